@@ -1,0 +1,284 @@
+"""Seeded synthetic inputs for the gated-retention (gRet) mixer.
+
+This module only draws numbers and rounds them to the storage dtype.  It holds
+none of the mixer's arithmetic, so both the fp64 oracle (``oracle/``) and the
+CUDA library may be fed from it without sharing any of the method.
+
+Generator (counter-based, so any element can be drawn on its own):
+
+* stream key      k = mix(mix(seed) XOR (tensor_id * phi))
+* 64-bit word i   w_i = mix(k + (i + 1) * phi)
+  where ``mix`` is the SplitMix64 output function (Steele, Lea and Flood,
+  "Fast splittable pseudorandom number generators", OOPSLA 2014) and
+  phi = 0x9E3779B97F4A7C15.
+* element e of a normal tensor uses the Box-Muller pair p = e // 2:
+  u1 = ((w_{2p} >> 11) + 1) 2^-53 in (0, 1], u2 = (w_{2p+1} >> 11) 2^-53,
+  r = sqrt(-2 ln u1); even e takes r cos(2 pi u2), odd e takes r sin(2 pi u2).
+* value = mean + sqrt(var) * normal, computed in fp64, then rounded to fp32
+  (IEEE round-to-nearest-even) and, for bf16 storage, from fp32 to bf16 (RNE).
+
+The workload presets mirror the shapes of the pages' long-context settings:
+head dimension 128 (YOCO deep analysis, section 5.3.4), chunk lengths of the
+chunkwise form (section 5.3.2) and contexts of 4K-64K tokens.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+import os
+from concurrent.futures import ThreadPoolExecutor
+from typing import Dict, List, Optional, Sequence, Tuple
+
+import numpy as np
+import torch
+
+_PHI = np.uint64(0x9E3779B97F4A7C15)
+_M1 = np.uint64(0xBF58476D1CE4E5B9)
+_M2 = np.uint64(0x94D049BB133111EB)
+_TWO53 = 1.0 / 9007199254740992.0
+
+# Tensor ids of the draw streams.
+TID_Q, TID_K, TID_V, TID_G, TID_Z = 1, 2, 3, 4, 5
+TID_STEP = 20  # decode-step tensors use TID_STEP + {TID_Q..TID_Z}
+
+
+def _mix(x: np.ndarray) -> np.ndarray:
+    with np.errstate(over="ignore"):
+        x = (x ^ (x >> np.uint64(30))) * _M1
+        x = (x ^ (x >> np.uint64(27))) * _M2
+        return x ^ (x >> np.uint64(31))
+
+
+def _stream_key(seed: int, tensor_id: int) -> np.uint64:
+    with np.errstate(over="ignore"):
+        s = _mix(np.array([seed & 0xFFFFFFFFFFFFFFFF], dtype=np.uint64))
+        t = np.array([tensor_id & 0xFFFFFFFFFFFFFFFF], dtype=np.uint64) * _PHI
+        return _mix(s ^ t)[0]
+
+
+def _words(key: np.uint64, idx: np.ndarray) -> np.ndarray:
+    with np.errstate(over="ignore"):
+        return _mix(key + (idx.astype(np.uint64) + np.uint64(1)) * _PHI)
+
+
+def standard_normal_at(seed: int, tensor_id: int, flat_index: np.ndarray) -> np.ndarray:
+    """N(0,1) draws (fp64) for the given flat element indices of one stream."""
+    e = np.asarray(flat_index, dtype=np.int64)
+    key = _stream_key(seed, tensor_id)
+    p = e >> 1
+    w1 = _words(key, 2 * p)
+    w2 = _words(key, 2 * p + 1)
+    u1 = ((w1 >> np.uint64(11)).astype(np.float64) + 1.0) * _TWO53
+    u2 = (w2 >> np.uint64(11)).astype(np.float64) * _TWO53
+    r = np.sqrt(-2.0 * np.log(u1))
+    ang = 2.0 * math.pi * u2
+    return np.where((e & 1) == 0, r * np.cos(ang), r * np.sin(ang))
+
+
+def _round_fp32_to_bf16_bits(x32: np.ndarray) -> np.ndarray:
+    u = x32.view(np.uint32).astype(np.uint64)
+    r = (u + np.uint64(0x7FFF) + ((u >> np.uint64(16)) & np.uint64(1))) >> np.uint64(16)
+    return r.astype(np.uint16)
+
+
+def to_storage(x64: np.ndarray, io: str) -> torch.Tensor:
+    """Round fp64 values to the storage dtype ('f32' or 'bf16'); returns a CPU tensor."""
+    x32 = x64.astype(np.float32)
+    if io == "f32":
+        return torch.from_numpy(np.ascontiguousarray(x32))
+    if io == "bf16":
+        bits = _round_fp32_to_bf16_bits(np.ascontiguousarray(x32))
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
+    raise ValueError(f"unknown storage dtype {io!r}")
+
+
+def _normal_full(seed: int, tid: int, numel: int, mean, std, io: str,
+                 mean_std_fn=None, threads: Optional[int] = None) -> torch.Tensor:
+    """Whole tensor of numel draws; mean/std scalars or per-element via mean_std_fn(idx)."""
+    out = torch.empty(numel, dtype=torch.float32 if io == "f32" else torch.bfloat16)
+    block = 1 << 22
+    nblk = (numel + block - 1) // block
+
+    def work(b):
+        lo, hi = b * block, min(numel, (b + 1) * block)
+        idx = np.arange(lo, hi, dtype=np.int64)
+        z = standard_normal_at(seed, tid, idx)
+        if mean_std_fn is not None:
+            m, s = mean_std_fn(idx)
+            v = m + s * z
+        else:
+            v = mean + std * z
+        out[lo:hi] = to_storage(v, io)
+
+    nthreads = threads or min(32, os.cpu_count() or 1)
+    if nblk == 1:
+        work(0)
+    else:
+        with ThreadPoolExecutor(nthreads) as ex:
+            list(ex.map(work, range(nblk)))
+    return out
+
+
+@dataclasses.dataclass(frozen=True)
+class PrefillConfig:
+    """One prefill workload: shapes, storage dtype and input distributions."""
+    name: str
+    B: int
+    H: int
+    N: int
+    dk: int
+    dv: int
+    chunk: int
+    io: str                      # 'f32' or 'bf16' for Q, K, V, G and O
+    tau: float
+    seed: int
+    qkv_var: float               # Q, K, V ~ N(0, qkv_var)
+    z_dist: Tuple[Tuple[float, float], ...]  # per head (mean, var), or a single entry
+    g_dist: Tuple[float, float] = (0.0, 1.0)
+    eps: float = 1e-5
+
+    def z_mean_std(self, h: np.ndarray):
+        zd = self.z_dist
+        if len(zd) == 1:
+            return np.full(h.shape, zd[0][0]), np.full(h.shape, math.sqrt(zd[0][1]))
+        m = np.array([zd[i][0] for i in range(self.H)])[h]
+        s = np.sqrt(np.array([zd[i][1] for i in range(self.H)]))[h]
+        return m, s
+
+    @property
+    def tokens(self) -> int:
+        return self.B * self.N
+
+    def scaled(self, **kw) -> "PrefillConfig":
+        return dataclasses.replace(self, **kw)
+
+
+@dataclasses.dataclass(frozen=True)
+class DecodeConfig:
+    """Recurrent decode workload: num_seqs x H states, prior prefill, T steps."""
+    name: str
+    num_seqs: int
+    H: int
+    dk: int
+    dv: int
+    steps: int
+    prior_len: int
+    io: str
+    tau: float
+    seed: int
+    qkv_var: float
+    z_dist: Tuple[float, float]
+    g_dist: Tuple[float, float] = (0.0, 1.0)
+    eps: float = 1e-5
+    prior_chunk: int = 64
+
+    def prior_prefill(self) -> PrefillConfig:
+        """The seeded prefill whose final state seeds the decode states."""
+        return PrefillConfig(name=self.name + "-prior", B=self.num_seqs, H=self.H, N=self.prior_len,
+                             dk=self.dk, dv=self.dv, chunk=self.prior_chunk, io=self.io,
+                             tau=self.tau, seed=self.seed, qkv_var=self.qkv_var,
+                             z_dist=(self.z_dist,), g_dist=self.g_dist, eps=self.eps)
+
+
+# The five workloads (shapes and distributions as the benchmark list states them;
+# the seeds of the four bf16 workloads are this module's choice: 1..4).
+C1 = PrefillConfig("prefill-f32-B1-H2-N256-d64-C64", 1, 2, 256, 64, 64, 64, "f32", 16.0, 0,
+                   1.0 / 64, ((2.0, 1.0),))
+C2 = PrefillConfig("prefill-bf16-B4-H16-N4096-dk128-dv256-C64", 4, 16, 4096, 128, 256, 64, "bf16",
+                   16.0, 1, 1.0 / 128, ((3.0, 1.5),))
+C3 = PrefillConfig("prefill-bf16-B1-H32-N65536-dk128-dv128-C128", 1, 32, 65536, 128, 128, 128,
+                   "bf16", 16.0, 2, 1.0 / 128, ((4.0, 1.0),))
+C4 = DecodeConfig("decode-bf16-S256-H16-dk128-dv256-T64", 256, 16, 128, 256, 64, 512, "bf16",
+                  16.0, 3, 1.0 / 128, (3.0, 1.5))
+C5 = PrefillConfig("prefill-bf16-gate-stress-B2-H16-N32768-dk128-dv256-C64", 2, 16, 32768, 128,
+                   256, 64, "bf16", 16.0, 4, 1.0 / 128,
+                   tuple([(-4.0, 1.0)] * 8 + [(8.0, 0.5)] * 8))
+
+CONFIGS = {"c1": C1, "c2": C2, "c3": C3, "c4": C4, "c5": C5}
+
+
+def prefill_inputs(cfg: PrefillConfig, tid_base: int = 0) -> Dict[str, torch.Tensor]:
+    """Full CPU tensors: Q, K [B,N,H,dk]; V, G [B,N,H,dv] in cfg.io; z [B,N,H] fp32."""
+    B, N, H, dk, dv = cfg.B, cfg.N, cfg.H, cfg.dk, cfg.dv
+    sd = math.sqrt(cfg.qkv_var)
+    out = {
+        "Q": _normal_full(cfg.seed, tid_base + TID_Q, B * N * H * dk, 0.0, sd, cfg.io).view(B, N, H, dk),
+        "K": _normal_full(cfg.seed, tid_base + TID_K, B * N * H * dk, 0.0, sd, cfg.io).view(B, N, H, dk),
+        "V": _normal_full(cfg.seed, tid_base + TID_V, B * N * H * dv, 0.0, sd, cfg.io).view(B, N, H, dv),
+        "G": _normal_full(cfg.seed, tid_base + TID_G, B * N * H * dv, cfg.g_dist[0],
+                          math.sqrt(cfg.g_dist[1]), cfg.io).view(B, N, H, dv),
+    }
+    out["z"] = _normal_full(cfg.seed, tid_base + TID_Z, B * N * H, 0.0, 1.0, "f32",
+                            mean_std_fn=lambda idx: cfg.z_mean_std(idx % H)).view(B, N, H)
+    return out
+
+
+def prefill_unit_inputs(cfg: PrefillConfig, b: int, h: int, tid_base: int = 0) -> Dict[str, torch.Tensor]:
+    """The slice of prefill_inputs(cfg) for one (batch, head) unit, drawn on its own.
+
+    Returns Q, K [N,dk]; V, G [N,dv] in cfg.io and z [N] fp32, element-identical to
+    ``prefill_inputs(cfg)[name][b, :, h]``.
+    """
+    B, N, H, dk, dv = cfg.B, cfg.N, cfg.H, cfg.dk, cfg.dv
+    n = np.arange(N, dtype=np.int64)[:, None]
+    sd = math.sqrt(cfg.qkv_var)
+
+    def idx(d):
+        return (((b * N + n) * H + h) * d + np.arange(d, dtype=np.int64)[None, :]).reshape(-1)
+
+    out = {}
+    for name, tid, d, mean, std in (("Q", TID_Q, dk, 0.0, sd), ("K", TID_K, dk, 0.0, sd),
+                                     ("V", TID_V, dv, 0.0, sd),
+                                     ("G", TID_G, dv, cfg.g_dist[0], math.sqrt(cfg.g_dist[1]))):
+        v = mean + std * standard_normal_at(cfg.seed, tid_base + tid, idx(d))
+        out[name] = to_storage(v, cfg.io).view(N, d)
+    zi = ((b * N + n[:, 0]) * H + h)
+    m, s = cfg.z_mean_std(np.full(N, h))
+    out["z"] = to_storage(m + s * standard_normal_at(cfg.seed, tid_base + TID_Z, zi), "f32")
+    return out
+
+
+def decode_step_inputs(cfg: DecodeConfig) -> Dict[str, torch.Tensor]:
+    """Per-step tensors for all T steps: q, k [T,S,H,dk]; v, g [T,S,H,dv]; z [T,S,H] fp32."""
+    T, S, H, dk, dv = cfg.steps, cfg.num_seqs, cfg.H, cfg.dk, cfg.dv
+    sd = math.sqrt(cfg.qkv_var)
+    b = TID_STEP
+    return {
+        "q": _normal_full(cfg.seed, b + TID_Q, T * S * H * dk, 0.0, sd, cfg.io).view(T, S, H, dk),
+        "k": _normal_full(cfg.seed, b + TID_K, T * S * H * dk, 0.0, sd, cfg.io).view(T, S, H, dk),
+        "v": _normal_full(cfg.seed, b + TID_V, T * S * H * dv, 0.0, sd, cfg.io).view(T, S, H, dv),
+        "g": _normal_full(cfg.seed, b + TID_G, T * S * H * dv, cfg.g_dist[0],
+                          math.sqrt(cfg.g_dist[1]), cfg.io).view(T, S, H, dv),
+        "z": _normal_full(cfg.seed, b + TID_Z, T * S * H, cfg.z_dist[0],
+                          math.sqrt(cfg.z_dist[1]), "f32").view(T, S, H),
+    }
+
+
+def decode_unit_step_inputs(cfg: DecodeConfig, s: int, h: int) -> Dict[str, torch.Tensor]:
+    """Slice of decode_step_inputs(cfg) for one (sequence, head): q,k [T,dk]; v,g [T,dv]; z [T]."""
+    T, S, H, dk, dv = cfg.steps, cfg.num_seqs, cfg.H, cfg.dk, cfg.dv
+    t = np.arange(T, dtype=np.int64)[:, None]
+    sd = math.sqrt(cfg.qkv_var)
+
+    def idx(d):
+        return (((t * S + s) * H + h) * d + np.arange(d, dtype=np.int64)[None, :]).reshape(-1)
+
+    out = {}
+    b = TID_STEP
+    for name, tid, d, mean, std in (("q", TID_Q, dk, 0.0, sd), ("k", TID_K, dk, 0.0, sd),
+                                     ("v", TID_V, dv, 0.0, sd),
+                                     ("g", TID_G, dv, cfg.g_dist[0], math.sqrt(cfg.g_dist[1]))):
+        v = mean + std * standard_normal_at(cfg.seed, b + tid, idx(d))
+        out[name] = to_storage(v, cfg.io).view(T, d)
+    zi = (t[:, 0] * S + s) * H + h
+    out["z"] = to_storage(cfg.z_dist[0] + math.sqrt(cfg.z_dist[1]) *
+                          standard_normal_at(cfg.seed, b + TID_Z, zi), "f32")
+    return out
+
+
+def random_unit(seed: int, tensor_id: int, shape: Sequence[int], mean=0.0, var=1.0,
+                io: str = "f32") -> torch.Tensor:
+    """Small helper for tests: a seeded tensor of any shape (CPU)."""
+    numel = int(np.prod(shape)) if len(shape) else 1
+    v = mean + math.sqrt(var) * standard_normal_at(seed, tensor_id, np.arange(numel, dtype=np.int64))
+    return to_storage(v, io).view(*shape)
