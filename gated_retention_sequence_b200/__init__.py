@@ -1,0 +1,11 @@
+"""Gated-retention (gRet) mixer on NVIDIA B200: Python face of libgret.
+
+The mixer ("YOCO 深度技术分析", section 2.2; chunkwise form, section 5.3.2)
+runs entirely in the CUDA library ``libgret.so`` built from ``csrc/``; this
+package only marshals arguments (see ``gret.py``).
+"""
+from .gret import (  # noqa: F401
+    Dtype, Epilogue, GretError, LIB_PATH, Path, SIGNATURES, Status, check_device_status,
+    decode_step, gret_decode_step, gret_last_device_status, gret_prefill, gret_prefill_path,
+    gret_prefill_workspace_size, gret_status_string, gret_version, load, prefill, prefill_path,
+)

@@ -1,0 +1,189 @@
+// libgret C ABI: argument validation, kernel selection and launch.
+//
+// Nothing here allocates device memory, copies tensors or touches data: every
+// step of the mixer runs in the kernels.  Validation happens before any launch
+// so that a bad call has no effect on the stream.
+#include <math.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "gret_common.cuh"
+
+namespace gret {
+namespace {
+
+__device__ unsigned int g_device_status;
+
+constexpr int kMaxDevices = 64;
+unsigned int* g_status_ptr[kMaxDevices] = {};
+int g_num_sms[kMaxDevices] = {};
+std::mutex g_mu;
+
+// Device status word and SM count of the current device (looked up once per
+// device, with that device current).
+bool device_info(unsigned int** status, int* num_sms) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_status_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return false;
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
+        g_status_ptr[dev] = static_cast<unsigned int*>(p);
+        g_num_sms[dev] = sms;
+    }
+    if (status) *status = g_status_ptr[dev];
+    if (num_sms) *num_sms = g_num_sms[dev];
+    return true;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool shape_supported(int dk, int dv) {
+    return dk % 16 == 0 && dv % 16 == 0 && dk <= 256 && dv <= 256;
+}
+
+bool chunk_supported(int chunk) { return chunk == 16 || chunk == 32 || chunk == 64 || chunk == 128; }
+
+constexpr size_t kMaxSmem = 227 * 1024;
+
+// Kernel choice for a prefill; segments/seg_len describe the sequence split.
+gret_path select_path(int B, int H, int N, int dk, int dv, int chunk, gret_dtype io, int num_sms,
+                      int* segments, int* seg_len) {
+    if (segments) *segments = 1;
+    if (seg_len) *seg_len = N;
+    if (B <= 0 || H <= 0 || N <= 0 || dk <= 0 || dv <= 0) return GRET_PATH_NONE;
+    if (io != GRET_F32 && io != GRET_BF16) return GRET_PATH_NONE;
+    if (!shape_supported(dk, dv) || !chunk_supported(chunk)) return GRET_PATH_NONE;
+    if (io == GRET_BF16 && prefill_tc_supported(dk, dv, chunk, io)) {
+        int segs = 1, len = N;
+        prefill_tc_plan(B, H, N, chunk, num_sms, &segs, &len);
+        if (segments) *segments = segs;
+        if (seg_len) *seg_len = len;
+        return GRET_PATH_TC;
+    }
+    if (prefill_simt_smem_bytes(dk, dv, chunk) <= kMaxSmem) return GRET_PATH_SIMT;
+    return GRET_PATH_NONE;
+}
+
+}  // namespace
+}  // namespace gret
+
+using namespace gret;
+
+extern "C" {
+
+const char* gret_status_string(gret_status s) {
+    switch (s) {
+        case GRET_OK: return "GRET_OK";
+        case GRET_ERR_INVALID_ARG: return "GRET_ERR_INVALID_ARG";
+        case GRET_ERR_UNSUPPORTED: return "GRET_ERR_UNSUPPORTED";
+        case GRET_ERR_CUDA: return "GRET_ERR_CUDA";
+        case GRET_ERR_TIMEOUT: return "GRET_ERR_TIMEOUT";
+    }
+    return "GRET_ERR_UNKNOWN";
+}
+
+int gret_version(void) { return 10000; }
+
+gret_path gret_prefill_path(int B, int H, int N, int dk, int dv, int chunk, gret_dtype io_dtype,
+                            int* segments) {
+    int sms = 148;
+    device_info(nullptr, &sms);
+    return select_path(B, H, N, dk, dv, chunk, io_dtype, sms, segments, nullptr);
+}
+
+size_t gret_prefill_workspace_size(int B, int H, int N, int dk, int dv, int chunk,
+                                   gret_dtype io_dtype) {
+    int sms = 148, segs = 1;
+    device_info(nullptr, &sms);
+    gret_path p = select_path(B, H, N, dk, dv, chunk, io_dtype, sms, &segs, nullptr);
+    if (p != GRET_PATH_TC) return 0;
+    return prefill_tc_workspace_bytes(B, H, dk, dv, segs);
+}
+
+gret_status gret_prefill(const void* Q, const void* K, const void* V, const float* gate_logits,
+                         const void* G, float tau, int chunk, void* O, float* S_final, int B, int H,
+                         int N, int dk, int dv, gret_dtype io_dtype, float eps, gret_epilogue epi,
+                         void* workspace, size_t workspace_bytes, gret_stream_t stream) {
+    if (!Q || !K || !V || !gate_logits || !O) return GRET_ERR_INVALID_ARG;
+    if (epi != GRET_EPI_GN_SWISH && epi != GRET_EPI_NONE) return GRET_ERR_INVALID_ARG;
+    if (epi == GRET_EPI_GN_SWISH && !G) return GRET_ERR_INVALID_ARG;
+    if (io_dtype != GRET_F32 && io_dtype != GRET_BF16) return GRET_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || N <= 0 || dk <= 0 || dv <= 0 || chunk <= 0) return GRET_ERR_INVALID_ARG;
+    if (!(tau > 0.0f) || !isfinite(tau) || !(eps >= 0.0f) || !isfinite(eps)) return GRET_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(gate_logits) || !aligned16(O) ||
+        (G && !aligned16(G)) || (S_final && !aligned16(S_final)))
+        return GRET_ERR_INVALID_ARG;
+    if ((long long)B * H > (1LL << 30) || (long long)B * N > (1LL << 40)) return GRET_ERR_UNSUPPORTED;
+
+    unsigned int* status = nullptr;
+    int sms = 0;
+    if (!device_info(&status, &sms)) return GRET_ERR_CUDA;
+    int segs = 1, seg_len = N;
+    gret_path path = select_path(B, H, N, dk, dv, chunk, io_dtype, sms, &segs, &seg_len);
+    if (path == GRET_PATH_NONE) return GRET_ERR_UNSUPPORTED;
+
+    PrefillArgs a;
+    a.Q = Q; a.K = K; a.V = V; a.z = gate_logits; a.G = G; a.O = O; a.S_final = S_final;
+    a.B = B; a.H = H; a.N = N; a.dk = dk; a.dv = dv; a.chunk = chunk;
+    a.inv_tau = 1.0f / tau; a.eps = eps; a.io = io_dtype; a.epi = epi;
+    a.workspace = workspace; a.workspace_bytes = workspace_bytes;
+    a.status = status; a.segments = segs; a.seg_len = seg_len;
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t err;
+    if (path == GRET_PATH_TC) {
+        size_t need = prefill_tc_workspace_bytes(B, H, dk, dv, segs);
+        if (need > 0) {
+            if (!workspace || workspace_bytes < need) return GRET_ERR_INVALID_ARG;
+            if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return GRET_ERR_INVALID_ARG;
+        }
+        err = launch_prefill_tc(a, s);
+    } else {
+        err = launch_prefill_simt(a, s);
+    }
+    return err == cudaSuccess ? GRET_OK : GRET_ERR_CUDA;
+}
+
+gret_status gret_decode_step(const void* q, const void* k, const void* v, const float* gate_logit,
+                             const void* g, float* S_inout, void* o, int num_seqs, int H, int dk,
+                             int dv, float tau, gret_dtype io_dtype, float eps, gret_epilogue epi,
+                             gret_stream_t stream) {
+    if (!q || !k || !v || !gate_logit || !S_inout || !o) return GRET_ERR_INVALID_ARG;
+    if (epi != GRET_EPI_GN_SWISH && epi != GRET_EPI_NONE) return GRET_ERR_INVALID_ARG;
+    if (epi == GRET_EPI_GN_SWISH && !g) return GRET_ERR_INVALID_ARG;
+    if (io_dtype != GRET_F32 && io_dtype != GRET_BF16) return GRET_ERR_INVALID_ARG;
+    if (num_seqs <= 0 || H <= 0 || dk <= 0 || dv <= 0) return GRET_ERR_INVALID_ARG;
+    if (!(tau > 0.0f) || !isfinite(tau) || !(eps >= 0.0f) || !isfinite(eps)) return GRET_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(gate_logit) ||
+        !aligned16(S_inout) || !aligned16(o) || (g && !aligned16(g)))
+        return GRET_ERR_INVALID_ARG;
+    if (!shape_supported(dk, dv)) return GRET_ERR_UNSUPPORTED;
+    if ((long long)num_seqs * H > (1LL << 31) - 1) return GRET_ERR_UNSUPPORTED;
+
+    DecodeArgs a;
+    a.q = q; a.k = k; a.v = v; a.z = gate_logit; a.g = g; a.S = S_inout; a.o = o;
+    a.num_units = num_seqs * H; a.H = H; a.dk = dk; a.dv = dv;
+    a.inv_tau = 1.0f / tau; a.eps = eps; a.io = io_dtype; a.epi = epi;
+    cudaError_t err = launch_decode(a, reinterpret_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? GRET_OK : GRET_ERR_CUDA;
+}
+
+gret_status gret_last_device_status(gret_stream_t stream) {
+    unsigned int* status = nullptr;
+    if (!device_info(&status, nullptr)) return GRET_ERR_CUDA;
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return GRET_ERR_CUDA;
+    unsigned int word = 0;
+    if (cudaMemcpy(&word, status, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return GRET_ERR_CUDA;
+    if (word != kDevOk) {
+        unsigned int zero = 0;
+        if (cudaMemcpy(status, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return GRET_ERR_CUDA;
+        return GRET_ERR_TIMEOUT;
+    }
+    return GRET_OK;
+}
+
+}  // extern "C"

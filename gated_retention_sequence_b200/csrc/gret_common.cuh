@@ -1,0 +1,89 @@
+// Shared device helpers and launch descriptors of libgret (internal header).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "gret.h"
+
+namespace gret {
+
+// Status word values a kernel writes when it gives up (host maps them to
+// GRET_ERR_TIMEOUT).  Kernels never trap.
+enum : unsigned int { kDevOk = 0u, kDevTimeout = 1u };
+
+struct PrefillArgs {
+    const void* Q;
+    const void* K;
+    const void* V;
+    const float* z;
+    const void* G;
+    void* O;
+    float* S_final;
+    int B, H, N, dk, dv, chunk;
+    float inv_tau, eps;
+    gret_dtype io;
+    gret_epilogue epi;
+    void* workspace;
+    size_t workspace_bytes;
+    unsigned int* status;     // device status word
+    int segments;             // sequence segments per unit (TC path)
+    int seg_len;              // tokens per segment (multiple of chunk)
+};
+
+struct DecodeArgs {
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* z;
+    const void* g;
+    float* S;
+    void* o;
+    int num_units, H, dk, dv;
+    float inv_tau, eps;
+    gret_dtype io;
+    gret_epilogue epi;
+};
+
+// Gate ("YOCO 深度技术分析", section 2.2): gamma = sigmoid(z)^(1/tau), kept in
+// log space: log gamma = -softplus(-z) / tau with
+// softplus(x) = max(x, 0) + log1p(exp(-|x|)).  Clamped at kMinLogGamma: a
+// token with gamma below e^-64 (about 1.6e-28) is treated as gamma = e^-64.
+// This keeps z = -inf (gamma = 0) from producing -inf - (-inf) in the
+// chunk-local sums, and keeps those fp32 sums small enough that the decay
+// between two later tokens (a difference of two sums) keeps its precision.
+constexpr float kMinLogGamma = -64.0f;
+__device__ __forceinline__ float log_gamma(float z, float inv_tau) {
+    float x = -z;
+    float sp = fmaxf(x, 0.0f) + log1pf(expf(-fabsf(x)));
+    return fmaxf(-sp * inv_tau, kMinLogGamma);
+}
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+__device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + expf(-x)); }
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Host-side launchers (one per kernel family).
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_prefill_simt(const PrefillArgs& a, cudaStream_t s);
+size_t prefill_simt_smem_bytes(int dk, int dv, int chunk);
+cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s);
+bool prefill_tc_supported(int dk, int dv, int chunk, gret_dtype io);
+void prefill_tc_plan(int B, int H, int N, int chunk, int num_sms, int* segments, int* seg_len);
+size_t prefill_tc_workspace_bytes(int B, int H, int dk, int dv, int segments);
+
+}  // namespace gret

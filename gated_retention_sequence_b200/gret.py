@@ -1,0 +1,229 @@
+"""Thin ctypes binding of libgret (argument marshalling only).
+
+``gret_prefill``, ``gret_decode_step``, ``gret_prefill_workspace_size``,
+``gret_prefill_path``, ``gret_last_device_status``, ``gret_status_string`` and
+``gret_version`` call the C ABI of ``include/gret.h`` one to one with raw
+pointers.  ``prefill`` and ``decode_step`` are conveniences for torch CUDA
+tensors: they check dtypes and shapes, allocate outputs and scratch with
+torch's allocator and pass the current stream.  Every step of the mixer runs
+in the CUDA library; there is no fallback, and a missing library raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import enum
+import os
+import threading
+from typing import Optional, Tuple
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgret.so")
+_lib = None
+_lock = threading.Lock()
+
+
+class Status(enum.IntEnum):
+    OK = 0
+    ERR_INVALID_ARG = 1
+    ERR_UNSUPPORTED = 2
+    ERR_CUDA = 3
+    ERR_TIMEOUT = 4
+
+
+class Dtype(enum.IntEnum):
+    F32 = 0
+    BF16 = 1
+
+
+class Epilogue(enum.IntEnum):
+    GN_SWISH = 0
+    NONE = 1
+
+
+class Path(enum.IntEnum):
+    NONE = 0
+    SIMT = 1
+    TC = 2
+
+
+class GretError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = Status(status)
+        super().__init__(f"{what}: {self.status.name}" if what else self.status.name)
+
+
+# Exported C symbols and their signatures.
+_VP, _FP, _I, _F, _SZ = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+SIGNATURES = {
+    "gret_prefill": (_I, [_VP, _VP, _VP, _FP, _VP, _F, _I, _VP, _FP, _I, _I, _I, _I, _I, _I, _F, _I,
+                          _VP, _SZ, _VP]),
+    "gret_prefill_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
+    "gret_prefill_path": (_I, [_I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_int)]),
+    "gret_decode_step": (_I, [_VP, _VP, _VP, _FP, _VP, _FP, _VP, _I, _I, _I, _I, _F, _I, _F, _I, _VP]),
+    "gret_last_device_status": (_I, [_VP]),
+    "gret_status_string": (ctypes.c_char_p, [_I]),
+    "gret_version": (_I, []),
+}
+
+
+def load():
+    """Load libgret.so (built by ``gated_retention_sequence_b200.build``); raises if absent."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"libgret.so is not built ({LIB_PATH}); run __graft_entry__.build()")
+            lib = ctypes.CDLL(LIB_PATH)
+            for name, (res, args) in SIGNATURES.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = lib
+    return _lib
+
+
+# ---------------------------------------------------------------- raw C calls
+def gret_prefill(Q, K, V, gate_logits, G, tau, chunk, O, S_final, B, H, N, dk, dv, io_dtype, eps,
+                 epi, workspace, workspace_bytes, stream) -> int:
+    return load().gret_prefill(Q, K, V, gate_logits, G, tau, chunk, O, S_final, B, H, N, dk, dv,
+                               int(io_dtype), eps, int(epi), workspace, workspace_bytes, stream)
+
+
+def gret_prefill_workspace_size(B, H, N, dk, dv, chunk, io_dtype) -> int:
+    return load().gret_prefill_workspace_size(B, H, N, dk, dv, chunk, int(io_dtype))
+
+
+def gret_prefill_path(B, H, N, dk, dv, chunk, io_dtype) -> Tuple[Path, int]:
+    segs = ctypes.c_int(0)
+    p = load().gret_prefill_path(B, H, N, dk, dv, chunk, int(io_dtype), ctypes.byref(segs))
+    return Path(p), segs.value
+
+
+def gret_decode_step(q, k, v, gate_logit, g, S_inout, o, num_seqs, H, dk, dv, tau, io_dtype, eps,
+                     epi, stream) -> int:
+    return load().gret_decode_step(q, k, v, gate_logit, g, S_inout, o, num_seqs, H, dk, dv, tau,
+                                   int(io_dtype), eps, int(epi), stream)
+
+
+def gret_last_device_status(stream=None) -> int:
+    return load().gret_last_device_status(stream)
+
+
+def gret_status_string(status: int) -> str:
+    return load().gret_status_string(int(status)).decode()
+
+
+def gret_version() -> int:
+    return load().gret_version()
+
+
+# ---------------------------------------------------------------- torch helpers
+def _torch():
+    import torch
+    return torch
+
+
+def _io_of(t) -> Dtype:
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return Dtype.BF16
+    if t.dtype == torch.float32:
+        return Dtype.F32
+    raise TypeError(f"unsupported io dtype {t.dtype}")
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _check(t, name, dtype, shape, device):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def prefill(Q, K, V, z, G, tau: float, chunk: int, eps: float = 1e-5, epilogue: str = "gn_swish",
+            O=None, S_final=None, want_state: bool = True, workspace=None, stream=None):
+    """Chunkwise prefill from the zero state.
+
+    Q, K [B,N,H,dk] and V, G [B,N,H,dv] in bf16 or fp32; z [B,N,H] fp32 gate logits.
+    Returns (O [B,N,H,dv] in the io dtype, S_final [B,H,dk,dv] fp32 or None).
+    ``epilogue='none'`` returns the pre-norm Y in O (G may be None).
+    """
+    torch = _torch()
+    B, N, H, dk = Q.shape
+    dv = V.shape[-1]
+    dev = Q.device
+    io = _io_of(Q)
+    epi = Epilogue.NONE if epilogue == "none" else Epilogue.GN_SWISH
+    _check(Q, "Q", Q.dtype, (B, N, H, dk), dev)
+    _check(K, "K", Q.dtype, (B, N, H, dk), dev)
+    _check(V, "V", Q.dtype, (B, N, H, dv), dev)
+    _check(z, "z", torch.float32, (B, N, H), dev)
+    if epi == Epilogue.GN_SWISH or G is not None:
+        _check(G, "G", Q.dtype, (B, N, H, dv), dev)
+    if O is None:
+        O = torch.empty((B, N, H, dv), dtype=Q.dtype, device=dev)
+    _check(O, "O", Q.dtype, (B, N, H, dv), dev)
+    if S_final is None and want_state:
+        S_final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    if S_final is not None:
+        _check(S_final, "S_final", torch.float32, (B, H, dk, dv), dev)
+    with torch.cuda.device(dev):
+        ws_bytes = gret_prefill_workspace_size(B, H, N, dk, dv, chunk, io)
+        if ws_bytes and (workspace is None or workspace.numel() * workspace.element_size() < ws_bytes):
+            workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        st = stream if stream is not None else torch.cuda.current_stream(dev)
+        status = gret_prefill(_ptr(Q), _ptr(K), _ptr(V), _ptr(z), _ptr(G), float(tau), int(chunk),
+                              _ptr(O), _ptr(S_final), B, H, N, dk, dv, io, float(eps), epi,
+                              _ptr(workspace) if ws_bytes else None, ws_bytes, st.cuda_stream)
+    if status != Status.OK:
+        raise GretError(status, "gret_prefill")
+    return O, S_final
+
+
+def decode_step(q, k, v, z, g, S, tau: float, eps: float = 1e-5, epilogue: str = "gn_swish",
+                o=None, stream=None):
+    """One recurrent step; S [num_seqs,H,dk,dv] fp32 is updated in place. Returns o."""
+    torch = _torch()
+    ns, H, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    io = _io_of(q)
+    epi = Epilogue.NONE if epilogue == "none" else Epilogue.GN_SWISH
+    _check(q, "q", q.dtype, (ns, H, dk), dev)
+    _check(k, "k", q.dtype, (ns, H, dk), dev)
+    _check(v, "v", q.dtype, (ns, H, dv), dev)
+    _check(z, "z", torch.float32, (ns, H), dev)
+    if epi == Epilogue.GN_SWISH or g is not None:
+        _check(g, "g", q.dtype, (ns, H, dv), dev)
+    _check(S, "S", torch.float32, (ns, H, dk, dv), dev)
+    if o is None:
+        o = torch.empty((ns, H, dv), dtype=q.dtype, device=dev)
+    _check(o, "o", q.dtype, (ns, H, dv), dev)
+    with torch.cuda.device(dev):
+        st = stream if stream is not None else torch.cuda.current_stream(dev)
+        status = gret_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(z), _ptr(g), _ptr(S), _ptr(o), ns, H,
+                                  dk, dv, float(tau), io, float(eps), epi, st.cuda_stream)
+    if status != Status.OK:
+        raise GretError(status, "gret_decode_step")
+    return o
+
+
+def prefill_path(B, H, N, dk, dv, chunk, io: Dtype) -> Tuple[Path, int]:
+    """Kernel the library would pick, and the sequence segments per unit."""
+    return gret_prefill_path(B, H, N, dk, dv, chunk, io)
+
+
+def check_device_status(stream=None) -> None:
+    """Synchronise and raise GretError if a kernel's bounded wait gave up."""
+    s = gret_last_device_status(stream)
+    if s != Status.OK:
+        raise GretError(s, "device status")

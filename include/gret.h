@@ -1,0 +1,133 @@
+/*
+ * libgret -- gated retention (gRet) mixer on NVIDIA B200 (sm_100a).
+ *
+ * C ABI: plain pointers and sizes, no C++ or framework types.  Every call is
+ * asynchronous on the given stream, allocates nothing and never throws; errors
+ * come back as a gret_status.  All tensor pointers are DEVICE pointers owned
+ * by the caller unless stated otherwise.
+ *
+ * What the mixer computes (web pages on the YOCO decoder-decoder family):
+ *  - "YOCO 深度技术分析", section 2.2 "Gated Retention (gRet)":
+ *      gate            gamma_n = sigmoid(z_n)^(1/tau), z = x W_gamma, one scalar
+ *                      per token and head ("head-wise gate")
+ *      parallel form   Y = (Q K^T (.) D) V, D[n][m] = prod_{i=m+1..n} gamma_i
+ *      recurrent form  S_n = gamma_n S_{n-1} + K_n^T V_n,  Y_n = Q_n S_n
+ *      per-head output GroupNorm(Y) (.) swish(G)
+ *  - same page, section 5.3.2: the chunkwise form (parallel inside a block of
+ *    `chunk` tokens, recurrent between blocks) is exactly equivalent; prefill
+ *    uses it, decode uses the recurrent form (section 5.3.7), and prefill hands
+ *    its last state to decode.
+ * No 1/sqrt(d_k) scale is applied (none appears in either form).  GroupNorm
+ * normalises the d_v channels of one token of one head with the biased
+ * variance and `eps`, without affine parameters; swish(g) = g * sigmoid(g).
+ *
+ * Layouts (row-major, contiguous, element strides only):
+ *   Q, K        [B][N][H][dk]   io dtype
+ *   V, G, O     [B][N][H][dv]   io dtype
+ *   gate_logits [B][N][H]       fp32 (z; the gate stays fp32 in both paths)
+ *   S           [B][H][dk][dv]  fp32, d_v fastest
+ * The decode step uses the same layouts with N = 1 and B = num_seqs.
+ */
+#ifndef GRET_H
+#define GRET_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL means the legacy default stream. */
+typedef struct CUstream_st* gret_stream_t;
+
+typedef enum {
+    GRET_OK = 0,
+    GRET_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, non-positive size, bad enum */
+    GRET_ERR_UNSUPPORTED = 2,   /* valid arguments outside what the kernels implement */
+    GRET_ERR_CUDA = 3,          /* a CUDA runtime/driver call or kernel launch failed */
+    GRET_ERR_TIMEOUT = 4        /* a bounded device-side wait gave up (see below) */
+} gret_status;
+
+typedef enum { GRET_F32 = 0, GRET_BF16 = 1 } gret_dtype;
+
+typedef enum {
+    GRET_EPI_GN_SWISH = 0,      /* O = GroupNorm(Y) (.) swish(G)                    */
+    GRET_EPI_NONE = 1           /* O = Y (pre-norm output; G is ignored, may be NULL) */
+} gret_epilogue;
+
+/* Kernel a prefill call runs (see gret_prefill_path). */
+typedef enum {
+    GRET_PATH_NONE = 0,         /* arguments are unsupported                         */
+    GRET_PATH_SIMT = 1,         /* fp32 CUDA-core chunkwise kernel (any io dtype)    */
+    GRET_PATH_TC = 2            /* tcgen05/TMEM tensor-core chunkwise kernel (bf16)  */
+} gret_path;
+
+/*
+ * gret_prefill -- chunkwise prefill of B x H independent (batch, head) units.
+ *
+ *   Q, K, V, gate_logits, G : inputs (layouts above).  G may be NULL when
+ *                             epi == GRET_EPI_NONE.
+ *   tau                     : gate temperature, > 0.
+ *   chunk                   : block length of the chunkwise form.  Supported:
+ *                             16, 32, 64, 128 (TC path: 64 or 128).
+ *   O                       : output [B][N][H][dv] in io_dtype; must not alias an input.
+ *   S_final                 : fp32 [B][H][dk][dv] state after the last token, or NULL.
+ *   B, H, N, dk, dv         : > 0; dk, dv multiples of 16 and <= 256.
+ *   eps                     : GroupNorm epsilon (>= 0); 1e-5 is the usual value.
+ *   workspace, workspace_bytes : device scratch of at least
+ *                             gret_prefill_workspace_size(...) bytes, 256-byte
+ *                             aligned; may be NULL when that size is 0.  Its
+ *                             contents on entry do not matter.
+ * The prefill starts from the zero state.  Pointers must be 16-byte aligned.
+ * Calls that share a workspace must not overlap on the GPU.
+ */
+gret_status gret_prefill(const void* Q, const void* K, const void* V, const float* gate_logits,
+                         const void* G, float tau, int chunk, void* O, float* S_final,
+                         int B, int H, int N, int dk, int dv, gret_dtype io_dtype, float eps,
+                         gret_epilogue epi, void* workspace, size_t workspace_bytes,
+                         gret_stream_t stream);
+
+/* Device scratch (bytes) gret_prefill needs for these arguments; 0 if none.
+ * Returns 0 as well for unsupported arguments (gret_prefill then reports them). */
+size_t gret_prefill_workspace_size(int B, int H, int N, int dk, int dv, int chunk,
+                                   gret_dtype io_dtype);
+
+/* Which kernel gret_prefill would run for these arguments, and into how many
+ * sequence segments it splits each unit (1 = no split).  segments may be NULL. */
+gret_path gret_prefill_path(int B, int H, int N, int dk, int dv, int chunk, gret_dtype io_dtype,
+                            int* segments);
+
+/*
+ * gret_decode_step -- one recurrent step for num_seqs x H units
+ * ("YOCO 深度技术分析" sections 2.2 and 5.3.7):
+ *     S <- gamma S + k^T v ;  y = q S ;  o = GroupNorm(y) (.) swish(g)
+ *   q, k        [num_seqs][H][dk] io dtype
+ *   v, g, o     [num_seqs][H][dv] io dtype (g may be NULL when epi == GRET_EPI_NONE)
+ *   gate_logit  [num_seqs][H] fp32
+ *   S_inout     [num_seqs][H][dk][dv] fp32, updated in place
+ * o must not alias any input or S_inout.  Pointers must be 16-byte aligned;
+ * dk, dv multiples of 16 and <= 256.
+ */
+gret_status gret_decode_step(const void* q, const void* k, const void* v, const float* gate_logit,
+                             const void* g, float* S_inout, void* o, int num_seqs, int H, int dk,
+                             int dv, float tau, gret_dtype io_dtype, float eps, gret_epilogue epi,
+                             gret_stream_t stream);
+
+/* Synchronises `stream`, then reports (and clears) the device status word that
+ * kernels set when a bounded wait (an mbarrier or tensor-memory wait) gave up:
+ * GRET_ERR_TIMEOUT in that case, GRET_ERR_CUDA if the stream reports an error,
+ * else GRET_OK.  Kernels never trap; a timed-out kernel returns early and its
+ * outputs are undefined. */
+gret_status gret_last_device_status(gret_stream_t stream);
+
+/* Static, human-readable name of a status code. */
+const char* gret_status_string(gret_status status);
+
+/* Library version as major * 10000 + minor * 100 + patch. */
+int gret_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GRET_H */

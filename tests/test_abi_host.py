@@ -1,0 +1,90 @@
+"""Host-side checks of the C ABI: the library loads, exports every symbol the
+header declares, and rejects bad arguments before launching anything.
+None of these calls launches a kernel, so they run without a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_retention_sequence_b200 as gret
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from gated_retention_sequence_b200 import build
+    build.build()
+    return gret.load()
+
+
+def _declared_functions():
+    text = open(os.path.join(ROOT, "include", "gret.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gret_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_names():
+    assert _declared_functions() == sorted(gret.SIGNATURES)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings_and_version(lib):
+    for s in gret.Status:
+        assert gret.gret_status_string(s) == "GRET_" + s.name
+    assert gret.gret_version() >= 10000
+
+
+def _prefill_args(**over):
+    good = 0x10000  # any 16-byte aligned address: validation fails before it is used
+    a = dict(Q=good, K=good, V=good, gate_logits=good, G=good, tau=16.0, chunk=64, O=good,
+             S_final=None, B=1, H=2, N=256, dk=64, dv=64, io_dtype=gret.Dtype.F32, eps=1e-5,
+             epi=gret.Epilogue.GN_SWISH, workspace=None, workspace_bytes=0, stream=None)
+    a.update(over)
+    return a
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(Q=None), gret.Status.ERR_INVALID_ARG),
+    (dict(O=None), gret.Status.ERR_INVALID_ARG),
+    (dict(G=None), gret.Status.ERR_INVALID_ARG),
+    (dict(K=0x10008), gret.Status.ERR_INVALID_ARG),          # misaligned
+    (dict(B=0), gret.Status.ERR_INVALID_ARG),
+    (dict(N=-3), gret.Status.ERR_INVALID_ARG),
+    (dict(tau=0.0), gret.Status.ERR_INVALID_ARG),
+    (dict(tau=float("nan")), gret.Status.ERR_INVALID_ARG),
+    (dict(eps=-1.0), gret.Status.ERR_INVALID_ARG),
+    (dict(io_dtype=7), gret.Status.ERR_INVALID_ARG),
+    (dict(epi=5), gret.Status.ERR_INVALID_ARG),
+    (dict(chunk=0), gret.Status.ERR_INVALID_ARG),
+])
+def test_prefill_rejects_bad_arguments(lib, over, expect):
+    assert gret.gret_prefill(**_prefill_args(**over)) == expect
+
+
+def test_decode_rejects_bad_arguments(lib):
+    good = 0x10000
+    base = dict(q=good, k=good, v=good, gate_logit=good, g=good, S_inout=good, o=good, num_seqs=4,
+                H=2, dk=128, dv=256, tau=16.0, io_dtype=gret.Dtype.BF16, eps=1e-5,
+                epi=gret.Epilogue.GN_SWISH, stream=None)
+    for over in (dict(S_inout=None), dict(o=0x10004), dict(num_seqs=0), dict(tau=-1.0),
+                 dict(g=None)):
+        assert gret.gret_decode_step(**{**base, **over}) == gret.Status.ERR_INVALID_ARG
+    for over in (dict(dk=24), dict(dv=512)):
+        assert gret.gret_decode_step(**{**base, **over}) == gret.Status.ERR_UNSUPPORTED
+
+
+def test_path_selection(lib):
+    # fp32 io always takes the CUDA-core kernel
+    p, segs = gret.prefill_path(1, 2, 256, 64, 64, 64, gret.Dtype.F32)
+    assert p == gret.Path.SIMT and segs == 1
+    # shapes no kernel takes
+    assert gret.prefill_path(1, 2, 256, 24, 64, 64, gret.Dtype.F32)[0] == gret.Path.NONE
+    assert gret.prefill_path(1, 2, 256, 64, 64, 48, gret.Dtype.F32)[0] == gret.Path.NONE
+    assert gret.prefill_path(1, 2, 256, 256, 256, 128, gret.Dtype.F32)[0] == gret.Path.NONE
+    assert gret.gret_prefill_workspace_size(1, 2, 256, 64, 64, 64, gret.Dtype.F32) == 0
