@@ -1,0 +1,396 @@
+#!/usr/bin/env python
+"""Throughput of the gated-retention mixer on B200 through libgret.
+
+One step = one gret_prefill call (gate, chunk decay sums, intra-chunk scores
+and mask, intra and inter-chunk outputs, state carry, GroupNorm + swish
+epilogue, final state) over a batch of 4 x 4096 tokens, 16 heads, d_k 128,
+d_v 256, chunk 64, bf16 I/O with fp32 state and gate logits -- the long-context
+prefill shape of "YOCO 深度技术分析" (head dimension 128, chunkwise form).
+Inputs are seeded synthetic tensors already resident in HBM (546 MB, larger
+than the 126 MB L2, so no flush is needed between steps).
+
+The JSON line also carries the recurrent decode step (256 sequences x 16
+heads, 128 x 256 fp32 states, 64 consecutive launches) as ``decode``.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (weak scaling): one process per GPU, each runs its own batch; no
+collective is on the data path.  ``--impl reference`` times the fp64 CPU
+oracle on the host cores instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = "gRet prefill Mtok/s & % bf16 TC peak; decode-step state GB/s & % HBM peak"
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return dict(FALLBACK_PEAKS, source="fallback")
+
+
+def prefill_alg(cfg):
+    """Algorithmic bytes and flops of one prefill (per token and head:
+    bytes e(2 dk + 3 dv) + 4 for Q, K, V, G, O and the fp32 gate logit;
+    flops C(dk + dv) + 4 dk dv for the causal half of the intra-chunk products
+    plus Q S and K^T V; plus the fp32 final state, 4 dk dv bytes per unit)."""
+    e = 2 if cfg.io == "bf16" else 4
+    th = cfg.B * cfg.N * cfg.H
+    units = cfg.B * cfg.H
+    bytes_ = th * (e * (2 * cfg.dk + 3 * cfg.dv) + 4) + units * 4 * cfg.dk * cfg.dv
+    flops = th * (cfg.chunk * (cfg.dk + cfg.dv) + 4 * cfg.dk * cfg.dv)
+    return bytes_, flops
+
+
+def decode_alg(cfg):
+    """Bytes of one decode step: the fp32 state read and written once, plus
+    q, k, v, g, o and the gate logit."""
+    e = 2 if cfg.io == "bf16" else 4
+    units = cfg.num_seqs * cfg.H
+    return units * (8 * cfg.dk * cfg.dv + e * (2 * cfg.dk + 3 * cfg.dv) + 4)
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while the GPU works."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.tmp = None
+
+    def start(self):
+        try:
+            self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50",
+                 "-i", str(self.gpu)], stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.tmp.flush()
+        self.tmp.seek(0)
+        rows = [r.strip().split(", ") for r in self.tmp.read().splitlines() if r.strip()]
+        os.unlink(self.tmp.name)
+        load, maxc, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm, mx, util = float(r[1]), float(r[2]), float(r[4])
+            except (ValueError, IndexError):
+                continue
+            maxc = mx
+            if util > 0:
+                load.append(sm)
+                for n, v in zip(names, r[6:10]):
+                    if v.strip() == "Active":
+                        reasons.add(n)
+        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": maxc,
+                "reasons": sorted(reasons), "samples_under_load": len(load)}
+
+
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    import torch
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def cpu_oracle_sample(cfg, units, threads):
+    """Time the fp64 oracle (as it stands) on `units` (batch, head) units of cfg."""
+    import gret_inputs as gi
+    import oracle
+    import torch
+    per = []
+    for u in range(units):
+        b, h = divmod(u % (cfg.B * cfg.H), cfg.H)
+        per.append(gi.prefill_unit_inputs(cfg, b, h))
+
+    def stack(name):
+        return torch.stack([p[name] for p in per], 1)[None] if name != "z" else \
+            torch.stack([p["z"] for p in per], 1)[None]
+    Q, K, V, G, z = (stack(n) for n in ("Q", "K", "V", "G", "z"))
+    t0 = time.perf_counter()
+    oracle.prefill(Q, K, V, z, G, cfg.tau, cfg.eps, threads=threads)
+    dt = time.perf_counter() - t0
+    tokens = units * cfg.N / cfg.H     # one unit = N tokens of one of H heads
+    return tokens / dt / 1e6, dt
+
+
+def run_reference(args, world, rank):
+    """Reference arm: the fp64 CPU oracle on a bounded sample of the workload."""
+    import gret_inputs as gi
+    import oracle
+    if rank != 0:
+        return 0
+    cfg = gi.C2
+    threads = oracle.default_threads()
+    units = min(cfg.B * cfg.H, threads)
+    vals = []
+    for i in range(args.warmup + args.steps):
+        v, dt = cpu_oracle_sample(cfg, units, threads)
+        if i >= args.warmup:
+            vals.append((v, dt))
+    value = statistics.mean(v for v, _ in vals)
+    sample = (f"{units} of {cfg.B * cfg.H} (batch, head) units x {cfg.N} tokens per step, "
+              f"fp64 recurrent form + GroupNorm/swish, {threads} threads")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "Mtok/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * statistics.mean(dt for _, dt in vals), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "N": cfg.N, "dk": cfg.dk,
+                       "dv": cfg.dv, "chunk": cfg.chunk, "io": cfg.io},
+            "cpu_baseline": {"value": value, "unit": "Mtok/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "Mtok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args, world, rank, local):
+    import torch
+    import gated_retention_sequence_b200 as gret
+    import gret_inputs as gi
+
+    gret.load()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    cfg = gi.C2
+    io = gret.Dtype.BF16
+    path, segs = gret.prefill_path(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, cfg.chunk, io)
+    host = gi.prefill_inputs(cfg)
+    d = {k: v.to(dev) for k, v in host.items()}
+    O = torch.empty_like(d["V"])
+    S = torch.empty((cfg.B, cfg.H, cfg.dk, cfg.dv), dtype=torch.float32, device=dev)
+    ws_bytes = gret.gret_prefill_workspace_size(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, cfg.chunk, io)
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        gret.prefill(d["Q"], d["K"], d["V"], d["z"], d["G"], cfg.tau, cfg.chunk, eps=cfg.eps, O=O,
+                     S_final=S, workspace=ws, stream=stream)
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    for _ in range(args.warmup):
+        step()
+    gret.check_device_status()
+    barrier(world)
+    ks = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ke = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for e in ks + ke:
+        e.record(stream)          # materialise the CUDA events
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    t_start.record(stream)
+    for i in range(args.steps):
+        gret.gret_set_profile_events(ks[i].cuda_event, ke[i].cuda_event)
+        step()
+    t_end.record(stream)
+    gret.gret_set_profile_events(None, None)
+    barrier(world)
+    ms = t_start.elapsed_time(t_end)
+    ms = max_over_ranks(ms, world)
+    gret.check_device_status()
+    kern_ms = statistics.mean(ks[i].elapsed_time(ke[i]) for i in range(args.steps))
+
+    tokens = cfg.B * cfg.N
+    value = world * tokens * args.steps / (ms / 1e3) / 1e6
+    alg_bytes, alg_flops = prefill_alg(cfg)
+    step_s = ms / 1e3 / args.steps
+    launches_per_step = 2 + (2 if segs > 1 else 0)
+
+    # end to end through the public call: pinned host inputs in, O and S out
+    pin = {k: v.pin_memory() for k, v in host.items()}
+    O_h = torch.empty(O.shape, dtype=O.dtype, pin_memory=True)
+    S_h = torch.empty(S.shape, dtype=S.dtype, pin_memory=True)
+    e2e_steps = max(1, min(args.steps, 20))
+    h2d = sum(v.numel() * v.element_size() for v in pin.values())
+    d2h = O_h.numel() * O_h.element_size() + S_h.numel() * S_h.element_size()
+
+    def e2e_step():
+        for k, v in pin.items():
+            d[k].copy_(v, non_blocking=True)
+        step()
+        O_h.copy_(O, non_blocking=True)
+        S_h.copy_(S, non_blocking=True)
+
+    e2e_value = None
+    if not args.no_e2e:
+        e2e_step()
+        barrier(world)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        barrier(world)
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+        e2e_value = world * tokens * e2e_steps / (e2e_ms / 1e3) / 1e6
+
+    decode = None if args.no_decode else run_decode(args, world, dev, stream, peaks)
+    clk = clocks.stop()
+
+    line = None
+    if rank == 0:
+        achieved = alg_bytes / (kern_ms / 1e3) / 1e9
+        line = {
+            "metric": METRIC, "value": value, "unit": "Mtok/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "N": cfg.N, "dk": cfg.dk,
+                       "dv": cfg.dv, "chunk": cfg.chunk, "io": "bf16 (fp32 state, fp32 gate logits)",
+                       "segments": segs, "path": path.name,
+                       "l2": "inputs 546 MB > 126 MB L2 per step, no flush",
+                       "parallelism": f"dp{world} (independent batches)"},
+            "tc": {"alg_tflops": alg_flops / step_s / 1e12,
+                   "frac_of_bf16_peak": alg_flops / step_s / 1e12 / peaks["bf16_tflops"],
+                   "peak_tflops": peaks["bf16_tflops"], "peak_source": peaks["source"] + " burst"},
+            "path_hbm": {"alg_gbs": alg_bytes / step_s / 1e9,
+                         "frac": alg_bytes / step_s / 1e9 / peaks["hbm_gbs"]},
+            "roofline": {"kernel": "prefill_tc_kernel (fused chunk loop)", "bound": "hbm",
+                         "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                         "alg_bytes_per_launch": alg_bytes, "launch_ms": kern_ms,
+                         "peak_source": peaks["source"]},
+            "e2e": {"value": e2e_value, "unit": "Mtok/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk,
+            "decode": decode,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            import oracle
+            threads = oracle.default_threads()
+            units = min(cfg.B * cfg.H, 2 * threads)
+            v, dt = cpu_oracle_sample(cfg, units, threads)
+            line["cpu_baseline"] = {"value": v, "unit": "Mtok/s", "cores": threads, "kind": "oracle",
+                                    "sample": f"{units} (batch, head) units x {cfg.N} tokens of {cfg.name}, "
+                                              f"fp64 recurrent form + GroupNorm/swish, {dt:.1f} s"}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_decode(args, world, dev, stream, peaks):
+    """Recurrent decode: 64 consecutive single-token steps over 256 x 16 states."""
+    import torch
+    import gated_retention_sequence_b200 as gret
+    import gret_inputs as gi
+    cfg = gi.C4
+    p = cfg.prior_prefill()
+    prior = {k: v.to(dev) for k, v in gi.prefill_inputs(p).items()}
+    _, S = gret.prefill(prior["Q"], prior["K"], prior["V"], prior["z"], prior["G"], p.tau, p.chunk)
+    del prior
+    st = {k: v.to(dev) for k, v in gi.decode_step_inputs(cfg).items()}
+    o = torch.empty_like(st["v"][0])
+    T = cfg.steps
+    for t in range(min(3, T)):       # warm-up steps on a copy of the state
+        S_w = S.clone()
+        gret.decode_step(st["q"][t], st["k"][t], st["v"][t], st["z"][t], st["g"][t], S_w, cfg.tau, o=o)
+    del S_w
+    barrier(world)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(T + 1)]
+    ev[0].record(stream)
+    for t in range(T):
+        gret.decode_step(st["q"][t], st["k"][t], st["v"][t], st["z"][t], st["g"][t], S, cfg.tau, o=o)
+        ev[t + 1].record(stream)
+    barrier(world)
+    gret.check_device_status()
+    per = [ev[t].elapsed_time(ev[t + 1]) for t in range(T)]
+    mean_ms = max_over_ranks(statistics.mean(per), world)
+    med_ms = statistics.median(per)
+    bytes_ = decode_alg(cfg)
+    gbs = bytes_ / (mean_ms / 1e3) / 1e9
+    return {"workload": cfg.name, "steps": T, "ms_per_step_mean": mean_ms, "ms_per_step_median": med_ms,
+            "state_gbs": world * bytes_ / (mean_ms / 1e3) / 1e9, "unit": "GB/s",
+            "roofline": {"kernel": "decode_step_kernel", "bound": "hbm", "achieved": gbs,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                         "traffic": None, "alg_bytes_per_launch": bytes_,
+                         "peak_source": peaks["source"]},
+            "gpu_launches": T}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        return run_reference(args, world, rank)
+    world, rank, local = dist_setup()
+    try:
+        return run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -11,6 +11,10 @@
 #include "gret_common.cuh"
 
 namespace gret {
+
+thread_local cudaEvent_t g_profile_start = nullptr;
+thread_local cudaEvent_t g_profile_stop = nullptr;
+
 namespace {
 
 __device__ unsigned int g_device_status;
@@ -88,6 +92,11 @@ const char* gret_status_string(gret_status s) {
 
 int gret_version(void) { return 10000; }
 
+void gret_set_profile_events(void* start, void* stop) {
+    g_profile_start = static_cast<cudaEvent_t>(start);
+    g_profile_stop = static_cast<cudaEvent_t>(stop);
+}
+
 gret_path gret_prefill_path(int B, int H, int N, int dk, int dv, int chunk, gret_dtype io_dtype,
                             int* segments) {
     int sms = 148;
@@ -101,7 +110,7 @@ size_t gret_prefill_workspace_size(int B, int H, int N, int dk, int dv, int chun
     device_info(nullptr, &sms);
     gret_path p = select_path(B, H, N, dk, dv, chunk, io_dtype, sms, &segs, nullptr);
     if (p != GRET_PATH_TC) return 0;
-    return prefill_tc_workspace_bytes(B, H, dk, dv, segs);
+    return prefill_tc_workspace_bytes(B, H, N, dk, dv, chunk, segs);
 }
 
 gret_status gret_prefill(const void* Q, const void* K, const void* V, const float* gate_logits,
@@ -136,7 +145,7 @@ gret_status gret_prefill(const void* Q, const void* K, const void* V, const floa
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t err;
     if (path == GRET_PATH_TC) {
-        size_t need = prefill_tc_workspace_bytes(B, H, dk, dv, segs);
+        size_t need = prefill_tc_workspace_bytes(B, H, N, dk, dv, chunk, segs);
         if (need > 0) {
             if (!workspace || workspace_bytes < need) return GRET_ERR_INVALID_ARG;
             if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return GRET_ERR_INVALID_ARG;

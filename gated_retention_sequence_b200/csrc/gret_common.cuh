@@ -77,6 +77,10 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
+// Events gret_set_profile_events armed for this host thread (null when off).
+extern thread_local cudaEvent_t g_profile_start;
+extern thread_local cudaEvent_t g_profile_stop;
+
 // Host-side launchers (one per kernel family).
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_prefill_simt(const PrefillArgs& a, cudaStream_t s);
@@ -84,6 +88,6 @@ size_t prefill_simt_smem_bytes(int dk, int dv, int chunk);
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s);
 bool prefill_tc_supported(int dk, int dv, int chunk, gret_dtype io);
 void prefill_tc_plan(int B, int H, int N, int chunk, int num_sms, int* segments, int* seg_len);
-size_t prefill_tc_workspace_bytes(int B, int H, int dk, int dv, int segments);
+size_t prefill_tc_workspace_bytes(int B, int H, int N, int dk, int dv, int chunk, int segments);
 
 }  // namespace gret

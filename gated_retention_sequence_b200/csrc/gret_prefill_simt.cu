@@ -146,6 +146,7 @@ size_t prefill_simt_smem_bytes(int dk, int dv, int chunk) {
 cudaError_t launch_prefill_simt(const PrefillArgs& a, cudaStream_t s) {
     size_t smem = prefill_simt_smem_bytes(a.dk, a.dv, a.chunk);
     int units = a.B * a.H;
+    if (g_profile_start) cudaEventRecord(g_profile_start, s);
     if (a.io == GRET_BF16) {
         auto k = prefill_simt_kernel<__nv_bfloat16>;
         cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -155,6 +156,7 @@ cudaError_t launch_prefill_simt(const PrefillArgs& a, cudaStream_t s) {
         cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         k<<<units, kThreads, smem, s>>>(a);
     }
+    if (g_profile_stop) cudaEventRecord(g_profile_stop, s);
     return cudaGetLastError();
 }
 

@@ -61,6 +61,7 @@ SIGNATURES = {
     "gret_prefill_path": (_I, [_I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_int)]),
     "gret_decode_step": (_I, [_VP, _VP, _VP, _FP, _VP, _FP, _VP, _I, _I, _I, _I, _F, _I, _F, _I, _VP]),
     "gret_last_device_status": (_I, [_VP]),
+    "gret_set_profile_events": (None, [_VP, _VP]),
     "gret_status_string": (ctypes.c_char_p, [_I]),
     "gret_version": (_I, []),
 }
@@ -107,6 +108,10 @@ def gret_decode_step(q, k, v, gate_logit, g, S_inout, o, num_seqs, H, dk, dv, ta
 
 def gret_last_device_status(stream=None) -> int:
     return load().gret_last_device_status(stream)
+
+
+def gret_set_profile_events(start, stop) -> None:
+    load().gret_set_profile_events(start, stop)
 
 
 def gret_status_string(status: int) -> str:

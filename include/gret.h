@@ -120,6 +120,13 @@ gret_status gret_decode_step(const void* q, const void* k, const void* v, const 
  * outputs are undefined. */
 gret_status gret_last_device_status(gret_stream_t stream);
 
+/* Profiling aid.  While set (non-NULL), every gret_prefill call made from the
+ * calling host thread records `start` on its stream just before the launch of
+ * the fused chunk-loop kernel (the dominant kernel of a prefill) and `stop`
+ * just after it, so that cudaEventElapsedTime gives that kernel's duration.
+ * Both are cudaEvent_t handles owned by the caller; pass NULL, NULL to stop. */
+void gret_set_profile_events(void* start, void* stop);
+
 /* Static, human-readable name of a status code. */
 const char* gret_status_string(gret_status status);
 
