@@ -63,7 +63,7 @@ struct Cfg {
     static constexpr int V_BYTES = (DV / 64) * BOX;
     static constexpr int G_BYTES = (DV / 64) * BOX;
     static constexpr int P_BYTES = (C / 64) * BOX;          // rows t, C bf16 of s
-    static constexpr int TPT = (NH == 2) ? C : C / 2;       // tokens per thread, epilogue
+    static constexpr int HT = C / 2;                        // tokens per thread, epilogue
     // tensor-memory columns
     static constexpr int TM_S = 0;                          // S^T: NH x 128 fp32 columns
     static constexpr int TM_O = NH * 128;                   // O^T: NH x C
@@ -78,8 +78,8 @@ struct Cfg {
     static constexpr int OFF_G = OFF_V + NS * V_BYTES;
     static constexpr int OFF_P = OFF_G + NG * G_BYTES;
     static constexpr int OFF_B = OFF_P + P_BYTES;           // NS x C fp32 decay sums
-    static constexpr int OFF_RED = OFF_B + NS * C * 4;      // kCW x TPT x 2 fp32
-    static constexpr int OFF_STAT = OFF_RED + kCW * TPT * 2 * 4;  // C x (mean, rstd)
+    static constexpr int OFF_RED = OFF_B + NS * C * 4;      // kCW x HT x 2 fp32
+    static constexpr int OFF_STAT = OFF_RED + kCW * HT * 2 * 4;   // C x (rstd, -mean * rstd)
     static constexpr int OFF_BAR = OFF_STAT + C * 8;
     static constexpr int NUM_BARS = 2 * NS + 2 * NG + 2;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
@@ -383,76 +383,72 @@ __global__ void __launch_bounds__(kThreadsTC, 1) prefill_tc_kernel(const __grid_
 
             if (kFull) {
                 // ---------------------------------------------------- epilogue
-                constexpr int TPT = CF::TPT;
+                // Thread (q4, grp, lane) owns d_v channels h*128 + q4*32 + lane
+                // (h < NH) for tokens grp*HT .. grp*HT + HT - 1.
+                constexpr int HT = CF::HT;
                 const int g = i % NG;
                 if (p.has_g) mbar_wait(bar(BGF + g), (i / NG) & 1, p.status, abort_flag);
                 uint8_t* Gp = sm + CF::OFF_G + g * CF::G_BYTES;
-                const int half = NH == 2 ? grp : 0;
-                const int t0 = NH == 2 ? 0 : grp * TPT;
-                const int d = half * 128 + q4 * 32 + lane;
-                const uint32_t oaddr = tm + lq + CF::TM_O + half * C + t0;
+                const int t0 = grp * HT;
+                const uint32_t oaddr = tm + lq + CF::TM_O + t0;
                 float* red = reinterpret_cast<float*>(sm + CF::OFF_RED);
-                float* stat = reinterpret_cast<float*>(sm + CF::OFF_STAT);
+                float2* stat = reinterpret_cast<float2*>(sm + CF::OFF_STAT);
                 if (p.gn) {
-                    float v[TPT];
-                    {
-                        uint32_t r[TPT];
-                        tmem_ld<TPT>(oaddr, r);
-                        tmem_wait_ld();
+                    // per-token sums over this thread's channels, then over the
+                    // warp's lanes, then over the four lane quarters
 #pragma unroll
-                        for (int j = 0; j < TPT; ++j) v[j] = u2f(r[j]);
+                    for (int pass = 0; pass < 2; ++pass) {
+                        float v[HT];
+#pragma unroll
+                        for (int h = 0; h < NH; ++h) {
+                            uint32_t r[HT];
+                            tmem_ld<HT>(oaddr + h * C, r);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int j = 0; j < HT; ++j) {
+                                const float y = u2f(r[j]);
+                                const float x = pass == 0 ? y : y * y;
+                                v[j] = h == 0 ? x : v[j] + x;
+                            }
+                        }
+                        warp_transpose_sum<HT>(v, lane);
+#pragma unroll
+                        for (int j = 0; j < HT / 32; ++j) red[(warp * HT + lane * (HT / 32) + j) * 2 + pass] = v[j];
                     }
-                    warp_transpose_sum<TPT>(v, lane);
-#pragma unroll
-                    for (int j = 0; j < TPT / 32; ++j) red[(warp * TPT + lane * (TPT / 32) + j) * 2] = v[j];
-                    {
-                        uint32_t r[TPT];
-                        tmem_ld<TPT>(oaddr, r);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int j = 0; j < TPT; ++j) v[j] = u2f(r[j]) * u2f(r[j]);
-                    }
-                    warp_transpose_sum<TPT>(v, lane);
-#pragma unroll
-                    for (int j = 0; j < TPT / 32; ++j) red[(warp * TPT + lane * (TPT / 32) + j) * 2 + 1] = v[j];
                     named_bar_sync(1, kCT);
                     if (tid < C) {
+                        const int gg = tid / HT, tl = tid % HT;
                         float s1 = 0.f, s2 = 0.f;
-                        if (NH == 2) {
 #pragma unroll
-                            for (int w = 0; w < kCW; ++w) {
-                                s1 += red[(w * TPT + tid) * 2];
-                                s2 += red[(w * TPT + tid) * 2 + 1];
-                            }
-                        } else {
-                            const int gg = tid / TPT, tl = tid % TPT;
-#pragma unroll
-                            for (int qq = 0; qq < 4; ++qq) {
-                                s1 += red[((gg * 4 + qq) * TPT + tl) * 2];
-                                s2 += red[((gg * 4 + qq) * TPT + tl) * 2 + 1];
-                            }
+                        for (int qq = 0; qq < 4; ++qq) {
+                            s1 += red[((gg * 4 + qq) * HT + tl) * 2];
+                            s2 += red[((gg * 4 + qq) * HT + tl) * 2 + 1];
                         }
                         const float mean = s1 * (1.0f / DV);
                         const float var = fmaxf(s2 * (1.0f / DV) - mean * mean, 0.f);
-                        stat[2 * tid] = mean;
-                        stat[2 * tid + 1] = rsqrtf(var + p.eps);
+                        const float rstd = rsqrtf(var + p.eps);
+                        stat[tid] = make_float2(rstd, -mean * rstd);
                     }
                     named_bar_sync(1, kCT);
                 }
-                {
-                    uint32_t r[TPT];
-                    tmem_ld<TPT>(oaddr, r);
-                    tmem_wait_ld();
-                    const int dj = d >> 6, dc = (d & 63) >> 3, de = (d & 7) * 2;
 #pragma unroll
-                    for (int j = 0; j < TPT; ++j) {
+                for (int h = 0; h < NH; ++h) {
+                    uint32_t r[HT];
+                    tmem_ld<HT>(oaddr + h * C, r);
+                    tmem_wait_ld();
+                    const int d = h * 128 + q4 * 32 + lane;
+                    const int dj = d >> 6, dc = (d & 63) >> 3, de = (d & 7) * 2;
+                    uint8_t* gcol = Gp + dj * CF::BOX + de;
+#pragma unroll
+                    for (int j = 0; j < HT; ++j) {
                         const int t = t0 + j;
-                        __nv_bfloat16* gp = reinterpret_cast<__nv_bfloat16*>(
-                            Gp + dj * CF::BOX + t * 128 + ((dc ^ (t & 7)) << 4) + de);
+                        __nv_bfloat16* gp = reinterpret_cast<__nv_bfloat16*>(gcol + t * 128 + ((dc ^ (t & 7)) << 4));
                         float o = u2f(r[j]);
                         if (p.gn) {
+                            const float2 st = stat[t];
                             const float gv = __bfloat162float(*gp);
-                            o = (o - stat[2 * t]) * stat[2 * t + 1] * gv / (1.0f + __expf(-gv));
+                            // GroupNorm as one FMA, then swish(g) = g * sigmoid(g)
+                            o = fmaf(o, st.x, st.y) * __fdividef(gv, 1.0f + __expf(-gv));
                         }
                         *gp = __float2bfloat16_rn(o);
                     }
