@@ -47,15 +47,17 @@ namespace {
 using namespace sm100;
 
 constexpr int DK = 128;
-constexpr int kCW = 8;                  // compute warps
-constexpr int kCT = kCW * 32;           // compute threads
-constexpr int kThreadsTC = kCT + 32;    // + one producer warp
+constexpr int kCW = 16;                 // compute warps: four per tensor-memory lane quarter
+constexpr int kCT = kCW * 32;           // threads per CTA (thread 0 also issues loads and MMAs)
+constexpr float kLazyMax = 40.0f;       // largest exponent the lazy state scale may reach
 
 template <int DV, int C>
 struct Cfg {
     static constexpr int NH = DV / 128;                     // d_v halves (MMA M = 128 each)
-    static constexpr int NS = (DV == 128 && C == 128) ? 1 : 2;  // Q/K/V stages
-    static constexpr int NG = 2;                            // G/O stages
+    static constexpr bool TF32 = (C == 64);                 // inter-chunk product in tf32
+    static constexpr int NQK = 2;                           // Q/K stages
+    static constexpr int NV = (DV == 128 && C == 64) ? 2 : 1;   // V stages
+    static constexpr int NG = (C == 128) ? 1 : 2;           // G/O stages
     static constexpr int ROWB = 128;                        // bytes per swizzled row
     static constexpr int BOX = C * ROWB;                    // one [C x 64] bf16 box
     static constexpr int Q_BYTES = 2 * BOX;                 // d_k = 128 -> 2 boxes
@@ -63,33 +65,39 @@ struct Cfg {
     static constexpr int V_BYTES = (DV / 64) * BOX;
     static constexpr int G_BYTES = (DV / 64) * BOX;
     static constexpr int P_BYTES = (C / 64) * BOX;          // rows t, C bf16 of s
-    static constexpr int HT = C / 2;                        // tokens per thread, epilogue
+    static constexpr int QT_BYTES = TF32 ? 4 * BOX : 0;     // rows t, 128 fp32 of k
+    static constexpr int HT = C / 4;                        // tokens per thread, epilogue
+    static constexpr int W = NH * 32;                       // state columns per thread
     // tensor-memory columns
-    static constexpr int TM_S = 0;                          // S^T: NH x 128 fp32 columns
+    static constexpr int TM_S = 0;                          // T^T: NH x 128 fp32
     static constexpr int TM_O = NH * 128;                   // O^T: NH x C
-    static constexpr int TM_X = NH * 128 + NH * C;          // scores (C) / bf16 S^T (NH x 64)
-    static constexpr int X_COLS = (C > NH * 64) ? C : NH * 64;
-    static constexpr int TM_USED = TM_X + X_COLS;
+    static constexpr int TM_SC = TM_O + NH * C;             // scores: C
+    static constexpr int TM_CP = TM_SC + C;                 // bf16 copy of T^T (bf16 mode): NH x 64
+    static constexpr int TM_USED = TM_CP + (TF32 ? 0 : NH * 64);
     static constexpr int TM_ALLOC = TM_USED <= 256 ? 256 : 512;
-    // shared-memory layout (bytes from a 1024-aligned base)
+    // shared memory (bytes from a 1024-aligned base)
     static constexpr int OFF_Q = 0;
-    static constexpr int OFF_K = OFF_Q + NS * Q_BYTES;
-    static constexpr int OFF_V = OFF_K + NS * K_BYTES;
-    static constexpr int OFF_G = OFF_V + NS * V_BYTES;
+    static constexpr int OFF_K = OFF_Q + NQK * Q_BYTES;
+    static constexpr int OFF_V = OFF_K + NQK * K_BYTES;
+    static constexpr int OFF_G = OFF_V + NV * V_BYTES;
     static constexpr int OFF_P = OFF_G + NG * G_BYTES;
-    static constexpr int OFF_B = OFF_P + P_BYTES;           // NS x C fp32 decay sums
-    static constexpr int OFF_RED = OFF_B + NS * C * 4;      // kCW x HT x 2 fp32
-    static constexpr int OFF_STAT = OFF_RED + kCW * HT * 2 * 4;   // C x (rstd, -mean * rstd)
-    static constexpr int OFF_BAR = OFF_STAT + C * 8;
-    static constexpr int NUM_BARS = 2 * NS + 2 * NG + 2;
+    static constexpr int OFF_QT = OFF_P + P_BYTES;
+    static constexpr int OFF_B = OFF_QT + QT_BYTES;         // NQK x C fp32 decay sums
+    static constexpr int OFF_BAR = OFF_B + NQK * C * 4;
+    static constexpr int NUM_BARS = NQK + NV + NG + 3;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int SMEM = OFF_MISC + 16 + 1024;      // + alignment slack
+    // epilogue scratch lives in the P buffer (P is dead during the epilogue)
+    static constexpr int OFF_RED = OFF_P;                   // kCW x HT x 2 fp32
+    static constexpr int OFF_STAT = OFF_P + kCW * HT * 2 * 4;  // C x (rstd, -mean * rstd)
+    static_assert(kCW * HT * 8 + C * 8 <= P_BYTES, "epilogue scratch fits in P");
     static_assert(TM_USED <= 512, "tensor memory budget");
     static_assert(SMEM <= 227 * 1024, "shared memory budget");
-    static_assert(C % 32 == 0 && C <= 128, "chunk");
-    // the padded rows (C..127) of the 128-row scores A operand must stay in
-    // the allocation: they read the bytes after the last Q stage's boxes.
-    static_assert(OFF_K + 2 * (128 - C) * ROWB <= SMEM, "scores padding rows");
+    static_assert(C == 64 || C == 128, "chunk");
+    static_assert(TF32 || NH == 1, "bf16 copy mode is laid out for one d_v half");
+    // the padded rows (C..127) of the 128-row scores A operand read the bytes
+    // after a Q stage's second box: the next Q stage or the first K stage.
+    static_assert(OFF_K + (128 - C) * ROWB <= OFF_V, "scores padding rows stay in the allocation");
 };
 
 struct TcParams {
@@ -128,30 +136,66 @@ __device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t (&r)[N]) {
     else tmem_ld_x64(taddr, r);
 }
 
-// Sum each of the N values of a lane over the 32 lanes of the warp; on return
-// v[j], j < N / 32, holds the total for value index lane * (N / 32) + j.
 template <int N>
-__device__ __forceinline__ void warp_transpose_sum(float (&v)[N], int lane) {
+__device__ __forceinline__ void tmem_st(uint32_t taddr, const uint32_t (&r)[N]) {
+    if constexpr (N == 16) tmem_st_x16(taddr, r);
+    else if constexpr (N == 32) tmem_st_x32(taddr, r);
+    else tmem_st_x64(taddr, r);
+}
+
+// One halving step of the cross-lane transpose-sum: lanes with bit OFF set
+// keep the upper N/2 values, the others the lower N/2, and each adds its
+// partner's copy of the half it keeps.
+template <int N, int OFF>
+__device__ __forceinline__ void transpose_sum_step(float (&v)[N], int lane) {
+    if constexpr (OFF >= 1) {
+        if constexpr (N >= 2) {
+            constexpr int n = N / 2;
+            const bool up = (lane & OFF) != 0;
 #pragma unroll
-    for (int off = 16, n = N / 2; off >= 1; off >>= 1, n >>= 1) {
-        const bool up = (lane & off) != 0;
-#pragma unroll
-        for (int j = 0; j < n; ++j) {
-            float send = up ? v[j] : v[j + n];
-            float keep = up ? v[j + n] : v[j];
-            v[j] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+            for (int j = 0; j < n; ++j) {
+                const float send = up ? v[j] : v[j + n];
+                const float keep = up ? v[j + n] : v[j];
+                v[j] = keep + __shfl_xor_sync(0xffffffffu, send, OFF);
+            }
+            transpose_sum_step<(n > 1 ? n : 1), OFF / 2>(reinterpret_cast<float(&)[(n > 1 ? n : 1)]>(v), lane);
+        } else {
+            v[0] += __shfl_xor_sync(0xffffffffu, v[0], OFF);
+            transpose_sum_step<1, OFF / 2>(v, lane);
         }
     }
 }
 
+// Sum each of the N values of a lane over the 32 lanes of the warp.  On
+// return, for N >= 32, v[j] (j < N / 32) holds the total of value index
+// lane * (N / 32) + j; for N = 16, v[0] holds the total of index lane >> 1.
+template <int N>
+__device__ __forceinline__ void warp_transpose_sum(float (&v)[N], int lane) {
+    static_assert(N == 16 || N % 32 == 0, "values per lane");
+    transpose_sum_step<N, 16>(v, lane);
+}
+
+// Fused chunk loop (kFull) or state-only pass (!kFull) for one (unit, segment).
+//
+// State scaling.  Tensor memory holds T = S / E with E = e^Lambda, Lambda <= 0
+// and the same in every thread.  A chunk is "lazy" when its largest K scale
+// e^{-b_s - Lambda} stays within e^kLazyMax: then K~_s = e^{-b_s - Lambda} K_s,
+// T += V^T K~ and Lambda += b_C, and T itself is not touched.  Otherwise the
+// chunk is "eager": T is rescaled in place by e^{Lambda + b_C},
+// K~_s = e^{b_C - b_s} K_s and Lambda = 0.  The inter-chunk read uses
+// Q~_t = e^{b_t + Lambda} Q_t against T, and the state leaves as e^Lambda T.
 template <int DV, int C, bool kFull>
-__global__ void __launch_bounds__(kThreadsTC, 1) prefill_tc_kernel(const __grid_constant__ TcParams p) {
+__global__ void __launch_bounds__(kCT, 1) prefill_tc_kernel(const __grid_constant__ TcParams p) {
     using CF = Cfg<DV, C>;
-    constexpr int NS = CF::NS, NG = CF::NG, NH = CF::NH;
+    constexpr int NQK = CF::NQK, NV = CF::NV, NG = CF::NG, NH = CF::NH, W = CF::W, HT = CF::HT;
+    constexpr bool TF32 = CF::TF32;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int q4 = warp & 3;       // tensor-memory lane quarter of this warp
+    const int grp = warp >> 2;     // which of the four warps sharing the quarter
+    const uint32_t lq = (uint32_t)(32 * q4) << 16;
 
     const int nseg = kFull ? p.P : p.P - 1;
     const int u = blockIdx.x / nseg, seg = blockIdx.x % nseg;
@@ -160,7 +204,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1) prefill_tc_kernel(const __grid_
     const int n_end = min(p.N, n_begin + p.seg_len);
     const int nchunks = (n_end - n_begin + C - 1) / C;
 
-    const int BF = 0, BE = NS, BGF = 2 * NS, BGE = 2 * NS + NG, BSC = 2 * NS + 2 * NG, BMMA = BSC + 1;
+    const int BQK = 0, BV = NQK, BG = NQK + NV, BSC = NQK + NV + NG, BO = BSC + 1, BMMA = BSC + 2;
     auto bar = [&](int i) -> uint32_t { return sb + CF::OFF_BAR + 8 * i; };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + CF::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + CF::OFF_MISC + 4);
@@ -186,319 +230,372 @@ __global__ void __launch_bounds__(kThreadsTC, 1) prefill_tc_kernel(const __grid_
     tc_fence_after();
     const uint32_t tm = *tmem_slot;
 
-    if (warp == kCW) {
-        // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            int iq = 0, ig = (kFull && p.has_g) ? 0 : nchunks;
-            while (iq < nchunks || ig < nchunks) {
-                const bool do_q = iq < nchunks && (ig >= nchunks || iq <= ig + (NS - 1));
-                if (do_q) {
-                    const int s = iq % NS;
-                    if (!mbar_wait(bar(BE + s), ((iq / NS) & 1) ^ 1, p.status, abort_flag)) break;
-                    const int n0 = n_begin + iq * C;
-                    const uint32_t bytes = CF::K_BYTES + CF::V_BYTES + C * 4 + (kFull ? CF::Q_BYTES : 0);
-                    const uint32_t fb = bar(BF + s);
-                    mbar_arrive_expect_tx(fb, bytes);
-                    if (kFull) {
-                        for (int j = 0; j < 2; ++j)
-                            tma_load_4d(sb + CF::OFF_Q + s * CF::Q_BYTES + j * CF::BOX, &p.tmQ, j * 64, hh, n0, bb, fb);
+    // ---- loads and MMAs, all issued by thread 0
+    auto issue_qk = [&](int j) {
+        const int s = j % NQK, n0 = n_begin + j * C;
+        const uint32_t fb = bar(BQK + s);
+        mbar_arrive_expect_tx(fb, CF::K_BYTES + C * 4 + (kFull ? CF::Q_BYTES : 0));
+        if (kFull)
+            for (int x = 0; x < 2; ++x)
+                tma_load_4d(sb + CF::OFF_Q + s * CF::Q_BYTES + x * CF::BOX, &p.tmQ, x * 64, hh, n0, bb, fb);
+        for (int x = 0; x < 2; ++x)
+            tma_load_4d(sb + CF::OFF_K + s * CF::K_BYTES + x * CF::BOX, &p.tmK, x * 64, hh, n0, bb, fb);
+        bulk_load(sb + CF::OFF_B + s * C * 4, p.bcum + (size_t)u * p.Npad + n0, C * 4, fb);
+    };
+    auto issue_v = [&](int j) {
+        const int s = j % NV, n0 = n_begin + j * C;
+        const uint32_t fb = bar(BV + s);
+        mbar_arrive_expect_tx(fb, CF::V_BYTES);
+        for (int x = 0; x < DV / 64; ++x)
+            tma_load_4d(sb + CF::OFF_V + s * CF::V_BYTES + x * CF::BOX, &p.tmV, x * 64, hh, n0, bb, fb);
+    };
+    auto issue_g = [&](int j) {
+        const int s = j % NG, n0 = n_begin + j * C;
+        const uint32_t fb = bar(BG + s);
+        mbar_arrive_expect_tx(fb, CF::G_BYTES);
+        for (int x = 0; x < DV / 64; ++x)
+            tma_load_4d(sb + CF::OFF_G + s * CF::G_BYTES + x * CF::BOX, &p.tmG, x * 64, hh, n0, bb, fb);
+    };
+    // scores D[t][s] = Q K^T over d_k (M = 128 rows of t; rows >= C unused)
+    auto issue_scores = [&](int j) {
+        const int s = j % NQK;
+        mbar_wait(bar(BQK + s), (j / NQK) & 1, p.status, abort_flag);
+        tc_fence_after();
+        const uint32_t sQ = sb + CF::OFF_Q + s * CF::Q_BYTES, sK = sb + CF::OFF_K + s * CF::K_BYTES;
+        constexpr uint32_t id = idesc_bf16(128, C, false, false);
+#pragma unroll
+        for (int k = 0; k < DK / 16; ++k) {
+            const uint32_t off = (k >> 2) * CF::BOX + (k & 3) * 32;
+            mma_ss(tm + CF::TM_SC, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(sK + off, 16, 1024), id, k > 0);
+        }
+        mma_commit(bar(BSC));
+    };
+    // T^T += V^T K~ for both d_v halves
+    auto issue_state = [&](uint32_t sV, uint32_t sK) {
+        constexpr uint32_t id_kv = idesc_bf16(128, DK, true, true);
+#pragma unroll
+        for (int h = 0; h < NH; ++h) {
+#pragma unroll
+            for (int k = 0; k < C / 16; ++k)
+                mma_ss(tm + CF::TM_S + h * 128, sdesc_sw128(sV + 2 * h * CF::BOX + k * 2048, CF::BOX, 1024),
+                       sdesc_sw128(sK + k * 2048, CF::BOX, 1024), id_kv, 1);
+        }
+    };
+
+    if (tid == 0) {
+        issue_qk(0);
+        if (nchunks > 1) issue_qk(1);
+        issue_v(0);
+        if (NV == 2 && nchunks > 1) issue_v(1);
+        if (kFull && p.has_g) {
+            issue_g(0);
+            if (NG == 2 && nchunks > 1) issue_g(1);
+        }
+        if (kFull) issue_scores(0);
+    }
+
+    // this thread's slice of T^T: lanes of quarter q4, columns col0 .. col0 + W - 1
+    const int col0 = grp * W;
+    const int s_half = col0 / 128, s_k0 = col0 % 128;
+    const int s_d = s_half * 128 + q4 * 32 + lane;
+    {
+        uint32_t r[W];
+        if (kFull && seg > 0) {
+            const float* src = p.seg_state + ((size_t)u * (p.P - 1) + (seg - 1)) * DV * DK + (size_t)s_d * DK + s_k0;
+            const float4* s4 = reinterpret_cast<const float4*>(src);
+#pragma unroll
+            for (int j = 0; j < W / 4; ++j) {
+                const float4 v = s4[j];
+                r[4 * j] = f2u(v.x); r[4 * j + 1] = f2u(v.y); r[4 * j + 2] = f2u(v.z); r[4 * j + 3] = f2u(v.w);
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < W; ++j) r[j] = 0u;
+        }
+        tmem_st<W>(tm + lq + CF::TM_S + col0, r);
+        tmem_wait_st();
+    }
+
+    float lam = 0.f;          // Lambda
+    float seg_decay = 0.f;
+    uint32_t eager_count = 0;
+    for (int i = 0; i < nchunks; ++i) {
+        const int sq = i % NQK, sv = i % NV;
+        const uint32_t sQ = sb + CF::OFF_Q + sq * CF::Q_BYTES;
+        const uint32_t sK = sb + CF::OFF_K + sq * CF::K_BYTES;
+        const uint32_t sV = sb + CF::OFF_V + sv * CF::V_BYTES;
+        const float* bc = reinterpret_cast<const float*>(sm + CF::OFF_B + sq * C * 4);
+        mbar_wait(bar(BQK + sq), (i / NQK) & 1, p.status, abort_flag);
+        const float bC = bc[C - 1];
+        const bool eager = (-bC - lam) > kLazyMax;
+
+        if (kFull) {
+            mbar_wait(bar(BSC), i & 1, p.status, abort_flag);
+            tc_fence_after();
+            // P[t][s] = A[t][s] e^{b_t - b_s} (s <= t) -> bf16, K-major rows t
+            if (q4 * 32 < C) {
+                constexpr int PC = C / 4;
+                const int t = q4 * 32 + lane;
+                uint32_t r[PC];
+                tmem_ld<PC>(tm + lq + CF::TM_SC + grp * PC, r);
+                tmem_wait_ld();
+                const float bt = bc[t];
+#pragma unroll
+                for (int c8 = 0; c8 < PC / 8; ++c8) {
+                    const int s0 = grp * PC + c8 * 8;
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int sa = s0 + 2 * e, sb2 = sa + 1;
+                        const float v0 = sa <= t ? u2f(r[c8 * 8 + 2 * e]) * __expf(bt - bc[sa]) : 0.f;
+                        const float v1 = sb2 <= t ? u2f(r[c8 * 8 + 2 * e + 1]) * __expf(bt - bc[sb2]) : 0.f;
+                        w[e] = pack_bf16x2(v0, v1);
                     }
-                    for (int j = 0; j < 2; ++j)
-                        tma_load_4d(sb + CF::OFF_K + s * CF::K_BYTES + j * CF::BOX, &p.tmK, j * 64, hh, n0, bb, fb);
-                    for (int j = 0; j < DV / 64; ++j)
-                        tma_load_4d(sb + CF::OFF_V + s * CF::V_BYTES + j * CF::BOX, &p.tmV, j * 64, hh, n0, bb, fb);
-                    bulk_load(sb + CF::OFF_B + s * C * 4, p.bcum + (size_t)u * p.Npad + n0, C * 4, fb);
-                    ++iq;
-                } else {
-                    const int g = ig % NG;
-                    if (!mbar_wait(bar(BGE + g), ((ig / NG) & 1) ^ 1, p.status, abort_flag)) break;
-                    const int n0 = n_begin + ig * C;
-                    const uint32_t gb = bar(BGF + g);
-                    mbar_arrive_expect_tx(gb, CF::G_BYTES);
-                    for (int j = 0; j < DV / 64; ++j)
-                        tma_load_4d(sb + CF::OFF_G + g * CF::G_BYTES + j * CF::BOX, &p.tmG, j * 64, hh, n0, bb, gb);
-                    ++ig;
+                    const int region = s0 >> 6, chunk = (s0 & 63) >> 3;
+                    uint8_t* dst = sm + CF::OFF_P + region * CF::BOX + t * 128 + ((chunk ^ (t & 7)) << 4);
+                    *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+            // Q~ = e^{b_t + Lambda} Q: fp32 copy (tf32 mode) or in place (bf16 mode)
+            uint8_t* Qp = sm + CF::OFF_Q + sq * CF::Q_BYTES;
+            if constexpr (TF32) {
+                uint8_t* QT = sm + CF::OFF_QT;
+                for (int ci = tid; ci < C * 16; ci += kCT) {
+                    const int t = ci >> 4, c = ci & 15;    // row t, bf16 16-byte chunk c (d_k 8c .. 8c+7)
+                    const float f = __expf(bc[t] + lam);
+                    const uint4 w = *reinterpret_cast<const uint4*>(Qp + (c >> 3) * CF::BOX + t * 128 +
+                                                                    (((c & 7) ^ (t & 7)) << 4));
+                    const uint32_t* e = reinterpret_cast<const uint32_t*>(&w);
+                    float x[8];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&e[j]));
+                        x[2 * j] = f2.x * f;
+                        x[2 * j + 1] = f2.y * f;
+                    }
+                    uint8_t* row = QT + (c >> 2) * CF::BOX + t * 128;
+                    const int lc = 2 * (c & 3);
+                    *reinterpret_cast<float4*>(row + ((lc ^ (t & 7)) << 4)) = make_float4(x[0], x[1], x[2], x[3]);
+                    *reinterpret_cast<float4*>(row + (((lc + 1) ^ (t & 7)) << 4)) =
+                        make_float4(x[4], x[5], x[6], x[7]);
+                }
+            } else {
+                for (int ci = tid; ci < C * 16; ci += kCT) {
+                    const int row = (ci >> 3) % C;
+                    scale_bf16x8(Qp + ci * 16, __expf(bc[row] + lam));
                 }
             }
         }
-    } else {
-        // ------------------------------------------------------------ compute warps
-        const int q4 = warp & 3;       // tensor-memory lane quarter of this warp
-        const int grp = warp >> 2;     // which of the two warps sharing the quarter
-        const uint32_t lq = (uint32_t)(32 * q4) << 16;
-
-        // Initial state S^T: zero, or the segment's S_in.
+        // K~: e^{-b_s - Lambda} (lazy) or e^{b_C - b_s} (eager), in place
         {
-            const float* src = nullptr;
-            if (kFull && seg > 0) src = p.seg_state + ((size_t)u * (p.P - 1) + (seg - 1)) * DV * DK;
+            uint8_t* Kp = sm + CF::OFF_K + sq * CF::K_BYTES;
+            for (int ci = tid; ci < C * 16; ci += kCT) {
+                const int row = (ci >> 3) % C;
+                const float ex = eager ? (bC - bc[row]) : (-bc[row] - lam);
+                scale_bf16x8(Kp + ci * 16, __expf(ex));
+            }
+        }
+        // pass over T before the MMAs: bf16 copy (bf16 mode) and / or eager rescale
+        const float escale = __expf(lam + bC);
+        if (kFull ? !TF32 : eager) {
+            uint32_t r[W];
+            tmem_ld<W>(tm + lq + CF::TM_S + col0, r);
+            tmem_wait_ld();
+            if constexpr (kFull && !TF32) {
+                uint32_t pk[W / 2];
 #pragma unroll
-            for (int cb = 0; cb < (NH == 2 ? 2 : 1); ++cb) {
-                const int half = NH == 2 ? grp : 0;
-                const int k0 = NH == 2 ? cb * 64 : grp * 64;
-                const int d = half * 128 + q4 * 32 + lane;
-                uint32_t r[64];
-                if (src) {
-                    const float4* s4 = reinterpret_cast<const float4*>(src + (size_t)d * DK + k0);
+                for (int j = 0; j < W / 2; ++j) pk[j] = pack_bf16x2(u2f(r[2 * j]), u2f(r[2 * j + 1]));
+                tmem_st<W / 2>(tm + lq + CF::TM_CP + col0 / 2, pk);
+            }
+            if (eager) {
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        float4 v = s4[j];
-                        r[4 * j] = f2u(v.x); r[4 * j + 1] = f2u(v.y); r[4 * j + 2] = f2u(v.z); r[4 * j + 3] = f2u(v.w);
-                    }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 64; ++j) r[j] = 0u;
-                }
-                tmem_st_x64(tm + lq + CF::TM_S + half * 128 + k0, r);
+                for (int j = 0; j < W; ++j) r[j] = f2u(u2f(r[j]) * escale);
+                tmem_st<W>(tm + lq + CF::TM_S + col0, r);
             }
             tmem_wait_st();
         }
-
-        float seg_decay = 0.f;
-        for (int i = 0; i < nchunks; ++i) {
-            const int s = i % NS;
-            const uint32_t sQ = sb + CF::OFF_Q + s * CF::Q_BYTES;
-            const uint32_t sK = sb + CF::OFF_K + s * CF::K_BYTES;
-            const uint32_t sV = sb + CF::OFF_V + s * CF::V_BYTES;
-            const float* bc = reinterpret_cast<const float*>(sm + CF::OFF_B + s * C * 4);
-            mbar_wait(bar(BF + s), (i / NS) & 1, p.status, abort_flag);
-            const float bC = bc[C - 1];
-
-            if (kFull) {
-                // scores D[t][s] = Q K^T over d_k (M = 128 rows of t; rows >= C unused)
-                if (tid == 0) {
-                    tc_fence_after();
-                    constexpr uint32_t id = idesc_bf16(128, C, false, false);
-#pragma unroll
-                    for (int k = 0; k < DK / 16; ++k) {
-                        const uint32_t off = (k >> 2) * CF::BOX + (k & 3) * 32;
-                        mma_ss(tm + CF::TM_X, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(sK + off, 16, 1024), id,
-                               k > 0);
-                    }
-                    mma_commit(bar(BSC));
-                }
-                mbar_wait(bar(BSC), i & 1, p.status, abort_flag);
-                tc_fence_after();
-                // P[t][s] = A[t][s] e^{b_t - b_s} (s <= t) -> bf16, K-major rows t
-                if (q4 * 32 < C) {
-                    constexpr int HC = C / 2;
-                    const int t = q4 * 32 + lane;
-                    uint32_t r[HC];
-                    tmem_ld<HC>(tm + lq + CF::TM_X + grp * HC, r);
-                    tmem_wait_ld();
-                    const float bt = bc[t];
-#pragma unroll
-                    for (int c8 = 0; c8 < HC / 8; ++c8) {
-                        const int s0 = grp * HC + c8 * 8;
-                        uint32_t w[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int sa = s0 + 2 * e, sb2 = sa + 1;
-                            const float v0 = sa <= t ? u2f(r[c8 * 8 + 2 * e]) * __expf(bt - bc[sa]) : 0.f;
-                            const float v1 = sb2 <= t ? u2f(r[c8 * 8 + 2 * e + 1]) * __expf(bt - bc[sb2]) : 0.f;
-                            w[e] = pack_bf16x2(v0, v1);
-                        }
-                        const int region = s0 >> 6, chunk = (s0 & 63) >> 3;
-                        uint8_t* dst = sm + CF::OFF_P + region * CF::BOX + t * 128 + ((chunk ^ (t & 7)) << 4);
-                        *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
-                    }
-                }
-            }
-            // K~ = diag(e^{b_C - b_s}) K and Q~ = diag(e^{b_t}) Q, in place.
-            {
-                uint8_t* Kp = sm + CF::OFF_K + s * CF::K_BYTES;
-                for (int ci = tid; ci < C * 16; ci += kCT) {
-                    const int row = (ci >> 3) % C;
-                    scale_bf16x8(Kp + ci * 16, __expf(bC - bc[row]));
-                }
-                if (kFull) {
-                    uint8_t* Qp = sm + CF::OFF_Q + s * CF::Q_BYTES;
-                    for (int ci = tid; ci < C * 16; ci += kCT) {
-                        const int row = (ci >> 3) % C;
-                        scale_bf16x8(Qp + ci * 16, __expf(bc[row]));
-                    }
-                }
-            }
-            tc_fence_before();
-            named_bar_sync(1, kCT);   // every read of the scores is done
+        fence_proxy_async_smem();
+        tc_fence_before();
+        named_bar_sync(1, kCT);
+        const bool split = kFull && TF32 && eager;   // rescale T between the inter read and the state MMA
+        if (tid == 0) {
             tc_fence_after();
-            // bf16 copy of S^T (A operand of the inter-chunk product), then S^T *= e^{b_C}
-            {
-                const float eC = __expf(bC);
+            mbar_wait(bar(BV + sv), (i / NV) & 1, p.status, abort_flag);
+            if (kFull) {
+                constexpr uint32_t id_pv = idesc_bf16(128, C, true, false);
+                constexpr uint32_t id_qs = idesc_bf16(128, C, false, false);
+                constexpr uint32_t id_qs32 = idesc_tf32(128, C, false, false);
 #pragma unroll
-                for (int cb = 0; cb < (NH == 2 ? 2 : 1); ++cb) {
-                    const int half = NH == 2 ? grp : 0;
-                    const int k0 = NH == 2 ? cb * 64 : grp * 64;
-                    uint32_t r[64];
-                    tmem_ld_x64(tm + lq + CF::TM_S + half * 128 + k0, r);
-                    tmem_wait_ld();
-                    if (kFull) {
-                        uint32_t pk[32];
+                for (int h = 0; h < NH; ++h) {
+                    const uint32_t vA = sV + 2 * h * CF::BOX;   // d_v rows h*128 .. +127 (two boxes)
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) pk[j] = pack_bf16x2(u2f(r[2 * j]), u2f(r[2 * j + 1]));
-                        tmem_st_x32(tm + lq + CF::TM_X + half * 64 + k0 / 2, pk);
+                    for (int k = 0; k < C / 16; ++k) {
+                        const uint32_t poff = (k >> 2) * CF::BOX + (k & 3) * 32;
+                        mma_ss(tm + CF::TM_O + h * C, sdesc_sw128(vA + k * 2048, CF::BOX, 1024),
+                               sdesc_sw128(sb + CF::OFF_P + poff, 16, 1024), id_pv, k > 0);
                     }
+                    if constexpr (TF32) {
 #pragma unroll
-                    for (int j = 0; j < 64; ++j) r[j] = f2u(u2f(r[j]) * eC);
-                    tmem_st_x64(tm + lq + CF::TM_S + half * 128 + k0, r);
+                        for (int k = 0; k < DK / 8; ++k) {
+                            const uint32_t qoff = (k >> 2) * CF::BOX + (k & 3) * 32;
+                            mma_ts_tf32(tm + CF::TM_O + h * C, tm + CF::TM_S + h * 128 + k * 8,
+                                        sdesc_sw128(sb + CF::OFF_QT + qoff, 16, 1024), id_qs32, 1);
+                        }
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < DK / 16; ++k) {
+                            const uint32_t qoff = (k >> 2) * CF::BOX + (k & 3) * 32;
+                            mma_ts(tm + CF::TM_O + h * C, tm + CF::TM_CP + h * 64 + k * 8,
+                                   sdesc_sw128(sQ + qoff, 16, 1024), id_qs, 1);
+                        }
+                    }
                 }
-                tmem_wait_st();
+                if (split) mma_commit(bar(BO));
             }
-            fence_proxy_async_smem();
+            if (!split) {
+                issue_state(sV, sK);
+                mma_commit(bar(BMMA));
+                if (kFull && i + 1 < nchunks) issue_scores(i + 1);
+            }
+        }
+        if (split) {
+            mbar_wait(bar(BO), eager_count & 1, p.status, abort_flag);
+            tc_fence_after();
+            uint32_t r[W];
+            tmem_ld<W>(tm + lq + CF::TM_S + col0, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < W; ++j) r[j] = f2u(u2f(r[j]) * escale);
+            tmem_st<W>(tm + lq + CF::TM_S + col0, r);
+            tmem_wait_st();
             tc_fence_before();
             named_bar_sync(1, kCT);
             if (tid == 0) {
                 tc_fence_after();
-#pragma unroll
-                for (int h = 0; h < NH; ++h) {
-                    const uint32_t vA = sV + 2 * h * CF::BOX;   // d_v rows h*128 .. +127 (two boxes)
-                    if (kFull) {
-                        constexpr uint32_t id_pv = idesc_bf16(128, C, true, false);
-#pragma unroll
-                        for (int k = 0; k < C / 16; ++k) {
-                            const uint32_t poff = (k >> 2) * CF::BOX + (k & 3) * 32;
-                            mma_ss(tm + CF::TM_O + h * C, sdesc_sw128(vA + k * 2048, CF::BOX, 1024),
-                                   sdesc_sw128(sb + CF::OFF_P + poff, 16, 1024), id_pv, k > 0);
-                        }
-                        constexpr uint32_t id_qs = idesc_bf16(128, C, false, false);
-#pragma unroll
-                        for (int k = 0; k < DK / 16; ++k) {
-                            const uint32_t qoff = (k >> 2) * CF::BOX + (k & 3) * 32;
-                            mma_ts(tm + CF::TM_O + h * C, tm + CF::TM_X + h * 64 + k * 8,
-                                   sdesc_sw128(sQ + qoff, 16, 1024), id_qs, 1);
-                        }
-                    }
-                    constexpr uint32_t id_kv = idesc_bf16(128, DK, true, true);
-#pragma unroll
-                    for (int k = 0; k < C / 16; ++k) {
-                        mma_ss(tm + CF::TM_S + h * 128, sdesc_sw128(vA + k * 2048, CF::BOX, 1024),
-                               sdesc_sw128(sK + k * 2048, CF::BOX, 1024), id_kv, 1);
-                    }
-                }
+                issue_state(sV, sK);
                 mma_commit(bar(BMMA));
-                mma_commit(bar(BE + s));   // frees this Q/K/V stage for the producer
+                if (i + 1 < nchunks) issue_scores(i + 1);
             }
-            seg_decay += bC;
-            mbar_wait(bar(BMMA), i & 1, p.status, abort_flag);
-            tc_fence_after();
-
-            if (kFull) {
-                // ---------------------------------------------------- epilogue
-                // Thread (q4, grp, lane) owns d_v channels h*128 + q4*32 + lane
-                // (h < NH) for tokens grp*HT .. grp*HT + HT - 1.
-                constexpr int HT = CF::HT;
-                const int g = i % NG;
-                if (p.has_g) mbar_wait(bar(BGF + g), (i / NG) & 1, p.status, abort_flag);
-                uint8_t* Gp = sm + CF::OFF_G + g * CF::G_BYTES;
-                const int t0 = grp * HT;
-                const uint32_t oaddr = tm + lq + CF::TM_O + t0;
-                float* red = reinterpret_cast<float*>(sm + CF::OFF_RED);
-                float2* stat = reinterpret_cast<float2*>(sm + CF::OFF_STAT);
-                if (p.gn) {
-                    // per-token sums over this thread's channels, then over the
-                    // warp's lanes, then over the four lane quarters
-#pragma unroll
-                    for (int pass = 0; pass < 2; ++pass) {
-                        float v[HT];
-#pragma unroll
-                        for (int h = 0; h < NH; ++h) {
-                            uint32_t r[HT];
-                            tmem_ld<HT>(oaddr + h * C, r);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int j = 0; j < HT; ++j) {
-                                const float y = u2f(r[j]);
-                                const float x = pass == 0 ? y : y * y;
-                                v[j] = h == 0 ? x : v[j] + x;
-                            }
-                        }
-                        warp_transpose_sum<HT>(v, lane);
-#pragma unroll
-                        for (int j = 0; j < HT / 32; ++j) red[(warp * HT + lane * (HT / 32) + j) * 2 + pass] = v[j];
-                    }
-                    named_bar_sync(1, kCT);
-                    if (tid < C) {
-                        const int gg = tid / HT, tl = tid % HT;
-                        float s1 = 0.f, s2 = 0.f;
-#pragma unroll
-                        for (int qq = 0; qq < 4; ++qq) {
-                            s1 += red[((gg * 4 + qq) * HT + tl) * 2];
-                            s2 += red[((gg * 4 + qq) * HT + tl) * 2 + 1];
-                        }
-                        const float mean = s1 * (1.0f / DV);
-                        const float var = fmaxf(s2 * (1.0f / DV) - mean * mean, 0.f);
-                        const float rstd = rsqrtf(var + p.eps);
-                        stat[tid] = make_float2(rstd, -mean * rstd);
-                    }
-                    named_bar_sync(1, kCT);
-                }
-#pragma unroll
-                for (int h = 0; h < NH; ++h) {
-                    uint32_t r[HT];
-                    tmem_ld<HT>(oaddr + h * C, r);
-                    tmem_wait_ld();
-                    const int d = h * 128 + q4 * 32 + lane;
-                    const int dj = d >> 6, dc = (d & 63) >> 3, de = (d & 7) * 2;
-                    uint8_t* gcol = Gp + dj * CF::BOX + de;
-#pragma unroll
-                    for (int j = 0; j < HT; ++j) {
-                        const int t = t0 + j;
-                        __nv_bfloat16* gp = reinterpret_cast<__nv_bfloat16*>(gcol + t * 128 + ((dc ^ (t & 7)) << 4));
-                        float o = u2f(r[j]);
-                        if (p.gn) {
-                            const float2 st = stat[t];
-                            const float gv = __bfloat162float(*gp);
-                            // GroupNorm as one FMA, then swish(g) = g * sigmoid(g)
-                            o = fmaf(o, st.x, st.y) * __fdividef(gv, 1.0f + __expf(-gv));
-                        }
-                        *gp = __float2bfloat16_rn(o);
-                    }
-                }
-                tc_fence_before();
-                fence_proxy_async_smem();
-                named_bar_sync(1, kCT);
-                if (tid == 0) {
-                    const int n0 = n_begin + i * C;
-                    for (int j = 0; j < DV / 64; ++j)
-                        tma_store_4d(&p.tmO, smem_u32(Gp + j * CF::BOX), j * 64, hh, n0, bb);
-                    bulk_commit();
-                    bulk_wait_read<1>();   // the store issued one chunk ago has read its buffer
-                    if (i >= 1 && p.has_g) mbar_arrive(bar(BGE + (i - 1) % NG));
-                }
-            }
+            ++eager_count;
+        }
+        seg_decay += bC;
+        lam = eager ? 0.f : lam + bC;
+        mbar_wait(bar(BMMA), i & 1, p.status, abort_flag);
+        tc_fence_after();
+        if (tid == 0) {
+            if (i + NQK < nchunks) issue_qk(i + NQK);   // this Q/K stage is free now
+            if (i + NV < nchunks) issue_v(i + NV);      // and this V stage
         }
 
-        // ---------------------------------------------------------------- state out
         if (kFull) {
-            if (tid == 0) bulk_wait<0>();
+            // ---------------------------------------------------- epilogue
+            // Thread (q4, grp, lane) owns d_v channels h*128 + q4*32 + lane
+            // (h < NH) for tokens grp*HT .. grp*HT + HT - 1.
+            const int g = i % NG;
+            if (p.has_g) mbar_wait(bar(BG + g), (i / NG) & 1, p.status, abort_flag);
+            uint8_t* Gp = sm + CF::OFF_G + g * CF::G_BYTES;
+            const int t0 = grp * HT;
+            const uint32_t oaddr = tm + lq + CF::TM_O + t0;
+            float* red = reinterpret_cast<float*>(sm + CF::OFF_RED);
+            float2* stat = reinterpret_cast<float2*>(sm + CF::OFF_STAT);
+            if (p.gn) {
+                // per-token sums over this thread's channels, then over the
+                // warp's lanes, then over the four lane quarters
+#pragma unroll
+                for (int pass = 0; pass < 2; ++pass) {
+                    float v[HT];
+#pragma unroll
+                    for (int h = 0; h < NH; ++h) {
+                        uint32_t r[HT];
+                        tmem_ld<HT>(oaddr + h * C, r);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < HT; ++j) {
+                            const float y = u2f(r[j]);
+                            const float x = pass == 0 ? y : y * y;
+                            v[j] = h == 0 ? x : v[j] + x;
+                        }
+                    }
+                    warp_transpose_sum<HT>(v, lane);
+                    if constexpr (HT >= 32) {
+#pragma unroll
+                        for (int j = 0; j < HT / 32; ++j) red[(warp * HT + lane * (HT / 32) + j) * 2 + pass] = v[j];
+                    } else {
+                        if ((lane & 1) == 0) red[(warp * HT + (lane >> 1)) * 2 + pass] = v[0];
+                    }
+                }
+                named_bar_sync(1, kCT);
+                if (tid < C) {
+                    const int gg = tid / HT, tl = tid % HT;
+                    float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+                    for (int qq = 0; qq < 4; ++qq) {
+                        s1 += red[((gg * 4 + qq) * HT + tl) * 2];
+                        s2 += red[((gg * 4 + qq) * HT + tl) * 2 + 1];
+                    }
+                    const float mean = s1 * (1.0f / DV);
+                    const float var = fmaxf(s2 * (1.0f / DV) - mean * mean, 0.f);
+                    const float rstd = rsqrtf(var + p.eps);
+                    stat[tid] = make_float2(rstd, -mean * rstd);
+                }
+                named_bar_sync(1, kCT);
+            }
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
+                uint32_t r[HT];
+                tmem_ld<HT>(oaddr + h * C, r);
+                tmem_wait_ld();
+                const int d = h * 128 + q4 * 32 + lane;
+                const int dj = d >> 6, dc = (d & 63) >> 3, de = (d & 7) * 2;
+                uint8_t* gcol = Gp + dj * CF::BOX + de;
+#pragma unroll
+                for (int j = 0; j < HT; ++j) {
+                    const int t = t0 + j;
+                    __nv_bfloat16* gp = reinterpret_cast<__nv_bfloat16*>(gcol + t * 128 + ((dc ^ (t & 7)) << 4));
+                    float o = u2f(r[j]);
+                    if (p.gn) {
+                        const float2 st = stat[t];
+                        const float gv = __bfloat162float(*gp);
+                        // GroupNorm as one FMA, then swish(g) = g * sigmoid(g)
+                        o = fmaf(o, st.x, st.y) * __fdividef(gv, 1.0f + __expf(-gv));
+                    }
+                    *gp = __float2bfloat16_rn(o);
+                }
+            }
+            tc_fence_before();
+            fence_proxy_async_smem();
+            named_bar_sync(1, kCT);
+            if (tid == 0) {
+                const int n0 = n_begin + i * C;
+                for (int x = 0; x < DV / 64; ++x) tma_store_4d(&p.tmO, smem_u32(Gp + x * CF::BOX), x * 64, hh, n0, bb);
+                bulk_commit();
+                bulk_wait_read<NG - 1>();   // every store but the newest has read its buffer
+                const int j = i + 1;
+                if (p.has_g && j >= NG && j < nchunks) issue_g(j);
+            }
+        }
+    }
+
+    // ---------------------------------------------------------------- state out: e^Lambda T
+    {
+        if (kFull && tid == 0) bulk_wait<0>();
+        const float sc = __expf(lam);
+        uint32_t r[W];
+        tmem_ld<W>(tm + lq + CF::TM_S + col0, r);
+        tmem_wait_ld();
+        if (kFull) {
             if (p.S_final && seg == p.P - 1) {
                 float* dst = p.S_final + (size_t)u * DK * DV;
 #pragma unroll
-                for (int cb = 0; cb < (NH == 2 ? 2 : 1); ++cb) {
-                    const int half = NH == 2 ? grp : 0;
-                    const int k0 = NH == 2 ? cb * 64 : grp * 64;
-                    const int d = half * 128 + q4 * 32 + lane;
-                    uint32_t r[64];
-                    tmem_ld_x64(tm + lq + CF::TM_S + half * 128 + k0, r);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < 64; ++j) dst[(size_t)(k0 + j) * DV + d] = u2f(r[j]);
-                }
+                for (int j = 0; j < W; ++j) dst[(size_t)(s_k0 + j) * DV + s_d] = u2f(r[j]) * sc;
             }
         } else {
-            float* dst = p.seg_state + ((size_t)u * (p.P - 1) + seg) * DV * DK;
+            float4* d4 = reinterpret_cast<float4*>(p.seg_state + ((size_t)u * (p.P - 1) + seg) * DV * DK +
+                                                   (size_t)s_d * DK + s_k0);
 #pragma unroll
-            for (int cb = 0; cb < (NH == 2 ? 2 : 1); ++cb) {
-                const int half = NH == 2 ? grp : 0;
-                const int k0 = NH == 2 ? cb * 64 : grp * 64;
-                const int d = half * 128 + q4 * 32 + lane;
-                uint32_t r[64];
-                tmem_ld_x64(tm + lq + CF::TM_S + half * 128 + k0, r);
-                tmem_wait_ld();
-                float4* d4 = reinterpret_cast<float4*>(dst + (size_t)d * DK + k0);
-#pragma unroll
-                for (int j = 0; j < 16; ++j)
-                    d4[j] = make_float4(u2f(r[4 * j]), u2f(r[4 * j + 1]), u2f(r[4 * j + 2]), u2f(r[4 * j + 3]));
-            }
+            for (int j = 0; j < W / 4; ++j)
+                d4[j] = make_float4(u2f(r[4 * j]) * sc, u2f(r[4 * j + 1]) * sc, u2f(r[4 * j + 2]) * sc,
+                                    u2f(r[4 * j + 3]) * sc);
             if (tid == 0) p.seg_decay[(size_t)u * (p.P - 1) + seg] = seg_decay;
         }
     }
@@ -614,13 +711,13 @@ cudaError_t run_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t s) {
     gate_scan_kernel<<<dim3(units, npad / C), C, 0, s>>>(a.z, const_cast<float*>(tp.bcum), a.H, a.N, npad,
                                                          a.inv_tau);
     if (tp.P > 1) {
-        ks<<<units * (tp.P - 1), kThreadsTC, CF::SMEM, s>>>(tp);
+        ks<<<units * (tp.P - 1), kCT, CF::SMEM, s>>>(tp);
         const int elems4 = DV * DK / 4;
         seg_combine_kernel<<<dim3((elems4 + 255) / 256, units), 256, 0, s>>>(tp.seg_state, tp.seg_decay, tp.P,
                                                                              elems4);
     }
     if (g_profile_start) cudaEventRecord(g_profile_start, s);
-    kf<<<units * tp.P, kThreadsTC, CF::SMEM, s>>>(tp);
+    kf<<<units * tp.P, kCT, CF::SMEM, s>>>(tp);
     if (g_profile_stop) cudaEventRecord(g_profile_stop, s);
     return cudaGetLastError();
 }

@@ -102,3 +102,27 @@ def test_full_workload_b1_h32_n65536_dv128():
 @pytest.mark.slow
 def test_full_workload_gate_stress_b2_h16_n32768():
     _full_workload_sampled(gi.C5, [(0, 0), (1, 8), (1, 15)])
+
+
+@pytest.mark.parametrize("dv,chunk", [(256, 64), (128, 128), (128, 64)])
+def test_lazy_and_eager_state_scaling(dv, chunk):
+    """148 units (one segment each, 8-16 chunks): moderate gates (z ~ N(-2,1),
+    log-decay about -8.5 per 64 tokens) run several lazy chunks between eager
+    rescales; the other heads stay near gamma = 1 (lazy throughout)."""
+    H = 148
+    cfg = _cfg(1, H, 1024, dv, chunk, 91, z_dist=tuple((-2.0, 1.0) if h % 2 else (6.0, 1.0) for h in range(H)))
+    path, segs = gret.prefill_path(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, cfg.chunk, gret.Dtype.BF16)
+    assert path == gret.Path.TC and segs == 1
+    inp = gi.prefill_inputs(cfg)
+    d = {k: v.cuda() for k, v in inp.items()}
+    O, Sf = gret.prefill(d["Q"], d["K"], d["V"], d["z"], d["G"], cfg.tau, cfg.chunk, eps=cfg.eps)
+    Y, _ = gret.prefill(d["Q"], d["K"], d["V"], d["z"], None, cfg.tau, cfg.chunk, epilogue="none",
+                        want_state=False)
+    gret.check_device_status()
+    for h in (0, 1, 77, 146, 147):
+        sl = lambda x: x[:, :, h:h + 1]
+        O_ref, Y_ref, S_ref = oracle.prefill(sl(inp["Q"]), sl(inp["K"]), sl(inp["V"]), sl(inp["z"]),
+                                             sl(inp["G"]), cfg.tau, cfg.eps)
+        assert_close(Y[:, :, h:h + 1], Y_ref, "bf16", f"Y head {h}")
+        assert_close(O[:, :, h:h + 1], O_ref, "bf16", f"O head {h}")
+        assert_close(Sf[:, h:h + 1], S_ref, "bf16", f"S head {h}")
