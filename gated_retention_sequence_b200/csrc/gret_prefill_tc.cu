@@ -58,6 +58,8 @@ struct Cfg {
     static constexpr int NQK = 2;                           // Q/K stages
     static constexpr int NV = (DV == 128 && C == 64) ? 2 : 1;   // V stages
     static constexpr int NG = (C == 128) ? 1 : 2;           // G/O stages
+    // with two G stages the swish gate is computed while the output MMAs run
+    static constexpr bool EARLY_SWISH = (NG == 2);
     static constexpr int ROWB = 128;                        // bytes per swizzled row
     static constexpr int BOX = C * ROWB;                    // one [C x 64] bf16 box
     static constexpr int Q_BYTES = 2 * BOX;                 // d_k = 128 -> 2 boxes
@@ -318,7 +320,6 @@ __global__ void __launch_bounds__(kCT, 1) prefill_tc_kernel(const __grid_constan
 
     float lam = 0.f;          // Lambda
     float seg_decay = 0.f;
-    uint32_t eager_count = 0;
     for (int i = 0; i < nchunks; ++i) {
         const int sq = i % NQK, sv = i % NV;
         const uint32_t sQ = sb + CF::OFF_Q + sq * CF::Q_BYTES;
@@ -343,12 +344,15 @@ __global__ void __launch_bounds__(kCT, 1) prefill_tc_kernel(const __grid_constan
 #pragma unroll
                 for (int c8 = 0; c8 < PC / 8; ++c8) {
                     const int s0 = grp * PC + c8 * 8;
+                    const float4 b0 = *reinterpret_cast<const float4*>(bc + s0);
+                    const float4 b1 = *reinterpret_cast<const float4*>(bc + s0 + 4);
+                    const float bs[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
                     uint32_t w[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int sa = s0 + 2 * e, sb2 = sa + 1;
-                        const float v0 = sa <= t ? u2f(r[c8 * 8 + 2 * e]) * __expf(bt - bc[sa]) : 0.f;
-                        const float v1 = sb2 <= t ? u2f(r[c8 * 8 + 2 * e + 1]) * __expf(bt - bc[sb2]) : 0.f;
+                        const int sa = s0 + 2 * e;
+                        const float v0 = sa <= t ? u2f(r[c8 * 8 + 2 * e]) * __expf(bt - bs[2 * e]) : 0.f;
+                        const float v1 = sa + 1 <= t ? u2f(r[c8 * 8 + 2 * e + 1]) * __expf(bt - bs[2 * e + 1]) : 0.f;
                         w[e] = pack_bf16x2(v0, v1);
                     }
                     const int region = s0 >> 6, chunk = (s0 & 63) >> 3;
@@ -356,48 +360,65 @@ __global__ void __launch_bounds__(kCT, 1) prefill_tc_kernel(const __grid_constan
                     *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
                 }
             }
-            // Q~ = e^{b_t + Lambda} Q: fp32 copy (tf32 mode) or in place (bf16 mode)
-            uint8_t* Qp = sm + CF::OFF_Q + sq * CF::Q_BYTES;
-            if constexpr (TF32) {
-                uint8_t* QT = sm + CF::OFF_QT;
-                for (int ci = tid; ci < C * 16; ci += kCT) {
-                    const int t = ci >> 4, c = ci & 15;    // row t, bf16 16-byte chunk c (d_k 8c .. 8c+7)
-                    const float f = __expf(bc[t] + lam);
-                    const uint4 w = *reinterpret_cast<const uint4*>(Qp + (c >> 3) * CF::BOX + t * 128 +
-                                                                    (((c & 7) ^ (t & 7)) << 4));
-                    const uint32_t* e = reinterpret_cast<const uint32_t*>(&w);
-                    float x[8];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&e[j]));
-                        x[2 * j] = f2.x * f;
-                        x[2 * j + 1] = f2.y * f;
-                    }
-                    uint8_t* row = QT + (c >> 2) * CF::BOX + t * 128;
-                    const int lc = 2 * (c & 3);
-                    *reinterpret_cast<float4*>(row + ((lc ^ (t & 7)) << 4)) = make_float4(x[0], x[1], x[2], x[3]);
-                    *reinterpret_cast<float4*>(row + (((lc + 1) ^ (t & 7)) << 4)) =
-                        make_float4(x[4], x[5], x[6], x[7]);
-                }
-            } else {
-                for (int ci = tid; ci < C * 16; ci += kCT) {
-                    const int row = (ci >> 3) % C;
-                    scale_bf16x8(Qp + ci * 16, __expf(bc[row] + lam));
-                }
-            }
         }
-        // K~: e^{-b_s - Lambda} (lazy) or e^{b_C - b_s} (eager), in place
+        // Q~ = e^{b_t + Lambda} Q (fp32 copy in tf32 mode, in place otherwise) and
+        // K~ = e^{-b_s - Lambda} K (lazy) or e^{b_C - b_s} K (eager), in place, as
+        // one list of 16-byte items.  With 64-token chunks the warps that own
+        // tensor-memory lanes 64..127 compute no P, so they take 3/4 of the list.
         {
+            constexpr int NQI = kFull ? C * 16 : 0;
+            constexpr int NI = NQI + C * 16;
+            int it0, it1, step;
+            if constexpr (kFull && C == 64) {
+                constexpr int cut = NI * 3 / 4;
+                step = kCT / 2;
+                if (q4 >= 2) { it0 = (((grp << 1) | (q4 - 2)) << 5) + lane; it1 = cut; }
+                else { it0 = cut + (((grp << 1) | q4) << 5) + lane; it1 = NI; }
+            } else {
+                it0 = tid; it1 = NI; step = kCT;
+            }
+            uint8_t* Qp = sm + CF::OFF_Q + sq * CF::Q_BYTES;
             uint8_t* Kp = sm + CF::OFF_K + sq * CF::K_BYTES;
-            for (int ci = tid; ci < C * 16; ci += kCT) {
-                const int row = (ci >> 3) % C;
-                const float ex = eager ? (bC - bc[row]) : (-bc[row] - lam);
-                scale_bf16x8(Kp + ci * 16, __expf(ex));
+            for (int it = it0; it < it1; it += step) {
+                if (it < NQI) {
+                    if constexpr (TF32) {
+                        const int t = it >> 4, c = it & 15;   // row t, bf16 16-byte chunk c (d_k 8c .. 8c+7)
+                        const float f = __expf(bc[t] + lam);
+                        const uint4 w = *reinterpret_cast<const uint4*>(Qp + (c >> 3) * CF::BOX + t * 128 +
+                                                                        (((c & 7) ^ (t & 7)) << 4));
+                        const uint32_t* e = reinterpret_cast<const uint32_t*>(&w);
+                        float x[8];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&e[j]));
+                            x[2 * j] = f2.x * f;
+                            x[2 * j + 1] = f2.y * f;
+                        }
+                        uint8_t* row = sm + CF::OFF_QT + (c >> 2) * CF::BOX + t * 128;
+                        const int lc = 2 * (c & 3);
+                        *reinterpret_cast<float4*>(row + ((lc ^ (t & 7)) << 4)) = make_float4(x[0], x[1], x[2], x[3]);
+                        *reinterpret_cast<float4*>(row + (((lc + 1) ^ (t & 7)) << 4)) =
+                            make_float4(x[4], x[5], x[6], x[7]);
+                    } else {
+                        const int row = (it >> 3) % C;
+                        scale_bf16x8(Qp + it * 16, __expf(bc[row] + lam));
+                    }
+                } else {
+                    const int ci = it - NQI;
+                    const int row = (ci >> 3) % C;
+                    const float ex = eager ? (bC - bc[row]) : (-bc[row] - lam);
+                    scale_bf16x8(Kp + ci * 16, __expf(ex));
+                }
             }
         }
-        // pass over T before the MMAs: bf16 copy (bf16 mode) and / or eager rescale
+        // pass over T before the MMAs: bf16 copy (bf16 mode) and / or eager rescale;
+        // it needs the previous chunk's state MMA to have finished
         const float escale = __expf(lam + bC);
         if (kFull ? !TF32 : eager) {
+            if (kFull && i > 0) {
+                mbar_wait(bar(BMMA), (i - 1) & 1, p.status, abort_flag);
+                tc_fence_after();
+            }
             uint32_t r[W];
             tmem_ld<W>(tm + lq + CF::TM_S + col0, r);
             tmem_wait_ld();
@@ -450,7 +471,14 @@ __global__ void __launch_bounds__(kCT, 1) prefill_tc_kernel(const __grid_constan
                         }
                     }
                 }
-                if (split) mma_commit(bar(BO));
+                mma_commit(bar(BO));
+            }
+            if (kFull && NG == 1 && p.has_g && i >= 1) {
+                // single G stage: the previous chunk's output store has to have
+                // read the buffer before this chunk's G lands there; it arrives
+                // while the MMAs run
+                bulk_wait_read<0>();
+                issue_g(i);
             }
             if (!split) {
                 issue_state(sV, sK);
@@ -458,9 +486,34 @@ __global__ void __launch_bounds__(kCT, 1) prefill_tc_kernel(const __grid_constan
                 if (kFull && i + 1 < nchunks) issue_scores(i + 1);
             }
         }
-        if (split) {
-            mbar_wait(bar(BO), eager_count & 1, p.status, abort_flag);
+        // swish(G) while the output MMAs run (two G stages: G(i) landed long ago)
+        float sw[NH][HT];
+        if constexpr (kFull && CF::EARLY_SWISH) {
+            if (p.gn) {
+                const int g = i % NG;
+                if (p.has_g) mbar_wait(bar(BG + g), (i / NG) & 1, p.status, abort_flag);
+                const uint8_t* Gp = sm + CF::OFF_G + g * CF::G_BYTES;
+#pragma unroll
+                for (int h = 0; h < NH; ++h) {
+                    const int d = h * 128 + q4 * 32 + lane;
+                    const int dj = d >> 6, dc = (d & 63) >> 3, de = (d & 7) * 2;
+                    const uint8_t* gcol = Gp + dj * CF::BOX + de;
+#pragma unroll
+                    for (int j = 0; j < HT; ++j) {
+                        const int t = grp * HT + j;
+                        const float gv = __bfloat162float(
+                            *reinterpret_cast<const __nv_bfloat16*>(gcol + t * 128 + ((dc ^ (t & 7)) << 4)));
+                        sw[h][j] = __fdividef(gv, 1.0f + __expf(-gv));
+                    }
+                }
+            }
+        }
+        if (kFull) {
+            // the epilogue needs only the output MMAs; the state MMA runs on
+            mbar_wait(bar(BO), i & 1, p.status, abort_flag);
             tc_fence_after();
+        }
+        if (split) {
             uint32_t r[W];
             tmem_ld<W>(tm + lq + CF::TM_S + col0, r);
             tmem_wait_ld();
@@ -476,15 +529,16 @@ __global__ void __launch_bounds__(kCT, 1) prefill_tc_kernel(const __grid_constan
                 mma_commit(bar(BMMA));
                 if (i + 1 < nchunks) issue_scores(i + 1);
             }
-            ++eager_count;
         }
         seg_decay += bC;
         lam = eager ? 0.f : lam + bC;
-        mbar_wait(bar(BMMA), i & 1, p.status, abort_flag);
-        tc_fence_after();
-        if (tid == 0) {
-            if (i + NQK < nchunks) issue_qk(i + NQK);   // this Q/K stage is free now
-            if (i + NV < nchunks) issue_v(i + NV);      // and this V stage
+        if (!kFull) {
+            mbar_wait(bar(BMMA), i & 1, p.status, abort_flag);
+            tc_fence_after();
+            if (tid == 0) {
+                if (i + NQK < nchunks) issue_qk(i + NQK);   // this K stage is free now
+                if (i + NV < nchunks) issue_v(i + NV);      // and this V stage
+            }
         }
 
         if (kFull) {
@@ -492,12 +546,20 @@ __global__ void __launch_bounds__(kCT, 1) prefill_tc_kernel(const __grid_constan
             // Thread (q4, grp, lane) owns d_v channels h*128 + q4*32 + lane
             // (h < NH) for tokens grp*HT .. grp*HT + HT - 1.
             const int g = i % NG;
-            if (p.has_g) mbar_wait(bar(BG + g), (i / NG) & 1, p.status, abort_flag);
+            if (p.has_g && !CF::EARLY_SWISH) mbar_wait(bar(BG + g), (i / NG) & 1, p.status, abort_flag);
             uint8_t* Gp = sm + CF::OFF_G + g * CF::G_BYTES;
             const int t0 = grp * HT;
-            const uint32_t oaddr = tm + lq + CF::TM_O + t0;
             float* red = reinterpret_cast<float*>(sm + CF::OFF_RED);
             float2* stat = reinterpret_cast<float2*>(sm + CF::OFF_STAT);
+            float y[NH][HT];
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
+                uint32_t r[HT];
+                tmem_ld<HT>(tm + lq + CF::TM_O + h * C + t0, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < HT; ++j) y[h][j] = u2f(r[j]);
+            }
             if (p.gn) {
                 // per-token sums over this thread's channels, then over the
                 // warp's lanes, then over the four lane quarters
@@ -505,16 +567,11 @@ __global__ void __launch_bounds__(kCT, 1) prefill_tc_kernel(const __grid_constan
                 for (int pass = 0; pass < 2; ++pass) {
                     float v[HT];
 #pragma unroll
-                    for (int h = 0; h < NH; ++h) {
-                        uint32_t r[HT];
-                        tmem_ld<HT>(oaddr + h * C, r);
-                        tmem_wait_ld();
+                    for (int j = 0; j < HT; ++j) {
+                        float acc = pass == 0 ? y[0][j] : y[0][j] * y[0][j];
 #pragma unroll
-                        for (int j = 0; j < HT; ++j) {
-                            const float y = u2f(r[j]);
-                            const float x = pass == 0 ? y : y * y;
-                            v[j] = h == 0 ? x : v[j] + x;
-                        }
+                        for (int h = 1; h < NH; ++h) acc += pass == 0 ? y[h][j] : y[h][j] * y[h][j];
+                        v[j] = acc;
                     }
                     warp_transpose_sum<HT>(v, lane);
                     if constexpr (HT >= 32) {
@@ -525,6 +582,13 @@ __global__ void __launch_bounds__(kCT, 1) prefill_tc_kernel(const __grid_constan
                     }
                 }
                 named_bar_sync(1, kCT);
+                if (tid == 0) {
+                    // this chunk's state MMA has had the whole reduction to finish:
+                    // its Q/K and V stages take the next loads
+                    mbar_wait(bar(BMMA), i & 1, p.status, abort_flag);
+                    if (i + NQK < nchunks) issue_qk(i + NQK);
+                    if (i + NV < nchunks) issue_v(i + NV);
+                }
                 if (tid < C) {
                     const int gg = tid / HT, tl = tid % HT;
                     float s1 = 0.f, s2 = 0.f;
@@ -540,24 +604,38 @@ __global__ void __launch_bounds__(kCT, 1) prefill_tc_kernel(const __grid_constan
                 }
                 named_bar_sync(1, kCT);
             }
+            if (!p.gn && tid == 0) {
+                mbar_wait(bar(BMMA), i & 1, p.status, abort_flag);
+                if (i + NQK < nchunks) issue_qk(i + NQK);
+                if (i + NV < nchunks) issue_v(i + NV);
+            }
+            int goff[NH];
 #pragma unroll
             for (int h = 0; h < NH; ++h) {
-                uint32_t r[HT];
-                tmem_ld<HT>(oaddr + h * C, r);
-                tmem_wait_ld();
                 const int d = h * 128 + q4 * 32 + lane;
-                const int dj = d >> 6, dc = (d & 63) >> 3, de = (d & 7) * 2;
-                uint8_t* gcol = Gp + dj * CF::BOX + de;
+                goff[h] = (d >> 6) * CF::BOX + (d & 7) * 2;
+            }
+            const int dc = ((q4 * 32 + lane) & 63) >> 3;   // the same for both halves
 #pragma unroll
-                for (int j = 0; j < HT; ++j) {
-                    const int t = t0 + j;
-                    __nv_bfloat16* gp = reinterpret_cast<__nv_bfloat16*>(gcol + t * 128 + ((dc ^ (t & 7)) << 4));
-                    float o = u2f(r[j]);
+            for (int j = 0; j < HT; ++j) {
+                const int t = t0 + j;
+                const int rowoff = t * 128 + ((dc ^ (t & 7)) << 4);
+                float2 st = make_float2(1.f, 0.f);
+                if (p.gn) st = stat[t];
+#pragma unroll
+                for (int h = 0; h < NH; ++h) {
+                    __nv_bfloat16* gp = reinterpret_cast<__nv_bfloat16*>(Gp + goff[h] + rowoff);
+                    float o = y[h][j];
                     if (p.gn) {
-                        const float2 st = stat[t];
-                        const float gv = __bfloat162float(*gp);
-                        // GroupNorm as one FMA, then swish(g) = g * sigmoid(g)
-                        o = fmaf(o, st.x, st.y) * __fdividef(gv, 1.0f + __expf(-gv));
+                        float swv;
+                        if constexpr (CF::EARLY_SWISH) {
+                            swv = sw[h][j];
+                        } else {
+                            const float gv = __bfloat162float(*gp);
+                            swv = __fdividef(gv, 1.0f + __expf(-gv));
+                        }
+                        // GroupNorm as one FMA, then times swish(g) = g * sigmoid(g)
+                        o = fmaf(o, st.x, st.y) * swv;
                     }
                     *gp = __float2bfloat16_rn(o);
                 }
@@ -569,16 +647,24 @@ __global__ void __launch_bounds__(kCT, 1) prefill_tc_kernel(const __grid_constan
                 const int n0 = n_begin + i * C;
                 for (int x = 0; x < DV / 64; ++x) tma_store_4d(&p.tmO, smem_u32(Gp + x * CF::BOX), x * 64, hh, n0, bb);
                 bulk_commit();
-                bulk_wait_read<NG - 1>();   // every store but the newest has read its buffer
                 const int j = i + 1;
-                if (p.has_g && j >= NG && j < nchunks) issue_g(j);
+                if constexpr (NG == 2) {
+                    bulk_wait_read<1>();   // the store issued one chunk ago has read its buffer
+                    if (p.has_g && j >= NG && j < nchunks) issue_g(j);
+                }
             }
         }
     }
 
     // ---------------------------------------------------------------- state out: e^Lambda T
     {
-        if (kFull && tid == 0) bulk_wait<0>();
+        if (kFull) {
+            if (tid == 0) bulk_wait<0>();
+            if (nchunks > 0) {
+                mbar_wait(bar(BMMA), (nchunks - 1) & 1, p.status, abort_flag);
+                tc_fence_after();
+            }
+        }
         const float sc = __expf(lam);
         uint32_t r[W];
         tmem_ld<W>(tm + lq + CF::TM_S + col0, r);
