@@ -57,6 +57,8 @@ _VP, _FP, _I, _F, _SZ = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c
 SIGNATURES = {
     "gret_prefill": (_I, [_VP, _VP, _VP, _FP, _VP, _F, _I, _VP, _FP, _I, _I, _I, _I, _I, _I, _F, _I,
                           _VP, _SZ, _VP]),
+    "gret_prefill_noalloc": (_I, [_VP, _VP, _VP, _FP, _VP, _F, _I, _VP, _FP, _I, _I, _I, _I, _I, _I, _F,
+                                  _I, _VP]),
     "gret_prefill_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
     "gret_prefill_path": (_I, [_I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_int)]),
     "gret_decode_step": (_I, [_VP, _VP, _VP, _FP, _VP, _FP, _VP, _I, _I, _I, _I, _F, _I, _F, _I, _VP]),
@@ -88,6 +90,12 @@ def gret_prefill(Q, K, V, gate_logits, G, tau, chunk, O, S_final, B, H, N, dk, d
                  epi, workspace, workspace_bytes, stream) -> int:
     return load().gret_prefill(Q, K, V, gate_logits, G, tau, chunk, O, S_final, B, H, N, dk, dv,
                                int(io_dtype), eps, int(epi), workspace, workspace_bytes, stream)
+
+
+def gret_prefill_noalloc(Q, K, V, gate_logits, G, tau, chunk, O, S_final, B, H, N, dk, dv, io_dtype, eps,
+                         epi, stream) -> int:
+    return load().gret_prefill_noalloc(Q, K, V, gate_logits, G, tau, chunk, O, S_final, B, H, N, dk, dv,
+                                       int(io_dtype), eps, int(epi), stream)
 
 
 def gret_prefill_workspace_size(B, H, N, dk, dv, chunk, io_dtype) -> int:

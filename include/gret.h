@@ -87,6 +87,36 @@ gret_status gret_prefill(const void* Q, const void* K, const void* V, const floa
                          gret_epilogue epi, void* workspace, size_t workspace_bytes,
                          gret_stream_t stream);
 
+/* Size of the device scratch array gret_prefill_noalloc draws on (32 MiB). */
+#define GRET_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+
+/*
+ * gret_prefill_noalloc -- gret_prefill without a workspace argument, for
+ * callers that cannot allocate device memory: plugins and custom-op hosts that
+ * are handed only the tensors' device pointers and have no allocator of their
+ * own to ask, and code paths where calling cudaMalloc is not allowed because
+ * it can synchronise the device or take memory from a pool someone else owns.
+ * The pages describe no such entry point; it is an addition of this library.
+ *
+ * Arguments, layouts and results are those of gret_prefill.  Instead of a
+ * caller workspace the call uses a fixed array of GRET_NOALLOC_SCRATCH_BYTES
+ * that the library reserves in device memory on every GPU that loads it, for
+ * the life of the process.  Calls whose gret_prefill_workspace_size exceeds
+ * that return GRET_ERR_UNSUPPORTED before touching the GPU.  The call
+ * allocates nothing itself.
+ *
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  All calls share the one array, and nothing in
+ * it needs clearing between calls (each call writes what it reads), but two
+ * calls whose work overlaps on the GPU (different streams, or different host
+ * threads on one device) race on it: serialise them.
+ */
+gret_status gret_prefill_noalloc(const void* Q, const void* K, const void* V, const float* gate_logits,
+                                 const void* G, float tau, int chunk, void* O, float* S_final,
+                                 int B, int H, int N, int dk, int dv, gret_dtype io_dtype, float eps,
+                                 gret_epilogue epi, gret_stream_t stream);
+
 /* Device scratch (bytes) gret_prefill needs for these arguments; 0 if none.
  * Returns 0 as well for unsupported arguments (gret_prefill then reports them). */
 size_t gret_prefill_workspace_size(int B, int H, int N, int dk, int dv, int chunk,
