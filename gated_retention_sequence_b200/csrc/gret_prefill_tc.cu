@@ -693,6 +693,194 @@ __global__ void __launch_bounds__(kCT, 1) prefill_tc_kernel(const __grid_constan
     }
 }
 
+// ---------------------------------------------------------------------------
+// Segment state pass: dS_p = sum over the segment's tokens of
+// e^{a_p - B_s} K_s^T V_s (B_s the log-decay from the segment start through s,
+// a_p the segment total), from K, V and the decay sums alone.  The same
+// lazy/eager state scaling as the fused kernels; a 3-4 stage ring of K/V
+// tiles keeps about 190 KB of loads in flight per SM.
+constexpr int kStateThreads = 256;
+
+template <int DV, int C>
+struct StateCfg {
+    static constexpr int NH = DV / 128;
+    static constexpr int NS = (C * (2 * 128 + DV) * 2 <= 48 * 1024) ? 4 : 3;   // stages of K + V
+    static constexpr int BOX = C * 128;
+    static constexpr int K_BYTES = 2 * BOX;
+    static constexpr int V_BYTES = (DV / 64) * BOX;
+    static constexpr int W = NH * 64;                       // state columns per thread
+    static constexpr int TM_ALLOC = NH * 128 <= 128 ? 128 : 256;
+    static constexpr int OFF_K = 0;
+    static constexpr int OFF_V = OFF_K + NS * K_BYTES;
+    static constexpr int OFF_B = OFF_V + NS * V_BYTES;
+    static constexpr int OFF_BAR = OFF_B + NS * C * 4;
+    static constexpr int OFF_MISC = OFF_BAR + 2 * NS * 8;
+    static constexpr int SMEM = OFF_MISC + 16 + 1024;
+    static_assert(SMEM <= 227 * 1024, "shared memory budget");
+};
+
+template <int DV, int C>
+__global__ void __launch_bounds__(kStateThreads, 1) prefill_state_kernel(const __grid_constant__ TcParams p) {
+    using CF = StateCfg<DV, C>;
+    constexpr int NS = CF::NS, NH = CF::NH, W = CF::W;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sb = smem_u32(sm);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int q4 = warp & 3, gi = warp >> 2;
+    const uint32_t lq = (uint32_t)(32 * q4) << 16;
+
+    const int nseg = p.P - 1;
+    const int u = blockIdx.x / nseg, seg = blockIdx.x % nseg;
+    const int bb = u / p.H, hh = u % p.H;
+    const int n_begin = seg * p.seg_len;
+    const int n_end = min(p.N, n_begin + p.seg_len);
+    const int nchunks = (n_end - n_begin + C - 1) / C;
+
+    auto full = [&](int s) -> uint32_t { return sb + CF::OFF_BAR + 8 * s; };
+    auto empty = [&](int s) -> uint32_t { return sb + CF::OFF_BAR + 8 * (NS + s); };
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + CF::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + CF::OFF_MISC + 4);
+
+    if (tid == 0) {
+        for (int i = 0; i < 2 * NS; ++i) mbar_init(sb + CF::OFF_BAR + 8 * i, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&p.tmK);
+        tma_prefetch_desc(&p.tmV);
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(tmem_slot), CF::TM_ALLOC);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = *tmem_slot;
+
+    auto issue = [&](int j) {
+        const int s = j % NS, n0 = n_begin + j * C;
+        mbar_arrive_expect_tx(full(s), CF::K_BYTES + CF::V_BYTES + C * 4);
+        for (int x = 0; x < 2; ++x)
+            tma_load_4d(sb + CF::OFF_K + s * CF::K_BYTES + x * CF::BOX, &p.tmK, x * 64, hh, n0, bb, full(s));
+        for (int x = 0; x < DV / 64; ++x)
+            tma_load_4d(sb + CF::OFF_V + s * CF::V_BYTES + x * CF::BOX, &p.tmV, x * 64, hh, n0, bb, full(s));
+        bulk_load(sb + CF::OFF_B + s * C * 4, p.bcum + (size_t)u * p.Npad + n0, C * 4, full(s));
+    };
+    if (tid == 0)
+        for (int j = 0; j < NS && j < nchunks; ++j) issue(j);
+
+    const int col0 = gi * W;
+#pragma unroll 1
+    for (int cb = 0; cb < W / 32; ++cb) {
+        uint32_t r[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) r[j] = 0u;
+        tmem_st<32>(tm + lq + col0 + cb * 32, r);
+    }
+    tmem_wait_st();
+
+    float lam = 0.f, seg_decay = 0.f;
+    for (int i = 0; i < nchunks; ++i) {
+        const int s = i % NS;
+        const float* bc = reinterpret_cast<const float*>(sm + CF::OFF_B + s * C * 4);
+        mbar_wait(full(s), (i / NS) & 1, p.status, abort_flag);
+        const float bC = bc[C - 1];
+        const bool eager = (-bC - lam) > kLazyMax;
+        uint8_t* Kp = sm + CF::OFF_K + s * CF::K_BYTES;
+        {
+            constexpr int NIT = C * 16 / kStateThreads;   // 4 or 8 items per thread
+            uint4 w[NIT];
+            float e[NIT];
+#pragma unroll
+            for (int k = 0; k < NIT; ++k) {
+                const int ci = tid + k * kStateThreads;
+                w[k] = *reinterpret_cast<const uint4*>(Kp + ci * 16);
+                e[k] = bc[(ci >> 3) % C];
+            }
+#pragma unroll
+            for (int k = 0; k < NIT; ++k) {
+                const float sc = __expf(eager ? (bC - e[k]) : (-e[k] - lam));
+                uint32_t* x = reinterpret_cast<uint32_t*>(&w[k]);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x[j]));
+                    x[j] = pack_bf16x2(f2.x * sc, f2.y * sc);
+                }
+                *reinterpret_cast<uint4*>(Kp + (tid + k * kStateThreads) * 16) = w[k];
+            }
+        }
+        if (eager) {
+            // T *= e^{Lambda + b_C}, after the previous chunk's state MMA
+            if (i > 0) {
+                mbar_wait(empty((i - 1) % NS), ((i - 1) / NS) & 1, p.status, abort_flag);
+                tc_fence_after();
+            }
+            const float escale = __expf(lam + bC);
+#pragma unroll 1
+            for (int cb = 0; cb < W / 32; ++cb) {
+                uint32_t r[32];
+                tmem_ld<32>(tm + lq + col0 + cb * 32, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) r[j] = f2u(u2f(r[j]) * escale);
+                tmem_st<32>(tm + lq + col0 + cb * 32, r);
+            }
+            tmem_wait_st();
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+            // the stage the previous chunk used is free once its MMA is done
+            if (i > 0 && i - 1 + NS < nchunks) {
+                mbar_wait(empty((i - 1) % NS), ((i - 1) / NS) & 1, p.status, abort_flag);
+                issue(i - 1 + NS);
+            }
+            const uint32_t sK = sb + CF::OFF_K + s * CF::K_BYTES, sV = sb + CF::OFF_V + s * CF::V_BYTES;
+            constexpr uint32_t id_kv = idesc_bf16(128, DK, true, true);
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
+#pragma unroll
+                for (int k = 0; k < C / 16; ++k)
+                    mma_ss(tm + h * 128, sdesc_sw128(sV + 2 * h * CF::BOX + k * 2048, CF::BOX, 1024),
+                           sdesc_sw128(sK + k * 2048, CF::BOX, 1024), id_kv, 1);
+            }
+            mma_commit(empty(s));
+        }
+        seg_decay += bC;
+        lam = eager ? 0.f : lam + bC;
+    }
+    if (nchunks > 0) {
+        mbar_wait(empty((nchunks - 1) % NS), ((nchunks - 1) / NS) & 1, p.status, abort_flag);
+        tc_fence_after();
+    }
+    {
+        const float sc = __expf(lam);
+        const int s_d = (col0 / 128) * 128 + q4 * 32 + lane, s_k0 = col0 % 128;
+        float* dst = p.seg_state + ((size_t)u * (p.P - 1) + seg) * DV * DK + (size_t)s_d * DK + s_k0;
+#pragma unroll 1
+        for (int cb = 0; cb < W / 32; ++cb) {
+            uint32_t r[32];
+            tmem_ld<32>(tm + lq + col0 + cb * 32, r);
+            tmem_wait_ld();
+            float4* d4 = reinterpret_cast<float4*>(dst + cb * 32);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                d4[j] = make_float4(u2f(r[4 * j]) * sc, u2f(r[4 * j + 1]) * sc, u2f(r[4 * j + 2]) * sc,
+                                    u2f(r[4 * j + 3]) * sc);
+        }
+        if (tid == 0) p.seg_decay[(size_t)u * (p.P - 1) + seg] = seg_decay;
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tm, CF::TM_ALLOC);
+    }
+}
+
 // Chunk-local inclusive sums of log gamma: bcum[u][n] = sum_{j in chunk, j <= n} lg_j.
 // Padding tokens (n >= N) carry lg = 0, so they repeat the chunk total.
 __global__ void gate_scan_kernel(const float* __restrict__ z, float* __restrict__ bcum, int H, int N,
@@ -783,13 +971,13 @@ template <int DV, int C>
 cudaError_t run_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t s) {
     using CF = Cfg<DV, C>;
     auto kf = prefill_tc_kernel<DV, C, true>;
-    auto ks = prefill_tc_kernel<DV, C, false>;
+    auto ks = prefill_state_kernel<DV, C>;
     static bool attr_done[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || !attr_done[dev]) {
         cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, CF::SMEM);
-        cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, CF::SMEM);
+        cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, StateCfg<DV, C>::SMEM);
         if (dev >= 0 && dev < 64) attr_done[dev] = true;
     }
     const int units = a.B * a.H;
@@ -797,7 +985,7 @@ cudaError_t run_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t s) {
     gate_scan_kernel<<<dim3(units, npad / C), C, 0, s>>>(a.z, const_cast<float*>(tp.bcum), a.H, a.N, npad,
                                                          a.inv_tau);
     if (tp.P > 1) {
-        ks<<<units * (tp.P - 1), kCT, CF::SMEM, s>>>(tp);
+        ks<<<units * (tp.P - 1), kStateThreads, StateCfg<DV, C>::SMEM, s>>>(tp);
         const int elems4 = DV * DK / 4;
         seg_combine_kernel<<<dim3((elems4 + 255) / 256, units), 256, 0, s>>>(tp.seg_state, tp.seg_decay, tp.P,
                                                                              elems4);
