@@ -133,13 +133,21 @@ def dist_setup():
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """Largest value of x over all ranks (the job's time is its slowest rank's)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(world: int, units_per_rank: float, steps: int, max_ms: float) -> float:
+    """Whole-job rate (units per second) of `world` ranks that each processed
+    `units_per_rank` per step for `steps` steps, timed by the slowest rank."""
+    return world * units_per_rank * steps / (max_ms / 1e3)
 
 
 def barrier(world):
@@ -147,7 +155,8 @@ def barrier(world):
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
 
 
 def cpu_oracle_sample(cfg, units, threads):
@@ -251,7 +260,7 @@ def run_ours(args, world, rank, local):
     kern_ms = statistics.mean(ks[i].elapsed_time(ke[i]) for i in range(args.steps))
 
     tokens = cfg.B * cfg.N
-    value = world * tokens * args.steps / (ms / 1e3) / 1e6
+    value = job_throughput(world, tokens, args.steps, ms) / 1e6
     alg_bytes, alg_flops = prefill_alg(cfg)
     step_s = ms / 1e3 / args.steps
     launches_per_step = 2 + (2 if segs > 1 else 0)
@@ -283,7 +292,7 @@ def run_ours(args, world, rank, local):
         e1.record(stream)
         barrier(world)
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-        e2e_value = world * tokens * e2e_steps / (e2e_ms / 1e3) / 1e6
+        e2e_value = job_throughput(world, tokens, e2e_steps, e2e_ms) / 1e6
 
     decode = None if args.no_decode else run_decode(args, world, dev, stream, peaks)
     clk = clocks.stop()

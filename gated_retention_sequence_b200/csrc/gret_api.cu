@@ -55,17 +55,19 @@ constexpr size_t kMaxSmem = 227 * 1024;
 
 // Kernel choice for a prefill; segments/seg_len describe the sequence split.
 gret_path select_path(int B, int H, int N, int dk, int dv, int chunk, gret_dtype io, int num_sms,
-                      int* segments, int* seg_len) {
+                      int* segments, int* seg_len, int* pieces = nullptr) {
     if (segments) *segments = 1;
     if (seg_len) *seg_len = N;
+    if (pieces) *pieces = 1;
     if (B <= 0 || H <= 0 || N <= 0 || dk <= 0 || dv <= 0) return GRET_PATH_NONE;
     if (io != GRET_F32 && io != GRET_BF16) return GRET_PATH_NONE;
     if (!shape_supported(dk, dv) || !chunk_supported(chunk)) return GRET_PATH_NONE;
     if (io == GRET_BF16 && prefill_tc_supported(dk, dv, chunk, io)) {
-        int segs = 1, len = N;
-        prefill_tc_plan(B, H, N, chunk, num_sms, &segs, &len);
+        int segs = 1, len = N, pcs = 1;
+        prefill_tc_plan(B, H, N, chunk, num_sms, &segs, &len, &pcs);
         if (segments) *segments = segs;
         if (seg_len) *seg_len = len;
+        if (pieces) *pieces = pcs;
         return GRET_PATH_TC;
     }
     if (prefill_simt_smem_bytes(dk, dv, chunk) <= kMaxSmem) return GRET_PATH_SIMT;
@@ -106,11 +108,11 @@ gret_path gret_prefill_path(int B, int H, int N, int dk, int dv, int chunk, gret
 
 size_t gret_prefill_workspace_size(int B, int H, int N, int dk, int dv, int chunk,
                                    gret_dtype io_dtype) {
-    int sms = 148, segs = 1;
+    int sms = 148, segs = 1, pcs = 1;
     device_info(nullptr, &sms);
-    gret_path p = select_path(B, H, N, dk, dv, chunk, io_dtype, sms, &segs, nullptr);
+    gret_path p = select_path(B, H, N, dk, dv, chunk, io_dtype, sms, &segs, nullptr, &pcs);
     if (p != GRET_PATH_TC) return 0;
-    return prefill_tc_workspace_bytes(B, H, N, dk, dv, chunk, segs);
+    return prefill_tc_workspace_bytes(B, H, N, dk, dv, chunk, segs, pcs);
 }
 
 gret_status gret_prefill(const void* Q, const void* K, const void* V, const float* gate_logits,
@@ -131,8 +133,8 @@ gret_status gret_prefill(const void* Q, const void* K, const void* V, const floa
     unsigned int* status = nullptr;
     int sms = 0;
     if (!device_info(&status, &sms)) return GRET_ERR_CUDA;
-    int segs = 1, seg_len = N;
-    gret_path path = select_path(B, H, N, dk, dv, chunk, io_dtype, sms, &segs, &seg_len);
+    int segs = 1, seg_len = N, pcs = 1;
+    gret_path path = select_path(B, H, N, dk, dv, chunk, io_dtype, sms, &segs, &seg_len, &pcs);
     if (path == GRET_PATH_NONE) return GRET_ERR_UNSUPPORTED;
 
     PrefillArgs a;
@@ -140,12 +142,12 @@ gret_status gret_prefill(const void* Q, const void* K, const void* V, const floa
     a.B = B; a.H = H; a.N = N; a.dk = dk; a.dv = dv; a.chunk = chunk;
     a.inv_tau = 1.0f / tau; a.eps = eps; a.io = io_dtype; a.epi = epi;
     a.workspace = workspace; a.workspace_bytes = workspace_bytes;
-    a.status = status; a.segments = segs; a.seg_len = seg_len;
+    a.status = status; a.segments = segs; a.seg_len = seg_len; a.pieces = pcs;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t err;
     if (path == GRET_PATH_TC) {
-        size_t need = prefill_tc_workspace_bytes(B, H, N, dk, dv, chunk, segs);
+        size_t need = prefill_tc_workspace_bytes(B, H, N, dk, dv, chunk, segs, pcs);
         if (need > 0) {
             if (!workspace || workspace_bytes < need) return GRET_ERR_INVALID_ARG;
             if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return GRET_ERR_INVALID_ARG;

@@ -30,6 +30,7 @@ struct PrefillArgs {
     unsigned int* status;     // device status word
     int segments;             // sequence segments per unit (TC path)
     int seg_len;              // tokens per segment (multiple of chunk)
+    int pieces;               // state-pass pieces per segment (divides seg_len / chunk)
 };
 
 struct DecodeArgs {
@@ -87,7 +88,7 @@ cudaError_t launch_prefill_simt(const PrefillArgs& a, cudaStream_t s);
 size_t prefill_simt_smem_bytes(int dk, int dv, int chunk);
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s);
 bool prefill_tc_supported(int dk, int dv, int chunk, gret_dtype io);
-void prefill_tc_plan(int B, int H, int N, int chunk, int num_sms, int* segments, int* seg_len);
-size_t prefill_tc_workspace_bytes(int B, int H, int N, int dk, int dv, int chunk, int segments);
+void prefill_tc_plan(int B, int H, int N, int chunk, int num_sms, int* segments, int* seg_len, int* pieces);
+size_t prefill_tc_workspace_bytes(int B, int H, int N, int dk, int dv, int chunk, int segments, int pieces);
 
 }  // namespace gret

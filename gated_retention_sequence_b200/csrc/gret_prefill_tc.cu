@@ -105,11 +105,12 @@ struct Cfg {
 struct TcParams {
     CUtensorMap tmQ, tmK, tmV, tmG, tmO;
     const float* bcum;       // [units][Npad] chunk-local cumulative log-decay
-    float* seg_state;        // [units][P-1][DV][DK]  (S^T, fp32)
-    float* seg_decay;        // [units][P-1]
+    float* seg_state;        // [units][(P-1)*K][DV][DK]  (S^T, fp32)
+    float* seg_decay;        // [units][(P-1)*K]
     float* S_final;          // [units][DK][DV] or null
     unsigned int* status;
     int H, N, Npad, P, seg_len;
+    int K, piece_len;        // state-pass pieces per segment and their length
     float eps;
     int gn;                  // 1: GroupNorm + swish; 0: O = Y
     int has_g;
@@ -303,7 +304,8 @@ __global__ void __launch_bounds__(kCT, 1) prefill_tc_kernel(const __grid_constan
     {
         uint32_t r[W];
         if (kFull && seg > 0) {
-            const float* src = p.seg_state + ((size_t)u * (p.P - 1) + (seg - 1)) * DV * DK + (size_t)s_d * DK + s_k0;
+            const float* src = p.seg_state + ((size_t)u * (p.P - 1) * p.K + (size_t)seg * p.K - 1) * DV * DK +
+                               (size_t)s_d * DK + s_k0;
             const float4* s4 = reinterpret_cast<const float4*>(src);
 #pragma unroll
             for (int j = 0; j < W / 4; ++j) {
@@ -730,11 +732,11 @@ __global__ void __launch_bounds__(kStateThreads, 1) prefill_state_kernel(const _
     const int q4 = warp & 3, gi = warp >> 2;
     const uint32_t lq = (uint32_t)(32 * q4) << 16;
 
-    const int nseg = p.P - 1;
+    const int nseg = (p.P - 1) * p.K;           // pieces of all segments but the last
     const int u = blockIdx.x / nseg, seg = blockIdx.x % nseg;
     const int bb = u / p.H, hh = u % p.H;
-    const int n_begin = seg * p.seg_len;
-    const int n_end = min(p.N, n_begin + p.seg_len);
+    const int n_begin = seg * p.piece_len;
+    const int n_end = min(p.N, n_begin + p.piece_len);
     const int nchunks = (n_end - n_begin + C - 1) / C;
 
     auto full = [&](int s) -> uint32_t { return sb + CF::OFF_BAR + 8 * s; };
@@ -859,7 +861,7 @@ __global__ void __launch_bounds__(kStateThreads, 1) prefill_state_kernel(const _
     {
         const float sc = __expf(lam);
         const int s_d = (col0 / 128) * 128 + q4 * 32 + lane, s_k0 = col0 % 128;
-        float* dst = p.seg_state + ((size_t)u * (p.P - 1) + seg) * DV * DK + (size_t)s_d * DK + s_k0;
+        float* dst = p.seg_state + ((size_t)u * nseg + seg) * DV * DK + (size_t)s_d * DK + s_k0;
 #pragma unroll 1
         for (int cb = 0; cb < W / 32; ++cb) {
             uint32_t r[32];
@@ -871,7 +873,7 @@ __global__ void __launch_bounds__(kStateThreads, 1) prefill_state_kernel(const _
                 d4[j] = make_float4(u2f(r[4 * j]) * sc, u2f(r[4 * j + 1]) * sc, u2f(r[4 * j + 2]) * sc,
                                     u2f(r[4 * j + 3]) * sc);
         }
-        if (tid == 0) p.seg_decay[(size_t)u * (p.P - 1) + seg] = seg_decay;
+        if (tid == 0) p.seg_decay[(size_t)u * nseg + seg] = seg_decay;
     }
     tc_fence_before();
     __syncthreads();
@@ -904,15 +906,15 @@ __global__ void gate_scan_kernel(const float* __restrict__ z, float* __restrict_
 
 // Fold the segment increments into initial states, in place:
 // slot p <- S_in(p + 1) = e^{a_p} S_in(p) + dS_p, with S_in(0) = 0.
-__global__ void seg_combine_kernel(float* __restrict__ seg_state, const float* __restrict__ seg_decay, int P,
+__global__ void seg_combine_kernel(float* __restrict__ seg_state, const float* __restrict__ seg_decay, int nslots,
                                    int elems4) {
     const int u = blockIdx.y;
     const int e = blockIdx.x * blockDim.x + threadIdx.x;
     if (e >= elems4) return;
     float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int p = 0; p < P - 1; ++p) {
-        float4* slot = reinterpret_cast<float4*>(seg_state) + ((size_t)u * (P - 1) + p) * elems4 + e;
-        const float f = __expf(seg_decay[(size_t)u * (P - 1) + p]);
+    for (int p = 0; p < nslots; ++p) {
+        float4* slot = reinterpret_cast<float4*>(seg_state) + ((size_t)u * nslots + p) * elems4 + e;
+        const float f = __expf(seg_decay[(size_t)u * nslots + p]);
         const float4 d = *slot;
         run = make_float4(fmaf(f, run.x, d.x), fmaf(f, run.y, d.y), fmaf(f, run.z, d.z), fmaf(f, run.w, d.w));
         *slot = run;
@@ -956,14 +958,15 @@ struct WsLayout {
     size_t bcum, state, decay, total;
 };
 
-WsLayout ws_layout(int B, int H, int N, int dk, int dv, int chunk, int segments) {
+WsLayout ws_layout(int B, int H, int N, int dk, int dv, int chunk, int segments, int pieces) {
     const size_t units = (size_t)B * H;
     const size_t npad = (size_t)((N + chunk - 1) / chunk) * chunk;
     WsLayout w;
     w.bcum = 0;
     w.state = align256(units * npad * 4);
-    w.decay = w.state + align256(segments > 1 ? units * (segments - 1) * (size_t)dk * dv * 4 : 0);
-    w.total = w.decay + align256(segments > 1 ? units * (segments - 1) * 4 : 0);
+    const size_t slots = segments > 1 ? (size_t)(segments - 1) * pieces : 0;
+    w.decay = w.state + align256(units * slots * (size_t)dk * dv * 4);
+    w.total = w.decay + align256(units * slots * 4);
     return w;
 }
 
@@ -985,9 +988,9 @@ cudaError_t run_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t s) {
     gate_scan_kernel<<<dim3(units, npad / C), C, 0, s>>>(a.z, const_cast<float*>(tp.bcum), a.H, a.N, npad,
                                                          a.inv_tau);
     if (tp.P > 1) {
-        ks<<<units * (tp.P - 1), kStateThreads, StateCfg<DV, C>::SMEM, s>>>(tp);
+        ks<<<units * (tp.P - 1) * tp.K, kStateThreads, StateCfg<DV, C>::SMEM, s>>>(tp);
         const int elems4 = DV * DK / 4;
-        seg_combine_kernel<<<dim3((elems4 + 255) / 256, units), 256, 0, s>>>(tp.seg_state, tp.seg_decay, tp.P,
+        seg_combine_kernel<<<dim3((elems4 + 255) / 256, units), 256, 0, s>>>(tp.seg_state, tp.seg_decay, (tp.P - 1) * tp.K,
                                                                              elems4);
     }
     if (g_profile_start) cudaEventRecord(g_profile_start, s);
@@ -1003,19 +1006,29 @@ bool prefill_tc_supported(int dk, int dv, int chunk, gret_dtype io) {
     return (dv == 128 && (chunk == 64 || chunk == 128)) || (dv == 256 && chunk == 64);
 }
 
-void prefill_tc_plan(int B, int H, int N, int chunk, int num_sms, int* segments, int* seg_len) {
-    const int units = B * H;
+// Segments: about one fused CTA per SM.  State-pass pieces: each of the first
+// P-1 segments is cut into K pieces (K divides the segment's chunk count) so
+// that the state pass, too, has about one CTA per SM.
+void prefill_tc_plan(int B, int H, int N, int chunk, int num_sms, int* segments, int* seg_len, int* pieces) {
+    const int units = B * H > 0 ? B * H : 1;
     const int nchunks = (N + chunk - 1) / chunk;
-    int P = num_sms / (units > 0 ? units : 1);
+    int P = num_sms / units;
     if (P < 1) P = 1;
     if (P > nchunks) P = nchunks;
     const int per = (nchunks + P - 1) / P;
     *seg_len = per * chunk;
     *segments = (nchunks + per - 1) / per;
+    int K = 1;
+    if (*segments > 1) {
+        const int kmax = num_sms / (units * (*segments - 1));
+        for (int k = kmax < per ? kmax : per; k >= 1; --k)
+            if (per % k == 0) { K = k; break; }
+    }
+    *pieces = K;
 }
 
-size_t prefill_tc_workspace_bytes(int B, int H, int N, int dk, int dv, int chunk, int segments) {
-    return ws_layout(B, H, N, dk, dv, chunk, segments).total;
+size_t prefill_tc_workspace_bytes(int B, int H, int N, int dk, int dv, int chunk, int segments, int pieces) {
+    return ws_layout(B, H, N, dk, dv, chunk, segments, pieces).total;
 }
 
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
@@ -1026,7 +1039,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
         !make_map(&tp.tmV, a.V, a.dv, a.H, a.N, a.B, C) || !make_map(&tp.tmO, a.O, a.dv, a.H, a.N, a.B, C) ||
         !make_map(&tp.tmG, a.G ? a.G : a.O, a.dv, a.H, a.N, a.B, C))
         return cudaErrorInvalidValue;
-    const WsLayout w = ws_layout(a.B, a.H, a.N, a.dk, a.dv, C, a.segments);
+    const WsLayout w = ws_layout(a.B, a.H, a.N, a.dk, a.dv, C, a.segments, a.pieces);
     uint8_t* ws = static_cast<uint8_t*>(a.workspace);
     tp.bcum = reinterpret_cast<const float*>(ws + w.bcum);
     tp.seg_state = reinterpret_cast<float*>(ws + w.state);
@@ -1038,6 +1051,8 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
     tp.Npad = (a.N + C - 1) / C * C;
     tp.P = a.segments;
     tp.seg_len = a.seg_len;
+    tp.K = a.pieces;
+    tp.piece_len = a.seg_len / a.pieces;
     tp.eps = a.eps;
     tp.gn = a.epi == GRET_EPI_GN_SWISH ? 1 : 0;
     tp.has_g = (a.epi == GRET_EPI_GN_SWISH && a.G) ? 1 : 0;

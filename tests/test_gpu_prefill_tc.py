@@ -126,3 +126,22 @@ def test_lazy_and_eager_state_scaling(dv, chunk):
         assert_close(Y[:, :, h:h + 1], Y_ref, "bf16", f"Y head {h}")
         assert_close(O[:, :, h:h + 1], O_ref, "bf16", f"O head {h}")
         assert_close(Sf[:, h:h + 1], S_ref, "bf16", f"S head {h}")
+
+
+def test_state_pass_pieces():
+    """50 units split into 2 segments of 8 chunks: the state pass cuts the first
+    segment into pieces (about one CTA per SM) folded back by the combine pass."""
+    H = 50
+    cfg = _cfg(1, H, 1024, 128, 64, 93, z_dist=tuple((0.0, 2.0) if h % 2 else (5.0, 1.0) for h in range(H)))
+    path, segs = gret.prefill_path(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, cfg.chunk, gret.Dtype.BF16)
+    assert path == gret.Path.TC and segs == 2
+    inp = gi.prefill_inputs(cfg)
+    d = {k: v.cuda() for k, v in inp.items()}
+    O, Sf = gret.prefill(d["Q"], d["K"], d["V"], d["z"], d["G"], cfg.tau, cfg.chunk, eps=cfg.eps)
+    gret.check_device_status()
+    for h in (0, 1, 25, 49):
+        sl = lambda x: x[:, :, h:h + 1]
+        O_ref, _, S_ref = oracle.prefill(sl(inp["Q"]), sl(inp["K"]), sl(inp["V"]), sl(inp["z"]),
+                                         sl(inp["G"]), cfg.tau, cfg.eps)
+        assert_close(O[:, :, h:h + 1], O_ref, "bf16", f"O head {h}")
+        assert_close(Sf[:, h:h + 1], S_ref, "bf16", f"S head {h}")
