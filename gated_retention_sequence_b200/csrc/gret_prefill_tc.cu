@@ -48,7 +48,8 @@ using namespace sm100;
 
 constexpr int DK = 128;
 constexpr int kCW = 16;                 // compute warps: four per tensor-memory lane quarter
-constexpr int kCT = kCW * 32;           // threads per CTA (thread 0 also issues loads and MMAs)
+constexpr int kCT = kCW * 32;           // compute threads per fused CTA
+constexpr int kFusedThreads = kCT + 32; // + one issuer warp
 constexpr float kLazyMax = 40.0f;       // largest exponent the lazy state scale may reach
 
 template <int DV, int C>
@@ -86,13 +87,18 @@ struct Cfg {
     static constexpr int OFF_QT = OFF_P + P_BYTES;
     static constexpr int OFF_B = OFF_QT + QT_BYTES;         // NQK x C fp32 decay sums
     static constexpr int OFF_BAR = OFF_B + NQK * C * 4;
-    static constexpr int NUM_BARS = NQK + NV + NG + 3;
+    static constexpr int NUM_BARS = NQK + NV + NG + 6;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-    static constexpr int SMEM = OFF_MISC + 16 + 1024;      // + alignment slack
-    // epilogue scratch lives in the P buffer (P is dead during the epilogue)
-    static constexpr int OFF_RED = OFF_P;                   // kCW x HT x 2 fp32
-    static constexpr int OFF_STAT = OFF_P + kCW * HT * 2 * 4;  // C x (rstd, -mean * rstd)
-    static_assert(kCW * HT * 8 + C * 8 <= P_BYTES, "epilogue scratch fits in P");
+    // epilogue scratch: kCW x HT x 2 fp32 partial sums, then C x (rstd, -mean * rstd).
+    // It gets its own space when that fits; otherwise it lives in the P buffer
+    // (dead during the epilogue) and the warps meet once more before the next P.
+    static constexpr int RED_BYTES = kCW * HT * 2 * 4 + C * 8;
+    static constexpr int OFF_XRED = OFF_MISC + 16;
+    static constexpr bool SEP_RED = OFF_XRED + RED_BYTES + 1024 <= 227 * 1024;
+    static constexpr int OFF_RED = SEP_RED ? OFF_XRED : OFF_P;
+    static constexpr int OFF_STAT = OFF_RED + kCW * HT * 2 * 4;
+    static constexpr int SMEM = OFF_XRED + (SEP_RED ? RED_BYTES : 0) + 1024;   // + alignment slack
+    static_assert(SEP_RED || RED_BYTES <= P_BYTES, "epilogue scratch fits in P");
     static_assert(TM_USED <= 512, "tensor memory budget");
     static_assert(SMEM <= 227 * 1024, "shared memory budget");
     static_assert(C == 64 || C == 128, "chunk");
@@ -178,7 +184,15 @@ __device__ __forceinline__ void warp_transpose_sum(float (&v)[N], int lane) {
     transpose_sum_step<N, 16>(v, lane);
 }
 
-// Fused chunk loop (kFull) or state-only pass (!kFull) for one (unit, segment).
+// Fused chunk loop for one (unit, segment).
+//
+// Warps 0-15 compute, four per tensor-memory lane quarter.  Warp 16 is the
+// issuer: its lane 0 alone issues the TMA loads and stores and the tcgen05
+// MMAs and waits on their completion, so no compute warp ever stalls behind
+// the tensor pipe.  Each compute warp tells the issuer when its share of a
+// chunk's operands is ready (BPREP), when its share of an eager state rescale
+// is done (BTSC) and when its share of the output tile is staged in shared
+// memory (BSTAGED).
 //
 // State scaling.  Tensor memory holds T = S / E with E = e^Lambda, Lambda <= 0
 // and the same in every thread.  A chunk is "lazy" when its largest K scale
@@ -187,8 +201,10 @@ __device__ __forceinline__ void warp_transpose_sum(float (&v)[N], int lane) {
 // chunk is "eager": T is rescaled in place by e^{Lambda + b_C},
 // K~_s = e^{b_C - b_s} K_s and Lambda = 0.  The inter-chunk read uses
 // Q~_t = e^{b_t + Lambda} Q_t against T, and the state leaves as e^Lambda T.
-template <int DV, int C, bool kFull>
-__global__ void __launch_bounds__(kCT, 1) prefill_tc_kernel(const __grid_constant__ TcParams p) {
+// The issuer repeats the lazy/eager decision from the same decay sums with
+// the same float operations, so both sides agree on it.
+template <int DV, int C>
+__global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __grid_constant__ TcParams p) {
     using CF = Cfg<DV, C>;
     constexpr int NQK = CF::NQK, NV = CF::NV, NG = CF::NG, NH = CF::NH, W = CF::W, HT = CF::HT;
     constexpr bool TF32 = CF::TF32;
@@ -196,33 +212,34 @@ __global__ void __launch_bounds__(kCT, 1) prefill_tc_kernel(const __grid_constan
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int q4 = warp & 3;       // tensor-memory lane quarter of this warp
-    const int grp = warp >> 2;     // which of the four warps sharing the quarter
-    const uint32_t lq = (uint32_t)(32 * q4) << 16;
 
-    const int nseg = kFull ? p.P : p.P - 1;
-    const int u = blockIdx.x / nseg, seg = blockIdx.x % nseg;
+    const int u = blockIdx.x / p.P, seg = blockIdx.x % p.P;
     const int bb = u / p.H, hh = u % p.H;
     const int n_begin = seg * p.seg_len;
     const int n_end = min(p.N, n_begin + p.seg_len);
     const int nchunks = (n_end - n_begin + C - 1) / C;
 
-    const int BQK = 0, BV = NQK, BG = NQK + NV, BSC = NQK + NV + NG, BO = BSC + 1, BMMA = BSC + 2;
+    constexpr int BQK = 0, BV = NQK, BG = NQK + NV, BSC = NQK + NV + NG, BO = BSC + 1, BMMA = BSC + 2;
+    constexpr int BPREP = BSC + 3, BTSC = BSC + 4, BSTAGED = BSC + 5;
+    static_assert(BSTAGED + 1 == CF::NUM_BARS, "barrier count");
     auto bar = [&](int i) -> uint32_t { return sb + CF::OFF_BAR + 8 * i; };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + CF::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + CF::OFF_MISC + 4);
 
     if (tid == 0) {
-        for (int i = 0; i < CF::NUM_BARS; ++i) mbar_init(bar(i), 1);
+        for (int i = 0; i < CF::NUM_BARS; ++i) {
+            // per-warp arrivals; BSTAGED takes one arrival after a block barrier
+            // when the epilogue scratch shares the P buffer
+            const bool per_warp = i == BPREP || i == BTSC || (i == BSTAGED && CF::SEP_RED);
+            mbar_init(bar(i), per_warp ? kCW : 1);
+        }
         *abort_flag = 0;
         fence_mbar_init();
+        tma_prefetch_desc(&p.tmQ);
         tma_prefetch_desc(&p.tmK);
         tma_prefetch_desc(&p.tmV);
-        if (kFull) {
-            tma_prefetch_desc(&p.tmQ);
-            tma_prefetch_desc(&p.tmG);
-            tma_prefetch_desc(&p.tmO);
-        }
+        tma_prefetch_desc(&p.tmG);
+        tma_prefetch_desc(&p.tmO);
     }
     if (warp == 0) {
         tmem_alloc(smem_u32(tmem_slot), CF::TM_ALLOC);
@@ -233,106 +250,189 @@ __global__ void __launch_bounds__(kCT, 1) prefill_tc_kernel(const __grid_constan
     tc_fence_after();
     const uint32_t tm = *tmem_slot;
 
-    // ---- loads and MMAs, all issued by thread 0
-    auto issue_qk = [&](int j) {
-        const int s = j % NQK, n0 = n_begin + j * C;
-        const uint32_t fb = bar(BQK + s);
-        mbar_arrive_expect_tx(fb, CF::K_BYTES + C * 4 + (kFull ? CF::Q_BYTES : 0));
-        if (kFull)
-            for (int x = 0; x < 2; ++x)
-                tma_load_4d(sb + CF::OFF_Q + s * CF::Q_BYTES + x * CF::BOX, &p.tmQ, x * 64, hh, n0, bb, fb);
-        for (int x = 0; x < 2; ++x)
-            tma_load_4d(sb + CF::OFF_K + s * CF::K_BYTES + x * CF::BOX, &p.tmK, x * 64, hh, n0, bb, fb);
-        bulk_load(sb + CF::OFF_B + s * C * 4, p.bcum + (size_t)u * p.Npad + n0, C * 4, fb);
-    };
-    auto issue_v = [&](int j) {
-        const int s = j % NV, n0 = n_begin + j * C;
-        const uint32_t fb = bar(BV + s);
-        mbar_arrive_expect_tx(fb, CF::V_BYTES);
-        for (int x = 0; x < DV / 64; ++x)
-            tma_load_4d(sb + CF::OFF_V + s * CF::V_BYTES + x * CF::BOX, &p.tmV, x * 64, hh, n0, bb, fb);
-    };
-    auto issue_g = [&](int j) {
-        const int s = j % NG, n0 = n_begin + j * C;
-        const uint32_t fb = bar(BG + s);
-        mbar_arrive_expect_tx(fb, CF::G_BYTES);
-        for (int x = 0; x < DV / 64; ++x)
-            tma_load_4d(sb + CF::OFF_G + s * CF::G_BYTES + x * CF::BOX, &p.tmG, x * 64, hh, n0, bb, fb);
-    };
-    // scores D[t][s] = Q K^T over d_k (M = 128 rows of t; rows >= C unused)
-    auto issue_scores = [&](int j) {
-        const int s = j % NQK;
-        mbar_wait(bar(BQK + s), (j / NQK) & 1, p.status, abort_flag);
-        tc_fence_after();
-        const uint32_t sQ = sb + CF::OFF_Q + s * CF::Q_BYTES, sK = sb + CF::OFF_K + s * CF::K_BYTES;
-        constexpr uint32_t id = idesc_bf16(128, C, false, false);
+    if (warp == kCW) {
+        if (lane == 0 && nchunks > 0) {
+            // ============================================================ issuer
+            auto issue_qk = [&](int j) {
+                const int s = j % NQK, n0 = n_begin + j * C;
+                const uint32_t fb = bar(BQK + s);
+                mbar_arrive_expect_tx(fb, CF::Q_BYTES + CF::K_BYTES + C * 4);
+                for (int x = 0; x < 2; ++x) {
+                    tma_load_4d(sb + CF::OFF_Q + s * CF::Q_BYTES + x * CF::BOX, &p.tmQ, x * 64, hh, n0, bb, fb);
+                    tma_load_4d(sb + CF::OFF_K + s * CF::K_BYTES + x * CF::BOX, &p.tmK, x * 64, hh, n0, bb, fb);
+                }
+                bulk_load(sb + CF::OFF_B + s * C * 4, p.bcum + (size_t)u * p.Npad + n0, C * 4, fb);
+            };
+            auto issue_v = [&](int j) {
+                const int s = j % NV, n0 = n_begin + j * C;
+                const uint32_t fb = bar(BV + s);
+                mbar_arrive_expect_tx(fb, CF::V_BYTES);
+                for (int x = 0; x < DV / 64; ++x)
+                    tma_load_4d(sb + CF::OFF_V + s * CF::V_BYTES + x * CF::BOX, &p.tmV, x * 64, hh, n0, bb, fb);
+            };
+            auto issue_g = [&](int j) {
+                const int s = j % NG, n0 = n_begin + j * C;
+                const uint32_t fb = bar(BG + s);
+                mbar_arrive_expect_tx(fb, CF::G_BYTES);
+                for (int x = 0; x < DV / 64; ++x)
+                    tma_load_4d(sb + CF::OFF_G + s * CF::G_BYTES + x * CF::BOX, &p.tmG, x * 64, hh, n0, bb, fb);
+            };
+            // scores D[t][s] = Q K^T over d_k (M = 128 rows of t; rows >= C unused)
+            auto issue_scores = [&](int j) {
+                const int s = j % NQK;
+                mbar_wait(bar(BQK + s), (j / NQK) & 1, p.status, abort_flag);
+                tc_fence_after();
+                const uint32_t sQ = sb + CF::OFF_Q + s * CF::Q_BYTES, sK = sb + CF::OFF_K + s * CF::K_BYTES;
+                constexpr uint32_t id = idesc_bf16(128, C, false, false);
 #pragma unroll
-        for (int k = 0; k < DK / 16; ++k) {
-            const uint32_t off = (k >> 2) * CF::BOX + (k & 3) * 32;
-            mma_ss(tm + CF::TM_SC, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(sK + off, 16, 1024), id, k > 0);
-        }
-        mma_commit(bar(BSC));
-    };
-    // T^T += V^T K~ for both d_v halves
-    auto issue_state = [&](uint32_t sV, uint32_t sK) {
-        constexpr uint32_t id_kv = idesc_bf16(128, DK, true, true);
-#pragma unroll
-        for (int h = 0; h < NH; ++h) {
-#pragma unroll
-            for (int k = 0; k < C / 16; ++k)
-                mma_ss(tm + CF::TM_S + h * 128, sdesc_sw128(sV + 2 * h * CF::BOX + k * 2048, CF::BOX, 1024),
-                       sdesc_sw128(sK + k * 2048, CF::BOX, 1024), id_kv, 1);
-        }
-    };
-
-    if (tid == 0) {
-        issue_qk(0);
-        if (nchunks > 1) issue_qk(1);
-        issue_v(0);
-        if (NV == 2 && nchunks > 1) issue_v(1);
-        if (kFull && p.has_g) {
-            issue_g(0);
-            if (NG == 2 && nchunks > 1) issue_g(1);
-        }
-        if (kFull) issue_scores(0);
-    }
-
-    // this thread's slice of T^T: lanes of quarter q4, columns col0 .. col0 + W - 1
-    const int col0 = grp * W;
-    const int s_half = col0 / 128, s_k0 = col0 % 128;
-    const int s_d = s_half * 128 + q4 * 32 + lane;
-    {
-        uint32_t r[W];
-        if (kFull && seg > 0) {
-            const float* src = p.seg_state + ((size_t)u * (p.P - 1) * p.K + (size_t)seg * p.K - 1) * DV * DK +
-                               (size_t)s_d * DK + s_k0;
-            const float4* s4 = reinterpret_cast<const float4*>(src);
-#pragma unroll
-            for (int j = 0; j < W / 4; ++j) {
-                const float4 v = s4[j];
-                r[4 * j] = f2u(v.x); r[4 * j + 1] = f2u(v.y); r[4 * j + 2] = f2u(v.z); r[4 * j + 3] = f2u(v.w);
+                for (int k = 0; k < DK / 16; ++k) {
+                    const uint32_t off = (k >> 2) * CF::BOX + (k & 3) * 32;
+                    mma_ss(tm + CF::TM_SC, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(sK + off, 16, 1024), id,
+                           k > 0);
+                }
+                mma_commit(bar(BSC));
+            };
+            issue_qk(0);
+            if (nchunks > 1) issue_qk(1);
+            issue_v(0);
+            if (NV == 2 && nchunks > 1) issue_v(1);
+            if (p.has_g) {
+                issue_g(0);
+                if (NG == 2 && nchunks > 1) issue_g(1);
             }
-        } else {
+            issue_scores(0);
+
+            float lam = 0.f;
+            int nsplit = 0;
+            for (int i = 0; i < nchunks; ++i) {
+                const int sq = i % NQK, sv = i % NV, g = i % NG;
+                const uint32_t sQ = sb + CF::OFF_Q + sq * CF::Q_BYTES;
+                const uint32_t sK = sb + CF::OFF_K + sq * CF::K_BYTES;
+                const uint32_t sV = sb + CF::OFF_V + sv * CF::V_BYTES;
+                // the decay sums of chunk i landed before its scores were issued
+                const float bC = reinterpret_cast<const float*>(sm + CF::OFF_B + sq * C * 4)[C - 1];
+                const bool eager = (-bC - lam) > kLazyMax;
+
+                // P, Q~, K~ (and, with bf16 inter products, the bf16 copy of T) ready
+                mbar_wait(bar(BPREP), i & 1, p.status, abort_flag);
+                tc_fence_after();
+                mbar_wait(bar(BV + sv), (i / NV) & 1, p.status, abort_flag);
+                {
+                    constexpr uint32_t id_pv = idesc_bf16(128, C, true, false);
+                    constexpr uint32_t id_qs = idesc_bf16(128, C, false, false);
+                    constexpr uint32_t id_qs32 = idesc_tf32(128, C, false, false);
 #pragma unroll
-            for (int j = 0; j < W; ++j) r[j] = 0u;
+                    for (int h = 0; h < NH; ++h) {
+                        const uint32_t vA = sV + 2 * h * CF::BOX;   // d_v rows h*128 .. +127 (two boxes)
+                        // intra-chunk: O^T = V^T P^T
+#pragma unroll
+                        for (int k = 0; k < C / 16; ++k) {
+                            const uint32_t poff = (k >> 2) * CF::BOX + (k & 3) * 32;
+                            mma_ss(tm + CF::TM_O + h * C, sdesc_sw128(vA + k * 2048, CF::BOX, 1024),
+                                   sdesc_sw128(sb + CF::OFF_P + poff, 16, 1024), id_pv, k > 0);
+                        }
+                        // inter-chunk: O^T += T^T Q~^T
+                        if constexpr (TF32) {
+#pragma unroll
+                            for (int k = 0; k < DK / 8; ++k) {
+                                const uint32_t qoff = (k >> 2) * CF::BOX + (k & 3) * 32;
+                                mma_ts_tf32(tm + CF::TM_O + h * C, tm + CF::TM_S + h * 128 + k * 8,
+                                            sdesc_sw128(sb + CF::OFF_QT + qoff, 16, 1024), id_qs32, 1);
+                            }
+                        } else {
+#pragma unroll
+                            for (int k = 0; k < DK / 16; ++k) {
+                                const uint32_t qoff = (k >> 2) * CF::BOX + (k & 3) * 32;
+                                mma_ts(tm + CF::TM_O + h * C, tm + CF::TM_CP + h * 64 + k * 8,
+                                       sdesc_sw128(sQ + qoff, 16, 1024), id_qs, 1);
+                            }
+                        }
+                    }
+                    mma_commit(bar(BO));
+                }
+                if (TF32 && eager) {
+                    // T is rescaled between the inter-chunk read and the state MMA
+                    mbar_wait(bar(BTSC), nsplit & 1, p.status, abort_flag);
+                    ++nsplit;
+                    tc_fence_after();
+                }
+                // T^T += V^T K~ for both d_v halves
+                {
+                    constexpr uint32_t id_kv = idesc_bf16(128, DK, true, true);
+#pragma unroll
+                    for (int h = 0; h < NH; ++h) {
+#pragma unroll
+                        for (int k = 0; k < C / 16; ++k)
+                            mma_ss(tm + CF::TM_S + h * 128,
+                                   sdesc_sw128(sV + 2 * h * CF::BOX + k * 2048, CF::BOX, 1024),
+                                   sdesc_sw128(sK + k * 2048, CF::BOX, 1024), id_kv, 1);
+                    }
+                    mma_commit(bar(BMMA));
+                }
+                if (i + 1 < nchunks) issue_scores(i + 1);
+                lam = eager ? 0.f : lam + bC;
+
+                // once the state MMA is done this chunk's Q/K and V stages are free
+                mbar_wait(bar(BMMA), i & 1, p.status, abort_flag);
+                if (i + NQK < nchunks) issue_qk(i + NQK);
+                if (i + NV < nchunks) issue_v(i + NV);
+
+                // the output tile, written over G(i) in shared memory, goes out
+                mbar_wait(bar(BSTAGED), i & 1, p.status, abort_flag);
+                {
+                    const uint32_t sG = sb + CF::OFF_G + g * CF::G_BYTES;
+                    const int n0 = n_begin + i * C;
+                    for (int x = 0; x < DV / 64; ++x) tma_store_4d(&p.tmO, sG + x * CF::BOX, x * 64, hh, n0, bb);
+                    bulk_commit();
+                }
+                // as soon as the store has read the stage, it takes the G of chunk i + NG
+                bulk_wait_read<0>();
+                if (p.has_g && i + NG < nchunks) issue_g(i + NG);
+            }
+            bulk_wait<0>();
         }
-        tmem_st<W>(tm + lq + CF::TM_S + col0, r);
-        tmem_wait_st();
-    }
+    } else {
+        // ================================================================ compute warps
+        const int q4 = warp & 3;       // tensor-memory lane quarter of this warp
+        const int grp = warp >> 2;     // which of the four compute warps sharing the quarter
+        const uint32_t lq = (uint32_t)(32 * q4) << 16;
+        // every lane of this warp has finished its part of a step: one arrival
+        auto warp_arrive = [&](int b) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(b));
+        };
 
-    float lam = 0.f;          // Lambda
-    float seg_decay = 0.f;
-    for (int i = 0; i < nchunks; ++i) {
-        const int sq = i % NQK, sv = i % NV;
-        const uint32_t sQ = sb + CF::OFF_Q + sq * CF::Q_BYTES;
-        const uint32_t sK = sb + CF::OFF_K + sq * CF::K_BYTES;
-        const uint32_t sV = sb + CF::OFF_V + sv * CF::V_BYTES;
-        const float* bc = reinterpret_cast<const float*>(sm + CF::OFF_B + sq * C * 4);
-        mbar_wait(bar(BQK + sq), (i / NQK) & 1, p.status, abort_flag);
-        const float bC = bc[C - 1];
-        const bool eager = (-bC - lam) > kLazyMax;
+        // this thread's slice of T^T: lanes of quarter q4, columns col0 .. col0 + W - 1
+        const int col0 = grp * W;
+        const int s_half = col0 / 128, s_k0 = col0 % 128;
+        const int s_d = s_half * 128 + q4 * 32 + lane;
+        {
+            uint32_t r[W];
+            if (seg > 0) {
+                const float* src = p.seg_state + ((size_t)u * (p.P - 1) * p.K + (size_t)seg * p.K - 1) * DV * DK +
+                                   (size_t)s_d * DK + s_k0;
+                const float4* s4 = reinterpret_cast<const float4*>(src);
+#pragma unroll
+                for (int j = 0; j < W / 4; ++j) {
+                    const float4 v = s4[j];
+                    r[4 * j] = f2u(v.x); r[4 * j + 1] = f2u(v.y); r[4 * j + 2] = f2u(v.z); r[4 * j + 3] = f2u(v.w);
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < W; ++j) r[j] = 0u;
+            }
+            tmem_st<W>(tm + lq + CF::TM_S + col0, r);
+            tmem_wait_st();
+        }
 
-        if (kFull) {
+        float lam = 0.f;          // Lambda
+        for (int i = 0; i < nchunks; ++i) {
+            const int sq = i % NQK;
+            const float* bc = reinterpret_cast<const float*>(sm + CF::OFF_B + sq * C * 4);
+            mbar_wait(bar(BQK + sq), (i / NQK) & 1, p.status, abort_flag);
+            const float bC = bc[C - 1];
+            const bool eager = (-bC - lam) > kLazyMax;
+
             mbar_wait(bar(BSC), i & 1, p.status, abort_flag);
             tc_fence_after();
             // P[t][s] = A[t][s] e^{b_t - b_s} (s <= t) -> bf16, K-major rows t
@@ -362,189 +462,123 @@ __global__ void __launch_bounds__(kCT, 1) prefill_tc_kernel(const __grid_constan
                     *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
                 }
             }
-        }
-        // Q~ = e^{b_t + Lambda} Q (fp32 copy in tf32 mode, in place otherwise) and
-        // K~ = e^{-b_s - Lambda} K (lazy) or e^{b_C - b_s} K (eager), in place, as
-        // one list of 16-byte items.  With 64-token chunks the warps that own
-        // tensor-memory lanes 64..127 compute no P, so they take 3/4 of the list.
-        {
-            constexpr int NQI = kFull ? C * 16 : 0;
-            constexpr int NI = NQI + C * 16;
-            int it0, it1, step;
-            if constexpr (kFull && C == 64) {
-                constexpr int cut = NI * 3 / 4;
-                step = kCT / 2;
-                if (q4 >= 2) { it0 = (((grp << 1) | (q4 - 2)) << 5) + lane; it1 = cut; }
-                else { it0 = cut + (((grp << 1) | q4) << 5) + lane; it1 = NI; }
-            } else {
-                it0 = tid; it1 = NI; step = kCT;
-            }
-            uint8_t* Qp = sm + CF::OFF_Q + sq * CF::Q_BYTES;
-            uint8_t* Kp = sm + CF::OFF_K + sq * CF::K_BYTES;
-            for (int it = it0; it < it1; it += step) {
-                if (it < NQI) {
-                    if constexpr (TF32) {
-                        const int t = it >> 4, c = it & 15;   // row t, bf16 16-byte chunk c (d_k 8c .. 8c+7)
-                        const float f = __expf(bc[t] + lam);
-                        const uint4 w = *reinterpret_cast<const uint4*>(Qp + (c >> 3) * CF::BOX + t * 128 +
-                                                                        (((c & 7) ^ (t & 7)) << 4));
-                        const uint32_t* e = reinterpret_cast<const uint32_t*>(&w);
-                        float x[8];
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&e[j]));
-                            x[2 * j] = f2.x * f;
-                            x[2 * j + 1] = f2.y * f;
-                        }
-                        uint8_t* row = sm + CF::OFF_QT + (c >> 2) * CF::BOX + t * 128;
-                        const int lc = 2 * (c & 3);
-                        *reinterpret_cast<float4*>(row + ((lc ^ (t & 7)) << 4)) = make_float4(x[0], x[1], x[2], x[3]);
-                        *reinterpret_cast<float4*>(row + (((lc + 1) ^ (t & 7)) << 4)) =
-                            make_float4(x[4], x[5], x[6], x[7]);
-                    } else {
-                        const int row = (it >> 3) % C;
-                        scale_bf16x8(Qp + it * 16, __expf(bc[row] + lam));
-                    }
+            // Q~ = e^{b_t + Lambda} Q (fp32 copy in tf32 mode, in place otherwise) and
+            // K~ = e^{-b_s - Lambda} K (lazy) or e^{b_C - b_s} K (eager), in place, as
+            // one list of 16-byte items.  With 64-token chunks the warps that own
+            // tensor-memory lanes 64..127 compute no P, so they take 3/4 of the list.
+            {
+                constexpr int NQI = C * 16;
+                constexpr int NI = NQI + C * 16;
+                int it0, it1, step;
+                if constexpr (C == 64) {
+                    constexpr int cut = NI * 3 / 4;
+                    step = kCT / 2;
+                    if (q4 >= 2) { it0 = (((grp << 1) | (q4 - 2)) << 5) + lane; it1 = cut; }
+                    else { it0 = cut + (((grp << 1) | q4) << 5) + lane; it1 = NI; }
                 } else {
-                    const int ci = it - NQI;
-                    const int row = (ci >> 3) % C;
-                    const float ex = eager ? (bC - bc[row]) : (-bc[row] - lam);
-                    scale_bf16x8(Kp + ci * 16, __expf(ex));
+                    it0 = tid; it1 = NI; step = kCT;
+                }
+                uint8_t* Qp = sm + CF::OFF_Q + sq * CF::Q_BYTES;
+                uint8_t* Kp = sm + CF::OFF_K + sq * CF::K_BYTES;
+                for (int it = it0; it < it1; it += step) {
+                    if (it < NQI) {
+                        if constexpr (TF32) {
+                            const int t = it >> 4, c = it & 15;   // row t, bf16 16-byte chunk c (d_k 8c .. 8c+7)
+                            const float f = __expf(bc[t] + lam);
+                            const uint4 w = *reinterpret_cast<const uint4*>(Qp + (c >> 3) * CF::BOX + t * 128 +
+                                                                            (((c & 7) ^ (t & 7)) << 4));
+                            const uint32_t* e = reinterpret_cast<const uint32_t*>(&w);
+                            float x[8];
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&e[j]));
+                                x[2 * j] = f2.x * f;
+                                x[2 * j + 1] = f2.y * f;
+                            }
+                            uint8_t* row = sm + CF::OFF_QT + (c >> 2) * CF::BOX + t * 128;
+                            const int lc = 2 * (c & 3);
+                            *reinterpret_cast<float4*>(row + ((lc ^ (t & 7)) << 4)) =
+                                make_float4(x[0], x[1], x[2], x[3]);
+                            *reinterpret_cast<float4*>(row + (((lc + 1) ^ (t & 7)) << 4)) =
+                                make_float4(x[4], x[5], x[6], x[7]);
+                        } else {
+                            const int row = (it >> 3) % C;
+                            scale_bf16x8(Qp + it * 16, __expf(bc[row] + lam));
+                        }
+                    } else {
+                        const int ci = it - NQI;
+                        const int row = (ci >> 3) % C;
+                        const float ex = eager ? (bC - bc[row]) : (-bc[row] - lam);
+                        scale_bf16x8(Kp + ci * 16, __expf(ex));
+                    }
                 }
             }
-        }
-        // pass over T before the MMAs: bf16 copy (bf16 mode) and / or eager rescale;
-        // it needs the previous chunk's state MMA to have finished
-        const float escale = __expf(lam + bC);
-        if (kFull ? !TF32 : eager) {
-            if (kFull && i > 0) {
-                mbar_wait(bar(BMMA), (i - 1) & 1, p.status, abort_flag);
-                tc_fence_after();
-            }
-            uint32_t r[W];
-            tmem_ld<W>(tm + lq + CF::TM_S + col0, r);
-            tmem_wait_ld();
-            if constexpr (kFull && !TF32) {
+            // bf16 inter products: bf16 copy of T (and the eager rescale) before the
+            // MMAs; it needs the previous chunk's state MMA to have finished
+            const float escale = __expf(lam + bC);
+            if constexpr (!TF32) {
+                if (i > 0) {
+                    mbar_wait(bar(BMMA), (i - 1) & 1, p.status, abort_flag);
+                    tc_fence_after();
+                }
+                uint32_t r[W];
+                tmem_ld<W>(tm + lq + CF::TM_S + col0, r);
+                tmem_wait_ld();
                 uint32_t pk[W / 2];
 #pragma unroll
                 for (int j = 0; j < W / 2; ++j) pk[j] = pack_bf16x2(u2f(r[2 * j]), u2f(r[2 * j + 1]));
                 tmem_st<W / 2>(tm + lq + CF::TM_CP + col0 / 2, pk);
+                if (eager) {
+#pragma unroll
+                    for (int j = 0; j < W; ++j) r[j] = f2u(u2f(r[j]) * escale);
+                    tmem_st<W>(tm + lq + CF::TM_S + col0, r);
+                }
+                tmem_wait_st();
             }
-            if (eager) {
+            fence_proxy_async_smem();
+            tc_fence_before();
+            warp_arrive(BPREP);
+
+            // swish(G) while the output MMAs run (two G stages: G(i) landed long ago)
+            float sw[NH][HT];
+            if constexpr (CF::EARLY_SWISH) {
+                if (p.gn) {
+                    const int g = i % NG;
+                    if (p.has_g) mbar_wait(bar(BG + g), (i / NG) & 1, p.status, abort_flag);
+                    const uint8_t* Gp = sm + CF::OFF_G + g * CF::G_BYTES;
 #pragma unroll
-                for (int j = 0; j < W; ++j) r[j] = f2u(u2f(r[j]) * escale);
-                tmem_st<W>(tm + lq + CF::TM_S + col0, r);
-            }
-            tmem_wait_st();
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        named_bar_sync(1, kCT);
-        const bool split = kFull && TF32 && eager;   // rescale T between the inter read and the state MMA
-        if (tid == 0) {
-            tc_fence_after();
-            mbar_wait(bar(BV + sv), (i / NV) & 1, p.status, abort_flag);
-            if (kFull) {
-                constexpr uint32_t id_pv = idesc_bf16(128, C, true, false);
-                constexpr uint32_t id_qs = idesc_bf16(128, C, false, false);
-                constexpr uint32_t id_qs32 = idesc_tf32(128, C, false, false);
+                    for (int h = 0; h < NH; ++h) {
+                        const int d = h * 128 + q4 * 32 + lane;
+                        const int dj = d >> 6, dc = (d & 63) >> 3, de = (d & 7) * 2;
+                        const uint8_t* gcol = Gp + dj * CF::BOX + de;
 #pragma unroll
-                for (int h = 0; h < NH; ++h) {
-                    const uint32_t vA = sV + 2 * h * CF::BOX;   // d_v rows h*128 .. +127 (two boxes)
-#pragma unroll
-                    for (int k = 0; k < C / 16; ++k) {
-                        const uint32_t poff = (k >> 2) * CF::BOX + (k & 3) * 32;
-                        mma_ss(tm + CF::TM_O + h * C, sdesc_sw128(vA + k * 2048, CF::BOX, 1024),
-                               sdesc_sw128(sb + CF::OFF_P + poff, 16, 1024), id_pv, k > 0);
-                    }
-                    if constexpr (TF32) {
-#pragma unroll
-                        for (int k = 0; k < DK / 8; ++k) {
-                            const uint32_t qoff = (k >> 2) * CF::BOX + (k & 3) * 32;
-                            mma_ts_tf32(tm + CF::TM_O + h * C, tm + CF::TM_S + h * 128 + k * 8,
-                                        sdesc_sw128(sb + CF::OFF_QT + qoff, 16, 1024), id_qs32, 1);
-                        }
-                    } else {
-#pragma unroll
-                        for (int k = 0; k < DK / 16; ++k) {
-                            const uint32_t qoff = (k >> 2) * CF::BOX + (k & 3) * 32;
-                            mma_ts(tm + CF::TM_O + h * C, tm + CF::TM_CP + h * 64 + k * 8,
-                                   sdesc_sw128(sQ + qoff, 16, 1024), id_qs, 1);
+                        for (int j = 0; j < HT; ++j) {
+                            const int t = grp * HT + j;
+                            const float gv = __bfloat162float(
+                                *reinterpret_cast<const __nv_bfloat16*>(gcol + t * 128 + ((dc ^ (t & 7)) << 4)));
+                            sw[h][j] = __fdividef(gv, 1.0f + __expf(-gv));
                         }
                     }
                 }
-                mma_commit(bar(BO));
             }
-            if (kFull && NG == 1 && p.has_g && i >= 1) {
-                // single G stage: the previous chunk's output store has to have
-                // read the buffer before this chunk's G lands there; it arrives
-                // while the MMAs run
-                bulk_wait_read<0>();
-                issue_g(i);
-            }
-            if (!split) {
-                issue_state(sV, sK);
-                mma_commit(bar(BMMA));
-                if (kFull && i + 1 < nchunks) issue_scores(i + 1);
-            }
-        }
-        // swish(G) while the output MMAs run (two G stages: G(i) landed long ago)
-        float sw[NH][HT];
-        if constexpr (kFull && CF::EARLY_SWISH) {
-            if (p.gn) {
-                const int g = i % NG;
-                if (p.has_g) mbar_wait(bar(BG + g), (i / NG) & 1, p.status, abort_flag);
-                const uint8_t* Gp = sm + CF::OFF_G + g * CF::G_BYTES;
-#pragma unroll
-                for (int h = 0; h < NH; ++h) {
-                    const int d = h * 128 + q4 * 32 + lane;
-                    const int dj = d >> 6, dc = (d & 63) >> 3, de = (d & 7) * 2;
-                    const uint8_t* gcol = Gp + dj * CF::BOX + de;
-#pragma unroll
-                    for (int j = 0; j < HT; ++j) {
-                        const int t = grp * HT + j;
-                        const float gv = __bfloat162float(
-                            *reinterpret_cast<const __nv_bfloat16*>(gcol + t * 128 + ((dc ^ (t & 7)) << 4)));
-                        sw[h][j] = __fdividef(gv, 1.0f + __expf(-gv));
-                    }
-                }
-            }
-        }
-        if (kFull) {
             // the epilogue needs only the output MMAs; the state MMA runs on
             mbar_wait(bar(BO), i & 1, p.status, abort_flag);
             tc_fence_after();
-        }
-        if (split) {
-            uint32_t r[W];
-            tmem_ld<W>(tm + lq + CF::TM_S + col0, r);
-            tmem_wait_ld();
+            if (TF32 && eager) {
+                // the inter-chunk read has used T: rescale it before the state MMA
+                uint32_t r[W];
+                tmem_ld<W>(tm + lq + CF::TM_S + col0, r);
+                tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < W; ++j) r[j] = f2u(u2f(r[j]) * escale);
-            tmem_st<W>(tm + lq + CF::TM_S + col0, r);
-            tmem_wait_st();
-            tc_fence_before();
-            named_bar_sync(1, kCT);
-            if (tid == 0) {
-                tc_fence_after();
-                issue_state(sV, sK);
-                mma_commit(bar(BMMA));
-                if (i + 1 < nchunks) issue_scores(i + 1);
+                for (int j = 0; j < W; ++j) r[j] = f2u(u2f(r[j]) * escale);
+                tmem_st<W>(tm + lq + CF::TM_S + col0, r);
+                tmem_wait_st();
+                tc_fence_before();
+                warp_arrive(BTSC);
             }
-        }
-        seg_decay += bC;
-        lam = eager ? 0.f : lam + bC;
-        if (!kFull) {
-            mbar_wait(bar(BMMA), i & 1, p.status, abort_flag);
-            tc_fence_after();
-            if (tid == 0) {
-                if (i + NQK < nchunks) issue_qk(i + NQK);   // this K stage is free now
-                if (i + NV < nchunks) issue_v(i + NV);      // and this V stage
-            }
-        }
+            lam = eager ? 0.f : lam + bC;
 
-        if (kFull) {
-            // ---------------------------------------------------- epilogue
+            // -------------------------------------------------------- epilogue
             // Thread (q4, grp, lane) owns d_v channels h*128 + q4*32 + lane
             // (h < NH) for tokens grp*HT .. grp*HT + HT - 1.
             const int g = i % NG;
@@ -584,13 +618,6 @@ __global__ void __launch_bounds__(kCT, 1) prefill_tc_kernel(const __grid_constan
                     }
                 }
                 named_bar_sync(1, kCT);
-                if (tid == 0) {
-                    // this chunk's state MMA has had the whole reduction to finish:
-                    // its Q/K and V stages take the next loads
-                    mbar_wait(bar(BMMA), i & 1, p.status, abort_flag);
-                    if (i + NQK < nchunks) issue_qk(i + NQK);
-                    if (i + NV < nchunks) issue_v(i + NV);
-                }
                 if (tid < C) {
                     const int gg = tid / HT, tl = tid % HT;
                     float s1 = 0.f, s2 = 0.f;
@@ -605,11 +632,6 @@ __global__ void __launch_bounds__(kCT, 1) prefill_tc_kernel(const __grid_constan
                     stat[tid] = make_float2(rstd, -mean * rstd);
                 }
                 named_bar_sync(1, kCT);
-            }
-            if (!p.gn && tid == 0) {
-                mbar_wait(bar(BMMA), i & 1, p.status, abort_flag);
-                if (i + NQK < nchunks) issue_qk(i + NQK);
-                if (i + NV < nchunks) issue_v(i + NV);
             }
             int goff[NH];
 #pragma unroll
@@ -644,47 +666,28 @@ __global__ void __launch_bounds__(kCT, 1) prefill_tc_kernel(const __grid_constan
             }
             tc_fence_before();
             fence_proxy_async_smem();
-            named_bar_sync(1, kCT);
-            if (tid == 0) {
-                const int n0 = n_begin + i * C;
-                for (int x = 0; x < DV / 64; ++x) tma_store_4d(&p.tmO, smem_u32(Gp + x * CF::BOX), x * 64, hh, n0, bb);
-                bulk_commit();
-                const int j = i + 1;
-                if constexpr (NG == 2) {
-                    bulk_wait_read<1>();   // the store issued one chunk ago has read its buffer
-                    if (p.has_g && j >= NG && j < nchunks) issue_g(j);
-                }
+            if constexpr (CF::SEP_RED) {
+                warp_arrive(BSTAGED);
+            } else {
+                // the next chunk's P overwrites the statistics: every warp has read them
+                named_bar_sync(1, kCT);
+                if (tid == 0) mbar_arrive(bar(BSTAGED));
             }
         }
-    }
 
-    // ---------------------------------------------------------------- state out: e^Lambda T
-    {
-        if (kFull) {
-            if (tid == 0) bulk_wait<0>();
-            if (nchunks > 0) {
-                mbar_wait(bar(BMMA), (nchunks - 1) & 1, p.status, abort_flag);
-                tc_fence_after();
-            }
+        // ------------------------------------------------------------ state out: e^Lambda T
+        if (nchunks > 0) {
+            mbar_wait(bar(BMMA), (nchunks - 1) & 1, p.status, abort_flag);
+            tc_fence_after();
         }
-        const float sc = __expf(lam);
-        uint32_t r[W];
-        tmem_ld<W>(tm + lq + CF::TM_S + col0, r);
-        tmem_wait_ld();
-        if (kFull) {
-            if (p.S_final && seg == p.P - 1) {
-                float* dst = p.S_final + (size_t)u * DK * DV;
+        if (p.S_final && seg == p.P - 1) {
+            const float sc = __expf(lam);
+            uint32_t r[W];
+            tmem_ld<W>(tm + lq + CF::TM_S + col0, r);
+            tmem_wait_ld();
+            float* dst = p.S_final + (size_t)u * DK * DV;
 #pragma unroll
-                for (int j = 0; j < W; ++j) dst[(size_t)(s_k0 + j) * DV + s_d] = u2f(r[j]) * sc;
-            }
-        } else {
-            float4* d4 = reinterpret_cast<float4*>(p.seg_state + ((size_t)u * (p.P - 1) + seg) * DV * DK +
-                                                   (size_t)s_d * DK + s_k0);
-#pragma unroll
-            for (int j = 0; j < W / 4; ++j)
-                d4[j] = make_float4(u2f(r[4 * j]) * sc, u2f(r[4 * j + 1]) * sc, u2f(r[4 * j + 2]) * sc,
-                                    u2f(r[4 * j + 3]) * sc);
-            if (tid == 0) p.seg_decay[(size_t)u * (p.P - 1) + seg] = seg_decay;
+            for (int j = 0; j < W; ++j) dst[(size_t)(s_k0 + j) * DV + s_d] = u2f(r[j]) * sc;
         }
     }
     tc_fence_before();
@@ -973,7 +976,7 @@ WsLayout ws_layout(int B, int H, int N, int dk, int dv, int chunk, int segments,
 template <int DV, int C>
 cudaError_t run_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t s) {
     using CF = Cfg<DV, C>;
-    auto kf = prefill_tc_kernel<DV, C, true>;
+    auto kf = prefill_tc_kernel<DV, C>;
     auto ks = prefill_state_kernel<DV, C>;
     static bool attr_done[64] = {};
     int dev = 0;
@@ -994,7 +997,7 @@ cudaError_t run_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t s) {
                                                                              elems4);
     }
     if (g_profile_start) cudaEventRecord(g_profile_start, s);
-    kf<<<units * tp.P, kCT, CF::SMEM, s>>>(tp);
+    kf<<<units * tp.P, kFusedThreads, CF::SMEM, s>>>(tp);
     if (g_profile_stop) cudaEventRecord(g_profile_stop, s);
     return cudaGetLastError();
 }
