@@ -192,7 +192,7 @@ gret_status gret_last_device_status(gret_stream_t stream) {
     if (word != kDevOk) {
         unsigned int zero = 0;
         if (cudaMemcpy(status, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return GRET_ERR_CUDA;
-        return GRET_ERR_TIMEOUT;
+        return word == kDevTimeout ? GRET_ERR_TIMEOUT : GRET_ERR_CUDA;
     }
     return GRET_OK;
 }

@@ -9,9 +9,11 @@
 
 namespace gret {
 
-// Status word values a kernel writes when it gives up (host maps them to
-// GRET_ERR_TIMEOUT).  Kernels never trap.
-enum : unsigned int { kDevOk = 0u, kDevTimeout = 1u };
+// Status word values a kernel writes when it gives up: a bounded wait ran out
+// (host: GRET_ERR_TIMEOUT), or the dynamic shared memory base was not aligned
+// enough for the kernel's layout and it did nothing (host: GRET_ERR_CUDA).
+// Kernels never trap.
+enum : unsigned int { kDevOk = 0u, kDevTimeout = 1u, kDevSmemLayout = 2u };
 
 struct PrefillArgs {
     const void* Q;

@@ -37,6 +37,7 @@
 #include <cuda.h>
 
 #include <cstring>
+#include <type_traits>
 
 #include "gret_common.cuh"
 #include "gret_sm100.cuh"
@@ -51,6 +52,8 @@ constexpr int kCW = 16;                 // compute warps: four per tensor-memory
 constexpr int kCT = kCW * 32;           // compute threads per fused CTA
 constexpr int kFusedThreads = kCT + 32; // + one issuer warp
 constexpr float kLazyMax = 40.0f;       // largest exponent the lazy state scale may reach
+constexpr float kBlockMax = 40.0f;      // largest log-decay drop within one block of P columns
+constexpr int kMaxSmem = 227 * 1024;    // dynamic shared memory per block
 
 template <int DV, int C>
 struct Cfg {
@@ -85,22 +88,27 @@ struct Cfg {
     static constexpr int OFF_G = OFF_V + NV * V_BYTES;
     static constexpr int OFF_P = OFF_G + NG * G_BYTES;
     static constexpr int OFF_QT = OFF_P + P_BYTES;
-    static constexpr int OFF_B = OFF_QT + QT_BYTES;         // NQK x C fp32 decay sums
-    static constexpr int OFF_BAR = OFF_B + NQK * C * 4;
-    static constexpr int NUM_BARS = NQK + NV + NG + 6;
+    // per Q/K stage: C fp32 decay sums b_t, then C fp32 block factors (gate scan)
+    static constexpr int OFF_B = OFF_QT + QT_BYTES;
+    static constexpr int OFF_BAR = OFF_B + NQK * 2 * C * 4;
+    static constexpr int NUM_BARS = NQK + NV + NG + 7;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     // epilogue scratch: kCW x HT x 2 fp32 partial sums, then C x (rstd, -mean * rstd).
     // It gets its own space when that fits; otherwise it lives in the P buffer
     // (dead during the epilogue) and the warps meet once more before the next P.
     static constexpr int RED_BYTES = kCW * HT * 2 * 4 + C * 8;
     static constexpr int OFF_XRED = OFF_MISC + 16;
-    static constexpr bool SEP_RED = OFF_XRED + RED_BYTES + 1024 <= 227 * 1024;
+    static constexpr bool SEP_RED = OFF_XRED + RED_BYTES + 1024 <= kMaxSmem;
     static constexpr int OFF_RED = SEP_RED ? OFF_XRED : OFF_P;
     static constexpr int OFF_STAT = OFF_RED + kCW * HT * 2 * 4;
-    static constexpr int SMEM = OFF_XRED + (SEP_RED ? RED_BYTES : 0) + 1024;   // + alignment slack
+    static constexpr int USED = OFF_XRED + (SEP_RED ? RED_BYTES : 0);
+    // room to round the dynamic shared memory base up to 1024 bytes; where less
+    // than 1024 is left the kernel checks the base it got
+    static constexpr int SLACK = USED + 1024 <= kMaxSmem ? 1024 : kMaxSmem - USED;
+    static constexpr int SMEM = USED + SLACK;
+    static_assert(SLACK >= 0, "shared memory budget");
     static_assert(SEP_RED || RED_BYTES <= P_BYTES, "epilogue scratch fits in P");
     static_assert(TM_USED <= 512, "tensor memory budget");
-    static_assert(SMEM <= 227 * 1024, "shared memory budget");
     static_assert(C == 64 || C == 128, "chunk");
     static_assert(TF32 || NH == 1, "bf16 copy mode is laid out for one d_v half");
     // the padded rows (C..127) of the 128-row scores A operand read the bytes
@@ -111,6 +119,7 @@ struct Cfg {
 struct TcParams {
     CUtensorMap tmQ, tmK, tmV, tmG, tmO;
     const float* bcum;       // [units][Npad] chunk-local cumulative log-decay
+    const float* eblk;       // [units][Npad] block factors of the P columns (gate scan)
     float* seg_state;        // [units][(P-1)*K][DV][DK]  (S^T, fp32)
     float* seg_decay;        // [units][(P-1)*K]
     float* S_final;          // [units][DK][DV] or null
@@ -136,6 +145,15 @@ __device__ __forceinline__ void scale_bf16x8(uint8_t* p, float f) {
         e[j] = pack_bf16x2(x.x * f, x.y * f);
     }
     *reinterpret_cast<uint4*>(p) = w;
+}
+
+// swish(g) = g sigmoid(g) = h (1 + tanh h) with h = g / 2, so that it costs one
+// special-function operation (tanh.approx) instead of an exponential and a divide
+__device__ __forceinline__ float swish_fast(float g) {
+    const float h = 0.5f * g;
+    float th;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(th) : "f"(h));
+    return fmaf(h, th, h);
 }
 
 template <int N>
@@ -190,9 +208,10 @@ __device__ __forceinline__ void warp_transpose_sum(float (&v)[N], int lane) {
 // issuer: its lane 0 alone issues the TMA loads and stores and the tcgen05
 // MMAs and waits on their completion, so no compute warp ever stalls behind
 // the tensor pipe.  Each compute warp tells the issuer when its share of a
-// chunk's operands is ready (BPREP), when its share of an eager state rescale
-// is done (BTSC) and when its share of the output tile is staged in shared
-// memory (BSTAGED).
+// chunk's Q~ is ready (BQT: the inter-chunk MMAs start while P and K~ are
+// still being computed), when its share of P and K~ is ready (BPREP), when
+// its share of an eager state rescale is done (BTSC) and when its share of the
+// output tile is staged in shared memory (BSTAGED).
 //
 // State scaling.  Tensor memory holds T = S / E with E = e^Lambda, Lambda <= 0
 // and the same in every thread.  A chunk is "lazy" when its largest K scale
@@ -212,6 +231,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if constexpr (CF::SLACK < 1024) {
+        if (sm + CF::USED > smem_raw + CF::SMEM) {   // the base is not aligned enough: report, do nothing
+            if (tid == 0) atomicExch(p.status, kDevSmemLayout);
+            return;
+        }
+    }
 
     const int u = blockIdx.x / p.P, seg = blockIdx.x % p.P;
     const int bb = u / p.H, hh = u % p.H;
@@ -220,7 +245,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
     const int nchunks = (n_end - n_begin + C - 1) / C;
 
     constexpr int BQK = 0, BV = NQK, BG = NQK + NV, BSC = NQK + NV + NG, BO = BSC + 1, BMMA = BSC + 2;
-    constexpr int BPREP = BSC + 3, BTSC = BSC + 4, BSTAGED = BSC + 5;
+    constexpr int BQT = BSC + 3, BPREP = BSC + 4, BTSC = BSC + 5, BSTAGED = BSC + 6;
     static_assert(BSTAGED + 1 == CF::NUM_BARS, "barrier count");
     auto bar = [&](int i) -> uint32_t { return sb + CF::OFF_BAR + 8 * i; };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + CF::OFF_MISC);
@@ -230,7 +255,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
         for (int i = 0; i < CF::NUM_BARS; ++i) {
             // per-warp arrivals; BSTAGED takes one arrival after a block barrier
             // when the epilogue scratch shares the P buffer
-            const bool per_warp = i == BPREP || i == BTSC || (i == BSTAGED && CF::SEP_RED);
+            const bool per_warp = i == BQT || i == BPREP || i == BTSC || (i == BSTAGED && CF::SEP_RED);
             mbar_init(bar(i), per_warp ? kCW : 1);
         }
         *abort_flag = 0;
@@ -256,12 +281,13 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
             auto issue_qk = [&](int j) {
                 const int s = j % NQK, n0 = n_begin + j * C;
                 const uint32_t fb = bar(BQK + s);
-                mbar_arrive_expect_tx(fb, CF::Q_BYTES + CF::K_BYTES + C * 4);
+                mbar_arrive_expect_tx(fb, CF::Q_BYTES + CF::K_BYTES + 2 * C * 4);
                 for (int x = 0; x < 2; ++x) {
                     tma_load_4d(sb + CF::OFF_Q + s * CF::Q_BYTES + x * CF::BOX, &p.tmQ, x * 64, hh, n0, bb, fb);
                     tma_load_4d(sb + CF::OFF_K + s * CF::K_BYTES + x * CF::BOX, &p.tmK, x * 64, hh, n0, bb, fb);
                 }
-                bulk_load(sb + CF::OFF_B + s * C * 4, p.bcum + (size_t)u * p.Npad + n0, C * 4, fb);
+                bulk_load(sb + CF::OFF_B + s * 2 * C * 4, p.bcum + (size_t)u * p.Npad + n0, C * 4, fb);
+                bulk_load(sb + CF::OFF_B + (s * 2 + 1) * C * 4, p.eblk + (size_t)u * p.Npad + n0, C * 4, fb);
             };
             auto issue_v = [&](int j) {
                 const int s = j % NV, n0 = n_begin + j * C;
@@ -310,42 +336,49 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
                 const uint32_t sK = sb + CF::OFF_K + sq * CF::K_BYTES;
                 const uint32_t sV = sb + CF::OFF_V + sv * CF::V_BYTES;
                 // the decay sums of chunk i landed before its scores were issued
-                const float bC = reinterpret_cast<const float*>(sm + CF::OFF_B + sq * C * 4)[C - 1];
+                const float bC = reinterpret_cast<const float*>(sm + CF::OFF_B + sq * 2 * C * 4)[C - 1];
                 const bool eager = (-bC - lam) > kLazyMax;
 
-                // P, Q~, K~ (and, with bf16 inter products, the bf16 copy of T) ready
-                mbar_wait(bar(BPREP), i & 1, p.status, abort_flag);
+                // inter-chunk: O^T = T^T Q~^T, as soon as Q~ (and, with bf16 inter
+                // products, the bf16 copy of T) is ready
+                mbar_wait(bar(BQT), i & 1, p.status, abort_flag);
                 tc_fence_after();
-                mbar_wait(bar(BV + sv), (i / NV) & 1, p.status, abort_flag);
                 {
-                    constexpr uint32_t id_pv = idesc_bf16(128, C, true, false);
                     constexpr uint32_t id_qs = idesc_bf16(128, C, false, false);
                     constexpr uint32_t id_qs32 = idesc_tf32(128, C, false, false);
 #pragma unroll
                     for (int h = 0; h < NH; ++h) {
-                        const uint32_t vA = sV + 2 * h * CF::BOX;   // d_v rows h*128 .. +127 (two boxes)
-                        // intra-chunk: O^T = V^T P^T
-#pragma unroll
-                        for (int k = 0; k < C / 16; ++k) {
-                            const uint32_t poff = (k >> 2) * CF::BOX + (k & 3) * 32;
-                            mma_ss(tm + CF::TM_O + h * C, sdesc_sw128(vA + k * 2048, CF::BOX, 1024),
-                                   sdesc_sw128(sb + CF::OFF_P + poff, 16, 1024), id_pv, k > 0);
-                        }
-                        // inter-chunk: O^T += T^T Q~^T
                         if constexpr (TF32) {
 #pragma unroll
                             for (int k = 0; k < DK / 8; ++k) {
                                 const uint32_t qoff = (k >> 2) * CF::BOX + (k & 3) * 32;
                                 mma_ts_tf32(tm + CF::TM_O + h * C, tm + CF::TM_S + h * 128 + k * 8,
-                                            sdesc_sw128(sb + CF::OFF_QT + qoff, 16, 1024), id_qs32, 1);
+                                            sdesc_sw128(sb + CF::OFF_QT + qoff, 16, 1024), id_qs32, k > 0);
                             }
                         } else {
 #pragma unroll
                             for (int k = 0; k < DK / 16; ++k) {
                                 const uint32_t qoff = (k >> 2) * CF::BOX + (k & 3) * 32;
                                 mma_ts(tm + CF::TM_O + h * C, tm + CF::TM_CP + h * 64 + k * 8,
-                                       sdesc_sw128(sQ + qoff, 16, 1024), id_qs, 1);
+                                       sdesc_sw128(sQ + qoff, 16, 1024), id_qs, k > 0);
                             }
+                        }
+                    }
+                }
+                // intra-chunk: O^T += V^T P^T once P and K~ are ready
+                mbar_wait(bar(BPREP), i & 1, p.status, abort_flag);
+                tc_fence_after();
+                mbar_wait(bar(BV + sv), (i / NV) & 1, p.status, abort_flag);
+                {
+                    constexpr uint32_t id_pv = idesc_bf16(128, C, true, false);
+#pragma unroll
+                    for (int h = 0; h < NH; ++h) {
+                        const uint32_t vA = sV + 2 * h * CF::BOX;   // d_v rows h*128 .. +127 (two boxes)
+#pragma unroll
+                        for (int k = 0; k < C / 16; ++k) {
+                            const uint32_t poff = (k >> 2) * CF::BOX + (k & 3) * 32;
+                            mma_ss(tm + CF::TM_O + h * C, sdesc_sw128(vA + k * 2048, CF::BOX, 1024),
+                                   sdesc_sw128(sb + CF::OFF_P + poff, 16, 1024), id_pv, 1);
                         }
                     }
                     mma_commit(bar(BO));
@@ -428,95 +461,47 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
         float lam = 0.f;          // Lambda
         for (int i = 0; i < nchunks; ++i) {
             const int sq = i % NQK;
-            const float* bc = reinterpret_cast<const float*>(sm + CF::OFF_B + sq * C * 4);
+            const float* bc = reinterpret_cast<const float*>(sm + CF::OFF_B + sq * 2 * C * 4);
+            const float* eb = bc + C;     // block factors E_s
+            uint8_t* Qp = sm + CF::OFF_Q + sq * CF::Q_BYTES;
+            uint8_t* Kp = sm + CF::OFF_K + sq * CF::K_BYTES;
             mbar_wait(bar(BQK + sq), (i / NQK) & 1, p.status, abort_flag);
             const float bC = bc[C - 1];
             const bool eager = (-bC - lam) > kLazyMax;
-
-            mbar_wait(bar(BSC), i & 1, p.status, abort_flag);
-            tc_fence_after();
-            // P[t][s] = A[t][s] e^{b_t - b_s} (s <= t) -> bf16, K-major rows t
-            if (q4 * 32 < C) {
-                constexpr int PC = C / 4;
-                const int t = q4 * 32 + lane;
-                uint32_t r[PC];
-                tmem_ld<PC>(tm + lq + CF::TM_SC + grp * PC, r);
-                tmem_wait_ld();
-                const float bt = bc[t];
-#pragma unroll
-                for (int c8 = 0; c8 < PC / 8; ++c8) {
-                    const int s0 = grp * PC + c8 * 8;
-                    const float4 b0 = *reinterpret_cast<const float4*>(bc + s0);
-                    const float4 b1 = *reinterpret_cast<const float4*>(bc + s0 + 4);
-                    const float bs[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-                    uint32_t w[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int sa = s0 + 2 * e;
-                        const float v0 = sa <= t ? u2f(r[c8 * 8 + 2 * e]) * __expf(bt - bs[2 * e]) : 0.f;
-                        const float v1 = sa + 1 <= t ? u2f(r[c8 * 8 + 2 * e + 1]) * __expf(bt - bs[2 * e + 1]) : 0.f;
-                        w[e] = pack_bf16x2(v0, v1);
-                    }
-                    const int region = s0 >> 6, chunk = (s0 & 63) >> 3;
-                    uint8_t* dst = sm + CF::OFF_P + region * CF::BOX + t * 128 + ((chunk ^ (t & 7)) << 4);
-                    *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
-                }
-            }
-            // Q~ = e^{b_t + Lambda} Q (fp32 copy in tf32 mode, in place otherwise) and
-            // K~ = e^{-b_s - Lambda} K (lazy) or e^{b_C - b_s} K (eager), in place, as
-            // one list of 16-byte items.  With 64-token chunks the warps that own
-            // tensor-memory lanes 64..127 compute no P, so they take 3/4 of the list.
-            {
-                constexpr int NQI = C * 16;
-                constexpr int NI = NQI + C * 16;
-                int it0, it1, step;
-                if constexpr (C == 64) {
-                    constexpr int cut = NI * 3 / 4;
-                    step = kCT / 2;
-                    if (q4 >= 2) { it0 = (((grp << 1) | (q4 - 2)) << 5) + lane; it1 = cut; }
-                    else { it0 = cut + (((grp << 1) | q4) << 5) + lane; it1 = NI; }
-                } else {
-                    it0 = tid; it1 = NI; step = kCT;
-                }
-                uint8_t* Qp = sm + CF::OFF_Q + sq * CF::Q_BYTES;
-                uint8_t* Kp = sm + CF::OFF_K + sq * CF::K_BYTES;
-                for (int it = it0; it < it1; it += step) {
-                    if (it < NQI) {
-                        if constexpr (TF32) {
-                            const int t = it >> 4, c = it & 15;   // row t, bf16 16-byte chunk c (d_k 8c .. 8c+7)
-                            const float f = __expf(bc[t] + lam);
-                            const uint4 w = *reinterpret_cast<const uint4*>(Qp + (c >> 3) * CF::BOX + t * 128 +
-                                                                            (((c & 7) ^ (t & 7)) << 4));
-                            const uint32_t* e = reinterpret_cast<const uint32_t*>(&w);
-                            float x[8];
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&e[j]));
-                                x[2 * j] = f2.x * f;
-                                x[2 * j + 1] = f2.y * f;
-                            }
-                            uint8_t* row = sm + CF::OFF_QT + (c >> 2) * CF::BOX + t * 128;
-                            const int lc = 2 * (c & 3);
-                            *reinterpret_cast<float4*>(row + ((lc ^ (t & 7)) << 4)) =
-                                make_float4(x[0], x[1], x[2], x[3]);
-                            *reinterpret_cast<float4*>(row + (((lc + 1) ^ (t & 7)) << 4)) =
-                                make_float4(x[4], x[5], x[6], x[7]);
-                        } else {
-                            const int row = (it >> 3) % C;
-                            scale_bf16x8(Qp + it * 16, __expf(bc[row] + lam));
-                        }
-                    } else {
-                        const int ci = it - NQI;
-                        const int row = (ci >> 3) % C;
-                        const float ex = eager ? (bC - bc[row]) : (-bc[row] - lam);
-                        scale_bf16x8(Kp + ci * 16, __expf(ex));
-                    }
-                }
-            }
-            // bf16 inter products: bf16 copy of T (and the eager rescale) before the
-            // MMAs; it needs the previous chunk's state MMA to have finished
             const float escale = __expf(lam + bC);
-            if constexpr (!TF32) {
+
+            // ---- phase A: Q~ = e^{b_t + Lambda} Q for the inter-chunk read, which
+            // the issuer starts as soon as every warp has done its share
+            if constexpr (TF32) {
+                // fp32 copy in its own buffer, so the scores MMA may still be reading Q
+                for (int it = tid; it < C * 16; it += kCT) {
+                    const int t = it >> 4, c = it & 15;   // row t, bf16 16-byte chunk c (d_k 8c .. 8c+7)
+                    const float f = __expf(bc[t] + lam);
+                    const uint4 w = *reinterpret_cast<const uint4*>(Qp + (c >> 3) * CF::BOX + t * 128 +
+                                                                    (((c & 7) ^ (t & 7)) << 4));
+                    const uint32_t* e = reinterpret_cast<const uint32_t*>(&w);
+                    float x[8];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&e[j]));
+                        x[2 * j] = f2.x * f;
+                        x[2 * j + 1] = f2.y * f;
+                    }
+                    uint8_t* row = sm + CF::OFF_QT + (c >> 2) * CF::BOX + t * 128;
+                    const int lc = 2 * (c & 3);
+                    *reinterpret_cast<float4*>(row + ((lc ^ (t & 7)) << 4)) = make_float4(x[0], x[1], x[2], x[3]);
+                    *reinterpret_cast<float4*>(row + (((lc + 1) ^ (t & 7)) << 4)) =
+                        make_float4(x[4], x[5], x[6], x[7]);
+                }
+            } else {
+                // in place, once the scores MMA has read Q
+                mbar_wait(bar(BSC), i & 1, p.status, abort_flag);
+                tc_fence_after();
+                for (int it = tid; it < C * 16; it += kCT) {
+                    const int row = (it >> 3) % C;
+                    scale_bf16x8(Qp + it * 16, __expf(bc[row] + lam));
+                }
+                // bf16 copy of T (and the eager rescale); needs the previous state MMA
                 if (i > 0) {
                     mbar_wait(bar(BMMA), (i - 1) & 1, p.status, abort_flag);
                     tc_fence_after();
@@ -534,6 +519,77 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
                     tmem_st<W>(tm + lq + CF::TM_S + col0, r);
                 }
                 tmem_wait_st();
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            warp_arrive(BQT);
+
+            // ---- phase B: P and K~, for the intra-chunk and state MMAs
+            if constexpr (TF32) {
+                mbar_wait(bar(BSC), i & 1, p.status, abort_flag);
+                tc_fence_after();
+            }
+            // P[t][s] = A[t][s] e^{b_t - b_s} (s <= t) -> bf16, K-major rows t.  The
+            // gate scan gives E_s = e^{b_{s0} - b_s} with s0 the first of the C/4
+            // columns this warp owns, so e^{b_t - b_s} = e^{b_t - b_{s0}} E_s takes
+            // one exponential per row.  A block whose decay drops by more than
+            // kBlockMax is marked (E_{s0} < 0) and takes e^{b_t - b_s} directly.
+            if (q4 * 32 < C) {
+                constexpr int PC = C / 4;
+                const int t = q4 * 32 + lane;
+                const int sb0 = grp * PC;
+                uint32_t r[PC];
+                tmem_ld<PC>(tm + lq + CF::TM_SC + sb0, r);
+                const float bt = bc[t];
+                const bool fac = eb[sb0] >= 0.f;                 // the same for the whole warp
+                const float f = __expf(fminf(bt - bc[sb0], 0.f));
+                tmem_wait_ld();
+                auto emit = [&](auto fac_tag) {
+                    constexpr bool FAC = decltype(fac_tag)::value;
+                    const float* src = FAC ? eb : bc;
+#pragma unroll
+                    for (int c8 = 0; c8 < PC / 8; ++c8) {
+                        const int s0 = sb0 + c8 * 8;
+                        const float4 a0 = *reinterpret_cast<const float4*>(src + s0);
+                        const float4 a1 = *reinterpret_cast<const float4*>(src + s0 + 4);
+                        const float xs[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+                        uint32_t w[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int sa = s0 + 2 * e;
+                            const float m0 = FAC ? f * xs[2 * e] : __expf(bt - xs[2 * e]);
+                            const float m1 = FAC ? f * xs[2 * e + 1] : __expf(bt - xs[2 * e + 1]);
+                            const float v0 = sa <= t ? u2f(r[c8 * 8 + 2 * e]) * m0 : 0.f;
+                            const float v1 = sa + 1 <= t ? u2f(r[c8 * 8 + 2 * e + 1]) * m1 : 0.f;
+                            w[e] = pack_bf16x2(v0, v1);
+                        }
+                        const int region = s0 >> 6, chunk = (s0 & 63) >> 3;
+                        uint8_t* dst = sm + CF::OFF_P + region * CF::BOX + t * 128 + ((chunk ^ (t & 7)) << 4);
+                        *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+                    }
+                };
+                if (fac) emit(std::true_type{});
+                else emit(std::false_type{});
+            }
+            // K~ = e^{-b_s - Lambda} K (lazy) or e^{b_C - b_s} K (eager), in place, as
+            // 16-byte items.  With 64-token chunks the warps that own tensor-memory
+            // lanes 64..127 compute no P, so they take 3/4 of the items.
+            {
+                constexpr int NKI = C * 16;
+                int it0, it1, step;
+                if constexpr (C == 64) {
+                    constexpr int cut = NKI * 3 / 4;
+                    step = kCT / 2;
+                    if (q4 >= 2) { it0 = (((grp << 1) | (q4 - 2)) << 5) + lane; it1 = cut; }
+                    else { it0 = cut + (((grp << 1) | q4) << 5) + lane; it1 = NKI; }
+                } else {
+                    it0 = tid; it1 = NKI; step = kCT;
+                }
+                for (int it = it0; it < it1; it += step) {
+                    const int row = (it >> 3) % C;
+                    const float ex = eager ? (bC - bc[row]) : (-bc[row] - lam);
+                    scale_bf16x8(Kp + it * 16, __expf(ex));
+                }
             }
             fence_proxy_async_smem();
             tc_fence_before();
@@ -556,7 +612,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
                             const int t = grp * HT + j;
                             const float gv = __bfloat162float(
                                 *reinterpret_cast<const __nv_bfloat16*>(gcol + t * 128 + ((dc ^ (t & 7)) << 4)));
-                            sw[h][j] = __fdividef(gv, 1.0f + __expf(-gv));
+                            sw[h][j] = swish_fast(gv);
                         }
                     }
                 }
@@ -655,8 +711,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
                         if constexpr (CF::EARLY_SWISH) {
                             swv = sw[h][j];
                         } else {
-                            const float gv = __bfloat162float(*gp);
-                            swv = __fdividef(gv, 1.0f + __expf(-gv));
+                            swv = swish_fast(__bfloat162float(*gp));
                         }
                         // GroupNorm as one FMA, then times swish(g) = g * sigmoid(g)
                         o = fmaf(o, st.x, st.y) * swv;
@@ -886,10 +941,11 @@ __global__ void __launch_bounds__(kStateThreads, 1) prefill_state_kernel(const _
     }
 }
 
-// Chunk-local inclusive sums of log gamma: bcum[u][n] = sum_{j in chunk, j <= n} lg_j.
+// Chunk-local inclusive sums of log gamma: bcum[u][n] = sum_{j in chunk, j <= n} lg_j,
+// and the P step's block factors eblk (below).
 // Padding tokens (n >= N) carry lg = 0, so they repeat the chunk total.
-__global__ void gate_scan_kernel(const float* __restrict__ z, float* __restrict__ bcum, int H, int N,
-                                 int Npad, float inv_tau) {
+__global__ void gate_scan_kernel(const float* __restrict__ z, float* __restrict__ bcum, float* __restrict__ eblk,
+                                 int H, int N, int Npad, float inv_tau) {
     __shared__ float wsum[4];
     const int C = blockDim.x;
     const int u = blockIdx.x, b = u / H, h = u % H;
@@ -905,6 +961,16 @@ __global__ void gate_scan_kernel(const float* __restrict__ z, float* __restrict_
     __syncthreads();
     for (int j = 0; j < w; ++j) x += wsum[j];
     bcum[(size_t)u * Npad + n] = x;
+    // block factors for the P step: E_n = e^{b_{s0} - b_n}, s0 the first token of
+    // n's block of C/4 (16 or 32, within one warp); a block whose decay drops by
+    // more than kBlockMax gets E_{s0} = -1 instead, so the P step takes the
+    // exponentials directly there
+    const int bw = C / 4;
+    const float x0 = __shfl_sync(0xffffffffu, x, lane & ~(bw - 1));
+    const float xl = __shfl_sync(0xffffffffu, x, lane | (bw - 1));
+    float e = expf(x0 - x);
+    if (x0 - xl > kBlockMax) e = (lane & (bw - 1)) == 0 ? -1.f : 0.f;
+    eblk[(size_t)u * Npad + n] = e;
 }
 
 // Fold the segment increments into initial states, in place:
@@ -958,7 +1024,7 @@ bool make_map(CUtensorMap* m, const void* base, int d, int H, int N, int B, int 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct WsLayout {
-    size_t bcum, state, decay, total;
+    size_t bcum, eblk, state, decay, total;
 };
 
 WsLayout ws_layout(int B, int H, int N, int dk, int dv, int chunk, int segments, int pieces) {
@@ -966,7 +1032,8 @@ WsLayout ws_layout(int B, int H, int N, int dk, int dv, int chunk, int segments,
     const size_t npad = (size_t)((N + chunk - 1) / chunk) * chunk;
     WsLayout w;
     w.bcum = 0;
-    w.state = align256(units * npad * 4);
+    w.eblk = align256(units * npad * 4);
+    w.state = w.eblk + align256(units * npad * 4);
     const size_t slots = segments > 1 ? (size_t)(segments - 1) * pieces : 0;
     w.decay = w.state + align256(units * slots * (size_t)dk * dv * 4);
     w.total = w.decay + align256(units * slots * 4);
@@ -988,8 +1055,8 @@ cudaError_t run_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t s) {
     }
     const int units = a.B * a.H;
     const int npad = tp.Npad;
-    gate_scan_kernel<<<dim3(units, npad / C), C, 0, s>>>(a.z, const_cast<float*>(tp.bcum), a.H, a.N, npad,
-                                                         a.inv_tau);
+    gate_scan_kernel<<<dim3(units, npad / C), C, 0, s>>>(a.z, const_cast<float*>(tp.bcum), const_cast<float*>(tp.eblk),
+                                                         a.H, a.N, npad, a.inv_tau);
     if (tp.P > 1) {
         ks<<<units * (tp.P - 1) * tp.K, kStateThreads, StateCfg<DV, C>::SMEM, s>>>(tp);
         const int elems4 = DV * DK / 4;
@@ -1045,6 +1112,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
     const WsLayout w = ws_layout(a.B, a.H, a.N, a.dk, a.dv, C, a.segments, a.pieces);
     uint8_t* ws = static_cast<uint8_t*>(a.workspace);
     tp.bcum = reinterpret_cast<const float*>(ws + w.bcum);
+    tp.eblk = reinterpret_cast<const float*>(ws + w.eblk);
     tp.seg_state = reinterpret_cast<float*>(ws + w.state);
     tp.seg_decay = reinterpret_cast<float*>(ws + w.decay);
     tp.S_final = a.S_final;

@@ -144,10 +144,11 @@ gret_status gret_decode_step(const void* q, const void* k, const void* v, const 
                              gret_stream_t stream);
 
 /* Synchronises `stream`, then reports (and clears) the device status word that
- * kernels set when a bounded wait (an mbarrier or tensor-memory wait) gave up:
- * GRET_ERR_TIMEOUT in that case, GRET_ERR_CUDA if the stream reports an error,
- * else GRET_OK.  Kernels never trap; a timed-out kernel returns early and its
- * outputs are undefined. */
+ * kernels set when they give up: GRET_ERR_TIMEOUT when a bounded wait (an
+ * mbarrier or tensor-memory wait) ran out; GRET_ERR_CUDA when a kernel found
+ * its dynamic shared memory base too poorly aligned for its layout, or when the
+ * stream reports an error; else GRET_OK.  Kernels never trap; a kernel that
+ * gave up returns early and its outputs are undefined. */
 gret_status gret_last_device_status(gret_stream_t stream);
 
 /* Profiling aid.  While set (non-NULL), every gret_prefill call made from the
