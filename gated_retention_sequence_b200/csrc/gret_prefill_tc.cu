@@ -50,7 +50,14 @@ using namespace sm100;
 constexpr int DK = 128;
 constexpr int kCW = 16;                 // compute warps: four per tensor-memory lane quarter
 constexpr int kCT = kCW * 32;           // compute threads per fused CTA
-constexpr int kFusedThreads = kCT + 32; // + one issuer warp
+constexpr int kFusedThreads = kCT + 128; // + a warpgroup: an MMA-issuing warp, a TMA warp, two idle
+// Register split of the fused kernel: it is launched with 96 registers a
+// thread (65536 / 640, rounded down to 8); the issuing warpgroup gives up all
+// but kIssueRegs and the four compute warpgroups take kComputeRegs.
+constexpr int kLaunchRegs = 96;
+constexpr int kIssueRegs = 64;
+constexpr int kComputeRegs = 104;
+static_assert(4 * 128 * kComputeRegs + 128 * kIssueRegs <= kFusedThreads * kLaunchRegs, "register split");
 constexpr float kLazyMax = 40.0f;       // largest exponent the lazy state scale may reach
 constexpr float kBlockMax = 40.0f;      // largest log-decay drop within one block of P columns
 constexpr int kMaxSmem = 227 * 1024;    // dynamic shared memory per block
@@ -62,8 +69,11 @@ struct Cfg {
     static constexpr int NQK = 2;                           // Q/K stages
     static constexpr int NV = (DV == 128 && C == 64) ? 2 : 1;   // V stages
     static constexpr int NG = (C == 128) ? 1 : 2;           // G/O stages
-    // with two G stages the swish gate is computed while the output MMAs run
-    static constexpr bool EARLY_SWISH = (NG == 2);
+    // software pipeline: chunk i + 1 is prepared (and its MMAs run) while the
+    // epilogue of chunk i works from registers; needs two score buffers and
+    // epilogue scratch of its own
+    static constexpr bool PIPE = (C == 64);
+    static constexpr int NSCB = PIPE ? 2 : 1;               // score buffers
     static constexpr int ROWB = 128;                        // bytes per swizzled row
     static constexpr int BOX = C * ROWB;                    // one [C x 64] bf16 box
     static constexpr int Q_BYTES = 2 * BOX;                 // d_k = 128 -> 2 boxes
@@ -77,8 +87,8 @@ struct Cfg {
     // tensor-memory columns
     static constexpr int TM_S = 0;                          // T^T: NH x 128 fp32
     static constexpr int TM_O = NH * 128;                   // O^T: NH x C
-    static constexpr int TM_SC = TM_O + NH * C;             // scores: C
-    static constexpr int TM_CP = TM_SC + C;                 // bf16 copy of T^T (bf16 mode): NH x 64
+    static constexpr int TM_SC = TM_O + NH * C;             // scores: NSCB x C
+    static constexpr int TM_CP = TM_SC + NSCB * C;          // bf16 copy of T^T (bf16 mode): NH x 64
     static constexpr int TM_USED = TM_CP + (TF32 ? 0 : NH * 64);
     static constexpr int TM_ALLOC = TM_USED <= 256 ? 256 : 512;
     // shared memory (bytes from a 1024-aligned base)
@@ -91,7 +101,7 @@ struct Cfg {
     // per Q/K stage: C fp32 decay sums b_t, then C fp32 block factors (gate scan)
     static constexpr int OFF_B = OFF_QT + QT_BYTES;
     static constexpr int OFF_BAR = OFF_B + NQK * 2 * C * 4;
-    static constexpr int NUM_BARS = NQK + NV + NG + 7;
+    static constexpr int NUM_BARS = NQK + NV + NG + 10;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     // epilogue scratch: kCW x HT x 2 fp32 partial sums, then C x (rstd, -mean * rstd).
     // It gets its own space when that fits; otherwise it lives in the P buffer
@@ -108,6 +118,7 @@ struct Cfg {
     static constexpr int SMEM = USED + SLACK;
     static_assert(SLACK >= 0, "shared memory budget");
     static_assert(SEP_RED || RED_BYTES <= P_BYTES, "epilogue scratch fits in P");
+    static_assert(!PIPE || SEP_RED, "the pipelined epilogue needs scratch of its own");
     static_assert(TM_USED <= 512, "tensor memory budget");
     static_assert(C == 64 || C == 128, "chunk");
     static_assert(TF32 || NH == 1, "bf16 copy mode is laid out for one d_v half");
@@ -204,14 +215,21 @@ __device__ __forceinline__ void warp_transpose_sum(float (&v)[N], int lane) {
 
 // Fused chunk loop for one (unit, segment).
 //
-// Warps 0-15 compute, four per tensor-memory lane quarter.  Warp 16 is the
-// issuer: its lane 0 alone issues the TMA loads and stores and the tcgen05
-// MMAs and waits on their completion, so no compute warp ever stalls behind
-// the tensor pipe.  Each compute warp tells the issuer when its share of a
-// chunk's Q~ is ready (BQT: the inter-chunk MMAs start while P and K~ are
-// still being computed), when its share of P and K~ is ready (BPREP), when
-// its share of an eager state rescale is done (BTSC) and when its share of the
-// output tile is staged in shared memory (BSTAGED).
+// Roles.  Warps 0-15 compute, four per tensor-memory lane quarter.  In the
+// fifth warpgroup, lane 0 of warp 16 issues every tcgen05 MMA and lane 0 of
+// warp 17 every TMA load and store (warps 18-19 idle); the warpgroup hands
+// most of its registers to the compute warps (kIssueRegs / kComputeRegs).
+// Each compute warp tells the MMA warp when its share of a chunk's Q~ is
+// ready (BQT: the inter-chunk MMAs start while P and K~ are still being
+// computed), when its share of P and K~ is ready (BPREP), when its share of an
+// eager state rescale is done (BTSC), and tells the TMA warp when its share of
+// the output tile is staged in shared memory (BSTAGED).
+//
+// Schedule.  With 64-token chunks (PIPE) the compute warps take the output of
+// chunk i from tensor memory into registers, prepare chunk i + 1 -- whose
+// MMAs then run, its scores into the second score buffer -- and only then do
+// the GroupNorm epilogue of chunk i.  With 128-token chunks there is no room
+// for that, and each chunk is prepared, multiplied and finished in turn.
 //
 // State scaling.  Tensor memory holds T = S / E with E = e^Lambda, Lambda <= 0
 // and the same in every thread.  A chunk is "lazy" when its largest K scale
@@ -220,13 +238,13 @@ __device__ __forceinline__ void warp_transpose_sum(float (&v)[N], int lane) {
 // chunk is "eager": T is rescaled in place by e^{Lambda + b_C},
 // K~_s = e^{b_C - b_s} K_s and Lambda = 0.  The inter-chunk read uses
 // Q~_t = e^{b_t + Lambda} Q_t against T, and the state leaves as e^Lambda T.
-// The issuer repeats the lazy/eager decision from the same decay sums with
+// The MMA warp repeats the lazy/eager decision from the same decay sums with
 // the same float operations, so both sides agree on it.
 template <int DV, int C>
 __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __grid_constant__ TcParams p) {
     using CF = Cfg<DV, C>;
     constexpr int NQK = CF::NQK, NV = CF::NV, NG = CF::NG, NH = CF::NH, W = CF::W, HT = CF::HT;
-    constexpr bool TF32 = CF::TF32;
+    constexpr bool TF32 = CF::TF32, PIPE = CF::PIPE;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_u32(sm);
@@ -244,9 +262,17 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
     const int n_end = min(p.N, n_begin + p.seg_len);
     const int nchunks = (n_end - n_begin + C - 1) / C;
 
-    constexpr int BQK = 0, BV = NQK, BG = NQK + NV, BSC = NQK + NV + NG, BO = BSC + 1, BMMA = BSC + 2;
-    constexpr int BQT = BSC + 3, BPREP = BSC + 4, BTSC = BSC + 5, BSTAGED = BSC + 6;
-    static_assert(BSTAGED + 1 == CF::NUM_BARS, "barrier count");
+    // Barriers.  The scores, the state MMA and the staged output have one
+    // barrier per chunk parity, so that none of them can complete a phase
+    // twice before its slowest waiter has seen the first: the next phase of
+    // each pair needs a load that the waiter issues after its wait, or a step
+    // of its own.  (Unpipelined, the scores use the first of their pair.)
+    constexpr int BQK = 0, BV = NQK, BG = NQK + NV, BSC = NQK + NV + NG, BO = BSC + 2, BMMA = BSC + 3;
+    constexpr int BQT = BSC + 5, BPREP = BSC + 6, BTSC = BSC + 7, BSTAGED = BSC + 8;
+    static_assert(BSTAGED + 2 == CF::NUM_BARS, "barrier count");
+    // barrier and parity of the scores of chunk j
+    auto bsc = [&](int j) -> int { return PIPE ? BSC + (j & 1) : BSC; };
+    auto bsc_par = [&](int j) -> uint32_t { return PIPE ? (j >> 1) & 1 : j & 1; };
     auto bar = [&](int i) -> uint32_t { return sb + CF::OFF_BAR + 8 * i; };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + CF::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + CF::OFF_MISC + 4);
@@ -255,7 +281,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
         for (int i = 0; i < CF::NUM_BARS; ++i) {
             // per-warp arrivals; BSTAGED takes one arrival after a block barrier
             // when the epilogue scratch shares the P buffer
-            const bool per_warp = i == BQT || i == BPREP || i == BTSC || (i == BSTAGED && CF::SEP_RED);
+            const bool per_warp =
+                i == BQT || i == BPREP || i == BTSC || ((i == BSTAGED || i == BSTAGED + 1) && CF::SEP_RED);
             mbar_init(bar(i), per_warp ? kCW : 1);
         }
         *abort_flag = 0;
@@ -274,10 +301,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
     __syncthreads();
     tc_fence_after();
     const uint32_t tm = *tmem_slot;
-
-    if (warp == kCW) {
+    if (warp >= kCW) {
+      // ================================================================ issuing warpgroup
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" : : "n"(kIssueRegs));
+      if (warp == kCW + 1) {
         if (lane == 0 && nchunks > 0) {
-            // ============================================================ issuer
+            // ============================================================ producer
             auto issue_qk = [&](int j) {
                 const int s = j % NQK, n0 = n_begin + j * C;
                 const uint32_t fb = bar(BQK + s);
@@ -303,20 +332,16 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
                 for (int x = 0; x < DV / 64; ++x)
                     tma_load_4d(sb + CF::OFF_G + s * CF::G_BYTES + x * CF::BOX, &p.tmG, x * 64, hh, n0, bb, fb);
             };
-            // scores D[t][s] = Q K^T over d_k (M = 128 rows of t; rows >= C unused)
-            auto issue_scores = [&](int j) {
-                const int s = j % NQK;
-                mbar_wait(bar(BQK + s), (j / NQK) & 1, p.status, abort_flag);
-                tc_fence_after();
-                const uint32_t sQ = sb + CF::OFF_Q + s * CF::Q_BYTES, sK = sb + CF::OFF_K + s * CF::K_BYTES;
-                constexpr uint32_t id = idesc_bf16(128, C, false, false);
-#pragma unroll
-                for (int k = 0; k < DK / 16; ++k) {
-                    const uint32_t off = (k >> 2) * CF::BOX + (k & 3) * 32;
-                    mma_ss(tm + CF::TM_SC, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(sK + off, 16, 1024), id,
-                           k > 0);
-                }
-                mma_commit(bar(BSC));
+            // the output tile of chunk j, written over G(j) in shared memory, goes
+            // out; once the store has read the stage it takes the G of chunk j + NG
+            auto store_out = [&](int j) {
+                mbar_wait(bar(BSTAGED + (j & 1)), (j >> 1) & 1, p.status, abort_flag);
+                const uint32_t sG = sb + CF::OFF_G + (j % NG) * CF::G_BYTES;
+                const int n0 = n_begin + j * C;
+                for (int x = 0; x < DV / 64; ++x) tma_store_4d(&p.tmO, sG + x * CF::BOX, x * 64, hh, n0, bb);
+                bulk_commit();
+                bulk_wait_read<0>();
+                if (p.has_g && j + NG < nchunks) issue_g(j + NG);
             };
             issue_qk(0);
             if (nchunks > 1) issue_qk(1);
@@ -326,12 +351,46 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
                 issue_g(0);
                 if (NG == 2 && nchunks > 1) issue_g(1);
             }
+            for (int i = 0; i < nchunks; ++i) {
+                // pipelined, the epilogue of chunk i - 1 ends after chunk i's preparation
+                if (PIPE && i >= 1) store_out(i - 1);
+                // once the state MMA of chunk i is done, its Q/K and V stages are free
+                mbar_wait(bar(BMMA + (i & 1)), (i >> 1) & 1, p.status, abort_flag);
+                if (i + NQK < nchunks) issue_qk(i + NQK);
+                if (i + NV < nchunks) issue_v(i + NV);
+                if (!PIPE) store_out(i);
+            }
+            if (PIPE) store_out(nchunks - 1);
+            bulk_wait<0>();
+        }
+      } else if (warp == kCW) {
+        if (lane == 0 && nchunks > 0) {
+            // ============================================================ MMA issuer
+            constexpr uint32_t id_sc = idesc_bf16(128, C, false, false);
+            constexpr uint32_t id_qs = idesc_bf16(128, C, false, false);
+            constexpr uint32_t id_qs32 = idesc_tf32(128, C, false, false);
+            constexpr uint32_t id_pv = idesc_bf16(128, C, true, false);
+            constexpr uint32_t id_kv = idesc_bf16(128, DK, true, true);
+            // scores D[t][s] = Q K^T over d_k (M = 128 rows of t; rows >= C unused)
+            auto issue_scores = [&](int j) {
+                const int s = j % NQK;
+                mbar_wait(bar(BQK + s), (j / NQK) & 1, p.status, abort_flag);
+                tc_fence_after();
+                const uint32_t sQ = sb + CF::OFF_Q + s * CF::Q_BYTES, sK = sb + CF::OFF_K + s * CF::K_BYTES;
+                const uint32_t dst = tm + CF::TM_SC + (PIPE ? (j & 1) * C : 0);
+#pragma unroll
+                for (int k = 0; k < DK / 16; ++k) {
+                    const uint32_t off = (k >> 2) * CF::BOX + (k & 3) * 32;
+                    mma_ss(dst, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(sK + off, 16, 1024), id_sc, k > 0);
+                }
+                mma_commit(bar(bsc(j)));
+            };
             issue_scores(0);
 
             float lam = 0.f;
             int nsplit = 0;
             for (int i = 0; i < nchunks; ++i) {
-                const int sq = i % NQK, sv = i % NV, g = i % NG;
+                const int sq = i % NQK, sv = i % NV;
                 const uint32_t sQ = sb + CF::OFF_Q + sq * CF::Q_BYTES;
                 const uint32_t sK = sb + CF::OFF_K + sq * CF::K_BYTES;
                 const uint32_t sV = sb + CF::OFF_V + sv * CF::V_BYTES;
@@ -340,49 +399,47 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
                 const bool eager = (-bC - lam) > kLazyMax;
 
                 // inter-chunk: O^T = T^T Q~^T, as soon as Q~ (and, with bf16 inter
-                // products, the bf16 copy of T) is ready
+                // products, the bf16 copy of T) is ready and the previous state
+                // MMA has written T
                 mbar_wait(bar(BQT), i & 1, p.status, abort_flag);
+                if (i > 0) mbar_wait(bar(BMMA + ((i - 1) & 1)), ((i - 1) >> 1) & 1, p.status, abort_flag);
                 tc_fence_after();
-                {
-                    constexpr uint32_t id_qs = idesc_bf16(128, C, false, false);
-                    constexpr uint32_t id_qs32 = idesc_tf32(128, C, false, false);
 #pragma unroll
-                    for (int h = 0; h < NH; ++h) {
-                        if constexpr (TF32) {
+                for (int h = 0; h < NH; ++h) {
+                    if constexpr (TF32) {
 #pragma unroll
-                            for (int k = 0; k < DK / 8; ++k) {
-                                const uint32_t qoff = (k >> 2) * CF::BOX + (k & 3) * 32;
-                                mma_ts_tf32(tm + CF::TM_O + h * C, tm + CF::TM_S + h * 128 + k * 8,
-                                            sdesc_sw128(sb + CF::OFF_QT + qoff, 16, 1024), id_qs32, k > 0);
-                            }
-                        } else {
+                        for (int k = 0; k < DK / 8; ++k) {
+                            const uint32_t qoff = (k >> 2) * CF::BOX + (k & 3) * 32;
+                            mma_ts_tf32(tm + CF::TM_O + h * C, tm + CF::TM_S + h * 128 + k * 8,
+                                        sdesc_sw128(sb + CF::OFF_QT + qoff, 16, 1024), id_qs32, k > 0);
+                        }
+                    } else {
 #pragma unroll
-                            for (int k = 0; k < DK / 16; ++k) {
-                                const uint32_t qoff = (k >> 2) * CF::BOX + (k & 3) * 32;
-                                mma_ts(tm + CF::TM_O + h * C, tm + CF::TM_CP + h * 64 + k * 8,
-                                       sdesc_sw128(sQ + qoff, 16, 1024), id_qs, k > 0);
-                            }
+                        for (int k = 0; k < DK / 16; ++k) {
+                            const uint32_t qoff = (k >> 2) * CF::BOX + (k & 3) * 32;
+                            mma_ts(tm + CF::TM_O + h * C, tm + CF::TM_CP + h * 64 + k * 8,
+                                   sdesc_sw128(sQ + qoff, 16, 1024), id_qs, k > 0);
                         }
                     }
                 }
+                // pipelined: the next chunk's scores go to the other score buffer
+                // now, so that its P is ready to start when this chunk's output is
+                if (PIPE && i + 1 < nchunks) issue_scores(i + 1);
                 // intra-chunk: O^T += V^T P^T once P and K~ are ready
                 mbar_wait(bar(BPREP), i & 1, p.status, abort_flag);
                 tc_fence_after();
                 mbar_wait(bar(BV + sv), (i / NV) & 1, p.status, abort_flag);
-                {
-                    constexpr uint32_t id_pv = idesc_bf16(128, C, true, false);
 #pragma unroll
-                    for (int h = 0; h < NH; ++h) {
-                        const uint32_t vA = sV + 2 * h * CF::BOX;   // d_v rows h*128 .. +127 (two boxes)
+                for (int h = 0; h < NH; ++h) {
+                    const uint32_t vA = sV + 2 * h * CF::BOX;   // d_v rows h*128 .. +127 (two boxes)
 #pragma unroll
-                        for (int k = 0; k < C / 16; ++k) {
-                            const uint32_t poff = (k >> 2) * CF::BOX + (k & 3) * 32;
-                            mma_ss(tm + CF::TM_O + h * C, sdesc_sw128(vA + k * 2048, CF::BOX, 1024),
-                                   sdesc_sw128(sb + CF::OFF_P + poff, 16, 1024), id_pv, 1);
-                        }
+                    for (int k = 0; k < C / 16; ++k) {
+                        const uint32_t poff = (k >> 2) * CF::BOX + (k & 3) * 32;
+                        mma_ss(tm + CF::TM_O + h * C, sdesc_sw128(vA + k * 2048, CF::BOX, 1024),
+                               sdesc_sw128(sb + CF::OFF_P + poff, 16, 1024), id_pv, 1);
                     }
-                    mma_commit(bar(BO));
                 }
+                mma_commit(bar(BO));
                 if (TF32 && eager) {
                     // T is rescaled between the inter-chunk read and the state MMA
                     mbar_wait(bar(BTSC), nsplit & 1, p.status, abort_flag);
@@ -390,42 +447,22 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
                     tc_fence_after();
                 }
                 // T^T += V^T K~ for both d_v halves
-                {
-                    constexpr uint32_t id_kv = idesc_bf16(128, DK, true, true);
 #pragma unroll
-                    for (int h = 0; h < NH; ++h) {
+                for (int h = 0; h < NH; ++h) {
 #pragma unroll
-                        for (int k = 0; k < C / 16; ++k)
-                            mma_ss(tm + CF::TM_S + h * 128,
-                                   sdesc_sw128(sV + 2 * h * CF::BOX + k * 2048, CF::BOX, 1024),
-                                   sdesc_sw128(sK + k * 2048, CF::BOX, 1024), id_kv, 1);
-                    }
-                    mma_commit(bar(BMMA));
+                    for (int k = 0; k < C / 16; ++k)
+                        mma_ss(tm + CF::TM_S + h * 128, sdesc_sw128(sV + 2 * h * CF::BOX + k * 2048, CF::BOX, 1024),
+                               sdesc_sw128(sK + k * 2048, CF::BOX, 1024), id_kv, 1);
                 }
-                if (i + 1 < nchunks) issue_scores(i + 1);
+                mma_commit(bar(BMMA + (i & 1)));
+                if (!PIPE && i + 1 < nchunks) issue_scores(i + 1);
                 lam = eager ? 0.f : lam + bC;
-
-                // once the state MMA is done this chunk's Q/K and V stages are free
-                mbar_wait(bar(BMMA), i & 1, p.status, abort_flag);
-                if (i + NQK < nchunks) issue_qk(i + NQK);
-                if (i + NV < nchunks) issue_v(i + NV);
-
-                // the output tile, written over G(i) in shared memory, goes out
-                mbar_wait(bar(BSTAGED), i & 1, p.status, abort_flag);
-                {
-                    const uint32_t sG = sb + CF::OFF_G + g * CF::G_BYTES;
-                    const int n0 = n_begin + i * C;
-                    for (int x = 0; x < DV / 64; ++x) tma_store_4d(&p.tmO, sG + x * CF::BOX, x * 64, hh, n0, bb);
-                    bulk_commit();
-                }
-                // as soon as the store has read the stage, it takes the G of chunk i + NG
-                bulk_wait_read<0>();
-                if (p.has_g && i + NG < nchunks) issue_g(i + NG);
             }
-            bulk_wait<0>();
         }
+      }
     } else {
         // ================================================================ compute warps
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" : : "n"(kComputeRegs));
         const int q4 = warp & 3;       // tensor-memory lane quarter of this warp
         const int grp = warp >> 2;     // which of the four compute warps sharing the quarter
         const uint32_t lq = (uint32_t)(32 * q4) << 16;
@@ -459,7 +496,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
         }
 
         float lam = 0.f;          // Lambda
-        for (int i = 0; i < nchunks; ++i) {
+        struct ChunkGate { float bC, escale; bool eager; };
+
+        // ---- preparation of chunk i: Q~ (phase A), then P and K~ (phase B)
+        auto prep = [&](int i) -> ChunkGate {
             const int sq = i % NQK;
             const float* bc = reinterpret_cast<const float*>(sm + CF::OFF_B + sq * 2 * C * 4);
             const float* eb = bc + C;     // block factors E_s
@@ -470,8 +510,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
             const bool eager = (-bC - lam) > kLazyMax;
             const float escale = __expf(lam + bC);
 
-            // ---- phase A: Q~ = e^{b_t + Lambda} Q for the inter-chunk read, which
-            // the issuer starts as soon as every warp has done its share
+            // phase A: Q~ = e^{b_t + Lambda} Q for the inter-chunk read, which the
+            // issuer starts as soon as every warp has done its share
             if constexpr (TF32) {
                 // fp32 copy in its own buffer, so the scores MMA may still be reading Q
                 for (int it = tid; it < C * 16; it += kCT) {
@@ -495,7 +535,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
                 }
             } else {
                 // in place, once the scores MMA has read Q
-                mbar_wait(bar(BSC), i & 1, p.status, abort_flag);
+                mbar_wait(bar(bsc(i)), bsc_par(i), p.status, abort_flag);
                 tc_fence_after();
                 for (int it = tid; it < C * 16; it += kCT) {
                     const int row = (it >> 3) % C;
@@ -503,7 +543,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
                 }
                 // bf16 copy of T (and the eager rescale); needs the previous state MMA
                 if (i > 0) {
-                    mbar_wait(bar(BMMA), (i - 1) & 1, p.status, abort_flag);
+                    mbar_wait(bar(BMMA + ((i - 1) & 1)), ((i - 1) >> 1) & 1, p.status, abort_flag);
                     tc_fence_after();
                 }
                 uint32_t r[W];
@@ -524,9 +564,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
             tc_fence_before();
             warp_arrive(BQT);
 
-            // ---- phase B: P and K~, for the intra-chunk and state MMAs
+            // phase B: P and K~, for the intra-chunk and state MMAs
             if constexpr (TF32) {
-                mbar_wait(bar(BSC), i & 1, p.status, abort_flag);
+                mbar_wait(bar(bsc(i)), bsc_par(i), p.status, abort_flag);
                 tc_fence_after();
             }
             // P[t][s] = A[t][s] e^{b_t - b_s} (s <= t) -> bf16, K-major rows t.  The
@@ -539,7 +579,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
                 const int t = q4 * 32 + lane;
                 const int sb0 = grp * PC;
                 uint32_t r[PC];
-                tmem_ld<PC>(tm + lq + CF::TM_SC + sb0, r);
+                tmem_ld<PC>(tm + lq + CF::TM_SC + (PIPE ? (i & 1) * C : 0) + sb0, r);
                 const float bt = bc[t];
                 const bool fac = eb[sb0] >= 0.f;                 // the same for the whole warp
                 const float f = __expf(fminf(bt - bc[sb0], 0.f));
@@ -594,64 +634,51 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
             fence_proxy_async_smem();
             tc_fence_before();
             warp_arrive(BPREP);
+            return ChunkGate{bC, escale, eager};
+        };
 
-            // swish(G) while the output MMAs run (two G stages: G(i) landed long ago)
-            float sw[NH][HT];
-            if constexpr (CF::EARLY_SWISH) {
-                if (p.gn) {
-                    const int g = i % NG;
-                    if (p.has_g) mbar_wait(bar(BG + g), (i / NG) & 1, p.status, abort_flag);
-                    const uint8_t* Gp = sm + CF::OFF_G + g * CF::G_BYTES;
-#pragma unroll
-                    for (int h = 0; h < NH; ++h) {
-                        const int d = h * 128 + q4 * 32 + lane;
-                        const int dj = d >> 6, dc = (d & 63) >> 3, de = (d & 7) * 2;
-                        const uint8_t* gcol = Gp + dj * CF::BOX + de;
-#pragma unroll
-                        for (int j = 0; j < HT; ++j) {
-                            const int t = grp * HT + j;
-                            const float gv = __bfloat162float(
-                                *reinterpret_cast<const __nv_bfloat16*>(gcol + t * 128 + ((dc ^ (t & 7)) << 4)));
-                            sw[h][j] = swish_fast(gv);
-                        }
-                    }
-                }
-            }
-            // the epilogue needs only the output MMAs; the state MMA runs on
+        // ---- the output MMAs of chunk i are done: Y^T into registers, and the
+        // eager state rescale where the inter-chunk read had to see T unscaled
+        auto drain = [&](int i, const ChunkGate& cg, float (&y)[NH][HT]) {
             mbar_wait(bar(BO), i & 1, p.status, abort_flag);
             tc_fence_after();
-            if (TF32 && eager) {
-                // the inter-chunk read has used T: rescale it before the state MMA
-                uint32_t r[W];
-                tmem_ld<W>(tm + lq + CF::TM_S + col0, r);
-                tmem_wait_ld();
+            if (TF32 && cg.eager) {
+                // in two halves, to keep the live registers down
 #pragma unroll
-                for (int j = 0; j < W; ++j) r[j] = f2u(u2f(r[j]) * escale);
-                tmem_st<W>(tm + lq + CF::TM_S + col0, r);
+                for (int hw = 0; hw < 2; ++hw) {
+                    uint32_t r[W / 2];
+                    tmem_ld<W / 2>(tm + lq + CF::TM_S + col0 + hw * (W / 2), r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < W / 2; ++j) r[j] = f2u(u2f(r[j]) * cg.escale);
+                    tmem_st<W / 2>(tm + lq + CF::TM_S + col0 + hw * (W / 2), r);
+                }
                 tmem_wait_st();
                 tc_fence_before();
                 warp_arrive(BTSC);
             }
-            lam = eager ? 0.f : lam + bC;
-
-            // -------------------------------------------------------- epilogue
-            // Thread (q4, grp, lane) owns d_v channels h*128 + q4*32 + lane
-            // (h < NH) for tokens grp*HT .. grp*HT + HT - 1.
-            const int g = i % NG;
-            if (p.has_g && !CF::EARLY_SWISH) mbar_wait(bar(BG + g), (i / NG) & 1, p.status, abort_flag);
-            uint8_t* Gp = sm + CF::OFF_G + g * CF::G_BYTES;
-            const int t0 = grp * HT;
-            float* red = reinterpret_cast<float*>(sm + CF::OFF_RED);
-            float2* stat = reinterpret_cast<float2*>(sm + CF::OFF_STAT);
-            float y[NH][HT];
 #pragma unroll
             for (int h = 0; h < NH; ++h) {
                 uint32_t r[HT];
-                tmem_ld<HT>(tm + lq + CF::TM_O + h * C + t0, r);
+                tmem_ld<HT>(tm + lq + CF::TM_O + h * C + grp * HT, r);
                 tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < HT; ++j) y[h][j] = u2f(r[j]);
             }
+            tc_fence_before();
+        };
+
+        // ---- epilogue of chunk i from Y in registers: GroupNorm over d_v, times
+        // swish(G), as bf16 over G in its stage, then handed to the issuer for
+        // the store.  Thread (q4, grp, lane) owns d_v channels h*128 + q4*32 + lane
+        // (h < NH) for tokens grp*HT .. grp*HT + HT - 1.
+        auto epilogue = [&](int i, const float (&y)[NH][HT]) {
+            const int g = i % NG;
+            if (p.has_g) mbar_wait(bar(BG + g), (i / NG) & 1, p.status, abort_flag);
+            uint8_t* Gp = sm + CF::OFF_G + g * CF::G_BYTES;
+            const int t0 = grp * HT;
+            float* red = reinterpret_cast<float*>(sm + CF::OFF_RED);
+            float2* stat = reinterpret_cast<float2*>(sm + CF::OFF_STAT);
             if (p.gn) {
                 // per-token sums over this thread's channels, then over the
                 // warp's lanes, then over the four lane quarters
@@ -706,33 +733,44 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
                 for (int h = 0; h < NH; ++h) {
                     __nv_bfloat16* gp = reinterpret_cast<__nv_bfloat16*>(Gp + goff[h] + rowoff);
                     float o = y[h][j];
-                    if (p.gn) {
-                        float swv;
-                        if constexpr (CF::EARLY_SWISH) {
-                            swv = sw[h][j];
-                        } else {
-                            swv = swish_fast(__bfloat162float(*gp));
-                        }
-                        // GroupNorm as one FMA, then times swish(g) = g * sigmoid(g)
-                        o = fmaf(o, st.x, st.y) * swv;
-                    }
+                    // GroupNorm as one FMA, then times swish(g) = g * sigmoid(g)
+                    if (p.gn) o = fmaf(o, st.x, st.y) * swish_fast(__bfloat162float(*gp));
                     *gp = __float2bfloat16_rn(o);
                 }
             }
-            tc_fence_before();
             fence_proxy_async_smem();
             if constexpr (CF::SEP_RED) {
-                warp_arrive(BSTAGED);
+                warp_arrive(BSTAGED + (i & 1));
             } else {
                 // the next chunk's P overwrites the statistics: every warp has read them
                 named_bar_sync(1, kCT);
-                if (tid == 0) mbar_arrive(bar(BSTAGED));
+                if (tid == 0) mbar_arrive(bar(BSTAGED + (i & 1)));
+            }
+        };
+
+        if constexpr (PIPE) {
+            // Y(i) -> registers; prepare chunk i + 1 (its MMAs start); epilogue of i
+            ChunkGate cg = nchunks > 0 ? prep(0) : ChunkGate{0.f, 1.f, false};
+            for (int i = 0; i < nchunks; ++i) {
+                float y[NH][HT];
+                drain(i, cg, y);
+                lam = cg.eager ? 0.f : lam + cg.bC;
+                if (i + 1 < nchunks) cg = prep(i + 1);
+                epilogue(i, y);
+            }
+        } else {
+            for (int i = 0; i < nchunks; ++i) {
+                const ChunkGate cg = prep(i);
+                float y[NH][HT];
+                drain(i, cg, y);
+                lam = cg.eager ? 0.f : lam + cg.bC;
+                epilogue(i, y);
             }
         }
 
         // ------------------------------------------------------------ state out: e^Lambda T
         if (nchunks > 0) {
-            mbar_wait(bar(BMMA), (nchunks - 1) & 1, p.status, abort_flag);
+            mbar_wait(bar(BMMA + ((nchunks - 1) & 1)), ((nchunks - 1) >> 1) & 1, p.status, abort_flag);
             tc_fence_after();
         }
         if (p.S_final && seg == p.P - 1) {
@@ -1049,6 +1087,11 @@ cudaError_t run_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t s) {
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || !attr_done[dev]) {
+        // the register split inside the fused kernel draws on the registers it
+        // was launched with: never launch a build that has fewer
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, kf) != cudaSuccess) return cudaErrorInvalidDeviceFunction;
+        if (fa.numRegs * kFusedThreads < 4 * 128 * kComputeRegs + 128 * kIssueRegs) return cudaErrorInvalidConfiguration;
         cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, CF::SMEM);
         cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, StateCfg<DV, C>::SMEM);
         if (dev >= 0 && dev < 64) attr_done[dev] = true;
