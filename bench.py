@@ -34,6 +34,9 @@ sys.path.insert(0, ROOT)
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 METRIC = "gRet prefill Mtok/s & % bf16 TC peak; decode-step state GB/s & % HBM peak"
+# ncu summaries (under profiles/) that carry the DRAM traffic of the timed kernels
+PREFILL_PROFILE = "prefill_tc_kernel_B4_H16_N4096_dk128_dv256_C64.md"
+DECODE_PROFILE = "decode_step_kernel_S256_H16_dk128_dv256.md"
 
 
 def load_peaks():
@@ -159,8 +162,29 @@ def barrier(world):
         torch.cuda.synchronize()
 
 
-def cpu_oracle_sample(cfg, units, threads):
-    """Time the fp64 oracle (as it stands) on `units` (batch, head) units of cfg."""
+def profiled_traffic(kernel_file, source):
+    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) that
+    an ncu capture recorded in profiles/<kernel_file>, provided the capture was
+    taken of the kernel source as it is now (its sha256 prefix is written next
+    to the figure); None otherwise."""
+    import hashlib
+    import re
+    try:
+        with open(os.path.join(ROOT, "profiles", kernel_file)) as f:
+            text = f.read()
+        with open(os.path.join(ROOT, source), "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()
+    except OSError:
+        return None
+    m = re.search(r"^traffic_bytes_per_launch: (\d+) .*sha256 ([0-9a-f]{16})", text, re.M)
+    if not m or not digest.startswith(m.group(2)):
+        return None
+    return int(m.group(1))
+
+
+def cpu_oracle_sample(cfg, units, threads, min_seconds=0.0):
+    """Time the fp64 oracle (as it stands) on `units` (batch, head) units of cfg,
+    repeating the call until at least `min_seconds` have passed."""
     import gret_inputs as gi
     import oracle
     import torch
@@ -174,10 +198,15 @@ def cpu_oracle_sample(cfg, units, threads):
             torch.stack([p["z"] for p in per], 1)[None]
     Q, K, V, G, z = (stack(n) for n in ("Q", "K", "V", "G", "z"))
     t0 = time.perf_counter()
-    oracle.prefill(Q, K, V, z, G, cfg.tau, cfg.eps, threads=threads)
-    dt = time.perf_counter() - t0
-    tokens = units * cfg.N / cfg.H     # one unit = N tokens of one of H heads
-    return tokens / dt / 1e6, dt
+    passes = 0
+    while True:
+        oracle.prefill(Q, K, V, z, G, cfg.tau, cfg.eps, threads=threads)
+        passes += 1
+        dt = time.perf_counter() - t0
+        if dt >= min_seconds:
+            break
+    tokens = passes * units * cfg.N / cfg.H     # one unit = N tokens of one of H heads
+    return tokens / dt / 1e6, dt, passes
 
 
 def run_reference(args, world, rank):
@@ -191,7 +220,7 @@ def run_reference(args, world, rank):
     units = min(cfg.B * cfg.H, threads)
     vals = []
     for i in range(args.warmup + args.steps):
-        v, dt = cpu_oracle_sample(cfg, units, threads)
+        v, dt, _ = cpu_oracle_sample(cfg, units, threads)
         if i >= args.warmup:
             vals.append((v, dt))
     value = statistics.mean(v for v, _ in vals)
@@ -316,7 +345,8 @@ def run_ours(args, world, rank, local):
                          "frac": alg_bytes / step_s / 1e9 / peaks["hbm_gbs"]},
             "roofline": {"kernel": "prefill_tc_kernel (fused chunk loop)", "bound": "hbm",
                          "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                         "frac": achieved / peaks["hbm_gbs"],
+                         "traffic": profiled_traffic(PREFILL_PROFILE, "gated_retention_sequence_b200/csrc/gret_prefill_tc.cu"),
                          "alg_bytes_per_launch": alg_bytes, "launch_ms": kern_ms,
                          "peak_source": peaks["source"]},
             "e2e": {"value": e2e_value, "unit": "Mtok/s", "h2d_bytes_per_step": h2d,
@@ -328,11 +358,12 @@ def run_ours(args, world, rank, local):
         if world == 1 and not args.no_cpu_baseline:
             import oracle
             threads = oracle.default_threads()
-            units = min(cfg.B * cfg.H, 2 * threads)
-            v, dt = cpu_oracle_sample(cfg, units, threads)
+            units = cfg.B * cfg.H
+            v, dt, passes = cpu_oracle_sample(cfg, units, threads, min_seconds=10.0)
             line["cpu_baseline"] = {"value": v, "unit": "Mtok/s", "cores": threads, "kind": "oracle",
-                                    "sample": f"{units} (batch, head) units x {cfg.N} tokens of {cfg.name}, "
-                                              f"fp64 recurrent form + GroupNorm/swish, {dt:.1f} s"}
+                                    "sample": f"{passes} passes over all {units} (batch, head) units x {cfg.N} "
+                                              f"tokens of {cfg.name}, fp64 recurrent form + GroupNorm/swish, "
+                                              f"{dt:.1f} s"}
         print(json.dumps(line), flush=True)
     return 0
 
@@ -371,7 +402,8 @@ def run_decode(args, world, dev, stream, peaks):
             "state_gbs": world * bytes_ / (mean_ms / 1e3) / 1e9, "unit": "GB/s",
             "roofline": {"kernel": "decode_step_kernel", "bound": "hbm", "achieved": gbs,
                          "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
-                         "traffic": None, "alg_bytes_per_launch": bytes_,
+                         "traffic": profiled_traffic(DECODE_PROFILE, "gated_retention_sequence_b200/csrc/gret_decode.cu"),
+                         "alg_bytes_per_launch": bytes_,
                          "peak_source": peaks["source"]},
             "gpu_launches": T}
 

@@ -115,10 +115,10 @@ size_t gret_prefill_workspace_size(int B, int H, int N, int dk, int dv, int chun
     return prefill_tc_workspace_bytes(B, H, N, dk, dv, chunk, segs, pcs);
 }
 
-gret_status gret_prefill(const void* Q, const void* K, const void* V, const float* gate_logits,
-                         const void* G, float tau, int chunk, void* O, float* S_final, int B, int H,
-                         int N, int dk, int dv, gret_dtype io_dtype, float eps, gret_epilogue epi,
-                         void* workspace, size_t workspace_bytes, gret_stream_t stream) {
+static gret_status prefill_impl(const void* Q, const void* K, const void* V, const float* gate_logits,
+                                const void* G, const float* S0, float tau, int chunk, void* O, float* S_final,
+                                int B, int H, int N, int dk, int dv, gret_dtype io_dtype, float eps,
+                                gret_epilogue epi, void* workspace, size_t workspace_bytes, gret_stream_t stream) {
     if (!Q || !K || !V || !gate_logits || !O) return GRET_ERR_INVALID_ARG;
     if (epi != GRET_EPI_GN_SWISH && epi != GRET_EPI_NONE) return GRET_ERR_INVALID_ARG;
     if (epi == GRET_EPI_GN_SWISH && !G) return GRET_ERR_INVALID_ARG;
@@ -126,9 +126,15 @@ gret_status gret_prefill(const void* Q, const void* K, const void* V, const floa
     if (B <= 0 || H <= 0 || N <= 0 || dk <= 0 || dv <= 0 || chunk <= 0) return GRET_ERR_INVALID_ARG;
     if (!(tau > 0.0f) || !isfinite(tau) || !(eps >= 0.0f) || !isfinite(eps)) return GRET_ERR_INVALID_ARG;
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(gate_logits) || !aligned16(O) ||
-        (G && !aligned16(G)) || (S_final && !aligned16(S_final)))
+        (G && !aligned16(G)) || (S_final && !aligned16(S_final)) || (S0 && !aligned16(S0)))
         return GRET_ERR_INVALID_ARG;
     if ((long long)B * H > (1LL << 30) || (long long)B * N > (1LL << 40)) return GRET_ERR_UNSUPPORTED;
+    if (S0 && S_final) {
+        // segments of one unit run in different CTAs: S_final must not overwrite S0
+        const size_t bytes = (size_t)B * H * dk * dv * sizeof(float);
+        const uintptr_t a0 = reinterpret_cast<uintptr_t>(S0), a1 = reinterpret_cast<uintptr_t>(S_final);
+        if (a0 < a1 + bytes && a1 < a0 + bytes) return GRET_ERR_INVALID_ARG;
+    }
 
     unsigned int* status = nullptr;
     int sms = 0;
@@ -138,7 +144,7 @@ gret_status gret_prefill(const void* Q, const void* K, const void* V, const floa
     if (path == GRET_PATH_NONE) return GRET_ERR_UNSUPPORTED;
 
     PrefillArgs a;
-    a.Q = Q; a.K = K; a.V = V; a.z = gate_logits; a.G = G; a.O = O; a.S_final = S_final;
+    a.Q = Q; a.K = K; a.V = V; a.z = gate_logits; a.G = G; a.O = O; a.S_final = S_final; a.S0 = S0;
     a.B = B; a.H = H; a.N = N; a.dk = dk; a.dv = dv; a.chunk = chunk;
     a.inv_tau = 1.0f / tau; a.eps = eps; a.io = io_dtype; a.epi = epi;
     a.workspace = workspace; a.workspace_bytes = workspace_bytes;
@@ -157,6 +163,23 @@ gret_status gret_prefill(const void* Q, const void* K, const void* V, const floa
         err = launch_prefill_simt(a, s);
     }
     return err == cudaSuccess ? GRET_OK : GRET_ERR_CUDA;
+}
+
+gret_status gret_prefill(const void* Q, const void* K, const void* V, const float* gate_logits,
+                         const void* G, float tau, int chunk, void* O, float* S_final, int B, int H,
+                         int N, int dk, int dv, gret_dtype io_dtype, float eps, gret_epilogue epi,
+                         void* workspace, size_t workspace_bytes, gret_stream_t stream) {
+    return prefill_impl(Q, K, V, gate_logits, G, nullptr, tau, chunk, O, S_final, B, H, N, dk, dv, io_dtype, eps,
+                        epi, workspace, workspace_bytes, stream);
+}
+
+gret_status gret_prefill_from_state(const void* Q, const void* K, const void* V, const float* gate_logits,
+                                    const void* G, const float* S0, float tau, int chunk, void* O,
+                                    float* S_final, int B, int H, int N, int dk, int dv, gret_dtype io_dtype,
+                                    float eps, gret_epilogue epi, void* workspace, size_t workspace_bytes,
+                                    gret_stream_t stream) {
+    return prefill_impl(Q, K, V, gate_logits, G, S0, tau, chunk, O, S_final, B, H, N, dk, dv, io_dtype, eps, epi,
+                        workspace, workspace_bytes, stream);
 }
 
 gret_status gret_decode_step(const void* q, const void* k, const void* v, const float* gate_logit,

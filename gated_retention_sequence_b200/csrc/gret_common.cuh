@@ -23,6 +23,7 @@ struct PrefillArgs {
     const void* G;
     void* O;
     float* S_final;
+    const float* S0;          // initial state [B][H][dk][dv] fp32, or null for zero
     int B, H, N, dk, dv, chunk;
     float inv_tau, eps;
     gret_dtype io;

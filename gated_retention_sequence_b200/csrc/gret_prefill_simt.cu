@@ -37,7 +37,8 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(PrefillArgs a) {
     float* bc = As + (size_t)C * C;       // [C] cumulative log-decay
     float* wl = bc + C;                   // [C] e^{b_L - b_s}
 
-    for (int e = tid; e < dk * dv; e += kThreads) S[e] = 0.f;
+    const float* S0 = a.S0 ? a.S0 + (size_t)u * dk * dv : nullptr;
+    for (int e = tid; e < dk * dv; e += kThreads) S[e] = S0 ? S0[e] : 0.f;
 
     const T* Qg = static_cast<const T*>(a.Q);
     const T* Kg = static_cast<const T*>(a.K);

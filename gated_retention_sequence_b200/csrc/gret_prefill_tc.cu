@@ -134,6 +134,7 @@ struct TcParams {
     float* seg_state;        // [units][(P-1)*K][DV][DK]  (S^T, fp32)
     float* seg_decay;        // [units][(P-1)*K]
     float* S_final;          // [units][DK][DV] or null
+    const float* S0;         // [units][DK][DV] initial state, or null for zero
     unsigned int* status;
     int H, N, Npad, P, seg_len;
     int K, piece_len;        // state-pass pieces per segment and their length
@@ -487,6 +488,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
                     const float4 v = s4[j];
                     r[4 * j] = f2u(v.x); r[4 * j + 1] = f2u(v.y); r[4 * j + 2] = f2u(v.z); r[4 * j + 3] = f2u(v.w);
                 }
+            } else if (p.S0) {
+                // the caller's initial state, [DK][DV]: lanes read consecutive d_v
+                const float* src = p.S0 + (size_t)u * DK * DV + (size_t)s_k0 * DV + s_d;
+#pragma unroll
+                for (int j = 0; j < W; ++j) r[j] = f2u(src[(size_t)j * DV]);
             } else {
 #pragma unroll
                 for (int j = 0; j < W; ++j) r[j] = 0u;
@@ -1012,13 +1018,19 @@ __global__ void gate_scan_kernel(const float* __restrict__ z, float* __restrict_
 }
 
 // Fold the segment increments into initial states, in place:
-// slot p <- S_in(p + 1) = e^{a_p} S_in(p) + dS_p, with S_in(0) = 0.
-__global__ void seg_combine_kernel(float* __restrict__ seg_state, const float* __restrict__ seg_decay, int nslots,
-                                   int elems4) {
+// slot p <- S_in(p + 1) = e^{a_p} S_in(p) + dS_p, with S_in(0) = S0 (or 0).
+__global__ void seg_combine_kernel(float* __restrict__ seg_state, const float* __restrict__ seg_decay,
+                                   const float* __restrict__ S0, int nslots, int dk, int dv) {
     const int u = blockIdx.y;
+    const int elems4 = dk * dv / 4;
     const int e = blockIdx.x * blockDim.x + threadIdx.x;
     if (e >= elems4) return;
     float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (S0) {   // slots hold S^T [dv][dk]; S0 is [dk][dv]
+        const int d = (4 * e) / dk, k = (4 * e) % dk;
+        const float* s0 = S0 + (size_t)u * dk * dv + (size_t)k * dv + d;
+        run = make_float4(s0[0], s0[dv], s0[2 * dv], s0[3 * dv]);
+    }
     for (int p = 0; p < nslots; ++p) {
         float4* slot = reinterpret_cast<float4*>(seg_state) + ((size_t)u * nslots + p) * elems4 + e;
         const float f = __expf(seg_decay[(size_t)u * nslots + p]);
@@ -1103,8 +1115,8 @@ cudaError_t run_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t s) {
     if (tp.P > 1) {
         ks<<<units * (tp.P - 1) * tp.K, kStateThreads, StateCfg<DV, C>::SMEM, s>>>(tp);
         const int elems4 = DV * DK / 4;
-        seg_combine_kernel<<<dim3((elems4 + 255) / 256, units), 256, 0, s>>>(tp.seg_state, tp.seg_decay, (tp.P - 1) * tp.K,
-                                                                             elems4);
+        seg_combine_kernel<<<dim3((elems4 + 255) / 256, units), 256, 0, s>>>(tp.seg_state, tp.seg_decay, tp.S0,
+                                                                             (tp.P - 1) * tp.K, DK, DV);
     }
     if (g_profile_start) cudaEventRecord(g_profile_start, s);
     kf<<<units * tp.P, kFusedThreads, CF::SMEM, s>>>(tp);
@@ -1159,6 +1171,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
     tp.seg_state = reinterpret_cast<float*>(ws + w.state);
     tp.seg_decay = reinterpret_cast<float*>(ws + w.decay);
     tp.S_final = a.S_final;
+    tp.S0 = a.S0;
     tp.status = a.status;
     tp.H = a.H;
     tp.N = a.N;

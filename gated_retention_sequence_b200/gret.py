@@ -59,6 +59,8 @@ SIGNATURES = {
                           _VP, _SZ, _VP]),
     "gret_prefill_noalloc": (_I, [_VP, _VP, _VP, _FP, _VP, _F, _I, _VP, _FP, _I, _I, _I, _I, _I, _I, _F,
                                   _I, _VP]),
+    "gret_prefill_from_state": (_I, [_VP, _VP, _VP, _FP, _VP, _FP, _F, _I, _VP, _FP, _I, _I, _I, _I, _I, _I,
+                                     _F, _I, _VP, _SZ, _VP]),
     "gret_prefill_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
     "gret_prefill_path": (_I, [_I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_int)]),
     "gret_decode_step": (_I, [_VP, _VP, _VP, _FP, _VP, _FP, _VP, _I, _I, _I, _I, _F, _I, _F, _I, _VP]),
@@ -90,6 +92,12 @@ def gret_prefill(Q, K, V, gate_logits, G, tau, chunk, O, S_final, B, H, N, dk, d
                  epi, workspace, workspace_bytes, stream) -> int:
     return load().gret_prefill(Q, K, V, gate_logits, G, tau, chunk, O, S_final, B, H, N, dk, dv,
                                int(io_dtype), eps, int(epi), workspace, workspace_bytes, stream)
+
+
+def gret_prefill_from_state(Q, K, V, gate_logits, G, S0, tau, chunk, O, S_final, B, H, N, dk, dv, io_dtype,
+                            eps, epi, workspace, workspace_bytes, stream) -> int:
+    return load().gret_prefill_from_state(Q, K, V, gate_logits, G, S0, tau, chunk, O, S_final, B, H, N, dk, dv,
+                                          int(io_dtype), eps, int(epi), workspace, workspace_bytes, stream)
 
 
 def gret_prefill_noalloc(Q, K, V, gate_logits, G, tau, chunk, O, S_final, B, H, N, dk, dv, io_dtype, eps,
@@ -163,10 +171,11 @@ def _check(t, name, dtype, shape, device):
 
 
 def prefill(Q, K, V, z, G, tau: float, chunk: int, eps: float = 1e-5, epilogue: str = "gn_swish",
-            O=None, S_final=None, want_state: bool = True, workspace=None, stream=None):
-    """Chunkwise prefill from the zero state.
+            O=None, S_final=None, want_state: bool = True, workspace=None, stream=None, S0=None):
+    """Chunkwise prefill from the zero state, or from ``S0`` (gret_prefill_from_state).
 
-    Q, K [B,N,H,dk] and V, G [B,N,H,dv] in bf16 or fp32; z [B,N,H] fp32 gate logits.
+    Q, K [B,N,H,dk] and V, G [B,N,H,dv] in bf16 or fp32; z [B,N,H] fp32 gate logits;
+    S0 [B,H,dk,dv] fp32 or None.
     Returns (O [B,N,H,dv] in the io dtype, S_final [B,H,dk,dv] fp32 or None).
     ``epilogue='none'`` returns the pre-norm Y in O (G may be None).
     """
@@ -189,16 +198,24 @@ def prefill(Q, K, V, z, G, tau: float, chunk: int, eps: float = 1e-5, epilogue: 
         S_final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
     if S_final is not None:
         _check(S_final, "S_final", torch.float32, (B, H, dk, dv), dev)
+    if S0 is not None:
+        _check(S0, "S0", torch.float32, (B, H, dk, dv), dev)
     with torch.cuda.device(dev):
         ws_bytes = gret_prefill_workspace_size(B, H, N, dk, dv, chunk, io)
         if ws_bytes and (workspace is None or workspace.numel() * workspace.element_size() < ws_bytes):
             workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
         st = stream if stream is not None else torch.cuda.current_stream(dev)
-        status = gret_prefill(_ptr(Q), _ptr(K), _ptr(V), _ptr(z), _ptr(G), float(tau), int(chunk),
-                              _ptr(O), _ptr(S_final), B, H, N, dk, dv, io, float(eps), epi,
-                              _ptr(workspace) if ws_bytes else None, ws_bytes, st.cuda_stream)
+        ws = _ptr(workspace) if ws_bytes else None
+        if S0 is None:
+            status = gret_prefill(_ptr(Q), _ptr(K), _ptr(V), _ptr(z), _ptr(G), float(tau), int(chunk),
+                                  _ptr(O), _ptr(S_final), B, H, N, dk, dv, io, float(eps), epi, ws, ws_bytes,
+                                  st.cuda_stream)
+        else:
+            status = gret_prefill_from_state(_ptr(Q), _ptr(K), _ptr(V), _ptr(z), _ptr(G), _ptr(S0), float(tau),
+                                             int(chunk), _ptr(O), _ptr(S_final), B, H, N, dk, dv, io,
+                                             float(eps), epi, ws, ws_bytes, st.cuda_stream)
     if status != Status.OK:
-        raise GretError(status, "gret_prefill")
+        raise GretError(status, "gret_prefill" if S0 is None else "gret_prefill_from_state")
     return O, S_final
 
 

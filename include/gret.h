@@ -87,6 +87,30 @@ gret_status gret_prefill(const void* Q, const void* K, const void* V, const floa
                          gret_epilogue epi, void* workspace, size_t workspace_bytes,
                          gret_stream_t stream);
 
+/*
+ * gret_prefill_from_state -- gret_prefill that continues from a given state.
+ *
+ * "YOCO 深度技术分析", sections 5.3.2 and 5.3.3: between blocks, and between
+ * the devices of Chunk Parallelism, the only thing carried forward is the
+ * state S; a prefill that starts from S0 instead of zero is the step that
+ * continues a sequence (the next piece of a chunked prefill, or the next
+ * device's slice of a long one).  With S0 = S_prev the result equals one
+ * gret_prefill over the concatenated tokens, up to rounding.
+ *
+ *   S0 : fp32 [B][H][dk][dv] state before the first token (DEVICE, read
+ *        only), or NULL for the zero state (then this is gret_prefill).
+ *        16-byte aligned; must not overlap S_final (units are split into
+ *        segments that run concurrently, so S_final may be written before
+ *        every segment has read S0): keep two state buffers and alternate.
+ * Every other argument, the workspace size and the errors are those of
+ * gret_prefill; an S0 that overlaps S_final returns GRET_ERR_INVALID_ARG.
+ */
+gret_status gret_prefill_from_state(const void* Q, const void* K, const void* V, const float* gate_logits,
+                                    const void* G, const float* S0, float tau, int chunk, void* O,
+                                    float* S_final, int B, int H, int N, int dk, int dv,
+                                    gret_dtype io_dtype, float eps, gret_epilogue epi, void* workspace,
+                                    size_t workspace_bytes, gret_stream_t stream);
+
 /* Size of the device scratch array gret_prefill_noalloc draws on (32 MiB). */
 #define GRET_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
 

@@ -67,6 +67,20 @@ def test_prefill_rejects_bad_arguments(lib, over, expect):
     assert gret.gret_prefill(**_prefill_args(**over)) == expect
 
 
+def test_prefill_from_state_rejects_overlapping_states(lib):
+    # S0 and S_final overlapping: rejected before any GPU work (the pointers
+    # are never dereferenced, so this runs without a GPU)
+    a = _prefill_args(S_final=0x20000)
+    base = {k: a[k] for k in ("Q", "K", "V", "gate_logits", "G")}
+    rest = {k: a[k] for k in ("tau", "chunk", "O", "S_final", "B", "H", "N", "dk", "dv", "io_dtype", "eps", "epi",
+                              "workspace", "workspace_bytes", "stream")}
+    state_bytes = 1 * 2 * 64 * 64 * 4
+    for s0 in (0x20000, 0x20000 + state_bytes - 16, 0x20000 - state_bytes + 16):
+        assert gret.gret_prefill_from_state(**base, S0=s0, **rest) == gret.Status.ERR_INVALID_ARG
+    assert gret.gret_prefill_from_state(**base, S0=0x20008, **dict(rest, S_final=None)) == \
+        gret.Status.ERR_INVALID_ARG                                   # misaligned S0
+
+
 def test_decode_rejects_bad_arguments(lib):
     good = 0x10000
     base = dict(q=good, k=good, v=good, gate_logit=good, g=good, S_inout=good, o=good, num_seqs=4,
