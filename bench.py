@@ -292,7 +292,7 @@ def run_ours(args, world, rank, local):
     value = job_throughput(world, tokens, args.steps, ms) / 1e6
     alg_bytes, alg_flops = prefill_alg(cfg)
     step_s = ms / 1e3 / args.steps
-    launches_per_step = 2 + (2 if segs > 1 else 0)
+    launches_per_step = gret.gret_prefill_launches(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, cfg.chunk, io)
 
     # end to end through the public call: pinned host inputs in, O and S out
     pin = {k: v.pin_memory() for k, v in host.items()}

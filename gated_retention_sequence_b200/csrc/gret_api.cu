@@ -106,6 +106,14 @@ gret_path gret_prefill_path(int B, int H, int N, int dk, int dv, int chunk, gret
     return select_path(B, H, N, dk, dv, chunk, io_dtype, sms, segments, nullptr);
 }
 
+int gret_prefill_launches(int B, int H, int N, int dk, int dv, int chunk, gret_dtype io_dtype) {
+    int sms = 148, segs = 1, pcs = 1;
+    device_info(nullptr, &sms);
+    gret_path p = select_path(B, H, N, dk, dv, chunk, io_dtype, sms, &segs, nullptr, &pcs);
+    if (p == GRET_PATH_TC) return prefill_tc_launches(segs, pcs);
+    return p == GRET_PATH_SIMT ? 1 : 0;
+}
+
 size_t gret_prefill_workspace_size(int B, int H, int N, int dk, int dv, int chunk,
                                    gret_dtype io_dtype) {
     int sms = 148, segs = 1, pcs = 1;

@@ -93,5 +93,6 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s);
 bool prefill_tc_supported(int dk, int dv, int chunk, gret_dtype io);
 void prefill_tc_plan(int B, int H, int N, int chunk, int num_sms, int* segments, int* seg_len, int* pieces);
 size_t prefill_tc_workspace_bytes(int B, int H, int N, int dk, int dv, int chunk, int segments, int pieces);
+int prefill_tc_launches(int segments, int pieces);
 
 }  // namespace gret

@@ -58,7 +58,7 @@ constexpr int kLaunchRegs = 96;
 constexpr int kIssueRegs = 64;
 constexpr int kComputeRegs = 104;
 static_assert(4 * 128 * kComputeRegs + 128 * kIssueRegs <= kFusedThreads * kLaunchRegs, "register split");
-constexpr float kLazyMax = 40.0f;       // largest exponent the lazy state scale may reach
+constexpr float kLazyMax = 64.0f;       // largest exponent the lazy state scale may reach
 constexpr float kBlockMax = 40.0f;      // largest log-decay drop within one block of P columns
 constexpr int kMaxSmem = 227 * 1024;    // dynamic shared memory per block
 
@@ -521,7 +521,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
             if constexpr (TF32) {
                 // fp32 copy in its own buffer, so the scores MMA may still be reading Q
                 for (int it = tid; it < C * 16; it += kCT) {
-                    const int t = it >> 4, c = it & 15;   // row t, bf16 16-byte chunk c (d_k 8c .. 8c+7)
+                    // row t, bf16 16-byte chunk c (d_k 8c .. 8c+7); consecutive items are
+                    // consecutive rows, so the swizzle spreads each access phase over
+                    // eight different bank groups
+                    const int t = it % C, c = it / C;
                     const float f = __expf(bc[t] + lam);
                     const uint4 w = *reinterpret_cast<const uint4*>(Qp + (c >> 3) * CF::BOX + t * 128 +
                                                                     (((c & 7) ^ (t & 7)) << 4));
@@ -808,10 +811,13 @@ constexpr int kStateThreads = 256;
 template <int DV, int C>
 struct StateCfg {
     static constexpr int NH = DV / 128;
-    static constexpr int NS = (C * (2 * 128 + DV) * 2 <= 48 * 1024) ? 4 : 3;   // stages of K + V
     static constexpr int BOX = C * 128;
     static constexpr int K_BYTES = 2 * BOX;
     static constexpr int V_BYTES = (DV / 64) * BOX;
+    // as many K + V stages as about 200 KB hold (3-6), to keep loads in flight
+    static constexpr int NS_FIT = (200 * 1024) / (K_BYTES + V_BYTES);
+    static constexpr int NS = NS_FIT > 6 ? 6 : NS_FIT;
+    static_assert(NS >= 3, "state pass stages");
     static constexpr int W = NH * 64;                       // state columns per thread
     static constexpr int TM_ALLOC = NH * 128 <= 128 ? 128 : 256;
     static constexpr int OFF_K = 0;
@@ -937,11 +943,6 @@ __global__ void __launch_bounds__(kStateThreads, 1) prefill_state_kernel(const _
         __syncthreads();
         if (tid == 0) {
             tc_fence_after();
-            // the stage the previous chunk used is free once its MMA is done
-            if (i > 0 && i - 1 + NS < nchunks) {
-                mbar_wait(empty((i - 1) % NS), ((i - 1) / NS) & 1, p.status, abort_flag);
-                issue(i - 1 + NS);
-            }
             const uint32_t sK = sb + CF::OFF_K + s * CF::K_BYTES, sV = sb + CF::OFF_V + s * CF::V_BYTES;
             constexpr uint32_t id_kv = idesc_bf16(128, DK, true, true);
 #pragma unroll
@@ -952,6 +953,12 @@ __global__ void __launch_bounds__(kStateThreads, 1) prefill_state_kernel(const _
                            sdesc_sw128(sK + k * 2048, CF::BOX, 1024), id_kv, 1);
             }
             mma_commit(empty(s));
+            // the stage the previous chunk used is free once its MMAs are done
+            // (they run before this chunk's, which queue behind them)
+            if (i > 0 && i - 1 + NS < nchunks) {
+                mbar_wait(empty((i - 1) % NS), ((i - 1) / NS) & 1, p.status, abort_flag);
+                issue(i - 1 + NS);
+            }
         }
         seg_decay += bC;
         lam = eager ? 0.f : lam + bC;
@@ -1150,6 +1157,13 @@ void prefill_tc_plan(int B, int H, int N, int chunk, int num_sms, int* segments,
             if (per % k == 0) { K = k; break; }
     }
     *pieces = K;
+}
+
+// Kernel launches of one call: gate scan and fused loop, plus the state pass
+// and the combine for a split sequence.
+int prefill_tc_launches(int segments, int pieces) {
+    (void)pieces;
+    return segments <= 1 ? 2 : 4;
 }
 
 size_t prefill_tc_workspace_bytes(int B, int H, int N, int dk, int dv, int chunk, int segments, int pieces) {

@@ -62,6 +62,7 @@ SIGNATURES = {
     "gret_prefill_from_state": (_I, [_VP, _VP, _VP, _FP, _VP, _FP, _F, _I, _VP, _FP, _I, _I, _I, _I, _I, _I,
                                      _F, _I, _VP, _SZ, _VP]),
     "gret_prefill_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
+    "gret_prefill_launches": (_I, [_I, _I, _I, _I, _I, _I, _I]),
     "gret_prefill_path": (_I, [_I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_int)]),
     "gret_decode_step": (_I, [_VP, _VP, _VP, _FP, _VP, _FP, _VP, _I, _I, _I, _I, _F, _I, _F, _I, _VP]),
     "gret_last_device_status": (_I, [_VP]),
@@ -108,6 +109,10 @@ def gret_prefill_noalloc(Q, K, V, gate_logits, G, tau, chunk, O, S_final, B, H, 
 
 def gret_prefill_workspace_size(B, H, N, dk, dv, chunk, io_dtype) -> int:
     return load().gret_prefill_workspace_size(B, H, N, dk, dv, chunk, int(io_dtype))
+
+
+def gret_prefill_launches(B, H, N, dk, dv, chunk, io_dtype) -> int:
+    return load().gret_prefill_launches(B, H, N, dk, dv, chunk, int(io_dtype))
 
 
 def gret_prefill_path(B, H, N, dk, dv, chunk, io_dtype) -> Tuple[Path, int]:

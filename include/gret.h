@@ -146,6 +146,11 @@ gret_status gret_prefill_noalloc(const void* Q, const void* K, const void* V, co
 size_t gret_prefill_workspace_size(int B, int H, int N, int dk, int dv, int chunk,
                                    gret_dtype io_dtype);
 
+/* How many kernels one gret_prefill call with these arguments launches on its
+ * stream (gate scan, fused chunk loop, and for a split sequence the state pass
+ * and, with many pieces, the combine pass); 0 for unsupported arguments. */
+int gret_prefill_launches(int B, int H, int N, int dk, int dv, int chunk, gret_dtype io_dtype);
+
 /* Which kernel gret_prefill would run for these arguments, and into how many
  * sequence segments it splits each unit (1 = no split).  segments may be NULL. */
 gret_path gret_prefill_path(int B, int H, int N, int dk, int dv, int chunk, gret_dtype io_dtype,
