@@ -38,6 +38,7 @@
 
 #include <cstring>
 #include <type_traits>
+#include <utility>
 
 #include "gret_common.cuh"
 #include "gret_sm100.cuh"
@@ -302,6 +303,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
     __syncthreads();
     tc_fence_after();
     const uint32_t tm = *tmem_slot;
+    // the setup above overlaps the previous kernel's tail; from here on this
+    // kernel reads what the earlier ones wrote (decay sums, segment states)
+    grid_dep_launch();
+    grid_dep_wait();
     if (warp >= kCW) {
       // ================================================================ issuing warpgroup
       asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" : : "n"(kIssueRegs));
@@ -877,6 +882,10 @@ __global__ void __launch_bounds__(kStateThreads, 1) prefill_state_kernel(const _
             tma_load_4d(sb + CF::OFF_V + s * CF::V_BYTES + x * CF::BOX, &p.tmV, x * 64, hh, n0, bb, full(s));
         bulk_load(sb + CF::OFF_B + s * C * 4, p.bcum + (size_t)u * p.Npad + n0, C * 4, full(s));
     };
+    // everything above overlaps the previous kernel's tail; the loads need its
+    // decay sums
+    grid_dep_launch();
+    grid_dep_wait();
     if (tid == 0)
         for (int j = 0; j < NS && j < nchunks; ++j) issue(j);
 
@@ -998,6 +1007,10 @@ __global__ void __launch_bounds__(kStateThreads, 1) prefill_state_kernel(const _
 __global__ void gate_scan_kernel(const float* __restrict__ z, float* __restrict__ bcum, float* __restrict__ eblk,
                                  int H, int N, int Npad, float inv_tau) {
     __shared__ float wsum[4];
+    // the gate logits may come from the kernel before this one, and the kernels
+    // before that may still read the workspace: wait for them first
+    grid_dep_launch();
+    grid_dep_wait();
     const int C = blockDim.x;
     const int u = blockIdx.x, b = u / H, h = u % H;
     const int t = threadIdx.x, lane = t & 31, w = t >> 5;
@@ -1028,6 +1041,8 @@ __global__ void gate_scan_kernel(const float* __restrict__ z, float* __restrict_
 // slot p <- S_in(p + 1) = e^{a_p} S_in(p) + dS_p, with S_in(0) = S0 (or 0).
 __global__ void seg_combine_kernel(float* __restrict__ seg_state, const float* __restrict__ seg_decay,
                                    const float* __restrict__ S0, int nslots, int dk, int dv) {
+    grid_dep_launch();
+    grid_dep_wait();       // the state pass's increments
     const int u = blockIdx.y;
     const int elems4 = dk * dv / 4;
     const int e = blockIdx.x * blockDim.x + threadIdx.x;
@@ -1097,6 +1112,25 @@ WsLayout ws_layout(int B, int H, int N, int dk, int dv, int chunk, int segments,
     return w;
 }
 
+// Launch with programmatic stream serialisation: the kernel may start while the
+// one before it in the stream finishes; each kernel waits (grid_dep_wait)
+// before it touches what the earlier ones wrote.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 template <int DV, int C>
 cudaError_t run_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t s) {
     using CF = Cfg<DV, C>;
@@ -1117,17 +1151,21 @@ cudaError_t run_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t s) {
     }
     const int units = a.B * a.H;
     const int npad = tp.Npad;
-    gate_scan_kernel<<<dim3(units, npad / C), C, 0, s>>>(a.z, const_cast<float*>(tp.bcum), const_cast<float*>(tp.eblk),
-                                                         a.H, a.N, npad, a.inv_tau);
+    cudaError_t e = launch_pdl(gate_scan_kernel, dim3(units, npad / C), dim3(C), 0, s, a.z,
+                               const_cast<float*>(tp.bcum), const_cast<float*>(tp.eblk), a.H, a.N, npad, a.inv_tau);
+    if (e != cudaSuccess) return e;
     if (tp.P > 1) {
-        ks<<<units * (tp.P - 1) * tp.K, kStateThreads, StateCfg<DV, C>::SMEM, s>>>(tp);
+        e = launch_pdl(ks, dim3(units * (tp.P - 1) * tp.K), dim3(kStateThreads), StateCfg<DV, C>::SMEM, s, tp);
+        if (e != cudaSuccess) return e;
         const int elems4 = DV * DK / 4;
-        seg_combine_kernel<<<dim3((elems4 + 255) / 256, units), 256, 0, s>>>(tp.seg_state, tp.seg_decay, tp.S0,
-                                                                             (tp.P - 1) * tp.K, DK, DV);
+        e = launch_pdl(seg_combine_kernel, dim3((elems4 + 255) / 256, units), dim3(256), 0, s, tp.seg_state,
+                       static_cast<const float*>(tp.seg_decay), tp.S0, (tp.P - 1) * tp.K, DK, DV);
+        if (e != cudaSuccess) return e;
     }
     if (g_profile_start) cudaEventRecord(g_profile_start, s);
-    kf<<<units * tp.P, kFusedThreads, CF::SMEM, s>>>(tp);
+    e = launch_pdl(kf, dim3(units * tp.P), dim3(kFusedThreads), CF::SMEM, s, tp);
     if (g_profile_stop) cudaEventRecord(g_profile_stop, s);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

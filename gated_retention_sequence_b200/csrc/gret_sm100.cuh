@@ -63,6 +63,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigne
 }
 
 // ---------------------------------------------------------------- fences
+// Programmatic dependent launch.  grid_dep_wait: block until the grid this one
+// was launched behind has completed and its writes are visible (returns at once
+// for a normal launch).  grid_dep_launch: let the next grid in the stream start
+// launching now; it still waits for this one before it reads what this one writes.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
