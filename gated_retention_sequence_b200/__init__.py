@@ -5,7 +5,8 @@ runs entirely in the CUDA library ``libgret.so`` built from ``csrc/``; this
 package only marshals arguments (see ``gret.py``).
 """
 from .gret import (  # noqa: F401
-    Dtype, Epilogue, GretError, LIB_PATH, Path, SIGNATURES, Status, check_device_status,
-    decode_step, gret_decode_step, gret_last_device_status, gret_prefill, gret_prefill_from_state, gret_prefill_launches, gret_prefill_noalloc, gret_prefill_path,
-    gret_prefill_workspace_size, gret_set_profile_events, gret_status_string, gret_version, load, prefill, prefill_path,
+    Dtype, Epilogue, GretError, LIB_PATH, Path, SIGNATURES, Status, check_device_status, decode_step,
+    gret_decode_step, gret_last_device_status, gret_prefill, gret_prefill_from_state, gret_prefill_launches,
+    gret_prefill_noalloc, gret_prefill_path, gret_prefill_varlen, gret_prefill_workspace_size,
+    gret_set_profile_events, gret_status_string, gret_version, load, prefill, prefill_path, prefill_varlen,
 )

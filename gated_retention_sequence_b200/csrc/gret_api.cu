@@ -124,9 +124,10 @@ size_t gret_prefill_workspace_size(int B, int H, int N, int dk, int dv, int chun
 }
 
 static gret_status prefill_impl(const void* Q, const void* K, const void* V, const float* gate_logits,
-                                const void* G, const float* S0, float tau, int chunk, void* O, float* S_final,
-                                int B, int H, int N, int dk, int dv, gret_dtype io_dtype, float eps,
-                                gret_epilogue epi, void* workspace, size_t workspace_bytes, gret_stream_t stream) {
+                                const void* G, const float* S0, const int* cu_seqlens, int total, float tau,
+                                int chunk, void* O, float* S_final, int B, int H, int N, int dk, int dv,
+                                gret_dtype io_dtype, float eps, gret_epilogue epi, void* workspace,
+                                size_t workspace_bytes, gret_stream_t stream) {
     if (!Q || !K || !V || !gate_logits || !O) return GRET_ERR_INVALID_ARG;
     if (epi != GRET_EPI_GN_SWISH && epi != GRET_EPI_NONE) return GRET_ERR_INVALID_ARG;
     if (epi == GRET_EPI_GN_SWISH && !G) return GRET_ERR_INVALID_ARG;
@@ -137,6 +138,7 @@ static gret_status prefill_impl(const void* Q, const void* K, const void* V, con
         (G && !aligned16(G)) || (S_final && !aligned16(S_final)) || (S0 && !aligned16(S0)))
         return GRET_ERR_INVALID_ARG;
     if ((long long)B * H > (1LL << 30) || (long long)B * N > (1LL << 40)) return GRET_ERR_UNSUPPORTED;
+    if (cu_seqlens && ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0 || total <= 0)) return GRET_ERR_INVALID_ARG;
     if (S0 && S_final) {
         // segments of one unit run in different CTAs: S_final must not overwrite S0
         const size_t bytes = (size_t)B * H * dk * dv * sizeof(float);
@@ -153,6 +155,7 @@ static gret_status prefill_impl(const void* Q, const void* K, const void* V, con
 
     PrefillArgs a;
     a.Q = Q; a.K = K; a.V = V; a.z = gate_logits; a.G = G; a.O = O; a.S_final = S_final; a.S0 = S0;
+    a.cu_seqlens = cu_seqlens; a.total = total;
     a.B = B; a.H = H; a.N = N; a.dk = dk; a.dv = dv; a.chunk = chunk;
     a.inv_tau = 1.0f / tau; a.eps = eps; a.io = io_dtype; a.epi = epi;
     a.workspace = workspace; a.workspace_bytes = workspace_bytes;
@@ -177,8 +180,8 @@ gret_status gret_prefill(const void* Q, const void* K, const void* V, const floa
                          const void* G, float tau, int chunk, void* O, float* S_final, int B, int H,
                          int N, int dk, int dv, gret_dtype io_dtype, float eps, gret_epilogue epi,
                          void* workspace, size_t workspace_bytes, gret_stream_t stream) {
-    return prefill_impl(Q, K, V, gate_logits, G, nullptr, tau, chunk, O, S_final, B, H, N, dk, dv, io_dtype, eps,
-                        epi, workspace, workspace_bytes, stream);
+    return prefill_impl(Q, K, V, gate_logits, G, nullptr, nullptr, 0, tau, chunk, O, S_final, B, H, N, dk, dv,
+                        io_dtype, eps, epi, workspace, workspace_bytes, stream);
 }
 
 gret_status gret_prefill_from_state(const void* Q, const void* K, const void* V, const float* gate_logits,
@@ -186,8 +189,18 @@ gret_status gret_prefill_from_state(const void* Q, const void* K, const void* V,
                                     float* S_final, int B, int H, int N, int dk, int dv, gret_dtype io_dtype,
                                     float eps, gret_epilogue epi, void* workspace, size_t workspace_bytes,
                                     gret_stream_t stream) {
-    return prefill_impl(Q, K, V, gate_logits, G, S0, tau, chunk, O, S_final, B, H, N, dk, dv, io_dtype, eps, epi,
-                        workspace, workspace_bytes, stream);
+    return prefill_impl(Q, K, V, gate_logits, G, S0, nullptr, 0, tau, chunk, O, S_final, B, H, N, dk, dv, io_dtype,
+                        eps, epi, workspace, workspace_bytes, stream);
+}
+
+gret_status gret_prefill_varlen(const void* Q, const void* K, const void* V, const float* gate_logits,
+                                const void* G, const float* S0, const int* cu_seqlens, int num_seqs,
+                                int total_tokens, int max_seqlen, float tau, int chunk, void* O, float* S_final,
+                                int H, int dk, int dv, gret_dtype io_dtype, float eps, gret_epilogue epi,
+                                void* workspace, size_t workspace_bytes, gret_stream_t stream) {
+    if (!cu_seqlens) return GRET_ERR_INVALID_ARG;
+    return prefill_impl(Q, K, V, gate_logits, G, S0, cu_seqlens, total_tokens, tau, chunk, O, S_final, num_seqs, H,
+                        max_seqlen, dk, dv, io_dtype, eps, epi, workspace, workspace_bytes, stream);
 }
 
 gret_status gret_decode_step(const void* q, const void* k, const void* v, const float* gate_logit,

@@ -15,6 +15,17 @@ namespace gret {
 // Kernels never trap.
 enum : unsigned int { kDevOk = 0u, kDevTimeout = 1u, kDevSmemLayout = 2u };
 
+// Token rows row0 .. row0 + len - 1 of sequence b in a packed batch of `total`
+// rows, clamped into [0, total] so that malformed offsets can neither address
+// memory outside the tensors nor give a negative row.
+__device__ __forceinline__ void packed_range(const int* cu, int b, int total, int& row0, int& len) {
+    int a0 = cu[b], a1 = cu[b + 1];
+    a0 = a0 < 0 ? 0 : (a0 > total ? total : a0);
+    a1 = a1 < a0 ? a0 : (a1 > total ? total : a1);
+    row0 = a0;
+    len = a1 - a0;
+}
+
 struct PrefillArgs {
     const void* Q;
     const void* K;
@@ -24,6 +35,11 @@ struct PrefillArgs {
     void* O;
     float* S_final;
     const float* S0;          // initial state [B][H][dk][dv] fp32, or null for zero
+    // packed variable-length batch: B sequences, sequence b holds token rows
+    // cu_seqlens[b] .. cu_seqlens[b + 1] - 1 of [total][H][d] tensors (device
+    // array), N is the longest; null for the uniform [B][N][H][d] layout
+    const int* cu_seqlens;
+    int total;
     int B, H, N, dk, dv, chunk;
     float inv_tau, eps;
     gret_dtype io;

@@ -47,9 +47,13 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(PrefillArgs a) {
     T* Og = static_cast<T*>(a.O);
     const size_t rowk = (size_t)H * dk, rowv = (size_t)H * dv;
 
-    for (int c0 = 0; c0 < N; c0 += C) {
-        const int L = min(C, N - c0);
-        const size_t tok0 = (size_t)b * N + c0;
+    // this unit's tokens: rows base .. base + Nu - 1
+    int row0 = 0, Nu = N;
+    if (a.cu_seqlens) packed_range(a.cu_seqlens, b, a.total, row0, Nu);
+    const size_t base = a.cu_seqlens ? (size_t)row0 : (size_t)b * N;
+    for (int c0 = 0; c0 < Nu; c0 += C) {
+        const int L = min(C, Nu - c0);
+        const size_t tok0 = base + c0;
         for (int e = tid; e < L * dk; e += kThreads) {
             int t = e / dk, i = e % dk;
             Qs[e] = to_f32(Qg[(tok0 + t) * rowk + (size_t)h * dk + i]);

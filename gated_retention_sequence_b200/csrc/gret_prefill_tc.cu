@@ -136,6 +136,9 @@ struct TcParams {
     float* seg_decay;        // [units][(P-1)*K]
     float* S_final;          // [units][DK][DV] or null
     const float* S0;         // [units][DK][DV] initial state, or null for zero
+    const int* cu;           // packed batch: sequence b is token rows cu[b] .. cu[b+1]-1; or null
+    int total;               // rows of the packed tensors
+    void* O;                 // output base (tail rows of packed sequences are stored directly)
     unsigned int* status;
     int H, N, Npad, P, seg_len;
     int K, piece_len;        // state-pass pieces per segment and their length
@@ -242,7 +245,7 @@ __device__ __forceinline__ void warp_transpose_sum(float (&v)[N], int lane) {
 // Q~_t = e^{b_t + Lambda} Q_t against T, and the state leaves as e^Lambda T.
 // The MMA warp repeats the lazy/eager decision from the same decay sums with
 // the same float operations, so both sides agree on it.
-template <int DV, int C>
+template <int DV, int C, bool PACKED>
 __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __grid_constant__ TcParams p) {
     using CF = Cfg<DV, C>;
     constexpr int NQK = CF::NQK, NV = CF::NV, NG = CF::NG, NH = CF::NH, W = CF::W, HT = CF::HT;
@@ -259,10 +262,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
     }
 
     const int u = blockIdx.x / p.P, seg = blockIdx.x % p.P;
-    const int bb = u / p.H, hh = u % p.H;
+    const int hh = u % p.H;
     const int n_begin = seg * p.seg_len;
-    const int n_end = min(p.N, n_begin + p.seg_len);
-    const int nchunks = (n_end - n_begin + C - 1) / C;
 
     // Barriers.  The scores, the state MMA and the staged output have one
     // barrier per chunk parity, so that none of them can complete a phase
@@ -307,6 +308,18 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
     // kernel reads what the earlier ones wrote (decay sums, segment states)
     grid_dep_launch();
     grid_dep_wait();
+    // this unit's sequence: batch bb of the uniform layout, or token rows
+    // row0 .. row0 + Nu - 1 of a packed batch (PACKED)
+    int bb = u / p.H, row0 = 0, Nu = p.N;
+    if constexpr (PACKED) {
+        bb = 0;
+        packed_range(p.cu, u / p.H, p.total, row0, Nu);
+    }
+    const int n_end = min(Nu, n_begin + p.seg_len);
+    const int nchunks = n_end > n_begin ? (n_end - n_begin + C - 1) / C : 0;
+    // a packed sequence's last chunk stops at its end: its output rows are
+    // stored directly, since a full tile would overwrite the next sequence
+    auto direct_tail = [&](int j) { return PACKED && n_end - (n_begin + j * C) < C; };
     if (warp >= kCW) {
       // ================================================================ issuing warpgroup
       asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" : : "n"(kIssueRegs));
@@ -318,8 +331,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
                 const uint32_t fb = bar(BQK + s);
                 mbar_arrive_expect_tx(fb, CF::Q_BYTES + CF::K_BYTES + 2 * C * 4);
                 for (int x = 0; x < 2; ++x) {
-                    tma_load_4d(sb + CF::OFF_Q + s * CF::Q_BYTES + x * CF::BOX, &p.tmQ, x * 64, hh, n0, bb, fb);
-                    tma_load_4d(sb + CF::OFF_K + s * CF::K_BYTES + x * CF::BOX, &p.tmK, x * 64, hh, n0, bb, fb);
+                    tma_load_4d(sb + CF::OFF_Q + s * CF::Q_BYTES + x * CF::BOX, &p.tmQ, x * 64, hh, row0 + n0, bb, fb);
+                    tma_load_4d(sb + CF::OFF_K + s * CF::K_BYTES + x * CF::BOX, &p.tmK, x * 64, hh, row0 + n0, bb, fb);
                 }
                 bulk_load(sb + CF::OFF_B + s * 2 * C * 4, p.bcum + (size_t)u * p.Npad + n0, C * 4, fb);
                 bulk_load(sb + CF::OFF_B + (s * 2 + 1) * C * 4, p.eblk + (size_t)u * p.Npad + n0, C * 4, fb);
@@ -329,14 +342,14 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
                 const uint32_t fb = bar(BV + s);
                 mbar_arrive_expect_tx(fb, CF::V_BYTES);
                 for (int x = 0; x < DV / 64; ++x)
-                    tma_load_4d(sb + CF::OFF_V + s * CF::V_BYTES + x * CF::BOX, &p.tmV, x * 64, hh, n0, bb, fb);
+                    tma_load_4d(sb + CF::OFF_V + s * CF::V_BYTES + x * CF::BOX, &p.tmV, x * 64, hh, row0 + n0, bb, fb);
             };
             auto issue_g = [&](int j) {
                 const int s = j % NG, n0 = n_begin + j * C;
                 const uint32_t fb = bar(BG + s);
                 mbar_arrive_expect_tx(fb, CF::G_BYTES);
                 for (int x = 0; x < DV / 64; ++x)
-                    tma_load_4d(sb + CF::OFF_G + s * CF::G_BYTES + x * CF::BOX, &p.tmG, x * 64, hh, n0, bb, fb);
+                    tma_load_4d(sb + CF::OFF_G + s * CF::G_BYTES + x * CF::BOX, &p.tmG, x * 64, hh, row0 + n0, bb, fb);
             };
             // the output tile of chunk j, written over G(j) in shared memory, goes
             // out; once the store has read the stage it takes the G of chunk j + NG
@@ -344,9 +357,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
                 mbar_wait(bar(BSTAGED + (j & 1)), (j >> 1) & 1, p.status, abort_flag);
                 const uint32_t sG = sb + CF::OFF_G + (j % NG) * CF::G_BYTES;
                 const int n0 = n_begin + j * C;
-                for (int x = 0; x < DV / 64; ++x) tma_store_4d(&p.tmO, sG + x * CF::BOX, x * 64, hh, n0, bb);
-                bulk_commit();
-                bulk_wait_read<0>();
+                if (!direct_tail(j)) {
+                    for (int x = 0; x < DV / 64; ++x)
+                        tma_store_4d(&p.tmO, sG + x * CF::BOX, x * 64, hh, row0 + n0, bb);
+                    bulk_commit();
+                    bulk_wait_read<0>();
+                }
                 if (p.has_g && j + NG < nchunks) issue_g(j + NG);
             };
             issue_qk(0);
@@ -520,6 +536,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
             const float bC = bc[C - 1];
             const bool eager = (-bC - lam) > kLazyMax;
             const float escale = __expf(lam + bC);
+            const int valid = n_end - (n_begin + i * C);   // rows of this unit in the chunk (PACKED)
 
             // phase A: Q~ = e^{b_t + Lambda} Q for the inter-chunk read, which the
             // issuer starts as soon as every warp has done its share
@@ -642,7 +659,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
                 for (int it = it0; it < it1; it += step) {
                     const int row = (it >> 3) % C;
                     const float ex = eager ? (bC - bc[row]) : (-bc[row] - lam);
-                    scale_bf16x8(Kp + it * 16, __expf(ex));
+                    // rows past a packed unit's end (the next sequence's) add nothing;
+                    // in the uniform layout they load as zeros
+                    scale_bf16x8(Kp + it * 16, (!PACKED || row < valid) ? __expf(ex) : 0.f);
                 }
             }
             fence_proxy_async_smem();
@@ -730,13 +749,13 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
                 }
                 named_bar_sync(1, kCT);
             }
+            auto d_of = [&](int h) { return h * 128 + q4 * 32 + lane; };
             int goff[NH];
 #pragma unroll
-            for (int h = 0; h < NH; ++h) {
-                const int d = h * 128 + q4 * 32 + lane;
-                goff[h] = (d >> 6) * CF::BOX + (d & 7) * 2;
-            }
+            for (int h = 0; h < NH; ++h) goff[h] = (d_of(h) >> 6) * CF::BOX + (d_of(h) & 7) * 2;
             const int dc = ((q4 * 32 + lane) & 63) >> 3;   // the same for both halves
+            // the last chunk of a packed sequence: its rows go straight to global memory
+            const bool tail = direct_tail(i);
 #pragma unroll
             for (int j = 0; j < HT; ++j) {
                 const int t = t0 + j;
@@ -749,7 +768,13 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
                     float o = y[h][j];
                     // GroupNorm as one FMA, then times swish(g) = g * sigmoid(g)
                     if (p.gn) o = fmaf(o, st.x, st.y) * swish_fast(__bfloat162float(*gp));
-                    *gp = __float2bfloat16_rn(o);
+                    if (!PACKED || !tail) {
+                        *gp = __float2bfloat16_rn(o);
+                    } else if (t < n_end - (n_begin + i * C)) {
+                        __nv_bfloat16* Ot = static_cast<__nv_bfloat16*>(p.O) +
+                                            ((size_t)(row0 + n_begin + i * C + t) * p.H + hh) * DV + d_of(h);
+                        *Ot = __float2bfloat16_rn(o);
+                    }
                 }
             }
             fence_proxy_async_smem();
@@ -834,7 +859,7 @@ struct StateCfg {
     static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
 
-template <int DV, int C>
+template <int DV, int C, bool PACKED>
 __global__ void __launch_bounds__(kStateThreads, 1) prefill_state_kernel(const __grid_constant__ TcParams p) {
     using CF = StateCfg<DV, C>;
     constexpr int NS = CF::NS, NH = CF::NH, W = CF::W;
@@ -847,10 +872,8 @@ __global__ void __launch_bounds__(kStateThreads, 1) prefill_state_kernel(const _
 
     const int nseg = (p.P - 1) * p.K;           // pieces of all segments but the last
     const int u = blockIdx.x / nseg, seg = blockIdx.x % nseg;
-    const int bb = u / p.H, hh = u % p.H;
+    const int hh = u % p.H;
     const int n_begin = seg * p.piece_len;
-    const int n_end = min(p.N, n_begin + p.piece_len);
-    const int nchunks = (n_end - n_begin + C - 1) / C;
 
     auto full = [&](int s) -> uint32_t { return sb + CF::OFF_BAR + 8 * s; };
     auto empty = [&](int s) -> uint32_t { return sb + CF::OFF_BAR + 8 * (NS + s); };
@@ -873,19 +896,27 @@ __global__ void __launch_bounds__(kStateThreads, 1) prefill_state_kernel(const _
     tc_fence_after();
     const uint32_t tm = *tmem_slot;
 
-    auto issue = [&](int j) {
-        const int s = j % NS, n0 = n_begin + j * C;
-        mbar_arrive_expect_tx(full(s), CF::K_BYTES + CF::V_BYTES + C * 4);
-        for (int x = 0; x < 2; ++x)
-            tma_load_4d(sb + CF::OFF_K + s * CF::K_BYTES + x * CF::BOX, &p.tmK, x * 64, hh, n0, bb, full(s));
-        for (int x = 0; x < DV / 64; ++x)
-            tma_load_4d(sb + CF::OFF_V + s * CF::V_BYTES + x * CF::BOX, &p.tmV, x * 64, hh, n0, bb, full(s));
-        bulk_load(sb + CF::OFF_B + s * C * 4, p.bcum + (size_t)u * p.Npad + n0, C * 4, full(s));
-    };
     // everything above overlaps the previous kernel's tail; the loads need its
     // decay sums
     grid_dep_launch();
     grid_dep_wait();
+    // this unit's sequence (see the fused kernel)
+    int bb = u / p.H, row0 = 0, Nu = p.N;
+    if constexpr (PACKED) {
+        bb = 0;
+        packed_range(p.cu, u / p.H, p.total, row0, Nu);
+    }
+    const int n_end = min(Nu, n_begin + p.piece_len);
+    const int nchunks = n_end > n_begin ? (n_end - n_begin + C - 1) / C : 0;
+    auto issue = [&](int j) {
+        const int s = j % NS, n0 = n_begin + j * C;
+        mbar_arrive_expect_tx(full(s), CF::K_BYTES + CF::V_BYTES + C * 4);
+        for (int x = 0; x < 2; ++x)
+            tma_load_4d(sb + CF::OFF_K + s * CF::K_BYTES + x * CF::BOX, &p.tmK, x * 64, hh, row0 + n0, bb, full(s));
+        for (int x = 0; x < DV / 64; ++x)
+            tma_load_4d(sb + CF::OFF_V + s * CF::V_BYTES + x * CF::BOX, &p.tmV, x * 64, hh, row0 + n0, bb, full(s));
+        bulk_load(sb + CF::OFF_B + s * C * 4, p.bcum + (size_t)u * p.Npad + n0, C * 4, full(s));
+    };
     if (tid == 0)
         for (int j = 0; j < NS && j < nchunks; ++j) issue(j);
 
@@ -917,9 +948,12 @@ __global__ void __launch_bounds__(kStateThreads, 1) prefill_state_kernel(const _
                 w[k] = *reinterpret_cast<const uint4*>(Kp + ci * 16);
                 e[k] = bc[(ci >> 3) % C];
             }
+            const int valid = n_end - (n_begin + i * C);   // rows of this unit in the chunk
 #pragma unroll
             for (int k = 0; k < NIT; ++k) {
-                const float sc = __expf(eager ? (bC - e[k]) : (-e[k] - lam));
+                // rows past the unit's end (the next packed sequence's) add nothing
+                const float sc = (!PACKED || ((tid + k * kStateThreads) >> 3) % C < valid)
+                                     ? __expf(eager ? (bC - e[k]) : (-e[k] - lam)) : 0.f;
                 uint32_t* x = reinterpret_cast<uint32_t*>(&w[k]);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
@@ -1004,8 +1038,9 @@ __global__ void __launch_bounds__(kStateThreads, 1) prefill_state_kernel(const _
 // Chunk-local inclusive sums of log gamma: bcum[u][n] = sum_{j in chunk, j <= n} lg_j,
 // and the P step's block factors eblk (below).
 // Padding tokens (n >= N) carry lg = 0, so they repeat the chunk total.
-__global__ void gate_scan_kernel(const float* __restrict__ z, float* __restrict__ bcum, float* __restrict__ eblk,
-                                 int H, int N, int Npad, float inv_tau) {
+__global__ void gate_scan_kernel(const float* __restrict__ z, const int* __restrict__ cu_seqlens, int total,
+                                 float* __restrict__ bcum, float* __restrict__ eblk, int H, int N, int Npad,
+                                 float inv_tau) {
     __shared__ float wsum[4];
     // the gate logits may come from the kernel before this one, and the kernels
     // before that may still read the workspace: wait for them first
@@ -1015,7 +1050,12 @@ __global__ void gate_scan_kernel(const float* __restrict__ z, float* __restrict_
     const int u = blockIdx.x, b = u / H, h = u % H;
     const int t = threadIdx.x, lane = t & 31, w = t >> 5;
     const int n = blockIdx.y * C + t;
-    float x = n < N ? log_gamma(z[((size_t)b * N + n) * H + h], inv_tau) : 0.f;
+    // this unit's tokens are rows base .. base + Nu - 1; past its end the
+    // decay stays flat (log gamma = 0), so a chunk's last sum is its decay
+    int row0 = 0, Nu = N;
+    if (cu_seqlens) packed_range(cu_seqlens, b, total, row0, Nu);
+    const size_t base = cu_seqlens ? (size_t)row0 : (size_t)b * N;
+    float x = n < Nu ? log_gamma(z[(base + n) * H + h], inv_tau) : 0.f;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         float y = __shfl_up_sync(0xffffffffu, x, o);
@@ -1131,11 +1171,11 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
-template <int DV, int C>
+template <int DV, int C, bool PACKED>
 cudaError_t run_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t s) {
     using CF = Cfg<DV, C>;
-    auto kf = prefill_tc_kernel<DV, C>;
-    auto ks = prefill_state_kernel<DV, C>;
+    auto kf = prefill_tc_kernel<DV, C, PACKED>;
+    auto ks = prefill_state_kernel<DV, C, PACKED>;
     static bool attr_done[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -1151,7 +1191,7 @@ cudaError_t run_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t s) {
     }
     const int units = a.B * a.H;
     const int npad = tp.Npad;
-    cudaError_t e = launch_pdl(gate_scan_kernel, dim3(units, npad / C), dim3(C), 0, s, a.z,
+    cudaError_t e = launch_pdl(gate_scan_kernel, dim3(units, npad / C), dim3(C), 0, s, a.z, a.cu_seqlens, a.total,
                                const_cast<float*>(tp.bcum), const_cast<float*>(tp.eblk), a.H, a.N, npad, a.inv_tau);
     if (e != cudaSuccess) return e;
     if (tp.P > 1) {
@@ -1212,10 +1252,16 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
     TcParams tp;
     memset(&tp, 0, sizeof(tp));
     const int C = a.chunk;
-    if (!make_map(&tp.tmQ, a.Q, DK, a.H, a.N, a.B, C) || !make_map(&tp.tmK, a.K, DK, a.H, a.N, a.B, C) ||
-        !make_map(&tp.tmV, a.V, a.dv, a.H, a.N, a.B, C) || !make_map(&tp.tmO, a.O, a.dv, a.H, a.N, a.B, C) ||
-        !make_map(&tp.tmG, a.G ? a.G : a.O, a.dv, a.H, a.N, a.B, C))
+    // a packed batch is one [total][H][d] tensor: (d, H, total, 1) maps, each
+    // unit addressing its own rows
+    const int mN = a.cu_seqlens ? a.total : a.N, mB = a.cu_seqlens ? 1 : a.B;
+    if (!make_map(&tp.tmQ, a.Q, DK, a.H, mN, mB, C) || !make_map(&tp.tmK, a.K, DK, a.H, mN, mB, C) ||
+        !make_map(&tp.tmV, a.V, a.dv, a.H, mN, mB, C) || !make_map(&tp.tmO, a.O, a.dv, a.H, mN, mB, C) ||
+        !make_map(&tp.tmG, a.G ? a.G : a.O, a.dv, a.H, mN, mB, C))
         return cudaErrorInvalidValue;
+    tp.cu = a.cu_seqlens;
+    tp.total = a.total;
+    tp.O = a.O;
     const WsLayout w = ws_layout(a.B, a.H, a.N, a.dk, a.dv, C, a.segments, a.pieces);
     uint8_t* ws = static_cast<uint8_t*>(a.workspace);
     tp.bcum = reinterpret_cast<const float*>(ws + w.bcum);
@@ -1235,9 +1281,10 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
     tp.eps = a.eps;
     tp.gn = a.epi == GRET_EPI_GN_SWISH ? 1 : 0;
     tp.has_g = (a.epi == GRET_EPI_GN_SWISH && a.G) ? 1 : 0;
-    if (a.dv == 256 && C == 64) return run_tc<256, 64>(a, tp, s);
-    if (a.dv == 128 && C == 128) return run_tc<128, 128>(a, tp, s);
-    if (a.dv == 128 && C == 64) return run_tc<128, 64>(a, tp, s);
+    const bool packed = a.cu_seqlens != nullptr;
+    if (a.dv == 256 && C == 64) return packed ? run_tc<256, 64, true>(a, tp, s) : run_tc<256, 64, false>(a, tp, s);
+    if (a.dv == 128 && C == 128) return packed ? run_tc<128, 128, true>(a, tp, s) : run_tc<128, 128, false>(a, tp, s);
+    if (a.dv == 128 && C == 64) return packed ? run_tc<128, 64, true>(a, tp, s) : run_tc<128, 64, false>(a, tp, s);
     return cudaErrorNotSupported;
 }
 

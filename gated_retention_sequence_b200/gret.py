@@ -61,6 +61,8 @@ SIGNATURES = {
                                   _I, _VP]),
     "gret_prefill_from_state": (_I, [_VP, _VP, _VP, _FP, _VP, _FP, _F, _I, _VP, _FP, _I, _I, _I, _I, _I, _I,
                                      _F, _I, _VP, _SZ, _VP]),
+    "gret_prefill_varlen": (_I, [_VP, _VP, _VP, _FP, _VP, _FP, _VP, _I, _I, _I, _F, _I, _VP, _FP, _I, _I, _I, _I,
+                                 _F, _I, _VP, _SZ, _VP]),
     "gret_prefill_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
     "gret_prefill_launches": (_I, [_I, _I, _I, _I, _I, _I, _I]),
     "gret_prefill_path": (_I, [_I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_int)]),
@@ -99,6 +101,13 @@ def gret_prefill_from_state(Q, K, V, gate_logits, G, S0, tau, chunk, O, S_final,
                             eps, epi, workspace, workspace_bytes, stream) -> int:
     return load().gret_prefill_from_state(Q, K, V, gate_logits, G, S0, tau, chunk, O, S_final, B, H, N, dk, dv,
                                           int(io_dtype), eps, int(epi), workspace, workspace_bytes, stream)
+
+
+def gret_prefill_varlen(Q, K, V, gate_logits, G, S0, cu_seqlens, num_seqs, total_tokens, max_seqlen, tau, chunk,
+                        O, S_final, H, dk, dv, io_dtype, eps, epi, workspace, workspace_bytes, stream) -> int:
+    return load().gret_prefill_varlen(Q, K, V, gate_logits, G, S0, cu_seqlens, num_seqs, total_tokens, max_seqlen,
+                                      tau, chunk, O, S_final, H, dk, dv, int(io_dtype), eps, int(epi), workspace,
+                                      workspace_bytes, stream)
 
 
 def gret_prefill_noalloc(Q, K, V, gate_logits, G, tau, chunk, O, S_final, B, H, N, dk, dv, io_dtype, eps,
@@ -221,6 +230,52 @@ def prefill(Q, K, V, z, G, tau: float, chunk: int, eps: float = 1e-5, epilogue: 
                                              float(eps), epi, ws, ws_bytes, st.cuda_stream)
     if status != Status.OK:
         raise GretError(status, "gret_prefill" if S0 is None else "gret_prefill_from_state")
+    return O, S_final
+
+
+def prefill_varlen(Q, K, V, z, G, cu_seqlens, max_seqlen: int, tau: float, chunk: int, eps: float = 1e-5,
+                   epilogue: str = "gn_swish", O=None, S_final=None, want_state: bool = True, workspace=None,
+                   stream=None, S0=None):
+    """Prefill of a packed batch of sequences (gret_prefill_varlen).
+
+    Q, K [T,H,dk]; V, G [T,H,dv] (bf16 or fp32); z [T,H] fp32; cu_seqlens int32 [S+1] on the
+    device (sequence b is rows cu_seqlens[b] .. cu_seqlens[b+1]-1); S0 [S,H,dk,dv] fp32 or None.
+    Returns (O [T,H,dv], S_final [S,H,dk,dv] fp32 or None).
+    """
+    torch = _torch()
+    T, H, dk = Q.shape
+    dv = V.shape[-1]
+    S = cu_seqlens.numel() - 1
+    dev = Q.device
+    io = _io_of(Q)
+    epi = Epilogue.NONE if epilogue == "none" else Epilogue.GN_SWISH
+    _check(Q, "Q", Q.dtype, (T, H, dk), dev)
+    _check(K, "K", Q.dtype, (T, H, dk), dev)
+    _check(V, "V", Q.dtype, (T, H, dv), dev)
+    _check(z, "z", torch.float32, (T, H), dev)
+    _check(cu_seqlens, "cu_seqlens", torch.int32, (S + 1,), dev)
+    if epi == Epilogue.GN_SWISH or G is not None:
+        _check(G, "G", Q.dtype, (T, H, dv), dev)
+    if O is None:
+        O = torch.empty((T, H, dv), dtype=Q.dtype, device=dev)
+    _check(O, "O", Q.dtype, (T, H, dv), dev)
+    if S_final is None and want_state:
+        S_final = torch.empty((S, H, dk, dv), dtype=torch.float32, device=dev)
+    if S_final is not None:
+        _check(S_final, "S_final", torch.float32, (S, H, dk, dv), dev)
+    if S0 is not None:
+        _check(S0, "S0", torch.float32, (S, H, dk, dv), dev)
+    with torch.cuda.device(dev):
+        ws_bytes = gret_prefill_workspace_size(S, H, max_seqlen, dk, dv, chunk, io)
+        if ws_bytes and (workspace is None or workspace.numel() * workspace.element_size() < ws_bytes):
+            workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        st = stream if stream is not None else torch.cuda.current_stream(dev)
+        status = gret_prefill_varlen(_ptr(Q), _ptr(K), _ptr(V), _ptr(z), _ptr(G), _ptr(S0), _ptr(cu_seqlens), S, T,
+                                     int(max_seqlen), float(tau), int(chunk), _ptr(O), _ptr(S_final), H, dk, dv, io,
+                                     float(eps), epi, _ptr(workspace) if ws_bytes else None, ws_bytes,
+                                     st.cuda_stream)
+    if status != Status.OK:
+        raise GretError(status, "gret_prefill_varlen")
     return O, S_final
 
 

@@ -111,6 +111,34 @@ gret_status gret_prefill_from_state(const void* Q, const void* K, const void* V,
                                     gret_dtype io_dtype, float eps, gret_epilogue epi, void* workspace,
                                     size_t workspace_bytes, gret_stream_t stream);
 
+/*
+ * gret_prefill_varlen -- prefill of a packed batch of sequences of different
+ * lengths (the layout a serving batch of prompts has), each from its own
+ * initial state or zero.
+ *
+ *   Q, K        [total_tokens][H][dk]   io dtype
+ *   V, G, O     [total_tokens][H][dv]   io dtype
+ *   gate_logits [total_tokens][H]       fp32
+ *   cu_seqlens  int32 [num_seqs + 1] (DEVICE): sequence b is token rows
+ *               cu_seqlens[b] .. cu_seqlens[b + 1] - 1, so cu_seqlens[0] = 0,
+ *               non-decreasing, cu_seqlens[num_seqs] = total_tokens; a sequence
+ *               may be empty (its S_final is then S0, or zero).
+ *   max_seqlen  the longest sequence (>= every length; sizes the work split).
+ *   S0, S_final fp32 [num_seqs][H][dk][dv]; S0 may be NULL (zero state); the
+ *               rule of gret_prefill_from_state on overlap applies.
+ * Workspace: gret_prefill_workspace_size(num_seqs, H, max_seqlen, dk, dv,
+ * chunk, io_dtype) bytes.  Every sequence gives what gret_prefill_from_state
+ * gives for it alone; nothing is written outside its rows.  Offsets outside
+ * [0, total_tokens] are clamped into it; tokens past max_seqlen in a sequence
+ * are not processed.  cu_seqlens must be 4-byte aligned; total_tokens > 0.
+ */
+gret_status gret_prefill_varlen(const void* Q, const void* K, const void* V, const float* gate_logits,
+                                const void* G, const float* S0, const int* cu_seqlens, int num_seqs,
+                                int total_tokens, int max_seqlen, float tau, int chunk, void* O,
+                                float* S_final, int H, int dk, int dv, gret_dtype io_dtype, float eps,
+                                gret_epilogue epi, void* workspace, size_t workspace_bytes,
+                                gret_stream_t stream);
+
 /* Size of the device scratch array gret_prefill_noalloc draws on (32 MiB). */
 #define GRET_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
 

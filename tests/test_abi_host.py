@@ -81,6 +81,17 @@ def test_prefill_from_state_rejects_overlapping_states(lib):
         gret.Status.ERR_INVALID_ARG                                   # misaligned S0
 
 
+def test_prefill_varlen_rejects_bad_arguments(lib):
+    good = 0x10000
+    a = dict(Q=good, K=good, V=good, gate_logits=good, G=good, S0=None, cu_seqlens=good, num_seqs=2,
+             total_tokens=100, max_seqlen=60, tau=16.0, chunk=64, O=good, S_final=None, H=2, dk=64, dv=64,
+             io_dtype=gret.Dtype.F32, eps=1e-5, epi=gret.Epilogue.GN_SWISH, workspace=None, workspace_bytes=0,
+             stream=None)
+    for over in (dict(cu_seqlens=None), dict(cu_seqlens=good + 2), dict(total_tokens=0), dict(num_seqs=0),
+                 dict(max_seqlen=0), dict(Q=None)):
+        assert gret.gret_prefill_varlen(**dict(a, **over)) == gret.Status.ERR_INVALID_ARG, over
+
+
 def test_decode_rejects_bad_arguments(lib):
     good = 0x10000
     base = dict(q=good, k=good, v=good, gate_logit=good, g=good, S_inout=good, o=good, num_seqs=4,
