@@ -4,6 +4,7 @@
 // step of the mixer runs in the kernels.  Validation happens before any launch
 // so that a bad call has no effect on the stream.
 #include <math.h>
+#include <string.h>
 #include <stdint.h>
 
 #include <mutex>
@@ -153,7 +154,7 @@ static gret_status prefill_impl(const void* Q, const void* K, const void* V, con
     gret_path path = select_path(B, H, N, dk, dv, chunk, io_dtype, sms, &segs, &seg_len, &pcs);
     if (path == GRET_PATH_NONE) return GRET_ERR_UNSUPPORTED;
 
-    PrefillArgs a;
+    PrefillArgs a = {};
     a.Q = Q; a.K = K; a.V = V; a.z = gate_logits; a.G = G; a.O = O; a.S_final = S_final; a.S0 = S0;
     a.cu_seqlens = cu_seqlens; a.total = total;
     a.B = B; a.H = H; a.N = N; a.dk = dk; a.dv = dv; a.chunk = chunk;
@@ -219,7 +220,7 @@ gret_status gret_decode_step(const void* q, const void* k, const void* v, const 
     if (!shape_supported(dk, dv)) return GRET_ERR_UNSUPPORTED;
     if ((long long)num_seqs * H > (1LL << 31) - 1) return GRET_ERR_UNSUPPORTED;
 
-    DecodeArgs a;
+    DecodeArgs a = {};
     a.q = q; a.k = k; a.v = v; a.z = gate_logit; a.g = g; a.S = S_inout; a.o = o;
     a.num_units = num_seqs * H; a.H = H; a.dk = dk; a.dv = dv;
     a.inv_tau = 1.0f / tau; a.eps = eps; a.io = io_dtype; a.epi = epi;
@@ -239,6 +240,60 @@ gret_status gret_last_device_status(gret_stream_t stream) {
         return word == kDevTimeout ? GRET_ERR_TIMEOUT : GRET_ERR_CUDA;
     }
     return GRET_OK;
+}
+
+size_t gret_prefill_state_workspace_size(int B, int H, int N, int dk, int dv, int chunk, gret_dtype io_dtype) {
+    int sms = 148;
+    device_info(nullptr, &sms);
+    if (select_path(B, H, N, dk, dv, chunk, io_dtype, sms, nullptr, nullptr) != GRET_PATH_TC) return 0;
+    return prefill_tc_state_workspace_bytes(B, H, N, dk, dv, chunk, sms);
+}
+
+gret_status gret_prefill_state(const void* K, const void* V, const float* gate_logits, float tau, int chunk,
+                               float* dS, float* decay, int B, int H, int N, int dk, int dv, gret_dtype io_dtype,
+                               void* workspace, size_t workspace_bytes, gret_stream_t stream) {
+    if (!K || !V || !gate_logits || !dS || !decay) return GRET_ERR_INVALID_ARG;
+    if (io_dtype != GRET_F32 && io_dtype != GRET_BF16) return GRET_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || N <= 0 || dk <= 0 || dv <= 0 || chunk <= 0) return GRET_ERR_INVALID_ARG;
+    if (!(tau > 0.0f) || !isfinite(tau)) return GRET_ERR_INVALID_ARG;
+    if (!aligned16(K) || !aligned16(V) || !aligned16(gate_logits) || !aligned16(dS) ||
+        (reinterpret_cast<uintptr_t>(decay) & 3u) != 0)
+        return GRET_ERR_INVALID_ARG;
+    if ((long long)B * H > (1LL << 30) || (long long)B * N > (1LL << 40)) return GRET_ERR_UNSUPPORTED;
+    unsigned int* status = nullptr;
+    int sms = 0;
+    if (!device_info(&status, &sms)) return GRET_ERR_CUDA;
+    gret_path path = select_path(B, H, N, dk, dv, chunk, io_dtype, sms, nullptr, nullptr);
+    if (path == GRET_PATH_NONE) return GRET_ERR_UNSUPPORTED;
+    PrefillArgs a = {};
+    memset(&a, 0, sizeof(a));
+    a.Q = K; a.K = K; a.V = V; a.z = gate_logits; a.S_final = dS; a.decay_out = decay; a.state_only = 1;
+    a.B = B; a.H = H; a.N = N; a.dk = dk; a.dv = dv; a.chunk = chunk;
+    a.inv_tau = 1.0f / tau; a.eps = 0.f; a.io = io_dtype; a.epi = GRET_EPI_NONE;
+    a.workspace = workspace; a.workspace_bytes = workspace_bytes; a.status = status;
+    a.segments = 1; a.seg_len = N; a.pieces = 1;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t err;
+    if (path == GRET_PATH_TC) {
+        const size_t need = prefill_tc_state_workspace_bytes(B, H, N, dk, dv, chunk, sms);
+        if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+            return GRET_ERR_INVALID_ARG;
+        err = launch_prefill_state_tc(a, sms, s);
+    } else {
+        err = launch_prefill_simt(a, s);
+    }
+    return err == cudaSuccess ? GRET_OK : GRET_ERR_CUDA;
+}
+
+gret_status gret_state_fold(const float* dS_all, const float* decay_all, int num_slices, int slice,
+                            const float* S0, float* S_in, int B, int H, int dk, int dv, gret_stream_t stream) {
+    if (!S_in || (slice > 0 && (!dS_all || !decay_all))) return GRET_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || dk <= 0 || dv <= 0 || num_slices <= 0 || slice < 0 || slice > num_slices)
+        return GRET_ERR_INVALID_ARG;
+    if ((long long)B * H * dk * dv > (1LL << 40)) return GRET_ERR_UNSUPPORTED;
+    const cudaError_t err = launch_state_fold(dS_all, decay_all, num_slices, slice, S0, S_in, B * H, dk * dv,
+                                              reinterpret_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? GRET_OK : GRET_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -40,6 +40,10 @@ struct PrefillArgs {
     // array), N is the longest; null for the uniform [B][N][H][d] layout
     const int* cu_seqlens;
     int total;
+    // state-only pass (sequence-parallel prefill): no outputs; the state
+    // increment goes to S_final and the slice's total log-decay to decay_out
+    int state_only;
+    float* decay_out;
     int B, H, N, dk, dv, chunk;
     float inv_tau, eps;
     gret_dtype io;
@@ -106,6 +110,12 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_prefill_simt(const PrefillArgs& a, cudaStream_t s);
 size_t prefill_simt_smem_bytes(int dk, int dv, int chunk);
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s);
+// state-only pass of the tensor-core path (a.state_only): workspace bytes and launch
+size_t prefill_tc_state_workspace_bytes(int B, int H, int N, int dk, int dv, int chunk, int num_sms);
+cudaError_t launch_prefill_state_tc(const PrefillArgs& a, int num_sms, cudaStream_t s);
+// S_in = fold over slices q < slice of (decay_q, dS_q), from S0 or zero
+cudaError_t launch_state_fold(const float* dS_all, const float* decay_all, int num_slices, int slice,
+                              const float* S0, float* S_in, int units, int elems, cudaStream_t s);
 bool prefill_tc_supported(int dk, int dv, int chunk, gret_dtype io);
 void prefill_tc_plan(int B, int H, int N, int chunk, int num_sms, int* segments, int* seg_len, int* pieces);
 size_t prefill_tc_workspace_bytes(int B, int H, int N, int dk, int dv, int chunk, int segments, int pieces);

@@ -51,12 +51,13 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(PrefillArgs a) {
     int row0 = 0, Nu = N;
     if (a.cu_seqlens) packed_range(a.cu_seqlens, b, a.total, row0, Nu);
     const size_t base = a.cu_seqlens ? (size_t)row0 : (size_t)b * N;
+    float decay = 0.f;      // the unit's total log-decay (state-only pass)
     for (int c0 = 0; c0 < Nu; c0 += C) {
         const int L = min(C, Nu - c0);
         const size_t tok0 = base + c0;
         for (int e = tid; e < L * dk; e += kThreads) {
             int t = e / dk, i = e % dk;
-            Qs[e] = to_f32(Qg[(tok0 + t) * rowk + (size_t)h * dk + i]);
+            if (!a.state_only) Qs[e] = to_f32(Qg[(tok0 + t) * rowk + (size_t)h * dk + i]);
             Ks[e] = to_f32(Kg[(tok0 + t) * rowk + (size_t)h * dk + i]);
         }
         for (int e = tid; e < L * dv; e += kThreads) {
@@ -81,7 +82,21 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(PrefillArgs a) {
         }
         __syncthreads();
         const float bL = bc[L - 1];
+        decay += bL;
         for (int s = tid; s < L; s += kThreads) wl[s] = expf(bL - bc[s]);
+        if (a.state_only) {
+            // state increment only: S <- e^{b_L} S + sum_s e^{b_L - b_s} K_s^T V_s
+            __syncthreads();
+            const float eL = expf(bL);
+            for (int e = tid; e < dk * dv; e += kThreads) {
+                int i = e / dv, j = e % dv;
+                float acc = 0.f;
+                for (int s = 0; s < L; ++s) acc = fmaf(wl[s] * Ks[s * dk + i], Vs[s * dv + j], acc);
+                S[e] = fmaf(eL, S[e], acc);
+            }
+            __syncthreads();
+            continue;
+        }
         // intra-chunk scores with the decay mask
         for (int e = tid; e < L * L; e += kThreads) {
             int t = e / L, s = e % L;
@@ -139,6 +154,7 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(PrefillArgs a) {
         float* Sf = a.S_final + (size_t)u * dk * dv;
         for (int e = tid; e < dk * dv; e += kThreads) Sf[e] = S[e];
     }
+    if (a.state_only && a.decay_out && tid == 0) a.decay_out[u] = decay;
 }
 
 }  // namespace

@@ -1102,6 +1102,42 @@ __global__ void seg_combine_kernel(float* __restrict__ seg_state, const float* _
     }
 }
 
+// State-only pass: the folded pieces (slot K-1, S^T layout [DV][DK]) become the
+// slice's increment dS [DK][DV] through a shared-memory tile transpose, and the
+// pieces' log-decays sum to the slice's total.
+template <int DV>
+__global__ void state_finish_kernel(const float* __restrict__ seg_state, const float* __restrict__ seg_decay,
+                                    int K, float* __restrict__ dS, float* __restrict__ decay) {
+    __shared__ float tile[32][33];
+    const int u = blockIdx.z;
+    const int d0 = blockIdx.x * 32, k0 = blockIdx.y * 32;     // tile of d_v rows, d_k columns of S^T
+    const float* src = seg_state + ((size_t)u * K + K - 1) * DV * DK;
+    for (int r = threadIdx.y; r < 32; r += blockDim.y) tile[r][threadIdx.x] = src[(size_t)(d0 + r) * DK + k0 + threadIdx.x];
+    __syncthreads();
+    float* dst = dS + (size_t)u * DK * DV;
+    for (int r = threadIdx.y; r < 32; r += blockDim.y) dst[(size_t)(k0 + r) * DV + d0 + threadIdx.x] = tile[threadIdx.x][r];
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0 && threadIdx.y == 0) {
+        float a = 0.f;
+        for (int k = 0; k < K; ++k) a += seg_decay[(size_t)u * K + k];
+        decay[u] = a;
+    }
+}
+
+// Sequence-parallel fold: S_in = e^{a_{p-1}} (... (e^{a_0} S0 + dS_0) ...) + dS_{p-1}
+// over the slices before `slice`, elementwise.
+__global__ void state_fold_kernel(const float* __restrict__ dS_all, const float* __restrict__ decay_all,
+                                  int slice, const float* __restrict__ S0, float* __restrict__ S_in, int units,
+                                  int elems) {
+    const int u = blockIdx.y;
+    const int e = blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= elems) return;
+    const size_t at = (size_t)u * elems + e;
+    float run = S0 ? S0[at] : 0.f;
+    for (int q = 0; q < slice; ++q)
+        run = fmaf(__expf(decay_all[(size_t)q * units + u]), run, dS_all[(size_t)q * units * elems + at]);
+    S_in[at] = run;
+}
+
 // ---------------------------------------------------------------- host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -1244,6 +1280,21 @@ int prefill_tc_launches(int segments, int pieces) {
     return segments <= 1 ? 2 : 4;
 }
 
+// State-only pass: the whole slice is one segment, cut into K pieces (about
+// one CTA per SM; K divides the chunk count).
+static int state_pass_pieces(int B, int H, int N, int chunk, int num_sms) {
+    const int units = B * H > 0 ? B * H : 1;
+    const int nchunks = (N + chunk - 1) / chunk;
+    const int kmax = num_sms / units > 1 ? num_sms / units : 1;
+    for (int k = kmax < nchunks ? kmax : nchunks; k >= 1; --k)
+        if (nchunks % k == 0) return k;
+    return 1;
+}
+
+size_t prefill_tc_state_workspace_bytes(int B, int H, int N, int dk, int dv, int chunk, int num_sms) {
+    return ws_layout(B, H, N, dk, dv, chunk, 2, state_pass_pieces(B, H, N, chunk, num_sms)).total;
+}
+
 size_t prefill_tc_workspace_bytes(int B, int H, int N, int dk, int dv, int chunk, int segments, int pieces) {
     return ws_layout(B, H, N, dk, dv, chunk, segments, pieces).total;
 }
@@ -1286,6 +1337,62 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
     if (a.dv == 128 && C == 128) return packed ? run_tc<128, 128, true>(a, tp, s) : run_tc<128, 128, false>(a, tp, s);
     if (a.dv == 128 && C == 64) return packed ? run_tc<128, 64, true>(a, tp, s) : run_tc<128, 64, false>(a, tp, s);
     return cudaErrorNotSupported;
+}
+
+template <int DV, int C>
+static cudaError_t run_state_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t s) {
+    auto ks = prefill_state_kernel<DV, C, false>;
+    cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, StateCfg<DV, C>::SMEM);
+    const int units = a.B * a.H;
+    cudaError_t e = launch_pdl(gate_scan_kernel, dim3(units, tp.Npad / C), dim3(C), 0, s, a.z,
+                               static_cast<const int*>(nullptr), 0, const_cast<float*>(tp.bcum),
+                               const_cast<float*>(tp.eblk), a.H, a.N, tp.Npad, a.inv_tau);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(ks, dim3(units * tp.K), dim3(kStateThreads), StateCfg<DV, C>::SMEM, s, tp);
+    if (e != cudaSuccess) return e;
+    const int elems4 = DV * DK / 4;
+    e = launch_pdl(seg_combine_kernel, dim3((elems4 + 255) / 256, units), dim3(256), 0, s, tp.seg_state,
+                   static_cast<const float*>(tp.seg_decay), static_cast<const float*>(nullptr), tp.K, DK, DV);
+    if (e != cudaSuccess) return e;
+    state_finish_kernel<DV><<<dim3(DV / 32, DK / 32, units), dim3(32, 8), 0, s>>>(tp.seg_state, tp.seg_decay, tp.K,
+                                                                             a.S_final, a.decay_out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_prefill_state_tc(const PrefillArgs& a, int num_sms, cudaStream_t s) {
+    TcParams tp;
+    memset(&tp, 0, sizeof(tp));
+    const int C = a.chunk;
+    if (!make_map(&tp.tmK, a.K, DK, a.H, a.N, a.B, C) || !make_map(&tp.tmV, a.V, a.dv, a.H, a.N, a.B, C))
+        return cudaErrorInvalidValue;
+    const int nchunks = (a.N + C - 1) / C;
+    const int K = state_pass_pieces(a.B, a.H, a.N, C, num_sms);
+    const WsLayout w = ws_layout(a.B, a.H, a.N, a.dk, a.dv, C, 2, K);
+    uint8_t* ws = static_cast<uint8_t*>(a.workspace);
+    tp.bcum = reinterpret_cast<const float*>(ws + w.bcum);
+    tp.eblk = reinterpret_cast<const float*>(ws + w.eblk);
+    tp.seg_state = reinterpret_cast<float*>(ws + w.state);
+    tp.seg_decay = reinterpret_cast<float*>(ws + w.decay);
+    tp.status = a.status;
+    tp.H = a.H;
+    tp.N = a.N;
+    tp.Npad = nchunks * C;
+    tp.P = 2;                      // the state kernel runs over the first P - 1 = 1 segment: all of it
+    tp.seg_len = nchunks * C;
+    tp.K = K;
+    tp.piece_len = tp.seg_len / K;
+    if (a.dv == 256 && C == 64) return run_state_tc<256, 64>(a, tp, s);
+    if (a.dv == 128 && C == 128) return run_state_tc<128, 128>(a, tp, s);
+    if (a.dv == 128 && C == 64) return run_state_tc<128, 64>(a, tp, s);
+    return cudaErrorNotSupported;
+}
+
+cudaError_t launch_state_fold(const float* dS_all, const float* decay_all, int num_slices, int slice,
+                              const float* S0, float* S_in, int units, int elems, cudaStream_t s) {
+    (void)num_slices;
+    state_fold_kernel<<<dim3((elems + 255) / 256, units), 256, 0, s>>>(dS_all, decay_all, slice, S0, S_in, units,
+                                                                      elems);
+    return cudaGetLastError();
 }
 
 }  // namespace gret

@@ -61,6 +61,9 @@ SIGNATURES = {
                                   _I, _VP]),
     "gret_prefill_from_state": (_I, [_VP, _VP, _VP, _FP, _VP, _FP, _F, _I, _VP, _FP, _I, _I, _I, _I, _I, _I,
                                      _F, _I, _VP, _SZ, _VP]),
+    "gret_prefill_state_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
+    "gret_prefill_state": (_I, [_VP, _VP, _FP, _F, _I, _FP, _FP, _I, _I, _I, _I, _I, _I, _VP, _SZ, _VP]),
+    "gret_state_fold": (_I, [_FP, _FP, _I, _I, _FP, _FP, _I, _I, _I, _I, _VP]),
     "gret_prefill_varlen": (_I, [_VP, _VP, _VP, _FP, _VP, _FP, _VP, _I, _I, _I, _F, _I, _VP, _FP, _I, _I, _I, _I,
                                  _F, _I, _VP, _SZ, _VP]),
     "gret_prefill_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
@@ -108,6 +111,20 @@ def gret_prefill_varlen(Q, K, V, gate_logits, G, S0, cu_seqlens, num_seqs, total
     return load().gret_prefill_varlen(Q, K, V, gate_logits, G, S0, cu_seqlens, num_seqs, total_tokens, max_seqlen,
                                       tau, chunk, O, S_final, H, dk, dv, int(io_dtype), eps, int(epi), workspace,
                                       workspace_bytes, stream)
+
+
+def gret_prefill_state_workspace_size(B, H, N, dk, dv, chunk, io_dtype) -> int:
+    return load().gret_prefill_state_workspace_size(B, H, N, dk, dv, chunk, int(io_dtype))
+
+
+def gret_prefill_state(K, V, gate_logits, tau, chunk, dS, decay, B, H, N, dk, dv, io_dtype, workspace,
+                       workspace_bytes, stream) -> int:
+    return load().gret_prefill_state(K, V, gate_logits, tau, chunk, dS, decay, B, H, N, dk, dv, int(io_dtype),
+                                     workspace, workspace_bytes, stream)
+
+
+def gret_state_fold(dS_all, decay_all, num_slices, slice_, S0, S_in, B, H, dk, dv, stream) -> int:
+    return load().gret_state_fold(dS_all, decay_all, num_slices, slice_, S0, S_in, B, H, dk, dv, stream)
 
 
 def gret_prefill_noalloc(Q, K, V, gate_logits, G, tau, chunk, O, S_final, B, H, N, dk, dv, io_dtype, eps,
@@ -277,6 +294,55 @@ def prefill_varlen(Q, K, V, z, G, cu_seqlens, max_seqlen: int, tau: float, chunk
     if status != Status.OK:
         raise GretError(status, "gret_prefill_varlen")
     return O, S_final
+
+
+def prefill_state(K, V, z, tau: float, chunk: int, workspace=None, stream=None):
+    """State increment and total log-decay of a token slice (gret_prefill_state).
+
+    K [B,N,H,dk], V [B,N,H,dv] (bf16 or fp32), z [B,N,H] fp32.
+    Returns (dS [B,H,dk,dv] fp32, decay [B,H] fp32)."""
+    torch = _torch()
+    B, N, H, dk = K.shape
+    dv = V.shape[-1]
+    dev = K.device
+    io = _io_of(K)
+    _check(V, "V", K.dtype, (B, N, H, dv), dev)
+    _check(z, "z", torch.float32, (B, N, H), dev)
+    dS = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    decay = torch.empty((B, H), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        ws_bytes = gret_prefill_state_workspace_size(B, H, N, dk, dv, chunk, io)
+        if ws_bytes and (workspace is None or workspace.numel() * workspace.element_size() < ws_bytes):
+            workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        st = stream if stream is not None else torch.cuda.current_stream(dev)
+        status = gret_prefill_state(_ptr(K), _ptr(V), _ptr(z), float(tau), int(chunk), _ptr(dS), _ptr(decay), B, H,
+                                    N, dk, dv, io, _ptr(workspace) if ws_bytes else None, ws_bytes, st.cuda_stream)
+    if status != Status.OK:
+        raise GretError(status, "gret_prefill_state")
+    return dS, decay
+
+
+def state_fold(dS_all, decay_all, slice_: int, S0=None, out=None, stream=None):
+    """S_in of slice ``slice_`` from the gathered increments (gret_state_fold).
+
+    dS_all [P,B,H,dk,dv] fp32, decay_all [P,B,H] fp32, S0 [B,H,dk,dv] fp32 or None."""
+    torch = _torch()
+    P, B, H, dk, dv = dS_all.shape
+    dev = dS_all.device
+    _check(dS_all, "dS_all", torch.float32, (P, B, H, dk, dv), dev)
+    _check(decay_all, "decay_all", torch.float32, (P, B, H), dev)
+    if S0 is not None:
+        _check(S0, "S0", torch.float32, (B, H, dk, dv), dev)
+    if out is None:
+        out = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    _check(out, "out", torch.float32, (B, H, dk, dv), dev)
+    with torch.cuda.device(dev):
+        st = stream if stream is not None else torch.cuda.current_stream(dev)
+        status = gret_state_fold(_ptr(dS_all), _ptr(decay_all), P, int(slice_), _ptr(S0), _ptr(out), B, H, dk, dv,
+                                 st.cuda_stream)
+    if status != Status.OK:
+        raise GretError(status, "gret_state_fold")
+    return out
 
 
 def decode_step(q, k, v, z, g, S, tau: float, eps: float = 1e-5, epilogue: str = "gn_swish",

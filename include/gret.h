@@ -139,6 +139,40 @@ gret_status gret_prefill_varlen(const void* Q, const void* K, const void* V, con
                                 gret_epilogue epi, void* workspace, size_t workspace_bytes,
                                 gret_stream_t stream);
 
+/*
+ * Sequence-parallel prefill ("YOCO 深度技术分析", section 5.3.3, Chunk
+ * Parallelism: the devices holding consecutive slices of one sequence pass
+ * only the state between them).  For P slices of the same B x H units:
+ *
+ *   1. each slice: gret_prefill_state -> its increment dS_p (the final state
+ *      of a zero-state prefill of the slice alone) and its total log-decay
+ *      a_p = sum of log gamma over the slice;
+ *   2. exchange (dS_p, a_p) among the slices (an all-gather across devices);
+ *   3. each slice: gret_state_fold -> S_in(p) = e^{a_{p-1}} S_in(p-1) + dS_{p-1},
+ *      S_in(0) = S0 or zero (the state decomposition of the recurrence);
+ *   4. each slice: gret_prefill_from_state(..., S0 = S_in(p), ...).
+ *
+ * gret_prefill_state -- step 1.  K [B][N][H][dk], V [B][N][H][dv] (io dtype),
+ * gate_logits [B][N][H] fp32; dS fp32 [B][H][dk][dv]; decay fp32 [B][H].
+ * Workspace: gret_prefill_state_workspace_size(...) bytes, 256-byte aligned.
+ * Q, G and O play no part.
+ */
+size_t gret_prefill_state_workspace_size(int B, int H, int N, int dk, int dv, int chunk, gret_dtype io_dtype);
+gret_status gret_prefill_state(const void* K, const void* V, const float* gate_logits, float tau, int chunk,
+                               float* dS, float* decay, int B, int H, int N, int dk, int dv,
+                               gret_dtype io_dtype, void* workspace, size_t workspace_bytes,
+                               gret_stream_t stream);
+
+/*
+ * gret_state_fold -- step 3.  dS_all fp32 [num_slices][B][H][dk][dv] and
+ * decay_all fp32 [num_slices][B][H] as gathered; writes S_in fp32
+ * [B][H][dk][dv] for slice `slice` (0 <= slice <= num_slices; slice =
+ * num_slices gives the state after the whole sequence).  S0 may be NULL (zero)
+ * and may be S_in itself; dS_all/decay_all may be NULL when slice = 0.
+ */
+gret_status gret_state_fold(const float* dS_all, const float* decay_all, int num_slices, int slice,
+                            const float* S0, float* S_in, int B, int H, int dk, int dv, gret_stream_t stream);
+
 /* Size of the device scratch array gret_prefill_noalloc draws on (32 MiB). */
 #define GRET_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
 

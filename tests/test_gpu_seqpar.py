@@ -1,0 +1,77 @@
+"""GPU parity of the sequence-parallel prefill's computing steps on one device.
+
+The slices of one sequence are processed in turn on the same GPU: the
+state-only pass of each slice (gret_prefill_state), the fold of the slices
+before it (gret_state_fold), and the prefill of the slice from that state.
+The concatenated outputs and the last state are compared with one oracle
+prefill of the whole sequence; the state-only pass is also compared with the
+oracle's state and decay of each slice alone.  (The all-gather between devices
+is covered by the gloo test of the same code on the CPU.)"""
+import numpy as np
+import pytest
+import torch
+
+import gated_retention_sequence_b200 as gret
+import gret_inputs as gi
+import oracle
+from parity import assert_close
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from gated_retention_sequence_b200 import build
+    build.build()
+    gret.load()
+
+
+def _run(cfg, cuts, expect_path, with_s0):
+    io = gret.Dtype.BF16 if cfg.io == "bf16" else gret.Dtype.F32
+    assert gret.prefill_path(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, cfg.chunk, io)[0] == expect_path
+    inp = gi.prefill_inputs(cfg)
+    d = {k: v.cuda() for k, v in inp.items()}
+    S0 = gi.random_unit(cfg.seed, 904, (cfg.B, cfg.H, cfg.dk, cfg.dv), var=0.04) if with_s0 else None
+    S0d = S0.cuda() if with_s0 else None
+    sl = [{k: v[:, a:b].contiguous() for k, v in d.items()} for a, b in zip(cuts[:-1], cuts[1:])]
+    parts = [gret.prefill_state(s["K"], s["V"], s["z"], cfg.tau, cfg.chunk) for s in sl]
+    gret.check_device_status()
+    # the state-only pass alone, against the oracle on each slice
+    for (a, b), (dS, decay) in zip(zip(cuts[:-1], cuts[1:]), parts):
+        lg = oracle.log_gamma(inp["z"][:, a:b], cfg.tau)
+        _, S_ref = oracle.recurrent(inp["K"][:, a:b], inp["K"][:, a:b], inp["V"][:, a:b], lg)
+        assert_close(dS, S_ref, cfg.io, f"dS of slice {a}:{b}")
+        np.testing.assert_allclose(decay.cpu().double().numpy(), np.asarray(lg).sum(axis=1), rtol=1e-4, atol=1e-3)
+    dS_all = torch.stack([p[0] for p in parts])
+    decay_all = torch.stack([p[1] for p in parts])
+    outs = []
+    for r, s in enumerate(sl):
+        S_in = gret.state_fold(dS_all, decay_all, r, S0=S0d)
+        O, S = gret.prefill(s["Q"], s["K"], s["V"], s["z"], s["G"], cfg.tau, cfg.chunk, eps=cfg.eps, S0=S_in)
+        outs.append((O, S))
+    S_whole = gret.state_fold(dS_all, decay_all, len(sl), S0=S0d)
+    gret.check_device_status()
+    O_ref, _, S_ref = oracle.prefill(inp["Q"], inp["K"], inp["V"], inp["z"], inp["G"], cfg.tau, cfg.eps, S0=S0)
+    assert_close(torch.cat([o for o, _ in outs], dim=1), O_ref, cfg.io, "O of all slices")
+    assert_close(outs[-1][1], S_ref, cfg.io, "state after the last slice")
+    assert_close(S_whole, S_ref, cfg.io, "fold of every slice")
+
+
+def test_tc_three_ragged_slices():
+    cfg = gi.C2.scaled(B=1, H=4, N=3000, chunk=64, seed=61)
+    _run(cfg, (0, 700, 1500, 3000), gret.Path.TC, with_s0=True)
+
+
+def test_tc_dv128_chunk128():
+    cfg = gi.C2.scaled(B=2, H=2, N=2000, dv=128, chunk=128, seed=62, z_dist=((4.0, 1.0),))
+    _run(cfg, (0, 1000, 1130, 2000), gret.Path.TC, with_s0=False)
+
+
+def test_tc_gate_stress():
+    cfg = gi.C2.scaled(B=1, H=2, N=2048, chunk=64, seed=63, z_dist=((-4.0, 1.0), (8.0, 0.5)))
+    _run(cfg, (0, 1024, 2048), gret.Path.TC, with_s0=True)
+
+
+def test_simt_fp32():
+    cfg = gi.C1.scaled(N=256, seed=64)
+    _run(cfg, (0, 100, 256), gret.Path.SIMT, with_s0=True)
