@@ -11,21 +11,22 @@
 //   out    = GroupNorm(O_c) (.) swish(G_c)
 // All exponents are <= 0.
 //
-// B200 mapping.  Every product runs as a 128-row tcgen05.mma (bf16 operands,
-// fp32 accumulation in tensor memory):
+// B200 mapping.  Every product runs as a 128-row tcgen05.mma with fp32
+// accumulation in tensor memory:
 //   scores   D[t][s]          = Q K^T        A = Q (smem, K-major), B = K (K-major)
-//   output   D[d][t] = O^T    = V^T P^T      A = V (smem, MN-major), B = P (K-major)
-//                            + S^T Q~^T     A = bf16 copy of S^T (TMEM), B = Q~ (K-major)
-//   state    D[d][k] = S^T   += V^T K~      A = V (MN-major), B = K~ (MN-major)
+//   output   D[d][t] = O^T    = T^T Q~^T     A = T^T in TMEM (tf32; 64-token chunks)
+//                                            or its bf16 copy (128-token chunks), B = Q~
+//                            + V^T P^T      A = V (smem, MN-major), B = P (K-major)
+//   state    D[d][k] = T^T   += V^T K~      A = V (MN-major), B = K~ (MN-major)
 // so d_v (128 per half) is the MMA's M dimension and the chunk is its N
-// dimension; a 64-token chunk needs no padding except in the small scores
-// product.  S^T stays in fp32 tensor memory for the whole segment; once per
-// chunk the compute warps read it, write a bf16 copy (the A operand of the
-// inter-chunk product) and scale it by e^{b_C} in place before the state MMA
-// accumulates.  Q, K and V tiles arrive by TMA (128-byte swizzle) into a
-// 1-2 stage ring; G arrives into a 2-stage ring and the normalised output is
-// written over it and stored by TMA.  Warp 8 issues the loads, thread 0 the
-// MMAs; eight warps do the decay, the bf16 conversions and the epilogue.
+// dimension.  The state lives in tensor memory for a whole segment as
+// T = S / e^Lambda, rescaled only when the decay since the last rescale grows
+// past e^kLazyMax ("lazy" scaling).  Q, K, V and G tiles arrive by TMA
+// (128-byte swizzle); the normalised output is written over the G tile and
+// stored by TMA.  One warp issues the MMAs, one the TMA traffic, and sixteen
+// compute the decays, P, Q~, K~ and the GroupNorm * swish epilogue; with
+// 64-token chunks they prepare chunk i + 1 before finishing chunk i (see
+// prefill_tc_kernel).
 //
 // Parallelism.  A unit is split into P sequence segments (the chunkwise form
 // applied to segments): a first pass computes each segment's state increment
@@ -539,7 +540,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
             const int valid = n_end - (n_begin + i * C);   // rows of this unit in the chunk (PACKED)
 
             // phase A: Q~ = e^{b_t + Lambda} Q for the inter-chunk read, which the
-            // issuer starts as soon as every warp has done its share
+            // MMA warp starts as soon as every warp has done its share
             if constexpr (TF32) {
                 // fp32 copy in its own buffer, so the scores MMA may still be reading Q
                 for (int it = tid; it < C * 16; it += kCT) {
@@ -702,7 +703,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
         };
 
         // ---- epilogue of chunk i from Y in registers: GroupNorm over d_v, times
-        // swish(G), as bf16 over G in its stage, then handed to the issuer for
+        // swish(G), as bf16 over G in its stage, then handed to the TMA warp for
         // the store.  Thread (q4, grp, lane) owns d_v channels h*128 + q4*32 + lane
         // (h < NH) for tokens grp*HT .. grp*HT + HT - 1.
         auto epilogue = [&](int i, const float (&y)[NH][HT]) {
