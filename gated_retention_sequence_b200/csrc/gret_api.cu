@@ -296,4 +296,37 @@ gret_status gret_state_fold(const float* dS_all, const float* decay_all, int num
     return err == cudaSuccess ? GRET_OK : GRET_ERR_CUDA;
 }
 
+size_t gret_prefill_backward_workspace_size(int B, int H, int N, int dk, int dv) {
+    if (B <= 0 || H <= 0 || N <= 0 || !shape_supported(dk, dv) || !prefill_backward_supported(dk, dv)) return 0;
+    return prefill_backward_workspace_bytes(B, H, N, dk, dv);
+}
+
+gret_status gret_prefill_backward(const void* Q, const void* K, const void* V, const float* gate_logits,
+                                  const void* G, const float* S0, const void* dO, const float* dS_final, float tau,
+                                  float eps, gret_epilogue epi, void* dQ, void* dK, void* dV, float* dz, void* dG,
+                                  float* dS0, int B, int H, int N, int dk, int dv, gret_dtype io_dtype,
+                                  void* workspace, size_t workspace_bytes, gret_stream_t stream) {
+    if (!Q || !K || !V || !gate_logits || !dO || !dQ || !dK || !dV || !dz) return GRET_ERR_INVALID_ARG;
+    if (epi != GRET_EPI_GN_SWISH && epi != GRET_EPI_NONE) return GRET_ERR_INVALID_ARG;
+    if (epi == GRET_EPI_GN_SWISH && (!G || !dG)) return GRET_ERR_INVALID_ARG;
+    if (io_dtype != GRET_F32 && io_dtype != GRET_BF16) return GRET_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || N <= 0 || dk <= 0 || dv <= 0) return GRET_ERR_INVALID_ARG;
+    if (!(tau > 0.0f) || !isfinite(tau) || !(eps >= 0.0f) || !isfinite(eps)) return GRET_ERR_INVALID_ARG;
+    const void* ptrs[] = {Q, K, V, gate_logits, dO, dQ, dK, dV, dz, G, dG, S0, dS_final, dS0};
+    for (const void* q : ptrs)
+        if (q && !aligned16(q)) return GRET_ERR_INVALID_ARG;
+    if ((long long)B * H > (1LL << 30) || (long long)B * N > (1LL << 40)) return GRET_ERR_UNSUPPORTED;
+    if (!shape_supported(dk, dv) || !prefill_backward_supported(dk, dv)) return GRET_ERR_UNSUPPORTED;
+    const size_t need = prefill_backward_workspace_bytes(B, H, N, dk, dv);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return GRET_ERR_INVALID_ARG;
+    BackwardArgs a = {};
+    a.Q = Q; a.K = K; a.V = V; a.G = G; a.dO = dO; a.z = gate_logits; a.S0 = S0; a.dS_final = dS_final;
+    a.dQ = dQ; a.dK = dK; a.dV = dV; a.dG = dG; a.dz = dz; a.dS0 = dS0; a.workspace = workspace;
+    a.B = B; a.H = H; a.N = N; a.dk = dk; a.dv = dv; a.inv_tau = 1.0f / tau; a.eps = eps;
+    a.gn = epi == GRET_EPI_GN_SWISH ? 1 : 0; a.io = io_dtype;
+    return launch_prefill_backward(a, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? GRET_OK
+                                                                                        : GRET_ERR_CUDA;
+}
+
 }  // extern "C"

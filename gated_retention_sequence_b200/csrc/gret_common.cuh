@@ -110,6 +110,22 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_prefill_simt(const PrefillArgs& a, cudaStream_t s);
 size_t prefill_simt_smem_bytes(int dk, int dv, int chunk);
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s);
+
+// Backward of the prefill (CUDA cores, gret_backward.cu).
+struct BackwardArgs {
+    const void *Q, *K, *V, *G, *dO;
+    const float *z, *S0, *dS_final;
+    void *dQ, *dK, *dV, *dG;
+    float *dz, *dS0;
+    void* workspace;
+    int B, H, N, dk, dv;
+    float inv_tau, eps;
+    int gn;
+    gret_dtype io;
+};
+size_t prefill_backward_workspace_bytes(int B, int H, int N, int dk, int dv);
+bool prefill_backward_supported(int dk, int dv);
+cudaError_t launch_prefill_backward(const BackwardArgs& a, cudaStream_t s);
 // state-only pass of the tensor-core path (a.state_only): workspace bytes and launch
 size_t prefill_tc_state_workspace_bytes(int B, int H, int N, int dk, int dv, int chunk, int num_sms);
 cudaError_t launch_prefill_state_tc(const PrefillArgs& a, int num_sms, cudaStream_t s);

@@ -64,6 +64,9 @@ SIGNATURES = {
     "gret_prefill_state_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
     "gret_prefill_state": (_I, [_VP, _VP, _FP, _F, _I, _FP, _FP, _I, _I, _I, _I, _I, _I, _VP, _SZ, _VP]),
     "gret_state_fold": (_I, [_FP, _FP, _I, _I, _FP, _FP, _I, _I, _I, _I, _VP]),
+    "gret_prefill_backward_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
+    "gret_prefill_backward": (_I, [_VP, _VP, _VP, _FP, _VP, _FP, _VP, _FP, _F, _F, _I, _VP, _VP, _VP, _FP, _VP, _FP,
+                                   _I, _I, _I, _I, _I, _I, _VP, _SZ, _VP]),
     "gret_prefill_varlen": (_I, [_VP, _VP, _VP, _FP, _VP, _FP, _VP, _I, _I, _I, _F, _I, _VP, _FP, _I, _I, _I, _I,
                                  _F, _I, _VP, _SZ, _VP]),
     "gret_prefill_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
@@ -125,6 +128,17 @@ def gret_prefill_state(K, V, gate_logits, tau, chunk, dS, decay, B, H, N, dk, dv
 
 def gret_state_fold(dS_all, decay_all, num_slices, slice_, S0, S_in, B, H, dk, dv, stream) -> int:
     return load().gret_state_fold(dS_all, decay_all, num_slices, slice_, S0, S_in, B, H, dk, dv, stream)
+
+
+def gret_prefill_backward_workspace_size(B, H, N, dk, dv) -> int:
+    return load().gret_prefill_backward_workspace_size(B, H, N, dk, dv)
+
+
+def gret_prefill_backward(Q, K, V, gate_logits, G, S0, dO, dS_final, tau, eps, epi, dQ, dK, dV, dz, dG, dS0, B, H,
+                          N, dk, dv, io_dtype, workspace, workspace_bytes, stream) -> int:
+    return load().gret_prefill_backward(Q, K, V, gate_logits, G, S0, dO, dS_final, tau, eps, int(epi), dQ, dK, dV,
+                                        dz, dG, dS0, B, H, N, dk, dv, int(io_dtype), workspace, workspace_bytes,
+                                        stream)
 
 
 def gret_prefill_noalloc(Q, K, V, gate_logits, G, tau, chunk, O, S_final, B, H, N, dk, dv, io_dtype, eps,
@@ -342,6 +356,45 @@ def state_fold(dS_all, decay_all, slice_: int, S0=None, out=None, stream=None):
                                  st.cuda_stream)
     if status != Status.OK:
         raise GretError(status, "gret_state_fold")
+    return out
+
+
+def prefill_backward(Q, K, V, z, G, dO, tau: float, eps: float = 1e-5, epilogue: str = "gn_swish", S0=None,
+                     dS_final=None, want_dS0: bool = False, workspace=None, stream=None):
+    """Gradients of <O, dO> + <S_final, dS_final> (gret_prefill_backward).
+
+    Shapes as for ``prefill``.  Returns a dict: dQ, dK, dV (io dtype), dz (fp32),
+    dG (io dtype; None for epilogue='none'), dS0 (fp32, when S0 is given or
+    want_dS0)."""
+    torch = _torch()
+    B, N, H, dk = Q.shape
+    dv = V.shape[-1]
+    dev = Q.device
+    io = _io_of(Q)
+    epi = Epilogue.NONE if epilogue == "none" else Epilogue.GN_SWISH
+    for t, name, shape in ((K, "K", (B, N, H, dk)), (V, "V", (B, N, H, dv)), (dO, "dO", (B, N, H, dv))):
+        _check(t, name, Q.dtype, shape, dev)
+    _check(z, "z", torch.float32, (B, N, H), dev)
+    if epi == Epilogue.GN_SWISH:
+        _check(G, "G", Q.dtype, (B, N, H, dv), dev)
+    for t, name in ((S0, "S0"), (dS_final, "dS_final")):
+        if t is not None:
+            _check(t, name, torch.float32, (B, H, dk, dv), dev)
+    out = {"dQ": torch.empty_like(Q), "dK": torch.empty_like(K), "dV": torch.empty_like(V),
+           "dz": torch.empty_like(z), "dG": torch.empty_like(V) if epi == Epilogue.GN_SWISH else None,
+           "dS0": torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev) if (S0 is not None or want_dS0)
+           else None}
+    with torch.cuda.device(dev):
+        ws_bytes = gret_prefill_backward_workspace_size(B, H, N, dk, dv)
+        if ws_bytes and (workspace is None or workspace.numel() * workspace.element_size() < ws_bytes):
+            workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        st = stream if stream is not None else torch.cuda.current_stream(dev)
+        status = gret_prefill_backward(_ptr(Q), _ptr(K), _ptr(V), _ptr(z), _ptr(G), _ptr(S0), _ptr(dO), _ptr(dS_final),
+                                       float(tau), float(eps), epi, _ptr(out["dQ"]), _ptr(out["dK"]), _ptr(out["dV"]),
+                                       _ptr(out["dz"]), _ptr(out["dG"]), _ptr(out["dS0"]), B, H, N, dk, dv, io,
+                                       _ptr(workspace) if ws_bytes else None, ws_bytes, st.cuda_stream)
+    if status != Status.OK:
+        raise GretError(status, "gret_prefill_backward")
     return out
 
 

@@ -173,6 +173,29 @@ gret_status gret_prefill_state(const void* K, const void* V, const float* gate_l
 gret_status gret_state_fold(const float* dS_all, const float* decay_all, int num_slices, int slice,
                             const float* S0, float* S_in, int B, int H, int dk, int dv, gret_stream_t stream);
 
+/*
+ * gret_prefill_backward -- gradients of the prefill (for training).
+ *
+ * The pages give the forward; this is its exact derivative.  For an upstream
+ * gradient dO of O (and optionally dS_final of S_final), returns the gradients
+ * of <O, dO> + <S_final, dS_final> with respect to Q, K, V (io dtype, their
+ * layouts), the gate logits dz (fp32 [B][N][H]), G (io dtype; GN_SWISH only)
+ * and the initial state dS0 (fp32 [B][H][dk][dv]; may be NULL).  S0 and
+ * dS_final may be NULL (zero).  Arithmetic is fp32 on CUDA cores; the state at
+ * every 32-token block is kept as a checkpoint in the workspace
+ * (gret_prefill_backward_workspace_size bytes: B*H*ceil(N/32)*dk*dv*4 plus one
+ * state per unit), then the blocks are walked in reverse.  Where the forward
+ * clamps a log-decay at -64 the gate gradient is zero.  dk, dv multiples of 16
+ * up to 256 (GRET_ERR_UNSUPPORTED beyond what fits in shared memory).
+ */
+size_t gret_prefill_backward_workspace_size(int B, int H, int N, int dk, int dv);
+gret_status gret_prefill_backward(const void* Q, const void* K, const void* V, const float* gate_logits,
+                                  const void* G, const float* S0, const void* dO, const float* dS_final,
+                                  float tau, float eps, gret_epilogue epi, void* dQ, void* dK, void* dV,
+                                  float* dz, void* dG, float* dS0, int B, int H, int N, int dk, int dv,
+                                  gret_dtype io_dtype, void* workspace, size_t workspace_bytes,
+                                  gret_stream_t stream);
+
 /* Size of the device scratch array gret_prefill_noalloc draws on (32 MiB). */
 #define GRET_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
 
