@@ -1039,33 +1039,38 @@ __global__ void __launch_bounds__(kStateThreads, 1) prefill_state_kernel(const _
 // Chunk-local inclusive sums of log gamma: bcum[u][n] = sum_{j in chunk, j <= n} lg_j,
 // and the P step's block factors eblk (below).
 // Padding tokens (n >= N) carry lg = 0, so they repeat the chunk total.
-__global__ void gate_scan_kernel(const float* __restrict__ z, const int* __restrict__ cu_seqlens, int total,
-                                 float* __restrict__ bcum, float* __restrict__ eblk, int H, int N, int Npad,
-                                 float inv_tau) {
-    __shared__ float wsum[4];
+constexpr int kScanThreads = 256;   // a block scans 256 / C chunks of one unit
+
+__global__ void __launch_bounds__(kScanThreads) gate_scan_kernel(const float* __restrict__ z,
+                                                                 const int* __restrict__ cu_seqlens, int total,
+                                                                 float* __restrict__ bcum, float* __restrict__ eblk,
+                                                                 int H, int N, int Npad, int C, float inv_tau) {
+    __shared__ float wsum[kScanThreads / 32];
     // the gate logits may come from the kernel before this one, and the kernels
     // before that may still read the workspace: wait for them first
     grid_dep_launch();
     grid_dep_wait();
-    const int C = blockDim.x;
     const int u = blockIdx.x, b = u / H, h = u % H;
-    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
-    const int n = blockIdx.y * C + t;
+    const int lane = threadIdx.x & 31, wg = threadIdx.x >> 5;
+    const int t = threadIdx.x % C, w = t >> 5;                 // token and warp within the chunk
+    const int ch = blockIdx.y * (kScanThreads / C) + threadIdx.x / C;
+    const bool live = ch * C < Npad;
+    const int n = ch * C + t;
     // this unit's tokens are rows base .. base + Nu - 1; past its end the
     // decay stays flat (log gamma = 0), so a chunk's last sum is its decay
     int row0 = 0, Nu = N;
     if (cu_seqlens) packed_range(cu_seqlens, b, total, row0, Nu);
     const size_t base = cu_seqlens ? (size_t)row0 : (size_t)b * N;
-    float x = n < Nu ? log_gamma(z[(base + n) * H + h], inv_tau) : 0.f;
+    float x = (live && n < Nu) ? log_gamma(z[(base + n) * H + h], inv_tau) : 0.f;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         float y = __shfl_up_sync(0xffffffffu, x, o);
         if (lane >= o) x += y;
     }
-    if (lane == 31) wsum[w] = x;
+    if (lane == 31) wsum[wg] = x;
     __syncthreads();
-    for (int j = 0; j < w; ++j) x += wsum[j];
-    bcum[(size_t)u * Npad + n] = x;
+    for (int j = 0; j < w; ++j) x += wsum[wg - w + j];      // the chunk's earlier warps
+    if (live) bcum[(size_t)u * Npad + n] = x;
     // block factors for the P step: E_n = e^{b_{s0} - b_n}, s0 the first token of
     // n's block of C/4 (16 or 32, within one warp); a block whose decay drops by
     // more than kBlockMax gets E_{s0} = -1 instead, so the P step takes the
@@ -1075,7 +1080,7 @@ __global__ void gate_scan_kernel(const float* __restrict__ z, const int* __restr
     const float xl = __shfl_sync(0xffffffffu, x, lane | (bw - 1));
     float e = expf(x0 - x);
     if (x0 - xl > kBlockMax) e = (lane & (bw - 1)) == 0 ? -1.f : 0.f;
-    eblk[(size_t)u * Npad + n] = e;
+    if (live) eblk[(size_t)u * Npad + n] = e;
 }
 
 // Fold the segment increments into initial states, in place:
@@ -1228,8 +1233,10 @@ cudaError_t run_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t s) {
     }
     const int units = a.B * a.H;
     const int npad = tp.Npad;
-    cudaError_t e = launch_pdl(gate_scan_kernel, dim3(units, npad / C), dim3(C), 0, s, a.z, a.cu_seqlens, a.total,
-                               const_cast<float*>(tp.bcum), const_cast<float*>(tp.eblk), a.H, a.N, npad, a.inv_tau);
+    const int per = kScanThreads / C;
+    cudaError_t e = launch_pdl(gate_scan_kernel, dim3(units, (npad / C + per - 1) / per), dim3(kScanThreads), 0, s,
+                               a.z, a.cu_seqlens, a.total, const_cast<float*>(tp.bcum), const_cast<float*>(tp.eblk),
+                               a.H, a.N, npad, C, a.inv_tau);
     if (e != cudaSuccess) return e;
     if (tp.P > 1) {
         e = launch_pdl(ks, dim3(units * (tp.P - 1) * tp.K), dim3(kStateThreads), StateCfg<DV, C>::SMEM, s, tp);
@@ -1345,9 +1352,10 @@ static cudaError_t run_state_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t
     auto ks = prefill_state_kernel<DV, C, false>;
     cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, StateCfg<DV, C>::SMEM);
     const int units = a.B * a.H;
-    cudaError_t e = launch_pdl(gate_scan_kernel, dim3(units, tp.Npad / C), dim3(C), 0, s, a.z,
-                               static_cast<const int*>(nullptr), 0, const_cast<float*>(tp.bcum),
-                               const_cast<float*>(tp.eblk), a.H, a.N, tp.Npad, a.inv_tau);
+    const int per = kScanThreads / C;
+    cudaError_t e = launch_pdl(gate_scan_kernel, dim3(units, (tp.Npad / C + per - 1) / per), dim3(kScanThreads), 0, s,
+                               a.z, static_cast<const int*>(nullptr), 0, const_cast<float*>(tp.bcum),
+                               const_cast<float*>(tp.eblk), a.H, a.N, tp.Npad, C, a.inv_tau);
     if (e != cudaSuccess) return e;
     e = launch_pdl(ks, dim3(units * tp.K), dim3(kStateThreads), StateCfg<DV, C>::SMEM, s, tp);
     if (e != cudaSuccess) return e;
