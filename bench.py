@@ -324,6 +324,8 @@ def run_ours(args, world, rank, local):
         e2e_value = job_throughput(world, tokens, e2e_steps, e2e_ms) / 1e6
 
     decode = None if args.no_decode else run_decode(args, world, dev, stream, peaks)
+    varlen = None if args.no_varlen else run_varlen(args, world, dev, stream, d, cfg, peaks)
+    backward = None if args.no_backward else run_backward(args, world, dev, stream, d, O, cfg, peaks)
     clk = clocks.stop()
 
     line = None
@@ -354,6 +356,8 @@ def run_ours(args, world, rank, local):
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk,
             "decode": decode,
+            "varlen": varlen,
+            "backward": backward,
         }
         if world == 1 and not args.no_cpu_baseline:
             import oracle
@@ -366,6 +370,113 @@ def run_ours(args, world, rank, local):
                                               f"{dt:.1f} s"}
         print(json.dumps(line), flush=True)
     return 0
+
+
+def varlen_lengths(total: int, max_len: int, seed: int):
+    """A ragged mix of sequence lengths summing to `total`: log-uniform draws in
+    [1, max_len] (short prompts next to long documents), with a one-token
+    sequence and lengths that are no multiple of the chunk."""
+    import numpy as np
+    rng = np.random.default_rng(seed)
+    lengths = [1]
+    while sum(lengths) < total:
+        lengths.append(int(np.exp(rng.uniform(0.0, np.log(max_len)))))
+    lengths[-1] -= sum(lengths) - total
+    if lengths[-1] == 0:
+        lengths.pop()
+    return lengths
+
+
+def run_varlen(args, world, dev, stream, d, cfg, peaks):
+    """gret_prefill_varlen over the benchmark's own tokens (B*N of them, same
+    heads and head sizes) packed as a ragged batch of sequences."""
+    import numpy as np
+    import torch
+    import gated_retention_sequence_b200 as gret
+    T = cfg.B * cfg.N
+    lengths = varlen_lengths(T, cfg.N, seed=17)
+    cu = torch.from_numpy(np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)).to(dev)
+    flat = {k: v.view((T,) + tuple(v.shape[2:])) for k, v in d.items()}
+    S_n, max_len = len(lengths), max(lengths)
+    O = torch.empty_like(flat["V"])
+    S = torch.empty((S_n, cfg.H, cfg.dk, cfg.dv), dtype=torch.float32, device=dev)
+    io = gret.Dtype.BF16
+    ws_bytes = gret.gret_prefill_workspace_size(S_n, cfg.H, max_len, cfg.dk, cfg.dv, cfg.chunk, io)
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+
+    def step():
+        gret.prefill_varlen(flat["Q"], flat["K"], flat["V"], flat["z"], flat["G"], cu, max_len, cfg.tau,
+                            cfg.chunk, eps=cfg.eps, O=O, S_final=S, workspace=ws, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    gret.check_device_status()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    barrier(world)
+    gret.check_device_status()
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    path, segs = gret.prefill_path(S_n, cfg.H, max_len, cfg.dk, cfg.dv, cfg.chunk, io)
+    bytes_, _ = prefill_alg(cfg)
+    bytes_ += (S_n - cfg.B) * cfg.H * 4 * cfg.dk * cfg.dv       # one final state per sequence
+    step_s = ms / 1e3 / args.steps
+    return {"workload": f"{cfg.name} tokens packed as {S_n} sequences of 1..{max_len} tokens",
+            "sequences": S_n, "tokens": T, "steps": args.steps, "ms_per_step": ms / args.steps,
+            "value": job_throughput(world, T, args.steps, ms) / 1e6, "unit": "Mtok/s",
+            "path": path.name, "segments": segs,
+            "path_hbm": {"alg_gbs": bytes_ / step_s / 1e9, "frac": bytes_ / step_s / 1e9 / peaks["hbm_gbs"]},
+            "gpu_launches": gret.gret_prefill_launches(S_n, cfg.H, max_len, cfg.dk, cfg.dv, cfg.chunk, io)
+            * args.steps}
+
+
+def backward_alg(cfg):
+    """Algorithmic bytes of one backward: Q, K, V, G and dO read, dQ, dK, dV, dG
+    written (io dtype), z read and dz written (fp32)."""
+    e = 2 if cfg.io == "bf16" else 4
+    return cfg.B * cfg.N * cfg.H * (e * (4 * cfg.dk + 5 * cfg.dv) + 8)
+
+
+def run_backward(args, world, dev, stream, d, O, cfg, peaks):
+    """gret_prefill_backward on the benchmark workload (CUDA-core kernels).
+    The upstream gradient dO is the forward's own output O (any tensor of O's
+    shape and dtype serves; the cost does not depend on its values)."""
+    import torch
+    import gated_retention_sequence_b200 as gret
+    steps = max(1, min(args.steps, 5))
+    dO = O.clone()
+    io = gret.Dtype.BF16
+    ws_bytes = gret.gret_prefill_backward_workspace_size(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, io)
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+
+    def step():
+        return gret.prefill_backward(d["Q"], d["K"], d["V"], d["z"], d["G"], dO, cfg.tau, eps=cfg.eps,
+                                     workspace=ws, stream=stream)
+
+    for _ in range(2):
+        step()
+    gret.check_device_status()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    barrier(world)
+    gret.check_device_status()
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    bytes_ = backward_alg(cfg)
+    step_s = ms / 1e3 / steps
+    tokens = cfg.B * cfg.N
+    return {"workload": cfg.name, "steps": steps, "warmup": 2, "ms_per_step": ms / steps,
+            "value": job_throughput(world, tokens, steps, ms) / 1e6, "unit": "Mtok/s",
+            "kernels": "bwd_inc, bwd_fwd_scan, bwd_dy, bwd_rev_scan, bwd_grad (CUDA cores, fp32 arithmetic)",
+            "path_hbm": {"alg_bytes": bytes_, "alg_gbs": bytes_ / step_s / 1e9,
+                         "frac": bytes_ / step_s / 1e9 / peaks["hbm_gbs"]},
+            "gpu_launches": gret.gret_prefill_backward_launches(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, io) * steps}
 
 
 def run_decode(args, world, dev, stream, peaks):
@@ -415,6 +526,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-varlen", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()

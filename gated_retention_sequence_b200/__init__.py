@@ -7,7 +7,8 @@ package only marshals arguments (see ``gret.py``).
 from .gret import (  # noqa: F401
     Dtype, Epilogue, GretError, LIB_PATH, Path, SIGNATURES, Status, check_device_status, decode_step,
     gret_decode_step, gret_last_device_status, gret_prefill, gret_prefill_backward,
-    gret_prefill_backward_workspace_size, gret_prefill_from_state, gret_prefill_launches,
+    gret_prefill_backward_launches, gret_prefill_backward_workspace_size, gret_prefill_from_state,
+    gret_prefill_launches,
     gret_prefill_noalloc, gret_prefill_path, gret_prefill_state, gret_prefill_state_workspace_size,
     gret_prefill_varlen, gret_prefill_workspace_size, gret_state_fold,
     gret_set_profile_events, gret_status_string, gret_version, load, prefill, prefill_backward, prefill_path, prefill_state,

@@ -296,9 +296,16 @@ gret_status gret_state_fold(const float* dS_all, const float* decay_all, int num
     return err == cudaSuccess ? GRET_OK : GRET_ERR_CUDA;
 }
 
-size_t gret_prefill_backward_workspace_size(int B, int H, int N, int dk, int dv) {
+size_t gret_prefill_backward_workspace_size(int B, int H, int N, int dk, int dv, gret_dtype io_dtype) {
     if (B <= 0 || H <= 0 || N <= 0 || !shape_supported(dk, dv) || !prefill_backward_supported(dk, dv)) return 0;
-    return prefill_backward_workspace_bytes(B, H, N, dk, dv);
+    if (io_dtype != GRET_F32 && io_dtype != GRET_BF16) return 0;
+    return prefill_backward_workspace_bytes(B, H, N, dk, dv, io_dtype);
+}
+
+int gret_prefill_backward_launches(int B, int H, int N, int dk, int dv, gret_dtype io_dtype) {
+    if (B <= 0 || H <= 0 || N <= 0 || !shape_supported(dk, dv) || !prefill_backward_supported(dk, dv)) return 0;
+    if (io_dtype != GRET_F32 && io_dtype != GRET_BF16) return 0;
+    return prefill_backward_launches(B, H, N, dk, dv, io_dtype);
 }
 
 gret_status gret_prefill_backward(const void* Q, const void* K, const void* V, const float* gate_logits,
@@ -317,7 +324,7 @@ gret_status gret_prefill_backward(const void* Q, const void* K, const void* V, c
         if (q && !aligned16(q)) return GRET_ERR_INVALID_ARG;
     if ((long long)B * H > (1LL << 30) || (long long)B * N > (1LL << 40)) return GRET_ERR_UNSUPPORTED;
     if (!shape_supported(dk, dv) || !prefill_backward_supported(dk, dv)) return GRET_ERR_UNSUPPORTED;
-    const size_t need = prefill_backward_workspace_bytes(B, H, N, dk, dv);
+    const size_t need = prefill_backward_workspace_bytes(B, H, N, dk, dv, io_dtype);
     if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
         return GRET_ERR_INVALID_ARG;
     BackwardArgs a = {};

@@ -345,7 +345,8 @@ size_t bwd_ckpt_smem(int dk, int dv) { return sizeof(float) * ((size_t)kBlk * (d
 
 }  // namespace
 
-size_t prefill_backward_workspace_bytes(int B, int H, int N, int dk, int dv) {
+size_t prefill_backward_workspace_bytes(int B, int H, int N, int dk, int dv, gret_dtype io) {
+    if (bwd_chunked_supported(B, H, N, dk, dv, io)) return bwd_chunked_workspace_bytes(B, H, N, dk, dv, io);
     const size_t units = (size_t)B * H, nblk = (N + kBlk - 1) / kBlk, E = (size_t)dk * dv;
     const size_t ck = (units * nblk * E * 4 + 255) & ~size_t(255);
     return ck + units * E * 4;
@@ -353,7 +354,12 @@ size_t prefill_backward_workspace_bytes(int B, int H, int N, int dk, int dv) {
 
 bool prefill_backward_supported(int dk, int dv) { return bwd_block_smem(dk, dv) <= 227 * 1024; }
 
+int prefill_backward_launches(int B, int H, int N, int dk, int dv, gret_dtype io) {
+    return bwd_chunked_supported(B, H, N, dk, dv, io) ? 5 : 2;
+}
+
 cudaError_t launch_prefill_backward(const BackwardArgs& in, cudaStream_t s) {
+    if (bwd_chunked_supported(in.B, in.H, in.N, in.dk, in.dv, in.io)) return launch_bwd_chunked(in, s);
     BwdArgs a;
     a.Q = in.Q; a.K = in.K; a.V = in.V; a.G = in.G; a.dO = in.dO;
     a.z = in.z; a.S0 = in.S0; a.dS_final = in.dS_final;

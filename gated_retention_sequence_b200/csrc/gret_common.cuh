@@ -123,9 +123,16 @@ struct BackwardArgs {
     int gn;
     gret_dtype io;
 };
-size_t prefill_backward_workspace_bytes(int B, int H, int N, int dk, int dv);
+size_t prefill_backward_workspace_bytes(int B, int H, int N, int dk, int dv, gret_dtype io);
 bool prefill_backward_supported(int dk, int dv);
+// launches one backward call makes (5 on the chunk-parallel path, 2 on the serial one)
+int prefill_backward_launches(int B, int H, int N, int dk, int dv, gret_dtype io);
 cudaError_t launch_prefill_backward(const BackwardArgs& a, cudaStream_t s);
+// chunk-parallel backward (gret_backward_chunk.cu): head sizes multiples of 32,
+// dk <= 128, dv <= 256
+bool bwd_chunked_supported(int B, int H, int N, int dk, int dv, gret_dtype io);
+size_t bwd_chunked_workspace_bytes(int B, int H, int N, int dk, int dv, gret_dtype io);
+cudaError_t launch_bwd_chunked(const BackwardArgs& a, cudaStream_t s);
 // state-only pass of the tensor-core path (a.state_only): workspace bytes and launch
 size_t prefill_tc_state_workspace_bytes(int B, int H, int N, int dk, int dv, int chunk, int num_sms);
 cudaError_t launch_prefill_state_tc(const PrefillArgs& a, int num_sms, cudaStream_t s);

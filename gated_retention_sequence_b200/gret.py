@@ -64,7 +64,8 @@ SIGNATURES = {
     "gret_prefill_state_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
     "gret_prefill_state": (_I, [_VP, _VP, _FP, _F, _I, _FP, _FP, _I, _I, _I, _I, _I, _I, _VP, _SZ, _VP]),
     "gret_state_fold": (_I, [_FP, _FP, _I, _I, _FP, _FP, _I, _I, _I, _I, _VP]),
-    "gret_prefill_backward_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
+    "gret_prefill_backward_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
+    "gret_prefill_backward_launches": (_I, [_I, _I, _I, _I, _I, _I]),
     "gret_prefill_backward": (_I, [_VP, _VP, _VP, _FP, _VP, _FP, _VP, _FP, _F, _F, _I, _VP, _VP, _VP, _FP, _VP, _FP,
                                    _I, _I, _I, _I, _I, _I, _VP, _SZ, _VP]),
     "gret_prefill_varlen": (_I, [_VP, _VP, _VP, _FP, _VP, _FP, _VP, _I, _I, _I, _F, _I, _VP, _FP, _I, _I, _I, _I,
@@ -130,8 +131,12 @@ def gret_state_fold(dS_all, decay_all, num_slices, slice_, S0, S_in, B, H, dk, d
     return load().gret_state_fold(dS_all, decay_all, num_slices, slice_, S0, S_in, B, H, dk, dv, stream)
 
 
-def gret_prefill_backward_workspace_size(B, H, N, dk, dv) -> int:
-    return load().gret_prefill_backward_workspace_size(B, H, N, dk, dv)
+def gret_prefill_backward_workspace_size(B, H, N, dk, dv, io_dtype) -> int:
+    return load().gret_prefill_backward_workspace_size(B, H, N, dk, dv, int(io_dtype))
+
+
+def gret_prefill_backward_launches(B, H, N, dk, dv, io_dtype) -> int:
+    return load().gret_prefill_backward_launches(B, H, N, dk, dv, int(io_dtype))
 
 
 def gret_prefill_backward(Q, K, V, gate_logits, G, S0, dO, dS_final, tau, eps, epi, dQ, dK, dV, dz, dG, dS0, B, H,
@@ -385,7 +390,7 @@ def prefill_backward(Q, K, V, z, G, dO, tau: float, eps: float = 1e-5, epilogue:
            "dS0": torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev) if (S0 is not None or want_dS0)
            else None}
     with torch.cuda.device(dev):
-        ws_bytes = gret_prefill_backward_workspace_size(B, H, N, dk, dv)
+        ws_bytes = gret_prefill_backward_workspace_size(B, H, N, dk, dv, io)
         if ws_bytes and (workspace is None or workspace.numel() * workspace.element_size() < ws_bytes):
             workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
         st = stream if stream is not None else torch.cuda.current_stream(dev)

@@ -181,14 +181,22 @@ gret_status gret_state_fold(const float* dS_all, const float* decay_all, int num
  * of <O, dO> + <S_final, dS_final> with respect to Q, K, V (io dtype, their
  * layouts), the gate logits dz (fp32 [B][N][H]), G (io dtype; GN_SWISH only)
  * and the initial state dS0 (fp32 [B][H][dk][dv]; may be NULL).  S0 and
- * dS_final may be NULL (zero).  Arithmetic is fp32 on CUDA cores; the state at
- * every 32-token block is kept as a checkpoint in the workspace
- * (gret_prefill_backward_workspace_size bytes: B*H*ceil(N/32)*dk*dv*4 plus one
- * state per unit), then the blocks are walked in reverse.  Where the forward
- * clamps a log-decay at -64 the gate gradient is zero.  dk, dv multiples of 16
- * up to 256 (GRET_ERR_UNSUPPORTED beyond what fits in shared memory).
+ * dS_final may be NULL (zero).  Arithmetic is fp32 on CUDA cores.
+ *
+ * Head sizes that are multiples of 32 with dk <= 128 and dv <= 256 take the
+ * chunk-parallel path (5 launches; chunks of 64 tokens for bf16, 32 for fp32):
+ * the workspace holds the state before every chunk and the gradient at every
+ * chunk's end (2 * B*H*ceil(N/chunk)*dk*dv*4 bytes), the gradient of the
+ * pre-norm output (B*N*H*dv*4) and one decay per chunk.  Other head sizes
+ * (multiples of 16 up to 256) take a serial path (2 launches) that keeps the
+ * state at every 32-token block (B*H*ceil(N/32)*dk*dv*4 plus one state per
+ * unit) and walks the blocks in reverse.  The size depends on io_dtype; 0 for
+ * an unsupported shape.  Where the forward clamps a log-decay at -64 the gate
+ * gradient is zero.
  */
-size_t gret_prefill_backward_workspace_size(int B, int H, int N, int dk, int dv);
+size_t gret_prefill_backward_workspace_size(int B, int H, int N, int dk, int dv, gret_dtype io_dtype);
+/* Kernel launches one gret_prefill_backward call makes for this shape (0 if unsupported). */
+int gret_prefill_backward_launches(int B, int H, int N, int dk, int dv, gret_dtype io_dtype);
 gret_status gret_prefill_backward(const void* Q, const void* K, const void* V, const float* gate_logits,
                                   const void* G, const float* S0, const void* dO, const float* dS_final,
                                   float tau, float eps, gret_epilogue epi, void* dQ, void* dK, void* dV,

@@ -113,3 +113,25 @@ def test_path_selection(lib):
     assert gret.prefill_path(1, 2, 256, 64, 64, 48, gret.Dtype.F32)[0] == gret.Path.NONE
     assert gret.prefill_path(1, 2, 256, 256, 256, 128, gret.Dtype.F32)[0] == gret.Path.NONE
     assert gret.gret_prefill_workspace_size(1, 2, 256, 64, 64, 64, gret.Dtype.F32) == 0
+
+
+def test_backward_path_and_workspace(lib):
+    bf, f32 = gret.Dtype.BF16, gret.Dtype.F32
+    E = 128 * 256
+    # chunk-parallel path: chunks of 64 tokens (bf16) or 32 (fp32); two states per
+    # chunk, the fp32 gradient of the pre-norm output and one decay per chunk
+    assert gret.gret_prefill_backward_launches(4, 16, 4096, 128, 256, bf) == 5
+    want = 2 * (64 * 64 * E * 4) + 4 * 4096 * 16 * 256 * 4 + 64 * 64 * 4
+    assert gret.gret_prefill_backward_workspace_size(4, 16, 4096, 128, 256, bf) == want
+    nc = (100 + 31) // 32
+    assert gret.gret_prefill_backward_launches(1, 2, 100, 64, 64, f32) == 5
+    got = gret.gret_prefill_backward_workspace_size(1, 2, 100, 64, 64, f32)
+    assert got >= 2 * 2 * nc * 64 * 64 * 4 + 100 * 2 * 64 * 4 + 2 * nc * 4
+    # serial path: head sizes that are not multiples of 32, or dk above 128
+    for dk, dv in ((48, 80), (256, 64), (160, 64)):
+        assert gret.gret_prefill_backward_launches(1, 2, 100, dk, dv, bf) == 2
+        want = ((2 * 4 * dk * dv * 4 + 255) // 256) * 256 + 2 * dk * dv * 4
+        assert gret.gret_prefill_backward_workspace_size(1, 2, 100, dk, dv, bf) == want
+    # unsupported
+    assert gret.gret_prefill_backward_workspace_size(1, 2, 100, 24, 64, bf) == 0
+    assert gret.gret_prefill_backward_launches(1, 2, 100, 64, 64, 7) == 0

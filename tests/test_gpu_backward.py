@@ -2,9 +2,10 @@
 (autograd of the recurrent definition, itself pinned by finite differences).
 
 Cases: the fp32 path (1e-4 of max|ref|) with an initial state and a gradient
-on the final state, both epilogues, ragged block tails; bf16 inputs and
-gradients at the benchmark's head sizes (bf16 tolerance); a gate-stress mix of
-fast- and slow-decaying heads."""
+on the final state, both epilogues, ragged chunk tails; bf16 inputs and
+gradients at the benchmark's head sizes (bf16 tolerance) over one and several
+chunks; a gate-stress mix of fast- and slow-decaying heads; head sizes that are
+not multiples of 32 (the serial path)."""
 import numpy as np
 import pytest
 import torch
@@ -64,3 +65,23 @@ def test_bf16_benchmark_heads():
 
 def test_bf16_gate_stress():
     _run(gi.C2.scaled(B=1, H=2, N=160, dv=128, seed=74, z_dist=((-4.0, 1.0), (8.0, 0.5))))
+
+
+def test_bf16_several_chunks_ragged():
+    # five 64-token chunks, the last one 44 tokens long, both states given
+    cfg = gi.C2.scaled(B=2, H=1, N=300, seed=75)
+    assert gret.gret_prefill_backward_launches(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, gret.Dtype.BF16) == 5
+    _run(cfg)
+
+
+def test_fp32_prenorm_many_chunks():
+    _run(gi.C1.scaled(N=130, dk=32, dv=96, seed=76), epilogue="none")
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_serial_path_odd_head_sizes(io):
+    base = gi.C1 if io == "f32" else gi.C2
+    cfg = base.scaled(B=1, H=2, N=70, dk=48, dv=80, seed=77)
+    dt = gret.Dtype.F32 if io == "f32" else gret.Dtype.BF16
+    assert gret.gret_prefill_backward_launches(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, dt) == 2
+    _run(cfg)
