@@ -10,7 +10,10 @@ Inputs are seeded synthetic tensors already resident in HBM (546 MB, larger
 than the 126 MB L2, so no flush is needed between steps).
 
 The JSON line also carries the recurrent decode step (256 sequences x 16
-heads, 128 x 256 fp32 states, 64 consecutive launches) as ``decode``.
+heads, 128 x 256 fp32 states, 64 consecutive launches) as ``decode``; the same
+16384 tokens packed as a ragged batch of sequences (gret_prefill_varlen) as
+``varlen``; and the gradients of the benchmark prefill (gret_prefill_backward)
+as ``backward``.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -441,11 +444,17 @@ def backward_alg(cfg):
 
 
 def run_backward(args, world, dev, stream, d, O, cfg, peaks):
-    """gret_prefill_backward on the benchmark workload (CUDA-core kernels).
-    The upstream gradient dO is the forward's own output O (any tensor of O's
-    shape and dtype serves; the cost does not depend on its values)."""
+    """gret_prefill_backward on the benchmark workload (CUDA-core kernels), or
+    on its first --backward-batch sequences.  The upstream gradient dO is the
+    forward's own output O (any tensor of O's shape and dtype serves; the cost
+    does not depend on its values)."""
     import torch
     import gated_retention_sequence_b200 as gret
+    if args.backward_batch and args.backward_batch < cfg.B:
+        nb = args.backward_batch
+        cfg = cfg.scaled(B=nb, name=f"{cfg.name} (first {nb} sequences)")
+        d = {k: v[:nb] for k, v in d.items()}
+        O = O[:nb]
     steps = max(1, min(args.steps, 5))
     dO = O.clone()
     io = gret.Dtype.BF16
@@ -528,6 +537,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-varlen", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--backward-batch", type=int, default=0,
+                    help="run the backward sub-measurement on this many of the batch's sequences")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()

@@ -85,3 +85,15 @@ def test_serial_path_odd_head_sizes(io):
     dt = gret.Dtype.F32 if io == "f32" else gret.Dtype.BF16
     assert gret.gret_prefill_backward_launches(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, dt) == 2
     _run(cfg)
+
+
+def test_bf16_tensor_core_path_prenorm():
+    # d_k 128 bf16 takes the mma.sync kernels; the plain epilogue (dy = dO)
+    _run(gi.C2.scaled(B=1, H=2, N=200, seed=78), epilogue="none")
+
+
+def test_bf16_cuda_core_chunked_path():
+    # bf16 with d_k 64: the CUDA-core chunk kernels (chunks of 64 tokens)
+    cfg = gi.C2.scaled(B=1, H=2, N=150, dk=64, dv=128, seed=79)
+    assert gret.gret_prefill_backward_launches(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, gret.Dtype.BF16) == 5
+    _run(cfg)
