@@ -131,11 +131,11 @@ __device__ __forceinline__ void chunk_gate(const float* z, size_t zstride, int L
 
 // rows 0..rows-1 of a tile with `cols` elements per row (a multiple of 16 bytes):
 // row r < L from src + r * rstride, zeros after; dst row pitch P elements.
-template <typename T>
+template <typename T, int NTH = kCT>
 __device__ __forceinline__ void stage_rows(T* dst, int P, const T* src, size_t rstride, int L, int rows, int cols) {
     constexpr int VE = 16 / sizeof(T);
     const int vpr = cols / VE;
-    for (int e = threadIdx.x; e < rows * vpr; e += kCT) {
+    for (int e = threadIdx.x; e < rows * vpr; e += NTH) {
         const int r = e / vpr, cv = e - r * vpr;
         uint4 w = make_uint4(0u, 0u, 0u, 0u);
         if (r < L) w = __ldg(reinterpret_cast<const uint4*>(src + (size_t)r * rstride) + cv);
@@ -148,10 +148,10 @@ __device__ __forceinline__ void stage_rows(T* dst, int P, const T* src, size_t r
 }
 
 // the same into an fp32 tile, converting element by element
-template <typename T>
+template <typename T, int NTH = kCT>
 __device__ __forceinline__ void stage_rows_f32(float* dst, int P, const T* src, size_t rstride, int L, int rows,
                                                int cols) {
-    for (int e = threadIdx.x; e < rows * cols; e += kCT) {
+    for (int e = threadIdx.x; e < rows * cols; e += NTH) {
         const int r = e / cols, cc = e - r * cols;
         dst[(size_t)r * P + cc] = r < L ? to_f32(src[(size_t)r * rstride + cc]) : 0.f;
     }
@@ -851,6 +851,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi) {
     return *reinterpret_cast<const uint32_t*>(&v);
 }
 
+constexpr int kCTm = 512;   // threads per block of the tensor-core kernels (16 warps)
+
 struct IncMmaLayout {
     size_t k, v, total;
     int pk, pv;
@@ -864,14 +866,15 @@ struct IncMmaLayout {
     }
 };
 
-// ---- 1 (tensor cores): e^{b_L} and sum_s k_s^T (e^{b_L - b_s} v_s) into slot c + 1
+// ---- 1 (tensor cores): e^{b_L} and sum_s k_s^T (e^{b_L - b_s} v_s) into slot
+// c + 1.  Warp w owns rows 16 (w % 8) .. + 15 of d_k and the column half w / 8.
 template <int DV>
-__global__ void __launch_bounds__(kCT) bwd_inc_mma_kernel(ChunkArgs a) {
-    constexpr int C = kCm;
+__global__ void __launch_bounds__(kCTm, 1) bwd_inc_mma_kernel(ChunkArgs a) {
+    constexpr int C = kCm, NT = DV / 16;
     extern __shared__ __align__(16) unsigned char smraw[];
     const int H = a.H, N = a.N, nc = a.nc;
     const int u = blockIdx.x / nc, c = blockIdx.x - u * nc, b = u / H, h = u - b * H;
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, mi = warp & 7, nh = warp >> 3;
     const int n0 = c * C, L = min(C, N - n0);
     const size_t tok0 = (size_t)b * N + n0;
     const IncMmaLayout lay(DV);
@@ -886,23 +889,21 @@ __global__ void __launch_bounds__(kCT) bwd_inc_mma_kernel(ChunkArgs a) {
     if (tid == 0) a.decay[(size_t)u * nc + c] = expf(bL);
     if (c == nc - 1) return;
     if (tid < C) wl[tid] = tid < L ? expf(bL - bc[tid]) : 0.f;
-    stage_rows(Ks, lay.pk, static_cast<const __nv_bfloat16*>(a.K) + (tok0 * H + h) * kDKm, (size_t)H * kDKm, L, C,
-               kDKm);
+    stage_rows<__nv_bfloat16, kCTm>(Ks, lay.pk, static_cast<const __nv_bfloat16*>(a.K) + (tok0 * H + h) * kDKm,
+                                    (size_t)H * kDKm, L, C, kDKm);
     __syncthreads();
     const __nv_bfloat16* Vg = static_cast<const __nv_bfloat16*>(a.V) + (tok0 * H + h) * DV;
-    for (int e = tid; e < C * DV; e += kCT) {
+    for (int e = tid; e < C * DV; e += kCTm) {
         const int s = e / DV, j = e - s * DV;
         Vw[s * lay.pv + j] = s < L ? wl[s] * __bfloat162float(Vg[(size_t)s * H * DV + j]) : 0.f;
     }
     __syncthreads();
     float* out = a.Sst + ((size_t)u * nc + c + 1) * (size_t)kDKm * DV;
-    for (int j0 = 0; j0 < DV; j0 += 128) {
-        float acc[16][4];
-        frag_zero(acc);
-        // rows i = 16 warp .. 16 warp + 15: A(i, s) = K[s][i], B(s, j) = wl[s] V[s][j]
-        warp_mma<16, false, true>(acc, Ks + 16 * warp, 1, lay.pk, Vw + j0, lay.pv, 1, C);
-        frag_store(acc, out + (size_t)(16 * warp) * DV + j0, DV);
-    }
+    float acc[NT][4];
+    frag_zero(acc);
+    // A(i, s) = K[s][i], B(s, j) = wl[s] V[s][j]
+    warp_mma<NT, false, true>(acc, Ks + 16 * mi, 1, lay.pk, Vw + nh * (DV / 2), lay.pv, 1, C);
+    frag_store(acc, out + (size_t)(16 * mi) * DV + nh * (DV / 2), DV);
 }
 
 struct DyMmaLayout {
@@ -920,7 +921,7 @@ struct DyMmaLayout {
         v = o; o = al16(o + (size_t)kCm * pv * 2);
         dy = o; o = al16(o + (size_t)kCm * py * 4);
         sl = o; o = al16(o + (size_t)2 * kSW * ps * 4);
-        part = o; o = al16(o + (size_t)4 * kCm * 4);
+        part = o; o = al16(o + (size_t)8 * kCm * 4);
         total = o;
     }
 };
@@ -932,68 +933,87 @@ __device__ __forceinline__ float quad_sum(float v) {
     return v;
 }
 
+// Sum over the four column-quarter warps of a row: each quad writes its partial
+// to part[quarter][row]; after the barrier every lane reads the four.
+__device__ __forceinline__ float rows_total(const float* part, int t) {
+    return part[t] + part[kCm + t] + part[2 * kCm + t] + part[3 * kCm + t];
+}
+
 // ---- 3 (tensor cores): y, the GroupNorm * swish backward, G_c.  Warp w owns
-// rows 16 (w % 4) .. + 15 and the column half w / 4 of every C x C and C x d_v
-// product; G_c (d_k x d_v) is cut into 16-row slices, one per warp.
+// rows 16 (w % 4) .. + 15 and the column quarter w / 4 of the C x C and C x d_v
+// products; G_c (d_k x d_v) is cut into 16-row slices and column halves.
 template <int DV>
-__global__ void __launch_bounds__(kCT, 1) bwd_dy_mma_kernel(ChunkArgs a) {
-    constexpr int C = kCm, PA = C + 4, NT = DV / 16, HALF = DV / 2;
+__global__ void __launch_bounds__(kCTm, 1) bwd_dy_mma_kernel(ChunkArgs a) {
+    constexpr int C = kCm, PA = C + 4, NTQ = DV / 32, QUART = DV / 4;
     extern __shared__ __align__(16) unsigned char smraw[];
     const int H = a.H, N = a.N, nc = a.nc;
     const int u = blockIdx.x / nc, c = blockIdx.x - u * nc, b = u / H, h = u - b * H;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int g = lane >> 2, q = lane & 3, mb = warp & 3, nh = warp >> 2;
+    const int g = lane >> 2, q = lane & 3, mb = warp & 3, nq = warp >> 2;
     const int n0 = c * C, L = min(C, N - n0);
     const size_t tok0 = (size_t)b * N + n0;
     const DyMmaLayout lay(DV);
     const int pq = lay.pq, pv = lay.pv, py = lay.py, ps = lay.ps;
+    using bf = __nv_bfloat16;
     float* lg = reinterpret_cast<float*>(smraw);
     float* bc = lg + C;
     float* eb = bc + C;
     float* wsum = eb + C;
-    __nv_bfloat16* Qs = reinterpret_cast<__nv_bfloat16*>(smraw + lay.q);
-    __nv_bfloat16* Ks = reinterpret_cast<__nv_bfloat16*>(smraw + lay.k);
+    bf* Qs = reinterpret_cast<bf*>(smraw + lay.q);
+    bf* Ks = reinterpret_cast<bf*>(smraw + lay.k);
     float* As = reinterpret_cast<float*>(smraw + lay.a);
-    __nv_bfloat16* Vs = reinterpret_cast<__nv_bfloat16*>(smraw + lay.v);
+    bf* Vs = reinterpret_cast<bf*>(smraw + lay.v);
     float* dYs = reinterpret_cast<float*>(smraw + lay.dy);
     float* Sl = reinterpret_cast<float*>(smraw + lay.sl);
-    float* part = reinterpret_cast<float*>(smraw + lay.part);   // [4][C] row partial sums
+    float* part = reinterpret_cast<float*>(smraw + lay.part);   // [8][C] row partial sums
     const size_t qoff = (tok0 * H + h) * (size_t)kDKm, voff = (tok0 * H + h) * (size_t)DV;
-    using bf = __nv_bfloat16;
 
     chunk_gate<C>(a.z + tok0 * H + h, (size_t)H, L, a.inv_tau, lg, bc, wsum);
     if (tid < C) eb[tid] = tid < L ? expf(bc[tid]) : 0.f;
-    stage_rows(Qs, pq, static_cast<const bf*>(a.Q) + qoff, (size_t)H * kDKm, L, C, kDKm);
+    stage_rows<bf, kCTm>(Qs, pq, static_cast<const bf*>(a.Q) + qoff, (size_t)H * kDKm, L, C, kDKm);
     if (a.gn) {
-        stage_rows(Ks, pq, static_cast<const bf*>(a.K) + qoff, (size_t)H * kDKm, L, C, kDKm);
-        stage_rows(Vs, pv, static_cast<const bf*>(a.V) + voff, (size_t)H * DV, L, C, DV);
+        stage_rows<bf, kCTm>(Ks, pq, static_cast<const bf*>(a.K) + qoff, (size_t)H * kDKm, L, C, kDKm);
+        stage_rows<bf, kCTm>(Vs, pv, static_cast<const bf*>(a.V) + voff, (size_t)H * DV, L, C, DV);
     } else {
-        stage_rows_f32(dYs, py, static_cast<const bf*>(a.dO) + voff, (size_t)H * DV, L, C, DV);
+        stage_rows_f32<bf, kCTm>(dYs, py, static_cast<const bf*>(a.dO) + voff, (size_t)H * DV, L, C, DV);
     }
     __syncthreads();
 
     const int t0 = 16 * mb + g, t1 = t0 + 8;   // the two fragment rows of this lane
     if (a.gn) {
+        // G and dO of this lane's fragment elements, fetched now and used after the products
+        const bf* Gg = static_cast<const bf*>(a.G) + voff;
+        const bf* dOg = static_cast<const bf*>(a.dO) + voff;
+        uint32_t gpre[NTQ][2], opre[NTQ][2];
+#pragma unroll
+        for (int nt = 0; nt < NTQ; ++nt)
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                const int t = hf ? t1 : t0;
+                const size_t o = (size_t)t * H * DV + nq * QUART + 8 * nt + 2 * q;
+                gpre[nt][hf] = t < L ? *reinterpret_cast<const uint32_t*>(Gg + o) : 0u;
+                opre[nt][hf] = t < L ? *reinterpret_cast<const uint32_t*>(dOg + o) : 0u;
+            }
         // A = (Q K^T) o e^{b_t - b_s} on s <= t
         {
-            float acc[4][4];
+            float acc[2][4];
             frag_zero(acc);
-            warp_mma<4, false, false>(acc, Qs + 16 * mb * pq, pq, 1, Ks + 32 * nh * pq, 1, pq, kDKm);
+            warp_mma<2, false, false>(acc, Qs + 16 * mb * pq, pq, 1, Ks + 16 * nq * pq, 1, pq, kDKm);
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
+            for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const int t = e < 2 ? t0 : t1, s = 32 * nh + 8 * nt + 2 * q + (e & 1);
+                    const int t = e < 2 ? t0 : t1, s = 16 * nq + 8 * nt + 2 * q + (e & 1);
                     As[t * PA + s] = s <= t ? acc[nt][e] * expf(bc[t] - bc[s]) : 0.f;
                 }
         }
-        // y = e^{b_t} Q S_c + A V over this warp's rows and column half; S_c
-        // streams through shared memory in 32-row slabs (async copies, two buffers)
-        float y[NT][4];
+        // y = e^{b_t} Q S_c + A V; S_c streams through shared memory in 32-row
+        // slabs (async copies, two buffers)
+        float y[NTQ][4];
         frag_zero(y);
         const float* S = a.Sst + ((size_t)u * nc + c) * (size_t)kDKm * DV;
         constexpr int NSL = kDKm / kSW, VPR = DV / 4;
-        for (int e = tid; e < kSW * VPR; e += kCT) {
+        for (int e = tid; e < kSW * VPR; e += kCTm) {
             const int r = e / VPR, v = e - r * VPR;
             cp_async16(Sl + r * ps + 4 * v, S + (size_t)r * DV + 4 * v);
         }
@@ -1002,7 +1022,7 @@ __global__ void __launch_bounds__(kCT, 1) bwd_dy_mma_kernel(ChunkArgs a) {
             if (sl + 1 < NSL) {
                 const float* src = S + (size_t)(sl + 1) * kSW * DV;
                 float* dst = Sl + (size_t)((sl + 1) & 1) * kSW * ps;
-                for (int e = tid; e < kSW * VPR; e += kCT) {
+                for (int e = tid; e < kSW * VPR; e += kCTm) {
                     const int r = e / VPR, v = e - r * VPR;
                     cp_async16(dst + r * ps + 4 * v, src + (size_t)r * DV + 4 * v);
                 }
@@ -1013,42 +1033,42 @@ __global__ void __launch_bounds__(kCT, 1) bwd_dy_mma_kernel(ChunkArgs a) {
             }
             __syncthreads();
             const float* Sb = Sl + (size_t)(sl & 1) * kSW * ps;
-            warp_mma<NT, false, true>(y, Qs + 16 * mb * pq + sl * kSW, pq, 1, Sb + nh * HALF, ps, 1, kSW);
+            warp_mma<NTQ, false, true>(y, Qs + 16 * mb * pq + sl * kSW, pq, 1, Sb + nq * QUART, ps, 1, kSW);
             __syncthreads();   // this buffer is refilled two slabs on
         }
         {
             const float e0 = eb[t0], e1 = eb[t1];
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
+            for (int nt = 0; nt < NTQ; ++nt) {
                 y[nt][0] *= e0;
                 y[nt][1] *= e0;
                 y[nt][2] *= e1;
                 y[nt][3] *= e1;
             }
         }
-        warp_mma<NT, true, false>(y, As + 16 * mb * PA, PA, 1, Vs + nh * HALF, pv, 1, C);
+        warp_mma<NTQ, true, false>(y, As + 16 * mb * PA, PA, 1, Vs + nq * QUART, pv, 1, C);
 
         // GroupNorm (biased variance, no affine) * swish(G) backward.  A row's
-        // d_v values sit in the 4 lanes of a group in each of two warps: sums
+        // d_v values sit in the 4 lanes of a group in each of four warps: sums
         // go through the quad, then through `part`.
         const float inv_dv = 1.0f / (float)DV;
         float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
+        for (int nt = 0; nt < NTQ; ++nt) {
             s0 += y[nt][0] + y[nt][1];
             s1 += y[nt][2] + y[nt][3];
         }
         s0 = quad_sum(s0);
         s1 = quad_sum(s1);
         if (q == 0) {
-            part[nh * C + t0] = s0;
-            part[nh * C + t1] = s1;
+            part[nq * C + t0] = s0;
+            part[nq * C + t1] = s1;
         }
         __syncthreads();
-        const float mean0 = (part[t0] + part[C + t0]) * inv_dv, mean1 = (part[t1] + part[C + t1]) * inv_dv;
+        const float mean0 = rows_total(part, t0) * inv_dv, mean1 = rows_total(part, t1) * inv_dv;
         float v0 = 0.f, v1 = 0.f;
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
+        for (int nt = 0; nt < NTQ; ++nt) {
             float d = y[nt][0] - mean0;
             v0 = fmaf(d, d, v0);
             d = y[nt][1] - mean0;
@@ -1061,30 +1081,26 @@ __global__ void __launch_bounds__(kCT, 1) bwd_dy_mma_kernel(ChunkArgs a) {
         v0 = quad_sum(v0);
         v1 = quad_sum(v1);
         if (q == 0) {
-            part[2 * C + nh * C + t0] = v0;
-            part[2 * C + nh * C + t1] = v1;
+            part[4 * C + nq * C + t0] = v0;
+            part[4 * C + nq * C + t1] = v1;
         }
         __syncthreads();
-        const float rstd0 = rsqrtf((part[2 * C + t0] + part[3 * C + t0]) * inv_dv + a.eps);
-        const float rstd1 = rsqrtf((part[2 * C + t1] + part[3 * C + t1]) * inv_dv + a.eps);
+        const float rstd0 = rsqrtf(rows_total(part + 4 * C, t0) * inv_dv + a.eps);
+        const float rstd1 = rsqrtf(rows_total(part + 4 * C, t1) * inv_dv + a.eps);
         __syncthreads();   // every lane has read `part`; it is reused below
-        const bf* Gg = static_cast<const bf*>(a.G) + voff;
-        const bf* dOg = static_cast<const bf*>(a.dO) + voff;
         bf* dGg = static_cast<bf*>(a.dG) + voff;
         float m10 = 0.f, m11 = 0.f, m20 = 0.f, m21 = 0.f;
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
+        for (int nt = 0; nt < NTQ; ++nt)
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
-                const int t = hf ? t1 : t0, j = nh * HALF + 8 * nt + 2 * q;
+                const int t = hf ? t1 : t0, j = nq * QUART + 8 * nt + 2 * q;
                 const float mean = hf ? mean1 : mean0, rstd = hf ? rstd1 : rstd0;
                 float dn[2] = {0.f, 0.f}, nn[2] = {0.f, 0.f};
                 if (t < L) {
-                    const size_t o = (size_t)t * H * DV + j;
-                    const __nv_bfloat162 g2 = *reinterpret_cast<const __nv_bfloat162*>(Gg + o);
-                    const __nv_bfloat162 d2 = *reinterpret_cast<const __nv_bfloat162*>(dOg + o);
-                    const float gv[2] = {__low2float(g2), __high2float(g2)};
-                    const float gov[2] = {__low2float(d2), __high2float(d2)};
+                    const uint32_t gw = gpre[nt][hf], ow = opre[nt][hf];
+                    const float gv[2] = {__uint_as_float(gw << 16), __uint_as_float(gw & 0xffff0000u)};
+                    const float gov[2] = {__uint_as_float(ow << 16), __uint_as_float(ow & 0xffff0000u)};
                     float dg[2];
 #pragma unroll
                     for (int k = 0; k < 2; ++k) {
@@ -1094,7 +1110,7 @@ __global__ void __launch_bounds__(kCT, 1) bwd_dy_mma_kernel(ChunkArgs a) {
                         dg[k] = gov[k] * nn[k] * sg * (1.f + gv[k] * (1.f - sg));
                         dn[k] = gov[k] * gv[k] * sg;
                     }
-                    *reinterpret_cast<uint32_t*>(dGg + o) = pack_bf16x2_rn(dg[0], dg[1]);
+                    *reinterpret_cast<uint32_t*>(dGg + (size_t)t * H * DV + j) = pack_bf16x2_rn(dg[0], dg[1]);
                 }
                 *reinterpret_cast<float2*>(dYs + t * py + j) = make_float2(dn[0], dn[1]);
                 y[nt][2 * hf] = nn[0];
@@ -1112,21 +1128,20 @@ __global__ void __launch_bounds__(kCT, 1) bwd_dy_mma_kernel(ChunkArgs a) {
         m20 = quad_sum(m20);
         m21 = quad_sum(m21);
         if (q == 0) {
-            part[nh * C + t0] = m10;
-            part[nh * C + t1] = m11;
-            part[2 * C + nh * C + t0] = m20;
-            part[2 * C + nh * C + t1] = m21;
+            part[nq * C + t0] = m10;
+            part[nq * C + t1] = m11;
+            part[4 * C + nq * C + t0] = m20;
+            part[4 * C + nq * C + t1] = m21;
         }
         __syncthreads();
-        const float m1a = (part[t0] + part[C + t0]) * inv_dv, m1b = (part[t1] + part[C + t1]) * inv_dv;
-        const float m2a = (part[2 * C + t0] + part[3 * C + t0]) * inv_dv;
-        const float m2b = (part[2 * C + t1] + part[3 * C + t1]) * inv_dv;
+        const float m1a = rows_total(part, t0) * inv_dv, m1b = rows_total(part, t1) * inv_dv;
+        const float m2a = rows_total(part + 4 * C, t0) * inv_dv, m2b = rows_total(part + 4 * C, t1) * inv_dv;
         float* dyw = a.dyw + voff;
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
+        for (int nt = 0; nt < NTQ; ++nt)
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
-                const int t = hf ? t1 : t0, j = nh * HALF + 8 * nt + 2 * q;
+                const int t = hf ? t1 : t0, j = nq * QUART + 8 * nt + 2 * q;
                 if (t < L) {
                     const float rstd = hf ? rstd1 : rstd0, m1 = hf ? m1b : m1a, m2 = hf ? m2b : m2a;
                     const float2 dn = *reinterpret_cast<const float2*>(dYs + t * py + j);
@@ -1138,18 +1153,21 @@ __global__ void __launch_bounds__(kCT, 1) bwd_dy_mma_kernel(ChunkArgs a) {
             }
         __syncthreads();
     }
-    // G_c = sum_t q_t^T (e^{b_t} dy_t): scale the dy rows, then 16 rows of d_k per warp
-    for (int e = tid; e < C * DV; e += kCT) {
+    // G_c = sum_t q_t^T (e^{b_t} dy_t): scale the dy rows, then warp w takes
+    // rows 16 (w % 8) .. + 15 of d_k and the column half w / 8
+    for (int e = tid; e < C * DV; e += kCTm) {
         const int t = e / DV, j = e - t * DV;
         dYs[t * py + j] *= eb[t];
     }
     __syncthreads();
     float* Gc = a.dSt + ((size_t)u * nc + c) * (size_t)kDKm * DV;
-    for (int j0 = 0; j0 < DV; j0 += 128) {
-        float acc[16][4];
+    {
+        constexpr int NT = DV / 16;
+        const int mi = warp & 7, nh = warp >> 3;
+        float acc[NT][4];
         frag_zero(acc);
-        warp_mma<16, false, true>(acc, Qs + 16 * warp, 1, pq, dYs + j0, py, 1, C);
-        frag_store(acc, Gc + (size_t)(16 * warp) * DV + j0, DV);
+        warp_mma<NT, false, true>(acc, Qs + 16 * mi, 1, pq, dYs + nh * (DV / 2), py, 1, C);
+        frag_store(acc, Gc + (size_t)(16 * mi) * DV + nh * (DV / 2), DV);
     }
 }
 
@@ -1160,7 +1178,7 @@ struct GradMmaLayout {
         pq = kDKm + 4;
         pv = dv + 4;
         py = dv + 4;
-        size_t o = al16(sizeof(float) * (8 * kCm + 16));
+        size_t o = al16(sizeof(float) * (8 * kCm + 32));
         q = o; o = al16(o + (size_t)kCm * pq * 2);
         k = o; o = al16(o + (size_t)kCm * pq * 2);
         v = o; o = al16(o + (size_t)kCm * pv * 2);
@@ -1169,30 +1187,39 @@ struct GradMmaLayout {
         d = o; o = al16(o + (size_t)kCm * (kCm + 4) * 4);
         const size_t slabs = (size_t)2 * kDKm * (kSW + 4) * 4, scratch = (size_t)kCm * (kCm + 4) * 4;
         sl = o; o = al16(o + (slabs > scratch ? slabs : scratch));
-        part = o; o = al16(o + (size_t)4 * kCm * 4);
+        part = o; o = al16(o + (size_t)8 * kCm * 4);
         total = o;
     }
 };
 
-// 32-column state slab into shared memory with row pitch kSW + 4 (16-byte rows)
-__device__ __forceinline__ void slab_store16(float* dst, const uint4 (&pre)[4]) {
+// 32-column state slab (rows i < d_k = 128, columns j0 .. j0 + 31 of a [128][dv]
+// fp32 state): 1024 16-byte vectors, two per thread of a 512-thread block, held
+// in registers between the global load and the shared store (row pitch kSW + 4)
+__device__ __forceinline__ void slab_load_m(const float* src, int dv, int j0, uint4 (&pre)[2]) {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const int e = threadIdx.x + q * kCT;   // kDKm * 8 = 4 * kCT vectors
-        *reinterpret_cast<uint4*>(dst + (e >> 3) * (kSW + 4) + 4 * (e & 7)) = pre[q];
+    for (int k = 0; k < 2; ++k) {
+        const int e = threadIdx.x + k * kCTm;
+        pre[k] = *reinterpret_cast<const uint4*>(src + (size_t)(e >> 3) * dv + j0 + 4 * (e & 7));
+    }
+}
+__device__ __forceinline__ void slab_store_m(float* dst, const uint4 (&pre)[2]) {
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const int e = threadIdx.x + k * kCTm;
+        *reinterpret_cast<uint4*>(dst + (e >> 3) * (kSW + 4) + 4 * (e & 7)) = pre[k];
     }
 }
 
 // ---- 5 (tensor cores): dq, dk, dv, dz.  Warp w owns rows 16 (w % 4) .. + 15
-// and the column half w / 4 of each product.
+// and the column quarter w / 4 of each product.
 template <int DV>
-__global__ void __launch_bounds__(kCT, 1) bwd_grad_mma_kernel(ChunkArgs a) {
-    constexpr int C = kCm, PA = C + 4, PS = kSW + 4, NS = DV / kSW;
+__global__ void __launch_bounds__(kCTm, 1) bwd_grad_mma_kernel(ChunkArgs a) {
+    constexpr int C = kCm, PA = C + 4, PS = kSW + 4, NS = DV / kSW, NW = kCTm / 32;
     extern __shared__ __align__(16) unsigned char smraw[];
     const int H = a.H, N = a.N, nc = a.nc;
     const int u = blockIdx.x / nc, c = blockIdx.x - u * nc, b = u / H, h = u - b * H;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int g = lane >> 2, q = lane & 3, mb = warp & 3, nh = warp >> 2;
+    const int g = lane >> 2, q = lane & 3, mb = warp & 3, nq = warp >> 2;
     const int n0 = c * C, L = min(C, N - n0);
     const size_t tok0 = (size_t)b * N + n0;
     const GradMmaLayout lay(DV);
@@ -1206,7 +1233,7 @@ __global__ void __launch_bounds__(kCT, 1) bwd_grad_mma_kernel(ChunkArgs a) {
     float* us = rr + C;        // e^{b_L - b_s} k_s . (dS' v_s)
     float* Fj = us + C;        // sum_{t>=j, s<j} A_ts D_ts
     float* wsum = Fj + 2 * C;
-    float* red = wsum + 4;
+    float* red = wsum + 4;     // [NW]
     bf* Qs = reinterpret_cast<bf*>(smraw + lay.q);
     bf* Ks = reinterpret_cast<bf*>(smraw + lay.k);
     bf* Vs = reinterpret_cast<bf*>(smraw + lay.v);
@@ -1227,38 +1254,38 @@ __global__ void __launch_bounds__(kCT, 1) bwd_grad_mma_kernel(ChunkArgs a) {
         eb[tid] = tid < L ? expf(bc[tid]) : 0.f;
         wl[tid] = tid < L ? expf(bL - bc[tid]) : 0.f;
     }
-    stage_rows(Qs, pq, static_cast<const bf*>(a.Q) + qoff, (size_t)H * kDKm, L, C, kDKm);
-    stage_rows(Ks, pq, static_cast<const bf*>(a.K) + qoff, (size_t)H * kDKm, L, C, kDKm);
-    stage_rows(Vs, pv, static_cast<const bf*>(a.V) + voff, (size_t)H * DV, L, C, DV);
+    stage_rows<bf, kCTm>(Qs, pq, static_cast<const bf*>(a.Q) + qoff, (size_t)H * kDKm, L, C, kDKm);
+    stage_rows<bf, kCTm>(Ks, pq, static_cast<const bf*>(a.K) + qoff, (size_t)H * kDKm, L, C, kDKm);
+    stage_rows<bf, kCTm>(Vs, pv, static_cast<const bf*>(a.V) + voff, (size_t)H * DV, L, C, DV);
     if (a.gn)
-        stage_rows_f32(dYs, py, static_cast<const float*>(a.dyw) + voff, (size_t)H * DV, L, C, DV);
+        stage_rows_f32<float, kCTm>(dYs, py, static_cast<const float*>(a.dyw) + voff, (size_t)H * DV, L, C, DV);
     else
-        stage_rows_f32(dYs, py, static_cast<const bf*>(a.dO) + voff, (size_t)H * DV, L, C, DV);
+        stage_rows_f32<bf, kCTm>(dYs, py, static_cast<const bf*>(a.dO) + voff, (size_t)H * DV, L, C, DV);
     __syncthreads();
 
     // A = (Q K^T) o e^{b_t - b_s} on s <= t
     {
-        float acc[4][4];
+        float acc[2][4];
         frag_zero(acc);
-        warp_mma<4, false, false>(acc, Qs + 16 * mb * pq, pq, 1, Ks + 32 * nh * pq, 1, pq, kDKm);
+        warp_mma<2, false, false>(acc, Qs + 16 * mb * pq, pq, 1, Ks + 16 * nq * pq, 1, pq, kDKm);
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
+        for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const int t = e < 2 ? t0 : t1, s = 32 * nh + 8 * nt + 2 * q + (e & 1);
+                const int t = e < 2 ? t0 : t1, s = 16 * nq + 8 * nt + 2 * q + (e & 1);
                 As[t * PA + s] = s <= t ? acc[nt][e] * expf(bc[t] - bc[s]) : 0.f;
             }
     }
     // D = dy V^T on s <= t: Ds = D e^{b_t - b_s}; M = A o D into the slab scratch
     {
-        float acc[4][4];
+        float acc[2][4];
         frag_zero(acc);
-        warp_mma<4, true, false>(acc, dYs + 16 * mb * py, py, 1, Vs + 32 * nh * pv, 1, pv, DV);
+        warp_mma<2, true, false>(acc, dYs + 16 * mb * py, py, 1, Vs + 16 * nq * pv, 1, pv, DV);
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
+        for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const int t = e < 2 ? t0 : t1, s = 32 * nh + 8 * nt + 2 * q + (e & 1);
+                const int t = e < 2 ? t0 : t1, s = 16 * nq + 8 * nt + 2 * q + (e & 1);
                 const bool in = s <= t;
                 Ds[t * PA + s] = in ? acc[nt][e] * expf(bc[t] - bc[s]) : 0.f;
                 SL[t * PA + s] = in ? As[t * PA + s] * acc[nt][e] : 0.f;
@@ -1269,7 +1296,8 @@ __global__ void __launch_bounds__(kCT, 1) bwd_grad_mma_kernel(ChunkArgs a) {
         const float4* s4 = reinterpret_cast<const float4*>(S);
         const float4* d4 = reinterpret_cast<const float4*>(dSp);
         float acc = 0.f;
-        for (size_t e = tid; e < E / 4; e += kCT) {
+#pragma unroll 4
+        for (int e = tid; e < (int)(E / 4); e += kCTm) {
             const float4 x = s4[e], y = d4[e];
             acc = fmaf(x.x, y.x, acc);
             acc = fmaf(x.y, y.y, acc);
@@ -1298,66 +1326,62 @@ __global__ void __launch_bounds__(kCT, 1) bwd_grad_mma_kernel(ChunkArgs a) {
     }
     __syncthreads();
 
-    float accY[8][4], accW[8][4];   // dy S_c^T and V dS'^T: rows t0/t1, columns 64 nh + ...
+    float accY[4][4], accW[4][4];   // dy S_c^T and V dS'^T: rows t0/t1, columns 32 nq + ...
     frag_zero(accY);
     frag_zero(accW);
-    uint4 pre[4];
+    uint4 pre[2];
     // pass over S_c
-    slab_load(S, kDKm, DV, 0, pre);
-    slab_store16(SL, pre);
+    slab_load_m(S, DV, 0, pre);
+    slab_store_m(SL, pre);
     __syncthreads();
     for (int sl = 0; sl < NS; ++sl) {
         const float* cur = SL + (size_t)(sl & 1) * kDKm * PS;
-        if (sl + 1 < NS) slab_load(S, kDKm, DV, (sl + 1) * kSW, pre);
+        if (sl + 1 < NS) slab_load_m(S, DV, (sl + 1) * kSW, pre);
         // B(j, i) = S_c[i][j]
-        warp_mma<8, true, true>(accY, dYs + 16 * mb * py + sl * kSW, py, 1, cur + 64 * nh * PS, 1, PS, kSW);
-        if (sl + 1 < NS) slab_store16(SL + (size_t)((sl + 1) & 1) * kDKm * PS, pre);
+        warp_mma<4, true, true>(accY, dYs + 16 * mb * py + sl * kSW, py, 1, cur + 32 * nq * PS, 1, PS, kSW);
+        if (sl + 1 < NS) slab_store_m(SL + (size_t)((sl + 1) & 1) * kDKm * PS, pre);
         __syncthreads();
     }
     // pass over dS'_c: V dS'^T, and dv for the slab's 32 columns
     bf* dVg = static_cast<bf*>(a.dV) + voff;
-    slab_load(dSp, kDKm, DV, 0, pre);
-    slab_store16(SL, pre);
+    slab_load_m(dSp, DV, 0, pre);
+    slab_store_m(SL, pre);
     __syncthreads();
     for (int sl = 0; sl < NS; ++sl) {
         const float* cur = SL + (size_t)(sl & 1) * kDKm * PS;
-        if (sl + 1 < NS) slab_load(dSp, kDKm, DV, (sl + 1) * kSW, pre);
+        if (sl + 1 < NS) slab_load_m(dSp, DV, (sl + 1) * kSW, pre);
         const int j0 = sl * kSW;
-        warp_mma<8, false, true>(accW, Vs + 16 * mb * pv + j0, pv, 1, cur + 64 * nh * PS, 1, PS, kSW);
-        // dv_s = e^{b_L - b_s} (K dS')_s + sum_t A_ts dy_t over columns j0 + 16 nh .. + 15
-        float dva[2][4];
+        warp_mma<4, false, true>(accW, Vs + 16 * mb * pv + j0, pv, 1, cur + 32 * nq * PS, 1, PS, kSW);
+        // dv_s = e^{b_L - b_s} (K dS')_s + sum_t A_ts dy_t over columns j0 + 8 nq .. + 7
+        float dva[1][4];
         frag_zero(dva);
-        warp_mma<2, false, true>(dva, Ks + 16 * mb * pq, pq, 1, cur + 16 * nh, PS, 1, kDKm);
+        warp_mma<1, false, true>(dva, Ks + 16 * mb * pq, pq, 1, cur + 8 * nq, PS, 1, kDKm);
         {
             const float w0 = wl[t0], w1 = wl[t1];
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                dva[nt][0] *= w0;
-                dva[nt][1] *= w0;
-                dva[nt][2] *= w1;
-                dva[nt][3] *= w1;
-            }
+            dva[0][0] *= w0;
+            dva[0][1] *= w0;
+            dva[0][2] *= w1;
+            dva[0][3] *= w1;
         }
-        warp_mma<2, true, true>(dva, As + 16 * mb, 1, PA, dYs + j0 + 16 * nh, py, 1, C);
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            const int j = j0 + 16 * nh + 8 * nt + 2 * q;
+        warp_mma<1, true, true>(dva, As + 16 * mb, 1, PA, dYs + j0 + 8 * nq, py, 1, C);
+        {
+            const int j = j0 + 8 * nq + 2 * q;
             if (t0 < L)
-                *reinterpret_cast<uint32_t*>(dVg + (size_t)t0 * H * DV + j) = pack_bf16x2_rn(dva[nt][0], dva[nt][1]);
+                *reinterpret_cast<uint32_t*>(dVg + (size_t)t0 * H * DV + j) = pack_bf16x2_rn(dva[0][0], dva[0][1]);
             if (t1 < L)
-                *reinterpret_cast<uint32_t*>(dVg + (size_t)t1 * H * DV + j) = pack_bf16x2_rn(dva[nt][2], dva[nt][3]);
+                *reinterpret_cast<uint32_t*>(dVg + (size_t)t1 * H * DV + j) = pack_bf16x2_rn(dva[0][2], dva[0][3]);
         }
-        if (sl + 1 < NS) slab_store16(SL + (size_t)((sl + 1) & 1) * kDKm * PS, pre);
+        if (sl + 1 < NS) slab_store_m(SL + (size_t)((sl + 1) & 1) * kDKm * PS, pre);
         __syncthreads();
     }
 
-    // row dots q_t . (S dy_t) and k_s . (dS' v_s) (halves through `part`), then
+    // row dots q_t . (S dy_t) and k_s . (dS' v_s) (quarters through `part`), then
     // dq = Ds K + e^{b_t} dy S^T and dk = Ds^T Q + e^{b_L - b_s} V dS'^T
     {
         float r0 = 0.f, r1 = 0.f, u0 = 0.f, u1 = 0.f;
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-            const int i = 64 * nh + 8 * nt + 2 * q;
+        for (int nt = 0; nt < 4; ++nt) {
+            const int i = 32 * nq + 8 * nt + 2 * q;
             r0 += ldf(Qs + t0 * pq + i) * accY[nt][0] + ldf(Qs + t0 * pq + i + 1) * accY[nt][1];
             r1 += ldf(Qs + t1 * pq + i) * accY[nt][2] + ldf(Qs + t1 * pq + i + 1) * accY[nt][3];
             u0 += ldf(Ks + t0 * pq + i) * accW[nt][0] + ldf(Ks + t0 * pq + i + 1) * accW[nt][1];
@@ -1368,14 +1392,14 @@ __global__ void __launch_bounds__(kCT, 1) bwd_grad_mma_kernel(ChunkArgs a) {
         u0 = quad_sum(u0);
         u1 = quad_sum(u1);
         if (q == 0) {
-            part[nh * C + t0] = r0;
-            part[nh * C + t1] = r1;
-            part[2 * C + nh * C + t0] = u0;
-            part[2 * C + nh * C + t1] = u1;
+            part[nq * C + t0] = r0;
+            part[nq * C + t1] = r1;
+            part[4 * C + nq * C + t0] = u0;
+            part[4 * C + nq * C + t1] = u1;
         }
         const float e0 = eb[t0], e1 = eb[t1], w0 = wl[t0], w1 = wl[t1];
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
+        for (int nt = 0; nt < 4; ++nt) {
             accY[nt][0] *= e0;
             accY[nt][1] *= e0;
             accY[nt][2] *= e1;
@@ -1387,14 +1411,14 @@ __global__ void __launch_bounds__(kCT, 1) bwd_grad_mma_kernel(ChunkArgs a) {
         }
     }
     // dq: A(t, s) = Ds[t][s], B(s, i) = K[s][i];  dk: A(s, t) = Ds[t][s], B(t, i) = Q[t][i]
-    warp_mma<8, true, false>(accY, Ds + 16 * mb * PA, PA, 1, Ks + 64 * nh, pq, 1, C);
-    warp_mma<8, true, false>(accW, Ds + 16 * mb, 1, PA, Qs + 64 * nh, pq, 1, C);
+    warp_mma<4, true, false>(accY, Ds + 16 * mb * PA, PA, 1, Ks + 32 * nq, pq, 1, C);
+    warp_mma<4, true, false>(accW, Ds + 16 * mb, 1, PA, Qs + 32 * nq, pq, 1, C);
     {
         bf* dQg = static_cast<bf*>(a.dQ) + qoff;
         bf* dKg = static_cast<bf*>(a.dK) + qoff;
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-            const int i = 64 * nh + 8 * nt + 2 * q;
+        for (int nt = 0; nt < 4; ++nt) {
+            const int i = 32 * nq + 8 * nt + 2 * q;
             if (t0 < L) {
                 const size_t o = (size_t)t0 * H * kDKm + i;
                 *reinterpret_cast<uint32_t*>(dQg + o) = pack_bf16x2_rn(accY[nt][0], accY[nt][1]);
@@ -1409,15 +1433,15 @@ __global__ void __launch_bounds__(kCT, 1) bwd_grad_mma_kernel(ChunkArgs a) {
     }
     __syncthreads();
     if (tid < C) {
-        rr[tid] = eb[tid] * (part[tid] + part[C + tid]);
-        us[tid] = wl[tid] * (part[2 * C + tid] + part[3 * C + tid]);
+        rr[tid] = eb[tid] * rows_total(part, tid);
+        us[tid] = wl[tid] * rows_total(part + 4 * C, tid);
     }
     __syncthreads();
     // dz_j = dlg_j (1 - sigmoid(z_j)) / tau, zero where the forward clamps log gamma
     if (tid < L) {
         const int j = tid;
         float c0 = 0.f;
-        for (int w = 0; w < kCT / 32; ++w) c0 += red[w];
+        for (int w = 0; w < NW; ++w) c0 += red[w];
         float rs = 0.f, su = 0.f;
         for (int t = j; t < L; ++t) rs += rr[t];
         for (int s = 0; s < j; ++s) su += us[s];
@@ -1472,11 +1496,11 @@ static cudaError_t run_bwd_mma(const ChunkArgs& a, cudaStream_t s) {
     if ((e = cudaFuncSetAttribute(k3, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s3)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(k5, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s5)) != cudaSuccess) return e;
     const unsigned blocks = (unsigned)((size_t)a.B * a.H * a.nc);
-    k1<<<blocks, kCT, s1, s>>>(a);
+    k1<<<blocks, kCTm, s1, s>>>(a);
     bwd_fwd_scan_kernel<<<scan_blocks(a), kCT, 0, s>>>(a);
-    k3<<<blocks, kCT, s3, s>>>(a);
+    k3<<<blocks, kCTm, s3, s>>>(a);
     bwd_rev_scan_kernel<<<scan_blocks(a), kCT, 0, s>>>(a);
-    k5<<<blocks, kCT, s5, s>>>(a);
+    k5<<<blocks, kCTm, s5, s>>>(a);
     return cudaGetLastError();
 }
 
