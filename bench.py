@@ -443,9 +443,44 @@ def backward_alg(cfg):
     return cfg.B * cfg.N * cfg.H * (e * (4 * cfg.dk + 5 * cfg.dv) + 8)
 
 
+# chunk length of the backward (bf16 inputs); the flop count below depends on it
+BACKWARD_CHUNK = 64
+# tf32 / bf16 dense tensor peak (nominal 1.1 / 2.25 PFLOP/s per GPU)
+TF32_OVER_BF16 = 1.1 / 2.25
+
+
+def backward_alg_flops(cfg, chunk=BACKWARD_CHUNK):
+    """Algorithmic flops of one backward, per (token, head): six state-sized
+    products (the state increment, Q S, G_c, dy S^T, V dS'^T, K dS'), 2 dk dv
+    flops each, and the causal halves of the intra-chunk products (Q K^T twice,
+    A V, dy V^T, A^T dy, D K, D^T Q), chunk (4 dk + 3 dv) flops together."""
+    return cfg.B * cfg.N * cfg.H * (12 * cfg.dk * cfg.dv + chunk * (4 * cfg.dk + 3 * cfg.dv))
+
+
+def backward_summary(cfg, steps, ms, world, peaks, launches_per_call):
+    """The ``backward`` object of the JSON line for `steps` calls that took
+    `ms` (max over ranks) on each of `world` ranks."""
+    bytes_ = backward_alg(cfg)
+    flops = backward_alg_flops(cfg)
+    step_s = ms / 1e3 / steps
+    tflops = flops / step_s / 1e12
+    peak = peaks["bf16_tflops"] * TF32_OVER_BF16
+    return {"workload": cfg.name, "steps": steps, "warmup": 2, "ms_per_step": ms / steps,
+            "value": job_throughput(world, cfg.B * cfg.N, steps, ms) / 1e6, "unit": "Mtok/s",
+            "kernels": "bwd_inc_mma, bwd_fwd_scan, bwd_dy_mma, bwd_rev_scan, bwd_grad_mma "
+                       "(mma.sync m16n8k8 tf32 with split operands, fp32 accumulation)",
+            "roofline": {"kernel": "whole backward (5 launches)", "bound": "tensor", "achieved": tflops,
+                         "peak": peak, "unit": "TFLOP/s", "frac": tflops / peak, "traffic": None,
+                         "alg_flops_per_call": flops,
+                         "peak_source": peaks["source"] + " bf16 burst x nominal tf32/bf16 ratio"},
+            "path_hbm": {"alg_bytes": bytes_, "alg_gbs": bytes_ / step_s / 1e9,
+                         "frac": bytes_ / step_s / 1e9 / peaks["hbm_gbs"]},
+            "gpu_launches": launches_per_call * steps}
+
+
 def run_backward(args, world, dev, stream, d, O, cfg, peaks):
-    """gret_prefill_backward on the benchmark workload (CUDA-core kernels), or
-    on its first --backward-batch sequences.  The upstream gradient dO is the
+    """gret_prefill_backward on the benchmark workload, or on its first
+    --backward-batch sequences.  The upstream gradient dO is the
     forward's own output O (any tensor of O's shape and dtype serves; the cost
     does not depend on its values)."""
     import torch
@@ -477,15 +512,8 @@ def run_backward(args, world, dev, stream, d, O, cfg, peaks):
     barrier(world)
     gret.check_device_status()
     ms = max_over_ranks(e0.elapsed_time(e1), world)
-    bytes_ = backward_alg(cfg)
-    step_s = ms / 1e3 / steps
-    tokens = cfg.B * cfg.N
-    return {"workload": cfg.name, "steps": steps, "warmup": 2, "ms_per_step": ms / steps,
-            "value": job_throughput(world, tokens, steps, ms) / 1e6, "unit": "Mtok/s",
-            "kernels": "bwd_inc, bwd_fwd_scan, bwd_dy, bwd_rev_scan, bwd_grad (CUDA cores, fp32 arithmetic)",
-            "path_hbm": {"alg_bytes": bytes_, "alg_gbs": bytes_ / step_s / 1e9,
-                         "frac": bytes_ / step_s / 1e9 / peaks["hbm_gbs"]},
-            "gpu_launches": gret.gret_prefill_backward_launches(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, io) * steps}
+    return backward_summary(cfg, steps, ms, world, peaks,
+                            gret.gret_prefill_backward_launches(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, io))
 
 
 def run_decode(args, world, dev, stream, peaks):
