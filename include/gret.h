@@ -181,11 +181,15 @@ gret_status gret_state_fold(const float* dS_all, const float* decay_all, int num
  * of <O, dO> + <S_final, dS_final> with respect to Q, K, V (io dtype, their
  * layouts), the gate logits dz (fp32 [B][N][H]), G (io dtype; GN_SWISH only)
  * and the initial state dS0 (fp32 [B][H][dk][dv]; may be NULL).  S0 and
- * dS_final may be NULL (zero).  Arithmetic is fp32 on CUDA cores.
+ * dS_final may be NULL (zero).  Accumulation is fp32 throughout.
  *
  * Head sizes that are multiples of 32 with dk <= 128 and dv <= 256 take the
- * chunk-parallel path (5 launches; chunks of 64 tokens for bf16, 32 for fp32):
- * the workspace holds the state before every chunk and the gradient at every
+ * chunk-parallel path (5 launches; chunks of 64 tokens for bf16, 32 for fp32).
+ * With bf16 inputs, dk = 128 and dv = 128 or 256 its products run on the
+ * tensor cores (mma.sync tf32; every operand that is not a bf16 input is split
+ * into two tf32 parts, which keeps the products at fp32-level accuracy);
+ * otherwise on CUDA cores in fp32.
+ * The workspace holds the state before every chunk and the gradient at every
  * chunk's end (2 * B*H*ceil(N/chunk)*dk*dv*4 bytes), the gradient of the
  * pre-norm output (B*N*H*dv*4) and one decay per chunk.  Other head sizes
  * (multiples of 16 up to 256) take a serial path (2 launches) that keeps the
