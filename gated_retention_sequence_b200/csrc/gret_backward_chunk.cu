@@ -1,5 +1,8 @@
-// Chunk-parallel backward of the gated-retention prefill (CUDA cores, fp32
-// arithmetic, every (batch, head, chunk) its own thread block).
+// Chunk-parallel backward of the gated-retention prefill: every (batch, head,
+// chunk) its own thread block, fp32 accumulation.  Two variants of the
+// per-chunk kernels: tensor cores (mma.sync tf32 tiles, bf16 inputs with
+// d_k = 128 and d_v of 128 or 256; second half of this file) and CUDA cores
+// (fp32 arithmetic, other head sizes that are multiples of 32).
 //
 // The forward is the chunkwise form of "YOCO 深度技术分析" (sections 2.2 and
 // 5.3.2).  Per unit and chunk of L <= C tokens starting from state S_c, with
@@ -25,7 +28,7 @@
 // All exponents are <= 0.  The chunk length is a free parameter of the
 // chunkwise form: 64 for bf16 inputs, 32 for fp32 (shared-memory budget).
 //
-// Products are register-tiled on CUDA cores: a warp owns rows (warp + 8 r) of
+// On CUDA cores products are register-tiled: a warp owns rows (warp + 8 r) of
 // an output, its lanes own columns (lane + 32 c), so the row operand is a
 // shared-memory broadcast and the column operand a conflict-free row of 32
 // words.  Tiles read across their rows ("n-major") are padded to an odd word
