@@ -135,3 +135,22 @@ def test_backward_path_and_workspace(lib):
     # unsupported
     assert gret.gret_prefill_backward_workspace_size(1, 2, 100, 24, 64, bf) == 0
     assert gret.gret_prefill_backward_launches(1, 2, 100, 64, 64, 7) == 0
+
+
+def test_backward_rejects_bad_arguments(lib):
+    # every case fails validation before any GPU work (pointers never dereferenced)
+    good, ws = 0x10000, 0x100000
+    need = gret.gret_prefill_backward_workspace_size(1, 2, 100, 128, 256, gret.Dtype.BF16)
+    a = dict(Q=good, K=good, V=good, gate_logits=good, G=good, S0=None, dO=good, dS_final=None, tau=16.0,
+             eps=1e-5, epi=gret.Epilogue.GN_SWISH, dQ=good, dK=good, dV=good, dz=good, dG=good, dS0=None, B=1,
+             H=2, N=100, dk=128, dv=256, io_dtype=gret.Dtype.BF16, workspace=ws, workspace_bytes=need - 1,
+             stream=None)
+    invalid = [dict(Q=None), dict(dO=None), dict(dz=None), dict(G=None), dict(dG=None), dict(epi=5),
+               dict(io_dtype=7), dict(B=0), dict(N=0), dict(tau=0.0), dict(tau=float("inf")), dict(eps=-1.0),
+               dict(K=good + 8), dict(S0=good + 4), dict(workspace=None, workspace_bytes=need),
+               dict(workspace=ws + 128, workspace_bytes=need),      # workspace not 256-byte aligned
+               dict()]                                               # workspace one byte short
+    for over in invalid:
+        assert gret.gret_prefill_backward(**dict(a, **over)) == gret.Status.ERR_INVALID_ARG, over
+    for over in (dict(dk=24), dict(dv=512)):
+        assert gret.gret_prefill_backward(**dict(a, **over)) == gret.Status.ERR_UNSUPPORTED, over
