@@ -12,8 +12,9 @@ than the 126 MB L2, so no flush is needed between steps).
 The JSON line also carries the recurrent decode step (256 sequences x 16
 heads, 128 x 256 fp32 states, 64 consecutive launches) as ``decode``; the same
 16384 tokens packed as a ragged batch of sequences (gret_prefill_varlen) as
-``varlen``; and the gradients of the benchmark prefill (gret_prefill_backward)
-as ``backward``.
+``varlen``; one rank's computing steps of the sequence-parallel prefill (two
+slices of 2048 tokens) as ``seqpar``; and the gradients of the benchmark
+prefill (gret_prefill_backward) as ``backward``.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -328,6 +329,12 @@ def run_ours(args, world, rank, local):
 
     decode = None if args.no_decode else run_decode(args, world, dev, stream, peaks)
     varlen = None if args.no_varlen else run_varlen(args, world, dev, stream, d, cfg, peaks)
+    seqpar = None
+    if not args.no_seqpar:
+        try:
+            seqpar = run_seqpar(args, world, dev, stream, d, cfg, peaks)
+        except Exception as exc:          # a failed sub-measurement must not cost the line
+            seqpar = {"error": f"{type(exc).__name__}: {exc}"}
     backward = None if args.no_backward else run_backward(args, world, dev, stream, d, O, cfg, peaks)
     clk = clocks.stop()
 
@@ -360,6 +367,7 @@ def run_ours(args, world, rank, local):
             "clocks": clk,
             "decode": decode,
             "varlen": varlen,
+            "seqpar": seqpar,
             "backward": backward,
         }
         if world == 1 and not args.no_cpu_baseline:
@@ -434,6 +442,63 @@ def run_varlen(args, world, dev, stream, d, cfg, peaks):
             "path_hbm": {"alg_gbs": bytes_ / step_s / 1e9, "frac": bytes_ / step_s / 1e9 / peaks["hbm_gbs"]},
             "gpu_launches": gret.gret_prefill_launches(S_n, cfg.H, max_len, cfg.dk, cfg.dv, cfg.chunk, io)
             * args.steps}
+
+
+def run_seqpar(args, world, dev, stream, d, cfg, peaks):
+    """Chunk Parallelism ("YOCO 深度技术分析", section 5.3.3) on one GPU: the
+    benchmark's sequences cut into two slices of N/2 tokens.  Timed: one rank's
+    computing steps for the second slice (the state pass of its slice, the fold
+    of the first slice's increment -- what the all-gather delivers -- and the
+    prefill of its slice from the folded state), and a plain prefill of the same
+    slice from the zero state.  The all-gather itself (d_k d_v + 1 floats per
+    (batch, head) and rank) is not timed."""
+    import torch
+    import gated_retention_sequence_b200 as gret
+    half = cfg.N // 2
+    io = gret.Dtype.BF16
+    sl = [{k: v[:, a:a + half].contiguous() for k, v in d.items()} for a in (0, half)]
+    s = sl[1]
+    st_bytes = gret.gret_prefill_state_workspace_size(cfg.B, cfg.H, half, cfg.dk, cfg.dv, cfg.chunk, io)
+    st_ws = torch.empty(max(st_bytes, 256), dtype=torch.uint8, device=dev)
+    parts = [gret.prefill_state(p["K"], p["V"], p["z"], cfg.tau, cfg.chunk, workspace=st_ws, stream=stream)
+             for p in sl]
+    dS_all = torch.stack([p[0] for p in parts])
+    decay_all = torch.stack([p[1] for p in parts])
+    S_in = torch.empty((cfg.B, cfg.H, cfg.dk, cfg.dv), dtype=torch.float32, device=dev)
+    O = torch.empty_like(s["V"])
+    S_out = torch.empty_like(S_in)
+    ws_bytes = gret.gret_prefill_workspace_size(cfg.B, cfg.H, half, cfg.dk, cfg.dv, cfg.chunk, io)
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+
+    def rank_step():
+        gret.prefill_state(s["K"], s["V"], s["z"], cfg.tau, cfg.chunk, workspace=st_ws, stream=stream)
+        gret.state_fold(dS_all, decay_all, 1, out=S_in, stream=stream)
+        gret.prefill(s["Q"], s["K"], s["V"], s["z"], s["G"], cfg.tau, cfg.chunk, eps=cfg.eps, O=O,
+                     S_final=S_out, workspace=ws, stream=stream, S0=S_in)
+
+    def plain_step():
+        gret.prefill(s["Q"], s["K"], s["V"], s["z"], s["G"], cfg.tau, cfg.chunk, eps=cfg.eps, O=O,
+                     S_final=S_out, workspace=ws, stream=stream)
+
+    def timed(fn):
+        for _ in range(max(3, args.warmup)):
+            fn()
+        gret.check_device_status()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            fn()
+        e1.record(stream)
+        barrier(world)
+        gret.check_device_status()
+        return max_over_ranks(e0.elapsed_time(e1), world) / args.steps
+
+    rank_ms = timed(rank_step)
+    plain_ms = timed(plain_step)
+    return {"workload": f"{cfg.name} cut into 2 slices of {half} tokens; one rank's steps for the second slice",
+            "rank_ms": rank_ms, "plain_slice_ms": plain_ms, "overhead": rank_ms / plain_ms - 1.0,
+            "two_rank_mtoks_without_exchange": cfg.B * cfg.N / (rank_ms / 1e3) / 1e6, "steps": args.steps}
 
 
 def backward_alg(cfg):
@@ -564,6 +629,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-varlen", action="store_true")
+    ap.add_argument("--no-seqpar", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--backward-batch", type=int, default=0,
                     help="run the backward sub-measurement on this many of the batch's sequences")
