@@ -1,4 +1,7 @@
-// Backward of the gated-retention prefill on CUDA cores, fp32 arithmetic.
+// Backward of the gated-retention prefill: the host entry points (workspace
+// size, launch count, dispatch) and the serial CUDA-core path, fp32 arithmetic,
+// for head sizes the chunk-parallel kernels (gret_backward_chunk.cu) do not
+// take.
 //
 // The forward is the chunkwise form of "YOCO 深度技术分析", sections 2.2 and
 // 5.3.2; this file computes its exact derivative.  Per (batch, head) unit, a
