@@ -234,3 +234,43 @@ void oracle_decode_step(const double* q, const double* k, const double* v, const
         oracle_groupnorm_swish(yu, g + (size_t)u * dv, 1, dv, eps, o + (size_t)u * dv);
     }
 }
+
+/* Gate projection ("YOCO 深度技术分析", section 2.2: gamma = sigmoid(X W_gamma)^(1/tau),
+ * with W_gamma in R^{d x 1} per head -- the Medium-article translation's
+ * "门控保留率" paragraph gives the same shape): the gate logit of token n and
+ * head h is z[n][h] = sum_i X[n][i] W[i][h].
+ *   X [rows][d_model] (rows = B * N tokens), W [d_model][H], z [rows][H]. */
+void oracle_gate_project(const double* X, const double* W, long rows, int d_model, int H, double* z) {
+    for (long r = 0; r < rows; ++r)
+        for (int h = 0; h < H; ++h) {
+            double acc = 0.0;
+            for (int i = 0; i < d_model; ++i) acc += X[(size_t)r * d_model + i] * W[(size_t)i * H + h];
+            z[(size_t)r * H + h] = acc;
+        }
+}
+
+/* The rotation Theta of Q and K ("YOCO 深度技术分析" section 2.2:
+ * Q = (X W_Q) (.) Theta, K = (X W_K) (.) Theta; the "通用YOCO" page's notes on
+ * reproduction: the self-decoder's position encoding is RoPE; section 5.3.6 of
+ * the first page: the RoPE base grows 640K -> 5M -> 80M with context).  Theta_n
+ * is read as e^{i n theta_j} acting on consecutive pairs of channels taken as
+ * complex numbers x_{2j} + i x_{2j+1}, with theta_j = base^(-2j/d):
+ *   x'_{2j}   = x_{2j} cos(n theta_j) - x_{2j+1} sin(n theta_j)
+ *   x'_{2j+1} = x_{2j} sin(n theta_j) + x_{2j+1} cos(n theta_j)
+ * n is the token's position in its sequence (pos0 + index).
+ *   X, Xr [B][N][H][d] (d even). */
+void oracle_rotate(const double* X, int B, int N, int H, int d, double base, long pos0, double* Xr) {
+    for (int b = 0; b < B; ++b)
+        for (int n = 0; n < N; ++n)
+            for (int h = 0; h < H; ++h) {
+                const double* x = X + IDX4(b, n, h, 0, N, H, d);
+                double* y = Xr + IDX4(b, n, h, 0, N, H, d);
+                for (int j = 0; j < d / 2; ++j) {
+                    double theta = pow(base, -2.0 * j / d);
+                    double ang = (double)(pos0 + n) * theta;
+                    double c = cos(ang), s = sin(ang);
+                    y[2 * j] = x[2 * j] * c - x[2 * j + 1] * s;
+                    y[2 * j + 1] = x[2 * j] * s + x[2 * j + 1] * c;
+                }
+            }
+}

@@ -15,6 +15,10 @@ Parity status of each function (what pins it, checked in ``tests/test_oracle_pin
   groupnorm_swish  torch.nn.functional.group_norm and silu; mean-0 / variance
                    invariants
   decode_step      prefill(N0) + T steps == prefill(N0 + T)
+  gate_project     worked value; numpy matmul as a second route; linearity
+  rotate           worked values (position 0, one radian per position);
+                   pair norms; R(a) R(b) = R(a + b); rotated scores depend on
+                   positions only through their difference
 """
 from __future__ import annotations
 
@@ -34,7 +38,7 @@ _lock = threading.Lock()
 _lib = None
 
 __all__ = ["build", "build_variant", "source_text", "log_gamma", "recurrent", "parallel", "chunkwise", "groupnorm_swish",
-           "prefill", "decode_step", "as_f64", "default_threads"]
+           "prefill", "decode_step", "gate_project", "rotate", "prefill_projected", "as_f64", "default_threads"]
 
 
 def build(force: bool = False) -> str:
@@ -57,8 +61,11 @@ def _bind(path: str):
     lib.oracle_chunkwise.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, I, P, P]
     lib.oracle_groupnorm_swish.argtypes = [P, P, L, I, D, P]
     lib.oracle_decode_step.argtypes = [P, P, P, P, P, P, I, I, I, I, D, I, I, P, P]
+    lib.oracle_gate_project.argtypes = [P, P, L, I, I, P]
+    lib.oracle_rotate.argtypes = [P, I, I, I, I, D, L, P]
     for f in (lib.oracle_log_gamma, lib.oracle_recurrent, lib.oracle_parallel,
-              lib.oracle_chunkwise, lib.oracle_groupnorm_swish, lib.oracle_decode_step):
+              lib.oracle_chunkwise, lib.oracle_groupnorm_swish, lib.oracle_decode_step,
+              lib.oracle_gate_project, lib.oracle_rotate):
         f.restype = None
     return lib
 
@@ -215,3 +222,36 @@ def decode_step(q, k, v, z, g, S, tau: float, eps: float = 1e-5, lg=None,
                                                    dk, dv, float(eps), a, b, _p(y), _p(o)),
                ns * H, threads)
     return o, y, Sn
+
+
+def gate_project(X, W, lib=None) -> np.ndarray:
+    """Gate logits z = X W_gamma. X [..., d_model]; W [d_model, H]. Returns z [..., H] in fp64."""
+    X, W = as_f64(X), as_f64(W)
+    d_model, H = W.shape
+    assert X.shape[-1] == d_model
+    rows = X.size // d_model
+    z = np.empty(X.shape[:-1] + (H,))
+    _load(lib).oracle_gate_project(_p(X), _p(W), rows, d_model, H, _p(z))
+    return z
+
+
+def rotate(X, base: float, pos0: int = 0, lib=None) -> np.ndarray:
+    """The rotation Theta (RoPE on consecutive channel pairs) of X [B, N, H, d]
+    at positions pos0 .. pos0 + N - 1. Returns fp64."""
+    X = as_f64(X)
+    B, N, H, d = X.shape
+    assert d % 2 == 0
+    out = np.empty_like(X)
+    _load(lib).oracle_rotate(_p(X), B, N, H, d, float(base), int(pos0), _p(out))
+    return out
+
+
+def prefill_projected(Q, K, V, X, W, G, tau: float, eps: float = 1e-5, theta_base: float = 0.0,
+                      S0=None, threads: Optional[int] = None, lib=None):
+    """Prefill whose gate logits come from the projection z = X W_gamma, and whose
+    Q and K are rotated by Theta first when theta_base > 0.
+    X [B, N, d_model]; W [d_model, H]. Returns (O, Y, S_final) in fp64."""
+    z = gate_project(X, W, lib=lib)
+    if theta_base > 0:
+        Q, K = rotate(Q, theta_base, lib=lib), rotate(K, theta_base, lib=lib)
+    return prefill(Q, K, V, z, G, tau, eps, S0=S0, threads=threads, lib=lib)
