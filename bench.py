@@ -3,20 +3,30 @@
 
 One step = one gret_prefill call (gate, chunk decay sums, intra-chunk scores
 and mask, intra and inter-chunk outputs, state carry, GroupNorm + swish
-epilogue, final state) over a batch of 4 x 4096 tokens, 16 heads, d_k 128,
-d_v 256, chunk 64, bf16 I/O with fp32 state and gate logits -- the long-context
-prefill shape of "YOCO 深度技术分析" (head dimension 128, chunkwise form).
-Inputs are seeded synthetic tensors already resident in HBM (546 MB, larger
-than the 126 MB L2, so no flush is needed between steps).
+epilogue, final state) over one batch of a long-context prefill workload, bf16
+I/O with fp32 state and gate logits -- the chunkwise prefill of "YOCO 深度技术分析"
+(head dimension 128, contexts of 4K-64K tokens).  ``--config`` picks the
+headline workload:
 
-The JSON line also carries the recurrent decode step (256 sequences x 16
-heads, 128 x 256 fp32 states, 64 consecutive launches) as ``decode``; the same
-16384 tokens packed as a ragged batch of sequences (gret_prefill_varlen) as
-``varlen``; one rank's computing steps of the sequence-parallel prefill (two
-slices of 2048 tokens) as ``seqpar``; and the gradients of the benchmark
-prefill (gret_prefill_backward) as ``backward``.
+  c3  B1 H32 N65536, d_k = d_v = 128, chunk 128, gate logits ~ N(4, 1)  (default)
+  c2  B4 H16 N4096,  d_k 128, d_v 256, chunk 64, gate logits ~ N(3, 1.5)
+  c5  B2 H16 N32768, d_k 128, d_v 256, chunk 64, half the heads fast-decaying
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Inputs are seeded synthetic tensors already resident in HBM (0.55-2.7 GB,
+larger than the 126 MB L2, so no flush is needed between steps).  The other two
+prefill workloads ride in the same JSON line under ``prefill_configs``, each
+with its own roofline object.
+
+The line also carries the recurrent decode step (256 sequences x 16 heads,
+128 x 256 fp32 states, 64 consecutive launches) as ``decode``; the c2 tokens
+packed as a ragged batch of sequences (gret_prefill_varlen) as ``varlen``;
+one rank's computing steps of the sequence-parallel prefill (two slices of
+2048 tokens of c2) as ``seqpar``; the c2 prefill with its gate logits
+computed from z = X W_gamma in the gate prologue (gret_prefill_projected) as
+``projected``; and the gradients of the c2 prefill (gret_prefill_backward) as
+``backward``.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config c3|c2|c5] [--impl ours|reference]
 
 Multi-GPU (weak scaling): one process per GPU, each runs its own batch; no
 collective is on the data path.  ``--impl reference`` times the fp64 CPU
@@ -39,8 +49,16 @@ sys.path.insert(0, ROOT)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 METRIC = "gRet prefill Mtok/s & % bf16 TC peak; decode-step state GB/s & % HBM peak"
 # ncu summaries (under profiles/) that carry the DRAM traffic of the timed kernels
-PREFILL_PROFILE = "prefill_tc_kernel_B4_H16_N4096_dk128_dv256_C64.md"
 DECODE_PROFILE = "decode_step_kernel_S256_H16_dk128_dv256.md"
+PREFILL_SOURCE = "gated_retention_sequence_b200/csrc/gret_prefill_tc.cu"
+# the prefill workloads a --config may name (c1 is the small fp32 parity case,
+# c4 the decode workload)
+PREFILL_CONFIGS = ("c3", "c2", "c5")
+
+
+def prefill_profile(cfg):
+    """Name of the ncu summary of the fused kernel on this workload."""
+    return (f"prefill_tc_kernel_B{cfg.B}_H{cfg.H}_N{cfg.N}_dk{cfg.dk}_dv{cfg.dv}_C{cfg.chunk}.md")
 
 
 def load_peaks():
@@ -186,56 +204,86 @@ def profiled_traffic(kernel_file, source):
     return int(m.group(1))
 
 
-def cpu_oracle_sample(cfg, units, threads, min_seconds=0.0):
-    """Time the fp64 oracle (as it stands) on `units` (batch, head) units of cfg,
-    repeating the call until at least `min_seconds` have passed."""
+def oracle_sample_inputs(cfg, units, tokens):
+    """Per-unit inputs of the first `tokens` tokens of `units` (batch, head)
+    units of cfg, drawn on their own (element-identical to the full tensors),
+    stacked as a [1, tokens, units, d] batch for the oracle."""
     import gret_inputs as gi
-    import oracle
     import torch
     per = []
     for u in range(units):
         b, h = divmod(u % (cfg.B * cfg.H), cfg.H)
-        per.append(gi.prefill_unit_inputs(cfg, b, h))
+        per.append(gi.prefill_unit_inputs(cfg, b, h, tokens=tokens))
+    return {n: torch.stack([p[n] for p in per], 1)[None] for n in ("Q", "K", "V", "G", "z")}
 
-    def stack(name):
-        return torch.stack([p[name] for p in per], 1)[None] if name != "z" else \
-            torch.stack([p["z"] for p in per], 1)[None]
-    Q, K, V, G, z = (stack(n) for n in ("Q", "K", "V", "G", "z"))
+
+def oracle_sample_tokens(cfg, seconds):
+    """Tokens per unit of a bounded oracle sample: each unit runs on its own
+    host thread, and the fp64 recurrence costs about 4 dk dv flops per token
+    at roughly 1 GFLOP/s per core."""
+    return int(min(cfg.N, max(cfg.chunk, seconds * 1e9 / (4.0 * cfg.dk * cfg.dv))))
+
+
+def cpu_oracle_sample(cfg, units, threads, min_seconds=0.0, tokens=None, inputs=None):
+    """Time the fp64 oracle (as it stands) on the first `tokens` tokens of
+    `units` (batch, head) units of cfg, repeating the call until at least
+    `min_seconds` have passed.  Returns (Mtok/s, seconds, passes, tokens);
+    one token is one position of the sequence with all H heads."""
+    import oracle
+    tokens = cfg.N if tokens is None else min(tokens, cfg.N)
+    x = inputs if inputs is not None else oracle_sample_inputs(cfg, units, tokens)
     t0 = time.perf_counter()
     passes = 0
     while True:
-        oracle.prefill(Q, K, V, z, G, cfg.tau, cfg.eps, threads=threads)
+        oracle.prefill(x["Q"], x["K"], x["V"], x["z"], x["G"], cfg.tau, cfg.eps, threads=threads)
         passes += 1
         dt = time.perf_counter() - t0
         if dt >= min_seconds:
             break
-    tokens = passes * units * cfg.N / cfg.H     # one unit = N tokens of one of H heads
-    return tokens / dt / 1e6, dt, passes
+    token_heads = passes * units * tokens
+    return token_heads / cfg.H / dt / 1e6, dt, passes, tokens
+
+
+def config_of(name):
+    import gret_inputs as gi
+    return gi.CONFIGS[name]
+
+
+def config_dict(cfg, **extra):
+    d = {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "N": cfg.N, "dk": cfg.dk, "dv": cfg.dv,
+         "chunk": cfg.chunk, "io": "bf16 (fp32 state, fp32 gate logits)"}
+    d.update(extra)
+    return d
+
+
+# tokens per (batch, head) unit of one step of the reference arm: a bounded
+# prefix of the workload's sequences, so that a step is a fraction of a second
+REFERENCE_TOKENS = 4096
 
 
 def run_reference(args, world, rank):
     """Reference arm: the fp64 CPU oracle on a bounded sample of the workload."""
-    import gret_inputs as gi
     import oracle
     if rank != 0:
         return 0
-    cfg = gi.C2
+    cfg = config_of(args.config)
     threads = oracle.default_threads()
     units = min(cfg.B * cfg.H, threads)
+    tokens = min(cfg.N, REFERENCE_TOKENS)
+    x = oracle_sample_inputs(cfg, units, tokens)
     vals = []
     for i in range(args.warmup + args.steps):
-        v, dt, _ = cpu_oracle_sample(cfg, units, threads)
+        v, dt, _, _ = cpu_oracle_sample(cfg, units, threads, tokens=tokens, inputs=x)
         if i >= args.warmup:
             vals.append((v, dt))
     value = statistics.mean(v for v, _ in vals)
-    sample = (f"{units} of {cfg.B * cfg.H} (batch, head) units x {cfg.N} tokens per step, "
+    sample = (f"{units} of {cfg.B * cfg.H} (batch, head) units x the first {tokens} of {cfg.N} tokens per step, "
               f"fp64 recurrent form + GroupNorm/swish, {threads} threads")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "Mtok/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * statistics.mean(dt for _, dt in vals), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "N": cfg.N, "dk": cfg.dk,
-                       "dv": cfg.dv, "chunk": cfg.chunk, "io": cfg.io},
+            "config": config_dict(cfg),
             "cpu_baseline": {"value": value, "unit": "Mtok/s", "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "Mtok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -243,32 +291,23 @@ def run_reference(args, world, rank):
     return 0
 
 
-def run_ours(args, world, rank, local):
+def time_prefill(args, world, dev, stream, cfg, d):
+    """Warm up, then time args.steps prefill calls of cfg on inputs `d` already
+    in HBM: the whole call (events around the loop, max over ranks) and the
+    fused kernel alone (events the library records around its launch).
+    Returns (ms for all steps, mean fused-kernel ms, O, S, step function)."""
     import torch
     import gated_retention_sequence_b200 as gret
-    import gret_inputs as gi
-
-    gret.load()
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    peaks = load_peaks()
-    cfg = gi.C2
     io = gret.Dtype.BF16
-    path, segs = gret.prefill_path(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, cfg.chunk, io)
-    host = gi.prefill_inputs(cfg)
-    d = {k: v.to(dev) for k, v in host.items()}
     O = torch.empty_like(d["V"])
     S = torch.empty((cfg.B, cfg.H, cfg.dk, cfg.dv), dtype=torch.float32, device=dev)
     ws_bytes = gret.gret_prefill_workspace_size(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, cfg.chunk, io)
     ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
 
     def step():
         gret.prefill(d["Q"], d["K"], d["V"], d["z"], d["G"], cfg.tau, cfg.chunk, eps=cfg.eps, O=O,
                      S_final=S, workspace=ws, stream=stream)
 
-    clocks = ClockSampler(local)
-    clocks.start()
     for _ in range(args.warmup):
         step()
     gret.check_device_status()
@@ -287,22 +326,62 @@ def run_ours(args, world, rank, local):
     t_end.record(stream)
     gret.gret_set_profile_events(None, None)
     barrier(world)
-    ms = t_start.elapsed_time(t_end)
-    ms = max_over_ranks(ms, world)
+    ms = max_over_ranks(t_start.elapsed_time(t_end), world)
     gret.check_device_status()
     kern_ms = statistics.mean(ks[i].elapsed_time(ke[i]) for i in range(args.steps))
+    return ms, kern_ms, O, S, step
 
-    tokens = cfg.B * cfg.N
-    value = job_throughput(world, tokens, args.steps, ms) / 1e6
+
+def prefill_summary(cfg, world, steps, ms, kern_ms, peaks):
+    """Throughput, tensor and HBM fractions and the fused kernel's roofline
+    object of `steps` prefill calls of cfg that took `ms` (whole calls, max
+    over ranks) with the fused kernel taking `kern_ms` per launch."""
     alg_bytes, alg_flops = prefill_alg(cfg)
-    step_s = ms / 1e3 / args.steps
+    step_s = ms / 1e3 / steps
+    achieved = alg_bytes / (kern_ms / 1e3) / 1e9
+    return {
+        "value": job_throughput(world, cfg.B * cfg.N, steps, ms) / 1e6, "unit": "Mtok/s",
+        "ms_per_step": ms / steps,
+        "tc": {"alg_tflops": alg_flops / step_s / 1e12,
+               "frac_of_bf16_peak": alg_flops / step_s / 1e12 / peaks["bf16_tflops"],
+               "peak_tflops": peaks["bf16_tflops"], "peak_source": peaks["source"] + " burst"},
+        "path_hbm": {"alg_gbs": alg_bytes / step_s / 1e9, "frac": alg_bytes / step_s / 1e9 / peaks["hbm_gbs"]},
+        "roofline": {"kernel": f"prefill_tc_kernel<{cfg.dv}, {cfg.chunk}> (fused chunk loop)", "bound": "hbm",
+                     "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"],
+                     "traffic": profiled_traffic(prefill_profile(cfg), PREFILL_SOURCE),
+                     "alg_bytes_per_launch": alg_bytes, "launch_ms": kern_ms, "peak_source": peaks["source"]},
+    }
+
+
+def run_ours(args, world, rank, local):
+    import torch
+    import gated_retention_sequence_b200 as gret
+    import gret_inputs as gi
+
+    gret.load()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    cfg = config_of(args.config)
+    io = gret.Dtype.BF16
+    path, segs = gret.prefill_path(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, cfg.chunk, io)
+    host = gi.prefill_inputs(cfg)
+    d = {k: v.to(dev) for k, v in host.items()}
+    stream = torch.cuda.current_stream(dev)
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    ms, kern_ms, O, S, step = time_prefill(args, world, dev, stream, cfg, d)
+    head = prefill_summary(cfg, world, args.steps, ms, kern_ms, peaks)
     launches_per_step = gret.gret_prefill_launches(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, cfg.chunk, io)
 
     # end to end through the public call: pinned host inputs in, O and S out
     pin = {k: v.pin_memory() for k, v in host.items()}
+    del host
     O_h = torch.empty(O.shape, dtype=O.dtype, pin_memory=True)
     S_h = torch.empty(S.shape, dtype=S.dtype, pin_memory=True)
-    e2e_steps = max(1, min(args.steps, 20))
+    e2e_steps = max(1, min(args.steps, 10))
     h2d = sum(v.numel() * v.element_size() for v in pin.values())
     d2h = O_h.numel() * O_h.element_size() + S_h.numel() * S_h.element_size()
 
@@ -325,60 +404,92 @@ def run_ours(args, world, rank, local):
         e1.record(stream)
         barrier(world)
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-        e2e_value = job_throughput(world, tokens, e2e_steps, e2e_ms) / 1e6
+        e2e_value = job_throughput(world, cfg.B * cfg.N, e2e_steps, e2e_ms) / 1e6
+    gret.check_device_status()
+    del pin, O_h, S_h
+    # the fp64 oracle's sample reads the headline inputs back from the device
+    # (bounded: the first tokens of as many units as there are host threads)
+    sample_x = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        threads = oracle.default_threads()
+        units = min(cfg.B * cfg.H, threads)
+        tokens = oracle_sample_tokens(cfg, seconds=10.0)
+        sel = [divmod(u, cfg.H) for u in range(units)]
+        sample_x = {k: torch.stack([d[k][b, :tokens, h].cpu() for b, h in sel], 1)[None]
+                    for k in ("Q", "K", "V", "G", "z")}
+    del d, O, S
 
+    others = {}
+    if not args.no_other_configs:
+        for name in PREFILL_CONFIGS:
+            if name == args.config:
+                continue
+            c = config_of(name)
+            dd = {k: v.to(dev) for k, v in gi.prefill_inputs(c).items()}
+            o_ms, o_kern, *_ = time_prefill(args, world, dev, stream, c, dd)
+            p_, s_ = gret.prefill_path(c.B, c.H, c.N, c.dk, c.dv, c.chunk, io)
+            others[name] = dict(config_dict(c, segments=s_, path=p_.name),
+                                **prefill_summary(c, world, args.steps, o_ms, o_kern, peaks))
+            del dd
+
+    c2 = gi.C2
+    d2 = None
+    if not (args.no_varlen and args.no_seqpar and args.no_backward and args.no_projected):
+        d2 = {k: v.to(dev) for k, v in gi.prefill_inputs(c2).items()}
     decode = None if args.no_decode else run_decode(args, world, dev, stream, peaks)
-    varlen = None if args.no_varlen else run_varlen(args, world, dev, stream, d, cfg, peaks)
+    varlen = None if args.no_varlen else run_varlen(args, world, dev, stream, d2, c2, peaks)
     seqpar = None
     if not args.no_seqpar:
         try:
-            seqpar = run_seqpar(args, world, dev, stream, d, cfg, peaks)
+            seqpar = run_seqpar(args, world, dev, stream, d2, c2, peaks)
         except Exception as exc:          # a failed sub-measurement must not cost the line
             seqpar = {"error": f"{type(exc).__name__}: {exc}"}
-    backward = None if args.no_backward else run_backward(args, world, dev, stream, d, O, cfg, peaks)
+    projected = None
+    if not args.no_projected:
+        try:
+            projected = run_projected(args, world, dev, stream, d2, c2, peaks)
+        except Exception as exc:          # a failed sub-measurement must not cost the line
+            projected = {"error": f"{type(exc).__name__}: {exc}"}
+    backward = None
+    if not args.no_backward:
+        O2 = torch.empty_like(d2["V"])
+        gret.prefill(d2["Q"], d2["K"], d2["V"], d2["z"], d2["G"], c2.tau, c2.chunk, eps=c2.eps, O=O2)
+        backward = run_backward(args, world, dev, stream, d2, O2, c2, peaks)
     clk = clocks.stop()
 
     line = None
     if rank == 0:
-        achieved = alg_bytes / (kern_ms / 1e3) / 1e9
+        in_bytes = prefill_alg(cfg)[0]
         line = {
-            "metric": METRIC, "value": value, "unit": "Mtok/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+            "metric": METRIC, "value": head["value"], "unit": "Mtok/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "N": cfg.N, "dk": cfg.dk,
-                       "dv": cfg.dv, "chunk": cfg.chunk, "io": "bf16 (fp32 state, fp32 gate logits)",
-                       "segments": segs, "path": path.name,
-                       "l2": "inputs 546 MB > 126 MB L2 per step, no flush",
-                       "parallelism": f"dp{world} (independent batches)"},
-            "tc": {"alg_tflops": alg_flops / step_s / 1e12,
-                   "frac_of_bf16_peak": alg_flops / step_s / 1e12 / peaks["bf16_tflops"],
-                   "peak_tflops": peaks["bf16_tflops"], "peak_source": peaks["source"] + " burst"},
-            "path_hbm": {"alg_gbs": alg_bytes / step_s / 1e9,
-                         "frac": alg_bytes / step_s / 1e9 / peaks["hbm_gbs"]},
-            "roofline": {"kernel": "prefill_tc_kernel (fused chunk loop)", "bound": "hbm",
-                         "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": achieved / peaks["hbm_gbs"],
-                         "traffic": profiled_traffic(PREFILL_PROFILE, "gated_retention_sequence_b200/csrc/gret_prefill_tc.cu"),
-                         "alg_bytes_per_launch": alg_bytes, "launch_ms": kern_ms,
-                         "peak_source": peaks["source"]},
+            "config": config_dict(cfg, segments=segs, path=path.name,
+                                  l2=f"inputs and outputs {in_bytes / 1e6:.0f} MB > 126 MB L2 per step, no flush",
+                                  parallelism=f"dp{world} (independent batches)"),
+            "tc": head["tc"], "path_hbm": head["path_hbm"], "roofline": head["roofline"],
             "e2e": {"value": e2e_value, "unit": "Mtok/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk,
+            "prefill_configs": others,
             "decode": decode,
             "varlen": varlen,
             "seqpar": seqpar,
+            "projected": projected,
             "backward": backward,
         }
-        if world == 1 and not args.no_cpu_baseline:
+        if sample_x is not None:
             import oracle
             threads = oracle.default_threads()
-            units = cfg.B * cfg.H
-            v, dt, passes = cpu_oracle_sample(cfg, units, threads, min_seconds=10.0)
+            units = sample_x["Q"].shape[2]
+            v, dt, passes, tokens = cpu_oracle_sample(cfg, units, threads, min_seconds=10.0,
+                                                      tokens=sample_x["Q"].shape[1], inputs=sample_x)
             line["cpu_baseline"] = {"value": v, "unit": "Mtok/s", "cores": threads, "kind": "oracle",
-                                    "sample": f"{passes} passes over all {units} (batch, head) units x {cfg.N} "
-                                              f"tokens of {cfg.name}, fp64 recurrent form + GroupNorm/swish, "
-                                              f"{dt:.1f} s"}
+                                    "sample": f"{passes} passes over {units} of {cfg.B * cfg.H} (batch, head) "
+                                              f"units x the first {tokens} of {cfg.N} tokens of {cfg.name}, "
+                                              f"fp64 recurrent form + GroupNorm/swish, {dt:.1f} s"}
         print(json.dumps(line), flush=True)
     return 0
 
@@ -449,8 +560,8 @@ def run_seqpar(args, world, dev, stream, d, cfg, peaks):
     benchmark's sequences cut into two slices of N/2 tokens.  Timed: one rank's
     computing steps for the second slice (the state pass of its slice, the fold
     of the first slice's increment -- what the all-gather delivers -- and the
-    prefill of its slice from the folded state), and a plain prefill of the same
-    slice from the zero state.  The all-gather itself (d_k d_v + 1 floats per
+    prefill of its slice resumed from the state pass's workspace and the folded
+    state), and a plain prefill of the same slice from the zero state.  The all-gather itself (d_k d_v + 1 floats per
     (batch, head) and rank) is not timed."""
     import torch
     import gated_retention_sequence_b200 as gret
@@ -474,7 +585,7 @@ def run_seqpar(args, world, dev, stream, d, cfg, peaks):
         gret.prefill_state(s["K"], s["V"], s["z"], cfg.tau, cfg.chunk, workspace=st_ws, stream=stream)
         gret.state_fold(dS_all, decay_all, 1, out=S_in, stream=stream)
         gret.prefill(s["Q"], s["K"], s["V"], s["z"], s["G"], cfg.tau, cfg.chunk, eps=cfg.eps, O=O,
-                     S_final=S_out, workspace=ws, stream=stream, S0=S_in)
+                     S_final=S_out, workspace=st_ws, stream=stream, S0=S_in, resume=True)
 
     def plain_step():
         gret.prefill(s["Q"], s["K"], s["V"], s["z"], s["G"], cfg.tau, cfg.chunk, eps=cfg.eps, O=O,
@@ -581,6 +692,71 @@ def run_backward(args, world, dev, stream, d, O, cfg, peaks):
                             gret.gret_prefill_backward_launches(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, io))
 
 
+def projection_alg(cfg, d_model):
+    """Algorithmic bytes of the fused gate prologue of a projected prefill: X
+    read once (bf16), W_gamma read (fp32), and the decay sums and P-block
+    factors written (2 fp32 per token and head); flops 2 d_model per token and
+    head (z = X W_gamma; the two bf16 halves of W are an implementation detail)."""
+    units = cfg.B * cfg.H
+    npad = -(-cfg.N // cfg.chunk) * cfg.chunk
+    bytes_ = cfg.B * cfg.N * d_model * 2 + d_model * cfg.H * 4 + 2 * units * npad * 4
+    return bytes_, 2 * cfg.B * cfg.N * cfg.H * d_model
+
+
+def run_projected(args, world, dev, stream, d, cfg, peaks):
+    """gret_prefill_projected on the c2 tokens with X of d_model = H d_k
+    channels (67 MB of bf16 rows): the gate logits come from z = X W_gamma
+    inside the gate prologue.  Timed: the whole call, and the fused
+    projection-and-scan kernel alone (events around its launch)."""
+    import torch
+    import gated_retention_sequence_b200 as gret
+    import gret_inputs as gi
+    d_model = cfg.H * cfg.dk
+    X = gi.random_unit(cfg.seed, 41, (cfg.B, cfg.N, d_model), 0.0, 1.0 / d_model, "bf16").to(dev)
+    W = gi.random_unit(cfg.seed, 42, (d_model, cfg.H), 3.0, 1.5, "f32").to(dev)
+    O = torch.empty_like(d["V"])
+    S = torch.empty((cfg.B, cfg.H, cfg.dk, cfg.dv), dtype=torch.float32, device=dev)
+    io = gret.Dtype.BF16
+    ws_bytes = gret.gret_prefill_projected_workspace_size(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, cfg.chunk, d_model, io)
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+
+    def step():
+        gret.prefill_projected(d["Q"], d["K"], d["V"], X, W, d["G"], cfg.tau, cfg.chunk, eps=cfg.eps, O=O,
+                               S_final=S, workspace=ws, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    gret.check_device_status()
+    barrier(world)
+    ks = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ke = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for e in ks + ke:
+        e.record(stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    e0.record(stream)
+    for i in range(args.steps):
+        gret.gret_set_gate_profile_events(ks[i].cuda_event, ke[i].cuda_event)
+        step()
+    e1.record(stream)
+    gret.gret_set_gate_profile_events(None, None)
+    barrier(world)
+    gret.check_device_status()
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    kern_ms = statistics.mean(ks[i].elapsed_time(ke[i]) for i in range(args.steps))
+    bytes_, flops = projection_alg(cfg, d_model)
+    achieved = bytes_ / (kern_ms / 1e3) / 1e9
+    return {"workload": f"{cfg.name} with gate logits z = X W_gamma, X [{cfg.B}, {cfg.N}, {d_model}] bf16",
+            "steps": args.steps, "ms_per_step": ms / args.steps,
+            "value": job_throughput(world, cfg.B * cfg.N, args.steps, ms) / 1e6, "unit": "Mtok/s",
+            "roofline": {"kernel": "gate_project_scan_kernel (z = X W_gamma fused with the decay scan)",
+                         "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"], "traffic": None, "alg_bytes_per_launch": bytes_,
+                         "alg_flops_per_launch": flops, "launch_ms": kern_ms, "peak_source": peaks["source"]},
+            "gpu_launches": (1 + gret.gret_prefill_launches(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, cfg.chunk, io))
+            * args.steps}
+
+
 def run_decode(args, world, dev, stream, peaks):
     """Recurrent decode: 64 consecutive single-token steps over 256 x 16 states."""
     import torch
@@ -627,10 +803,15 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", choices=list(PREFILL_CONFIGS), default="c3",
+                    help="headline prefill workload (c3: B1 H32 N65536 d 128 chunk 128)")
+    ap.add_argument("--no-other-configs", action="store_true",
+                    help="skip the other prefill workloads' sub-measurements")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-varlen", action="store_true")
     ap.add_argument("--no-seqpar", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--no-projected", action="store_true")
     ap.add_argument("--backward-batch", type=int, default=0,
                     help="run the backward sub-measurement on this many of the batch's sequences")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -7,6 +7,7 @@
 #include <string.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "gret_common.cuh"
@@ -15,6 +16,8 @@ namespace gret {
 
 thread_local cudaEvent_t g_profile_start = nullptr;
 thread_local cudaEvent_t g_profile_stop = nullptr;
+thread_local cudaEvent_t g_profile_gate_start = nullptr;
+thread_local cudaEvent_t g_profile_gate_stop = nullptr;
 
 namespace {
 
@@ -24,6 +27,17 @@ constexpr int kMaxDevices = 64;
 unsigned int* g_status_ptr[kMaxDevices] = {};
 int g_num_sms[kMaxDevices] = {};
 std::mutex g_mu;
+
+// prefill calls on the tensor-core path still to carry an injected timeout
+std::atomic<int> g_inject_timeouts{0};
+
+// Take one pending injected timeout, if any.
+int take_injected_timeout() {
+    int n = g_inject_timeouts.load();
+    while (n > 0 && !g_inject_timeouts.compare_exchange_weak(n, n - 1)) {
+    }
+    return n > 0 ? 1 : 0;
+}
 
 // Device status word and SM count of the current device (looked up once per
 // device, with that device current).
@@ -50,7 +64,9 @@ bool shape_supported(int dk, int dv) {
     return dk % 16 == 0 && dv % 16 == 0 && dk <= 256 && dv <= 256;
 }
 
-bool chunk_supported(int chunk) { return chunk == 16 || chunk == 32 || chunk == 64 || chunk == 128; }
+bool chunk_supported(int chunk) {
+    return chunk == 16 || chunk == 32 || chunk == 64 || chunk == 128 || chunk == 256;
+}
 
 constexpr size_t kMaxSmem = 227 * 1024;
 
@@ -100,6 +116,11 @@ void gret_set_profile_events(void* start, void* stop) {
     g_profile_stop = static_cast<cudaEvent_t>(stop);
 }
 
+void gret_set_gate_profile_events(void* start, void* stop) {
+    g_profile_gate_start = static_cast<cudaEvent_t>(start);
+    g_profile_gate_stop = static_cast<cudaEvent_t>(stop);
+}
+
 gret_path gret_prefill_path(int B, int H, int N, int dk, int dv, int chunk, gret_dtype io_dtype,
                             int* segments) {
     int sms = 148;
@@ -124,11 +145,26 @@ size_t gret_prefill_workspace_size(int B, int H, int N, int dk, int dv, int chun
     return prefill_tc_workspace_bytes(B, H, N, dk, dv, chunk, segs, pcs);
 }
 
+// Workspace of a projected prefill: the prefill's own, then the split gate
+// weights (fused tensor-core prologue) or the gate logits (other paths).
+static size_t projected_extra_bytes(gret_path path, int B, int H, int N, int d_model) {
+    if (path == GRET_PATH_TC && gate_project_tc_supported(H, d_model)) return gate_project_tc_ws_bytes(H, d_model);
+    return ((size_t)B * N * H * 4 + 255) & ~size_t(255);
+}
+
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
 static gret_status prefill_impl(const void* Q, const void* K, const void* V, const float* gate_logits,
                                 const void* G, const float* S0, const int* cu_seqlens, int total, float tau,
                                 int chunk, void* O, float* S_final, int B, int H, int N, int dk, int dv,
                                 gret_dtype io_dtype, float eps, gret_epilogue epi, void* workspace,
-                                size_t workspace_bytes, gret_stream_t stream) {
+                                size_t workspace_bytes, gret_stream_t stream, const void* X = nullptr,
+                                const float* W_gamma = nullptr, int d_model = 0, bool resume = false) {
+    const bool projected = X != nullptr;
+    if (projected) {
+        if (!W_gamma || d_model <= 0 || !aligned16(X) || !aligned16(W_gamma) || cu_seqlens) return GRET_ERR_INVALID_ARG;
+        gate_logits = static_cast<const float*>(X);     // validated below like the logits it replaces
+    }
     if (!Q || !K || !V || !gate_logits || !O) return GRET_ERR_INVALID_ARG;
     if (epi != GRET_EPI_GN_SWISH && epi != GRET_EPI_NONE) return GRET_ERR_INVALID_ARG;
     if (epi == GRET_EPI_GN_SWISH && !G) return GRET_ERR_INVALID_ARG;
@@ -164,18 +200,62 @@ static gret_status prefill_impl(const void* Q, const void* K, const void* V, con
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t err;
-    if (path == GRET_PATH_TC) {
-        size_t need = prefill_tc_workspace_bytes(B, H, N, dk, dv, chunk, segs, pcs);
-        if (need > 0) {
-            if (!workspace || workspace_bytes < need) return GRET_ERR_INVALID_ARG;
-            if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return GRET_ERR_INVALID_ARG;
+    if (resume && path == GRET_PATH_TC) {
+        a.resume = 1;
+        a.pieces = prefill_tc_state_pieces(B, H, chunk, sms, segs, seg_len);
+    }
+    const size_t base = path != GRET_PATH_TC ? 0
+                        : resume ? prefill_tc_state_workspace_bytes(B, H, N, dk, dv, chunk, sms)
+                                 : prefill_tc_workspace_bytes(B, H, N, dk, dv, chunk, segs, pcs);
+    const size_t need = align256(base) + (projected ? projected_extra_bytes(path, B, H, N, d_model) : 0);
+    if (need > 0) {
+        if (!workspace || workspace_bytes < need) return GRET_ERR_INVALID_ARG;
+        if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return GRET_ERR_INVALID_ARG;
+    }
+    if (projected) {
+        a.X = X;
+        a.Wg = W_gamma;
+        a.d_model = d_model;
+        if (!(path == GRET_PATH_TC && gate_project_tc_supported(H, d_model))) {
+            // the gate logits first, into the workspace after the prefill's own
+            float* z = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + align256(base));
+            err = launch_gate_project_simt(a, z, s);
+            if (err != cudaSuccess) return GRET_ERR_CUDA;
+            a.z = z;
+            a.X = nullptr;
         }
+    }
+    if (path == GRET_PATH_TC) {
+        a.fault = take_injected_timeout();
         err = launch_prefill_tc(a, s);
     } else {
         err = launch_prefill_simt(a, s);
     }
     return err == cudaSuccess ? GRET_OK : GRET_ERR_CUDA;
 }
+
+size_t gret_prefill_projected_workspace_size(int B, int H, int N, int dk, int dv, int chunk, int d_model,
+                                             gret_dtype io_dtype) {
+    if (d_model <= 0) return 0;
+    int sms = 148, segs = 1, pcs = 1;
+    device_info(nullptr, &sms);
+    gret_path p = select_path(B, H, N, dk, dv, chunk, io_dtype, sms, &segs, nullptr, &pcs);
+    if (p == GRET_PATH_NONE) return 0;
+    const size_t base = p == GRET_PATH_TC ? prefill_tc_workspace_bytes(B, H, N, dk, dv, chunk, segs, pcs) : 0;
+    return align256(base) + projected_extra_bytes(p, B, H, N, d_model);
+}
+
+gret_status gret_prefill_projected(const void* Q, const void* K, const void* V, const void* X,
+                                   const float* W_gamma, int d_model, const void* G, float tau, int chunk,
+                                   void* O, float* S_final, int B, int H, int N, int dk, int dv,
+                                   gret_dtype io_dtype, float eps, gret_epilogue epi, void* workspace,
+                                   size_t workspace_bytes, gret_stream_t stream) {
+    if (!X) return GRET_ERR_INVALID_ARG;
+    return prefill_impl(Q, K, V, nullptr, G, nullptr, nullptr, 0, tau, chunk, O, S_final, B, H, N, dk, dv,
+                        io_dtype, eps, epi, workspace, workspace_bytes, stream, X, W_gamma, d_model);
+}
+
+void gret_debug_inject_timeout(int calls) { g_inject_timeouts.store(calls > 0 ? calls : 0); }
 
 gret_status gret_prefill(const void* Q, const void* K, const void* V, const float* gate_logits,
                          const void* G, float tau, int chunk, void* O, float* S_final, int B, int H,
@@ -192,6 +272,14 @@ gret_status gret_prefill_from_state(const void* Q, const void* K, const void* V,
                                     gret_stream_t stream) {
     return prefill_impl(Q, K, V, gate_logits, G, S0, nullptr, 0, tau, chunk, O, S_final, B, H, N, dk, dv, io_dtype,
                         eps, epi, workspace, workspace_bytes, stream);
+}
+
+gret_status gret_prefill_resume(const void* Q, const void* K, const void* V, const float* gate_logits,
+                                const void* G, const float* S0, float tau, int chunk, void* O, float* S_final, int B,
+                                int H, int N, int dk, int dv, gret_dtype io_dtype, float eps, gret_epilogue epi,
+                                void* workspace, size_t workspace_bytes, gret_stream_t stream) {
+    return prefill_impl(Q, K, V, gate_logits, G, S0, nullptr, 0, tau, chunk, O, S_final, B, H, N, dk, dv, io_dtype,
+                        eps, epi, workspace, workspace_bytes, stream, nullptr, nullptr, 0, true);
 }
 
 gret_status gret_prefill_varlen(const void* Q, const void* K, const void* V, const float* gate_logits,

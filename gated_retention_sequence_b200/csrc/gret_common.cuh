@@ -54,6 +54,17 @@ struct PrefillArgs {
     int segments;             // sequence segments per unit (TC path)
     int seg_len;              // tokens per segment (multiple of chunk)
     int pieces;               // state-pass pieces per segment (divides seg_len / chunk)
+    int fault;                // test only: inject a timed-out wait (gret_debug_inject_timeout)
+    // resumed prefill (gret_prefill_resume): the workspace already holds the
+    // decay sums and the folded state-pass pieces of these tokens; pieces is
+    // then the state pass's pieces per segment
+    int resume;
+    // gate projection (gret_prefill_projected): when X is set, the gate logits
+    // are z = X W_gamma, computed by the tensor-core path's gate prologue;
+    // X [B][N][d_model] bf16, Wg [d_model][H] fp32
+    const void* X;
+    const float* Wg;
+    int d_model;
 };
 
 struct DecodeArgs {
@@ -84,6 +95,21 @@ __device__ __forceinline__ float log_gamma(float z, float inv_tau) {
     return fmaxf(-sp * inv_tau, kMinLogGamma);
 }
 
+// P-block factors of the tensor-core prefill.  The P step forms
+// e^{b_t - b_s} as e^{b_t - b_{s0}} E_s with E_s = e^{b_{s0} - b_s}, s0 the
+// first token of s's block of C/4 columns (16 or 32 tokens, within one warp).
+// A block whose log-decay drops by more than kBlockMax gets E_{s0} = -1 (and
+// 0 elsewhere) instead, so the P step takes the exponentials directly there.
+// x is this lane's chunk-local decay sum b; every lane of the warp calls this.
+constexpr float kBlockMax = 40.0f;
+__device__ __forceinline__ float p_block_factor(float x, int lane, int bw) {
+    const float x0 = __shfl_sync(0xffffffffu, x, lane & ~(bw - 1));
+    const float xl = __shfl_sync(0xffffffffu, x, lane | (bw - 1));
+    float e = expf(x0 - x);
+    if (x0 - xl > kBlockMax) e = (lane & (bw - 1)) == 0 ? -1.f : 0.f;
+    return e;
+}
+
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
 
@@ -101,9 +127,12 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
-// Events gret_set_profile_events armed for this host thread (null when off).
+// Events gret_set_profile_events armed for this host thread (null when off),
+// and those of gret_set_gate_profile_events (around the gate prologue).
 extern thread_local cudaEvent_t g_profile_start;
 extern thread_local cudaEvent_t g_profile_stop;
+extern thread_local cudaEvent_t g_profile_gate_start;
+extern thread_local cudaEvent_t g_profile_gate_stop;
 
 // Host-side launchers (one per kernel family).
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
@@ -135,11 +164,20 @@ size_t bwd_chunked_workspace_bytes(int B, int H, int N, int dk, int dv, gret_dty
 cudaError_t launch_bwd_chunked(const BackwardArgs& a, cudaStream_t s);
 // state-only pass of the tensor-core path (a.state_only): workspace bytes and launch
 size_t prefill_tc_state_workspace_bytes(int B, int H, int N, int dk, int dv, int chunk, int num_sms);
+int prefill_tc_state_pieces(int B, int H, int chunk, int num_sms, int segments, int seg_len);
 cudaError_t launch_prefill_state_tc(const PrefillArgs& a, int num_sms, cudaStream_t s);
 // S_in = fold over slices q < slice of (decay_q, dS_q), from S0 or zero
 cudaError_t launch_state_fold(const float* dS_all, const float* decay_all, int num_slices, int slice,
                               const float* S0, float* S_in, int units, int elems, cudaStream_t s);
 bool prefill_tc_supported(int dk, int dv, int chunk, gret_dtype io);
+// gate projection (gret_gate_project.cu): the fused tensor-core prologue, which
+// writes the decay sums and P-block factors, and a CUDA-core projection to z
+int gate_project_heads_padded(int H);
+bool gate_project_tc_supported(int H, int d_model);
+size_t gate_project_tc_ws_bytes(int H, int d_model);
+cudaError_t launch_gate_project_tc(const PrefillArgs& a, float* bcum, float* eblk, int Npad, void* wsplit,
+                                   cudaStream_t s);
+cudaError_t launch_gate_project_simt(const PrefillArgs& a, float* z, cudaStream_t s);
 void prefill_tc_plan(int B, int H, int N, int chunk, int num_sms, int* segments, int* seg_len, int* pieces);
 size_t prefill_tc_workspace_bytes(int B, int H, int N, int dk, int dv, int chunk, int segments, int pieces);
 int prefill_tc_launches(int segments, int pieces);

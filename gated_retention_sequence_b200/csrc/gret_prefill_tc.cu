@@ -61,7 +61,6 @@ constexpr int kIssueRegs = 64;
 constexpr int kComputeRegs = 104;
 static_assert(4 * 128 * kComputeRegs + 128 * kIssueRegs <= kFusedThreads * kLaunchRegs, "register split");
 constexpr float kLazyMax = 64.0f;       // largest exponent the lazy state scale may reach
-constexpr float kBlockMax = 40.0f;      // largest log-decay drop within one block of P columns
 constexpr int kMaxSmem = 227 * 1024;    // dynamic shared memory per block
 
 template <int DV, int C>
@@ -103,7 +102,7 @@ struct Cfg {
     // per Q/K stage: C fp32 decay sums b_t, then C fp32 block factors (gate scan)
     static constexpr int OFF_B = OFF_QT + QT_BYTES;
     static constexpr int OFF_BAR = OFF_B + NQK * 2 * C * 4;
-    static constexpr int NUM_BARS = NQK + NV + NG + 10;
+    static constexpr int NUM_BARS = NQK + NV + NG + 12;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     // epilogue scratch: kCW x HT x 2 fp32 partial sums, then C x (rstd, -mean * rstd).
     // It gets its own space when that fits; otherwise it lives in the P buffer
@@ -133,8 +132,8 @@ struct TcParams {
     CUtensorMap tmQ, tmK, tmV, tmG, tmO;
     const float* bcum;       // [units][Npad] chunk-local cumulative log-decay
     const float* eblk;       // [units][Npad] block factors of the P columns (gate scan)
-    float* seg_state;        // [units][(P-1)*K][DV][DK]  (S^T, fp32)
-    float* seg_decay;        // [units][(P-1)*K]
+    float* seg_state;        // [units][slots][DV][DK]  (S^T, fp32)
+    float* seg_decay;        // [units][slots]
     float* S_final;          // [units][DK][DV] or null
     const float* S0;         // [units][DK][DV] initial state, or null for zero
     const int* cu;           // packed batch: sequence b is token rows cu[b] .. cu[b+1]-1; or null
@@ -143,9 +142,11 @@ struct TcParams {
     unsigned int* status;
     int H, N, Npad, P, seg_len;
     int K, piece_len;        // state-pass pieces per segment and their length
+    int slots;               // state-pass pieces (and seg_state slots) per unit
     float eps;
     int gn;                  // 1: GroupNorm + swish; 0: O = Y
     int has_g;
+    int fault;               // test only: the fused kernel's first wait gives up (see gret_debug_inject_timeout)
 };
 
 __device__ __forceinline__ float u2f(uint32_t x) { return __uint_as_float(x); }
@@ -273,7 +274,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
     // of its own.  (Unpipelined, the scores use the first of their pair.)
     constexpr int BQK = 0, BV = NQK, BG = NQK + NV, BSC = NQK + NV + NG, BO = BSC + 2, BMMA = BSC + 3;
     constexpr int BQT = BSC + 5, BPREP = BSC + 6, BTSC = BSC + 7, BSTAGED = BSC + 8;
-    static_assert(BSTAGED + 2 == CF::NUM_BARS, "barrier count");
+    // BDRAIN: the MMA warp's last commit, awaited before the tensor memory is
+    // freed; BNEVER: nothing arrives at it (the injected timeout waits there)
+    constexpr int BDRAIN = BSTAGED + 2, BNEVER = BSTAGED + 3;
+    static_assert(BNEVER + 1 == CF::NUM_BARS, "barrier count");
     // barrier and parity of the scores of chunk j
     auto bsc = [&](int j) -> int { return PIPE ? BSC + (j & 1) : BSC; };
     auto bsc_par = [&](int j) -> uint32_t { return PIPE ? (j >> 1) & 1 : j & 1; };
@@ -327,8 +331,15 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
       if (warp == kCW + 1) {
         if (lane == 0 && nchunks > 0) {
             // ============================================================ producer
+            // the last chunk whose loads went into each stage (-1: none): on the
+            // give-up path the loads still in flight are awaited before exit
+            int last_qk[NQK], last_v[NV], last_g[NG];
+            for (int x = 0; x < NQK; ++x) last_qk[x] = -1;
+            for (int x = 0; x < NV; ++x) last_v[x] = -1;
+            for (int x = 0; x < NG; ++x) last_g[x] = -1;
             auto issue_qk = [&](int j) {
                 const int s = j % NQK, n0 = n_begin + j * C;
+                last_qk[s] = j;
                 const uint32_t fb = bar(BQK + s);
                 mbar_arrive_expect_tx(fb, CF::Q_BYTES + CF::K_BYTES + 2 * C * 4);
                 for (int x = 0; x < 2; ++x) {
@@ -340,6 +351,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
             };
             auto issue_v = [&](int j) {
                 const int s = j % NV, n0 = n_begin + j * C;
+                last_v[s] = j;
                 const uint32_t fb = bar(BV + s);
                 mbar_arrive_expect_tx(fb, CF::V_BYTES);
                 for (int x = 0; x < DV / 64; ++x)
@@ -347,6 +359,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
             };
             auto issue_g = [&](int j) {
                 const int s = j % NG, n0 = n_begin + j * C;
+                last_g[s] = j;
                 const uint32_t fb = bar(BG + s);
                 mbar_arrive_expect_tx(fb, CF::G_BYTES);
                 for (int x = 0; x < DV / 64; ++x)
@@ -354,8 +367,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
             };
             // the output tile of chunk j, written over G(j) in shared memory, goes
             // out; once the store has read the stage it takes the G of chunk j + NG
-            auto store_out = [&](int j) {
-                mbar_wait(bar(BSTAGED + (j & 1)), (j >> 1) & 1, p.status, abort_flag);
+            auto store_out = [&](int j) -> bool {
+                if (!mbar_wait(bar(BSTAGED + (j & 1)), (j >> 1) & 1, p.status, abort_flag)) return false;
                 const uint32_t sG = sb + CF::OFF_G + (j % NG) * CF::G_BYTES;
                 const int n0 = n_begin + j * C;
                 if (!direct_tail(j)) {
@@ -365,25 +378,39 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
                     bulk_wait_read<0>();
                 }
                 if (p.has_g && j + NG < nchunks) issue_g(j + NG);
+                return true;
             };
-            issue_qk(0);
-            if (nchunks > 1) issue_qk(1);
-            issue_v(0);
-            if (NV == 2 && nchunks > 1) issue_v(1);
-            if (p.has_g) {
-                issue_g(0);
-                if (NG == 2 && nchunks > 1) issue_g(1);
+            if (p.fault) mbar_wait_injected_timeout(bar(BNEVER), p.status, abort_flag);
+            if (!*abort_flag) {
+                issue_qk(0);
+                if (nchunks > 1) issue_qk(1);
+                issue_v(0);
+                if (NV == 2 && nchunks > 1) issue_v(1);
+                if (p.has_g) {
+                    issue_g(0);
+                    if (NG == 2 && nchunks > 1) issue_g(1);
+                }
+                for (int i = 0; i < nchunks; ++i) {
+                    // pipelined, the epilogue of chunk i - 1 ends after chunk i's preparation
+                    if (PIPE && i >= 1 && !store_out(i - 1)) break;
+                    // once the state MMA of chunk i is done, its Q/K and V stages are free
+                    if (!mbar_wait(bar(BMMA + (i & 1)), (i >> 1) & 1, p.status, abort_flag)) break;
+                    if (i + NQK < nchunks) issue_qk(i + NQK);
+                    if (i + NV < nchunks) issue_v(i + NV);
+                    if (!PIPE && !store_out(i)) break;
+                }
+                if (PIPE && !*abort_flag) store_out(nchunks - 1);
             }
-            for (int i = 0; i < nchunks; ++i) {
-                // pipelined, the epilogue of chunk i - 1 ends after chunk i's preparation
-                if (PIPE && i >= 1) store_out(i - 1);
-                // once the state MMA of chunk i is done, its Q/K and V stages are free
-                mbar_wait(bar(BMMA + (i & 1)), (i >> 1) & 1, p.status, abort_flag);
-                if (i + NQK < nchunks) issue_qk(i + NQK);
-                if (i + NV < nchunks) issue_v(i + NV);
-                if (!PIPE) store_out(i);
+            if (*abort_flag) {
+                // gave up: no more loads are issued; let those in flight land
+                // (at most one per stage) before the shared memory is released
+                for (int x = 0; x < NQK; ++x)
+                    if (last_qk[x] >= 0) mbar_wait_drain(bar(BQK + x), (last_qk[x] / NQK) & 1, kWaitCycles);
+                for (int x = 0; x < NV; ++x)
+                    if (last_v[x] >= 0) mbar_wait_drain(bar(BV + x), (last_v[x] / NV) & 1, kWaitCycles);
+                for (int x = 0; x < NG; ++x)
+                    if (last_g[x] >= 0) mbar_wait_drain(bar(BG + x), (last_g[x] / NG) & 1, kWaitCycles);
             }
-            if (PIPE) store_out(nchunks - 1);
             bulk_wait<0>();
         }
       } else if (warp == kCW) {
@@ -397,7 +424,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
             // scores D[t][s] = Q K^T over d_k (M = 128 rows of t; rows >= C unused)
             auto issue_scores = [&](int j) {
                 const int s = j % NQK;
-                mbar_wait(bar(BQK + s), (j / NQK) & 1, p.status, abort_flag);
+                if (!mbar_wait(bar(BQK + s), (j / NQK) & 1, p.status, abort_flag)) return;
                 tc_fence_after();
                 const uint32_t sQ = sb + CF::OFF_Q + s * CF::Q_BYTES, sK = sb + CF::OFF_K + s * CF::K_BYTES;
                 const uint32_t dst = tm + CF::TM_SC + (PIPE ? (j & 1) * C : 0);
@@ -424,8 +451,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
                 // inter-chunk: O^T = T^T Q~^T, as soon as Q~ (and, with bf16 inter
                 // products, the bf16 copy of T) is ready and the previous state
                 // MMA has written T
-                mbar_wait(bar(BQT), i & 1, p.status, abort_flag);
-                if (i > 0) mbar_wait(bar(BMMA + ((i - 1) & 1)), ((i - 1) >> 1) & 1, p.status, abort_flag);
+                if (!mbar_wait(bar(BQT), i & 1, p.status, abort_flag)) break;
+                if (i > 0 && !mbar_wait(bar(BMMA + ((i - 1) & 1)), ((i - 1) >> 1) & 1, p.status, abort_flag)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int h = 0; h < NH; ++h) {
@@ -449,9 +476,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
                 // now, so that its P is ready to start when this chunk's output is
                 if (PIPE && i + 1 < nchunks) issue_scores(i + 1);
                 // intra-chunk: O^T += V^T P^T once P and K~ are ready
-                mbar_wait(bar(BPREP), i & 1, p.status, abort_flag);
+                if (!mbar_wait(bar(BPREP), i & 1, p.status, abort_flag)) break;
                 tc_fence_after();
-                mbar_wait(bar(BV + sv), (i / NV) & 1, p.status, abort_flag);
+                if (!mbar_wait(bar(BV + sv), (i / NV) & 1, p.status, abort_flag)) break;
 #pragma unroll
                 for (int h = 0; h < NH; ++h) {
                     const uint32_t vA = sV + 2 * h * CF::BOX;   // d_v rows h*128 .. +127 (two boxes)
@@ -465,7 +492,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
                 mma_commit(bar(BO));
                 if (TF32 && eager) {
                     // T is rescaled between the inter-chunk read and the state MMA
-                    mbar_wait(bar(BTSC), nsplit & 1, p.status, abort_flag);
+                    if (!mbar_wait(bar(BTSC), nsplit & 1, p.status, abort_flag)) break;
                     ++nsplit;
                     tc_fence_after();
                 }
@@ -481,6 +508,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
                 if (!PIPE && i + 1 < nchunks) issue_scores(i + 1);
                 lam = eager ? 0.f : lam + bC;
             }
+            // every MMA this thread issued has completed before the tensor
+            // memory is freed, on the give-up path too
+            mma_commit(bar(BDRAIN));
+            mbar_wait_drain(bar(BDRAIN), 0, kWaitCycles);
         }
       }
     } else {
@@ -502,7 +533,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
         {
             uint32_t r[W];
             if (seg > 0) {
-                const float* src = p.seg_state + ((size_t)u * (p.P - 1) * p.K + (size_t)seg * p.K - 1) * DV * DK +
+                const float* src = p.seg_state + ((size_t)u * p.slots + (size_t)seg * p.K - 1) * DV * DK +
                                    (size_t)s_d * DK + s_k0;
                 const float4* s4 = reinterpret_cast<const float4*>(src);
 #pragma unroll
@@ -855,7 +886,8 @@ struct StateCfg {
     static constexpr int OFF_V = OFF_K + NS * K_BYTES;
     static constexpr int OFF_B = OFF_V + NS * V_BYTES;
     static constexpr int OFF_BAR = OFF_B + NS * C * 4;
-    static constexpr int OFF_MISC = OFF_BAR + 2 * NS * 8;
+    // full and empty barrier per stage, then the drain barrier of the last commit
+    static constexpr int OFF_MISC = OFF_BAR + (2 * NS + 1) * 8;
     static constexpr int SMEM = OFF_MISC + 16 + 1024;
     static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
@@ -871,18 +903,19 @@ __global__ void __launch_bounds__(kStateThreads, 1) prefill_state_kernel(const _
     const int q4 = warp & 3, gi = warp >> 2;
     const uint32_t lq = (uint32_t)(32 * q4) << 16;
 
-    const int nseg = (p.P - 1) * p.K;           // pieces of all segments but the last
+    const int nseg = p.slots;                   // pieces of the segments that need one
     const int u = blockIdx.x / nseg, seg = blockIdx.x % nseg;
     const int hh = u % p.H;
     const int n_begin = seg * p.piece_len;
 
     auto full = [&](int s) -> uint32_t { return sb + CF::OFF_BAR + 8 * s; };
     auto empty = [&](int s) -> uint32_t { return sb + CF::OFF_BAR + 8 * (NS + s); };
+    const uint32_t drain_bar = sb + CF::OFF_BAR + 8 * (2 * NS);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + CF::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + CF::OFF_MISC + 4);
 
     if (tid == 0) {
-        for (int i = 0; i < 2 * NS; ++i) mbar_init(sb + CF::OFF_BAR + 8 * i, 1);
+        for (int i = 0; i < 2 * NS + 1; ++i) mbar_init(sb + CF::OFF_BAR + 8 * i, 1);
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&p.tmK);
@@ -909,8 +942,10 @@ __global__ void __launch_bounds__(kStateThreads, 1) prefill_state_kernel(const _
     }
     const int n_end = min(Nu, n_begin + p.piece_len);
     const int nchunks = n_end > n_begin ? (n_end - n_begin + C - 1) / C : 0;
+    int last_issued = -1;     // thread 0: the last chunk whose loads it issued
     auto issue = [&](int j) {
         const int s = j % NS, n0 = n_begin + j * C;
+        last_issued = j;
         mbar_arrive_expect_tx(full(s), CF::K_BYTES + CF::V_BYTES + C * 4);
         for (int x = 0; x < 2; ++x)
             tma_load_4d(sb + CF::OFF_K + s * CF::K_BYTES + x * CF::BOX, &p.tmK, x * 64, hh, row0 + n0, bb, full(s));
@@ -985,7 +1020,7 @@ __global__ void __launch_bounds__(kStateThreads, 1) prefill_state_kernel(const _
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
-        if (tid == 0) {
+        if (tid == 0 && !*abort_flag) {
             tc_fence_after();
             const uint32_t sK = sb + CF::OFF_K + s * CF::K_BYTES, sV = sb + CF::OFF_V + s * CF::V_BYTES;
             constexpr uint32_t id_kv = idesc_bf16(128, DK, true, true);
@@ -999,13 +1034,23 @@ __global__ void __launch_bounds__(kStateThreads, 1) prefill_state_kernel(const _
             mma_commit(empty(s));
             // the stage the previous chunk used is free once its MMAs are done
             // (they run before this chunk's, which queue behind them)
-            if (i > 0 && i - 1 + NS < nchunks) {
-                mbar_wait(empty((i - 1) % NS), ((i - 1) / NS) & 1, p.status, abort_flag);
+            if (i > 0 && i - 1 + NS < nchunks &&
+                mbar_wait(empty((i - 1) % NS), ((i - 1) / NS) & 1, p.status, abort_flag))
                 issue(i - 1 + NS);
-            }
         }
         seg_decay += bC;
         lam = eager ? 0.f : lam + bC;
+    }
+    if (tid == 0) {
+        // every MMA issued has completed, and on the give-up path every load
+        // issued has landed, before the tensor and shared memory are released
+        // (loads into a stage are issued only after the previous chunk in
+        // it was consumed, so the last NS chunks issued are the ones in flight)
+        mma_commit(drain_bar);
+        mbar_wait_drain(drain_bar, 0, kWaitCycles);
+        if (*abort_flag)
+            for (int j = last_issued; j >= 0 && j > last_issued - NS; --j)
+                mbar_wait_drain(full(j % NS), (j / NS) & 1, kWaitCycles);
     }
     if (nchunks > 0) {
         mbar_wait(empty((nchunks - 1) % NS), ((nchunks - 1) / NS) & 1, p.status, abort_flag);
@@ -1044,7 +1089,8 @@ constexpr int kScanThreads = 256;   // a block scans 256 / C chunks of one unit
 __global__ void __launch_bounds__(kScanThreads) gate_scan_kernel(const float* __restrict__ z,
                                                                  const int* __restrict__ cu_seqlens, int total,
                                                                  float* __restrict__ bcum, float* __restrict__ eblk,
-                                                                 int H, int N, int Npad, int C, float inv_tau) {
+                                                                 int H, int N, int Npad, int C, float inv_tau,
+                                                                 int nyb) {
     __shared__ float wsum[kScanThreads / 32];
     // the gate logits may come from the kernel before this one, and the kernels
     // before that may still read the workspace: wait for them first
@@ -1053,34 +1099,39 @@ __global__ void __launch_bounds__(kScanThreads) gate_scan_kernel(const float* __
     const int u = blockIdx.x, b = u / H, h = u % H;
     const int lane = threadIdx.x & 31, wg = threadIdx.x >> 5;
     const int t = threadIdx.x % C, w = t >> 5;                 // token and warp within the chunk
-    const int ch = blockIdx.y * (kScanThreads / C) + threadIdx.x / C;
-    const bool live = ch * C < Npad;
-    const int n = ch * C + t;
     // this unit's tokens are rows base .. base + Nu - 1; past its end the
     // decay stays flat (log gamma = 0), so a chunk's last sum is its decay
     int row0 = 0, Nu = N;
     if (cu_seqlens) packed_range(cu_seqlens, b, total, row0, Nu);
     const size_t base = cu_seqlens ? (size_t)row0 : (size_t)b * N;
-    float x = (live && n < Nu) ? log_gamma(z[(base + n) * H + h], inv_tau) : 0.f;
+    // blocks of kScanThreads / C chunks, strided over the grid's y extent
+    for (int by = blockIdx.y; by < nyb; by += gridDim.y) {
+        const int ch = by * (kScanThreads / C) + threadIdx.x / C;
+        const bool live = ch * C < Npad;
+        const int n = ch * C + t;
+        float x = (live && n < Nu) ? log_gamma(z[(base + n) * H + h], inv_tau) : 0.f;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        float y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
+        for (int o = 1; o < 32; o <<= 1) {
+            float y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) wsum[wg] = x;
+        __syncthreads();
+        for (int j = 0; j < w; ++j) x += wsum[wg - w + j];      // the chunk's earlier warps
+        if (live) bcum[(size_t)u * Npad + n] = x;
+        // block factors for the P step (p_block_factor)
+        const float e = p_block_factor(x, lane, C / 4);
+        if (live) eblk[(size_t)u * Npad + n] = e;
+        __syncthreads();       // wsum is rewritten by the next block of chunks
     }
-    if (lane == 31) wsum[wg] = x;
-    __syncthreads();
-    for (int j = 0; j < w; ++j) x += wsum[wg - w + j];      // the chunk's earlier warps
-    if (live) bcum[(size_t)u * Npad + n] = x;
-    // block factors for the P step: E_n = e^{b_{s0} - b_n}, s0 the first token of
-    // n's block of C/4 (16 or 32, within one warp); a block whose decay drops by
-    // more than kBlockMax gets E_{s0} = -1 instead, so the P step takes the
-    // exponentials directly there
-    const int bw = C / 4;
-    const float x0 = __shfl_sync(0xffffffffu, x, lane & ~(bw - 1));
-    const float xl = __shfl_sync(0xffffffffu, x, lane | (bw - 1));
-    float e = expf(x0 - x);
-    if (x0 - xl > kBlockMax) e = (lane & (bw - 1)) == 0 ? -1.f : 0.f;
-    if (live) eblk[(size_t)u * Npad + n] = e;
+}
+
+// Launch shape of the gate scan: units in x, blocks of chunks in y (at most
+// the grid's y limit; the kernel strides over the rest).
+static dim3 gate_scan_grid(int units, int npad, int C, int* nyb) {
+    const int per = kScanThreads / C;
+    *nyb = (npad / C + per - 1) / per;
+    return dim3(units, *nyb < 65535 ? *nyb : 65535);
 }
 
 // Fold the segment increments into initial states, in place:
@@ -1089,9 +1140,9 @@ __global__ void seg_combine_kernel(float* __restrict__ seg_state, const float* _
                                    const float* __restrict__ S0, int nslots, int dk, int dv) {
     grid_dep_launch();
     grid_dep_wait();       // the state pass's increments
-    const int u = blockIdx.y;
+    const int u = blockIdx.x;
     const int elems4 = dk * dv / 4;
-    const int e = blockIdx.x * blockDim.x + threadIdx.x;
+    const int e = blockIdx.y * blockDim.x + threadIdx.x;
     if (e >= elems4) return;
     float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
     if (S0) {   // slots hold S^T [dv][dk]; S0 is [dk][dv]
@@ -1108,24 +1159,51 @@ __global__ void seg_combine_kernel(float* __restrict__ seg_state, const float* _
     }
 }
 
-// State-only pass: the folded pieces (slot K-1, S^T layout [DV][DK]) become the
-// slice's increment dS [DK][DV] through a shared-memory tile transpose, and the
-// pieces' log-decays sum to the slice's total.
+// State-only pass: the folded pieces (the last slot, S^T layout [DV][DK]) become
+// the slice's increment dS [DK][DV] through a shared-memory tile transpose, and
+// the pieces' log-decays sum to the slice's total.
 template <int DV>
 __global__ void state_finish_kernel(const float* __restrict__ seg_state, const float* __restrict__ seg_decay,
-                                    int K, float* __restrict__ dS, float* __restrict__ decay) {
+                                    int slots, float* __restrict__ dS, float* __restrict__ decay) {
     __shared__ float tile[32][33];
-    const int u = blockIdx.z;
-    const int d0 = blockIdx.x * 32, k0 = blockIdx.y * 32;     // tile of d_v rows, d_k columns of S^T
-    const float* src = seg_state + ((size_t)u * K + K - 1) * DV * DK;
+    const int u = blockIdx.x;
+    const int d0 = (blockIdx.y % (DV / 32)) * 32, k0 = (blockIdx.y / (DV / 32)) * 32;   // tile of S^T
+    const float* src = seg_state + ((size_t)u * slots + slots - 1) * DV * DK;
     for (int r = threadIdx.y; r < 32; r += blockDim.y) tile[r][threadIdx.x] = src[(size_t)(d0 + r) * DK + k0 + threadIdx.x];
     __syncthreads();
     float* dst = dS + (size_t)u * DK * DV;
     for (int r = threadIdx.y; r < 32; r += blockDim.y) dst[(size_t)(k0 + r) * DV + d0 + threadIdx.x] = tile[threadIdx.x][r];
-    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0 && threadIdx.y == 0) {
+    if (blockIdx.y == 0 && threadIdx.x == 0 && threadIdx.y == 0) {
         float a = 0.f;
-        for (int k = 0; k < K; ++k) a += seg_decay[(size_t)u * K + k];
+        for (int k = 0; k < slots; ++k) a += seg_decay[(size_t)u * slots + k];
         decay[u] = a;
+    }
+}
+
+// Prefill resumed after a state-only pass of the same tokens, whose pieces
+// were folded from the zero state: every folded slot j (the state after piece
+// j, S^T layout) gains the initial state carried through the pieces' decays,
+// slot_j += e^{a_0 + ... + a_j} S0 -- the state decomposition with S0 as the
+// state before the first piece.
+__global__ void seg_shift_kernel(float* __restrict__ seg_state, const float* __restrict__ seg_decay,
+                                 const float* __restrict__ S0, int slots, int dk, int dv) {
+    grid_dep_launch();
+    grid_dep_wait();
+    const int u = blockIdx.x;
+    const int elems4 = dk * dv / 4;
+    const int e = blockIdx.y * blockDim.x + threadIdx.x;
+    if (e >= elems4) return;
+    const int d = (4 * e) / dk, k = (4 * e) % dk;       // S^T element (d, k .. k + 3); S0 is [dk][dv]
+    const float* s0 = S0 + (size_t)u * dk * dv + (size_t)k * dv + d;
+    const float4 x = make_float4(s0[0], s0[dv], s0[2 * dv], s0[3 * dv]);
+    float a = 0.f;
+    for (int j = 0; j < slots; ++j) {
+        a += seg_decay[(size_t)u * slots + j];
+        const float f = __expf(a);
+        float4* slot = reinterpret_cast<float4*>(seg_state) + ((size_t)u * slots + j) * elems4 + e;
+        float4 v = *slot;
+        v = make_float4(fmaf(f, x.x, v.x), fmaf(f, x.y, v.y), fmaf(f, x.z, v.z), fmaf(f, x.w, v.w));
+        *slot = v;
     }
 }
 
@@ -1134,14 +1212,476 @@ __global__ void state_finish_kernel(const float* __restrict__ seg_state, const f
 __global__ void state_fold_kernel(const float* __restrict__ dS_all, const float* __restrict__ decay_all,
                                   int slice, const float* __restrict__ S0, float* __restrict__ S_in, int units,
                                   int elems) {
-    const int u = blockIdx.y;
-    const int e = blockIdx.x * blockDim.x + threadIdx.x;
+    const int u = blockIdx.x;
+    const int e = blockIdx.y * blockDim.x + threadIdx.x;
     if (e >= elems) return;
     const size_t at = (size_t)u * elems + e;
     float run = S0 ? S0[at] : 0.f;
     for (int q = 0; q < slice; ++q)
         run = fmaf(__expf(decay_all[(size_t)q * units + u]), run, dS_all[(size_t)q * units * elems + at]);
     S_in[at] = run;
+}
+
+// ---------------------------------------------------------------------------
+// Fused chunk loop for 128-token chunks with d_v = 128, output held as rows.
+//
+// The same chunkwise form as prefill_tc_kernel, laid out the other way round
+// for the output: O[t][d] sits in tensor memory with one token per lane, so the
+// GroupNorm of a token is one thread's sum over its own row and G / O move as
+// 16-byte vectors, and P[t][s] feeds the intra-chunk product from tensor memory.
+//   scores  D[t][s]  = Q K~^T        A = Q (smem, K-major), B = K~ (K-major)
+//   inter   D[t][d]  = Q~ T           A = Q or Q~ (smem),    B = bf16 copy of T^T (smem, K-major)
+//   intra   D[t][d] += P V            A = P (tensor memory, bf16), B = V (smem, MN-major)
+//   state   D[d][k] += V^T K~         A = V (MN-major), B = K~ (MN-major): T^T, fp32, lanes = d
+// The epilogue warps read G from a TMA-loaded tile and write their output
+// rows straight to global memory (16-byte stores, 256 contiguous bytes per
+// token), so the next G tile can load as soon as this one has been read.
+//
+// Lazy chunks (the largest K scale e^{-b_s - Lambda} within e^kLazyMax) factor
+// the decay: K~_s = e^{-b_s - Lambda} K_s is scaled once, before the scores, so
+//   e^{-(b_t + Lambda)} Y_t = Q_t T + sum_{s <= t} (Q_t . K~_s) V_s,
+// P is the masked scores alone, Q needs no scaling, and the row factor
+// c_t = e^{b_t + Lambda} <= 1 enters the GroupNorm statistics (mean c mu,
+// variance c^2 var) in the epilogue; the state update T += V^T K~ uses the same
+// K~ and Lambda += b_C.  Eager chunks take the direct forms: P[t][s] =
+// A[t][s] e^{b_t - b_s}, Q~_t = e^{b_t + Lambda} Q_t against the unscaled T, then
+// T *= e^{Lambda + b_C}, K~_s = e^{b_C - b_s} K_s and Lambda = 0.  All exponents
+// stay <= kLazyMax, so nothing overflows.
+//
+// Roles (512 threads).  Warps 0-3 (E): epilogue, one token row per thread.
+// Warps 4-7 (P): masked scores -> bf16 P in tensor memory.  Warps 8-11 (S): K~
+// and Q~ in shared memory, the bf16 copy of T after each state update, the
+// eager rescale, the initial and final state.  Warp 12 lane 0 issues every
+// MMA, warp 13 lane 0 every TMA load and store; warps 14-15 idle.  The roles
+// work on different chunks at once: E finishes chunk i while S and P prepare
+// chunk i + 1 and the tensor cores run its products.
+constexpr int kRowsThreads = 512;
+constexpr int kRowsLaunchRegs = 128;   // 65536 / 512
+constexpr int kRowsERegs = 200;        // epilogue warps hold a token's 128 outputs
+constexpr int kRowsOtherRegs = 104;
+static_assert(128 * kRowsERegs + 384 * kRowsOtherRegs <= kRowsThreads * kRowsLaunchRegs, "register split");
+
+struct RowsCfg {
+    static constexpr int C = 128, DV = 128;
+    static constexpr int BOX = C * 128;             // one [128 rows x 64] bf16 box, 16 KB
+    static constexpr int TILE = 2 * BOX;            // [128 rows x 128] bf16
+    static constexpr int OFF_Q = 0;                 // 2 stages
+    static constexpr int OFF_K = OFF_Q + 2 * TILE;  // 2 stages
+    static constexpr int OFF_V = OFF_K + 2 * TILE;
+    static constexpr int OFF_G = OFF_V + TILE;      // G
+    static constexpr int OFF_T = OFF_G + TILE;      // bf16 T^T [d][k]
+    static constexpr int OFF_B = OFF_T + TILE;      // per Q/K stage: C fp32 decay sums
+    static constexpr int OFF_BAR = OFF_B + 2 * C * 4;
+    static constexpr int NUM_BARS = 17;
+    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+    static constexpr int USED = OFF_MISC + 16;
+    static constexpr int SMEM = USED + 1024;        // room to align the base to 1024 bytes
+    static_assert(SMEM <= kMaxSmem, "shared memory budget");
+    // tensor-memory columns
+    static constexpr int TM_O = 0, TM_SC = 128, TM_P = 256, TM_T = 320, TM_ALLOC = 512;
+};
+
+__global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __grid_constant__ TcParams p) {
+    using CF = RowsCfg;
+    constexpr int C = CF::C, DV = CF::DV;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sb = smem_u32(sm);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int u = blockIdx.x / p.P, seg = blockIdx.x % p.P;
+    const int hh = u % p.H, bb = u / p.H;
+    const int n_begin = seg * p.seg_len;
+    const int n_end = min(p.N, n_begin + p.seg_len);
+    const int nchunks = n_end > n_begin ? (n_end - n_begin + C - 1) / C : 0;
+
+    // barriers; KT has one per Q/K stage so that no phase can complete twice
+    // before the MMA warp has seen the first.  BGF: the epilogue has read the
+    // G tile (index 14 is unused)
+    constexpr int BQK = 0, BV = 2, BG = 3, BSC = 4, BOD = 5, BST = 6, BKT = 7, BTC = 9, BQT = 10, BPR = 11,
+                  BOF = 12, BGF = 13, BDRAIN = 15, BNEVER = 16;
+    static_assert(BNEVER + 1 == CF::NUM_BARS, "barrier count");
+    auto bar = [&](int i) -> uint32_t { return sb + CF::OFF_BAR + 8 * i; };
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + CF::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + CF::OFF_MISC + 4);
+
+    if (tid == 0) {
+        for (int i = 0; i < CF::NUM_BARS; ++i) {
+            // per-warp arrivals of a four-warp role
+            const bool four = i == BKT || i == BKT + 1 || i == BTC || i == BQT || i == BPR || i == BOF || i == BGF;
+            mbar_init(bar(i), four ? 4 : 1);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&p.tmQ);
+        tma_prefetch_desc(&p.tmK);
+        tma_prefetch_desc(&p.tmV);
+        tma_prefetch_desc(&p.tmG);
+        tma_prefetch_desc(&p.tmO);
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(tmem_slot), CF::TM_ALLOC);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = *tmem_slot;
+    grid_dep_launch();
+    grid_dep_wait();
+
+    const int role = warp >> 2;            // 0 E, 1 P, 2 S, 3 issuing warps
+    const int q4 = warp & 3;               // tensor-memory lane quarter
+    const uint32_t lq = (uint32_t)(32 * q4) << 16;
+    const int row = 32 * q4 + lane;        // token t (E, P) or channel d (S) of this thread
+    auto warp_arrive = [&](int b) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(b));
+    };
+    auto stage_bc = [&](int i) -> const float* {
+        return reinterpret_cast<const float*>(sm + CF::OFF_B + (i & 1) * C * 4);
+    };
+
+    if (role == 3) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" : : "n"(kRowsOtherRegs));
+        if (warp == 13 && lane == 0 && nchunks > 0) {
+            // ======================================================== TMA producer
+            int last_qk[2] = {-1, -1}, last_v = -1, last_g = -1;
+            auto issue_qk = [&](int j) {
+                const int s = j & 1, n0 = n_begin + j * C;
+                last_qk[s] = j;
+                const uint32_t fb = bar(BQK + s);
+                mbar_arrive_expect_tx(fb, 2 * CF::TILE + C * 4);
+                for (int x = 0; x < 2; ++x) {
+                    tma_load_4d(sb + CF::OFF_Q + s * CF::TILE + x * CF::BOX, &p.tmQ, x * 64, hh, n0, bb, fb);
+                    tma_load_4d(sb + CF::OFF_K + s * CF::TILE + x * CF::BOX, &p.tmK, x * 64, hh, n0, bb, fb);
+                }
+                bulk_load(sb + CF::OFF_B + s * C * 4, p.bcum + (size_t)u * p.Npad + n0, C * 4, fb);
+            };
+            auto issue_v = [&](int j) {
+                last_v = j;
+                mbar_arrive_expect_tx(bar(BV), CF::TILE);
+                for (int x = 0; x < 2; ++x)
+                    tma_load_4d(sb + CF::OFF_V + x * CF::BOX, &p.tmV, x * 64, hh, n_begin + j * C, bb, bar(BV));
+            };
+            auto issue_g = [&](int j) {
+                last_g = j;
+                mbar_arrive_expect_tx(bar(BG), CF::TILE);
+                for (int x = 0; x < 2; ++x)
+                    tma_load_4d(sb + CF::OFF_G + x * CF::BOX, &p.tmG, x * 64, hh, n_begin + j * C, bb, bar(BG));
+            };
+            if (p.fault) mbar_wait_injected_timeout(bar(BNEVER), p.status, abort_flag);
+            if (!*abort_flag) {
+                issue_qk(0);
+                if (nchunks > 1) issue_qk(1);
+                issue_v(0);
+                if (p.has_g) issue_g(0);
+                for (int i = 0; i < nchunks; ++i) {
+                    // the state MMA of chunk i is the last reader of its Q/K stage and of V
+                    if (!mbar_wait(bar(BST), i & 1, p.status, abort_flag)) break;
+                    if (i + 2 < nchunks) issue_qk(i + 2);
+                    if (i + 1 < nchunks) issue_v(i + 1);
+                    // G of chunk i + 1, once the epilogue has read that of chunk i
+                    if (p.has_g && i + 1 < nchunks) {
+                        if (!mbar_wait(bar(BGF), i & 1, p.status, abort_flag)) break;
+                        issue_g(i + 1);
+                    }
+                }
+            }
+            if (*abort_flag) {
+                for (int x = 0; x < 2; ++x)
+                    if (last_qk[x] >= 0) mbar_wait_drain(bar(BQK + x), (last_qk[x] >> 1) & 1, kWaitCycles);
+                if (last_v >= 0) mbar_wait_drain(bar(BV), last_v & 1, kWaitCycles);
+                if (last_g >= 0) mbar_wait_drain(bar(BG), last_g & 1, kWaitCycles);
+            }
+        } else if (warp == 12 && lane == 0 && nchunks > 0) {
+            // ======================================================== MMA issuer
+            constexpr uint32_t id_kk = idesc_bf16(128, 128, false, false);   // scores, inter
+            constexpr uint32_t id_pv = idesc_bf16(128, 128, false, true);    // intra: B = V MN-major
+            constexpr uint32_t id_kv = idesc_bf16(128, 128, true, true);     // state
+            float lam = 0.f;
+            int neager = 0;         // eager chunks so far: BQT completes once per eager chunk
+            for (int i = 0; i < nchunks; ++i) {
+                const int s = i & 1;
+                const uint32_t sQ = sb + CF::OFF_Q + s * CF::TILE, sK = sb + CF::OFF_K + s * CF::TILE;
+                const uint32_t sV = sb + CF::OFF_V, sT = sb + CF::OFF_T;
+                if (!mbar_wait(bar(BQK + s), (i >> 1) & 1, p.status, abort_flag)) break;
+                const float bC = stage_bc(i)[C - 1];
+                const bool eager = (-bC - lam) > kLazyMax;
+                // scores: lazy ones take K~ (scaled before), eager ones the raw K; the
+                // score buffer is free once P of the previous chunk is out
+                if (!eager && !mbar_wait(bar(BKT + s), (i >> 1) & 1, p.status, abort_flag)) break;
+                if (i > 0 && !mbar_wait(bar(BPR), (i - 1) & 1, p.status, abort_flag)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < DK / 16; ++k) {
+                    const uint32_t off = (k >> 2) * CF::BOX + (k & 3) * 32;
+                    mma_ss(tm + CF::TM_SC, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(sK + off, 16, 1024), id_kk,
+                           k > 0);
+                }
+                mma_commit(bar(BSC));
+                // inter-chunk: O = Q T (lazy) or Q~ T (eager), once the bf16 copy of T
+                // is ready and the epilogue has taken the previous output
+                if (!mbar_wait(bar(BTC), i & 1, p.status, abort_flag)) break;
+                if (eager && !mbar_wait(bar(BQT), neager & 1, p.status, abort_flag)) break;
+                neager += eager ? 1 : 0;
+                if (i > 0 && !mbar_wait(bar(BOF), (i - 1) & 1, p.status, abort_flag)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < DK / 16; ++k) {
+                    const uint32_t off = (k >> 2) * CF::BOX + (k & 3) * 32;
+                    mma_ss(tm + CF::TM_O, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(sT + off, 16, 1024), id_kk,
+                           k > 0);
+                }
+                // intra-chunk: O += P V
+                if (!mbar_wait(bar(BPR), i & 1, p.status, abort_flag)) break;
+                if (!mbar_wait(bar(BV), i & 1, p.status, abort_flag)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < C / 16; ++k)
+                    mma_ts(tm + CF::TM_O, tm + CF::TM_P + k * 8, sdesc_sw128(sV + k * 2048, CF::BOX, 1024), id_pv, 1);
+                mma_commit(bar(BOD));
+                // state: T^T += V^T K~ (eager: K~ is scaled after the scores)
+                if (eager && !mbar_wait(bar(BKT + s), (i >> 1) & 1, p.status, abort_flag)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < C / 16; ++k)
+                    mma_ss(tm + CF::TM_T, sdesc_sw128(sV + k * 2048, CF::BOX, 1024),
+                           sdesc_sw128(sK + k * 2048, CF::BOX, 1024), id_kv, 1);
+                mma_commit(bar(BST));
+                lam = eager ? 0.f : lam + bC;
+            }
+            // every MMA this thread issued has completed before tensor memory is freed
+            mma_commit(bar(BDRAIN));
+            mbar_wait_drain(bar(BDRAIN), 0, kWaitCycles);
+        }
+    } else if (role == 2) {
+        // ============================================================ S warps
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" : : "n"(kRowsOtherRegs));
+        const int st = tid - 256;              // 0..127
+        // initial state T^T[d][k] (lane d = row): zero, a caller's S0 [k][d], or a
+        // segment's folded state [d][k]
+        {
+            uint32_t r[32];
+            for (int cb = 0; cb < 4; ++cb) {
+                if (seg > 0) {
+                    const float4* s4 = reinterpret_cast<const float4*>(
+                        p.seg_state + ((size_t)u * p.slots + (size_t)seg * p.K - 1) * DV * DK +
+                        (size_t)row * DK + cb * 32);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const float4 v = s4[j];
+                        r[4 * j] = f2u(v.x); r[4 * j + 1] = f2u(v.y); r[4 * j + 2] = f2u(v.z); r[4 * j + 3] = f2u(v.w);
+                    }
+                } else if (p.S0) {
+                    const float* src = p.S0 + (size_t)u * DK * DV + (size_t)(cb * 32) * DV + row;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) r[j] = f2u(src[(size_t)j * DV]);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) r[j] = 0u;
+                }
+                tmem_st_x32(tm + lq + CF::TM_T + cb * 32, r);
+            }
+            tmem_wait_st();
+        }
+        // K~ (or Q~) in place: 16-byte items of a [128 x 128] bf16 tile, rows scaled
+        auto scale_rows = [&](uint8_t* tile, auto factor_of_row) {
+            for (int it = st; it < C * 16; it += 128) {
+                const int r = (it >> 3) % C;
+                scale_bf16x8(tile + it * 16, factor_of_row(r));
+            }
+        };
+        float lam = 0.f;
+        for (int i = 0; i < nchunks; ++i) {
+            const int s = i & 1;
+            const float* bc = stage_bc(i);
+            uint8_t* Qp = sm + CF::OFF_Q + s * CF::TILE;
+            uint8_t* Kp = sm + CF::OFF_K + s * CF::TILE;
+            mbar_wait(bar(BQK + s), (i >> 1) & 1, p.status, abort_flag);
+            const float bC = bc[C - 1];
+            const bool eager = (-bC - lam) > kLazyMax;
+            if (!eager) {
+                scale_rows(Kp, [&](int r) { return __expf(-bc[r] - lam); });
+                fence_proxy_async_smem();
+                warp_arrive(BKT + s);
+            }
+            // bf16 copy of T^T for this chunk's inter-chunk product, once the
+            // previous state update is done (it also finished the previous
+            // inter-chunk product, the last reader of the copy); eager chunks
+            // then rescale T for their state update
+            if (i > 0) mbar_wait(bar(BST), (i - 1) & 1, p.status, abort_flag);
+            tc_fence_after();
+            const float escale = __expf(lam + bC);
+#pragma unroll 1
+            for (int cb = 0; cb < 4; ++cb) {
+                uint32_t r[32];
+                tmem_ld_x32(tm + lq + CF::TM_T + cb * 32, r);
+                tmem_wait_ld();
+                uint8_t* trow = sm + CF::OFF_T + (cb >> 1) * CF::BOX + row * 128;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int chunk = (cb & 1) * 4 + c;        // 16-byte chunk of the 128-byte row
+                    uint4 w;
+                    w.x = pack_bf16x2(u2f(r[8 * c]), u2f(r[8 * c + 1]));
+                    w.y = pack_bf16x2(u2f(r[8 * c + 2]), u2f(r[8 * c + 3]));
+                    w.z = pack_bf16x2(u2f(r[8 * c + 4]), u2f(r[8 * c + 5]));
+                    w.w = pack_bf16x2(u2f(r[8 * c + 6]), u2f(r[8 * c + 7]));
+                    *reinterpret_cast<uint4*>(trow + ((chunk ^ (row & 7)) << 4)) = w;
+                }
+                if (eager) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) r[j] = f2u(u2f(r[j]) * escale);
+                    tmem_st_x32(tm + lq + CF::TM_T + cb * 32, r);
+                }
+            }
+            tmem_wait_st();
+            fence_proxy_async_smem();
+            tc_fence_before();
+            warp_arrive(BTC);
+            if (eager) {
+                // Q~ and K~ in place, once the scores have read Q and K
+                mbar_wait(bar(BSC), i & 1, p.status, abort_flag);
+                tc_fence_after();
+                scale_rows(Qp, [&](int r) { return __expf(bc[r] + lam); });
+                scale_rows(Kp, [&](int r) { return __expf(bC - bc[r]); });
+                fence_proxy_async_smem();
+                warp_arrive(BQT);
+                warp_arrive(BKT + s);
+            }
+            lam = eager ? 0.f : lam + bC;
+        }
+        // state out: e^Lambda T
+        if (nchunks > 0) {
+            mbar_wait(bar(BST), (nchunks - 1) & 1, p.status, abort_flag);
+            tc_fence_after();
+        }
+        if (p.S_final && seg == p.P - 1) {
+            const float sc = __expf(lam);
+            float* dst = p.S_final + (size_t)u * DK * DV;
+#pragma unroll 1
+            for (int cb = 0; cb < 4; ++cb) {
+                uint32_t r[32];
+                tmem_ld_x32(tm + lq + CF::TM_T + cb * 32, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) dst[(size_t)(cb * 32 + j) * DV + row] = u2f(r[j]) * sc;
+            }
+        }
+    } else if (role == 1) {
+        // ============================================================ P warps
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" : : "n"(kRowsOtherRegs));
+        float lam = 0.f;
+        for (int i = 0; i < nchunks; ++i) {
+            const float* bc = stage_bc(i);
+            mbar_wait(bar(BSC), i & 1, p.status, abort_flag);   // the scores landed (so did Q/K and bc)
+            tc_fence_after();
+            const float bC = bc[C - 1];
+            const bool eager = (-bC - lam) > kLazyMax;
+            const float bt = bc[row];
+#pragma unroll 1
+            for (int cb = 0; cb < 4; ++cb) {
+                uint32_t pk[16];
+                if (cb <= q4) {
+                    uint32_t r[32];
+                    tmem_ld_x32(tm + lq + CF::TM_SC + cb * 32, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int s0 = cb * 32 + 2 * j;
+                        float v0 = u2f(r[2 * j]), v1 = u2f(r[2 * j + 1]);
+                        if (eager) {
+                            v0 *= __expf(fminf(bt - bc[s0], 0.f));
+                            v1 *= __expf(fminf(bt - bc[s0 + 1], 0.f));
+                        }
+                        pk[j] = pack_bf16x2(s0 <= row ? v0 : 0.f, s0 + 1 <= row ? v1 : 0.f);
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) pk[j] = 0u;
+                }
+                tmem_st_x16(tm + lq + CF::TM_P + cb * 16, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            warp_arrive(BPR);
+            lam = eager ? 0.f : lam + bC;
+        }
+    } else {
+        // ============================================================ E warps
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" : : "n"(kRowsERegs));
+        float lam = 0.f;
+        const float* bsum = p.bcum + (size_t)u * p.Npad;
+        for (int i = 0; i < nchunks; ++i) {
+            const int n0 = n_begin + i * C;
+            const float bt = bsum[n0 + row], bC = bsum[n0 + C - 1];
+            mbar_wait(bar(BOD), i & 1, p.status, abort_flag);
+            tc_fence_after();
+            float y[DV];
+#pragma unroll
+            for (int cb = 0; cb < 4; ++cb) {
+                uint32_t r[32];
+                tmem_ld_x32(tm + lq + CF::TM_O + cb * 32, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) y[cb * 32 + j] = u2f(r[j]);
+            }
+            tc_fence_before();
+            warp_arrive(BOF);              // the next inter-chunk product may overwrite O
+            const bool eager = (-bC - lam) > kLazyMax;
+            // row factor c = e^{b_t + Lambda} of a lazy chunk; y = c u
+            const float c = eager ? 1.f : __expf(bt + lam);
+            float a = c, b0 = 0.f;
+            if (p.gn) {
+                // mean of u, then the variance of y = c u from the scaled
+                // deviations c (u - mean): u itself may be as large as e^64 y
+                float s1 = 0.f;
+#pragma unroll
+                for (int j = 0; j < DV; ++j) s1 += y[j];
+                const float mean = s1 * (1.0f / DV);
+                float s2 = 0.f;
+#pragma unroll
+                for (int j = 0; j < DV; ++j) {
+                    const float dv_ = (y[j] - mean) * c;
+                    s2 = fmaf(dv_, dv_, s2);
+                }
+                a = c * rsqrtf(s2 * (1.0f / DV) + p.eps);
+                b0 = -mean * a;
+            }
+            if (p.has_g) mbar_wait(bar(BG), i & 1, p.status, abort_flag);
+            // this token's output row: 256 contiguous bytes of O, written straight
+            // to global memory (rows past the sequence's end are not written)
+            const bool live = n0 + row < n_end;
+            uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.O) +
+                                                   (((size_t)bb * p.N + n0 + row) * p.H + hh) * DV);
+#pragma unroll
+            for (int ch = 0; ch < 16; ++ch) {
+                uint4 w = make_uint4(0u, 0u, 0u, 0u);
+                if (p.has_g)
+                    w = *reinterpret_cast<const uint4*>(sm + CF::OFF_G + (ch >> 3) * CF::BOX + row * 128 +
+                                                        (((ch & 7) ^ (row & 7)) << 4));
+                uint32_t* e = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    float o0 = fmaf(y[ch * 8 + 2 * j], a, b0), o1 = fmaf(y[ch * 8 + 2 * j + 1], a, b0);
+                    if (p.gn) {
+                        const float2 g = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&e[j]));
+                        o0 *= swish_fast(g.x);
+                        o1 *= swish_fast(g.y);
+                    }
+                    e[j] = pack_bf16x2(o0, o1);
+                }
+                if (live) orow[ch] = w;
+            }
+            warp_arrive(BGF);              // the G tile may be reloaded
+            lam = eager ? 0.f : lam + bC;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tm, CF::TM_ALLOC);
+    }
 }
 
 // ---------------------------------------------------------------- host side
@@ -1233,18 +1773,57 @@ cudaError_t run_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t s) {
     }
     const int units = a.B * a.H;
     const int npad = tp.Npad;
-    const int per = kScanThreads / C;
-    cudaError_t e = launch_pdl(gate_scan_kernel, dim3(units, (npad / C + per - 1) / per), dim3(kScanThreads), 0, s,
-                               a.z, a.cu_seqlens, a.total, const_cast<float*>(tp.bcum), const_cast<float*>(tp.eblk),
-                               a.H, a.N, npad, C, a.inv_tau);
+    cudaError_t e = cudaSuccess;
+    if (a.resume) {
+        // the gate scan and the state pass ran in gret_prefill_state: shift its
+        // folded slots by the initial state, then the fused loop
+        if (tp.P > 1 && tp.S0) {
+            const int elems4 = DV * DK / 4;
+            e = launch_pdl(seg_shift_kernel, dim3(units, (elems4 + 255) / 256), dim3(256), 0, s, tp.seg_state,
+                           static_cast<const float*>(tp.seg_decay), tp.S0, tp.slots, DK, DV);
+        }
+    } else if (a.X) {
+        // gate logits from the projection z = X W_gamma, fused with the scan
+        const WsLayout w = ws_layout(a.B, a.H, a.N, a.dk, a.dv, C, a.segments, a.pieces);
+        e = launch_gate_project_tc(a, const_cast<float*>(tp.bcum), const_cast<float*>(tp.eblk), npad,
+                                   static_cast<uint8_t*>(a.workspace) + w.total, s);
+    } else {
+        int nyb = 0;
+        const dim3 sgrid = gate_scan_grid(units, npad, C, &nyb);
+        if (g_profile_gate_start) cudaEventRecord(g_profile_gate_start, s);
+        e = launch_pdl(gate_scan_kernel, sgrid, dim3(kScanThreads), 0, s, a.z, a.cu_seqlens, a.total,
+                       const_cast<float*>(tp.bcum), const_cast<float*>(tp.eblk), a.H, a.N, npad, C, a.inv_tau, nyb);
+        if (g_profile_gate_stop) cudaEventRecord(g_profile_gate_stop, s);
+    }
     if (e != cudaSuccess) return e;
-    if (tp.P > 1) {
-        e = launch_pdl(ks, dim3(units * (tp.P - 1) * tp.K), dim3(kStateThreads), StateCfg<DV, C>::SMEM, s, tp);
+    if (tp.P > 1 && !a.resume) {
+        e = launch_pdl(ks, dim3(units * tp.slots), dim3(kStateThreads), StateCfg<DV, C>::SMEM, s, tp);
         if (e != cudaSuccess) return e;
         const int elems4 = DV * DK / 4;
-        e = launch_pdl(seg_combine_kernel, dim3((elems4 + 255) / 256, units), dim3(256), 0, s, tp.seg_state,
-                       static_cast<const float*>(tp.seg_decay), tp.S0, (tp.P - 1) * tp.K, DK, DV);
+        e = launch_pdl(seg_combine_kernel, dim3(units, (elems4 + 255) / 256), dim3(256), 0, s, tp.seg_state,
+                       static_cast<const float*>(tp.seg_decay), tp.S0, tp.slots, DK, DV);
         if (e != cudaSuccess) return e;
+    }
+#ifndef GRET_ROWS_KERNEL
+#define GRET_ROWS_KERNEL 1
+#endif
+    if constexpr (DV == 128 && C == 128 && !PACKED && GRET_ROWS_KERNEL) {
+        // 128-token chunks with d_v 128: the output-rows kernel
+        auto kr = prefill_rows_kernel;
+        static bool rows_attr_done[64] = {};
+        if (dev < 0 || dev >= 64 || !rows_attr_done[dev]) {
+            cudaFuncAttributes fa;
+            if (cudaFuncGetAttributes(&fa, kr) != cudaSuccess) return cudaErrorInvalidDeviceFunction;
+            if (fa.numRegs * kRowsThreads < 128 * kRowsERegs + 384 * kRowsOtherRegs)
+                return cudaErrorInvalidConfiguration;
+            cudaFuncSetAttribute(kr, cudaFuncAttributeMaxDynamicSharedMemorySize, RowsCfg::SMEM);
+            if (dev >= 0 && dev < 64) rows_attr_done[dev] = true;
+        }
+        if (g_profile_start) cudaEventRecord(g_profile_start, s);
+        e = launch_pdl(kr, dim3(units * tp.P), dim3(kRowsThreads), RowsCfg::SMEM, s, tp);
+        if (g_profile_stop) cudaEventRecord(g_profile_stop, s);
+        if (e != cudaSuccess) return e;
+        return cudaGetLastError();
     }
     if (g_profile_start) cudaEventRecord(g_profile_start, s);
     e = launch_pdl(kf, dim3(units * tp.P), dim3(kFusedThreads), CF::SMEM, s, tp);
@@ -1288,19 +1867,26 @@ int prefill_tc_launches(int segments, int pieces) {
     return segments <= 1 ? 2 : 4;
 }
 
-// State-only pass: the whole slice is one segment, cut into K pieces (about
-// one CTA per SM; K divides the chunk count).
-static int state_pass_pieces(int B, int H, int N, int chunk, int num_sms) {
+// State-only pass (gret_prefill_state): it follows the prefill's own plan --
+// P segments of seg_len tokens -- and cuts every segment into the same number
+// of pieces (about one CTA per SM; the count divides the segment's chunks),
+// so that a prefill resumed on the same tokens (gret_prefill_resume) finds the
+// state before each of its segments among the folded pieces.
+int prefill_tc_state_pieces(int B, int H, int chunk, int num_sms, int segments, int seg_len) {
     const int units = B * H > 0 ? B * H : 1;
-    const int nchunks = (N + chunk - 1) / chunk;
-    const int kmax = num_sms / units > 1 ? num_sms / units : 1;
-    for (int k = kmax < nchunks ? kmax : nchunks; k >= 1; --k)
-        if (nchunks % k == 0) return k;
+    const int per = seg_len / chunk;
+    int kmax = num_sms / (units * (segments > 0 ? segments : 1));
+    if (kmax < 1) kmax = 1;
+    for (int k = kmax < per ? kmax : per; k >= 1; --k)
+        if (per % k == 0) return k;
     return 1;
 }
 
 size_t prefill_tc_state_workspace_bytes(int B, int H, int N, int dk, int dv, int chunk, int num_sms) {
-    return ws_layout(B, H, N, dk, dv, chunk, 2, state_pass_pieces(B, H, N, chunk, num_sms)).total;
+    int P = 1, seg_len = N, K = 1;
+    prefill_tc_plan(B, H, N, chunk, num_sms, &P, &seg_len, &K);
+    const int Ks = prefill_tc_state_pieces(B, H, chunk, num_sms, P, seg_len);
+    return ws_layout(B, H, N, dk, dv, chunk, P + 1, Ks).total;
 }
 
 size_t prefill_tc_workspace_bytes(int B, int H, int N, int dk, int dv, int chunk, int segments, int pieces) {
@@ -1321,7 +1907,9 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
     tp.cu = a.cu_seqlens;
     tp.total = a.total;
     tp.O = a.O;
-    const WsLayout w = ws_layout(a.B, a.H, a.N, a.dk, a.dv, C, a.segments, a.pieces);
+    // a resumed prefill reads the layout gret_prefill_state wrote: a slot for
+    // every piece of every segment
+    const WsLayout w = ws_layout(a.B, a.H, a.N, a.dk, a.dv, C, a.segments + (a.resume ? 1 : 0), a.pieces);
     uint8_t* ws = static_cast<uint8_t*>(a.workspace);
     tp.bcum = reinterpret_cast<const float*>(ws + w.bcum);
     tp.eblk = reinterpret_cast<const float*>(ws + w.eblk);
@@ -1337,9 +1925,11 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
     tp.seg_len = a.seg_len;
     tp.K = a.pieces;
     tp.piece_len = a.seg_len / a.pieces;
+    tp.slots = (a.segments - (a.resume ? 0 : 1)) * a.pieces;
     tp.eps = a.eps;
     tp.gn = a.epi == GRET_EPI_GN_SWISH ? 1 : 0;
     tp.has_g = (a.epi == GRET_EPI_GN_SWISH && a.G) ? 1 : 0;
+    tp.fault = a.fault;
     const bool packed = a.cu_seqlens != nullptr;
     if (a.dv == 256 && C == 64) return packed ? run_tc<256, 64, true>(a, tp, s) : run_tc<256, 64, false>(a, tp, s);
     if (a.dv == 128 && C == 128) return packed ? run_tc<128, 128, true>(a, tp, s) : run_tc<128, 128, false>(a, tp, s);
@@ -1352,19 +1942,22 @@ static cudaError_t run_state_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t
     auto ks = prefill_state_kernel<DV, C, false>;
     cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, StateCfg<DV, C>::SMEM);
     const int units = a.B * a.H;
-    const int per = kScanThreads / C;
-    cudaError_t e = launch_pdl(gate_scan_kernel, dim3(units, (tp.Npad / C + per - 1) / per), dim3(kScanThreads), 0, s,
+    int nyb = 0;
+    const dim3 sgrid = gate_scan_grid(units, tp.Npad, C, &nyb);
+    cudaError_t e = launch_pdl(gate_scan_kernel, sgrid, dim3(kScanThreads), 0, s,
                                a.z, static_cast<const int*>(nullptr), 0, const_cast<float*>(tp.bcum),
-                               const_cast<float*>(tp.eblk), a.H, a.N, tp.Npad, C, a.inv_tau);
+                               const_cast<float*>(tp.eblk), a.H, a.N, tp.Npad, C, a.inv_tau, nyb);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(ks, dim3(units * tp.K), dim3(kStateThreads), StateCfg<DV, C>::SMEM, s, tp);
+    e = launch_pdl(ks, dim3(units * tp.slots), dim3(kStateThreads), StateCfg<DV, C>::SMEM, s, tp);
     if (e != cudaSuccess) return e;
+    // fold every piece from the zero state, in place: slot j becomes the
+    // increment from the slice's start through piece j
     const int elems4 = DV * DK / 4;
-    e = launch_pdl(seg_combine_kernel, dim3((elems4 + 255) / 256, units), dim3(256), 0, s, tp.seg_state,
-                   static_cast<const float*>(tp.seg_decay), static_cast<const float*>(nullptr), tp.K, DK, DV);
+    e = launch_pdl(seg_combine_kernel, dim3(units, (elems4 + 255) / 256), dim3(256), 0, s, tp.seg_state,
+                   static_cast<const float*>(tp.seg_decay), static_cast<const float*>(nullptr), tp.slots, DK, DV);
     if (e != cudaSuccess) return e;
-    state_finish_kernel<DV><<<dim3(DV / 32, DK / 32, units), dim3(32, 8), 0, s>>>(tp.seg_state, tp.seg_decay, tp.K,
-                                                                             a.S_final, a.decay_out);
+    state_finish_kernel<DV><<<dim3(units, (DV / 32) * (DK / 32)), dim3(32, 8), 0, s>>>(tp.seg_state, tp.seg_decay,
+                                                                                  tp.slots, a.S_final, a.decay_out);
     return cudaGetLastError();
 }
 
@@ -1375,8 +1968,10 @@ cudaError_t launch_prefill_state_tc(const PrefillArgs& a, int num_sms, cudaStrea
     if (!make_map(&tp.tmK, a.K, DK, a.H, a.N, a.B, C) || !make_map(&tp.tmV, a.V, a.dv, a.H, a.N, a.B, C))
         return cudaErrorInvalidValue;
     const int nchunks = (a.N + C - 1) / C;
-    const int K = state_pass_pieces(a.B, a.H, a.N, C, num_sms);
-    const WsLayout w = ws_layout(a.B, a.H, a.N, a.dk, a.dv, C, 2, K);
+    int P = 1, seg_len = a.N, Kp = 1;
+    prefill_tc_plan(a.B, a.H, a.N, C, num_sms, &P, &seg_len, &Kp);
+    const int K = prefill_tc_state_pieces(a.B, a.H, C, num_sms, P, seg_len);
+    const WsLayout w = ws_layout(a.B, a.H, a.N, a.dk, a.dv, C, P + 1, K);
     uint8_t* ws = static_cast<uint8_t*>(a.workspace);
     tp.bcum = reinterpret_cast<const float*>(ws + w.bcum);
     tp.eblk = reinterpret_cast<const float*>(ws + w.eblk);
@@ -1386,10 +1981,11 @@ cudaError_t launch_prefill_state_tc(const PrefillArgs& a, int num_sms, cudaStrea
     tp.H = a.H;
     tp.N = a.N;
     tp.Npad = nchunks * C;
-    tp.P = 2;                      // the state kernel runs over the first P - 1 = 1 segment: all of it
-    tp.seg_len = nchunks * C;
+    tp.P = P;
+    tp.seg_len = seg_len;
     tp.K = K;
-    tp.piece_len = tp.seg_len / K;
+    tp.piece_len = seg_len / K;
+    tp.slots = P * K;              // every piece of every segment
     if (a.dv == 256 && C == 64) return run_state_tc<256, 64>(a, tp, s);
     if (a.dv == 128 && C == 128) return run_state_tc<128, 128>(a, tp, s);
     if (a.dv == 128 && C == 64) return run_state_tc<128, 64>(a, tp, s);
@@ -1399,7 +1995,7 @@ cudaError_t launch_prefill_state_tc(const PrefillArgs& a, int num_sms, cudaStrea
 cudaError_t launch_state_fold(const float* dS_all, const float* decay_all, int num_slices, int slice,
                               const float* S0, float* S_in, int units, int elems, cudaStream_t s) {
     (void)num_slices;
-    state_fold_kernel<<<dim3((elems + 255) / 256, units), 256, 0, s>>>(dS_all, decay_all, slice, S0, S_in, units,
+    state_fold_kernel<<<dim3(units, (elems + 255) / 256), 256, 0, s>>>(dS_all, decay_all, slice, S0, S_in, units,
                                                                       elems);
     return cudaGetLastError();
 }

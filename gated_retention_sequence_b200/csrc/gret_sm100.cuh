@@ -62,6 +62,35 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigne
     return true;
 }
 
+// Wait for the phase of the given parity with a budget of `cycles`, whatever
+// the abort flag says: the give-up path uses it to let the asynchronous work a
+// role has already issued (TMA loads, MMAs) land before the CTA frees its
+// tensor memory and exits.  Returns false if the budget ran out.
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, long long cycles) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - t0 > cycles) return false;
+    }
+    return true;
+}
+
+// A wait that the caller knows cannot be satisfied (a barrier nothing arrives
+// at), with a short budget: it runs out, sets the status word and the abort
+// flag exactly as a real timeout does.  Used only when a test asks for it.
+__device__ __forceinline__ void mbar_wait_injected_timeout(uint32_t bar, unsigned int* status,
+                                                           volatile int* abort_flag) {
+    constexpr long long kInjectedBudget = 1LL << 20;   // about 0.5 ms
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, 0)) {
+        if (clock64() - t0 > kInjectedBudget) {
+            atomicExch(status, kDevTimeout);
+            *abort_flag = 1;
+            return;
+        }
+    }
+}
+
 // ---------------------------------------------------------------- fences
 // Programmatic dependent launch.  grid_dep_wait: block until the grid this one
 // was launched behind has completed and its writes are visible (returns at once
@@ -104,6 +133,22 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* tmap, int 
         "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, int c0, int c1, int c2, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int c0, int c1, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(bar)
         : "memory");
 }
 

@@ -61,6 +61,8 @@ SIGNATURES = {
                                   _I, _VP]),
     "gret_prefill_from_state": (_I, [_VP, _VP, _VP, _FP, _VP, _FP, _F, _I, _VP, _FP, _I, _I, _I, _I, _I, _I,
                                      _F, _I, _VP, _SZ, _VP]),
+    "gret_prefill_resume": (_I, [_VP, _VP, _VP, _FP, _VP, _FP, _F, _I, _VP, _FP, _I, _I, _I, _I, _I, _I,
+                                 _F, _I, _VP, _SZ, _VP]),
     "gret_prefill_state_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
     "gret_prefill_state": (_I, [_VP, _VP, _FP, _F, _I, _FP, _FP, _I, _I, _I, _I, _I, _I, _VP, _SZ, _VP]),
     "gret_state_fold": (_I, [_FP, _FP, _I, _I, _FP, _FP, _I, _I, _I, _I, _VP]),
@@ -76,6 +78,11 @@ SIGNATURES = {
     "gret_decode_step": (_I, [_VP, _VP, _VP, _FP, _VP, _FP, _VP, _I, _I, _I, _I, _F, _I, _F, _I, _VP]),
     "gret_last_device_status": (_I, [_VP]),
     "gret_set_profile_events": (None, [_VP, _VP]),
+    "gret_debug_inject_timeout": (None, [_I]),
+    "gret_set_gate_profile_events": (None, [_VP, _VP]),
+    "gret_prefill_projected": (_I, [_VP, _VP, _VP, _VP, _FP, _I, _VP, _F, _I, _VP, _FP, _I, _I, _I, _I, _I, _I,
+                                    _F, _I, _VP, _SZ, _VP]),
+    "gret_prefill_projected_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "gret_status_string": (ctypes.c_char_p, [_I]),
     "gret_version": (_I, []),
 }
@@ -108,6 +115,12 @@ def gret_prefill_from_state(Q, K, V, gate_logits, G, S0, tau, chunk, O, S_final,
                             eps, epi, workspace, workspace_bytes, stream) -> int:
     return load().gret_prefill_from_state(Q, K, V, gate_logits, G, S0, tau, chunk, O, S_final, B, H, N, dk, dv,
                                           int(io_dtype), eps, int(epi), workspace, workspace_bytes, stream)
+
+
+def gret_prefill_resume(Q, K, V, gate_logits, G, S0, tau, chunk, O, S_final, B, H, N, dk, dv, io_dtype,
+                        eps, epi, workspace, workspace_bytes, stream) -> int:
+    return load().gret_prefill_resume(Q, K, V, gate_logits, G, S0, tau, chunk, O, S_final, B, H, N, dk, dv,
+                                      int(io_dtype), eps, int(epi), workspace, workspace_bytes, stream)
 
 
 def gret_prefill_varlen(Q, K, V, gate_logits, G, S0, cu_seqlens, num_seqs, total_tokens, max_seqlen, tau, chunk,
@@ -180,6 +193,24 @@ def gret_set_profile_events(start, stop) -> None:
     load().gret_set_profile_events(start, stop)
 
 
+def gret_debug_inject_timeout(calls: int) -> None:
+    load().gret_debug_inject_timeout(int(calls))
+
+
+def gret_set_gate_profile_events(start, stop) -> None:
+    load().gret_set_gate_profile_events(start, stop)
+
+
+def gret_prefill_projected(Q, K, V, X, W_gamma, d_model, G, tau, chunk, O, S_final, B, H, N, dk, dv, io_dtype, eps,
+                           epi, workspace, workspace_bytes, stream) -> int:
+    return load().gret_prefill_projected(Q, K, V, X, W_gamma, d_model, G, tau, chunk, O, S_final, B, H, N, dk, dv,
+                                         int(io_dtype), eps, int(epi), workspace, workspace_bytes, stream)
+
+
+def gret_prefill_projected_workspace_size(B, H, N, dk, dv, chunk, d_model, io_dtype) -> int:
+    return load().gret_prefill_projected_workspace_size(B, H, N, dk, dv, chunk, d_model, int(io_dtype))
+
+
 def gret_status_string(status: int) -> str:
     return load().gret_status_string(int(status)).decode()
 
@@ -207,6 +238,28 @@ def _ptr(t) -> Optional[int]:
     return None if t is None else t.data_ptr()
 
 
+def _scratch(workspace, ws_bytes, dev, st):
+    """The caller's workspace when it is large enough, else a new one from
+    torch's allocator.  A new one is allocated on the current stream but used
+    by kernels on ``st``; it is dropped when the call returns, so it is
+    recorded on ``st`` to keep the caching allocator from handing its memory
+    out again before those kernels finish."""
+    torch = _torch()
+    if not ws_bytes:
+        return workspace
+    if workspace is not None and workspace.numel() * workspace.element_size() >= ws_bytes:
+        return workspace
+    workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    if st != torch.cuda.current_stream(dev):
+        workspace.record_stream(st)
+    return workspace
+
+
+def _need_g(G, epi, name="G"):
+    if epi == Epilogue.GN_SWISH and G is None:
+        raise ValueError(f"{name} is required for epilogue 'gn_swish' (pass epilogue='none' for the pre-norm Y)")
+
+
 def _check(t, name, dtype, shape, device):
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
@@ -221,8 +274,12 @@ def _check(t, name, dtype, shape, device):
 
 
 def prefill(Q, K, V, z, G, tau: float, chunk: int, eps: float = 1e-5, epilogue: str = "gn_swish",
-            O=None, S_final=None, want_state: bool = True, workspace=None, stream=None, S0=None):
+            O=None, S_final=None, want_state: bool = True, workspace=None, stream=None, S0=None,
+            resume: bool = False):
     """Chunkwise prefill from the zero state, or from ``S0`` (gret_prefill_from_state).
+
+    ``resume=True`` (gret_prefill_resume) reuses the decay sums and state-pass
+    pieces that ``prefill_state`` left in ``workspace`` for the same K, V, z.
 
     Q, K [B,N,H,dk] and V, G [B,N,H,dv] in bf16 or fp32; z [B,N,H] fp32 gate logits;
     S0 [B,H,dk,dv] fp32 or None.
@@ -235,11 +292,12 @@ def prefill(Q, K, V, z, G, tau: float, chunk: int, eps: float = 1e-5, epilogue: 
     dev = Q.device
     io = _io_of(Q)
     epi = Epilogue.NONE if epilogue == "none" else Epilogue.GN_SWISH
+    _need_g(G, epi)
     _check(Q, "Q", Q.dtype, (B, N, H, dk), dev)
     _check(K, "K", Q.dtype, (B, N, H, dk), dev)
     _check(V, "V", Q.dtype, (B, N, H, dv), dev)
     _check(z, "z", torch.float32, (B, N, H), dev)
-    if epi == Epilogue.GN_SWISH or G is not None:
+    if G is not None:
         _check(G, "G", Q.dtype, (B, N, H, dv), dev)
     if O is None:
         O = torch.empty((B, N, H, dv), dtype=Q.dtype, device=dev)
@@ -250,13 +308,21 @@ def prefill(Q, K, V, z, G, tau: float, chunk: int, eps: float = 1e-5, epilogue: 
         _check(S_final, "S_final", torch.float32, (B, H, dk, dv), dev)
     if S0 is not None:
         _check(S0, "S0", torch.float32, (B, H, dk, dv), dev)
+    if resume and workspace is None:
+        raise ValueError("resume=True needs the workspace prefill_state wrote")
     with torch.cuda.device(dev):
-        ws_bytes = gret_prefill_workspace_size(B, H, N, dk, dv, chunk, io)
-        if ws_bytes and (workspace is None or workspace.numel() * workspace.element_size() < ws_bytes):
-            workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        ws_bytes = (gret_prefill_state_workspace_size if resume else gret_prefill_workspace_size)(
+            B, H, N, dk, dv, chunk, io)
         st = stream if stream is not None else torch.cuda.current_stream(dev)
+        if resume and ws_bytes and workspace.numel() * workspace.element_size() < ws_bytes:
+            raise ValueError("the workspace is smaller than gret_prefill_state_workspace_size")
+        workspace = _scratch(workspace, ws_bytes, dev, st)
         ws = _ptr(workspace) if ws_bytes else None
-        if S0 is None:
+        if resume:
+            status = gret_prefill_resume(_ptr(Q), _ptr(K), _ptr(V), _ptr(z), _ptr(G), _ptr(S0), float(tau),
+                                         int(chunk), _ptr(O), _ptr(S_final), B, H, N, dk, dv, io, float(eps), epi,
+                                         ws, ws_bytes, st.cuda_stream)
+        elif S0 is None:
             status = gret_prefill(_ptr(Q), _ptr(K), _ptr(V), _ptr(z), _ptr(G), float(tau), int(chunk),
                                   _ptr(O), _ptr(S_final), B, H, N, dk, dv, io, float(eps), epi, ws, ws_bytes,
                                   st.cuda_stream)
@@ -265,7 +331,48 @@ def prefill(Q, K, V, z, G, tau: float, chunk: int, eps: float = 1e-5, epilogue: 
                                              int(chunk), _ptr(O), _ptr(S_final), B, H, N, dk, dv, io,
                                              float(eps), epi, ws, ws_bytes, st.cuda_stream)
     if status != Status.OK:
-        raise GretError(status, "gret_prefill" if S0 is None else "gret_prefill_from_state")
+        raise GretError(status, "gret_prefill_resume" if resume else
+                        "gret_prefill" if S0 is None else "gret_prefill_from_state")
+    return O, S_final
+
+
+def prefill_projected(Q, K, V, X, W_gamma, G, tau: float, chunk: int, eps: float = 1e-5, epilogue: str = "gn_swish",
+                      O=None, S_final=None, want_state: bool = True, workspace=None, stream=None):
+    """Prefill with the gate logits computed from z = X W_gamma (gret_prefill_projected).
+
+    Q, K [B,N,H,dk]; V, G [B,N,H,dv]; X [B,N,d_model] (all bf16 or all fp32);
+    W_gamma [d_model,H] fp32.  Returns (O, S_final) as ``prefill`` does."""
+    torch = _torch()
+    B, N, H, dk = Q.shape
+    dv = V.shape[-1]
+    d_model = X.shape[-1]
+    dev = Q.device
+    io = _io_of(Q)
+    epi = Epilogue.NONE if epilogue == "none" else Epilogue.GN_SWISH
+    _need_g(G, epi)
+    _check(K, "K", Q.dtype, (B, N, H, dk), dev)
+    _check(V, "V", Q.dtype, (B, N, H, dv), dev)
+    _check(X, "X", Q.dtype, (B, N, d_model), dev)
+    _check(W_gamma, "W_gamma", torch.float32, (d_model, H), dev)
+    if G is not None:
+        _check(G, "G", Q.dtype, (B, N, H, dv), dev)
+    if O is None:
+        O = torch.empty((B, N, H, dv), dtype=Q.dtype, device=dev)
+    _check(O, "O", Q.dtype, (B, N, H, dv), dev)
+    if S_final is None and want_state:
+        S_final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    if S_final is not None:
+        _check(S_final, "S_final", torch.float32, (B, H, dk, dv), dev)
+    with torch.cuda.device(dev):
+        ws_bytes = gret_prefill_projected_workspace_size(B, H, N, dk, dv, chunk, d_model, io)
+        st = stream if stream is not None else torch.cuda.current_stream(dev)
+        workspace = _scratch(workspace, ws_bytes, dev, st)
+        status = gret_prefill_projected(_ptr(Q), _ptr(K), _ptr(V), _ptr(X), _ptr(W_gamma), d_model, _ptr(G),
+                                        float(tau), int(chunk), _ptr(O), _ptr(S_final), B, H, N, dk, dv, io,
+                                        float(eps), epi, _ptr(workspace) if ws_bytes else None, ws_bytes,
+                                        st.cuda_stream)
+    if status != Status.OK:
+        raise GretError(status, "gret_prefill_projected")
     return O, S_final
 
 
@@ -285,12 +392,13 @@ def prefill_varlen(Q, K, V, z, G, cu_seqlens, max_seqlen: int, tau: float, chunk
     dev = Q.device
     io = _io_of(Q)
     epi = Epilogue.NONE if epilogue == "none" else Epilogue.GN_SWISH
+    _need_g(G, epi)
     _check(Q, "Q", Q.dtype, (T, H, dk), dev)
     _check(K, "K", Q.dtype, (T, H, dk), dev)
     _check(V, "V", Q.dtype, (T, H, dv), dev)
     _check(z, "z", torch.float32, (T, H), dev)
     _check(cu_seqlens, "cu_seqlens", torch.int32, (S + 1,), dev)
-    if epi == Epilogue.GN_SWISH or G is not None:
+    if G is not None:
         _check(G, "G", Q.dtype, (T, H, dv), dev)
     if O is None:
         O = torch.empty((T, H, dv), dtype=Q.dtype, device=dev)
@@ -303,9 +411,8 @@ def prefill_varlen(Q, K, V, z, G, cu_seqlens, max_seqlen: int, tau: float, chunk
         _check(S0, "S0", torch.float32, (S, H, dk, dv), dev)
     with torch.cuda.device(dev):
         ws_bytes = gret_prefill_workspace_size(S, H, max_seqlen, dk, dv, chunk, io)
-        if ws_bytes and (workspace is None or workspace.numel() * workspace.element_size() < ws_bytes):
-            workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
         st = stream if stream is not None else torch.cuda.current_stream(dev)
+        workspace = _scratch(workspace, ws_bytes, dev, st)
         status = gret_prefill_varlen(_ptr(Q), _ptr(K), _ptr(V), _ptr(z), _ptr(G), _ptr(S0), _ptr(cu_seqlens), S, T,
                                      int(max_seqlen), float(tau), int(chunk), _ptr(O), _ptr(S_final), H, dk, dv, io,
                                      float(eps), epi, _ptr(workspace) if ws_bytes else None, ws_bytes,
@@ -331,9 +438,8 @@ def prefill_state(K, V, z, tau: float, chunk: int, workspace=None, stream=None):
     decay = torch.empty((B, H), dtype=torch.float32, device=dev)
     with torch.cuda.device(dev):
         ws_bytes = gret_prefill_state_workspace_size(B, H, N, dk, dv, chunk, io)
-        if ws_bytes and (workspace is None or workspace.numel() * workspace.element_size() < ws_bytes):
-            workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
         st = stream if stream is not None else torch.cuda.current_stream(dev)
+        workspace = _scratch(workspace, ws_bytes, dev, st)
         status = gret_prefill_state(_ptr(K), _ptr(V), _ptr(z), float(tau), int(chunk), _ptr(dS), _ptr(decay), B, H,
                                     N, dk, dv, io, _ptr(workspace) if ws_bytes else None, ws_bytes, st.cuda_stream)
     if status != Status.OK:
@@ -377,6 +483,7 @@ def prefill_backward(Q, K, V, z, G, dO, tau: float, eps: float = 1e-5, epilogue:
     dev = Q.device
     io = _io_of(Q)
     epi = Epilogue.NONE if epilogue == "none" else Epilogue.GN_SWISH
+    _need_g(G, epi)
     for t, name, shape in ((K, "K", (B, N, H, dk)), (V, "V", (B, N, H, dv)), (dO, "dO", (B, N, H, dv))):
         _check(t, name, Q.dtype, shape, dev)
     _check(z, "z", torch.float32, (B, N, H), dev)
@@ -391,9 +498,8 @@ def prefill_backward(Q, K, V, z, G, dO, tau: float, eps: float = 1e-5, epilogue:
            else None}
     with torch.cuda.device(dev):
         ws_bytes = gret_prefill_backward_workspace_size(B, H, N, dk, dv, io)
-        if ws_bytes and (workspace is None or workspace.numel() * workspace.element_size() < ws_bytes):
-            workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
         st = stream if stream is not None else torch.cuda.current_stream(dev)
+        workspace = _scratch(workspace, ws_bytes, dev, st)
         status = gret_prefill_backward(_ptr(Q), _ptr(K), _ptr(V), _ptr(z), _ptr(G), _ptr(S0), _ptr(dO), _ptr(dS_final),
                                        float(tau), float(eps), epi, _ptr(out["dQ"]), _ptr(out["dK"]), _ptr(out["dV"]),
                                        _ptr(out["dz"]), _ptr(out["dG"]), _ptr(out["dS0"]), B, H, N, dk, dv, io,
@@ -412,11 +518,12 @@ def decode_step(q, k, v, z, g, S, tau: float, eps: float = 1e-5, epilogue: str =
     dev = q.device
     io = _io_of(q)
     epi = Epilogue.NONE if epilogue == "none" else Epilogue.GN_SWISH
+    _need_g(g, epi, "g")
     _check(q, "q", q.dtype, (ns, H, dk), dev)
     _check(k, "k", q.dtype, (ns, H, dk), dev)
     _check(v, "v", q.dtype, (ns, H, dv), dev)
     _check(z, "z", torch.float32, (ns, H), dev)
-    if epi == Epilogue.GN_SWISH or g is not None:
+    if g is not None:
         _check(g, "g", q.dtype, (ns, H, dv), dev)
     _check(S, "S", torch.float32, (ns, H, dk, dv), dev)
     if o is None:

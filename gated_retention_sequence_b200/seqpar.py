@@ -12,7 +12,9 @@ exchange step:
 3. every rank folds the slices before it into its initial state
    (``state_fold``: S_in(r) = e^{a_{r-1}} S_in(r-1) + dS_{r-1}, S_in(0) = S0);
 4. every rank runs the prefill of its slice from S_in(r)
-   (``prefill`` with ``S0``).
+   (``prefill`` with ``S0`` and ``resume``: the decay sums and state pieces
+   of step 1 are taken from its workspace, so the slice's K and V are read by
+   one state pass, as in a prefill on one device).
 
 The last rank's final state is the state after the whole sequence.  The
 collectives are torch.distributed calls (NCCL over NVLink on GPUs); every
@@ -23,14 +25,20 @@ from __future__ import annotations
 
 
 class LibraryOps:
-    """The three computing steps as libgret calls (CUDA tensors)."""
+    """The three computing steps as libgret calls (CUDA tensors).  The state
+    pass's workspace is kept for the prefill of the same slice."""
 
     def __init__(self, workspace=None):
         self.workspace = workspace
 
     def state(self, K, V, z, tau, chunk):
-        from .gret import prefill_state
-        return prefill_state(K, V, z, tau, chunk)
+        from .gret import gret_prefill_state_workspace_size, prefill_state, _io_of
+        import torch
+        B, N, H, dk = K.shape
+        need = gret_prefill_state_workspace_size(B, H, N, dk, V.shape[-1], chunk, _io_of(K))
+        if self.workspace is None or self.workspace.numel() * self.workspace.element_size() < need:
+            self.workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=K.device)
+        return prefill_state(K, V, z, tau, chunk, workspace=self.workspace)
 
     def fold(self, dS_all, decay_all, rank, S0):
         from .gret import state_fold
@@ -38,7 +46,7 @@ class LibraryOps:
 
     def prefill_from(self, Q, K, V, z, G, tau, chunk, eps, S_in):
         from .gret import prefill
-        return prefill(Q, K, V, z, G, tau, chunk, eps=eps, S0=S_in, workspace=self.workspace)
+        return prefill(Q, K, V, z, G, tau, chunk, eps=eps, S0=S_in, workspace=self.workspace, resume=True)
 
 
 def prefill_sequence_parallel(Q, K, V, z, G, tau: float, chunk: int, eps: float = 1e-5, S0=None, group=None,

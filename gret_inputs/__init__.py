@@ -213,14 +213,16 @@ def prefill_inputs(cfg: PrefillConfig, tid_base: int = 0) -> Dict[str, torch.Ten
     return out
 
 
-def prefill_unit_inputs(cfg: PrefillConfig, b: int, h: int, tid_base: int = 0) -> Dict[str, torch.Tensor]:
+def prefill_unit_inputs(cfg: PrefillConfig, b: int, h: int, tid_base: int = 0,
+                        tokens: Optional[int] = None) -> Dict[str, torch.Tensor]:
     """The slice of prefill_inputs(cfg) for one (batch, head) unit, drawn on its own.
 
-    Returns Q, K [N,dk]; V, G [N,dv] in cfg.io and z [N] fp32, element-identical to
-    ``prefill_inputs(cfg)[name][b, :, h]``.
+    Returns Q, K [T,dk]; V, G [T,dv] in cfg.io and z [T] fp32, element-identical to
+    ``prefill_inputs(cfg)[name][b, :T, h]``, with T = tokens (default: all N).
     """
     B, N, H, dk, dv = cfg.B, cfg.N, cfg.H, cfg.dk, cfg.dv
-    n = np.arange(N, dtype=np.int64)[:, None]
+    T = N if tokens is None else min(int(tokens), N)
+    n = np.arange(T, dtype=np.int64)[:, None]
     sd = math.sqrt(cfg.qkv_var)
 
     def idx(d):
@@ -231,9 +233,9 @@ def prefill_unit_inputs(cfg: PrefillConfig, b: int, h: int, tid_base: int = 0) -
                                      ("V", TID_V, dv, 0.0, sd),
                                      ("G", TID_G, dv, cfg.g_dist[0], math.sqrt(cfg.g_dist[1]))):
         v = mean + std * standard_normal_at(cfg.seed, tid_base + tid, idx(d))
-        out[name] = to_storage(v, cfg.io).view(N, d)
+        out[name] = to_storage(v, cfg.io).view(T, d)
     zi = ((b * N + n[:, 0]) * H + h)
-    m, s = cfg.z_mean_std(np.full(N, h))
+    m, s = cfg.z_mean_std(np.full(T, h))
     out["z"] = to_storage(m + s * standard_normal_at(cfg.seed, tid_base + TID_Z, zi), "f32")
     return out
 

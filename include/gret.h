@@ -69,7 +69,11 @@ typedef enum {
  *                             epi == GRET_EPI_NONE.
  *   tau                     : gate temperature, > 0.
  *   chunk                   : block length of the chunkwise form.  Supported:
- *                             16, 32, 64, 128 (TC path: 64 or 128).
+ *                             16, 32, 64, 128, 256 (TC path: 64 or 128; 256,
+ *                             the pages' own block size (section 5.3.8), runs
+ *                             on the CUDA-core kernel, which works through a
+ *                             chunk in blocks of rows and columns when the
+ *                             whole chunk does not fit in shared memory).
  *   O                       : output [B][N][H][dv] in io_dtype; must not alias an input.
  *   S_final                 : fp32 [B][H][dk][dv] state after the last token, or NULL.
  *   B, H, N, dk, dv         : > 0; dk, dv multiples of 16 and <= 256.
@@ -162,6 +166,27 @@ gret_status gret_prefill_state(const void* K, const void* V, const float* gate_l
                                float* dS, float* decay, int B, int H, int N, int dk, int dv,
                                gret_dtype io_dtype, void* workspace, size_t workspace_bytes,
                                gret_stream_t stream);
+
+/*
+ * gret_prefill_resume -- step 4 of a rank that ran gret_prefill_state on the
+ * same tokens: gret_prefill_from_state(Q, K, V, gate_logits, G, S0, ...) that
+ * takes the decay sums and the state pass's pieces from `workspace`, where
+ * gret_prefill_state left them, instead of computing them again.  The state
+ * pass folded its pieces from the zero state; this call adds S0 carried
+ * through each piece's decay (S(x || y) = e^{sum log gamma(y)} S(x) + S(y),
+ * the state decomposition) and runs the fused chunk loop: K, V and the gate
+ * are read once by the state pass and once here, as in a single-device
+ * prefill.  Arguments as gret_prefill_from_state; `workspace` must be the one
+ * gret_prefill_state was given (at least gret_prefill_state_workspace_size
+ * bytes) with the same K, V, gate_logits, tau, chunk, B, H, N, dk, dv and io
+ * dtype and nothing written to it in between (otherwise the result is
+ * undefined).  gate_logits is not read again.  On the CUDA-core path the call
+ * is gret_prefill_from_state.
+ */
+gret_status gret_prefill_resume(const void* Q, const void* K, const void* V, const float* gate_logits,
+                                const void* G, const float* S0, float tau, int chunk, void* O, float* S_final, int B,
+                                int H, int N, int dk, int dv, gret_dtype io_dtype, float eps, gret_epilogue epi,
+                                void* workspace, size_t workspace_bytes, gret_stream_t stream);
 
 /*
  * gret_state_fold -- step 3.  dS_all fp32 [num_slices][B][H][dk][dv] and
@@ -277,12 +302,55 @@ gret_status gret_decode_step(const void* q, const void* k, const void* v, const 
  * gave up returns early and its outputs are undefined. */
 gret_status gret_last_device_status(gret_stream_t stream);
 
+/*
+ * gret_prefill_projected -- gret_prefill whose gate logits come from the gate
+ * projection itself.
+ *
+ * "YOCO 深度技术分析", section 2.2: gamma = sigmoid(X W_gamma)^(1/tau), with one
+ * column of W_gamma per head, so z[b][n][h] = sum_i X[b][n][i] W_gamma[i][h].
+ * On the tensor-core path (bf16, as gret_prefill_path reports) with H <= 256
+ * and d_model a multiple of 8, z is a tcgen05 product inside the kernel that
+ * scans the gate (W_gamma fed as two bf16 halves for fp32-level accuracy) and
+ * never reaches memory; elsewhere a CUDA-core kernel writes z into the
+ * workspace first.  Everything else is gret_prefill.
+ *
+ *   X         [B][N][d_model] in io_dtype, the mixer's input rows
+ *   W_gamma   [d_model][H] fp32
+ *   workspace at least gret_prefill_projected_workspace_size(...) bytes
+ * Pointers must be 16-byte aligned.  Same errors as gret_prefill.
+ */
+gret_status gret_prefill_projected(const void* Q, const void* K, const void* V, const void* X,
+                                   const float* W_gamma, int d_model, const void* G, float tau, int chunk,
+                                   void* O, float* S_final, int B, int H, int N, int dk, int dv,
+                                   gret_dtype io_dtype, float eps, gret_epilogue epi, void* workspace,
+                                   size_t workspace_bytes, gret_stream_t stream);
+size_t gret_prefill_projected_workspace_size(int B, int H, int N, int dk, int dv, int chunk, int d_model,
+                                             gret_dtype io_dtype);
+
+/* Test aid for the give-up path of the bounded device waits.  The next `calls`
+ * prefill calls that run the tensor-core kernels (any gret_prefill* entry
+ * point on that path, from any host thread) make the fused kernel's TMA warp,
+ * before it issues any load, wait on an mbarrier that nothing ever arrives at,
+ * with a budget of about 2^20 cycles.  The wait runs out, the kernel records
+ * GRET_ERR_TIMEOUT in the device status word, every role of the CTA stops
+ * issuing work, the work already issued is awaited, and the kernel returns.
+ * The call's outputs are then undefined; gret_last_device_status reports
+ * GRET_ERR_TIMEOUT once and clears it, and later calls run normally.  No GPU
+ * fault, trap or hang is involved.  `calls` <= 0 cancels pending injections.
+ * Not for production use. */
+void gret_debug_inject_timeout(int calls);
+
 /* Profiling aid.  While set (non-NULL), every gret_prefill call made from the
  * calling host thread records `start` on its stream just before the launch of
  * the fused chunk-loop kernel (the dominant kernel of a prefill) and `stop`
  * just after it, so that cudaEventElapsedTime gives that kernel's duration.
  * Both are cudaEvent_t handles owned by the caller; pass NULL, NULL to stop. */
 void gret_set_profile_events(void* start, void* stop);
+
+/* The same for the gate prologue of a prefill (the gate scan, or on the
+ * tensor-core path of gret_prefill_projected the fused projection and scan;
+ * the CUDA-core projection of the other paths). */
+void gret_set_gate_profile_events(void* start, void* stop);
 
 /* Static, human-readable name of a status code. */
 const char* gret_status_string(gret_status status);

@@ -113,6 +113,14 @@ def test_path_selection(lib):
     assert gret.prefill_path(1, 2, 256, 64, 64, 48, gret.Dtype.F32)[0] == gret.Path.NONE
     assert gret.prefill_path(1, 2, 256, 256, 256, 128, gret.Dtype.F32)[0] == gret.Path.NONE
     assert gret.gret_prefill_workspace_size(1, 2, 256, 64, 64, 64, gret.Dtype.F32) == 0
+    # chunk 256 (the pages' block size) runs on the CUDA-core kernel, also for
+    # the benchmark's bf16 head sizes; 512 is no supported chunk
+    bf = gret.Dtype.BF16
+    assert gret.prefill_path(1, 2, 4096, 128, 128, 256, bf)[0] == gret.Path.SIMT
+    assert gret.prefill_path(1, 2, 4096, 128, 256, 256, bf)[0] == gret.Path.SIMT
+    assert gret.prefill_path(1, 2, 4096, 64, 64, 256, gret.Dtype.F32)[0] == gret.Path.SIMT
+    assert gret.prefill_path(1, 2, 4096, 64, 64, 512, gret.Dtype.F32)[0] == gret.Path.NONE
+    assert gret.prefill_path(1, 2, 4096, 128, 128, 128, bf)[0] == gret.Path.TC
 
 
 def test_backward_path_and_workspace(lib):
@@ -154,3 +162,19 @@ def test_backward_rejects_bad_arguments(lib):
         assert gret.gret_prefill_backward(**dict(a, **over)) == gret.Status.ERR_INVALID_ARG, over
     for over in (dict(dk=24), dict(dv=512)):
         assert gret.gret_prefill_backward(**dict(a, **over)) == gret.Status.ERR_UNSUPPORTED, over
+
+
+def test_python_binding_requires_g_for_gn_swish():
+    # the default epilogue needs the gate tensor G; without it the binding says
+    # so before touching any device (CPU tensors suffice for this check)
+    import torch
+    Q = torch.zeros(1, 4, 1, 16)
+    z = torch.zeros(1, 4, 1)
+    with pytest.raises(ValueError, match="G is required"):
+        gret.prefill(Q, Q, Q, z, None, 16.0, 64)
+    with pytest.raises(ValueError, match="G is required"):
+        gret.prefill_varlen(Q[0], Q[0], Q[0], z[0], None, torch.zeros(2, dtype=torch.int32), 4, 16.0, 64)
+    with pytest.raises(ValueError, match="G is required"):
+        gret.prefill_backward(Q, Q, Q, z, None, Q, 16.0)
+    with pytest.raises(ValueError, match="g is required"):
+        gret.decode_step(Q[0], Q[0], Q[0], z[0], None, torch.zeros(4, 1, 16, 16), 16.0)

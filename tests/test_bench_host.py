@@ -67,3 +67,12 @@ def test_varlen_mix():
     assert 1 in lengths                                  # a one-token sequence
     assert any(n % 64 for n in lengths)                  # ragged chunk tails
     assert bench.varlen_lengths(16384, 4096, seed=17) == lengths
+
+
+def test_projection_bytes():
+    # X rows of d_model bf16, W_gamma fp32, and two fp32 words (decay sum and
+    # P-block factor) per token and head of the padded sequence
+    cfg = gi.C2
+    d_model = 16 * 128
+    want = 4 * 4096 * d_model * 2 + d_model * 16 * 4 + 2 * 64 * 4096 * 4
+    assert bench.projection_alg(cfg, d_model) == (want, 2 * 4 * 4096 * 16 * d_model)

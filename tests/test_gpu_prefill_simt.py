@@ -58,6 +58,12 @@ def test_fp32_workload():
     (1, 1, 77, 64, 32, 32, "bf16"),     # bf16 io on the CUDA-core kernel
     (2, 2, 130, 128, 128, 16, "f32"),   # many short chunks, large heads
     (1, 2, 300, 64, 64, 128, "f32"),    # chunk larger than the remaining tail
+    # chunk 256, the pages' block size: the chunk does not fit in shared memory
+    # and is worked through in blocks of 64 or 16 rows and columns
+    (1, 2, 600, 64, 64, 256, "f32"),    # two full chunks and a ragged one
+    (1, 2, 700, 128, 128, 256, "bf16"), # the benchmark's head size, chunk 256
+    (1, 1, 300, 128, 256, 256, "bf16"), # d_v 256: blocks of 16
+    (1, 1, 200, 128, 256, 128, "bf16"), # chunk 128 with d_v 256 (no tensor-core variant)
 ])
 def test_shapes(B, H, N, dk, dv, chunk, io):
     cfg = gi.C1.scaled(B=B, H=H, N=N, dk=dk, dv=dv, chunk=chunk, io=io, seed=100 + N,

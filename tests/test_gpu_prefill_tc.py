@@ -74,18 +74,25 @@ def test_gate_stress_mixed_heads():
 
 
 def _full_workload_sampled(cfg, units):
+    """The whole workload in the benchmark's launch configuration; O, the
+    pre-norm Y (GroupNorm would hide a uniform scale error, and S_final an
+    error confined to the intra-chunk part) and S_final of sampled units
+    against the oracle run on each unit alone."""
     inp = gi.prefill_inputs(cfg)
     d = {k: v.cuda() for k, v in inp.items()}
     O, Sf = gret.prefill(d["Q"], d["K"], d["V"], d["z"], d["G"], cfg.tau, cfg.chunk, eps=cfg.eps)
+    Y, _ = gret.prefill(d["Q"], d["K"], d["V"], d["z"], None, cfg.tau, cfg.chunk, epilogue="none",
+                        want_state=False)
     gret.check_device_status()
-    assert torch.isfinite(O.float()).all() and torch.isfinite(Sf).all()
+    assert torch.isfinite(O.float()).all() and torch.isfinite(Sf).all() and torch.isfinite(Y.float()).all()
     for b, h in units:
         u = gi.prefill_unit_inputs(cfg, b, h)
         for name in ("Q", "V", "z"):
             assert torch.equal(u[name], inp[name][b, :, h])
-        O_ref, _, S_ref = oracle.prefill(u["Q"][None, :, None], u["K"][None, :, None], u["V"][None, :, None],
-                                         u["z"][None, :, None], u["G"][None, :, None], cfg.tau, cfg.eps)
+        O_ref, Y_ref, S_ref = oracle.prefill(u["Q"][None, :, None], u["K"][None, :, None], u["V"][None, :, None],
+                                             u["z"][None, :, None], u["G"][None, :, None], cfg.tau, cfg.eps)
         assert_close(O[b, :, h], O_ref[0, :, 0], "bf16", f"O unit {(b, h)}")
+        assert_close(Y[b, :, h], Y_ref[0, :, 0], "bf16", f"Y unit {(b, h)}")
         assert_close(Sf[b, h], S_ref[0, 0], "bf16", f"S unit {(b, h)}")
 
 

@@ -2,7 +2,10 @@
 
 The slices of one sequence are processed in turn on the same GPU: the
 state-only pass of each slice (gret_prefill_state), the fold of the slices
-before it (gret_state_fold), and the prefill of the slice from that state.
+before it (gret_state_fold), and the prefill of the slice from that state --
+either from scratch (gret_prefill_from_state) or resumed from the state pass's
+workspace (gret_prefill_resume), which shifts the pieces the state pass folded
+from zero by the slice's initial state.
 The concatenated outputs and the last state are compared with one oracle
 prefill of the whole sequence; the state-only pass is also compared with the
 oracle's state and decay of each slice alone.  (The all-gather between devices
@@ -26,7 +29,7 @@ def _lib():
     gret.load()
 
 
-def _run(cfg, cuts, expect_path, with_s0):
+def _run(cfg, cuts, expect_path, with_s0, resume=False):
     io = gret.Dtype.BF16 if cfg.io == "bf16" else gret.Dtype.F32
     assert gret.prefill_path(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, cfg.chunk, io)[0] == expect_path
     inp = gi.prefill_inputs(cfg)
@@ -34,7 +37,13 @@ def _run(cfg, cuts, expect_path, with_s0):
     S0 = gi.random_unit(cfg.seed, 904, (cfg.B, cfg.H, cfg.dk, cfg.dv), var=0.04) if with_s0 else None
     S0d = S0.cuda() if with_s0 else None
     sl = [{k: v[:, a:b].contiguous() for k, v in d.items()} for a, b in zip(cuts[:-1], cuts[1:])]
-    parts = [gret.prefill_state(s["K"], s["V"], s["z"], cfg.tau, cfg.chunk) for s in sl]
+    # one workspace per slice, kept for the resumed prefill of that slice
+    wss = []
+    for s in sl:
+        n = s["K"].shape[1]
+        need = gret.gret_prefill_state_workspace_size(cfg.B, cfg.H, n, cfg.dk, cfg.dv, cfg.chunk, io)
+        wss.append(torch.empty(max(need, 256), dtype=torch.uint8, device="cuda"))
+    parts = [gret.prefill_state(s["K"], s["V"], s["z"], cfg.tau, cfg.chunk, workspace=w) for s, w in zip(sl, wss)]
     gret.check_device_status()
     # the state-only pass alone, against the oracle on each slice
     for (a, b), (dS, decay) in zip(zip(cuts[:-1], cuts[1:]), parts):
@@ -47,7 +56,8 @@ def _run(cfg, cuts, expect_path, with_s0):
     outs = []
     for r, s in enumerate(sl):
         S_in = gret.state_fold(dS_all, decay_all, r, S0=S0d)
-        O, S = gret.prefill(s["Q"], s["K"], s["V"], s["z"], s["G"], cfg.tau, cfg.chunk, eps=cfg.eps, S0=S_in)
+        O, S = gret.prefill(s["Q"], s["K"], s["V"], s["z"], s["G"], cfg.tau, cfg.chunk, eps=cfg.eps, S0=S_in,
+                            workspace=wss[r] if resume else None, resume=resume)
         outs.append((O, S))
     S_whole = gret.state_fold(dS_all, decay_all, len(sl), S0=S0d)
     gret.check_device_status()
@@ -75,3 +85,17 @@ def test_tc_gate_stress():
 def test_simt_fp32():
     cfg = gi.C1.scaled(N=256, seed=64)
     _run(cfg, (0, 100, 256), gret.Path.SIMT, with_s0=True)
+
+
+@pytest.mark.parametrize("dv,chunk,N,cuts", [(256, 64, 3000, (0, 700, 1500, 3000)),
+                                             (128, 128, 2000, (0, 1000, 1130, 2000)),
+                                             (128, 64, 5000, (0, 2500, 5000))])
+def test_tc_resumed_from_the_state_pass(dv, chunk, N, cuts):
+    cfg = gi.C2.scaled(B=1, H=4, N=N, dv=dv, chunk=chunk, seed=65 + dv + chunk,
+                       z_dist=((-4.0, 1.0), (8.0, 0.5), (3.0, 1.5), (0.0, 2.0)))
+    _run(cfg, cuts, gret.Path.TC, with_s0=True, resume=True)
+
+
+def test_simt_resumed_is_from_state():
+    cfg = gi.C1.scaled(N=256, seed=66)
+    _run(cfg, (0, 100, 256), gret.Path.SIMT, with_s0=True, resume=True)

@@ -14,8 +14,10 @@ def test_unit_slice_matches_full_tensor():
     for b in range(cfg.B):
         for h in range(cfg.H):
             unit = gi.prefill_unit_inputs(cfg, b, h)
+            head = gi.prefill_unit_inputs(cfg, b, h, tokens=13)
             for name in ("Q", "K", "V", "G", "z"):
                 assert torch.equal(full[name][b, :, h], unit[name]), name
+                assert torch.equal(full[name][b, :13, h], head[name]), name
 
 
 def test_decode_unit_slice_matches_full():
