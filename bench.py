@@ -244,9 +244,12 @@ def cpu_oracle_sample(cfg, units, threads, min_seconds=0.0, tokens=None, inputs=
     return token_heads / cfg.H / dt / 1e6, dt, passes, tokens
 
 
-def config_of(name):
+def config_of(name, seq_len=0):
     import gret_inputs as gi
-    return gi.CONFIGS[name]
+    cfg = gi.CONFIGS[name]
+    if seq_len:
+        cfg = cfg.scaled(N=seq_len, name=cfg.name.replace(f"N{cfg.N}", f"N{seq_len}"))
+    return cfg
 
 
 def config_dict(cfg, **extra):
@@ -266,7 +269,7 @@ def run_reference(args, world, rank):
     import oracle
     if rank != 0:
         return 0
-    cfg = config_of(args.config)
+    cfg = config_of(args.config, args.seq_len)
     threads = oracle.default_threads()
     units = min(cfg.B * cfg.H, threads)
     tokens = min(cfg.N, REFERENCE_TOKENS)
@@ -363,7 +366,7 @@ def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     peaks = load_peaks()
-    cfg = config_of(args.config)
+    cfg = config_of(args.config, args.seq_len)
     io = gret.Dtype.BF16
     path, segs = gret.prefill_path(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, cfg.chunk, io)
     host = gi.prefill_inputs(cfg)
@@ -523,7 +526,7 @@ def run_varlen(args, world, dev, stream, d, cfg, peaks):
     O = torch.empty_like(flat["V"])
     S = torch.empty((S_n, cfg.H, cfg.dk, cfg.dv), dtype=torch.float32, device=dev)
     io = gret.Dtype.BF16
-    ws_bytes = gret.gret_prefill_workspace_size(S_n, cfg.H, max_len, cfg.dk, cfg.dv, cfg.chunk, io)
+    ws_bytes = gret.gret_prefill_varlen_workspace_size(S_n, T, max_len, cfg.H, cfg.dk, cfg.dv, cfg.chunk, io)
     ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
 
     def step():
@@ -549,9 +552,9 @@ def run_varlen(args, world, dev, stream, d, cfg, peaks):
     return {"workload": f"{cfg.name} tokens packed as {S_n} sequences of 1..{max_len} tokens",
             "sequences": S_n, "tokens": T, "steps": args.steps, "ms_per_step": ms / args.steps,
             "value": job_throughput(world, T, args.steps, ms) / 1e6, "unit": "Mtok/s",
-            "path": path.name, "segments": segs,
+            "path": path.name, "split": "long sequences cut on the device, longest segments first",
             "path_hbm": {"alg_gbs": bytes_ / step_s / 1e9, "frac": bytes_ / step_s / 1e9 / peaks["hbm_gbs"]},
-            "gpu_launches": gret.gret_prefill_launches(S_n, cfg.H, max_len, cfg.dk, cfg.dv, cfg.chunk, io)
+            "gpu_launches": gret.gret_prefill_varlen_launches(S_n, T, max_len, cfg.H, cfg.dk, cfg.dv, cfg.chunk, io)
             * args.steps}
 
 
@@ -807,6 +810,9 @@ def main():
                     help="headline prefill workload (c3: B1 H32 N65536 d 128 chunk 128)")
     ap.add_argument("--no-other-configs", action="store_true",
                     help="skip the other prefill workloads' sub-measurements")
+    ap.add_argument("--seq-len", type=int, default=0,
+                    help="profiling aid: run the headline workload with this many tokens per sequence "
+                         "(the JSON line then names the reduced workload)")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-varlen", action="store_true")
     ap.add_argument("--no-seqpar", action="store_true")

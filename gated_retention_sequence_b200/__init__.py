@@ -14,4 +14,5 @@ from .gret import (  # noqa: F401
     gret_set_profile_events, gret_status_string, gret_version, load, prefill, prefill_backward, prefill_path, prefill_state,
     prefill_varlen, state_fold, prefill_projected, gret_prefill_projected, gret_prefill_projected_workspace_size,
     gret_prefill_resume, gret_debug_inject_timeout, gret_set_gate_profile_events,
+    gret_prefill_varlen_workspace_size, gret_prefill_varlen_launches,
 )

@@ -196,7 +196,7 @@ static gret_status prefill_impl(const void* Q, const void* K, const void* V, con
     a.B = B; a.H = H; a.N = N; a.dk = dk; a.dv = dv; a.chunk = chunk;
     a.inv_tau = 1.0f / tau; a.eps = eps; a.io = io_dtype; a.epi = epi;
     a.workspace = workspace; a.workspace_bytes = workspace_bytes;
-    a.status = status; a.segments = segs; a.seg_len = seg_len; a.pieces = pcs;
+    a.status = status; a.segments = segs; a.seg_len = seg_len; a.pieces = pcs; a.num_sms = sms;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t err;
@@ -205,6 +205,7 @@ static gret_status prefill_impl(const void* Q, const void* K, const void* V, con
         a.pieces = prefill_tc_state_pieces(B, H, chunk, sms, segs, seg_len);
     }
     const size_t base = path != GRET_PATH_TC ? 0
+                        : cu_seqlens ? prefill_tc_varlen_workspace_bytes(B, H, N, total, dk, dv, chunk, sms)
                         : resume ? prefill_tc_state_workspace_bytes(B, H, N, dk, dv, chunk, sms)
                                  : prefill_tc_workspace_bytes(B, H, N, dk, dv, chunk, segs, pcs);
     const size_t need = align256(base) + (projected ? projected_extra_bytes(path, B, H, N, d_model) : 0);
@@ -280,6 +281,25 @@ gret_status gret_prefill_resume(const void* Q, const void* K, const void* V, con
                                 void* workspace, size_t workspace_bytes, gret_stream_t stream) {
     return prefill_impl(Q, K, V, gate_logits, G, S0, nullptr, 0, tau, chunk, O, S_final, B, H, N, dk, dv, io_dtype,
                         eps, epi, workspace, workspace_bytes, stream, nullptr, nullptr, 0, true);
+}
+
+size_t gret_prefill_varlen_workspace_size(int num_seqs, int total_tokens, int max_seqlen, int H, int dk, int dv,
+                                          int chunk, gret_dtype io_dtype) {
+    if (num_seqs <= 0 || total_tokens <= 0 || max_seqlen <= 0) return 0;
+    int sms = 148;
+    device_info(nullptr, &sms);
+    if (select_path(num_seqs, H, max_seqlen, dk, dv, chunk, io_dtype, sms, nullptr, nullptr) != GRET_PATH_TC) return 0;
+    return prefill_tc_varlen_workspace_bytes(num_seqs, H, max_seqlen, total_tokens, dk, dv, chunk, sms);
+}
+
+int gret_prefill_varlen_launches(int num_seqs, int total_tokens, int max_seqlen, int H, int dk, int dv, int chunk,
+                                 gret_dtype io_dtype) {
+    if (num_seqs <= 0 || total_tokens <= 0 || max_seqlen <= 0) return 0;
+    int sms = 148;
+    device_info(nullptr, &sms);
+    const gret_path p = select_path(num_seqs, H, max_seqlen, dk, dv, chunk, io_dtype, sms, nullptr, nullptr);
+    // tensor cores: gate scan, plan, state pass, combine, fused loop
+    return p == GRET_PATH_TC ? 5 : p == GRET_PATH_SIMT ? 1 : 0;
 }
 
 gret_status gret_prefill_varlen(const void* Q, const void* K, const void* V, const float* gate_logits,

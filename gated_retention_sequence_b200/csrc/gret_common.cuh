@@ -59,6 +59,7 @@ struct PrefillArgs {
     // decay sums and the folded state-pass pieces of these tokens; pieces is
     // then the state pass's pieces per segment
     int resume;
+    int num_sms;              // the device's SM count (plans of packed batches)
     // gate projection (gret_prefill_projected): when X is set, the gate logits
     // are z = X W_gamma, computed by the tensor-core path's gate prologue;
     // X [B][N][d_model] bf16, Wg [d_model][H] fp32
@@ -180,6 +181,8 @@ cudaError_t launch_gate_project_tc(const PrefillArgs& a, float* bcum, float* ebl
 cudaError_t launch_gate_project_simt(const PrefillArgs& a, float* z, cudaStream_t s);
 void prefill_tc_plan(int B, int H, int N, int chunk, int num_sms, int* segments, int* seg_len, int* pieces);
 size_t prefill_tc_workspace_bytes(int B, int H, int N, int dk, int dv, int chunk, int segments, int pieces);
+size_t prefill_tc_varlen_workspace_bytes(int S, int H, int max_seqlen, int total, int dk, int dv, int chunk,
+                                         int num_sms);
 int prefill_tc_launches(int segments, int pieces);
 
 }  // namespace gret

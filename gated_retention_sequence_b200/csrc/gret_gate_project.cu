@@ -12,9 +12,11 @@
 // accumulated in fp32 in tensor memory, with X tiles (bf16, 128-byte swizzle)
 // and W_gamma^T tiles arriving by TMA.  The gate precision is kept by feeding
 // W_gamma as two bf16 halves, hi = bf16(W) and lo = bf16(W - hi): X is exact in
-// bf16, so D = X hi + X lo carries W to about 2^-17 relative, against 2^-9 for
+// bf16, so z = X hi + X lo carries W to about 2^-17 relative, against 2^-9 for
 // a single bf16 copy (a z near 8 would otherwise move gamma's memory length by
-// percents).  The four epilogue warps then read z straight from tensor memory
+// percents).  The halves are stacked as the rows of one B operand, so that one
+// MMA of N = 2 x heads gives both products side by side.  The four epilogue
+// warps then read z = D[t][h] + D[t][HP + h] straight from tensor memory
 // (lane = token), form log gamma, and scan it along the tokens of each chunk
 // (warp shuffles, then the earlier warps' totals of the chunk through shared
 // memory), writing the same decay sums and P-block factors the plain gate scan
@@ -38,7 +40,7 @@ constexpr int kProjThreads = 160;   // warps 0-3: scan epilogue, lane = token; w
 constexpr int kProjBox = 64;        // d_model columns per TMA box (128 bytes of bf16)
 
 struct ProjParams {
-    CUtensorMap tmX, tmWhi, tmWlo;
+    CUtensorMap tmX, tmW;
     float* bcum;            // [B*H][Npad] chunk-local cumulative log-decay
     float* eblk;            // [B*H][Npad] P-block factors
     unsigned int* status;
@@ -49,17 +51,20 @@ struct ProjParams {
 template <int HP>
 struct ProjCfg {
     static constexpr int XB = kProjRows * 128;      // X tile: 128 tokens x 64 bf16
-    static constexpr int WB = HP * 128;             // one W^T tile: HP heads x 64 bf16
-    static constexpr int STAGE = XB + 2 * WB;       // X, W hi, W lo
+    static constexpr int WB = 2 * HP * 128;         // W^T tile: hi then lo rows, HP each, x 64 bf16
+    static constexpr int STAGE = XB + WB;           // X, stacked W
+    // as many stages as about 192 KB hold (2-8): the kernel streams X once, so
+    // the loads in flight per SM set its rate
     static constexpr int NS_FIT = (192 * 1024) / STAGE;
-    static constexpr int NS = NS_FIT > 4 ? 4 : NS_FIT;
+    static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;
     static_assert(NS >= 2, "projection stages");
     static constexpr int OFF_BAR = NS * STAGE;
     static constexpr int NBAR = 2 * NS + 1;         // full, empty per stage; all MMAs done
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int OFF_WSUM = OFF_MISC + 16;  // [HP][4] each warp's scan total
     static constexpr int SMEM = OFF_WSUM + HP * 4 * 4 + 1024;
-    static constexpr int TM_COLS = HP <= 32 ? 32 : HP <= 64 ? 64 : HP <= 128 ? 128 : 256;
+    static constexpr int TM_COLS = 2 * HP <= 32 ? 32 : 2 * HP <= 64 ? 64 : 2 * HP <= 128 ? 128 : 256;
+    static_assert(2 * HP <= 256, "one MMA of N = 2 HP");
     static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
 
@@ -85,8 +90,7 @@ __global__ void __launch_bounds__(kProjThreads, 1) gate_project_scan_kernel(cons
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&p.tmX);
-        tma_prefetch_desc(&p.tmWhi);
-        tma_prefetch_desc(&p.tmWlo);
+        tma_prefetch_desc(&p.tmW);
     }
     if (warp == 0) {
         tmem_alloc(smem_u32(tmem_slot), CF::TM_COLS);
@@ -110,24 +114,19 @@ __global__ void __launch_bounds__(kProjThreads, 1) gate_project_scan_kernel(cons
                 const uint32_t st = sb + s * CF::STAGE;
                 mbar_arrive_expect_tx(full(s), CF::STAGE);
                 tma_load_3d(st, &p.tmX, k * kProjBox, m * kProjRows, b, full(s));
-                tma_load_2d(st + CF::XB, &p.tmWhi, k * kProjBox, 0, full(s));
-                tma_load_2d(st + CF::XB + CF::WB, &p.tmWlo, k * kProjBox, 0, full(s));
+                tma_load_2d(st + CF::XB, &p.tmW, k * kProjBox, 0, full(s));
             };
             for (int k = 0; k < NS && k < p.nk; ++k) issue(k);
-            constexpr uint32_t idesc = idesc_bf16(kProjRows, HP, false, false);
+            constexpr uint32_t idesc = idesc_bf16(kProjRows, 2 * HP, false, false);
             for (int k = 0; k < p.nk; ++k) {
                 const int s = k % NS;
                 if (!mbar_wait(full(s), (k / NS) & 1, p.status, abort_flag)) break;
                 tc_fence_after();
                 const uint32_t st = sb + s * CF::STAGE;
 #pragma unroll
-                for (int w = 0; w < 2; ++w) {           // W hi, then W lo
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_ss(tm, sdesc_sw128(st + kk * 32, 16, 1024),
-                               sdesc_sw128(st + CF::XB + w * CF::WB + kk * 32, 16, 1024), idesc,
-                               (k | w | kk) != 0);
-                }
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_ss(tm, sdesc_sw128(st + kk * 32, 16, 1024), sdesc_sw128(st + CF::XB + kk * 32, 16, 1024),
+                           idesc, (k | kk) != 0);
                 mma_commit(empty(s));
                 if (k + NS < p.nk) {
                     // the stage is free once its MMAs have read it
@@ -152,15 +151,17 @@ __global__ void __launch_bounds__(kProjThreads, 1) gate_project_scan_kernel(cons
         const uint32_t lq = (uint32_t)(warp * 32) << 16;
 #pragma unroll 1
         for (int g = 0; g < HP / 16; ++g) {
-            uint32_t r[16];
-            tmem_ld_x16(tm + lq + g * 16, r);
+            uint32_t r[16], rl[16];
+            tmem_ld_x16(tm + lq + g * 16, r);             // X W_hi
+            tmem_ld_x16(tm + lq + HP + g * 16, rl);       // X W_lo
             tmem_wait_ld();
             float x[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 const int h = g * 16 + j;
+                const float z = __uint_as_float(r[j]) + __uint_as_float(rl[j]);
                 // past the sequence's end the decay stays flat (log gamma = 0)
-                x[j] = (h < p.H && n < p.N) ? log_gamma(__uint_as_float(r[j]), p.inv_tau) : 0.f;
+                x[j] = (h < p.H && n < p.N) ? log_gamma(z, p.inv_tau) : 0.f;
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
                     const float y = __shfl_up_sync(0xffffffffu, x[j], o);
@@ -190,7 +191,8 @@ __global__ void __launch_bounds__(kProjThreads, 1) gate_project_scan_kernel(cons
     }
 }
 
-// W_gamma [d_model][H] fp32 -> hi, lo [HP][d_model] bf16 (rows h >= H zero).
+// W_gamma [d_model][H] fp32 -> hi, lo [HP][d_model] bf16 (rows h >= H zero);
+// lo follows hi in memory, so the two form one [2 HP][d_model] operand.
 __global__ void gate_weight_split_kernel(const float* __restrict__ W, int d_model, int H, int HP,
                                          __nv_bfloat16* __restrict__ whi, __nv_bfloat16* __restrict__ wlo) {
     // the previous call's kernels may still read this workspace
@@ -286,7 +288,7 @@ cudaError_t run_project(ProjParams& pp, int B, cudaStream_t s) {
 }  // namespace
 
 int gate_project_heads_padded(int H) {
-    return H <= 16 ? 16 : H <= 32 ? 32 : H <= 64 ? 64 : H <= 128 ? 128 : H <= 256 ? 256 : 0;
+    return H <= 16 ? 16 : H <= 32 ? 32 : H <= 64 ? 64 : H <= 128 ? 128 : 0;
 }
 
 bool gate_project_tc_supported(int H, int d_model) {
@@ -295,16 +297,15 @@ bool gate_project_tc_supported(int H, int d_model) {
 }
 
 size_t gate_project_tc_ws_bytes(int H, int d_model) {
-    const size_t half = (size_t)gate_project_heads_padded(H) * d_model * 2;
-    return 2 * ((half + 255) & ~size_t(255));
+    const size_t both = 2 * (size_t)gate_project_heads_padded(H) * d_model * 2;
+    return (both + 255) & ~size_t(255);
 }
 
 cudaError_t launch_gate_project_tc(const PrefillArgs& a, float* bcum, float* eblk, int Npad, void* wsplit,
                                    cudaStream_t s) {
     const int HP = gate_project_heads_padded(a.H);
-    const size_t half = ((size_t)HP * a.d_model * 2 + 255) & ~size_t(255);
     __nv_bfloat16* whi = static_cast<__nv_bfloat16*>(wsplit);
-    __nv_bfloat16* wlo = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(wsplit) + half);
+    __nv_bfloat16* wlo = whi + (size_t)HP * a.d_model;
     const long long elems = (long long)HP * a.d_model;
     const int blocks = (int)std::min<long long>((elems + 255) / 256, 148 * 8);
     cudaError_t e = launch_pdl(gate_weight_split_kernel, dim3(blocks), dim3(256), 0, s, a.Wg, a.d_model, a.H, HP,
@@ -314,11 +315,9 @@ cudaError_t launch_gate_project_tc(const PrefillArgs& a, float* bcum, float* ebl
     memset(&pp, 0, sizeof(pp));
     const cuuint64_t xd[3] = {(cuuint64_t)a.d_model, (cuuint64_t)a.N, (cuuint64_t)a.B};
     const cuuint32_t xb[3] = {kProjBox, kProjRows, 1};
-    const cuuint64_t wd[2] = {(cuuint64_t)a.d_model, (cuuint64_t)HP};
-    const cuuint32_t wb[2] = {kProjBox, (cuuint32_t)HP};
-    if (!make_map(&pp.tmX, a.X, 3, xd, xb) || !make_map(&pp.tmWhi, whi, 2, wd, wb) ||
-        !make_map(&pp.tmWlo, wlo, 2, wd, wb))
-        return cudaErrorInvalidValue;
+    const cuuint64_t wd[2] = {(cuuint64_t)a.d_model, (cuuint64_t)(2 * HP)};
+    const cuuint32_t wb[2] = {kProjBox, (cuuint32_t)(2 * HP)};
+    if (!make_map(&pp.tmX, a.X, 3, xd, xb) || !make_map(&pp.tmW, whi, 2, wd, wb)) return cudaErrorInvalidValue;
     pp.bcum = bcum;
     pp.eblk = eblk;
     pp.status = a.status;
@@ -333,8 +332,7 @@ cudaError_t launch_gate_project_tc(const PrefillArgs& a, float* bcum, float* ebl
         case 16: e = run_project<16>(pp, a.B, s); break;
         case 32: e = run_project<32>(pp, a.B, s); break;
         case 64: e = run_project<64>(pp, a.B, s); break;
-        case 128: e = run_project<128>(pp, a.B, s); break;
-        default: e = run_project<256>(pp, a.B, s); break;
+        default: e = run_project<128>(pp, a.B, s); break;
     }
     if (g_profile_gate_stop) cudaEventRecord(g_profile_gate_stop, s);
     return e;

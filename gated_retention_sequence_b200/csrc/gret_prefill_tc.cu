@@ -37,6 +37,7 @@
 // decomposition S(x || y) = e^{sum log gamma(y)} S(x) + S(y from 0).
 #include <cuda.h>
 
+#include <algorithm>
 #include <cstring>
 #include <type_traits>
 #include <utility>
@@ -139,10 +140,18 @@ struct TcParams {
     const int* cu;           // packed batch: sequence b is token rows cu[b] .. cu[b+1]-1; or null
     int total;               // rows of the packed tensors
     void* O;                 // output base (tail rows of packed sequences are stored directly)
+    const void* G;           // gate tensor (read directly by the output-rows kernel), or null
     unsigned int* status;
     int H, N, Npad, P, seg_len;
     int K, piece_len;        // state-pass pieces per segment and their length
     int slots;               // state-pass pieces (and seg_state slots) per unit
+    // planned packed batch (varlen_plan_kernel): per unit {segments, segment
+    // length, first seg_state slot, -}; the fused and state-pass work items
+    // (unit, segment), longest segments first; the item counts
+    const int4* unit_info;
+    const int2* fused_items;
+    const int2* state_items;
+    const int* plan_count;
     float eps;
     int gn;                  // 1: GroupNorm + swish; 0: O = Y
     int has_g;
@@ -263,9 +272,27 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
         }
     }
 
-    const int u = blockIdx.x / p.P, seg = blockIdx.x % p.P;
+    // work item: a (unit, segment) of the uniform split, or of a packed
+    // batch's plan (a block past the plan's item count has nothing to do)
+    int u = 0, seg = 0, nseg_u = p.P, seg_len = p.seg_len;
+    size_t in_slot = 0;                       // seg_state slot of S_in (seg > 0)
+    if constexpr (!PACKED) {
+        u = blockIdx.x / p.P;
+        seg = blockIdx.x % p.P;
+        in_slot = (size_t)u * p.slots + (size_t)seg * p.K - 1;
+    } else {
+        grid_dep_wait();
+        if ((int)blockIdx.x >= p.plan_count[0]) return;
+        const int2 it = p.fused_items[blockIdx.x];
+        const int4 ui = p.unit_info[it.x];
+        u = it.x;
+        seg = it.y;
+        nseg_u = ui.x;
+        seg_len = ui.y;
+        in_slot = (size_t)ui.z + seg - 1;
+    }
     const int hh = u % p.H;
-    const int n_begin = seg * p.seg_len;
+    const int n_begin = seg * seg_len;
 
     // Barriers.  The scores, the state MMA and the staged output have one
     // barrier per chunk parity, so that none of them can complete a phase
@@ -319,8 +346,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
     if constexpr (PACKED) {
         bb = 0;
         packed_range(p.cu, u / p.H, p.total, row0, Nu);
+        Nu = min(Nu, p.N);                    // tokens past max_seqlen are not processed
     }
-    const int n_end = min(Nu, n_begin + p.seg_len);
+    const int n_end = min(Nu, n_begin + seg_len);
     const int nchunks = n_end > n_begin ? (n_end - n_begin + C - 1) / C : 0;
     // a packed sequence's last chunk stops at its end: its output rows are
     // stored directly, since a full tile would overwrite the next sequence
@@ -533,8 +561,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
         {
             uint32_t r[W];
             if (seg > 0) {
-                const float* src = p.seg_state + ((size_t)u * p.slots + (size_t)seg * p.K - 1) * DV * DK +
-                                   (size_t)s_d * DK + s_k0;
+                const float* src = p.seg_state + in_slot * DV * DK + (size_t)s_d * DK + s_k0;
                 const float4* s4 = reinterpret_cast<const float4*>(src);
 #pragma unroll
                 for (int j = 0; j < W / 4; ++j) {
@@ -844,7 +871,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
             mbar_wait(bar(BMMA + ((nchunks - 1) & 1)), ((nchunks - 1) >> 1) & 1, p.status, abort_flag);
             tc_fence_after();
         }
-        if (p.S_final && seg == p.P - 1) {
+        if (p.S_final && seg == nseg_u - 1) {
             const float sc = __expf(lam);
             uint32_t r[W];
             tmem_ld<W>(tm + lq + CF::TM_S + col0, r);
@@ -903,10 +930,27 @@ __global__ void __launch_bounds__(kStateThreads, 1) prefill_state_kernel(const _
     const int q4 = warp & 3, gi = warp >> 2;
     const uint32_t lq = (uint32_t)(32 * q4) << 16;
 
-    const int nseg = p.slots;                   // pieces of the segments that need one
-    const int u = blockIdx.x / nseg, seg = blockIdx.x % nseg;
+    // work item: a piece of the uniform split, or a segment of a packed
+    // batch's plan (one piece per segment; a block past the plan's count has
+    // nothing to do)
+    int u = 0, seg = 0, piece_len = p.piece_len;
+    size_t out_slot = 0;
+    if constexpr (!PACKED) {
+        u = blockIdx.x / p.slots;
+        seg = blockIdx.x % p.slots;
+        out_slot = (size_t)u * p.slots + seg;
+    } else {
+        grid_dep_wait();
+        if ((int)blockIdx.x >= p.plan_count[1]) return;
+        const int2 it = p.state_items[blockIdx.x];
+        const int4 ui = p.unit_info[it.x];
+        u = it.x;
+        seg = it.y;
+        piece_len = ui.y;
+        out_slot = (size_t)ui.z + seg;
+    }
     const int hh = u % p.H;
-    const int n_begin = seg * p.piece_len;
+    const int n_begin = seg * piece_len;
 
     auto full = [&](int s) -> uint32_t { return sb + CF::OFF_BAR + 8 * s; };
     auto empty = [&](int s) -> uint32_t { return sb + CF::OFF_BAR + 8 * (NS + s); };
@@ -939,8 +983,9 @@ __global__ void __launch_bounds__(kStateThreads, 1) prefill_state_kernel(const _
     if constexpr (PACKED) {
         bb = 0;
         packed_range(p.cu, u / p.H, p.total, row0, Nu);
+        Nu = min(Nu, p.N);                    // tokens past max_seqlen are not processed
     }
-    const int n_end = min(Nu, n_begin + p.piece_len);
+    const int n_end = min(Nu, n_begin + piece_len);
     const int nchunks = n_end > n_begin ? (n_end - n_begin + C - 1) / C : 0;
     int last_issued = -1;     // thread 0: the last chunk whose loads it issued
     auto issue = [&](int j) {
@@ -1059,7 +1104,7 @@ __global__ void __launch_bounds__(kStateThreads, 1) prefill_state_kernel(const _
     {
         const float sc = __expf(lam);
         const int s_d = (col0 / 128) * 128 + q4 * 32 + lane, s_k0 = col0 % 128;
-        float* dst = p.seg_state + ((size_t)u * nseg + seg) * DV * DK + (size_t)s_d * DK + s_k0;
+        float* dst = p.seg_state + out_slot * DV * DK + (size_t)s_d * DK + s_k0;
 #pragma unroll 1
         for (int cb = 0; cb < W / 32; ++cb) {
             uint32_t r[32];
@@ -1071,7 +1116,7 @@ __global__ void __launch_bounds__(kStateThreads, 1) prefill_state_kernel(const _
                 d4[j] = make_float4(u2f(r[4 * j]) * sc, u2f(r[4 * j + 1]) * sc, u2f(r[4 * j + 2]) * sc,
                                     u2f(r[4 * j + 3]) * sc);
         }
-        if (tid == 0) p.seg_decay[(size_t)u * nseg + seg] = seg_decay;
+        if (tid == 0) p.seg_decay[out_slot] = seg_decay;
     }
     tc_fence_before();
     __syncthreads();
@@ -1134,16 +1179,138 @@ static dim3 gate_scan_grid(int units, int npad, int C, int* nyb) {
     return dim3(units, *nyb < 65535 ? *nyb : 65535);
 }
 
+// Work plan of a packed batch (gret_prefill_varlen on the tensor-core path),
+// made on the device from cu_seqlens.  A sequence of more than seg_max tokens
+// is cut into ceil(chunks / (seg_max / C)) segments of equal chunk-multiple
+// length, every head alike; the others stay whole.  The fused loop's work
+// items (unit, segment) are listed longest segment first (a counting sort on
+// the chunks per segment), so that the block scheduler starts the long ones
+// first and no sequence finishes alone; the state pass's items are the
+// segments before each split sequence's last, one slot each, numbered so that
+// item i writes slot i.
+constexpr int kPlanThreads = 1024;
+constexpr int kPlanBuckets = 1024;
+
+struct PlanArgs {
+    const int* cu;
+    int total, S, H, C, seg_max, max_len;   // sequences are cut at max_len tokens
+    int4* unit_info;        // [S * H]
+    int2* fused_items;      // [max_fused]
+    int2* state_items;      // [max_state]
+    int* count;             // [2]: fused items, state items
+    int2* seq_info;         // [S] scratch: segments, chunks per segment
+    int* seq_order;         // [S] scratch: sequences, longest segments first
+    int max_fused, max_state;
+};
+
+// Exclusive prefix sum of v over the block's threads; *total gets the sum.
+__device__ __forceinline__ int block_exclusive_sum(int v, int* warp_sums, int* total) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_sums[w] = x;
+    __syncthreads();
+    if (w == 0) {
+        int t = lane < kPlanThreads / 32 ? warp_sums[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, t, o);
+            if (lane >= o) t += y;
+        }
+        warp_sums[lane] = t;             // inclusive over warps
+    }
+    __syncthreads();
+    const int excl = x - v + (w > 0 ? warp_sums[w - 1] : 0);
+    const int tot = warp_sums[kPlanThreads / 32 - 1];
+    __syncthreads();                     // warp_sums is reused by the next call
+    *total = tot;
+    return excl;
+}
+
+__global__ void __launch_bounds__(kPlanThreads) varlen_plan_kernel(const PlanArgs a) {
+    __shared__ int offs[kPlanBuckets];
+    __shared__ int warp_sums[kPlanThreads / 32];
+    // the previous call's kernels may still read the plan in the workspace
+    grid_dep_launch();
+    grid_dep_wait();
+    const int tid = threadIdx.x;
+    const int maxch = a.seg_max / a.C;
+    offs[tid] = 0;
+    __syncthreads();
+    auto bucket_of = [&](int per) { return kPlanBuckets - 1 - min(per, kPlanBuckets - 1); };
+    // segments per sequence, and a histogram of chunks per segment
+    for (int b = tid; b < a.S; b += kPlanThreads) {
+        int row0, len;
+        packed_range(a.cu, b, a.total, row0, len);
+        len = min(len, a.max_len);
+        const int nch = (len + a.C - 1) / a.C;
+        const int P = nch > maxch ? (nch + maxch - 1) / maxch : 1;
+        const int per = (nch + P - 1) / P;
+        a.seq_info[b] = make_int2(P, per);
+        atomicAdd(&offs[bucket_of(per)], 1);
+    }
+    __syncthreads();
+    int tot = 0;
+    const int start = block_exclusive_sum(offs[tid], warp_sums, &tot);
+    offs[tid] = start;
+    __syncthreads();
+    for (int b = tid; b < a.S; b += kPlanThreads)
+        a.seq_order[atomicAdd(&offs[bucket_of(a.seq_info[b].y)], 1)] = b;
+    __syncthreads();
+    // in that order: the fused items (sequence, segment, head) and, per split
+    // sequence, its state slots
+    int carry_f = 0, carry_s = 0;
+    for (int r0 = 0; r0 < a.S; r0 += kPlanThreads) {
+        const int r = r0 + tid;
+        const int b = r < a.S ? a.seq_order[r] : -1;
+        const int2 si = b >= 0 ? a.seq_info[b] : make_int2(0, 0);
+        int tf = 0, ts = 0;
+        const int ef = block_exclusive_sum(si.x, warp_sums, &tf) + carry_f;
+        const int es = block_exclusive_sum(b >= 0 ? si.x - 1 : 0, warp_sums, &ts) + carry_s;
+        if (b >= 0) {
+            for (int h = 0; h < a.H; ++h) {
+                const int u = b * a.H + h;
+                const int slot0 = es * a.H + h * (si.x - 1);
+                a.unit_info[u] = make_int4(si.x, si.y * a.C, slot0, 0);
+                for (int sg = 0; sg < si.x; ++sg) {
+                    const int it = (ef + sg) * a.H + h;
+                    if (it < a.max_fused) a.fused_items[it] = make_int2(u, sg);
+                }
+                for (int sg = 0; sg + 1 < si.x; ++sg)
+                    if (slot0 + sg < a.max_state) a.state_items[slot0 + sg] = make_int2(u, sg);
+            }
+        }
+        carry_f += tf;
+        carry_s += ts;
+    }
+    if (tid == 0) {
+        a.count[0] = min(carry_f * a.H, a.max_fused);
+        a.count[1] = min(carry_s * a.H, a.max_state);
+    }
+}
+
 // Fold the segment increments into initial states, in place:
 // slot p <- S_in(p + 1) = e^{a_p} S_in(p) + dS_p, with S_in(0) = S0 (or 0).
 __global__ void seg_combine_kernel(float* __restrict__ seg_state, const float* __restrict__ seg_decay,
-                                   const float* __restrict__ S0, int nslots, int dk, int dv) {
+                                   const float* __restrict__ S0, int nslots, int dk, int dv,
+                                   const int4* __restrict__ unit_info) {
     grid_dep_launch();
     grid_dep_wait();       // the state pass's increments
     const int u = blockIdx.x;
     const int elems4 = dk * dv / 4;
     const int e = blockIdx.y * blockDim.x + threadIdx.x;
     if (e >= elems4) return;
+    // a packed batch's plan gives each unit its own slot range
+    size_t base = (size_t)u * nslots;
+    if (unit_info) {
+        const int4 ui = unit_info[u];
+        nslots = ui.x - 1;
+        base = (size_t)ui.z;
+    }
     float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
     if (S0) {   // slots hold S^T [dv][dk]; S0 is [dk][dv]
         const int d = (4 * e) / dk, k = (4 * e) % dk;
@@ -1151,8 +1318,8 @@ __global__ void seg_combine_kernel(float* __restrict__ seg_state, const float* _
         run = make_float4(s0[0], s0[dv], s0[2 * dv], s0[3 * dv]);
     }
     for (int p = 0; p < nslots; ++p) {
-        float4* slot = reinterpret_cast<float4*>(seg_state) + ((size_t)u * nslots + p) * elems4 + e;
-        const float f = __expf(seg_decay[(size_t)u * nslots + p]);
+        float4* slot = reinterpret_cast<float4*>(seg_state) + (base + p) * elems4 + e;
+        const float f = __expf(seg_decay[base + p]);
         const float4 d = *slot;
         run = make_float4(fmaf(f, run.x, d.x), fmaf(f, run.y, d.y), fmaf(f, run.z, d.z), fmaf(f, run.w, d.w));
         *slot = run;
@@ -1227,39 +1394,45 @@ __global__ void state_fold_kernel(const float* __restrict__ dS_all, const float*
 //
 // The same chunkwise form as prefill_tc_kernel, laid out the other way round
 // for the output: O[t][d] sits in tensor memory with one token per lane, so the
-// GroupNorm of a token is one thread's sum over its own row and G / O move as
-// 16-byte vectors, and P[t][s] feeds the intra-chunk product from tensor memory.
+// GroupNorm of a token is a sum along its own row and G / O move as 16-byte
+// vectors, and P[t][s] feeds the intra-chunk product from tensor memory.
 //   scores  D[t][s]  = Q K~^T        A = Q (smem, K-major), B = K~ (K-major)
 //   inter   D[t][d]  = Q~ T           A = Q or Q~ (smem),    B = bf16 copy of T^T (smem, K-major)
 //   intra   D[t][d] += P V            A = P (tensor memory, bf16), B = V (smem, MN-major)
 //   state   D[d][k] += V^T K~         A = V (MN-major), B = K~ (MN-major): T^T, fp32, lanes = d
-// The epilogue warps read G from a TMA-loaded tile and write their output
-// rows straight to global memory (16-byte stores, 256 contiguous bytes per
-// token), so the next G tile can load as soon as this one has been read.
+// The epilogue warps read G from a TMA-loaded tile and write the output over
+// it in place; one TMA store per chunk then writes the tile to O, after which
+// the tile takes the next chunk's G.
 //
 // Lazy chunks (the largest K scale e^{-b_s - Lambda} within e^kLazyMax) factor
 // the decay: K~_s = e^{-b_s - Lambda} K_s is scaled once, before the scores, so
 //   e^{-(b_t + Lambda)} Y_t = Q_t T + sum_{s <= t} (Q_t . K~_s) V_s,
 // P is the masked scores alone, Q needs no scaling, and the row factor
-// c_t = e^{b_t + Lambda} <= 1 enters the GroupNorm statistics (mean c mu,
-// variance c^2 var) in the epilogue; the state update T += V^T K~ uses the same
-// K~ and Lambda += b_C.  Eager chunks take the direct forms: P[t][s] =
-// A[t][s] e^{b_t - b_s}, Q~_t = e^{b_t + Lambda} Q_t against the unscaled T, then
-// T *= e^{Lambda + b_C}, K~_s = e^{b_C - b_s} K_s and Lambda = 0.  All exponents
-// stay <= kLazyMax, so nothing overflows.
+// c_t = e^{b_t + Lambda} <= 1 enters the GroupNorm statistics in the
+// epilogue; the state update T += V^T K~ uses the same K~ and Lambda += b_C.
+// Eager chunks take the direct forms: P[t][s] = A[t][s] e^{b_t - b_s},
+// Q~_t = e^{b_t + Lambda} Q_t against the unscaled T, then T *= e^{Lambda + b_C},
+// K~_s = e^{b_C - b_s} K_s and Lambda = 0.  All exponents stay <= kLazyMax.
 //
-// Roles (512 threads).  Warps 0-3 (E): epilogue, one token row per thread.
-// Warps 4-7 (P): masked scores -> bf16 P in tensor memory.  Warps 8-11 (S): K~
-// and Q~ in shared memory, the bf16 copy of T after each state update, the
-// eager rescale, the initial and final state.  Warp 12 lane 0 issues every
-// MMA, warp 13 lane 0 every TMA load and store; warps 14-15 idle.  The roles
-// work on different chunks at once: E finishes chunk i while S and P prepare
-// chunk i + 1 and the tensor cores run its products.
-constexpr int kRowsThreads = 512;
-constexpr int kRowsLaunchRegs = 128;   // 65536 / 512
-constexpr int kRowsERegs = 200;        // epilogue warps hold a token's 128 outputs
-constexpr int kRowsOtherRegs = 104;
-static_assert(128 * kRowsERegs + 384 * kRowsOtherRegs <= kRowsThreads * kRowsLaunchRegs, "register split");
+// Roles (896 threads, seven warpgroups, 72 registers each).  Warps 0-15 (E):
+// epilogue, four warps per tensor-memory lane quarter, each owning 32 of a
+// token's 128 channels; the four quarters' partial sums of a token meet in
+// spare tensor-memory columns of its lane (two sets, by chunk parity).  Warps
+// 16-19 (P): masked scores -> bf16 P in tensor memory; causality leaves lane
+// quarter q with q + 1 nonzero 32-column blocks, so warps 26 and 27 (lane
+// quarters 2 and 3) take the blocks past the second of the two heaviest
+// quarters and no warp converts more than two.  The blocks above the diagonal
+// stay zero and are written once.  Warps 20-23 (S): K~ and Q~ in shared memory
+// (one token row per thread), the bf16 copy of T after each state update, the
+// eager rescale, the initial and final state.  Warp 24 lane 0 issues every
+// MMA; warp 25 lane 0 every TMA load and the output store.  The roles work on
+// different chunks at once: E finishes chunk i while S and P prepare chunk
+// i + 1 and the tensor cores run its products.
+constexpr int kRowsThreads = 896;
+constexpr int kRowsRegs = 72;          // 65536 / 896, rounded down to 8
+constexpr int kRowsSRegs = 64;         // the S warps hand registers to the issuing warps
+constexpr int kRowsIssueRegs = 80;
+static_assert(128 * kRowsSRegs + 128 * kRowsIssueRegs <= 256 * kRowsRegs, "register split");
 
 struct RowsCfg {
     static constexpr int C = 128, DV = 128;
@@ -1272,14 +1445,27 @@ struct RowsCfg {
     static constexpr int OFF_T = OFF_G + TILE;      // bf16 T^T [d][k]
     static constexpr int OFF_B = OFF_T + TILE;      // per Q/K stage: C fp32 decay sums
     static constexpr int OFF_BAR = OFF_B + 2 * C * 4;
-    static constexpr int NUM_BARS = 17;
+    static constexpr int NUM_BARS = 16;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int USED = OFF_MISC + 16;
     static constexpr int SMEM = USED + 1024;        // room to align the base to 1024 bytes
     static_assert(SMEM <= kMaxSmem, "shared memory budget");
-    // tensor-memory columns
-    static constexpr int TM_O = 0, TM_SC = 128, TM_P = 256, TM_T = 320, TM_ALLOC = 512;
+    // tensor-memory columns: O, scores, P, T^T, and the epilogue's exchange
+    // (two sets of four (sum, sum of squares) pairs)
+    static constexpr int TM_O = 0, TM_SC = 128, TM_P = 256, TM_T = 320, TM_X = 448, TM_ALLOC = 512;
+    static_assert(TM_X + 16 <= TM_ALLOC, "tensor-memory columns");
 };
+
+// Scale the 16-byte chunks of one token row of a [128 x 128] bf16 tile (two
+// 128-byte-swizzled boxes) by f; the logical chunk order spreads the 32 rows of
+// a warp over all banks.
+__device__ __forceinline__ void scale_tile_row(uint8_t* tile, int row, float f) {
+#pragma unroll
+    for (int x = 0; x < 2; ++x)
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+            scale_bf16x8(tile + x * RowsCfg::BOX + row * 128 + ((c ^ (row & 7)) << 4), f);
+}
 
 __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __grid_constant__ TcParams p) {
     using CF = RowsCfg;
@@ -1295,10 +1481,11 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
     const int nchunks = n_end > n_begin ? (n_end - n_begin + C - 1) / C : 0;
 
     // barriers; KT has one per Q/K stage so that no phase can complete twice
-    // before the MMA warp has seen the first.  BGF: the epilogue has read the
-    // G tile (index 14 is unused)
+    // before the MMA warp has seen the first.  BG: the G tile of a chunk is in
+    // (or, without G, the tile is free for the chunk's output); BGF: the
+    // epilogue has written the chunk's output into the tile.
     constexpr int BQK = 0, BV = 2, BG = 3, BSC = 4, BOD = 5, BST = 6, BKT = 7, BTC = 9, BQT = 10, BPR = 11,
-                  BOF = 12, BGF = 13, BDRAIN = 15, BNEVER = 16;
+                  BOF = 12, BGF = 13, BDRAIN = 14, BNEVER = 15;
     static_assert(BNEVER + 1 == CF::NUM_BARS, "barrier count");
     auto bar = [&](int i) -> uint32_t { return sb + CF::OFF_BAR + 8 * i; };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + CF::OFF_MISC);
@@ -1306,9 +1493,11 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
 
     if (tid == 0) {
         for (int i = 0; i < CF::NUM_BARS; ++i) {
-            // per-warp arrivals of a four-warp role
-            const bool four = i == BKT || i == BKT + 1 || i == BTC || i == BQT || i == BPR || i == BOF || i == BGF;
-            mbar_init(bar(i), four ? 4 : 1);
+            // per-warp arrivals: sixteen epilogue warps, six P warps, or one
+            // four-warp role
+            const bool sixteen = i == BOF || i == BGF;
+            const bool four = i == BKT || i == BKT + 1 || i == BTC || i == BQT;
+            mbar_init(bar(i), sixteen ? 16 : four ? 4 : i == BPR ? 6 : 1);
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -1329,10 +1518,10 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
     grid_dep_launch();
     grid_dep_wait();
 
-    const int role = warp >> 2;            // 0 E, 1 P, 2 S, 3 issuing warps
+    const int role = warp >> 2;            // 0-3 E; 4 P; 5 S; 6 issuing warps
     const int q4 = warp & 3;               // tensor-memory lane quarter
     const uint32_t lq = (uint32_t)(32 * q4) << 16;
-    const int row = 32 * q4 + lane;        // token t (E, P) or channel d (S) of this thread
+    const int row = 32 * q4 + lane;        // token t (E, P) or channel d / token row (S) of this thread
     auto warp_arrive = [&](int b) {
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(b));
@@ -1340,10 +1529,44 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
     auto stage_bc = [&](int i) -> const float* {
         return reinterpret_cast<const float*>(sm + CF::OFF_B + (i & 1) * C * 4);
     };
+    // masked scores -> bf16 P for the 32-column blocks cb_lo..cb_hi of this
+    // warp's lane quarter (a P warp, or a helper on the heavy quarters)
+    auto p_rows = [&](int cb_lo, int cb_hi) {
+        float lam = 0.f;
+        for (int i = 0; i < nchunks; ++i) {
+            const float* bc = stage_bc(i);
+            mbar_wait(bar(BSC), i & 1, p.status, abort_flag);   // the scores landed (so did Q/K and bc)
+            tc_fence_after();
+            const float bC = bc[C - 1];
+            const bool eager = (-bC - lam) > kLazyMax;
+            const float bt = bc[row];
+#pragma unroll 1
+            for (int cb = cb_lo; cb <= cb_hi; ++cb) {
+                uint32_t r[32], pk[16];
+                tmem_ld_x32(tm + lq + CF::TM_SC + cb * 32, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const int s0 = cb * 32 + 2 * j;
+                    float v0 = u2f(r[2 * j]), v1 = u2f(r[2 * j + 1]);
+                    if (eager) {
+                        v0 *= __expf(fminf(bt - bc[s0], 0.f));
+                        v1 *= __expf(fminf(bt - bc[s0 + 1], 0.f));
+                    }
+                    pk[j] = pack_bf16x2(s0 <= row ? v0 : 0.f, s0 + 1 <= row ? v1 : 0.f);
+                }
+                tmem_st_x16(tm + lq + CF::TM_P + cb * 16, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            warp_arrive(BPR);
+            lam = eager ? 0.f : lam + bC;
+        }
+    };
 
-    if (role == 3) {
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" : : "n"(kRowsOtherRegs));
-        if (warp == 13 && lane == 0 && nchunks > 0) {
+    if (role == 6) {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" : : "n"(kRowsIssueRegs));
+        if (warp == 25 && lane == 0 && nchunks > 0) {
             // ======================================================== TMA producer
             int last_qk[2] = {-1, -1}, last_v = -1, last_g = -1;
             auto issue_qk = [&](int j) {
@@ -1363,7 +1586,12 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
                 for (int x = 0; x < 2; ++x)
                     tma_load_4d(sb + CF::OFF_V + x * CF::BOX, &p.tmV, x * 64, hh, n_begin + j * C, bb, bar(BV));
             };
+            // the tile of chunk j: its G, or (without G) a plain release for its output
             auto issue_g = [&](int j) {
+                if (!p.has_g) {
+                    mbar_arrive(bar(BG));
+                    return;
+                }
                 last_g = j;
                 mbar_arrive_expect_tx(bar(BG), CF::TILE);
                 for (int x = 0; x < 2; ++x)
@@ -1374,26 +1602,31 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
                 issue_qk(0);
                 if (nchunks > 1) issue_qk(1);
                 issue_v(0);
-                if (p.has_g) issue_g(0);
+                issue_g(0);
                 for (int i = 0; i < nchunks; ++i) {
                     // the state MMA of chunk i is the last reader of its Q/K stage and of V
                     if (!mbar_wait(bar(BST), i & 1, p.status, abort_flag)) break;
                     if (i + 2 < nchunks) issue_qk(i + 2);
                     if (i + 1 < nchunks) issue_v(i + 1);
-                    // G of chunk i + 1, once the epilogue has read that of chunk i
-                    if (p.has_g && i + 1 < nchunks) {
-                        if (!mbar_wait(bar(BGF), i & 1, p.status, abort_flag)) break;
-                        issue_g(i + 1);
-                    }
+                    // the output of chunk i leaves from the tile (rows past the end of
+                    // the sequence fall outside the map and are not written); once the
+                    // store has read the tile it takes chunk i + 1
+                    if (!mbar_wait(bar(BGF), i & 1, p.status, abort_flag)) break;
+                    for (int x = 0; x < 2; ++x)
+                        tma_store_4d(&p.tmO, sb + CF::OFF_G + x * CF::BOX, x * 64, hh, n_begin + i * C, bb);
+                    bulk_commit();
+                    bulk_wait_read<0>();
+                    if (i + 1 < nchunks) issue_g(i + 1);
                 }
             }
+            bulk_wait<0>();
             if (*abort_flag) {
                 for (int x = 0; x < 2; ++x)
                     if (last_qk[x] >= 0) mbar_wait_drain(bar(BQK + x), (last_qk[x] >> 1) & 1, kWaitCycles);
                 if (last_v >= 0) mbar_wait_drain(bar(BV), last_v & 1, kWaitCycles);
                 if (last_g >= 0) mbar_wait_drain(bar(BG), last_g & 1, kWaitCycles);
             }
-        } else if (warp == 12 && lane == 0 && nchunks > 0) {
+        } else if (warp == 24 && lane == 0 && nchunks > 0) {
             // ======================================================== MMA issuer
             constexpr uint32_t id_kk = idesc_bf16(128, 128, false, false);   // scores, inter
             constexpr uint32_t id_pv = idesc_bf16(128, 128, false, true);    // intra: B = V MN-major
@@ -1453,11 +1686,13 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
             // every MMA this thread issued has completed before tensor memory is freed
             mma_commit(bar(BDRAIN));
             mbar_wait_drain(bar(BDRAIN), 0, kWaitCycles);
+        } else if (warp >= 26) {
+            // helpers on lane quarters 2 and 3: blocks 2..q4
+            p_rows(2, q4);
         }
-    } else if (role == 2) {
+    } else if (role == 5) {
         // ============================================================ S warps
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" : : "n"(kRowsOtherRegs));
-        const int st = tid - 256;              // 0..127
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" : : "n"(kRowsSRegs));
         // initial state T^T[d][k] (lane d = row): zero, a caller's S0 [k][d], or a
         // segment's folded state [d][k]
         {
@@ -1465,8 +1700,8 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
             for (int cb = 0; cb < 4; ++cb) {
                 if (seg > 0) {
                     const float4* s4 = reinterpret_cast<const float4*>(
-                        p.seg_state + ((size_t)u * p.slots + (size_t)seg * p.K - 1) * DV * DK +
-                        (size_t)row * DK + cb * 32);
+                        p.seg_state + ((size_t)u * p.slots + (size_t)seg * p.K - 1) * DV * DK + (size_t)row * DK +
+                        cb * 32);
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         const float4 v = s4[j];
@@ -1484,13 +1719,6 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
             }
             tmem_wait_st();
         }
-        // K~ (or Q~) in place: 16-byte items of a [128 x 128] bf16 tile, rows scaled
-        auto scale_rows = [&](uint8_t* tile, auto factor_of_row) {
-            for (int it = st; it < C * 16; it += 128) {
-                const int r = (it >> 3) % C;
-                scale_bf16x8(tile + it * 16, factor_of_row(r));
-            }
-        };
         float lam = 0.f;
         for (int i = 0; i < nchunks; ++i) {
             const int s = i & 1;
@@ -1500,8 +1728,9 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
             mbar_wait(bar(BQK + s), (i >> 1) & 1, p.status, abort_flag);
             const float bC = bc[C - 1];
             const bool eager = (-bC - lam) > kLazyMax;
+            const float brow = bc[row];
             if (!eager) {
-                scale_rows(Kp, [&](int r) { return __expf(-bc[r] - lam); });
+                scale_tile_row(Kp, row, __expf(-brow - lam));
                 fence_proxy_async_smem();
                 warp_arrive(BKT + s);
             }
@@ -1542,8 +1771,8 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
                 // Q~ and K~ in place, once the scores have read Q and K
                 mbar_wait(bar(BSC), i & 1, p.status, abort_flag);
                 tc_fence_after();
-                scale_rows(Qp, [&](int r) { return __expf(bc[r] + lam); });
-                scale_rows(Kp, [&](int r) { return __expf(bC - bc[r]); });
+                scale_tile_row(Qp, row, __expf(brow + lam));
+                scale_tile_row(Kp, row, __expf(bC - brow));
                 fence_proxy_async_smem();
                 warp_arrive(BQT);
                 warp_arrive(BKT + s);
@@ -1567,48 +1796,21 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
                 for (int j = 0; j < 32; ++j) dst[(size_t)(cb * 32 + j) * DV + row] = u2f(r[j]) * sc;
             }
         }
-    } else if (role == 1) {
+    } else if (role == 4) {
         // ============================================================ P warps
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" : : "n"(kRowsOtherRegs));
-        float lam = 0.f;
-        for (int i = 0; i < nchunks; ++i) {
-            const float* bc = stage_bc(i);
-            mbar_wait(bar(BSC), i & 1, p.status, abort_flag);   // the scores landed (so did Q/K and bc)
-            tc_fence_after();
-            const float bC = bc[C - 1];
-            const bool eager = (-bC - lam) > kLazyMax;
-            const float bt = bc[row];
-#pragma unroll 1
-            for (int cb = 0; cb < 4; ++cb) {
-                uint32_t pk[16];
-                if (cb <= q4) {
-                    uint32_t r[32];
-                    tmem_ld_x32(tm + lq + CF::TM_SC + cb * 32, r);
-                    tmem_wait_ld();
+        // the blocks above the diagonal, once
+        {
+            uint32_t z[16];
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int s0 = cb * 32 + 2 * j;
-                        float v0 = u2f(r[2 * j]), v1 = u2f(r[2 * j + 1]);
-                        if (eager) {
-                            v0 *= __expf(fminf(bt - bc[s0], 0.f));
-                            v1 *= __expf(fminf(bt - bc[s0 + 1], 0.f));
-                        }
-                        pk[j] = pack_bf16x2(s0 <= row ? v0 : 0.f, s0 + 1 <= row ? v1 : 0.f);
-                    }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) pk[j] = 0u;
-                }
-                tmem_st_x16(tm + lq + CF::TM_P + cb * 16, pk);
-            }
+            for (int j = 0; j < 16; ++j) z[j] = 0u;
+            for (int cb = q4 + 1; cb < 4; ++cb) tmem_st_x16(tm + lq + CF::TM_P + cb * 16, z);
             tmem_wait_st();
-            tc_fence_before();
-            warp_arrive(BPR);
-            lam = eager ? 0.f : lam + bC;
         }
+        p_rows(0, min(q4, 1));
     } else {
         // ============================================================ E warps
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" : : "n"(kRowsERegs));
+        const int hf = role;                       // which 32 channels of the token
+        constexpr int QC = DV / 4;
         float lam = 0.f;
         const float* bsum = p.bcum + (size_t)u * p.Npad;
         for (int i = 0; i < nchunks; ++i) {
@@ -1616,15 +1818,9 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
             const float bt = bsum[n0 + row], bC = bsum[n0 + C - 1];
             mbar_wait(bar(BOD), i & 1, p.status, abort_flag);
             tc_fence_after();
-            float y[DV];
-#pragma unroll
-            for (int cb = 0; cb < 4; ++cb) {
-                uint32_t r[32];
-                tmem_ld_x32(tm + lq + CF::TM_O + cb * 32, r);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 32; ++j) y[cb * 32 + j] = u2f(r[j]);
-            }
+            uint32_t y[QC];
+            tmem_ld_x32(tm + lq + CF::TM_O + hf * QC, y);
+            tmem_wait_ld();
             tc_fence_before();
             warp_arrive(BOF);              // the next inter-chunk product may overwrite O
             const bool eager = (-bC - lam) > kLazyMax;
@@ -1632,37 +1828,48 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
             const float c = eager ? 1.f : __expf(bt + lam);
             float a = c, b0 = 0.f;
             if (p.gn) {
-                // mean of u, then the variance of y = c u from the scaled
-                // deviations c (u - mean): u itself may be as large as e^64 y
-                float s1 = 0.f;
+                // sums of u and of y^2 = (c u)^2 over this quarter (u itself may be
+                // as large as e^64 y), then the token's four quarters through
+                // spare tensor-memory columns of its lane (the set alternates with
+                // the chunk, so a set is rewritten only after every quarter has
+                // passed the next chunk's barrier, i.e. read this one)
+                float s1 = 0.f, s2 = 0.f;
 #pragma unroll
-                for (int j = 0; j < DV; ++j) s1 += y[j];
-                const float mean = s1 * (1.0f / DV);
-                float s2 = 0.f;
-#pragma unroll
-                for (int j = 0; j < DV; ++j) {
-                    const float dv_ = (y[j] - mean) * c;
-                    s2 = fmaf(dv_, dv_, s2);
+                for (int j = 0; j < QC; ++j) {
+                    const float v = u2f(y[j]);
+                    s1 += v;
+                    const float yc = v * c;
+                    s2 = fmaf(yc, yc, s2);
                 }
-                a = c * rsqrtf(s2 * (1.0f / DV) + p.eps);
-                b0 = -mean * a;
+                const uint32_t xs = tm + lq + CF::TM_X + 8 * (i & 1);
+                const uint32_t mine[2] = {f2u(s1), f2u(s2)};
+                tmem_st_x2(xs + 2 * hf, mine);
+                tmem_wait_st();
+                tc_fence_before();
+                named_bar_sync(1 + q4, 128);
+                tc_fence_after();
+                uint32_t all[8];
+                tmem_ld_x8(xs, all);
+                tmem_wait_ld();
+                const float t1 = (u2f(all[0]) + u2f(all[2])) + (u2f(all[4]) + u2f(all[6]));
+                const float t2 = (u2f(all[1]) + u2f(all[3])) + (u2f(all[5]) + u2f(all[7]));
+                const float mean_u = t1 * (1.0f / DV);
+                const float mean_y = mean_u * c;
+                const float var = fmaxf(t2 * (1.0f / DV) - mean_y * mean_y, 0.f);
+                a = c * rsqrtf(var + p.eps);
+                b0 = -mean_u * a;
             }
-            if (p.has_g) mbar_wait(bar(BG), i & 1, p.status, abort_flag);
-            // this token's output row: 256 contiguous bytes of O, written straight
-            // to global memory (rows past the sequence's end are not written)
-            const bool live = n0 + row < n_end;
-            uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.O) +
-                                                   (((size_t)bb * p.N + n0 + row) * p.H + hh) * DV);
+            // this token's 32 output channels go over its G in the tile
+            mbar_wait(bar(BG), i & 1, p.status, abort_flag);
+            uint8_t* grow = sm + CF::OFF_G + (hf >> 1) * CF::BOX + row * 128;
 #pragma unroll
-            for (int ch = 0; ch < 16; ++ch) {
-                uint4 w = make_uint4(0u, 0u, 0u, 0u);
-                if (p.has_g)
-                    w = *reinterpret_cast<const uint4*>(sm + CF::OFF_G + (ch >> 3) * CF::BOX + row * 128 +
-                                                        (((ch & 7) ^ (row & 7)) << 4));
+            for (int ch = 0; ch < 4; ++ch) {
+                uint4* slot = reinterpret_cast<uint4*>(grow + ((((hf & 1) * 4 + ch) ^ (row & 7)) << 4));
+                uint4 w = p.has_g ? *slot : make_uint4(0u, 0u, 0u, 0u);
                 uint32_t* e = reinterpret_cast<uint32_t*>(&w);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    float o0 = fmaf(y[ch * 8 + 2 * j], a, b0), o1 = fmaf(y[ch * 8 + 2 * j + 1], a, b0);
+                    float o0 = fmaf(u2f(y[ch * 8 + 2 * j]), a, b0), o1 = fmaf(u2f(y[ch * 8 + 2 * j + 1]), a, b0);
                     if (p.gn) {
                         const float2 g = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&e[j]));
                         o0 *= swish_fast(g.x);
@@ -1670,9 +1877,10 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
                     }
                     e[j] = pack_bf16x2(o0, o1);
                 }
-                if (live) orow[ch] = w;
+                *slot = w;
             }
-            warp_arrive(BGF);              // the G tile may be reloaded
+            fence_proxy_async_smem();
+            warp_arrive(BGF);              // the tile holds this chunk's output
             lam = eager ? 0.f : lam + bC;
         }
     }
@@ -1734,6 +1942,46 @@ WsLayout ws_layout(int B, int H, int N, int dk, int dv, int chunk, int segments,
     return w;
 }
 
+// Workspace of a packed batch on the tensor-core path: decay sums, the state
+// pass's slots (at most max_state), and the plan.  seg_max is half of one SM's
+// share of the batch's token-heads (at least four chunks), so that the
+// longest-first order has pieces fine enough to even out; the item bounds follow
+// from sum over sequences of ceil(chunks / (seg_max / C)) <= S + (total / C + S) / (seg_max / C).
+struct VarlenLayout {
+    size_t bcum, eblk, state, decay, unit_info, fused, sitems, count, seq_info, seq_order, total;
+    int seg_max, max_fused, max_state, npad;
+};
+
+VarlenLayout varlen_layout(int S, int H, int max_seqlen, int total, int dk, int dv, int chunk, int num_sms) {
+    VarlenLayout w;
+    const long long units = (long long)S * H;
+    const long long share = ((long long)total * H + 2LL * num_sms - 1) / (2LL * (num_sms > 0 ? num_sms : 1));
+    long long seg_max = (share + chunk - 1) / chunk * chunk;
+    if (seg_max < 4LL * chunk) seg_max = 4LL * chunk;
+    if (seg_max > (1LL << 30)) seg_max = (1LL << 30) / chunk * chunk;
+    const long long maxch = seg_max / chunk;
+    const long long chunks_bound = ((long long)total + chunk - 1) / chunk + S;
+    const long long long_bound = (chunks_bound + maxch - 1) / maxch;
+    w.seg_max = (int)seg_max;
+    w.max_fused = (int)std::min<long long>((long long)H * (S + long_bound), 1LL << 30);
+    w.max_state = (int)std::min<long long>((long long)H * long_bound, 1LL << 30);
+    w.npad = (max_seqlen + chunk - 1) / chunk * chunk;
+    size_t off = 0;
+    auto take = [&](size_t bytes) { const size_t at = off; off += align256(bytes); return at; };
+    w.bcum = take((size_t)units * w.npad * 4);
+    w.eblk = take((size_t)units * w.npad * 4);
+    w.state = take((size_t)w.max_state * dk * dv * 4);
+    w.decay = take((size_t)w.max_state * 4);
+    w.unit_info = take((size_t)units * 16);
+    w.fused = take((size_t)w.max_fused * 8);
+    w.sitems = take((size_t)w.max_state * 8);
+    w.count = take(16);
+    w.seq_info = take((size_t)S * 8);
+    w.seq_order = take((size_t)S * 4);
+    w.total = off;
+    return w;
+}
+
 // Launch with programmatic stream serialisation: the kernel may start while the
 // one before it in the stream finishes; each kernel waits (grid_dep_wait)
 // before it touches what the earlier ones wrote.
@@ -1754,7 +2002,7 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 }
 
 template <int DV, int C, bool PACKED>
-cudaError_t run_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t s) {
+cudaError_t run_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t s, const PlanArgs* plan = nullptr) {
     using CF = Cfg<DV, C>;
     auto kf = prefill_tc_kernel<DV, C, PACKED>;
     auto ks = prefill_state_kernel<DV, C, PACKED>;
@@ -1774,6 +2022,29 @@ cudaError_t run_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t s) {
     const int units = a.B * a.H;
     const int npad = tp.Npad;
     cudaError_t e = cudaSuccess;
+    if constexpr (PACKED) {
+        // gate scan, plan, state pass and combine over the plan's slots, fused loop
+        int nyb = 0;
+        const dim3 sgrid = gate_scan_grid(units, npad, C, &nyb);
+        if (g_profile_gate_start) cudaEventRecord(g_profile_gate_start, s);
+        e = launch_pdl(gate_scan_kernel, sgrid, dim3(kScanThreads), 0, s, a.z, a.cu_seqlens, a.total,
+                       const_cast<float*>(tp.bcum), const_cast<float*>(tp.eblk), a.H, a.N, npad, C, a.inv_tau, nyb);
+        if (g_profile_gate_stop) cudaEventRecord(g_profile_gate_stop, s);
+        if (e != cudaSuccess) return e;
+        e = launch_pdl(varlen_plan_kernel, dim3(1), dim3(kPlanThreads), 0, s, *plan);
+        if (e != cudaSuccess) return e;
+        e = launch_pdl(ks, dim3(plan->max_state), dim3(kStateThreads), StateCfg<DV, C>::SMEM, s, tp);
+        if (e != cudaSuccess) return e;
+        const int elems4 = DV * DK / 4;
+        e = launch_pdl(seg_combine_kernel, dim3(units, (elems4 + 255) / 256), dim3(256), 0, s, tp.seg_state,
+                       static_cast<const float*>(tp.seg_decay), tp.S0, 0, DK, DV, tp.unit_info);
+        if (e != cudaSuccess) return e;
+        if (g_profile_start) cudaEventRecord(g_profile_start, s);
+        e = launch_pdl(kf, dim3(plan->max_fused), dim3(kFusedThreads), CF::SMEM, s, tp);
+        if (g_profile_stop) cudaEventRecord(g_profile_stop, s);
+        if (e != cudaSuccess) return e;
+        return cudaGetLastError();
+    }
     if (a.resume) {
         // the gate scan and the state pass ran in gret_prefill_state: shift its
         // folded slots by the initial state, then the fused loop
@@ -1801,7 +2072,8 @@ cudaError_t run_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t s) {
         if (e != cudaSuccess) return e;
         const int elems4 = DV * DK / 4;
         e = launch_pdl(seg_combine_kernel, dim3(units, (elems4 + 255) / 256), dim3(256), 0, s, tp.seg_state,
-                       static_cast<const float*>(tp.seg_decay), tp.S0, tp.slots, DK, DV);
+                       static_cast<const float*>(tp.seg_decay), tp.S0, tp.slots, DK, DV,
+                       static_cast<const int4*>(nullptr));
         if (e != cudaSuccess) return e;
     }
 #ifndef GRET_ROWS_KERNEL
@@ -1814,8 +2086,7 @@ cudaError_t run_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t s) {
         if (dev < 0 || dev >= 64 || !rows_attr_done[dev]) {
             cudaFuncAttributes fa;
             if (cudaFuncGetAttributes(&fa, kr) != cudaSuccess) return cudaErrorInvalidDeviceFunction;
-            if (fa.numRegs * kRowsThreads < 128 * kRowsERegs + 384 * kRowsOtherRegs)
-                return cudaErrorInvalidConfiguration;
+            if (fa.numRegs > kRowsRegs) return cudaErrorInvalidConfiguration;
             cudaFuncSetAttribute(kr, cudaFuncAttributeMaxDynamicSharedMemorySize, RowsCfg::SMEM);
             if (dev >= 0 && dev < 64) rows_attr_done[dev] = true;
         }
@@ -1893,6 +2164,11 @@ size_t prefill_tc_workspace_bytes(int B, int H, int N, int dk, int dv, int chunk
     return ws_layout(B, H, N, dk, dv, chunk, segments, pieces).total;
 }
 
+size_t prefill_tc_varlen_workspace_bytes(int S, int H, int max_seqlen, int total, int dk, int dv, int chunk,
+                                         int num_sms) {
+    return varlen_layout(S, H, max_seqlen, total, dk, dv, chunk, num_sms).total;
+}
+
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
     TcParams tp;
     memset(&tp, 0, sizeof(tp));
@@ -1907,14 +2183,45 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
     tp.cu = a.cu_seqlens;
     tp.total = a.total;
     tp.O = a.O;
-    // a resumed prefill reads the layout gret_prefill_state wrote: a slot for
-    // every piece of every segment
-    const WsLayout w = ws_layout(a.B, a.H, a.N, a.dk, a.dv, C, a.segments + (a.resume ? 1 : 0), a.pieces);
+    tp.G = a.G;
     uint8_t* ws = static_cast<uint8_t*>(a.workspace);
-    tp.bcum = reinterpret_cast<const float*>(ws + w.bcum);
-    tp.eblk = reinterpret_cast<const float*>(ws + w.eblk);
-    tp.seg_state = reinterpret_cast<float*>(ws + w.state);
-    tp.seg_decay = reinterpret_cast<float*>(ws + w.decay);
+    PlanArgs plan;
+    memset(&plan, 0, sizeof(plan));
+    if (a.cu_seqlens) {
+        // a packed batch works from the plan its own kernel makes
+        const VarlenLayout v = varlen_layout(a.B, a.H, a.N, a.total, a.dk, a.dv, C, a.num_sms);
+        tp.bcum = reinterpret_cast<const float*>(ws + v.bcum);
+        tp.eblk = reinterpret_cast<const float*>(ws + v.eblk);
+        tp.seg_state = reinterpret_cast<float*>(ws + v.state);
+        tp.seg_decay = reinterpret_cast<float*>(ws + v.decay);
+        tp.unit_info = reinterpret_cast<const int4*>(ws + v.unit_info);
+        tp.fused_items = reinterpret_cast<const int2*>(ws + v.fused);
+        tp.state_items = reinterpret_cast<const int2*>(ws + v.sitems);
+        tp.plan_count = reinterpret_cast<const int*>(ws + v.count);
+        plan.cu = a.cu_seqlens;
+        plan.total = a.total;
+        plan.S = a.B;
+        plan.H = a.H;
+        plan.C = C;
+        plan.seg_max = v.seg_max;
+        plan.max_len = a.N;
+        plan.unit_info = reinterpret_cast<int4*>(ws + v.unit_info);
+        plan.fused_items = reinterpret_cast<int2*>(ws + v.fused);
+        plan.state_items = reinterpret_cast<int2*>(ws + v.sitems);
+        plan.count = reinterpret_cast<int*>(ws + v.count);
+        plan.seq_info = reinterpret_cast<int2*>(ws + v.seq_info);
+        plan.seq_order = reinterpret_cast<int*>(ws + v.seq_order);
+        plan.max_fused = v.max_fused;
+        plan.max_state = v.max_state;
+    } else {
+        // a resumed prefill reads the layout gret_prefill_state wrote: a slot for
+        // every piece of every segment
+        const WsLayout w = ws_layout(a.B, a.H, a.N, a.dk, a.dv, C, a.segments + (a.resume ? 1 : 0), a.pieces);
+        tp.bcum = reinterpret_cast<const float*>(ws + w.bcum);
+        tp.eblk = reinterpret_cast<const float*>(ws + w.eblk);
+        tp.seg_state = reinterpret_cast<float*>(ws + w.state);
+        tp.seg_decay = reinterpret_cast<float*>(ws + w.decay);
+    }
     tp.S_final = a.S_final;
     tp.S0 = a.S0;
     tp.status = a.status;
@@ -1931,9 +2238,12 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
     tp.has_g = (a.epi == GRET_EPI_GN_SWISH && a.G) ? 1 : 0;
     tp.fault = a.fault;
     const bool packed = a.cu_seqlens != nullptr;
-    if (a.dv == 256 && C == 64) return packed ? run_tc<256, 64, true>(a, tp, s) : run_tc<256, 64, false>(a, tp, s);
-    if (a.dv == 128 && C == 128) return packed ? run_tc<128, 128, true>(a, tp, s) : run_tc<128, 128, false>(a, tp, s);
-    if (a.dv == 128 && C == 64) return packed ? run_tc<128, 64, true>(a, tp, s) : run_tc<128, 64, false>(a, tp, s);
+    if (a.dv == 256 && C == 64)
+        return packed ? run_tc<256, 64, true>(a, tp, s, &plan) : run_tc<256, 64, false>(a, tp, s);
+    if (a.dv == 128 && C == 128)
+        return packed ? run_tc<128, 128, true>(a, tp, s, &plan) : run_tc<128, 128, false>(a, tp, s);
+    if (a.dv == 128 && C == 64)
+        return packed ? run_tc<128, 64, true>(a, tp, s, &plan) : run_tc<128, 64, false>(a, tp, s);
     return cudaErrorNotSupported;
 }
 
@@ -1954,7 +2264,8 @@ static cudaError_t run_state_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t
     // increment from the slice's start through piece j
     const int elems4 = DV * DK / 4;
     e = launch_pdl(seg_combine_kernel, dim3(units, (elems4 + 255) / 256), dim3(256), 0, s, tp.seg_state,
-                   static_cast<const float*>(tp.seg_decay), static_cast<const float*>(nullptr), tp.slots, DK, DV);
+                   static_cast<const float*>(tp.seg_decay), static_cast<const float*>(nullptr), tp.slots, DK, DV,
+                   static_cast<const int4*>(nullptr));
     if (e != cudaSuccess) return e;
     state_finish_kernel<DV><<<dim3(units, (DV / 32) * (DK / 32)), dim3(32, 8), 0, s>>>(tp.seg_state, tp.seg_decay,
                                                                                   tp.slots, a.S_final, a.decay_out);

@@ -73,6 +73,8 @@ SIGNATURES = {
     "gret_prefill_varlen": (_I, [_VP, _VP, _VP, _FP, _VP, _FP, _VP, _I, _I, _I, _F, _I, _VP, _FP, _I, _I, _I, _I,
                                  _F, _I, _VP, _SZ, _VP]),
     "gret_prefill_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
+    "gret_prefill_varlen_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I, _I]),
+    "gret_prefill_varlen_launches": (_I, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "gret_prefill_launches": (_I, [_I, _I, _I, _I, _I, _I, _I]),
     "gret_prefill_path": (_I, [_I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_int)]),
     "gret_decode_step": (_I, [_VP, _VP, _VP, _FP, _VP, _FP, _VP, _I, _I, _I, _I, _F, _I, _F, _I, _VP]),
@@ -167,6 +169,15 @@ def gret_prefill_noalloc(Q, K, V, gate_logits, G, tau, chunk, O, S_final, B, H, 
 
 def gret_prefill_workspace_size(B, H, N, dk, dv, chunk, io_dtype) -> int:
     return load().gret_prefill_workspace_size(B, H, N, dk, dv, chunk, int(io_dtype))
+
+
+def gret_prefill_varlen_workspace_size(num_seqs, total_tokens, max_seqlen, H, dk, dv, chunk, io_dtype) -> int:
+    return load().gret_prefill_varlen_workspace_size(num_seqs, total_tokens, max_seqlen, H, dk, dv, chunk,
+                                                     int(io_dtype))
+
+
+def gret_prefill_varlen_launches(num_seqs, total_tokens, max_seqlen, H, dk, dv, chunk, io_dtype) -> int:
+    return load().gret_prefill_varlen_launches(num_seqs, total_tokens, max_seqlen, H, dk, dv, chunk, int(io_dtype))
 
 
 def gret_prefill_launches(B, H, N, dk, dv, chunk, io_dtype) -> int:
@@ -410,7 +421,7 @@ def prefill_varlen(Q, K, V, z, G, cu_seqlens, max_seqlen: int, tau: float, chunk
     if S0 is not None:
         _check(S0, "S0", torch.float32, (S, H, dk, dv), dev)
     with torch.cuda.device(dev):
-        ws_bytes = gret_prefill_workspace_size(S, H, max_seqlen, dk, dv, chunk, io)
+        ws_bytes = gret_prefill_varlen_workspace_size(S, T, max_seqlen, H, dk, dv, chunk, io)
         st = stream if stream is not None else torch.cuda.current_stream(dev)
         workspace = _scratch(workspace, ws_bytes, dev, st)
         status = gret_prefill_varlen(_ptr(Q), _ptr(K), _ptr(V), _ptr(z), _ptr(G), _ptr(S0), _ptr(cu_seqlens), S, T,

@@ -130,11 +130,20 @@ gret_status gret_prefill_from_state(const void* Q, const void* K, const void* V,
  *   max_seqlen  the longest sequence (>= every length; sizes the work split).
  *   S0, S_final fp32 [num_seqs][H][dk][dv]; S0 may be NULL (zero state); the
  *               rule of gret_prefill_from_state on overlap applies.
- * Workspace: gret_prefill_workspace_size(num_seqs, H, max_seqlen, dk, dv,
- * chunk, io_dtype) bytes.  Every sequence gives what gret_prefill_from_state
- * gives for it alone; nothing is written outside its rows.  Offsets outside
- * [0, total_tokens] are clamped into it; tokens past max_seqlen in a sequence
- * are not processed.  cu_seqlens must be 4-byte aligned; total_tokens > 0.
+ * Workspace: gret_prefill_varlen_workspace_size(num_seqs, total_tokens,
+ * max_seqlen, H, dk, dv, chunk, io_dtype) bytes.  Every sequence gives what
+ * gret_prefill_from_state gives for it alone; nothing is written outside its
+ * rows.  Offsets outside [0, total_tokens] are clamped into it; tokens past
+ * max_seqlen in a sequence are not processed.  cu_seqlens must be 4-byte
+ * aligned; total_tokens > 0.
+ *
+ * On the tensor-core path the work is planned on the device from cu_seqlens
+ * (no host synchronisation): a sequence longer than half of one SM's share of the
+ * batch's tokens and heads is cut into segments of equal length -- a state
+ * pass gives each segment its initial state -- while the others stay whole,
+ * and the segments start longest first, so that one long prompt among short
+ * ones does not finish alone.  The call then makes
+ * gret_prefill_varlen_launches(...) launches.
  */
 gret_status gret_prefill_varlen(const void* Q, const void* K, const void* V, const float* gate_logits,
                                 const void* G, const float* S0, const int* cu_seqlens, int num_seqs,
@@ -142,6 +151,10 @@ gret_status gret_prefill_varlen(const void* Q, const void* K, const void* V, con
                                 float* S_final, int H, int dk, int dv, gret_dtype io_dtype, float eps,
                                 gret_epilogue epi, void* workspace, size_t workspace_bytes,
                                 gret_stream_t stream);
+size_t gret_prefill_varlen_workspace_size(int num_seqs, int total_tokens, int max_seqlen, int H, int dk, int dv,
+                                          int chunk, gret_dtype io_dtype);
+int gret_prefill_varlen_launches(int num_seqs, int total_tokens, int max_seqlen, int H, int dk, int dv, int chunk,
+                                 gret_dtype io_dtype);
 
 /*
  * Sequence-parallel prefill ("YOCO 深度技术分析", section 5.3.3, Chunk
@@ -308,7 +321,7 @@ gret_status gret_last_device_status(gret_stream_t stream);
  *
  * "YOCO 深度技术分析", section 2.2: gamma = sigmoid(X W_gamma)^(1/tau), with one
  * column of W_gamma per head, so z[b][n][h] = sum_i X[b][n][i] W_gamma[i][h].
- * On the tensor-core path (bf16, as gret_prefill_path reports) with H <= 256
+ * On the tensor-core path (bf16, as gret_prefill_path reports) with H <= 128
  * and d_model a multiple of 8, z is a tcgen05 product inside the kernel that
  * scans the gate (W_gamma fed as two bf16 halves for fp32-level accuracy) and
  * never reaches memory; elsewhere a CUDA-core kernel writes z into the

@@ -97,3 +97,30 @@ def test_bf16_cuda_core_chunked_path():
     cfg = gi.C2.scaled(B=1, H=2, N=150, dk=64, dv=128, seed=79)
     assert gret.gret_prefill_backward_launches(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, gret.Dtype.BF16) == 5
     _run(cfg)
+
+
+@pytest.mark.slow
+def test_bf16_full_benchmark_length_sampled_units():
+    """The benchmark's whole backward (B4 H16 N4096, d_k 128, d_v 256, both
+    states given), as the bench launches it; sampled (batch, head) units -- each
+    depends on its own inputs only -- against the oracle run on that unit alone
+    over all 4096 tokens."""
+    cfg = gi.C2
+    inp = gi.prefill_inputs(cfg)
+    shape_o = (cfg.B, cfg.N, cfg.H, cfg.dv)
+    shape_s = (cfg.B, cfg.H, cfg.dk, cfg.dv)
+    dO = gi.random_unit(cfg.seed, 910, shape_o, io=cfg.io)
+    S0 = gi.random_unit(cfg.seed, 911, shape_s, var=0.04)
+    dSf = gi.random_unit(cfg.seed, 912, shape_s, var=0.01)
+    d = {k: v.cuda() for k, v in inp.items()}
+    got = gret.prefill_backward(d["Q"], d["K"], d["V"], d["z"], d["G"], dO.cuda(), cfg.tau, eps=cfg.eps,
+                                S0=S0.cuda(), dS_final=dSf.cuda())
+    gret.check_device_status()
+    for b, h in ((0, 0), (3, 15)):
+        u = lambda x: x[b:b + 1, :, h:h + 1]  # noqa: E731
+        ref = og.prefill_backward(u(inp["Q"]), u(inp["K"]), u(inp["V"]), u(inp["z"]), u(inp["G"]), cfg.tau,
+                                  cfg.eps, u(dO), S0=S0[b:b + 1, h:h + 1], dS_final=dSf[b:b + 1, h:h + 1])
+        for name in ("dQ", "dK", "dV", "dG"):
+            assert_close(u(got[name]), ref[name], "bf16", f"{name} unit {(b, h)}")
+        assert_close(got["dz"][b:b + 1, :, h:h + 1], ref["dz"], "bf16", f"dz unit {(b, h)}")
+        assert_close(got["dS0"][b:b + 1, h:h + 1], ref["dS0"], "bf16", f"dS0 unit {(b, h)}")
