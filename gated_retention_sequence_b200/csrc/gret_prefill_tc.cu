@@ -1414,20 +1414,23 @@ __global__ void state_fold_kernel(const float* __restrict__ dS_all, const float*
 // Q~_t = e^{b_t + Lambda} Q_t against the unscaled T, then T *= e^{Lambda + b_C},
 // K~_s = e^{b_C - b_s} K_s and Lambda = 0.  All exponents stay <= kLazyMax.
 //
-// Roles (896 threads, seven warpgroups, 72 registers each).  Warps 0-15 (E):
-// epilogue, four warps per tensor-memory lane quarter, each owning 32 of a
-// token's 128 channels; the four quarters' partial sums of a token meet in
-// spare tensor-memory columns of its lane (two sets, by chunk parity).  Warps
-// 16-19 (P): masked scores -> bf16 P in tensor memory; causality leaves lane
-// quarter q with q + 1 nonzero 32-column blocks, so warps 26 and 27 (lane
-// quarters 2 and 3) take the blocks past the second of the two heaviest
-// quarters and no warp converts more than two.  The blocks above the diagonal
-// stay zero and are written once.  Warps 20-23 (S): K~ and Q~ in shared memory
-// (one token row per thread), the bf16 copy of T after each state update, the
-// eager rescale, the initial and final state.  Warp 24 lane 0 issues every
-// MMA; warp 25 lane 0 every TMA load and the output store.  The roles work on
-// different chunks at once: E finishes chunk i while S and P prepare chunk
-// i + 1 and the tensor cores run its products.
+// Roles (896 threads, seven warpgroups).  Warps 0-15 (E): epilogue, four warps
+// per tensor-memory lane quarter, each owning 32 of a token's 128 channels; the
+// four quarters' partial sums of a token meet in spare tensor-memory columns of
+// its lane (two sets, by chunk parity).  After the output of chunk i they scale
+// K~ of a lazy chunk i + 2 (a quarter of a token row per thread).  Warps 16-19
+// (P): masked scores -> bf16 P in tensor memory; causality leaves lane quarter
+// q with q + 1 nonzero 32-column blocks, so warps 26 and 27 (lane quarters 2
+// and 3) take the blocks past the second of the two heaviest quarters and no
+// warp converts more than two.  The blocks above the diagonal stay zero and
+// are written once.  Warps 20-23 (S): the bf16 copy of T after each state
+// update, and for eager chunks the rescale of T and the scaling of Q~ and K~
+// after the scores; the initial and final state.  Warp 24 lane 0 issues every
+// MMA; warp 25 lane 0 every TMA load and the output store.  Per chunk the MMA
+// warp issues the scores, the inter-chunk product, the state update (which
+// needs neither P nor the output) and last the intra-chunk product, so that
+// the tensor cores work while the P warps convert the scores; a chunk's V is
+// released by its intra-chunk product, its Q and K by the state update.
 constexpr int kRowsThreads = 896;
 constexpr int kRowsRegs = 72;          // 65536 / 896, rounded down to 8
 constexpr int kRowsSRegs = 64;         // the S warps hand registers to the issuing warps
@@ -1496,8 +1499,9 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
             // per-warp arrivals: sixteen epilogue warps, six P warps, or one
             // four-warp role
             const bool sixteen = i == BOF || i == BGF;
-            const bool four = i == BKT || i == BKT + 1 || i == BTC || i == BQT;
-            mbar_init(bar(i), sixteen ? 16 : four ? 4 : i == BPR ? 6 : 1);
+            const bool four = i == BTC || i == BQT;
+            const bool kt = i == BKT || i == BKT + 1;   // every chunk: the E and the S warps
+            mbar_init(bar(i), sixteen ? 16 : four ? 4 : kt ? 20 : i == BPR ? 6 : 1);
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -1604,9 +1608,11 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
                 issue_v(0);
                 issue_g(0);
                 for (int i = 0; i < nchunks; ++i) {
-                    // the state MMA of chunk i is the last reader of its Q/K stage and of V
+                    // the state MMA of chunk i is the last reader of its Q/K stage,
+                    // the intra-chunk MMA the last reader of V
                     if (!mbar_wait(bar(BST), i & 1, p.status, abort_flag)) break;
                     if (i + 2 < nchunks) issue_qk(i + 2);
+                    if (!mbar_wait(bar(BOD), i & 1, p.status, abort_flag)) break;
                     if (i + 1 < nchunks) issue_v(i + 1);
                     // the output of chunk i leaves from the tile (rows past the end of
                     // the sequence fall outside the map and are not written); once the
@@ -1665,15 +1671,9 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
                     mma_ss(tm + CF::TM_O, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(sT + off, 16, 1024), id_kk,
                            k > 0);
                 }
-                // intra-chunk: O += P V
-                if (!mbar_wait(bar(BPR), i & 1, p.status, abort_flag)) break;
+                // state: T^T += V^T K~ (eager: K~ is scaled after the scores); it
+                // needs neither P nor the output, so it runs while P is converted
                 if (!mbar_wait(bar(BV), i & 1, p.status, abort_flag)) break;
-                tc_fence_after();
-#pragma unroll
-                for (int k = 0; k < C / 16; ++k)
-                    mma_ts(tm + CF::TM_O, tm + CF::TM_P + k * 8, sdesc_sw128(sV + k * 2048, CF::BOX, 1024), id_pv, 1);
-                mma_commit(bar(BOD));
-                // state: T^T += V^T K~ (eager: K~ is scaled after the scores)
                 if (eager && !mbar_wait(bar(BKT + s), (i >> 1) & 1, p.status, abort_flag)) break;
                 tc_fence_after();
 #pragma unroll
@@ -1681,6 +1681,13 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
                     mma_ss(tm + CF::TM_T, sdesc_sw128(sV + k * 2048, CF::BOX, 1024),
                            sdesc_sw128(sK + k * 2048, CF::BOX, 1024), id_kv, 1);
                 mma_commit(bar(BST));
+                // intra-chunk: O += P V
+                if (!mbar_wait(bar(BPR), i & 1, p.status, abort_flag)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < C / 16; ++k)
+                    mma_ts(tm + CF::TM_O, tm + CF::TM_P + k * 8, sdesc_sw128(sV + k * 2048, CF::BOX, 1024), id_pv, 1);
+                mma_commit(bar(BOD));
                 lam = eager ? 0.f : lam + bC;
             }
             // every MMA this thread issued has completed before tensor memory is freed
@@ -1729,11 +1736,9 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
             const float bC = bc[C - 1];
             const bool eager = (-bC - lam) > kLazyMax;
             const float brow = bc[row];
-            if (!eager) {
-                scale_tile_row(Kp, row, __expf(-brow - lam));
-                fence_proxy_async_smem();
-                warp_arrive(BKT + s);
-            }
+            // a lazy chunk's K~ is the E warps' (before its scores); an eager
+            // chunk's is scaled here after its scores
+            if (!eager) warp_arrive(BKT + s);
             // bf16 copy of T^T for this chunk's inter-chunk product, once the
             // previous state update is done (it also finished the previous
             // inter-chunk product, the last reader of the copy); eager chunks
@@ -1813,6 +1818,28 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
         constexpr int QC = DV / 4;
         float lam = 0.f;
         const float* bsum = p.bcum + (size_t)u * p.Npad;
+        // K~_s = e^{-b_s - Lambda} K_s of a lazy chunk j, in place: token row
+        // tid % 128, its 16-byte words 4 (tid / 128) .. + 3; an eager chunk's K
+        // stays raw for its scores (the S warps scale it after them).  Chunks
+        // are taken in order, so Lambda follows them.
+        float lam_k = 0.f;
+        auto scale_k = [&](int j) {
+            const int s = j & 1, kr = tid & (C - 1), part = tid >> 7;
+            const float* bc = stage_bc(j);
+            mbar_wait(bar(BQK + s), (j >> 1) & 1, p.status, abort_flag);
+            const float bCj = bc[C - 1];
+            const bool eg = (-bCj - lam_k) > kLazyMax;
+            if (!eg) {
+                const float f = __expf(-bc[kr] - lam_k);
+                uint8_t* krow = sm + CF::OFF_K + s * CF::TILE + (part >> 1) * CF::BOX + kr * 128;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) scale_bf16x8(krow + ((((part & 1) * 4 + c) ^ (kr & 7)) << 4), f);
+                fence_proxy_async_smem();
+            }
+            warp_arrive(BKT + s);
+            lam_k = eg ? 0.f : lam_k + bCj;
+        };
+        for (int j = 0; j < 2 && j < nchunks; ++j) scale_k(j);
         for (int i = 0; i < nchunks; ++i) {
             const int n0 = n_begin + i * C;
             const float bt = bsum[n0 + row], bC = bsum[n0 + C - 1];
@@ -1882,6 +1909,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
             fence_proxy_async_smem();
             warp_arrive(BGF);              // the tile holds this chunk's output
             lam = eager ? 0.f : lam + bC;
+            if (i + 2 < nchunks) scale_k(i + 2);
         }
     }
     tc_fence_before();
