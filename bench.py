@@ -56,9 +56,17 @@ PREFILL_SOURCE = "gated_retention_sequence_b200/csrc/gret_prefill_tc.cu"
 PREFILL_CONFIGS = ("c3", "c2", "c5")
 
 
+def fused_kernel_name(cfg):
+    """The fused chunk-loop kernel that runs this workload: 128-token chunks with
+    d_v = 128 (bf16) take the output-rows kernel, the others prefill_tc_kernel."""
+    if cfg.io == "bf16" and cfg.dv == 128 and cfg.chunk == 128:
+        return "prefill_rows_kernel"
+    return "prefill_tc_kernel"
+
+
 def prefill_profile(cfg):
     """Name of the ncu summary of the fused kernel on this workload."""
-    return (f"prefill_tc_kernel_B{cfg.B}_H{cfg.H}_N{cfg.N}_dk{cfg.dk}_dv{cfg.dv}_C{cfg.chunk}.md")
+    return (f"{fused_kernel_name(cfg)}_B{cfg.B}_H{cfg.H}_N{cfg.N}_dk{cfg.dk}_dv{cfg.dv}_C{cfg.chunk}.md")
 
 
 def load_peaks():
@@ -349,7 +357,9 @@ def prefill_summary(cfg, world, steps, ms, kern_ms, peaks):
                "frac_of_bf16_peak": alg_flops / step_s / 1e12 / peaks["bf16_tflops"],
                "peak_tflops": peaks["bf16_tflops"], "peak_source": peaks["source"] + " burst"},
         "path_hbm": {"alg_gbs": alg_bytes / step_s / 1e9, "frac": alg_bytes / step_s / 1e9 / peaks["hbm_gbs"]},
-        "roofline": {"kernel": f"prefill_tc_kernel<{cfg.dv}, {cfg.chunk}> (fused chunk loop)", "bound": "hbm",
+        "roofline": {"kernel": (f"{fused_kernel_name(cfg)}<{cfg.dv}, {cfg.chunk}> (fused chunk loop)"
+                                if fused_kernel_name(cfg) == "prefill_tc_kernel"
+                                else f"{fused_kernel_name(cfg)} (fused chunk loop, output rows)"), "bound": "hbm",
                      "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"],
                      "traffic": profiled_traffic(prefill_profile(cfg), PREFILL_SOURCE),

@@ -144,6 +144,7 @@ struct TcParams {
     unsigned int* status;
     int H, N, Npad, P, seg_len;
     int K, piece_len;        // state-pass pieces per segment and their length
+    int piece_split;         // > 0: K = 2 pieces of piece_split and seg_len / C - piece_split chunks
     int slots;               // state-pass pieces (and seg_state slots) per unit
     // planned packed batch (varlen_plan_kernel): per unit {segments, segment
     // length, first seg_state slot, -}; the fused and state-pass work items
@@ -933,11 +934,24 @@ __global__ void __launch_bounds__(kStateThreads, 1) prefill_state_kernel(const _
     // work item: a piece of the uniform split, or a segment of a packed
     // batch's plan (one piece per segment; a block past the plan's count has
     // nothing to do)
-    int u = 0, seg = 0, piece_len = p.piece_len;
+    int u = 0, seg = 0, piece_len = p.piece_len, n_begin = 0;
     size_t out_slot = 0;
     if constexpr (!PACKED) {
-        u = blockIdx.x / p.slots;
-        seg = blockIdx.x % p.slots;
+        if (p.piece_split > 0) {
+            // each segment in a long and a short piece: the long ones first (the
+            // lower block indices start first), the short ones after, two to an SM
+            const int nseg = p.slots / 2, nlong = (int)gridDim.x / 2;
+            const int b = (int)blockIdx.x, second = b >= nlong ? 1 : 0, bi = b - second * nlong;
+            u = bi / nseg;
+            const int sg = bi % nseg;
+            seg = 2 * sg + second;
+            n_begin = sg * p.seg_len + second * p.piece_split * C;
+            piece_len = second ? p.seg_len - p.piece_split * C : p.piece_split * C;
+        } else {
+            u = blockIdx.x / p.slots;
+            seg = blockIdx.x % p.slots;
+            n_begin = seg * piece_len;
+        }
         out_slot = (size_t)u * p.slots + seg;
     } else {
         grid_dep_wait();
@@ -947,10 +961,10 @@ __global__ void __launch_bounds__(kStateThreads, 1) prefill_state_kernel(const _
         u = it.x;
         seg = it.y;
         piece_len = ui.y;
+        n_begin = seg * piece_len;
         out_slot = (size_t)ui.z + seg;
     }
     const int hh = u % p.H;
-    const int n_begin = seg * piece_len;
 
     auto full = [&](int s) -> uint32_t { return sb + CF::OFF_BAR + 8 * s; };
     auto empty = [&](int s) -> uint32_t { return sb + CF::OFF_BAR + 8 * (NS + s); };
@@ -2138,9 +2152,34 @@ bool prefill_tc_supported(int dk, int dv, int chunk, gret_dtype io) {
     return (dv == 128 && (chunk == 64 || chunk == 128)) || (dv == 256 && chunk == 64);
 }
 
+// State-pass pieces of a split that leaves SMs idle with one piece per segment
+// but would need a second wave with two equal ones (units * (P - 1) segments,
+// between half the SMs and all of them): each segment is cut into a long piece
+// of a chunks and a short one of b, a = k b, where k is the number of short
+// pieces each remaining SM takes one after the other.  Returns a (0: no such cut).
+static int uneven_piece_split(long long units, int segments, int per, int num_sms) {
+    const long long n = units * (segments - 1);
+    if (segments < 2 || per < 3 || n >= num_sms || 2 * n <= num_sms) return 0;
+    const long long spare = num_sms - n;
+    const long long k = (n + spare - 1) / spare;
+    const int b = (int)(per / (k + 1));
+    return b >= 1 ? per - b : 0;
+}
+
+int prefill_tc_piece_split(int B, int H, int chunk, int num_sms, int segments, int seg_len, int pieces) {
+    const long long units = (long long)B * H;
+    const int per = seg_len / chunk;
+    if (pieces != 2 || segments < 2 || units < 1) return 0;
+    const long long kmax = num_sms / (units * (segments - 1));
+    if (kmax >= 2 && per % 2 == 0) return 0;                 // two equal pieces fit one wave
+    return uneven_piece_split(units, segments, per, num_sms);
+}
+
 // Segments: about one fused CTA per SM.  State-pass pieces: each of the first
 // P-1 segments is cut into K pieces (K divides the segment's chunk count) so
-// that the state pass, too, has about one CTA per SM.
+// that the state pass, too, has about one CTA per SM; where one piece per
+// segment would leave SMs idle and two equal ones need a second wave, a long and
+// a short piece (uneven_piece_split).
 void prefill_tc_plan(int B, int H, int N, int chunk, int num_sms, int* segments, int* seg_len, int* pieces) {
     const int units = B * H > 0 ? B * H : 1;
     const int nchunks = (N + chunk - 1) / chunk;
@@ -2155,6 +2194,7 @@ void prefill_tc_plan(int B, int H, int N, int chunk, int num_sms, int* segments,
         const int kmax = num_sms / (units * (*segments - 1));
         for (int k = kmax < per ? kmax : per; k >= 1; --k)
             if (per % k == 0) { K = k; break; }
+        if (K == 1 && uneven_piece_split(units, *segments, per, num_sms) > 0) K = 2;
     }
     *pieces = K;
 }
@@ -2261,6 +2301,8 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
     tp.K = a.pieces;
     tp.piece_len = a.seg_len / a.pieces;
     tp.slots = (a.segments - (a.resume ? 0 : 1)) * a.pieces;
+    tp.piece_split = (a.resume || a.cu_seqlens)
+                         ? 0 : prefill_tc_piece_split(a.B, a.H, C, a.num_sms, a.segments, a.seg_len, a.pieces);
     tp.eps = a.eps;
     tp.gn = a.epi == GRET_EPI_GN_SWISH ? 1 : 0;
     tp.has_g = (a.epi == GRET_EPI_GN_SWISH && a.G) ? 1 : 0;

@@ -152,3 +152,14 @@ def test_state_pass_pieces():
                                          sl(inp["G"]), cfg.tau, cfg.eps)
         assert_close(O[:, :, h:h + 1], O_ref, "bf16", f"O head {h}")
         assert_close(Sf[:, h:h + 1], S_ref, "bf16", f"S head {h}")
+
+
+@pytest.mark.parametrize("dv,chunk,N", [(128, 64, 14245), (128, 128, 28501)])
+def test_state_pass_long_and_short_pieces(dv, chunk, N):
+    """Eight units split into 18 segments: the 136 segments before the last of
+    each unit are fewer than the SMs but more than half of them, so the state
+    pass cuts each into a long and a short piece (more than 13 chunks per
+    segment); the carried states must be those of the unsplit recurrence."""
+    cfg = _cfg(1, 8, N, dv, chunk, 500 + chunk, z_dist=((4.0, 1.0),))
+    segs = _check_full(cfg)
+    assert segs == 18
