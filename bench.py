@@ -192,19 +192,35 @@ def barrier(world):
         torch.cuda.synchronize()
 
 
-def profiled_traffic(kernel_file, source):
+# The output-rows kernel's text within its source file (from the first marker
+# up to the second): its ncu summary records the sha256 of this text only.
+ROWS_KERNEL_TEXT = ("// Fused chunk loop for 128-token chunks with d_v = 128, output held as rows.",
+                    "// ---------------------------------------------------------------- host side")
+
+
+def kernel_digest(source, markers=None):
+    """sha256 of a kernel source file, or of the text between two markers in it."""
+    import hashlib
+    with open(os.path.join(ROOT, source), "rb") as f:
+        data = f.read()
+    if markers:
+        a = data.index(markers[0].encode())
+        b = data.index(markers[1].encode(), a)
+        data = data[a:b]
+    return hashlib.sha256(data).hexdigest()
+
+
+def profiled_traffic(kernel_file, source, markers=None):
     """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) that
     an ncu capture recorded in profiles/<kernel_file>, provided the capture was
     taken of the kernel source as it is now (its sha256 prefix is written next
     to the figure); None otherwise."""
-    import hashlib
     import re
     try:
         with open(os.path.join(ROOT, "profiles", kernel_file)) as f:
             text = f.read()
-        with open(os.path.join(ROOT, source), "rb") as f:
-            digest = hashlib.sha256(f.read()).hexdigest()
-    except OSError:
+        digest = kernel_digest(source, markers)
+    except (OSError, ValueError):
         return None
     m = re.search(r"^traffic_bytes_per_launch: (\d+) .*sha256 ([0-9a-f]{16})", text, re.M)
     if not m or not digest.startswith(m.group(2)):
@@ -362,7 +378,9 @@ def prefill_summary(cfg, world, steps, ms, kern_ms, peaks):
                                 else f"{fused_kernel_name(cfg)} (fused chunk loop, output rows)"), "bound": "hbm",
                      "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"],
-                     "traffic": profiled_traffic(prefill_profile(cfg), PREFILL_SOURCE),
+                     "traffic": profiled_traffic(prefill_profile(cfg), PREFILL_SOURCE,
+                                                 ROWS_KERNEL_TEXT if fused_kernel_name(cfg) == "prefill_rows_kernel"
+                                                 else None),
                      "alg_bytes_per_launch": alg_bytes, "launch_ms": kern_ms, "peak_source": peaks["source"]},
     }
 
