@@ -70,6 +70,17 @@ bool chunk_supported(int chunk) {
 
 constexpr size_t kMaxSmem = 227 * 1024;
 
+// Chunk the tensor-core kernels run for a requested chunk.  The chunkwise form is
+// the same function for every chunk length (only the rounding differs), so
+// d_v = 256 runs 128-token chunks for uniform batches (the output-rows CTA
+// pair) and 64-token ones for packed batches, whichever of the two was asked.
+int run_chunk(int dk, int dv, int chunk, gret_dtype io, bool packed) {
+    if (io != GRET_BF16 || dk != 128 || dv != 256) return chunk;
+    if (!packed && chunk == 64) return 128;
+    if (packed && chunk == 128) return 64;
+    return chunk;
+}
+
 // Kernel choice for a prefill; segments/seg_len describe the sequence split.
 gret_path select_path(int B, int H, int N, int dk, int dv, int chunk, gret_dtype io, int num_sms,
                       int* segments, int* seg_len, int* pieces = nullptr) {
@@ -81,7 +92,7 @@ gret_path select_path(int B, int H, int N, int dk, int dv, int chunk, gret_dtype
     if (!shape_supported(dk, dv) || !chunk_supported(chunk)) return GRET_PATH_NONE;
     if (io == GRET_BF16 && prefill_tc_supported(dk, dv, chunk, io)) {
         int segs = 1, len = N, pcs = 1;
-        prefill_tc_plan(B, H, N, chunk, num_sms, &segs, &len, &pcs);
+        prefill_tc_plan(B, H, N, chunk, num_sms, &segs, &len, &pcs, prefill_tc_ctas_per_item(dv, chunk));
         if (segments) *segments = segs;
         if (seg_len) *seg_len = len;
         if (pieces) *pieces = pcs;
@@ -123,12 +134,14 @@ void gret_set_gate_profile_events(void* start, void* stop) {
 
 gret_path gret_prefill_path(int B, int H, int N, int dk, int dv, int chunk, gret_dtype io_dtype,
                             int* segments) {
+    chunk = run_chunk(dk, dv, chunk, io_dtype, false);
     int sms = 148;
     device_info(nullptr, &sms);
     return select_path(B, H, N, dk, dv, chunk, io_dtype, sms, segments, nullptr);
 }
 
 int gret_prefill_launches(int B, int H, int N, int dk, int dv, int chunk, gret_dtype io_dtype) {
+    chunk = run_chunk(dk, dv, chunk, io_dtype, false);
     int sms = 148, segs = 1, pcs = 1;
     device_info(nullptr, &sms);
     gret_path p = select_path(B, H, N, dk, dv, chunk, io_dtype, sms, &segs, nullptr, &pcs);
@@ -138,6 +151,7 @@ int gret_prefill_launches(int B, int H, int N, int dk, int dv, int chunk, gret_d
 
 size_t gret_prefill_workspace_size(int B, int H, int N, int dk, int dv, int chunk,
                                    gret_dtype io_dtype) {
+    chunk = run_chunk(dk, dv, chunk, io_dtype, false);
     int sms = 148, segs = 1, pcs = 1;
     device_info(nullptr, &sms);
     gret_path p = select_path(B, H, N, dk, dv, chunk, io_dtype, sms, &segs, nullptr, &pcs);
@@ -183,6 +197,7 @@ static gret_status prefill_impl(const void* Q, const void* K, const void* V, con
         if (a0 < a1 + bytes && a1 < a0 + bytes) return GRET_ERR_INVALID_ARG;
     }
 
+    chunk = run_chunk(dk, dv, chunk, io_dtype, cu_seqlens != nullptr);
     unsigned int* status = nullptr;
     int sms = 0;
     if (!device_info(&status, &sms)) return GRET_ERR_CUDA;
@@ -238,6 +253,7 @@ static gret_status prefill_impl(const void* Q, const void* K, const void* V, con
 size_t gret_prefill_projected_workspace_size(int B, int H, int N, int dk, int dv, int chunk, int d_model,
                                              gret_dtype io_dtype) {
     if (d_model <= 0) return 0;
+    chunk = run_chunk(dk, dv, chunk, io_dtype, false);
     int sms = 148, segs = 1, pcs = 1;
     device_info(nullptr, &sms);
     gret_path p = select_path(B, H, N, dk, dv, chunk, io_dtype, sms, &segs, nullptr, &pcs);
@@ -286,6 +302,7 @@ gret_status gret_prefill_resume(const void* Q, const void* K, const void* V, con
 size_t gret_prefill_varlen_workspace_size(int num_seqs, int total_tokens, int max_seqlen, int H, int dk, int dv,
                                           int chunk, gret_dtype io_dtype) {
     if (num_seqs <= 0 || total_tokens <= 0 || max_seqlen <= 0) return 0;
+    chunk = run_chunk(dk, dv, chunk, io_dtype, true);
     int sms = 148;
     device_info(nullptr, &sms);
     if (select_path(num_seqs, H, max_seqlen, dk, dv, chunk, io_dtype, sms, nullptr, nullptr) != GRET_PATH_TC) return 0;
@@ -295,6 +312,7 @@ size_t gret_prefill_varlen_workspace_size(int num_seqs, int total_tokens, int ma
 int gret_prefill_varlen_launches(int num_seqs, int total_tokens, int max_seqlen, int H, int dk, int dv, int chunk,
                                  gret_dtype io_dtype) {
     if (num_seqs <= 0 || total_tokens <= 0 || max_seqlen <= 0) return 0;
+    chunk = run_chunk(dk, dv, chunk, io_dtype, true);
     int sms = 148;
     device_info(nullptr, &sms);
     const gret_path p = select_path(num_seqs, H, max_seqlen, dk, dv, chunk, io_dtype, sms, nullptr, nullptr);
@@ -351,6 +369,7 @@ gret_status gret_last_device_status(gret_stream_t stream) {
 }
 
 size_t gret_prefill_state_workspace_size(int B, int H, int N, int dk, int dv, int chunk, gret_dtype io_dtype) {
+    chunk = run_chunk(dk, dv, chunk, io_dtype, false);
     int sms = 148;
     device_info(nullptr, &sms);
     if (select_path(B, H, N, dk, dv, chunk, io_dtype, sms, nullptr, nullptr) != GRET_PATH_TC) return 0;
@@ -368,6 +387,7 @@ gret_status gret_prefill_state(const void* K, const void* V, const float* gate_l
         (reinterpret_cast<uintptr_t>(decay) & 3u) != 0)
         return GRET_ERR_INVALID_ARG;
     if ((long long)B * H > (1LL << 30) || (long long)B * N > (1LL << 40)) return GRET_ERR_UNSUPPORTED;
+    chunk = run_chunk(dk, dv, chunk, io_dtype, false);
     unsigned int* status = nullptr;
     int sms = 0;
     if (!device_info(&status, &sms)) return GRET_ERR_CUDA;

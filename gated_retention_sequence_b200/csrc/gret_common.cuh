@@ -179,7 +179,10 @@ size_t gate_project_tc_ws_bytes(int H, int d_model);
 cudaError_t launch_gate_project_tc(const PrefillArgs& a, float* bcum, float* eblk, int Npad, void* wsplit,
                                    cudaStream_t s);
 cudaError_t launch_gate_project_simt(const PrefillArgs& a, float* z, cudaStream_t s);
-void prefill_tc_plan(int B, int H, int N, int chunk, int num_sms, int* segments, int* seg_len, int* pieces);
+// ctas_per_item: CTAs that run one fused work item (2 for the d_v = 256 pair).
+void prefill_tc_plan(int B, int H, int N, int chunk, int num_sms, int* segments, int* seg_len, int* pieces,
+                     int ctas_per_item = 1);
+int prefill_tc_ctas_per_item(int dv, int chunk);
 size_t prefill_tc_workspace_bytes(int B, int H, int N, int dk, int dv, int chunk, int segments, int pieces);
 size_t prefill_tc_varlen_workspace_bytes(int S, int H, int max_seqlen, int total, int dk, int dv, int chunk,
                                          int num_sms);

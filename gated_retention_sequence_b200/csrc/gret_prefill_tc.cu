@@ -904,10 +904,10 @@ struct StateCfg {
     static constexpr int BOX = C * 128;
     static constexpr int K_BYTES = 2 * BOX;
     static constexpr int V_BYTES = (DV / 64) * BOX;
-    // as many K + V stages as about 200 KB hold (3-6), to keep loads in flight
-    static constexpr int NS_FIT = (200 * 1024) / (K_BYTES + V_BYTES);
+    // as many K + V stages as about 210 KB hold (2-6), to keep loads in flight
+    static constexpr int NS_FIT = (210 * 1024) / (K_BYTES + V_BYTES);
     static constexpr int NS = NS_FIT > 6 ? 6 : NS_FIT;
-    static_assert(NS >= 3, "state pass stages");
+    static_assert(NS >= 2, "state pass stages");
     static constexpr int W = NH * 64;                       // state columns per thread
     static constexpr int TM_ALLOC = NH * 128 <= 128 ? 128 : 256;
     static constexpr int OFF_K = 0;
@@ -1447,9 +1447,10 @@ __global__ void state_fold_kernel(const float* __restrict__ dS_all, const float*
 // released by its intra-chunk product, its Q and K by the state update.
 constexpr int kRowsThreads = 896;
 constexpr int kRowsRegs = 72;          // 65536 / 896, rounded down to 8
-constexpr int kRowsSRegs = 64;         // the S warps hand registers to the issuing warps
+constexpr int kRowsSRegs = 56;         // the S warps hand registers to the P and issuing warps
+constexpr int kRowsPRegs = 80;
 constexpr int kRowsIssueRegs = 80;
-static_assert(128 * kRowsSRegs + 128 * kRowsIssueRegs <= 256 * kRowsRegs, "register split");
+static_assert(128 * kRowsSRegs + 128 * kRowsPRegs + 128 * kRowsIssueRegs <= 384 * kRowsRegs, "register split");
 
 struct RowsCfg {
     static constexpr int C = 128, DV = 128;
@@ -1461,12 +1462,15 @@ struct RowsCfg {
     static constexpr int OFF_G = OFF_V + TILE;      // G
     static constexpr int OFF_T = OFF_G + TILE;      // bf16 T^T [d][k]
     static constexpr int OFF_B = OFF_T + TILE;      // per Q/K stage: C fp32 decay sums
-    static constexpr int OFF_BAR = OFF_B + 2 * C * 4;
-    static constexpr int NUM_BARS = 16;
+    static constexpr int OFF_XIN = OFF_B + 2 * C * 4;   // CTA pair: the other CTA's per-token sums
+    static constexpr int OFF_BAR = OFF_XIN + C * 8;
+    static constexpr int NUM_BARS = 19;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int USED = OFF_MISC + 16;
-    static constexpr int SMEM = USED + 1024;        // room to align the base to 1024 bytes
-    static_assert(SMEM <= kMaxSmem, "shared memory budget");
+    // the rest of the budget is slack for aligning the base to 1024 bytes (the
+    // kernel checks that it sufficed)
+    static constexpr int SMEM = kMaxSmem;
+    static_assert(USED <= SMEM, "shared memory budget");
     // tensor-memory columns: O, scores, P, T^T, and the epilogue's exchange
     // (two sets of four (sum, sum of squares) pairs)
     static constexpr int TM_O = 0, TM_SC = 128, TM_P = 256, TM_T = 320, TM_X = 448, TM_ALLOC = 512;
@@ -1484,14 +1488,25 @@ __device__ __forceinline__ void scale_tile_row(uint8_t* tile, int row, float f) 
             scale_bf16x8(tile + x * RowsCfg::BOX + row * 128 + ((c ^ (row & 7)) << 4), f);
 }
 
+template <bool PAIR>
 __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __grid_constant__ TcParams p) {
     using CF = RowsCfg;
-    constexpr int C = CF::C, DV = CF::DV;
+    constexpr int C = CF::C, DV = CF::DV;      // DV: the output channels (and state rows) of this CTA
+    constexpr int DVT = PAIR ? 2 * DV : DV;    // the unit's d_v
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int u = blockIdx.x / p.P, seg = blockIdx.x % p.P;
+    if (sm + CF::USED > smem_raw + CF::SMEM) {   // the base is not aligned enough: report, do nothing
+        if (tid == 0) atomicExch(p.status, kDevSmemLayout);
+        return;
+    }
+    // a CTA pair (cluster of two, consecutive blocks) shares one work item: rank r
+    // owns output channels and state rows r * DV .. r * DV + DV - 1
+    const int rank = PAIR ? (int)cluster_ctarank() : 0;
+    const int ch0 = rank * DV;
+    const int item = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+    const int u = item / p.P, seg = item % p.P;
     const int hh = u % p.H, bb = u / p.H;
     const int n_begin = seg * p.seg_len;
     const int n_end = min(p.N, n_begin + p.seg_len);
@@ -1501,9 +1516,11 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
     // before the MMA warp has seen the first.  BG: the G tile of a chunk is in
     // (or, without G, the tile is free for the chunk's output); BGF: the
     // epilogue has written the chunk's output into the tile.
-    constexpr int BQK = 0, BV = 2, BG = 3, BSC = 4, BOD = 5, BST = 6, BKT = 7, BTC = 9, BQT = 10, BPR = 11,
-                  BOF = 12, BGF = 13, BDRAIN = 14, BNEVER = 15;
-    static_assert(BNEVER + 1 == CF::NUM_BARS, "barrier count");
+    // BXF / BXE (CTA pair): the other CTA's per-token sums are in this CTA's
+    // exchange buffer / it has read the sums this CTA sent
+    constexpr int BQK = 0, BV = 2, BG = 3, BSC = 4, BOD = 6, BST = 7, BKT = 8, BTC = 10, BQT = 11, BPR = 12,
+                  BOF = 13, BGF = 14, BDRAIN = 15, BNEVER = 16, BXF = 17, BXE = 18;
+    static_assert(BXE + 1 == CF::NUM_BARS, "barrier count");
     auto bar = [&](int i) -> uint32_t { return sb + CF::OFF_BAR + 8 * i; };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + CF::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + CF::OFF_MISC + 4);
@@ -1512,10 +1529,10 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
         for (int i = 0; i < CF::NUM_BARS; ++i) {
             // per-warp arrivals: sixteen epilogue warps, six P warps, or one
             // four-warp role
-            const bool sixteen = i == BOF || i == BGF;
+            const bool sixteen = i == BOF || i == BGF || i == BKT || i == BKT + 1;
             const bool four = i == BTC || i == BQT;
-            const bool kt = i == BKT || i == BKT + 1;   // every chunk: the E and the S warps
-            mbar_init(bar(i), sixteen ? 16 : four ? 4 : kt ? 20 : i == BPR ? 6 : 1);
+            const bool xchg_full = i == BXF;            // one writer warp per lane quarter
+            mbar_init(bar(i), sixteen || i == BXE ? 16 : four || xchg_full ? 4 : i == BPR ? 6 : 1);
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -1532,6 +1549,8 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // the other CTA's barriers are initialised before either sends to them
+    if constexpr (PAIR) cluster_sync_all();
     const uint32_t tm = *tmem_slot;
     grid_dep_launch();
     grid_dep_wait();
@@ -1553,7 +1572,8 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
         float lam = 0.f;
         for (int i = 0; i < nchunks; ++i) {
             const float* bc = stage_bc(i);
-            mbar_wait(bar(BSC), i & 1, p.status, abort_flag);   // the scores landed (so did Q/K and bc)
+            // the scores landed (so did Q/K and bc)
+            mbar_wait(bar(BSC + (i & 1)), (i >> 1) & 1, p.status, abort_flag);
             tc_fence_after();
             const float bC = bc[C - 1];
             const bool eager = (-bC - lam) > kLazyMax;
@@ -1562,6 +1582,9 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
             for (int cb = cb_lo; cb <= cb_hi; ++cb) {
                 uint32_t r[32], pk[16];
                 tmem_ld_x32(tm + lq + CF::TM_SC + cb * 32, r);
+                // a lazy chunk's column factors e^{-b_s - Lambda} (<= e^kLazyMax), one
+                // per lane, shared by shuffles; the scores are Q K^T of the raw K
+                const float cf = __expf(-bc[cb * 32 + lane] - lam);
                 tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
@@ -1570,6 +1593,9 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
                     if (eager) {
                         v0 *= __expf(fminf(bt - bc[s0], 0.f));
                         v1 *= __expf(fminf(bt - bc[s0 + 1], 0.f));
+                    } else {
+                        v0 *= __shfl_sync(0xffffffffu, cf, 2 * j);
+                        v1 *= __shfl_sync(0xffffffffu, cf, 2 * j + 1);
                     }
                     pk[j] = pack_bf16x2(s0 <= row ? v0 : 0.f, s0 + 1 <= row ? v1 : 0.f);
                 }
@@ -1602,7 +1628,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
                 last_v = j;
                 mbar_arrive_expect_tx(bar(BV), CF::TILE);
                 for (int x = 0; x < 2; ++x)
-                    tma_load_4d(sb + CF::OFF_V + x * CF::BOX, &p.tmV, x * 64, hh, n_begin + j * C, bb, bar(BV));
+                    tma_load_4d(sb + CF::OFF_V + x * CF::BOX, &p.tmV, ch0 + x * 64, hh, n_begin + j * C, bb, bar(BV));
             };
             // the tile of chunk j: its G, or (without G) a plain release for its output
             auto issue_g = [&](int j) {
@@ -1613,7 +1639,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
                 last_g = j;
                 mbar_arrive_expect_tx(bar(BG), CF::TILE);
                 for (int x = 0; x < 2; ++x)
-                    tma_load_4d(sb + CF::OFF_G + x * CF::BOX, &p.tmG, x * 64, hh, n_begin + j * C, bb, bar(BG));
+                    tma_load_4d(sb + CF::OFF_G + x * CF::BOX, &p.tmG, ch0 + x * 64, hh, n_begin + j * C, bb, bar(BG));
             };
             if (p.fault) mbar_wait_injected_timeout(bar(BNEVER), p.status, abort_flag);
             if (!*abort_flag) {
@@ -1622,18 +1648,16 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
                 issue_v(0);
                 issue_g(0);
                 for (int i = 0; i < nchunks; ++i) {
-                    // the state MMA of chunk i is the last reader of its Q/K stage,
-                    // the intra-chunk MMA the last reader of V
+                    // the state MMA of chunk i is the last reader of its Q/K stage and of V
                     if (!mbar_wait(bar(BST), i & 1, p.status, abort_flag)) break;
                     if (i + 2 < nchunks) issue_qk(i + 2);
-                    if (!mbar_wait(bar(BOD), i & 1, p.status, abort_flag)) break;
                     if (i + 1 < nchunks) issue_v(i + 1);
                     // the output of chunk i leaves from the tile (rows past the end of
                     // the sequence fall outside the map and are not written); once the
                     // store has read the tile it takes chunk i + 1
                     if (!mbar_wait(bar(BGF), i & 1, p.status, abort_flag)) break;
                     for (int x = 0; x < 2; ++x)
-                        tma_store_4d(&p.tmO, sb + CF::OFF_G + x * CF::BOX, x * 64, hh, n_begin + i * C, bb);
+                        tma_store_4d(&p.tmO, sb + CF::OFF_G + x * CF::BOX, ch0 + x * 64, hh, n_begin + i * C, bb);
                     bulk_commit();
                     bulk_wait_read<0>();
                     if (i + 1 < nchunks) issue_g(i + 1);
@@ -1660,10 +1684,8 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
                 if (!mbar_wait(bar(BQK + s), (i >> 1) & 1, p.status, abort_flag)) break;
                 const float bC = stage_bc(i)[C - 1];
                 const bool eager = (-bC - lam) > kLazyMax;
-                // scores: lazy ones take K~ (scaled before), eager ones the raw K; the
-                // score buffer is free once P of the previous chunk is out
-                if (!eager && !mbar_wait(bar(BKT + s), (i >> 1) & 1, p.status, abort_flag)) break;
-                if (i > 0 && !mbar_wait(bar(BPR), (i - 1) & 1, p.status, abort_flag)) break;
+                // scores of the raw Q and K, once P of the previous chunk has left the
+                // score buffer (the intra-chunk product waited for it)
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < DK / 16; ++k) {
@@ -1671,7 +1693,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
                     mma_ss(tm + CF::TM_SC, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(sK + off, 16, 1024), id_kk,
                            k > 0);
                 }
-                mma_commit(bar(BSC));
+                mma_commit(bar(BSC + s));
                 // inter-chunk: O = Q T (lazy) or Q~ T (eager), once the bf16 copy of T
                 // is ready and the epilogue has taken the previous output
                 if (!mbar_wait(bar(BTC), i & 1, p.status, abort_flag)) break;
@@ -1685,23 +1707,23 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
                     mma_ss(tm + CF::TM_O, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(sT + off, 16, 1024), id_kk,
                            k > 0);
                 }
-                // state: T^T += V^T K~ (eager: K~ is scaled after the scores); it
-                // needs neither P nor the output, so it runs while P is converted
+                // intra-chunk: O += P V
+                if (!mbar_wait(bar(BPR), i & 1, p.status, abort_flag)) break;
                 if (!mbar_wait(bar(BV), i & 1, p.status, abort_flag)) break;
-                if (eager && !mbar_wait(bar(BKT + s), (i >> 1) & 1, p.status, abort_flag)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < C / 16; ++k)
+                    mma_ts(tm + CF::TM_O, tm + CF::TM_P + k * 8, sdesc_sw128(sV + k * 2048, CF::BOX, 1024), id_pv, 1);
+                mma_commit(bar(BOD));
+                // state: T^T += V^T K~, once the epilogue warps have scaled K~ in place
+                // (after the scores read the raw K)
+                if (!mbar_wait(bar(BKT + s), (i >> 1) & 1, p.status, abort_flag)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < C / 16; ++k)
                     mma_ss(tm + CF::TM_T, sdesc_sw128(sV + k * 2048, CF::BOX, 1024),
                            sdesc_sw128(sK + k * 2048, CF::BOX, 1024), id_kv, 1);
                 mma_commit(bar(BST));
-                // intra-chunk: O += P V
-                if (!mbar_wait(bar(BPR), i & 1, p.status, abort_flag)) break;
-                tc_fence_after();
-#pragma unroll
-                for (int k = 0; k < C / 16; ++k)
-                    mma_ts(tm + CF::TM_O, tm + CF::TM_P + k * 8, sdesc_sw128(sV + k * 2048, CF::BOX, 1024), id_pv, 1);
-                mma_commit(bar(BOD));
                 lam = eager ? 0.f : lam + bC;
             }
             // every MMA this thread issued has completed before tensor memory is freed
@@ -1721,17 +1743,17 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
             for (int cb = 0; cb < 4; ++cb) {
                 if (seg > 0) {
                     const float4* s4 = reinterpret_cast<const float4*>(
-                        p.seg_state + ((size_t)u * p.slots + (size_t)seg * p.K - 1) * DV * DK + (size_t)row * DK +
-                        cb * 32);
+                        p.seg_state + ((size_t)u * p.slots + (size_t)seg * p.K - 1) * DVT * DK +
+                        (size_t)(ch0 + row) * DK + cb * 32);
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         const float4 v = s4[j];
                         r[4 * j] = f2u(v.x); r[4 * j + 1] = f2u(v.y); r[4 * j + 2] = f2u(v.z); r[4 * j + 3] = f2u(v.w);
                     }
                 } else if (p.S0) {
-                    const float* src = p.S0 + (size_t)u * DK * DV + (size_t)(cb * 32) * DV + row;
+                    const float* src = p.S0 + (size_t)u * DK * DVT + (size_t)(cb * 32) * DVT + ch0 + row;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) r[j] = f2u(src[(size_t)j * DV]);
+                    for (int j = 0; j < 32; ++j) r[j] = f2u(src[(size_t)j * DVT]);
                 } else {
 #pragma unroll
                     for (int j = 0; j < 32; ++j) r[j] = 0u;
@@ -1745,14 +1767,10 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
             const int s = i & 1;
             const float* bc = stage_bc(i);
             uint8_t* Qp = sm + CF::OFF_Q + s * CF::TILE;
-            uint8_t* Kp = sm + CF::OFF_K + s * CF::TILE;
             mbar_wait(bar(BQK + s), (i >> 1) & 1, p.status, abort_flag);
             const float bC = bc[C - 1];
             const bool eager = (-bC - lam) > kLazyMax;
             const float brow = bc[row];
-            // a lazy chunk's K~ is the E warps' (before its scores); an eager
-            // chunk's is scaled here after its scores
-            if (!eager) warp_arrive(BKT + s);
             // bf16 copy of T^T for this chunk's inter-chunk product, once the
             // previous state update is done (it also finished the previous
             // inter-chunk product, the last reader of the copy); eager chunks
@@ -1787,14 +1805,12 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
             tc_fence_before();
             warp_arrive(BTC);
             if (eager) {
-                // Q~ and K~ in place, once the scores have read Q and K
-                mbar_wait(bar(BSC), i & 1, p.status, abort_flag);
+                // Q~ in place, once the scores have read Q (K~ is the E warps')
+                mbar_wait(bar(BSC + s), (i >> 1) & 1, p.status, abort_flag);
                 tc_fence_after();
                 scale_tile_row(Qp, row, __expf(brow + lam));
-                scale_tile_row(Kp, row, __expf(bC - brow));
                 fence_proxy_async_smem();
                 warp_arrive(BQT);
-                warp_arrive(BKT + s);
             }
             lam = eager ? 0.f : lam + bC;
         }
@@ -1805,18 +1821,19 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
         }
         if (p.S_final && seg == p.P - 1) {
             const float sc = __expf(lam);
-            float* dst = p.S_final + (size_t)u * DK * DV;
+            float* dst = p.S_final + (size_t)u * DK * DVT + ch0;
 #pragma unroll 1
             for (int cb = 0; cb < 4; ++cb) {
                 uint32_t r[32];
                 tmem_ld_x32(tm + lq + CF::TM_T + cb * 32, r);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) dst[(size_t)(cb * 32 + j) * DV + row] = u2f(r[j]) * sc;
+                for (int j = 0; j < 32; ++j) dst[(size_t)(cb * 32 + j) * DVT + row] = u2f(r[j]) * sc;
             }
         }
     } else if (role == 4) {
         // ============================================================ P warps
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" : : "n"(kRowsPRegs));
         // the blocks above the diagonal, once
         {
             uint32_t z[16];
@@ -1832,29 +1849,27 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
         constexpr int QC = DV / 4;
         float lam = 0.f;
         const float* bsum = p.bcum + (size_t)u * p.Npad;
-        // K~_s = e^{-b_s - Lambda} K_s of a lazy chunk j, in place: token row
-        // tid % 128, its 16-byte words 4 (tid / 128) .. + 3; an eager chunk's K
-        // stays raw for its scores (the S warps scale it after them).  Chunks
+        // K~ of chunk j in place for its state update, once its scores have read
+        // the raw K: e^{-b_s - Lambda} K_s (lazy) or e^{b_C - b_s} K_s (eager);
+        // token row tid % 128, its 16-byte words 4 (tid / 128) .. + 3.  Chunks
         // are taken in order, so Lambda follows them.
         float lam_k = 0.f;
         auto scale_k = [&](int j) {
             const int s = j & 1, kr = tid & (C - 1), part = tid >> 7;
             const float* bc = stage_bc(j);
-            mbar_wait(bar(BQK + s), (j >> 1) & 1, p.status, abort_flag);
+            mbar_wait(bar(BSC + s), (j >> 1) & 1, p.status, abort_flag);
             const float bCj = bc[C - 1];
             const bool eg = (-bCj - lam_k) > kLazyMax;
-            if (!eg) {
-                const float f = __expf(-bc[kr] - lam_k);
-                uint8_t* krow = sm + CF::OFF_K + s * CF::TILE + (part >> 1) * CF::BOX + kr * 128;
+            const float f = __expf(eg ? bCj - bc[kr] : -bc[kr] - lam_k);
+            uint8_t* krow = sm + CF::OFF_K + s * CF::TILE + (part >> 1) * CF::BOX + kr * 128;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) scale_bf16x8(krow + ((((part & 1) * 4 + c) ^ (kr & 7)) << 4), f);
-                fence_proxy_async_smem();
-            }
+            for (int c = 0; c < 4; ++c) scale_bf16x8(krow + ((((part & 1) * 4 + c) ^ (kr & 7)) << 4), f);
+            fence_proxy_async_smem();
             warp_arrive(BKT + s);
             lam_k = eg ? 0.f : lam_k + bCj;
         };
-        for (int j = 0; j < 2 && j < nchunks; ++j) scale_k(j);
         for (int i = 0; i < nchunks; ++i) {
+            scale_k(i);
             const int n0 = n_begin + i * C;
             const float bt = bsum[n0 + row], bC = bsum[n0 + C - 1];
             mbar_wait(bar(BOD), i & 1, p.status, abort_flag);
@@ -1892,11 +1907,30 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
                 uint32_t all[8];
                 tmem_ld_x8(xs, all);
                 tmem_wait_ld();
-                const float t1 = (u2f(all[0]) + u2f(all[2])) + (u2f(all[4]) + u2f(all[6]));
-                const float t2 = (u2f(all[1]) + u2f(all[3])) + (u2f(all[5]) + u2f(all[7]));
-                const float mean_u = t1 * (1.0f / DV);
+                float t1 = (u2f(all[0]) + u2f(all[2])) + (u2f(all[4]) + u2f(all[6]));
+                float t2 = (u2f(all[1]) + u2f(all[3])) + (u2f(all[5]) + u2f(all[7]));
+                if constexpr (PAIR) {
+                    // the token's other 128 channels are the other CTA's: the first
+                    // warp of each lane quarter sends this CTA's sums into the other's
+                    // exchange buffer (once it has read the previous chunk's), every
+                    // warp then reads the other's sums from its own buffer and says so
+                    const uint32_t other = (uint32_t)(rank ^ 1);
+                    if (hf == 0) {
+                        if (i > 0) mbar_wait_cluster(bar(BXE), (i - 1) & 1, p.status, abort_flag);
+                        st_cluster_f2(cluster_map(sb + CF::OFF_XIN + row * 8, other), t1, t2);
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive_remote(cluster_map(bar(BXF), other));
+                    }
+                    mbar_wait_cluster(bar(BXF), i & 1, p.status, abort_flag);
+                    const float2 o = *reinterpret_cast<const float2*>(sm + CF::OFF_XIN + row * 8);
+                    t1 += o.x;
+                    t2 += o.y;
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_remote(cluster_map(bar(BXE), other));
+                }
+                const float mean_u = t1 * (1.0f / DVT);
                 const float mean_y = mean_u * c;
-                const float var = fmaxf(t2 * (1.0f / DV) - mean_y * mean_y, 0.f);
+                const float var = fmaxf(t2 * (1.0f / DVT) - mean_y * mean_y, 0.f);
                 a = c * rsqrtf(var + p.eps);
                 b0 = -mean_u * a;
             }
@@ -1923,7 +1957,6 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
             fence_proxy_async_smem();
             warp_arrive(BGF);              // the tile holds this chunk's output
             lam = eager ? 0.f : lam + bC;
-            if (i + 2 < nchunks) scale_k(i + 2);
         }
     }
     tc_fence_before();
@@ -1931,6 +1964,11 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tm, CF::TM_ALLOC);
+    }
+    // neither CTA of a pair leaves while the other may still send to it
+    if constexpr (PAIR) {
+        __syncwarp();
+        cluster_sync_all();
     }
 }
 
@@ -2043,21 +2081,58 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+#ifndef GRET_ROWS_KERNEL
+#define GRET_ROWS_KERNEL 1
+#endif
+
+// Launch with programmatic stream serialisation and clusters of two CTAs.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl_pair(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                            Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// Chunk loop over a uniform batch, or a packed batch's plan.  128-token chunks
+// of d_v 128 or 256 (bf16) run the output-rows kernel (a CTA pair for 256),
+// the others prefill_tc_kernel.
 template <int DV, int C, bool PACKED>
 cudaError_t run_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t s, const PlanArgs* plan = nullptr) {
-    using CF = Cfg<DV, C>;
-    auto kf = prefill_tc_kernel<DV, C, PACKED>;
+    constexpr bool ROWS = !PACKED && C == 128 && (DV == 128 || DV == 256) && GRET_ROWS_KERNEL;
     auto ks = prefill_state_kernel<DV, C, PACKED>;
     static bool attr_done[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || !attr_done[dev]) {
-        // the register split inside the fused kernel draws on the registers it
-        // was launched with: never launch a build that has fewer
-        cudaFuncAttributes fa;
-        if (cudaFuncGetAttributes(&fa, kf) != cudaSuccess) return cudaErrorInvalidDeviceFunction;
-        if (fa.numRegs * kFusedThreads < 4 * 128 * kComputeRegs + 128 * kIssueRegs) return cudaErrorInvalidConfiguration;
-        cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, CF::SMEM);
+        if constexpr (!ROWS) {
+            // the register split inside the fused kernel draws on the registers it
+            // was launched with: never launch a build that has fewer
+            auto kf = prefill_tc_kernel<DV, C, PACKED>;
+            cudaFuncAttributes fa;
+            if (cudaFuncGetAttributes(&fa, kf) != cudaSuccess) return cudaErrorInvalidDeviceFunction;
+            if (fa.numRegs * kFusedThreads < 4 * 128 * kComputeRegs + 128 * kIssueRegs)
+                return cudaErrorInvalidConfiguration;
+            cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<DV, C>::SMEM);
+        } else {
+            auto kr = prefill_rows_kernel<DV == 256>;
+            cudaFuncAttributes fa;
+            if (cudaFuncGetAttributes(&fa, kr) != cudaSuccess) return cudaErrorInvalidDeviceFunction;
+            if (fa.numRegs > kRowsRegs) return cudaErrorInvalidConfiguration;
+            cudaFuncSetAttribute(kr, cudaFuncAttributeMaxDynamicSharedMemorySize, RowsCfg::SMEM);
+        }
         cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, StateCfg<DV, C>::SMEM);
         if (dev >= 0 && dev < 64) attr_done[dev] = true;
     }
@@ -2065,6 +2140,8 @@ cudaError_t run_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t s, const Pla
     const int npad = tp.Npad;
     cudaError_t e = cudaSuccess;
     if constexpr (PACKED) {
+        auto kf = prefill_tc_kernel<DV, C, PACKED>;
+        using CF = Cfg<DV, C>;
         // gate scan, plan, state pass and combine over the plan's slots, fused loop
         int nyb = 0;
         const dim3 sgrid = gate_scan_grid(units, npad, C, &nyb);
@@ -2118,39 +2195,37 @@ cudaError_t run_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t s, const Pla
                        static_cast<const int4*>(nullptr));
         if (e != cudaSuccess) return e;
     }
-#ifndef GRET_ROWS_KERNEL
-#define GRET_ROWS_KERNEL 1
-#endif
-    if constexpr (DV == 128 && C == 128 && !PACKED && GRET_ROWS_KERNEL) {
-        // 128-token chunks with d_v 128: the output-rows kernel
-        auto kr = prefill_rows_kernel;
-        static bool rows_attr_done[64] = {};
-        if (dev < 0 || dev >= 64 || !rows_attr_done[dev]) {
-            cudaFuncAttributes fa;
-            if (cudaFuncGetAttributes(&fa, kr) != cudaSuccess) return cudaErrorInvalidDeviceFunction;
-            if (fa.numRegs > kRowsRegs) return cudaErrorInvalidConfiguration;
-            cudaFuncSetAttribute(kr, cudaFuncAttributeMaxDynamicSharedMemorySize, RowsCfg::SMEM);
-            if (dev >= 0 && dev < 64) rows_attr_done[dev] = true;
-        }
+    if constexpr (ROWS) {
+        // 128-token chunks: the output-rows kernel (d_v 256: a pair of CTAs per
+        // work item, each owning half of the channels)
+        auto kr = prefill_rows_kernel<DV == 256>;
         if (g_profile_start) cudaEventRecord(g_profile_start, s);
-        e = launch_pdl(kr, dim3(units * tp.P), dim3(kRowsThreads), RowsCfg::SMEM, s, tp);
+        if constexpr (DV == 256)
+            e = launch_pdl_pair(kr, dim3(2 * units * tp.P), dim3(kRowsThreads), RowsCfg::SMEM, s, tp);
+        else
+            e = launch_pdl(kr, dim3(units * tp.P), dim3(kRowsThreads), RowsCfg::SMEM, s, tp);
+        if (g_profile_stop) cudaEventRecord(g_profile_stop, s);
+        if (e != cudaSuccess) return e;
+        return cudaGetLastError();
+    } else {
+        auto kf = prefill_tc_kernel<DV, C, PACKED>;
+        if (g_profile_start) cudaEventRecord(g_profile_start, s);
+        e = launch_pdl(kf, dim3(units * tp.P), dim3(kFusedThreads), Cfg<DV, C>::SMEM, s, tp);
         if (g_profile_stop) cudaEventRecord(g_profile_stop, s);
         if (e != cudaSuccess) return e;
         return cudaGetLastError();
     }
-    if (g_profile_start) cudaEventRecord(g_profile_start, s);
-    e = launch_pdl(kf, dim3(units * tp.P), dim3(kFusedThreads), CF::SMEM, s, tp);
-    if (g_profile_stop) cudaEventRecord(g_profile_stop, s);
-    if (e != cudaSuccess) return e;
-    return cudaGetLastError();
 }
 
 }  // namespace
 
 bool prefill_tc_supported(int dk, int dv, int chunk, gret_dtype io) {
     if (io != GRET_BF16 || dk != DK) return false;
-    return (dv == 128 && (chunk == 64 || chunk == 128)) || (dv == 256 && chunk == 64);
+    return (dv == 128 && (chunk == 64 || chunk == 128)) || (dv == 256 && (chunk == 64 || chunk == 128));
 }
+
+// CTAs of one fused work item: the output-rows kernel for d_v = 256 is a pair.
+int prefill_tc_ctas_per_item(int dv, int chunk) { return dv == 256 && chunk == 128 ? 2 : 1; }
 
 // State-pass pieces of a split that leaves SMs idle with one piece per segment
 // but would need a second wave with two equal ones (units * (P - 1) segments,
@@ -2180,10 +2255,11 @@ int prefill_tc_piece_split(int B, int H, int chunk, int num_sms, int segments, i
 // that the state pass, too, has about one CTA per SM; where one piece per
 // segment would leave SMs idle and two equal ones need a second wave, a long and
 // a short piece (uneven_piece_split).
-void prefill_tc_plan(int B, int H, int N, int chunk, int num_sms, int* segments, int* seg_len, int* pieces) {
+void prefill_tc_plan(int B, int H, int N, int chunk, int num_sms, int* segments, int* seg_len, int* pieces,
+                     int ctas_per_item) {
     const int units = B * H > 0 ? B * H : 1;
     const int nchunks = (N + chunk - 1) / chunk;
-    int P = num_sms / units;
+    int P = num_sms / (units * (ctas_per_item > 1 ? ctas_per_item : 1));
     if (P < 1) P = 1;
     if (P > nchunks) P = nchunks;
     const int per = (nchunks + P - 1) / P;
@@ -2223,7 +2299,7 @@ int prefill_tc_state_pieces(int B, int H, int chunk, int num_sms, int segments, 
 
 size_t prefill_tc_state_workspace_bytes(int B, int H, int N, int dk, int dv, int chunk, int num_sms) {
     int P = 1, seg_len = N, K = 1;
-    prefill_tc_plan(B, H, N, chunk, num_sms, &P, &seg_len, &K);
+    prefill_tc_plan(B, H, N, chunk, num_sms, &P, &seg_len, &K, prefill_tc_ctas_per_item(dv, chunk));
     const int Ks = prefill_tc_state_pieces(B, H, chunk, num_sms, P, seg_len);
     return ws_layout(B, H, N, dk, dv, chunk, P + 1, Ks).total;
 }
@@ -2310,6 +2386,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
     const bool packed = a.cu_seqlens != nullptr;
     if (a.dv == 256 && C == 64)
         return packed ? run_tc<256, 64, true>(a, tp, s, &plan) : run_tc<256, 64, false>(a, tp, s);
+    if (a.dv == 256 && C == 128 && !packed) return run_tc<256, 128, false>(a, tp, s);
     if (a.dv == 128 && C == 128)
         return packed ? run_tc<128, 128, true>(a, tp, s, &plan) : run_tc<128, 128, false>(a, tp, s);
     if (a.dv == 128 && C == 64)
@@ -2350,7 +2427,7 @@ cudaError_t launch_prefill_state_tc(const PrefillArgs& a, int num_sms, cudaStrea
         return cudaErrorInvalidValue;
     const int nchunks = (a.N + C - 1) / C;
     int P = 1, seg_len = a.N, Kp = 1;
-    prefill_tc_plan(a.B, a.H, a.N, C, num_sms, &P, &seg_len, &Kp);
+    prefill_tc_plan(a.B, a.H, a.N, C, num_sms, &P, &seg_len, &Kp, prefill_tc_ctas_per_item(a.dv, C));
     const int K = prefill_tc_state_pieces(a.B, a.H, C, num_sms, P, seg_len);
     const WsLayout w = ws_layout(a.B, a.H, a.N, a.dk, a.dv, C, P + 1, K);
     uint8_t* ws = static_cast<uint8_t*>(a.workspace);
@@ -2368,6 +2445,7 @@ cudaError_t launch_prefill_state_tc(const PrefillArgs& a, int num_sms, cudaStrea
     tp.piece_len = seg_len / K;
     tp.slots = P * K;              // every piece of every segment
     if (a.dv == 256 && C == 64) return run_state_tc<256, 64>(a, tp, s);
+    if (a.dv == 256 && C == 128) return run_state_tc<256, 128>(a, tp, s);
     if (a.dv == 128 && C == 128) return run_state_tc<128, 128>(a, tp, s);
     if (a.dv == 128 && C == 64) return run_state_tc<128, 64>(a, tp, s);
     return cudaErrorNotSupported;

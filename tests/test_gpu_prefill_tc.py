@@ -50,9 +50,23 @@ def test_dv256_chunk64(N):
     _check_full(_cfg(1, 2, N, 256, 64, 200 + N))
 
 
-@pytest.mark.parametrize("N", [128, 300, 1100])
+@pytest.mark.parametrize("N", [1, 2, 128, 300, 1100])
 def test_dv128_chunk128(N):
     _check_full(_cfg(1, 2, N, 128, 128, 300 + N, z_dist=((4.0, 1.0),)))
+
+
+@pytest.mark.parametrize("N", [1, 130, 700])
+def test_dv256_chunk128(N):
+    """d_v 256 in 128-token chunks: the output-rows kernel as a CTA pair, each
+    CTA owning half of the channels and of the state."""
+    _check_full(_cfg(1, 2, N, 256, 128, 600 + N))
+
+
+def test_dv256_pair_segment_carry():
+    """Four units cut into 16 segments each: the pair kernel resumes every
+    segment from the state pass's carried state (its own half of each)."""
+    segs = _check_full(_cfg(1, 4, 6000, 256, 64, 611, z_dist=((3.0, 1.5), (-4.0, 1.0), (8.0, 0.5), (0.0, 2.0))))
+    assert segs > 1
 
 
 @pytest.mark.parametrize("N", [64, 500])
