@@ -1531,9 +1531,10 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
             // four-warp role
             const bool sixteen = i == BOF || i == BGF || i == BKT || i == BKT + 1;
             const bool four = i == BTC || i == BQT;
-            const bool xchg_full = i == BXF;            // one writer warp per lane quarter
-            mbar_init(bar(i), sixteen || i == BXE ? 16 : four || xchg_full ? 4 : i == BPR ? 6 : 1);
+            mbar_init(bar(i), sixteen || i == BXE ? 16 : four ? 4 : i == BPR ? 6 : 1);
         }
+        // the pair's exchange: armed for the first chunk's 128 pairs of sums
+        if (PAIR && p.gn && nchunks > 0) mbar_arrive_expect_tx(bar(BXF), C * 8);
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&p.tmQ);
@@ -1912,21 +1913,24 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
                 if constexpr (PAIR) {
                     // the token's other 128 channels are the other CTA's: the first
                     // warp of each lane quarter sends this CTA's sums into the other's
-                    // exchange buffer (once it has read the previous chunk's), every
-                    // warp then reads the other's sums from its own buffer and says so
+                    // exchange buffer (once it has read the previous chunk's) with
+                    // asynchronous stores that complete the transaction count of the
+                    // other's BXF; every warp then reads the other's sums from its own
+                    // buffer and says so.  Thread 0 arms BXF for the next chunk (1 KB)
+                    // once it has seen this chunk's phase complete.
                     const uint32_t other = (uint32_t)(rank ^ 1);
                     if (hf == 0) {
                         if (i > 0) mbar_wait_cluster(bar(BXE), (i - 1) & 1, p.status, abort_flag);
-                        st_cluster_f2(cluster_map(sb + CF::OFF_XIN + row * 8, other), t1, t2);
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive_remote(cluster_map(bar(BXF), other));
+                        st_async_f2(cluster_map(sb + CF::OFF_XIN + row * 8, other), cluster_map(bar(BXF), other),
+                                    t1, t2);
                     }
                     mbar_wait_cluster(bar(BXF), i & 1, p.status, abort_flag);
+                    if (tid == 0 && i + 1 < nchunks) mbar_arrive_expect_tx(bar(BXF), C * 8);
                     const float2 o = *reinterpret_cast<const float2*>(sm + CF::OFF_XIN + row * 8);
                     t1 += o.x;
                     t2 += o.y;
                     __syncwarp();
-                    if (lane == 0) mbar_arrive_remote(cluster_map(bar(BXE), other));
+                    if (lane == 0) mbar_arrive_remote_relaxed(cluster_map(bar(BXE), other));
                 }
                 const float mean_u = t1 * (1.0f / DVT);
                 const float mean_y = mean_u * c;

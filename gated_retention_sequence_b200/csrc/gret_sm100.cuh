@@ -126,6 +126,21 @@ __device__ __forceinline__ void st_cluster_f2(uint32_t remote, float x, float y)
     asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(remote), "f"(x), "f"(y) : "memory");
 }
 
+// Asynchronous store of two floats into another CTA's shared memory that
+// completes 8 bytes of the transaction count of an mbarrier there (no fence:
+// the receiver sees the data once it sees the barrier's phase complete).
+__device__ __forceinline__ void st_async_f2(uint32_t remote, uint32_t remote_bar, float x, float y) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(remote),
+                 "f"(x), "f"(y), "r"(remote_bar)
+                 : "memory");
+}
+
+// Arrive on an mbarrier in another CTA of the cluster without ordering any
+// memory access (a signal whose data dependences are already resolved).
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t remote_bar) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
+}
+
 // Arrive on an mbarrier in another CTA of the cluster, releasing this thread's
 // prior writes (and, through a preceding __syncwarp, its warp's) at cluster scope.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t remote_bar) {
