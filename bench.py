@@ -57,10 +57,11 @@ PREFILL_CONFIGS = ("c3", "c2", "c5")
 
 
 def fused_kernel_name(cfg):
-    """The fused chunk-loop kernel that runs this workload: 128-token chunks with
-    d_v = 128 (bf16) take the output-rows kernel, the others prefill_tc_kernel."""
-    if cfg.io == "bf16" and cfg.dv == 128 and cfg.chunk == 128:
-        return "prefill_rows_kernel"
+    """The fused chunk-loop kernel that runs this workload (uniform batches):
+    128-token chunks with d_v = 128 and every d_v = 256 request (as a CTA pair in
+    128-token tiles) take the output-rows kernel, the others prefill_tc_kernel."""
+    if cfg.io == "bf16" and ((cfg.dv == 128 and cfg.chunk == 128) or cfg.dv == 256):
+        return "prefill_rows_kernel_pair" if cfg.dv == 256 else "prefill_rows_kernel"
     return "prefill_tc_kernel"
 
 
@@ -279,6 +280,10 @@ def config_of(name, seq_len=0):
 def config_dict(cfg, **extra):
     d = {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "N": cfg.N, "dk": cfg.dk, "dv": cfg.dv,
          "chunk": cfg.chunk, "io": "bf16 (fp32 state, fp32 gate logits)"}
+    if cfg.io == "bf16" and cfg.dv == 256:
+        # the chunkwise form is the same function for every chunk; d_v = 256 runs
+        # 128-token tiles on the CTA-pair output-rows kernel
+        d["tile"] = 128
     d.update(extra)
     return d
 
@@ -373,13 +378,15 @@ def prefill_summary(cfg, world, steps, ms, kern_ms, peaks):
                "frac_of_bf16_peak": alg_flops / step_s / 1e12 / peaks["bf16_tflops"],
                "peak_tflops": peaks["bf16_tflops"], "peak_source": peaks["source"] + " burst"},
         "path_hbm": {"alg_gbs": alg_bytes / step_s / 1e9, "frac": alg_bytes / step_s / 1e9 / peaks["hbm_gbs"]},
-        "roofline": {"kernel": (f"{fused_kernel_name(cfg)}<{cfg.dv}, {cfg.chunk}> (fused chunk loop)"
-                                if fused_kernel_name(cfg) == "prefill_tc_kernel"
-                                else f"{fused_kernel_name(cfg)} (fused chunk loop, output rows)"), "bound": "hbm",
+        "roofline": {"kernel": {"prefill_tc_kernel": f"prefill_tc_kernel<{cfg.dv}, {cfg.chunk}> (fused chunk loop)",
+                                "prefill_rows_kernel": "prefill_rows_kernel<false> (fused chunk loop, output rows)",
+                                "prefill_rows_kernel_pair": "prefill_rows_kernel<true> (fused chunk loop, output rows, "
+                                                            "CTA pair, 128-token tiles)"}[fused_kernel_name(cfg)],
+                     "bound": "hbm",
                      "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"],
                      "traffic": profiled_traffic(prefill_profile(cfg), PREFILL_SOURCE,
-                                                 ROWS_KERNEL_TEXT if fused_kernel_name(cfg) == "prefill_rows_kernel"
+                                                 ROWS_KERNEL_TEXT if fused_kernel_name(cfg).startswith("prefill_rows")
                                                  else None),
                      "alg_bytes_per_launch": alg_bytes, "launch_ms": kern_ms, "peak_source": peaks["source"]},
     }
