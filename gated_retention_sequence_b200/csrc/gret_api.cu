@@ -72,13 +72,12 @@ constexpr size_t kMaxSmem = 227 * 1024;
 
 // Chunk the tensor-core kernels run for a requested chunk.  The chunkwise form is
 // the same function for every chunk length (only the rounding differs), so
-// d_v = 256 runs 128-token chunks for uniform batches (the output-rows CTA
-// pair) and 64-token ones for packed batches, whichever of the two was asked.
+// d_v = 256 runs 128-token chunks (the output-rows CTA pair), uniform or packed,
+// whichever of 64 and 128 was asked.
 int run_chunk(int dk, int dv, int chunk, gret_dtype io, bool packed) {
+    (void)packed;
     if (io != GRET_BF16 || dk != 128 || dv != 256) return chunk;
-    if (!packed && chunk == 64) return 128;
-    if (packed && chunk == 128) return 64;
-    return chunk;
+    return chunk == 64 ? 128 : chunk;
 }
 
 // Kernel choice for a prefill; segments/seg_len describe the sequence split.

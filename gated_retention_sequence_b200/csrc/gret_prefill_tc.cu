@@ -1488,7 +1488,7 @@ __device__ __forceinline__ void scale_tile_row(uint8_t* tile, int row, float f) 
             scale_bf16x8(tile + x * RowsCfg::BOX + row * 128 + ((c ^ (row & 7)) << 4), f);
 }
 
-template <bool PAIR>
+template <bool PAIR, bool PACKED>
 __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __grid_constant__ TcParams p) {
     using CF = RowsCfg;
     constexpr int C = CF::C, DV = CF::DV;      // DV: the output channels (and state rows) of this CTA
@@ -1506,11 +1506,45 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
     const int rank = PAIR ? (int)cluster_ctarank() : 0;
     const int ch0 = rank * DV;
     const int item = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
-    const int u = item / p.P, seg = item % p.P;
-    const int hh = u % p.H, bb = u / p.H;
-    const int n_begin = seg * p.seg_len;
-    const int n_end = min(p.N, n_begin + p.seg_len);
+    // work item: a (unit, segment) of the uniform split, or of a packed batch's
+    // plan (a block past the plan's item count has nothing to do; both CTAs of a
+    // pair read the same count)
+    int u = 0, seg = 0, seg_len = p.seg_len;
+    if constexpr (PACKED) {
+        grid_dep_wait();
+        if (item >= p.plan_count[0]) return;
+        const int2 it = p.fused_items[item];
+        u = it.x;
+        seg = it.y;
+        seg_len = p.unit_info[u].y;
+    } else {
+        u = item / p.P;
+        seg = item % p.P;
+    }
+    // the seg_state slot of this segment's initial state (seg > 0), and whether
+    // it is its unit's last segment (worked out where they are needed)
+    auto in_slot = [&]() -> size_t {
+        if constexpr (PACKED) return (size_t)p.unit_info[u].z + seg - 1;
+        else return (size_t)u * p.slots + (size_t)seg * p.K - 1;
+    };
+    auto last_segment = [&]() -> bool {
+        if constexpr (PACKED) return seg == p.unit_info[u].x - 1;
+        else return seg == p.P - 1;
+    };
+    // this unit's tokens: rows row0 .. row0 + Nu - 1 of the (packed) tensors
+    const int hh = u % p.H;
+    int bb = u / p.H, row0 = 0, Nu = p.N;
+    if constexpr (PACKED) {
+        bb = 0;
+        packed_range(p.cu, u / p.H, p.total, row0, Nu);
+        Nu = min(Nu, p.N);                    // tokens past max_seqlen are not processed
+    }
+    const int n_begin = seg * seg_len;
+    const int n_end = min(Nu, n_begin + seg_len);
     const int nchunks = n_end > n_begin ? (n_end - n_begin + C - 1) / C : 0;
+    // rows of chunk j inside the sequence (a packed sequence's last chunk may
+    // end before its 128 rows; the rest are the next sequence's)
+    auto valid_rows = [&](int j) -> int { return min(C, n_end - (n_begin + j * C)); };
 
     // barriers; KT has one per Q/K stage so that no phase can complete twice
     // before the MMA warp has seen the first.  BG: the G tile of a chunk is in
@@ -1615,13 +1649,15 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
             // ======================================================== TMA producer
             int last_qk[2] = {-1, -1}, last_v = -1, last_g = -1;
             auto issue_qk = [&](int j) {
+                // n0: the chunk's first token within its unit (the decay sums are
+                // per unit); row0 + n0: its row in the (packed) tensors
                 const int s = j & 1, n0 = n_begin + j * C;
                 last_qk[s] = j;
                 const uint32_t fb = bar(BQK + s);
                 mbar_arrive_expect_tx(fb, 2 * CF::TILE + C * 4);
                 for (int x = 0; x < 2; ++x) {
-                    tma_load_4d(sb + CF::OFF_Q + s * CF::TILE + x * CF::BOX, &p.tmQ, x * 64, hh, n0, bb, fb);
-                    tma_load_4d(sb + CF::OFF_K + s * CF::TILE + x * CF::BOX, &p.tmK, x * 64, hh, n0, bb, fb);
+                    tma_load_4d(sb + CF::OFF_Q + s * CF::TILE + x * CF::BOX, &p.tmQ, x * 64, hh, row0 + n0, bb, fb);
+                    tma_load_4d(sb + CF::OFF_K + s * CF::TILE + x * CF::BOX, &p.tmK, x * 64, hh, row0 + n0, bb, fb);
                 }
                 bulk_load(sb + CF::OFF_B + s * C * 4, p.bcum + (size_t)u * p.Npad + n0, C * 4, fb);
             };
@@ -1629,7 +1665,8 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
                 last_v = j;
                 mbar_arrive_expect_tx(bar(BV), CF::TILE);
                 for (int x = 0; x < 2; ++x)
-                    tma_load_4d(sb + CF::OFF_V + x * CF::BOX, &p.tmV, ch0 + x * 64, hh, n_begin + j * C, bb, bar(BV));
+                    tma_load_4d(sb + CF::OFF_V + x * CF::BOX, &p.tmV, ch0 + x * 64, hh, row0 + n_begin + j * C, bb,
+                                bar(BV));
             };
             // the tile of chunk j: its G, or (without G) a plain release for its output
             auto issue_g = [&](int j) {
@@ -1640,7 +1677,8 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
                 last_g = j;
                 mbar_arrive_expect_tx(bar(BG), CF::TILE);
                 for (int x = 0; x < 2; ++x)
-                    tma_load_4d(sb + CF::OFF_G + x * CF::BOX, &p.tmG, ch0 + x * 64, hh, n_begin + j * C, bb, bar(BG));
+                    tma_load_4d(sb + CF::OFF_G + x * CF::BOX, &p.tmG, ch0 + x * 64, hh, row0 + n_begin + j * C, bb,
+                                bar(BG));
             };
             if (p.fault) mbar_wait_injected_timeout(bar(BNEVER), p.status, abort_flag);
             if (!*abort_flag) {
@@ -1654,13 +1692,17 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
                     if (i + 2 < nchunks) issue_qk(i + 2);
                     if (i + 1 < nchunks) issue_v(i + 1);
                     // the output of chunk i leaves from the tile (rows past the end of
-                    // the sequence fall outside the map and are not written); once the
-                    // store has read the tile it takes chunk i + 1
+                    // the tensors fall outside the map and are not written; a packed
+                    // sequence's short last chunk was stored row by row by the
+                    // epilogue); once the store has read the tile it takes chunk i + 1
                     if (!mbar_wait(bar(BGF), i & 1, p.status, abort_flag)) break;
-                    for (int x = 0; x < 2; ++x)
-                        tma_store_4d(&p.tmO, sb + CF::OFF_G + x * CF::BOX, ch0 + x * 64, hh, n_begin + i * C, bb);
-                    bulk_commit();
-                    bulk_wait_read<0>();
+                    if (!PACKED || valid_rows(i) == C) {
+                        for (int x = 0; x < 2; ++x)
+                            tma_store_4d(&p.tmO, sb + CF::OFF_G + x * CF::BOX, ch0 + x * 64, hh, row0 + n_begin + i * C,
+                                         bb);
+                        bulk_commit();
+                        bulk_wait_read<0>();
+                    }
                     if (i + 1 < nchunks) issue_g(i + 1);
                 }
             }
@@ -1744,7 +1786,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
             for (int cb = 0; cb < 4; ++cb) {
                 if (seg > 0) {
                     const float4* s4 = reinterpret_cast<const float4*>(
-                        p.seg_state + ((size_t)u * p.slots + (size_t)seg * p.K - 1) * DVT * DK +
+                        p.seg_state + in_slot() * DVT * DK +
                         (size_t)(ch0 + row) * DK + cb * 32);
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
@@ -1820,7 +1862,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
             mbar_wait(bar(BST), (nchunks - 1) & 1, p.status, abort_flag);
             tc_fence_after();
         }
-        if (p.S_final && seg == p.P - 1) {
+        if (p.S_final && last_segment()) {
             const float sc = __expf(lam);
             float* dst = p.S_final + (size_t)u * DK * DVT + ch0;
 #pragma unroll 1
@@ -1861,7 +1903,8 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
             mbar_wait(bar(BSC + s), (j >> 1) & 1, p.status, abort_flag);
             const float bCj = bc[C - 1];
             const bool eg = (-bCj - lam_k) > kLazyMax;
-            const float f = __expf(eg ? bCj - bc[kr] : -bc[kr] - lam_k);
+            // rows past the sequence's end (a packed batch's next sequence) add nothing
+            const float f = kr < valid_rows(j) ? __expf(eg ? bCj - bc[kr] : -bc[kr] - lam_k) : 0.f;
             uint8_t* krow = sm + CF::OFF_K + s * CF::TILE + (part >> 1) * CF::BOX + kr * 128;
 #pragma unroll
             for (int c = 0; c < 4; ++c) scale_bf16x8(krow + ((((part & 1) * 4 + c) ^ (kr & 7)) << 4), f);
@@ -1938,9 +1981,15 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
                 a = c * rsqrtf(var + p.eps);
                 b0 = -mean_u * a;
             }
-            // this token's 32 output channels go over its G in the tile
+            // this token's 32 output channels go over its G in the tile; a packed
+            // sequence's short last chunk is stored row by row instead (the rows
+            // after it are the next sequence's)
             mbar_wait(bar(BG), i & 1, p.status, abort_flag);
             uint8_t* grow = sm + CF::OFF_G + (hf >> 1) * CF::BOX + row * 128;
+            const bool direct = PACKED && valid_rows(i) < C;
+            uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.O) +
+                                                   ((size_t)(row0 + n0 + row) * p.H + hh) * DVT + ch0 + hf * QC);
+            const bool live = row < valid_rows(i);
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
                 uint4* slot = reinterpret_cast<uint4*>(grow + ((((hf & 1) * 4 + ch) ^ (row & 7)) << 4));
@@ -1957,6 +2006,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1) prefill_rows_kernel(const __g
                     e[j] = pack_bf16x2(o0, o1);
                 }
                 *slot = w;
+                if (direct && live) orow[ch] = w;
             }
             fence_proxy_async_smem();
             warp_arrive(BGF);              // the tile holds this chunk's output
@@ -2039,7 +2089,9 @@ struct VarlenLayout {
 VarlenLayout varlen_layout(int S, int H, int max_seqlen, int total, int dk, int dv, int chunk, int num_sms) {
     VarlenLayout w;
     const long long units = (long long)S * H;
-    const long long share = ((long long)total * H + 2LL * num_sms - 1) / (2LL * (num_sms > 0 ? num_sms : 1));
+    // concurrent work items: one per SM, or per pair of SMs for the d_v = 256 pair
+    const long long slots = std::max<long long>(1, num_sms / prefill_tc_ctas_per_item(dv, chunk));
+    const long long share = ((long long)total * H + 2LL * slots - 1) / (2LL * slots);
     long long seg_max = (share + chunk - 1) / chunk * chunk;
     if (seg_max < 4LL * chunk) seg_max = 4LL * chunk;
     if (seg_max > (1LL << 30)) seg_max = (1LL << 30) / chunk * chunk;
@@ -2115,7 +2167,7 @@ cudaError_t launch_pdl_pair(void (*kernel)(KArgs...), dim3 grid, dim3 block, siz
 // the others prefill_tc_kernel.
 template <int DV, int C, bool PACKED>
 cudaError_t run_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t s, const PlanArgs* plan = nullptr) {
-    constexpr bool ROWS = !PACKED && C == 128 && (DV == 128 || DV == 256) && GRET_ROWS_KERNEL;
+    constexpr bool ROWS = C == 128 && (DV == 128 || DV == 256) && GRET_ROWS_KERNEL;
     auto ks = prefill_state_kernel<DV, C, PACKED>;
     static bool attr_done[64] = {};
     int dev = 0;
@@ -2131,7 +2183,7 @@ cudaError_t run_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t s, const Pla
                 return cudaErrorInvalidConfiguration;
             cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<DV, C>::SMEM);
         } else {
-            auto kr = prefill_rows_kernel<DV == 256>;
+            auto kr = prefill_rows_kernel<DV == 256, PACKED>;
             cudaFuncAttributes fa;
             if (cudaFuncGetAttributes(&fa, kr) != cudaSuccess) return cudaErrorInvalidDeviceFunction;
             if (fa.numRegs > kRowsRegs) return cudaErrorInvalidConfiguration;
@@ -2144,8 +2196,6 @@ cudaError_t run_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t s, const Pla
     const int npad = tp.Npad;
     cudaError_t e = cudaSuccess;
     if constexpr (PACKED) {
-        auto kf = prefill_tc_kernel<DV, C, PACKED>;
-        using CF = Cfg<DV, C>;
         // gate scan, plan, state pass and combine over the plan's slots, fused loop
         int nyb = 0;
         const dim3 sgrid = gate_scan_grid(units, npad, C, &nyb);
@@ -2163,7 +2213,16 @@ cudaError_t run_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t s, const Pla
                        static_cast<const float*>(tp.seg_decay), tp.S0, 0, DK, DV, tp.unit_info);
         if (e != cudaSuccess) return e;
         if (g_profile_start) cudaEventRecord(g_profile_start, s);
-        e = launch_pdl(kf, dim3(plan->max_fused), dim3(kFusedThreads), CF::SMEM, s, tp);
+        if constexpr (ROWS) {
+            auto kr = prefill_rows_kernel<DV == 256, true>;
+            if constexpr (DV == 256)
+                e = launch_pdl_pair(kr, dim3(2 * plan->max_fused), dim3(kRowsThreads), RowsCfg::SMEM, s, tp);
+            else
+                e = launch_pdl(kr, dim3(plan->max_fused), dim3(kRowsThreads), RowsCfg::SMEM, s, tp);
+        } else {
+            e = launch_pdl(prefill_tc_kernel<DV, C, PACKED>, dim3(plan->max_fused), dim3(kFusedThreads),
+                           Cfg<DV, C>::SMEM, s, tp);
+        }
         if (g_profile_stop) cudaEventRecord(g_profile_stop, s);
         if (e != cudaSuccess) return e;
         return cudaGetLastError();
@@ -2202,7 +2261,7 @@ cudaError_t run_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t s, const Pla
     if constexpr (ROWS) {
         // 128-token chunks: the output-rows kernel (d_v 256: a pair of CTAs per
         // work item, each owning half of the channels)
-        auto kr = prefill_rows_kernel<DV == 256>;
+        auto kr = prefill_rows_kernel<DV == 256, false>;
         if (g_profile_start) cudaEventRecord(g_profile_start, s);
         if constexpr (DV == 256)
             e = launch_pdl_pair(kr, dim3(2 * units * tp.P), dim3(kRowsThreads), RowsCfg::SMEM, s, tp);
@@ -2390,7 +2449,8 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
     const bool packed = a.cu_seqlens != nullptr;
     if (a.dv == 256 && C == 64)
         return packed ? run_tc<256, 64, true>(a, tp, s, &plan) : run_tc<256, 64, false>(a, tp, s);
-    if (a.dv == 256 && C == 128 && !packed) return run_tc<256, 128, false>(a, tp, s);
+    if (a.dv == 256 && C == 128)
+        return packed ? run_tc<256, 128, true>(a, tp, s, &plan) : run_tc<256, 128, false>(a, tp, s);
     if (a.dv == 128 && C == 128)
         return packed ? run_tc<128, 128, true>(a, tp, s, &plan) : run_tc<128, 128, false>(a, tp, s);
     if (a.dv == 128 && C == 64)
