@@ -1311,16 +1311,22 @@ __global__ void __launch_bounds__(kPlanThreads) varlen_plan_kernel(const PlanArg
 // slot p <- S_in(p + 1) = e^{a_p} S_in(p) + dS_p, with S_in(0) = S0 (or 0).
 __global__ void seg_combine_kernel(float* __restrict__ seg_state, const float* __restrict__ seg_decay,
                                    const float* __restrict__ S0, int nslots, int dk, int dv,
-                                   const int4* __restrict__ unit_info) {
+                                   const int4* __restrict__ unit_info, const int2* __restrict__ state_items,
+                                   const int* __restrict__ plan_count) {
     grid_dep_launch();
     grid_dep_wait();       // the state pass's increments
-    const int u = blockIdx.x;
+    int u = blockIdx.x;
     const int elems4 = dk * dv / 4;
     const int e = blockIdx.y * blockDim.x + threadIdx.x;
     if (e >= elems4) return;
-    // a packed batch's plan gives each unit its own slot range
+    // a packed batch's plan: block x is state item x, and the first segment's
+    // item of each split unit folds that unit's slots (its own slot range)
     size_t base = (size_t)u * nslots;
     if (unit_info) {
+        if ((int)blockIdx.x >= plan_count[1]) return;
+        const int2 it = state_items[blockIdx.x];
+        if (it.y != 0) return;
+        u = it.x;
         const int4 ui = unit_info[u];
         nslots = ui.x - 1;
         base = (size_t)ui.z;
@@ -2209,8 +2215,9 @@ cudaError_t run_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t s, const Pla
         e = launch_pdl(ks, dim3(plan->max_state), dim3(kStateThreads), StateCfg<DV, C>::SMEM, s, tp);
         if (e != cudaSuccess) return e;
         const int elems4 = DV * DK / 4;
-        e = launch_pdl(seg_combine_kernel, dim3(units, (elems4 + 255) / 256), dim3(256), 0, s, tp.seg_state,
-                       static_cast<const float*>(tp.seg_decay), tp.S0, 0, DK, DV, tp.unit_info);
+        e = launch_pdl(seg_combine_kernel, dim3(plan->max_state, (elems4 + 255) / 256), dim3(256), 0, s,
+                       tp.seg_state, static_cast<const float*>(tp.seg_decay), tp.S0, 0, DK, DV, tp.unit_info,
+                       tp.state_items, tp.plan_count);
         if (e != cudaSuccess) return e;
         if (g_profile_start) cudaEventRecord(g_profile_start, s);
         if constexpr (ROWS) {
@@ -2255,7 +2262,8 @@ cudaError_t run_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t s, const Pla
         const int elems4 = DV * DK / 4;
         e = launch_pdl(seg_combine_kernel, dim3(units, (elems4 + 255) / 256), dim3(256), 0, s, tp.seg_state,
                        static_cast<const float*>(tp.seg_decay), tp.S0, tp.slots, DK, DV,
-                       static_cast<const int4*>(nullptr));
+                       static_cast<const int4*>(nullptr), static_cast<const int2*>(nullptr),
+                       static_cast<const int*>(nullptr));
         if (e != cudaSuccess) return e;
     }
     if constexpr (ROWS) {
@@ -2476,7 +2484,8 @@ static cudaError_t run_state_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t
     const int elems4 = DV * DK / 4;
     e = launch_pdl(seg_combine_kernel, dim3(units, (elems4 + 255) / 256), dim3(256), 0, s, tp.seg_state,
                    static_cast<const float*>(tp.seg_decay), static_cast<const float*>(nullptr), tp.slots, DK, DV,
-                   static_cast<const int4*>(nullptr));
+                   static_cast<const int4*>(nullptr), static_cast<const int2*>(nullptr),
+                   static_cast<const int*>(nullptr));
     if (e != cudaSuccess) return e;
     state_finish_kernel<DV><<<dim3(units, (DV / 32) * (DK / 32)), dim3(32, 8), 0, s>>>(tp.seg_state, tp.seg_decay,
                                                                                   tp.slots, a.S_final, a.decay_out);
