@@ -112,3 +112,14 @@ def test_equal_lengths_match_the_uniform_call():
     # the same values up to the bf16 rounding of the tensor-core path
     assert_close(O_v.reshape(B, N, H, -1), O_u.double().cpu().numpy(), "bf16", "O")
     assert_close(S_v, S_u.double().cpu().numpy(), "bf16", "S_final")
+
+
+@pytest.mark.parametrize("dv,chunk", [(128, 128), (256, 64)])
+def test_many_short_sequences(dv, chunk):
+    """200 sequences of 0 to 299 tokens and 4 heads: 800 units, more than five
+    times the SMs, in the plan's longest-first order; empty sequences keep
+    S_final = S0."""
+    lengths = [int(x) for x in np.random.default_rng(5).integers(0, 300, size=200)]
+    lengths[3] = 0
+    lengths[7] = 1
+    _run(lengths, dv, chunk, H=4, seed=48 + dv, with_s0=True)
