@@ -459,6 +459,7 @@ gret_status gret_prefill_backward(const void* Q, const void* K, const void* V, c
     a.dQ = dQ; a.dK = dK; a.dV = dV; a.dG = dG; a.dz = dz; a.dS0 = dS0; a.workspace = workspace;
     a.B = B; a.H = H; a.N = N; a.dk = dk; a.dv = dv; a.inv_tau = 1.0f / tau; a.eps = eps;
     a.gn = epi == GRET_EPI_GN_SWISH ? 1 : 0; a.io = io_dtype;
+    if (!device_info(&a.status, nullptr)) return GRET_ERR_CUDA;
     return launch_prefill_backward(a, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? GRET_OK
                                                                                         : GRET_ERR_CUDA;
 }

@@ -349,6 +349,7 @@ size_t bwd_ckpt_smem(int dk, int dv) { return sizeof(float) * ((size_t)kBlk * (d
 }  // namespace
 
 size_t prefill_backward_workspace_bytes(int B, int H, int N, int dk, int dv, gret_dtype io) {
+    if (bwd_tc_supported(B, H, N, dk, dv, io)) return bwd_tc_workspace_bytes(B, H, N, dv);
     if (bwd_chunked_supported(B, H, N, dk, dv, io)) return bwd_chunked_workspace_bytes(B, H, N, dk, dv, io);
     const size_t units = (size_t)B * H, nblk = (N + kBlk - 1) / kBlk, E = (size_t)dk * dv;
     const size_t ck = (units * nblk * E * 4 + 255) & ~size_t(255);
@@ -358,10 +359,11 @@ size_t prefill_backward_workspace_bytes(int B, int H, int N, int dk, int dv, gre
 bool prefill_backward_supported(int dk, int dv) { return bwd_block_smem(dk, dv) <= 227 * 1024; }
 
 int prefill_backward_launches(int B, int H, int N, int dk, int dv, gret_dtype io) {
-    return bwd_chunked_supported(B, H, N, dk, dv, io) ? 5 : 2;
+    return bwd_tc_supported(B, H, N, dk, dv, io) || bwd_chunked_supported(B, H, N, dk, dv, io) ? 5 : 2;
 }
 
 cudaError_t launch_prefill_backward(const BackwardArgs& in, cudaStream_t s) {
+    if (bwd_tc_supported(in.B, in.H, in.N, in.dk, in.dv, in.io)) return launch_bwd_tc(in, s);
     if (bwd_chunked_supported(in.B, in.H, in.N, in.dk, in.dv, in.io)) return launch_bwd_chunked(in, s);
     BwdArgs a;
     a.Q = in.Q; a.K = in.K; a.V = in.V; a.G = in.G; a.dO = in.dO;

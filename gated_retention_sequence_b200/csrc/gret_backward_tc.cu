@@ -1,0 +1,1375 @@
+// Tensor-core (tcgen05) backward of the gated-retention prefill for bf16 inputs
+// with d_k = 128 and d_v of 128 or 256, on chunks of 128 tokens.
+//
+// The forward is the chunkwise form of "YOCO 深度技术分析" (sections 2.2 and
+// 5.3.2).  Per unit and chunk c of L <= 128 tokens with state S_c before it,
+// b_t the chunk-local inclusive sum of log gamma, b_L its total and
+// E_ts = e^{b_t - b_s} on s <= t:
+//   y_t     = sum_s (q_t . k_s) E_ts v_s + e^{b_t} q_t S_c
+//   S_{c+1} = e^{b_L} S_c + sum_s e^{b_L - b_s} k_s^T v_s
+// With dy the gradient of y (GroupNorm * swish backward), D_ts = dy_t . v_s,
+// A_ts = q_t . k_s and dS'_c the gradient at chunk c's end
+// (dS'_{c-1} = e^{b_L} dS'_c + sum_t e^{b_t} q_t^T dy_t):
+//   dq_t = sum_s D_ts E_ts k_s + e^{b_t} dy_t S_c^T
+//   dk_s = sum_t D_ts E_ts q_t + e^{b_L - b_s} v_s dS'_c^T
+//   dv_s = sum_t A_ts E_ts dy_t + e^{b_L - b_s} k_s dS'_c
+// and the gate gradient of token j as four sums over the (s, t) pairs that
+// straddle it (s < j <= t), none of which cancels:
+//   dlg_j = sum_{t>=j, s<j} A_ts D_ts E_ts           (F_j, within the chunk)
+//         + sum_{t>=j} dy_t . (e^{b_t} q_t S_c)        (earlier chunks -> t)
+//         + e^{b_L} <dS'_c, S_c>                       (earlier -> later chunks)
+//         + sum_{s<j} e^{b_L - b_s} k_s . (dS'_c v_s)  (s -> later chunks)
+// (the final state's gradient enters through dS' of the last chunk).
+//
+// Five launches:
+//   1. bwd_inc_tc      per chunk: e^{b_L} and the increment K~^T V (tcgen05)
+//   2. bwd_scan_fwd    per state element: S_c of every chunk as a bf16 pair
+//                      (hi = bf16(S), lo = bf16(S - hi))
+//   3. bwd_dyq_tc      per chunk: y, the GroupNorm * swish backward (dG, dy),
+//                      G_c = sum_t e^{b_t} q_t^T dy_t and dq (tcgen05)
+//   4. bwd_scan_rev    per state element: dS'_c as a bf16 pair, dS0 and
+//                      e^{b_L} <dS'_c, S_c>
+//   5. bwd_kv_tc       per chunk: dk, dv and dz (tcgen05)
+// The products whose operands are not bf16 inputs take them as bf16 pairs:
+// a product with one such operand costs two MMAs (x_hi, x_lo), with two of
+// them three (hi hi, hi lo, lo hi), which keeps about 16 mantissa bits.  The
+// decay factors of a row (e^{b_t}, e^{b_L - b_s}) are applied to fp32
+// accumulator rows in tensor memory instead of being folded into an operand.
+// The masked score matrices (P, D o E, A o E) are single bf16 operands, as in
+// the forward.  With d_v = 256 a chunk runs on a cluster of two CTAs, each
+// owning 128 of the output channels: the GroupNorm row sums cross the pair
+// through distributed shared memory, and the partial dq (dk) of the two
+// channel halves are added by the CTA that stores the row.
+#include <cuda.h>
+
+#include <algorithm>
+#include <cstring>
+#include <utility>
+
+#include "gret_common.cuh"
+#include "gret_sm100.cuh"
+
+namespace gret {
+namespace {
+
+using namespace sm100;
+
+constexpr int kC = 128;                  // chunk length
+constexpr int kDK = 128;                 // d_k
+constexpr int kBox = 128 * 128;          // bytes of one [128 rows][64 bf16] swizzled box
+constexpr int kTile = 2 * kBox;          // [128 rows][128 bf16]
+constexpr int kRowThreads = 256;         // eight warps: lane quarter q = w & 3, column half w >> 2
+constexpr int kThreads = kRowThreads + 32;
+constexpr int kNamedBar = 1;             // named barrier among the row warps
+
+struct BwdTcParams {
+    CUtensorMap tmQ, tmK, tmV, tmDyH, tmDyL, tmSH, tmSL;
+    const void *Q, *K, *V, *G, *dO;
+    const float *z, *S0, *dS_final;
+    void *dQ, *dK, *dV, *dG;
+    float *dz, *dS0;
+    float* incg;              // [units][nc][dk][dv] fp32: increments, then G_c
+    __nv_bfloat16* sh;        // [units][nc][dk][dv]: S_c hi, then dS'_c hi
+    __nv_bfloat16* sl;        // the lo halves
+    __nv_bfloat16* dyh;       // [B][N][H][dv] dy hi
+    __nv_bfloat16* dyl;       // dy lo
+    float* rr;                // [2][B][N][H] per channel half: dy_t . (e^{b_t} q_t S_c)
+    float* xs;                // [units][nc] e^{b_L} <dS'_c, S_c>
+    float* decay;             // [units][nc] e^{b_L}
+    float* fus;               // [units][nc][256]: F and us partials of a pair's second CTA
+    unsigned int* status;
+    int B, H, N, dv, nc;
+    float inv_tau, eps;
+    int gn;
+};
+
+__device__ __forceinline__ float u2f(uint32_t x) { return __uint_as_float(x); }
+__device__ __forceinline__ uint32_t f2u(float x) { return __float_as_uint(x); }
+
+// bf16 pair of x: hi = bf16(x), lo = bf16(x - hi)
+__device__ __forceinline__ void split2(float x, float y, uint32_t& hi, uint32_t& lo) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
+    const float2 hf = __bfloat1622float2(h);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(x - hf.x, y - hf.y);
+    hi = *reinterpret_cast<const uint32_t*>(&h);
+    lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+// Byte offset of element (row r, column x < 64) of a [rows][64 bf16] box in
+// the 128-byte swizzle layout (16-byte chunk x / 8 of row r sits at chunk
+// (x / 8) ^ (r % 8)); boxes are 1024-byte aligned.
+__device__ __forceinline__ uint32_t sw128(int r, int x) {
+    return (uint32_t)(r * 128 + ((((x >> 3) ^ (r & 7)) & 7) << 4) + (x & 7) * 2);
+}
+
+// Chunk-local decay sums b_t of the chunk's tokens (0 past L: b_t = b_{L-1})
+// into bc[0..127], and e^{b_L} on request; threads 0..127 of the row warps
+// take part (warps 0-3), the row warps sync after.
+__device__ __forceinline__ void chunk_decay(const BwdTcParams& p, size_t tok0, int hh, int L, float* bc, float* wsum) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid < kC) {
+        float x = tid < L ? log_gamma(p.z[(tok0 + tid) * p.H + hh], p.inv_tau) : 0.f;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) wsum[warp] = x;
+        bc[tid] = x;
+    }
+    named_bar_sync(kNamedBar, kRowThreads);
+    if (tid < kC) {
+        float add = 0.f;
+        for (int w = 0; w < warp; ++w) add += wsum[w];
+        bc[tid] += add;
+    }
+    named_bar_sync(kNamedBar, kRowThreads);
+}
+
+// ---- 1. per chunk: e^{b_L} and inc_c = sum_s e^{b_L - b_s} k_s^T v_s into
+// slot c of incg ([d][j] fp32).  K~ = diag(e^{b_L - b}) K is formed in shared
+// memory as a bf16 pair; the MMA is D[d][j] = K~^T V (A = K~ MN-major,
+// B = V MN-major), two passes.
+template <int DV>
+struct IncCfg {
+    static constexpr int OFF_K = 0;                    // K~ hi (in place of K)
+    static constexpr int OFF_KL = kTile;               // K~ lo
+    static constexpr int OFF_V = 2 * kTile;            // DV / 64 boxes
+    static constexpr int OFF_BC = OFF_V + DV / 64 * kBox;
+    static constexpr int OFF_BAR = OFF_BC + kC * 4 + 64;
+    static constexpr int OFF_MISC = OFF_BAR + 64;
+    static constexpr int SMEM = OFF_MISC + 64 + 1024;  // + alignment slack
+};
+
+template <int DV>
+__global__ void __launch_bounds__(kThreads, 1) bwd_inc_tc(const __grid_constant__ BwdTcParams p) {
+    using CF = IncCfg<DV>;
+    extern __shared__ uint8_t smraw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sb = smem_u32(sm);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nc = p.nc, u = blockIdx.x / nc, c = blockIdx.x - u * nc, b = u / p.H, hh = u - b * p.H;
+    const int n0 = c * kC, L = min(kC, p.N - n0);
+    const size_t tok0 = (size_t)b * p.N + n0;
+    const bool need = c + 1 < nc;   // the last chunk's increment is never used
+    float* bc = reinterpret_cast<float*>(sm + CF::OFF_BC);
+    float* wsum = bc + kC;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + CF::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + CF::OFF_MISC + 4);
+    const uint32_t bar_ld = sb + CF::OFF_BAR, bar_mma = sb + CF::OFF_BAR + 8, bar_rdy = sb + CF::OFF_BAR + 16;
+    if (tid == kRowThreads) {
+        mbar_init(bar_ld, 1);
+        mbar_init(bar_mma, 1);
+        mbar_init(bar_rdy, kRowThreads / 32);
+        *abort_flag = 0;
+        fence_mbar_init();
+        if (need) {
+            mbar_arrive_expect_tx(bar_ld, kTile + DV / 64 * kBox);
+            for (int x = 0; x < 2; ++x)
+                tma_load_4d(sb + CF::OFF_K + x * kBox, &p.tmK, x * 64, hh, n0, b, bar_ld);
+            for (int x = 0; x < DV / 64; ++x)
+                tma_load_4d(sb + CF::OFF_V + x * kBox, &p.tmV, x * 64, hh, n0, b, bar_ld);
+        }
+    }
+    if (warp == kRowThreads / 32) {
+        tmem_alloc(smem_u32(tmem_slot), DV);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = *tmem_slot;
+
+    if (tid < kRowThreads) {
+        chunk_decay(p, tok0, hh, L, bc, wsum);
+        const float bL = bc[kC - 1];
+        if (tid == 0) {
+            p.decay[(size_t)u * nc + c] = __expf(bL);
+            p.xs[(size_t)u * nc + c] = 0.f;   // the reverse scan accumulates here
+        }
+        // K~ = e^{b_L - b_s} k_s as a bf16 pair: row s, 64 columns per thread
+        const int s = tid & 127, xb = tid >> 7;
+        const float w = s < L ? __expf(bL - bc[s]) : 0.f;
+        if (need && mbar_wait(bar_ld, 0, p.status, abort_flag)) {
+            uint8_t* row = sm + CF::OFF_K + xb * kBox + s * 128;
+            uint8_t* rowl = sm + CF::OFF_KL + xb * kBox + s * 128;
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+                uint4 v = *reinterpret_cast<const uint4*>(row + ch * 16), hi, lo;
+                const uint32_t* e = reinterpret_cast<const uint32_t*>(&v);
+                uint32_t* h = reinterpret_cast<uint32_t*>(&hi);
+                uint32_t* l = reinterpret_cast<uint32_t*>(&lo);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    split2(u2f(e[k] << 16) * w, u2f(e[k] & 0xffff0000u) * w, h[k], l[k]);
+                *reinterpret_cast<uint4*>(row + ch * 16) = hi;    // the swizzle permutes whole
+                *reinterpret_cast<uint4*>(rowl + ch * 16) = lo;   // 16-byte chunks of one row
+            }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_rdy);
+    } else if (lane == 0) {
+        // ============================================================ MMA issuer
+        constexpr uint32_t id = idesc_bf16(128, DV, true, true);
+        if (mbar_wait(bar_rdy, 0, p.status, abort_flag) && need) {
+            tc_fence_after();
+            for (int pass = 0; pass < 2; ++pass) {
+                const uint32_t sK = sb + (pass ? CF::OFF_KL : CF::OFF_K);
+#pragma unroll
+                for (int k = 0; k < kC / 16; ++k)
+                    mma_ss(tm, sdesc_sw128(sK + k * 2048, kBox, 1024), sdesc_sw128(sb + CF::OFF_V + k * 2048, kBox, 1024),
+                           id, pass > 0 || k > 0);
+            }
+        }
+        mma_commit(bar_mma);
+    }
+    // store: row d of the increment (TMEM lane d), DV / 2 columns per thread
+    if (tid < kRowThreads) {
+        const int q = warp & 3, half = warp >> 2, d = 32 * q + lane;
+        if (mbar_wait(bar_mma, 0, p.status, abort_flag) && need) {
+            tc_fence_after();
+            float* dst = p.incg + (((size_t)u * nc + c) * kDK + d) * DV + half * (DV / 2);
+#pragma unroll 1
+            for (int cb = 0; cb < DV / 64; ++cb) {
+                uint32_t r[32];
+                tmem_ld_x32(tm + ((uint32_t)(32 * q) << 16) + half * (DV / 2) + cb * 32, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    reinterpret_cast<float4*>(dst + cb * 32)[k] =
+                        make_float4(u2f(r[4 * k]), u2f(r[4 * k + 1]), u2f(r[4 * k + 2]), u2f(r[4 * k + 3]));
+            }
+        }
+    } else if (lane == 0 && *abort_flag) {
+        if (need) mbar_wait_drain(bar_ld, 0, kWaitCycles);
+        mbar_wait_drain(bar_mma, 0, kWaitCycles);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kRowThreads / 32) tmem_dealloc(tm, DV);
+}
+
+// ---- 2. per state element (4 per thread): S_0 = S0 (or 0), S_{c+1} =
+// e^{b_L(c)} S_c + inc_c; S_c of every chunk as a bf16 pair
+constexpr int kScanThreads = 256;
+__global__ void __launch_bounds__(kScanThreads) bwd_scan_fwd(const __grid_constant__ BwdTcParams p) {
+    const size_t E4 = (size_t)kDK * p.dv / 4;
+    const int nc = p.nc;
+    const size_t u = blockIdx.y, e4 = (size_t)blockIdx.x * kScanThreads + threadIdx.x;
+    const bool on = e4 < E4;
+    const float4* inc = reinterpret_cast<const float4*>(p.incg) + u * nc * E4 + e4;
+    uint2* hi = reinterpret_cast<uint2*>(p.sh) + u * nc * E4 + e4;
+    uint2* lo = reinterpret_cast<uint2*>(p.sl) + u * nc * E4 + e4;
+    const float* dec = p.decay + u * nc;
+    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (on && p.S0) s = reinterpret_cast<const float4*>(p.S0)[u * E4 + e4];
+    if (!on) return;
+    float4 nxt = nc > 1 ? inc[0] : s;
+    for (int c = 0; c < nc; ++c) {
+        uint2 h, l;
+        split2(s.x, s.y, h.x, l.x);
+        split2(s.z, s.w, h.y, l.y);
+        hi[(size_t)c * E4] = h;
+        lo[(size_t)c * E4] = l;
+        if (c + 1 == nc) break;
+        const float4 d = nxt;
+        if (c + 2 < nc) nxt = inc[(size_t)(c + 1) * E4];
+        const float g = dec[c];
+        s.x = fmaf(g, s.x, d.x);
+        s.y = fmaf(g, s.y, d.y);
+        s.z = fmaf(g, s.z, d.z);
+        s.w = fmaf(g, s.w, d.w);
+    }
+}
+
+// ---- 4. per state element, from the last chunk back: cur = dS_final (or 0);
+// for c = nc-1 .. 0: X_c += e^{b_L} <cur, S_c> (S_c from its bf16 pair, read
+// before it is overwritten), slot c <- cur as a bf16 pair, cur = e^{b_L} cur
+// + G_c; dS0 = cur
+__global__ void __launch_bounds__(kScanThreads) bwd_scan_rev(const __grid_constant__ BwdTcParams p) {
+    __shared__ float red[kScanThreads / 32];
+    const size_t E4 = (size_t)kDK * p.dv / 4;
+    const int nc = p.nc;
+    const size_t u = blockIdx.y, e4 = (size_t)blockIdx.x * kScanThreads + threadIdx.x;
+    const bool on = e4 < E4;
+    const float4* gc = reinterpret_cast<const float4*>(p.incg) + u * nc * E4 + e4;
+    uint2* hi = reinterpret_cast<uint2*>(p.sh) + u * nc * E4 + e4;
+    uint2* lo = reinterpret_cast<uint2*>(p.sl) + u * nc * E4 + e4;
+    const float* dec = p.decay + u * nc;
+    float4 cur = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (on && p.dS_final) cur = reinterpret_cast<const float4*>(p.dS_final)[u * E4 + e4];
+    for (int c = nc - 1; c >= 0; --c) {
+        float acc = 0.f;
+        float4 g = make_float4(0.f, 0.f, 0.f, 0.f);
+        const float e = dec[c];
+        if (on) {
+            g = gc[(size_t)c * E4];
+            const uint2 h = hi[(size_t)c * E4], l = lo[(size_t)c * E4];
+            const float s0 = u2f(h.x << 16) + u2f(l.x << 16), s1 = u2f(h.x & 0xffff0000u) + u2f(l.x & 0xffff0000u);
+            const float s2 = u2f(h.y << 16) + u2f(l.y << 16), s3 = u2f(h.y & 0xffff0000u) + u2f(l.y & 0xffff0000u);
+            acc = e * (cur.x * s0 + cur.y * s1 + cur.z * s2 + cur.w * s3);
+            uint2 nh, nl;
+            split2(cur.x, cur.y, nh.x, nl.x);
+            split2(cur.z, cur.w, nh.y, nl.y);
+            hi[(size_t)c * E4] = nh;
+            lo[(size_t)c * E4] = nl;
+            cur.x = fmaf(e, cur.x, g.x);
+            cur.y = fmaf(e, cur.y, g.y);
+            cur.z = fmaf(e, cur.z, g.z);
+            cur.w = fmaf(e, cur.w, g.w);
+        }
+        acc = warp_sum(acc);
+        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            float t = 0.f;
+            for (int w = 0; w < kScanThreads / 32; ++w) t += red[w];
+            atomicAdd(p.xs + u * nc + c, t);
+        }
+        __syncthreads();
+    }
+    if (on && p.dS0) reinterpret_cast<float4*>(p.dS0)[u * E4 + e4] = cur;
+}
+
+// Shared-memory layout of the two per-chunk gradient kernels: seven
+// [128][128] bf16 tiles (two 64-column swizzled boxes each), then small arrays.
+struct GradCfg {
+    static constexpr int OFF_T0 = 0;
+    static constexpr int OFF_BC = 7 * kTile;          // b_t [128], 4 warp sums
+    static constexpr int OFF_AUX = OFF_BC + 528;      // 2 KB: exchange buffers / row sums
+    static constexpr int NUM_BARS = 18;
+    static constexpr int OFF_BAR = OFF_AUX + 2048;
+    static constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;
+    static constexpr int SMEM = OFF_MISC + 16;
+    static_assert(SMEM <= 227 * 1024, "shared memory");
+};
+
+// ---- 3. per chunk: y = P V + e^{b_t} Q S_c, the GroupNorm * swish backward
+// (dG; dy as a bf16 pair to the workspace), G_c = sum_t e^{b_t} q_t^T dy_t into
+// slot c of incg, rr_t = dy_t . (e^{b_t} q_t S_c), and
+// dq = (D o E) K + e^{b_t} dy S_c^T.  With PAIR the CTA of cluster rank h owns
+// channels 128 h .. 128 h + 127 and rows 64 h .. 64 h + 63 of dq.
+//
+// Tensor memory (512 columns): [0,128) scores A, then D, then D o E (bf16);
+// [128,256) Y = P V, then e^{b_t} dy S^T + (D o E) K; [256,384) Yi = Q S, then
+// G_c; [384,512) P (bf16), then Q~^T as a bf16 pair.
+// Shared memory tiles: Q, K, V (this CTA's channels), S_c hi, S_c lo, dy hi,
+// dy lo; the dy lo tile is scratch for the row sums until dy is written.
+template <bool PAIR>
+__global__ void __launch_bounds__(kThreads, 1) bwd_dyq_tc(const __grid_constant__ BwdTcParams p) {
+    using CF = GradCfg;
+    constexpr int OFF_Q = 0, OFF_K = kTile, OFF_V = 2 * kTile, OFF_SH = 3 * kTile, OFF_SL = 4 * kTile,
+                  OFF_DYH = 5 * kTile, OFF_DYL = 6 * kTile;
+    constexpr uint32_t R_A = 0, R_Y = 128, R_YI = 256, R_P = 384;
+    constexpr int BQK = 0, BVS = 1, BA = 2, BYI = 3, BP = 4, BY = 5, BDY = 6, BD = 7, BQI = 8, BQT = 9, BGC = 10,
+                  BDS = 11, BDQ = 12, BX0 = 13, BX1 = 14, BX2 = 15, BXQ = 16, BDRAIN = 17;
+    extern __shared__ __align__(1024) uint8_t sm[];
+    const uint32_t sb = smem_u32(sm);
+    if (sb & 1023u) {
+        if (threadIdx.x == 0) atomicExch(p.status, kDevSmemLayout);
+        return;
+    }
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int rank = PAIR ? (int)cluster_ctarank() : 0;
+    const int item = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+    const int nc = p.nc, u = item / nc, c = item - u * nc, b = u / p.H, hh = u - b * p.H;
+    const int n0 = c * kC, L = min(kC, p.N - n0);
+    const size_t tok0 = (size_t)b * p.N + n0;
+    const int DV = p.dv, ch0 = 128 * rank;
+    auto bar = [&](int i) -> uint32_t { return sb + CF::OFF_BAR + 8 * i; };
+    float* bc = reinterpret_cast<float*>(sm + CF::OFF_BC);
+    float* wsum = bc + kC;
+    float* xch = reinterpret_cast<float*>(sm + CF::OFF_AUX);   // [128] round 0, [128] round 1, [128][2] round 2
+    float* scr = reinterpret_cast<float*>(sm + OFF_DYL);       // [9][128] row partial sums
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + CF::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + CF::OFF_MISC + 4);
+
+    if (tid == kRowThreads) {
+        for (int i = 0; i < CF::NUM_BARS; ++i)
+            mbar_init(bar(i), (i == BP || i == BDY || i == BQT || i == BDS) ? kRowThreads / 32 : 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        if (PAIR) {
+            // one-shot exchange barriers, armed for the bytes the other CTA sends
+            if (p.gn) {
+                mbar_arrive_expect_tx(bar(BX0), kC * 4);
+                mbar_arrive_expect_tx(bar(BX1), kC * 4);
+                mbar_arrive_expect_tx(bar(BX2), kC * 8);
+            }
+            mbar_arrive_expect_tx(bar(BXQ), 64 * 128 * 4);
+        }
+        tma_prefetch_desc(&p.tmQ);
+        tma_prefetch_desc(&p.tmK);
+        tma_prefetch_desc(&p.tmV);
+        tma_prefetch_desc(&p.tmSH);
+        tma_prefetch_desc(&p.tmSL);
+    }
+    if (warp == kRowThreads / 32) {
+        tmem_alloc(smem_u32(tmem_slot), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if constexpr (PAIR) cluster_sync_all();
+    const uint32_t tm = *tmem_slot;
+    const uint32_t peer = (uint32_t)(rank ^ 1);
+
+    float dq[64];
+    if (tid < kRowThreads) {
+        const int q = warp & 3, half = warp >> 2, t = 32 * q + lane;
+        const uint32_t lq = (uint32_t)(32 * q) << 16;
+        auto warp_arrive = [&](int i) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(i));
+        };
+        chunk_decay(p, tok0, hh, L, bc, wsum);
+        const float bt = bc[t], ebt = __expf(bt);
+
+        // ---------------------------------------------------- P = A o E, masked
+        if (mbar_wait(bar(BA), 0, p.status, abort_flag)) {
+            tc_fence_after();
+            uint32_t r[32], pk[16];
+#pragma unroll 1
+            for (int cb = 0; cb < 2; ++cb) {
+                tmem_ld_x32(tm + lq + R_A + 64 * half + 32 * cb, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const int s0 = 64 * half + 32 * cb + 2 * j;
+                    const float v0 = s0 <= t ? u2f(r[2 * j]) * __expf(fminf(bt - bc[s0], 0.f)) : 0.f;
+                    const float v1 = s0 + 1 <= t ? u2f(r[2 * j + 1]) * __expf(fminf(bt - bc[s0 + 1], 0.f)) : 0.f;
+                    pk[j] = pack_bf16x2(v0, v1);
+                }
+                tmem_st_x16(tm + lq + R_P + 32 * half + 16 * cb, pk);
+            }
+            tmem_wait_st();
+        }
+        tc_fence_before();
+        warp_arrive(BP);
+
+        // ---------------------------------------------------- GroupNorm * swish backward
+        const size_t rowoff = ((tok0 + t) * p.H + hh) * (size_t)DV + ch0 + 64 * half;
+        uint4 gv[8], ov[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            ov[k] = t < L ? reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.dO) + rowoff)[k]
+                          : make_uint4(0u, 0u, 0u, 0u);
+            gv[k] = (t < L && p.gn) ? reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.G) + rowoff)[k]
+                                    : make_uint4(0u, 0u, 0u, 0u);
+        }
+        // sum over the row's d_v channels of (a, b): the two column-half warps
+        // through `scr`, the pair through distributed shared memory
+        auto row_sum = [&](int slot, int xbar, float a, float bv, bool two, float& ra, float& rb) {
+            if (half) {
+                scr[(2 * slot) * kC + t] = a;
+                if (two) scr[(2 * slot + 1) * kC + t] = bv;
+            }
+            named_bar_sync(kNamedBar, kRowThreads);
+            if (!half) {
+                a += scr[(2 * slot) * kC + t];
+                if (two) bv += scr[(2 * slot + 1) * kC + t];
+                if constexpr (PAIR) {
+                    const int off = slot == 0 ? t : slot == 1 ? kC + t : 2 * kC + 2 * t;
+                    const uint32_t remote = cluster_map(smem_u32(xch + off), peer);
+                    const uint32_t rbar = cluster_map(bar(xbar), peer);
+                    if (two)
+                        st_async_f2(remote, rbar, a, bv);
+                    else
+                        st_async_f1(remote, rbar, a);
+                    if (mbar_wait_cluster(bar(xbar), 0, p.status, abort_flag)) {
+                        a += xch[off];
+                        if (two) bv += xch[off + 1];
+                    }
+                }
+                scr[(2 * slot) * kC + t] = a;
+                if (two) scr[(2 * slot + 1) * kC + t] = bv;
+            }
+            named_bar_sync(kNamedBar, kRowThreads);
+            ra = scr[(2 * slot) * kC + t];
+            rb = two ? scr[(2 * slot + 1) * kC + t] : 0.f;
+            named_bar_sync(kNamedBar, kRowThreads);
+        };
+        float y[64];
+        const bool ok_y = mbar_wait(bar(BY), 0, p.status, abort_flag) && mbar_wait(bar(BYI), 0, p.status, abort_flag);
+        tc_fence_after();
+        if (ok_y) {
+            uint32_t r[32], ri[32];
+#pragma unroll
+            for (int cb = 0; cb < 2; ++cb) {
+                tmem_ld_x32(tm + lq + R_Y + 64 * half + 32 * cb, r);
+                tmem_ld_x32(tm + lq + R_YI + 64 * half + 32 * cb, ri);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) y[32 * cb + j] = fmaf(ebt, u2f(ri[j]), u2f(r[j]));
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 64; ++j) y[j] = 0.f;
+        }
+        if (p.gn) {
+            const float inv_dv = 1.0f / (float)DV;
+            float s1 = 0.f, dummy;
+#pragma unroll
+            for (int j = 0; j < 64; ++j) s1 += y[j];
+            float mean;
+            row_sum(0, BX0, s1, 0.f, false, mean, dummy);
+            mean *= inv_dv;
+            float s2 = 0.f;
+#pragma unroll
+            for (int j = 0; j < 64; ++j) {
+                y[j] -= mean;
+                s2 = fmaf(y[j], y[j], s2);
+            }
+            float var;
+            row_sum(1, BX1, s2, 0.f, false, var, dummy);
+            const float rstd = rsqrtf(var * inv_dv + p.eps);
+            float m1 = 0.f, m2 = 0.f;
+            __nv_bfloat16* dGg = static_cast<__nv_bfloat16*>(p.dG) + rowoff;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const uint32_t* ge = reinterpret_cast<const uint32_t*>(&gv[k]);
+                const uint32_t* oe = reinterpret_cast<const uint32_t*>(&ov[k]);
+                uint4 dg;
+                uint32_t* dge = reinterpret_cast<uint32_t*>(&dg);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    float out[2];
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf) {
+                        const int j = 8 * k + 2 * e + hf;
+                        const float g = hf ? u2f(ge[e] & 0xffff0000u) : u2f(ge[e] << 16);
+                        const float o = hf ? u2f(oe[e] & 0xffff0000u) : u2f(oe[e] << 16);
+                        const float sg = sigmoidf_(g);
+                        const float n = y[j] * rstd;
+                        y[j] = n;
+                        // d/dg [g sigmoid(g)] = sigmoid(g) (1 + g (1 - sigmoid(g)))
+                        out[hf] = o * n * sg * (1.f + g * (1.f - sg));
+                        const float dn = o * g * sg;
+                        m1 += dn;
+                        m2 = fmaf(dn, n, m2);
+                    }
+                    dge[e] = pack_bf16x2(out[0], out[1]);
+                }
+                if (t < L) reinterpret_cast<uint4*>(dGg)[k] = dg;
+            }
+            row_sum(2, BX2, m1, m2, true, m1, m2);
+            m1 *= inv_dv;
+            m2 *= inv_dv;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const uint32_t* ge = reinterpret_cast<const uint32_t*>(&gv[k]);
+                const uint32_t* oe = reinterpret_cast<const uint32_t*>(&ov[k]);
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf) {
+                        const int j = 8 * k + 2 * e + hf;
+                        const float g = hf ? u2f(ge[e] & 0xffff0000u) : u2f(ge[e] << 16);
+                        const float o = hf ? u2f(oe[e] & 0xffff0000u) : u2f(oe[e] << 16);
+                        const float dn = o * g * sigmoidf_(g);
+                        y[j] = rstd * (dn - m1 - y[j] * m2);
+                    }
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const uint32_t* oe = reinterpret_cast<const uint32_t*>(&ov[k]);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    y[8 * k + 2 * e] = u2f(oe[e] << 16);
+                    y[8 * k + 2 * e + 1] = u2f(oe[e] & 0xffff0000u);
+                }
+            }
+        }
+        // rr_t = dy_t . (e^{b_t} q_t S_c) over this CTA's channels (Yi is still in
+        // tensor memory: G_c overwrites it only after every row warp arrived on BQT)
+        {
+            float rp = 0.f;
+            if (ok_y) {
+                uint32_t ri[32];
+#pragma unroll
+                for (int cb = 0; cb < 2; ++cb) {
+                    tmem_ld_x32(tm + lq + R_YI + 64 * half + 32 * cb, ri);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) rp = fmaf(y[32 * cb + j], u2f(ri[j]), rp);
+                }
+            }
+            rp *= ebt;
+            if (half) scr[8 * kC + t] = rp;
+            named_bar_sync(kNamedBar, kRowThreads);
+            if (!half && t < L) p.rr[(size_t)rank * p.B * p.N * p.H + (tok0 + t) * p.H + hh] = rp + scr[8 * kC + t];
+            named_bar_sync(kNamedBar, kRowThreads);   // the scratch is overwritten by dy below
+        }
+        // dy as a bf16 pair: shared-memory tiles (row t, box `half`) and the workspace
+        {
+            uint8_t* rh = sm + OFF_DYH + half * kBox;
+            uint8_t* rl = sm + OFF_DYL + half * kBox;
+            const size_t go = ((tok0 + t) * p.H + hh) * (size_t)DV + ch0 + 64 * half;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                uint4 h, l;
+                split2(y[8 * k], y[8 * k + 1], h.x, l.x);
+                split2(y[8 * k + 2], y[8 * k + 3], h.y, l.y);
+                split2(y[8 * k + 4], y[8 * k + 5], h.z, l.z);
+                split2(y[8 * k + 6], y[8 * k + 7], h.w, l.w);
+                *reinterpret_cast<uint4*>(rh + sw128(t, 8 * k)) = h;
+                *reinterpret_cast<uint4*>(rl + sw128(t, 8 * k)) = l;
+                if (t < L) {
+                    reinterpret_cast<uint4*>(p.dyh + go)[k] = h;
+                    reinterpret_cast<uint4*>(p.dyl + go)[k] = l;
+                }
+            }
+        }
+        fence_proxy_async_smem();
+        warp_arrive(BDY);
+
+        // ---------------------------------------------------- Q~^T = (diag(e^{b}) Q)^T as a bf16 pair
+        if (ok_y) {
+            const int d = 32 * q + lane;
+            const uint8_t* qb = sm + OFF_Q + (q >> 1) * kBox;
+            const int xq = 32 * (q & 1) + lane;
+            uint32_t hi[32], lo[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int t0 = 64 * half + 2 * j;
+                const float x0 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(qb + sw128(t0, xq)));
+                const float x1 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(qb + sw128(t0 + 1, xq)));
+                split2(x0 * __expf(bc[t0]), x1 * __expf(bc[t0 + 1]), hi[j], lo[j]);
+            }
+            (void)d;
+            tmem_st_x32(tm + lq + R_P + 32 * half, hi);
+            tmem_st_x32(tm + lq + R_P + 64 + 32 * half, lo);
+            tmem_wait_st();
+        }
+        tc_fence_before();
+        warp_arrive(BQT);
+
+        // ---------------------------------------------------- D o E (bf16) and e^{b_t} dy S^T
+        if (mbar_wait(bar(BD), 0, p.status, abort_flag)) {
+            tc_fence_after();
+            uint32_t r[64], pk[32];
+            tmem_ld_x32(tm + lq + R_A + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(r));
+            tmem_ld_x32(tm + lq + R_A + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int s0 = 64 * half + 2 * j;
+                const float v0 = s0 <= t ? u2f(r[2 * j]) * __expf(fminf(bt - bc[s0], 0.f)) : 0.f;
+                const float v1 = s0 + 1 <= t ? u2f(r[2 * j + 1]) * __expf(fminf(bt - bc[s0 + 1], 0.f)) : 0.f;
+                pk[j] = pack_bf16x2(v0, v1);
+            }
+            // every row warp has read D before D o E overwrites its first 64 columns
+            named_bar_sync(kNamedBar, kRowThreads);
+            tmem_st_x32(tm + lq + R_A + 32 * half, pk);
+            if (mbar_wait(bar(BQI), 0, p.status, abort_flag)) {
+                tc_fence_after();
+#pragma unroll
+                for (int cb = 0; cb < 2; ++cb) {
+                    uint32_t v[32];
+                    tmem_ld_x32(tm + lq + R_Y + 64 * half + 32 * cb, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = f2u(u2f(v[j]) * ebt);
+                    tmem_st_x32(tm + lq + R_Y + 64 * half + 32 * cb, v);
+                }
+            }
+            tmem_wait_st();
+        } else {
+            named_bar_sync(kNamedBar, kRowThreads);
+        }
+        tc_fence_before();
+        warp_arrive(BDS);
+
+        // ---------------------------------------------------- G_c rows (lane = d_k row)
+        if (mbar_wait(bar(BGC), 0, p.status, abort_flag)) {
+            tc_fence_after();
+            float* dst = p.incg + (((size_t)u * nc + c) * kDK + t) * DV + ch0 + 64 * half;
+#pragma unroll 1
+            for (int cb = 0; cb < 2; ++cb) {
+                uint32_t v[32];
+                tmem_ld_x32(tm + lq + R_YI + 64 * half + 32 * cb, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    reinterpret_cast<float4*>(dst + 32 * cb)[k] =
+                        make_float4(u2f(v[4 * k]), u2f(v[4 * k + 1]), u2f(v[4 * k + 2]), u2f(v[4 * k + 3]));
+            }
+        }
+        // ---------------------------------------------------- dq (this CTA's channel half)
+        if (mbar_wait(bar(BDQ), 0, p.status, abort_flag)) {
+            tc_fence_after();
+#pragma unroll
+            for (int cb = 0; cb < 2; ++cb) {
+                uint32_t v[32];
+                tmem_ld_x32(tm + lq + R_Y + 64 * half + 32 * cb, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) dq[32 * cb + j] = u2f(v[j]);
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 64; ++j) dq[j] = 0.f;
+        }
+    } else if (lane == 0) {
+        // ============================================================ TMA + MMA issuer
+        constexpr uint32_t id_kk = idesc_bf16(128, 128, false, false);
+        constexpr uint32_t id_kn = idesc_bf16(128, 128, false, true);
+        auto kmaj = [&](uint32_t base, int k) { return sdesc_sw128(base + (k >> 2) * kBox + (k & 3) * 32, 16, 1024); };
+        auto mnmaj = [&](uint32_t base, int k) { return sdesc_sw128(base + k * 2048, kBox, 1024); };
+        const int srow = (u * nc + c) * kDK;
+        mbar_arrive_expect_tx(bar(BQK), 2 * kTile);
+        for (int x = 0; x < 2; ++x) {
+            tma_load_4d(sb + OFF_Q + x * kBox, &p.tmQ, x * 64, hh, n0, b, bar(BQK));
+            tma_load_4d(sb + OFF_K + x * kBox, &p.tmK, x * 64, hh, n0, b, bar(BQK));
+        }
+        mbar_arrive_expect_tx(bar(BVS), 3 * kTile);
+        for (int x = 0; x < 2; ++x) {
+            tma_load_4d(sb + OFF_V + x * kBox, &p.tmV, ch0 + x * 64, hh, n0, b, bar(BVS));
+            tma_load_2d(sb + OFF_SH + x * kBox, &p.tmSH, ch0 + x * 64, srow, bar(BVS));
+            tma_load_2d(sb + OFF_SL + x * kBox, &p.tmSL, ch0 + x * 64, srow, bar(BVS));
+        }
+        bool ok = mbar_wait(bar(BQK), 0, p.status, abort_flag);
+        if (ok) {
+            tc_fence_after();
+            // scores A = Q K^T
+#pragma unroll
+            for (int k = 0; k < 8; ++k) mma_ss(tm + R_A, kmaj(sb + OFF_Q, k), kmaj(sb + OFF_K, k), id_kk, k > 0);
+        }
+        mma_commit(bar(BA));
+        ok = ok && mbar_wait(bar(BVS), 0, p.status, abort_flag);
+        if (ok) {
+            tc_fence_after();
+            // Yi = Q S_c (S as a bf16 pair)
+            for (int pass = 0; pass < 2; ++pass)
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_ss(tm + R_YI, kmaj(sb + OFF_Q, k), mnmaj(sb + (pass ? OFF_SL : OFF_SH), k), id_kn,
+                           pass > 0 || k > 0);
+        }
+        mma_commit(bar(BYI));
+        ok = ok && mbar_wait(bar(BP), 0, p.status, abort_flag);
+        if (ok) {
+            tc_fence_after();
+            // Y = P V
+#pragma unroll
+            for (int k = 0; k < 8; ++k) mma_ts(tm + R_Y, tm + R_P + k * 8, mnmaj(sb + OFF_V, k), id_kn, k > 0);
+        }
+        mma_commit(bar(BY));
+        ok = ok && mbar_wait(bar(BDY), 0, p.status, abort_flag);
+        if (ok) {
+            tc_fence_after();
+            // D = dy V^T (dy as a bf16 pair)
+            for (int pass = 0; pass < 2; ++pass)
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_ss(tm + R_A, kmaj(sb + (pass ? OFF_DYL : OFF_DYH), k), kmaj(sb + OFF_V, k), id_kk,
+                           pass > 0 || k > 0);
+        }
+        mma_commit(bar(BD));
+        if (ok) {
+            // dy S^T: hi hi + hi lo + lo hi
+            for (int pass = 0; pass < 3; ++pass)
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_ss(tm + R_Y, kmaj(sb + (pass == 2 ? OFF_DYL : OFF_DYH), k),
+                           kmaj(sb + (pass == 1 ? OFF_SL : OFF_SH), k), id_kk, pass > 0 || k > 0);
+        }
+        mma_commit(bar(BQI));
+        ok = ok && mbar_wait(bar(BQT), 0, p.status, abort_flag);
+        if (ok) {
+            tc_fence_after();
+            // G_c = Q~^T dy: A = Q~^T from tensor memory (lane = d_k row), B = dy MN-major
+            for (int pass = 0; pass < 3; ++pass)
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_ts(tm + R_YI, tm + R_P + (pass == 2 ? 64 : 0) + k * 8,
+                           mnmaj(sb + (pass == 1 ? OFF_DYL : OFF_DYH), k), id_kn, pass > 0 || k > 0);
+        }
+        mma_commit(bar(BGC));
+        ok = ok && mbar_wait(bar(BDS), 0, p.status, abort_flag);
+        if (ok) {
+            tc_fence_after();
+            // dq += (D o E) K
+#pragma unroll
+            for (int k = 0; k < 8; ++k) mma_ts(tm + R_Y, tm + R_A + k * 8, mnmaj(sb + OFF_K, k), id_kn, 1);
+        }
+        mma_commit(bar(BDQ));
+        mma_commit(bar(BDRAIN));
+        mbar_wait_drain(bar(BDRAIN), 0, kWaitCycles);
+        if (*abort_flag) {
+            mbar_wait_drain(bar(BQK), 0, kWaitCycles);
+            mbar_wait_drain(bar(BVS), 0, kWaitCycles);
+        }
+    }
+    __syncwarp();
+    // ---------------------------------------------------------------- dq rows
+    if constexpr (PAIR) cluster_sync_all();   // both CTAs are past their last MMA: the S tiles are free
+    if (tid < kRowThreads) {
+        const int q = warp & 3, half = warp >> 2, t = 32 * q + lane;
+        float* recv = reinterpret_cast<float*>(sm + OFF_SH);   // [64 rows][128] partials from the other CTA
+        bool mine = true;
+        if constexpr (PAIR) {
+            const int owner = t >> 6;
+            mine = owner == rank;
+            if (!mine) {
+                const uint32_t remote = cluster_map(smem_u32(recv + (t & 63) * 128 + 64 * half), peer);
+                const uint32_t rbar = cluster_map(bar(BXQ), peer);
+#pragma unroll
+                for (int k = 0; k < 16; ++k)
+                    st_async_f4(remote + 16 * k, rbar, dq[4 * k], dq[4 * k + 1], dq[4 * k + 2], dq[4 * k + 3]);
+            } else if (mbar_wait_cluster(bar(BXQ), 0, p.status, abort_flag)) {
+                const float* src = recv + (t & 63) * 128 + 64 * half;
+#pragma unroll
+                for (int j = 0; j < 64; ++j) dq[j] += src[j];
+            }
+        }
+        if (mine && t < L) {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dQ) + ((tok0 + t) * p.H + hh) * kDK +
+                                                  64 * half);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                dst[k] = make_uint4(pack_bf16x2(dq[8 * k], dq[8 * k + 1]), pack_bf16x2(dq[8 * k + 2], dq[8 * k + 3]),
+                                    pack_bf16x2(dq[8 * k + 4], dq[8 * k + 5]), pack_bf16x2(dq[8 * k + 6], dq[8 * k + 7]));
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if constexpr (PAIR) cluster_sync_all();   // no CTA leaves while the other still sends to it
+    if (warp == kRowThreads / 32) tmem_dealloc(tm, 512);
+}
+
+// Sum of v[0..31] over the warp's lanes for each of the 32 columns at once:
+// after the five halving steps lane l holds the sum of column l (31 shuffles).
+__device__ __forceinline__ float transpose_reduce32(float (&v)[32], int lane) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        const bool up = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < o; ++i) {
+            const float send = up ? v[i] : v[i + o];
+            const float keep = up ? v[i + o] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+    }
+    return v[0];
+}
+
+// ---- 5. per chunk: dk = (D o E)^T Q + e^{b_L - b_s} V dS'^T,
+// dv = (A o E)^T dy + e^{b_L - b_s} K dS' and the gate gradient
+//   dz_j = (F_j + sum_{t>=j} rr_t + X_c + sum_{s<j} us_s) (1 - sigmoid(z_j)) / tau
+// with F_j = sum_{s<j<=t} A_ts D_ts E_ts and us_s = e^{b_L - b_s} k_s . (dS' v_s).
+// The products are taken transposed (tensor-memory lane = key token s), so
+// that (A o E)^T and (D o E)^T serve as A operands from tensor memory.  With
+// PAIR the CTA of cluster rank h owns channels 128 h .. + 127 (the dv columns,
+// a partial dk, F and us) and rows 64 h .. 64 h + 63 of dk; rank 0 forms dz.
+//
+// Tensor memory: [0,128) A^T, then (A o E)^T (bf16); [128,256) D^T, then
+// (D o E)^T; [256,384) V dS'^T, scaled, + (D o E)^T Q; [384,512) K dS',
+// scaled, + (A o E)^T dy.  Shared tiles: Q, K, V, dy hi, dy lo, dS' hi, dS' lo.
+template <bool PAIR>
+__global__ void __launch_bounds__(kThreads, 1) bwd_kv_tc(const __grid_constant__ BwdTcParams p) {
+    using CF = GradCfg;
+    constexpr int OFF_Q = 0, OFF_K = kTile, OFF_V = 2 * kTile, OFF_DYH = 3 * kTile, OFF_DYL = 4 * kTile,
+                  OFF_DSH = 5 * kTile, OFF_DSL = 6 * kTile;
+    constexpr uint32_t R_AT = 0, R_DT = 128, R_DK = 256, R_DV = 384;
+    constexpr int BQK = 0, BVD = 1, BS = 2, BADT = 3, BINTER = 4, BROWS = 5, BOUT = 6, BXK = 7, BDRAIN = 8;
+    extern __shared__ __align__(1024) uint8_t sm[];
+    const uint32_t sb = smem_u32(sm);
+    if (sb & 1023u) {
+        if (threadIdx.x == 0) atomicExch(p.status, kDevSmemLayout);
+        return;
+    }
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int rank = PAIR ? (int)cluster_ctarank() : 0;
+    const int item = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+    const int nc = p.nc, u = item / nc, c = item - u * nc, b = u / p.H, hh = u - b * p.H;
+    const int n0 = c * kC, L = min(kC, p.N - n0);
+    const size_t tok0 = (size_t)b * p.N + n0;
+    const int DV = p.dv, ch0 = 128 * rank;
+    auto bar = [&](int i) -> uint32_t { return sb + CF::OFF_BAR + 8 * i; };
+    float* bc = reinterpret_cast<float*>(sm + CF::OFF_BC);
+    float* wsum = bc + kC;
+    float* Facc = reinterpret_cast<float*>(sm + CF::OFF_AUX);   // [128] F_j over this CTA's channels
+    float* T1 = Facc + kC;                                       // [128] scratch
+    float* ush = T1 + kC;                                        // [2][128] us_s per column half
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + CF::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + CF::OFF_MISC + 4);
+
+    if (tid == kRowThreads) {
+        for (int i = 0; i < CF::NUM_BARS; ++i) mbar_init(bar(i), i == BROWS ? kRowThreads / 32 : 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        if (PAIR) mbar_arrive_expect_tx(bar(BXK), 64 * 128 * 4);
+        tma_prefetch_desc(&p.tmQ);
+        tma_prefetch_desc(&p.tmK);
+        tma_prefetch_desc(&p.tmV);
+        tma_prefetch_desc(&p.tmDyH);
+        tma_prefetch_desc(&p.tmDyL);
+        tma_prefetch_desc(&p.tmSH);
+        tma_prefetch_desc(&p.tmSL);
+    }
+    if (warp == kRowThreads / 32) {
+        tmem_alloc(smem_u32(tmem_slot), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if constexpr (PAIR) cluster_sync_all();
+    const uint32_t tm = *tmem_slot;
+    const uint32_t peer = (uint32_t)(rank ^ 1);
+
+    float dk[64];
+    if (tid < kRowThreads) {
+        const int q = warp & 3, half = warp >> 2, s = 32 * q + lane;
+        const uint32_t lq = (uint32_t)(32 * q) << 16;
+        auto warp_arrive = [&](int i) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(i));
+        };
+        chunk_decay(p, tok0, hh, L, bc, wsum);
+        if (tid < kC) Facc[tid] = 0.f;
+        const float bs = bc[s], bL = bc[kC - 1];
+        const float ws = s < L ? __expf(bL - bs) : 0.f;
+        named_bar_sync(kNamedBar, kRowThreads);
+
+        // ---------------------------------------------------- (A o E)^T, (D o E)^T and F
+        const bool ok = mbar_wait(bar(BADT), 0, p.status, abort_flag);
+        tc_fence_after();
+        uint32_t pa[32], pd[32];
+        {
+            float m[64];
+            if (ok) {
+#pragma unroll
+                for (int cb = 0; cb < 2; ++cb) {
+                    uint32_t ra[32], rd[32];
+                    tmem_ld_x32(tm + lq + R_AT + 64 * half + 32 * cb, ra);
+                    tmem_ld_x32(tm + lq + R_DT + 64 * half + 32 * cb, rd);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        float av[2], dv2[2];
+#pragma unroll
+                        for (int hf = 0; hf < 2; ++hf) {
+                            const int jj = 32 * cb + 2 * j + hf, t = 64 * half + jj;
+                            const float e = (t >= s && t < L) ? __expf(fminf(bc[t] - bs, 0.f)) : 0.f;
+                            const float a = u2f(ra[2 * j + hf]), d = u2f(rd[2 * j + hf]);
+                            av[hf] = a * e;
+                            dv2[hf] = d * e;
+                            m[jj] = av[hf] * d;
+                        }
+                        pa[16 * cb + j] = pack_bf16x2(av[0], av[1]);
+                        pd[16 * cb + j] = pack_bf16x2(dv2[0], dv2[1]);
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 64; ++j) m[j] = 0.f;
+            }
+            // C_s(j) = sum_{t >= j} M_ts: suffix within this half, plus the second
+            // half's row total for the first half
+            float run = 0.f;
+#pragma unroll
+            for (int j = 63; j >= 0; --j) {
+                run += m[j];
+                m[j] = run;
+            }
+            if (half) T1[s] = run;
+            named_bar_sync(kNamedBar, kRowThreads);
+            const float add = half ? 0.f : T1[s];
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {
+                float v[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int j = 64 * half + 32 * g + i;   // the token j of F_j
+                    v[i] = s < j ? m[32 * g + i] + add : 0.f;
+                }
+                atomicAdd(Facc + 64 * half + 32 * g + lane, transpose_reduce32(v, lane));
+            }
+        }
+        // every row warp has read A^T and D^T before their first 64 columns are overwritten
+        named_bar_sync(kNamedBar, kRowThreads);
+        if (ok) {
+            tmem_st_x32(tm + lq + R_AT + 32 * half, pa);
+            tmem_st_x32(tm + lq + R_DT + 32 * half, pd);
+        }
+        // ---------------------------------------------------- e^{b_L - b_s} on the dS' products, us_s
+        float usp = 0.f;
+        if (mbar_wait(bar(BINTER), 0, p.status, abort_flag)) {
+            tc_fence_after();
+            const uint8_t* krow = sm + OFF_K + half * kBox;
+#pragma unroll
+            for (int cb = 0; cb < 2; ++cb) {
+                uint32_t v[32];
+                tmem_ld_x32(tm + lq + R_DK + 64 * half + 32 * cb, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint4 kw = *reinterpret_cast<const uint4*>(krow + sw128(s, 32 * cb + 8 * k));
+                    const uint32_t* ke = reinterpret_cast<const uint32_t*>(&kw);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float x0 = u2f(v[8 * k + 2 * e]) * ws, x1 = u2f(v[8 * k + 2 * e + 1]) * ws;
+                        usp = fmaf(u2f(ke[e] << 16), x0, fmaf(u2f(ke[e] & 0xffff0000u), x1, usp));
+                        v[8 * k + 2 * e] = f2u(x0);
+                        v[8 * k + 2 * e + 1] = f2u(x1);
+                    }
+                }
+                tmem_st_x32(tm + lq + R_DK + 64 * half + 32 * cb, v);
+                tmem_ld_x32(tm + lq + R_DV + 64 * half + 32 * cb, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] = f2u(u2f(v[j]) * ws);
+                tmem_st_x32(tm + lq + R_DV + 64 * half + 32 * cb, v);
+            }
+        }
+        ush[half * kC + s] = usp;
+        tmem_wait_st();
+        tc_fence_before();
+        warp_arrive(BROWS);
+
+        // ---------------------------------------------------- dv rows out, dk partial rows
+        if (mbar_wait(bar(BOUT), 0, p.status, abort_flag)) {
+            tc_fence_after();
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dV) + ((tok0 + s) * p.H + hh) * DV +
+                                                  ch0 + 64 * half);
+#pragma unroll
+            for (int cb = 0; cb < 2; ++cb) {
+                uint32_t v[32];
+                tmem_ld_x32(tm + lq + R_DV + 64 * half + 32 * cb, v);
+                tmem_wait_ld();
+                if (s < L)
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        dst[4 * cb + k] = make_uint4(pack_bf16x2(u2f(v[8 * k]), u2f(v[8 * k + 1])),
+                                                     pack_bf16x2(u2f(v[8 * k + 2]), u2f(v[8 * k + 3])),
+                                                     pack_bf16x2(u2f(v[8 * k + 4]), u2f(v[8 * k + 5])),
+                                                     pack_bf16x2(u2f(v[8 * k + 6]), u2f(v[8 * k + 7])));
+                tmem_ld_x32(tm + lq + R_DK + 64 * half + 32 * cb, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) dk[32 * cb + j] = u2f(v[j]);
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 64; ++j) dk[j] = 0.f;
+        }
+        named_bar_sync(kNamedBar, kRowThreads);   // F and us of this CTA are complete
+        if (PAIR && rank == 1 && tid < kC) {
+            float* dst = p.fus + (size_t)item * 2 * kC;
+            dst[tid] = Facc[tid];
+            dst[kC + tid] = ush[tid] + ush[kC + tid];
+            __threadfence();   // read by the other CTA after the cluster barrier
+        }
+    } else if (lane == 0) {
+        // ============================================================ TMA + MMA issuer
+        constexpr uint32_t id_kk = idesc_bf16(128, 128, false, false);
+        constexpr uint32_t id_kn = idesc_bf16(128, 128, false, true);
+        auto kmaj = [&](uint32_t base, int k) { return sdesc_sw128(base + (k >> 2) * kBox + (k & 3) * 32, 16, 1024); };
+        auto mnmaj = [&](uint32_t base, int k) { return sdesc_sw128(base + k * 2048, kBox, 1024); };
+        const int srow = (u * nc + c) * kDK;
+        mbar_arrive_expect_tx(bar(BQK), 2 * kTile);
+        for (int x = 0; x < 2; ++x) {
+            tma_load_4d(sb + OFF_Q + x * kBox, &p.tmQ, x * 64, hh, n0, b, bar(BQK));
+            tma_load_4d(sb + OFF_K + x * kBox, &p.tmK, x * 64, hh, n0, b, bar(BQK));
+        }
+        mbar_arrive_expect_tx(bar(BVD), 3 * kTile);
+        for (int x = 0; x < 2; ++x) {
+            tma_load_4d(sb + OFF_V + x * kBox, &p.tmV, ch0 + x * 64, hh, n0, b, bar(BVD));
+            tma_load_4d(sb + OFF_DYH + x * kBox, &p.tmDyH, ch0 + x * 64, hh, n0, b, bar(BVD));
+            tma_load_4d(sb + OFF_DYL + x * kBox, &p.tmDyL, ch0 + x * 64, hh, n0, b, bar(BVD));
+        }
+        mbar_arrive_expect_tx(bar(BS), 2 * kTile);
+        for (int x = 0; x < 2; ++x) {
+            tma_load_2d(sb + OFF_DSH + x * kBox, &p.tmSH, ch0 + x * 64, srow, bar(BS));
+            tma_load_2d(sb + OFF_DSL + x * kBox, &p.tmSL, ch0 + x * 64, srow, bar(BS));
+        }
+        bool ok = mbar_wait(bar(BQK), 0, p.status, abort_flag);
+        if (ok) {
+            tc_fence_after();
+            // A^T = K Q^T
+#pragma unroll
+            for (int k = 0; k < 8; ++k) mma_ss(tm + R_AT, kmaj(sb + OFF_K, k), kmaj(sb + OFF_Q, k), id_kk, k > 0);
+        }
+        ok = ok && mbar_wait(bar(BVD), 0, p.status, abort_flag);
+        if (ok) {
+            tc_fence_after();
+            // D^T = V dy^T (dy as a bf16 pair)
+            for (int pass = 0; pass < 2; ++pass)
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_ss(tm + R_DT, kmaj(sb + OFF_V, k), kmaj(sb + (pass ? OFF_DYL : OFF_DYH), k), id_kk,
+                           pass > 0 || k > 0);
+        }
+        mma_commit(bar(BADT));
+        ok = ok && mbar_wait(bar(BS), 0, p.status, abort_flag);
+        if (ok) {
+            tc_fence_after();
+            // V dS'^T and K dS' (dS' as a bf16 pair)
+            for (int pass = 0; pass < 2; ++pass)
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_ss(tm + R_DK, kmaj(sb + OFF_V, k), kmaj(sb + (pass ? OFF_DSL : OFF_DSH), k), id_kk,
+                           pass > 0 || k > 0);
+            for (int pass = 0; pass < 2; ++pass)
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_ss(tm + R_DV, kmaj(sb + OFF_K, k), mnmaj(sb + (pass ? OFF_DSL : OFF_DSH), k), id_kn,
+                           pass > 0 || k > 0);
+        }
+        mma_commit(bar(BINTER));
+        ok = ok && mbar_wait(bar(BROWS), 0, p.status, abort_flag);
+        if (ok) {
+            tc_fence_after();
+            // dk += (D o E)^T Q, dv += (A o E)^T dy
+#pragma unroll
+            for (int k = 0; k < 8; ++k) mma_ts(tm + R_DK, tm + R_DT + k * 8, mnmaj(sb + OFF_Q, k), id_kn, 1);
+            for (int pass = 0; pass < 2; ++pass)
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_ts(tm + R_DV, tm + R_AT + k * 8, mnmaj(sb + (pass ? OFF_DYL : OFF_DYH), k), id_kn, 1);
+        }
+        mma_commit(bar(BOUT));
+        mma_commit(bar(BDRAIN));
+        mbar_wait_drain(bar(BDRAIN), 0, kWaitCycles);
+        if (*abort_flag) {
+            mbar_wait_drain(bar(BQK), 0, kWaitCycles);
+            mbar_wait_drain(bar(BVD), 0, kWaitCycles);
+            mbar_wait_drain(bar(BS), 0, kWaitCycles);
+        }
+    }
+    __syncwarp();
+    if constexpr (PAIR) cluster_sync_all();   // both CTAs are past their last MMA; F and us exported
+    if (tid < kRowThreads) {
+        const int q = warp & 3, half = warp >> 2, s = 32 * q + lane;
+        // ---------------------------------------------------- dk rows
+        float* recv = reinterpret_cast<float*>(sm + OFF_DSH);   // [64 rows][128] partials from the other CTA
+        bool mine = true;
+        if constexpr (PAIR) {
+            const int owner = s >> 6;
+            mine = owner == rank;
+            if (!mine) {
+                const uint32_t remote = cluster_map(smem_u32(recv + (s & 63) * 128 + 64 * half), peer);
+                const uint32_t rbar = cluster_map(bar(BXK), peer);
+#pragma unroll
+                for (int k = 0; k < 16; ++k)
+                    st_async_f4(remote + 16 * k, rbar, dk[4 * k], dk[4 * k + 1], dk[4 * k + 2], dk[4 * k + 3]);
+            } else if (mbar_wait_cluster(bar(BXK), 0, p.status, abort_flag)) {
+                const float* src = recv + (s & 63) * 128 + 64 * half;
+#pragma unroll
+                for (int j = 0; j < 64; ++j) dk[j] += src[j];
+            }
+        }
+        if (mine && s < L) {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dK) + ((tok0 + s) * p.H + hh) * kDK +
+                                                  64 * half);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                dst[k] = make_uint4(pack_bf16x2(dk[8 * k], dk[8 * k + 1]), pack_bf16x2(dk[8 * k + 2], dk[8 * k + 3]),
+                                    pack_bf16x2(dk[8 * k + 4], dk[8 * k + 5]), pack_bf16x2(dk[8 * k + 6], dk[8 * k + 7]));
+        }
+        // ---------------------------------------------------- dz (rank 0)
+        if (rank == 0 && tid < kC) {
+            const int j = tid;
+            const float* other = PAIR ? p.fus + (size_t)item * 2 * kC : nullptr;
+            const size_t tk = (tok0 + j) * p.H + hh;
+            float F = Facc[j], us = ush[j] + ush[kC + j], rr = 0.f;
+            if (PAIR) {
+                F += other[j];
+                us += other[kC + j];
+            }
+            if (j < L) {
+                rr = p.rr[tk];
+                if (PAIR) rr += p.rr[(size_t)p.B * p.N * p.H + tk];
+            }
+            // R_j = sum_{t >= j} rr_t (suffix), U_j = sum_{s < j} us_s (exclusive prefix)
+            float R = rr, U = us;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float r2 = __shfl_down_sync(0xffffffffu, R, o);
+                const float u2 = __shfl_up_sync(0xffffffffu, U, o);
+                if (lane + o < 32) R += r2;
+                if (lane >= o) U += u2;
+            }
+            U -= us;
+            // warp totals: R of lane 0 is its warp's total, U + us of lane 31 likewise
+            float* tot = T1;   // [4] rr totals, [4] us totals (T1 is no longer needed)
+            named_bar_sync(2, kC);
+            if (lane == 0) tot[warp] = R;
+            if (lane == 31) tot[4 + warp] = U + us;
+            named_bar_sync(2, kC);
+            for (int w = warp + 1; w < 4; ++w) R += tot[w];
+            for (int w = 0; w < warp; ++w) U += tot[4 + w];
+            if (j < L) {
+                const float dlg = F + R + p.xs[(size_t)u * nc + c] + U;
+                const float zj = p.z[tk];
+                const float deriv = log_gamma(zj, p.inv_tau) > kMinLogGamma ? (1.f - sigmoidf_(zj)) * p.inv_tau : 0.f;
+                p.dz[tk] = dlg * deriv;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if constexpr (PAIR) cluster_sync_all();   // no CTA leaves while the other still sends to it
+    if (warp == kRowThreads / 32) tmem_dealloc(tm, 512);
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn_bwd() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+// bf16 tensor of `rank` dimensions (innermost first), 128-byte swizzle, box
+// (64, 1, ..., 128 at dimension `rowdim`, ...)
+bool encode_bf16(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint32_t* box) {
+    EncodeTiledFn fn = encode_fn_bwd();
+    if (!fn) return false;
+    cuuint64_t strides[4];
+    cuuint64_t st = 2;
+    for (int i = 0; i + 1 < rank; ++i) {
+        st *= dims[i];
+        strides[i] = st;
+    }
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [B][N][H][d] viewed as (d, H, N, B), box (64, 1, 128, 1)
+bool map_tokens(CUtensorMap* m, const void* base, int d, int H, int N, int B) {
+    const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
+    const cuuint32_t box[4] = {64, 1, (cuuint32_t)kC, 1};
+    return encode_bf16(m, base, 4, dims, box);
+}
+
+// per-chunk states [rows][dv] (rows = units * nc * 128), box (64, 128)
+bool map_states(CUtensorMap* m, const void* base, int dv, size_t rows) {
+    const cuuint64_t dims[2] = {(cuuint64_t)dv, (cuuint64_t)rows};
+    const cuuint32_t box[2] = {64, 128};
+    return encode_bf16(m, base, 2, dims, box);
+}
+
+size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct BwdTcWs {
+    size_t incg, sh, sl, dyh, dyl, rr, xs, decay, fus, total;
+};
+
+BwdTcWs bwd_tc_ws(int B, int H, int N, int dv) {
+    const size_t units = (size_t)B * H, nc = (size_t)(N + kC - 1) / kC, E = (size_t)kDK * dv;
+    const size_t tok = (size_t)B * N * H;
+    BwdTcWs w;
+    size_t o = 0;
+    w.incg = o; o += a256(units * nc * E * 4);
+    w.sh = o; o += a256(units * nc * E * 2);
+    w.sl = o; o += a256(units * nc * E * 2);
+    w.dyh = o; o += a256(tok * dv * 2);
+    w.dyl = o; o += a256(tok * dv * 2);
+    w.rr = o; o += a256(2 * tok * 4);
+    w.xs = o; o += a256(units * nc * 4);
+    w.decay = o; o += a256(units * nc * 4);
+    w.fus = o; o += a256(units * nc * 2 * kC * 4);
+    w.total = o;
+    return w;
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_cluster(void (*kernel)(KArgs...), unsigned grid, int cluster, size_t smem, cudaStream_t s,
+                           Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = cluster > 1 ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+template <int DV>
+cudaError_t run_bwd_tc(BwdTcParams& p, cudaStream_t s) {
+    constexpr bool PAIR = DV == 256;
+    const unsigned items = (unsigned)((size_t)p.B * p.H * p.nc);
+    auto k1 = bwd_inc_tc<DV>;
+    auto k3 = bwd_dyq_tc<PAIR>;
+    auto k5 = bwd_kv_tc<PAIR>;
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, IncCfg<DV>::SMEM)) != cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(k3, cudaFuncAttributeMaxDynamicSharedMemorySize, GradCfg::SMEM)) != cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(k5, cudaFuncAttributeMaxDynamicSharedMemorySize, GradCfg::SMEM)) != cudaSuccess)
+        return e;
+    const dim3 sgrid((unsigned)((kDK * DV / 4 + kScanThreads - 1) / kScanThreads), (unsigned)(p.B * p.H));
+    k1<<<items, kThreads, IncCfg<DV>::SMEM, s>>>(p);
+    bwd_scan_fwd<<<sgrid, kScanThreads, 0, s>>>(p);
+    if ((e = launch_cluster(k3, items * (PAIR ? 2 : 1), PAIR ? 2 : 1, GradCfg::SMEM, s, p)) != cudaSuccess) return e;
+    bwd_scan_rev<<<sgrid, kScanThreads, 0, s>>>(p);
+    if ((e = launch_cluster(k5, items * (PAIR ? 2 : 1), PAIR ? 2 : 1, GradCfg::SMEM, s, p)) != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool bwd_tc_supported(int B, int H, int N, int dk, int dv, gret_dtype io) {
+    if (io != GRET_BF16 || dk != kDK || (dv != 128 && dv != 256) || B <= 0 || H <= 0 || N <= 0) return false;
+    const long long items = (long long)B * H * ((N + kC - 1) / kC);
+    // the per-chunk state rows address a 2-D tensor map (rows < 2^31) and
+    // the grids one CTA (pair) per chunk
+    return items * kDK < (1LL << 31) && items * 2 < (1LL << 31);
+}
+
+size_t bwd_tc_workspace_bytes(int B, int H, int N, int dv) { return bwd_tc_ws(B, H, N, dv).total; }
+
+cudaError_t launch_bwd_tc(const BackwardArgs& in, cudaStream_t s) {
+    BwdTcParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.Q = in.Q; p.K = in.K; p.V = in.V; p.G = in.G; p.dO = in.dO;
+    p.z = in.z; p.S0 = in.S0; p.dS_final = in.dS_final;
+    p.dQ = in.dQ; p.dK = in.dK; p.dV = in.dV; p.dG = in.dG; p.dz = in.dz; p.dS0 = in.dS0;
+    p.status = in.status;
+    p.B = in.B; p.H = in.H; p.N = in.N; p.dv = in.dv; p.nc = (in.N + kC - 1) / kC;
+    p.inv_tau = in.inv_tau; p.eps = in.eps; p.gn = in.gn;
+    const BwdTcWs w = bwd_tc_ws(in.B, in.H, in.N, in.dv);
+    uint8_t* ws = static_cast<uint8_t*>(in.workspace);
+    p.incg = reinterpret_cast<float*>(ws + w.incg);
+    p.sh = reinterpret_cast<__nv_bfloat16*>(ws + w.sh);
+    p.sl = reinterpret_cast<__nv_bfloat16*>(ws + w.sl);
+    p.dyh = reinterpret_cast<__nv_bfloat16*>(ws + w.dyh);
+    p.dyl = reinterpret_cast<__nv_bfloat16*>(ws + w.dyl);
+    p.rr = reinterpret_cast<float*>(ws + w.rr);
+    p.xs = reinterpret_cast<float*>(ws + w.xs);
+    p.decay = reinterpret_cast<float*>(ws + w.decay);
+    p.fus = reinterpret_cast<float*>(ws + w.fus);
+    const size_t srows = (size_t)in.B * in.H * p.nc * kDK;
+    if (!map_tokens(&p.tmQ, in.Q, kDK, in.H, in.N, in.B) || !map_tokens(&p.tmK, in.K, kDK, in.H, in.N, in.B) ||
+        !map_tokens(&p.tmV, in.V, in.dv, in.H, in.N, in.B) || !map_tokens(&p.tmDyH, p.dyh, in.dv, in.H, in.N, in.B) ||
+        !map_tokens(&p.tmDyL, p.dyl, in.dv, in.H, in.N, in.B) || !map_states(&p.tmSH, p.sh, in.dv, srows) ||
+        !map_states(&p.tmSL, p.sl, in.dv, srows))
+        return cudaErrorInvalidValue;
+    return in.dv == 256 ? run_bwd_tc<256>(p, s) : run_bwd_tc<128>(p, s);
+}
+
+}  // namespace gret

@@ -152,6 +152,7 @@ struct BackwardArgs {
     float inv_tau, eps;
     int gn;
     gret_dtype io;
+    unsigned int* status;     // device status word (tensor-core path)
 };
 size_t prefill_backward_workspace_bytes(int B, int H, int N, int dk, int dv, gret_dtype io);
 bool prefill_backward_supported(int dk, int dv);
@@ -163,6 +164,10 @@ cudaError_t launch_prefill_backward(const BackwardArgs& a, cudaStream_t s);
 bool bwd_chunked_supported(int B, int H, int N, int dk, int dv, gret_dtype io);
 size_t bwd_chunked_workspace_bytes(int B, int H, int N, int dk, int dv, gret_dtype io);
 cudaError_t launch_bwd_chunked(const BackwardArgs& a, cudaStream_t s);
+// tensor-core backward (gret_backward_tc.cu): bf16, dk = 128, dv of 128 or 256
+bool bwd_tc_supported(int B, int H, int N, int dk, int dv, gret_dtype io);
+size_t bwd_tc_workspace_bytes(int B, int H, int N, int dv);
+cudaError_t launch_bwd_tc(const BackwardArgs& a, cudaStream_t s);
 // state-only pass of the tensor-core path (a.state_only): workspace bytes and launch
 size_t prefill_tc_state_workspace_bytes(int B, int H, int N, int dk, int dv, int chunk, int num_sms);
 int prefill_tc_state_pieces(int B, int H, int chunk, int num_sms, int segments, int seg_len);

@@ -135,6 +135,19 @@ __device__ __forceinline__ void st_async_f2(uint32_t remote, uint32_t remote_bar
                  : "memory");
 }
 
+// The same for one float and for four (16-byte aligned) floats.
+__device__ __forceinline__ void st_async_f1(uint32_t remote, uint32_t remote_bar, float x) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.f32 [%0], %1, [%2];" ::"r"(remote), "f"(x),
+                 "r"(remote_bar)
+                 : "memory");
+}
+__device__ __forceinline__ void st_async_f4(uint32_t remote, uint32_t remote_bar, float x, float y, float z, float w) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                     remote),
+                 "f"(x), "f"(y), "f"(z), "f"(w), "r"(remote_bar)
+                 : "memory");
+}
+
 // Arrive on an mbarrier in another CTA of the cluster without ordering any
 // memory access (a signal whose data dependences are already resolved).
 __device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t remote_bar) {

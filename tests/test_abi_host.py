@@ -126,10 +126,14 @@ def test_path_selection(lib):
 def test_backward_path_and_workspace(lib):
     bf, f32 = gret.Dtype.BF16, gret.Dtype.F32
     E = 128 * 256
-    # chunk-parallel path: chunks of 64 tokens (bf16) or 32 (fp32); two states per
-    # chunk, the fp32 gradient of the pre-norm output and one decay per chunk
+    # tensor-core path (bf16, d_k 128): chunks of 128 tokens; per chunk an fp32
+    # state-shaped buffer (increments, then G_c) and a state as a bf16 pair
+    # (S_c, then dS'_c); dy as a bf16 pair; per token the two channel halves'
+    # inter-chunk terms; per chunk X_c, e^{b_L} and a pair's F/us partials
     assert gret.gret_prefill_backward_launches(4, 16, 4096, 128, 256, bf) == 5
-    want = 2 * (64 * 64 * E * 4) + 4 * 4096 * 16 * 256 * 4 + 64 * 64 * 4
+    units, nc128, tok = 64, 32, 4 * 4096 * 16
+    want = (units * nc128 * E * 4 + 2 * units * nc128 * E * 2 + 2 * tok * 256 * 2 + 2 * tok * 4 + units * nc128 * 4
+            + units * nc128 * 4 + units * nc128 * 256 * 4)
     assert gret.gret_prefill_backward_workspace_size(4, 16, 4096, 128, 256, bf) == want
     nc = (100 + 31) // 32
     assert gret.gret_prefill_backward_launches(1, 2, 100, 64, 64, f32) == 5
