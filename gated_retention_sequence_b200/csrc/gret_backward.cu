@@ -359,7 +359,8 @@ size_t prefill_backward_workspace_bytes(int B, int H, int N, int dk, int dv, gre
 bool prefill_backward_supported(int dk, int dv) { return bwd_block_smem(dk, dv) <= 227 * 1024; }
 
 int prefill_backward_launches(int B, int H, int N, int dk, int dv, gret_dtype io) {
-    return bwd_tc_supported(B, H, N, dk, dv, io) || bwd_chunked_supported(B, H, N, dk, dv, io) ? 5 : 2;
+    if (bwd_tc_supported(B, H, N, dk, dv, io)) return 6;
+    return bwd_chunked_supported(B, H, N, dk, dv, io) ? 5 : 2;
 }
 
 cudaError_t launch_prefill_backward(const BackwardArgs& in, cudaStream_t s) {

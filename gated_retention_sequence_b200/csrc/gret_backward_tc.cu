@@ -22,13 +22,14 @@
 // (the final state's gradient enters through dS' of the last chunk).
 //
 // Five launches:
-//   1. bwd_inc_tc      per chunk: e^{b_L} and the increment K~^T V (tcgen05)
+//   1. bwd_inc_tc      per chunk and channel half: e^{b_L} and the increment
+//                      K~^T V (tcgen05)
 //   2. bwd_scan_fwd    per state element: S_c of every chunk as a bf16 pair
 //                      (hi = bf16(S), lo = bf16(S - hi))
 //   3. bwd_dyq_tc      per chunk: y, the GroupNorm * swish backward (dG, dy),
 //                      G_c = sum_t e^{b_t} q_t^T dy_t and dq (tcgen05)
-//   4. bwd_scan_rev    per state element: dS'_c as a bf16 pair, dS0 and
-//                      e^{b_L} <dS'_c, S_c>
+//   4. bwd_scan_rev    per state element: dS'_c as a bf16 pair, dS0 and the
+//                      shares of e^{b_L} <dS'_c, S_c>
 //   5. bwd_kv_tc       per chunk: dk, dv and dz (tcgen05)
 // The products whose operands are not bf16 inputs take them as bf16 pairs:
 // a product with one such operand costs two MMAs (x_hi, x_lo), with two of
@@ -74,9 +75,9 @@ struct BwdTcParams {
     __nv_bfloat16* dyh;       // [B][N][H][dv] dy hi
     __nv_bfloat16* dyl;       // dy lo
     float* rr;                // [2][B][N][H] per channel half: dy_t . (e^{b_t} q_t S_c)
-    float* xs;                // [units][nc] e^{b_L} <dS'_c, S_c>
+    float* xs;                // [units][nc][dv]: e^{b_L} <dS'_c, S_c> in shares of 128 elements
     float* decay;             // [units][nc] e^{b_L}
-    float* fus;               // [units][nc][256]: F and us partials of a pair's second CTA
+    float* fus;               // [units][nc][2][256]: F and us per channel half
     unsigned int* status;
     int B, H, N, dv, nc;
     float inv_tau, eps;
@@ -84,6 +85,19 @@ struct BwdTcParams {
 };
 
 __device__ __forceinline__ float u2f(uint32_t x) { return __uint_as_float(x); }
+
+// logistic sigmoid with the fast exponential and divide (a few ulp)
+__device__ __forceinline__ float sigmoid_fast(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
+
+// 16-byte global load through the non-coherent path, issued where it is written
+// (volatile), for data read once well after it is requested
+__device__ __forceinline__ uint4 ldg_nc_v4(const uint4* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
 __device__ __forceinline__ uint32_t f2u(float x) { return __float_as_uint(x); }
 
 // bf16 pair of x: hi = bf16(x), lo = bf16(x - hi)
@@ -103,8 +117,9 @@ __device__ __forceinline__ uint32_t sw128(int r, int x) {
 }
 
 // Chunk-local decay sums b_t of the chunk's tokens (0 past L: b_t = b_{L-1})
-// into bc[0..127], and e^{b_L} on request; threads 0..127 of the row warps
-// take part (warps 0-3), the row warps sync after.
+// into bc[0..127]; threads 0..127 of the NRT row threads compute them, all
+// row threads sync after.
+template <int NRT = kRowThreads>
 __device__ __forceinline__ void chunk_decay(const BwdTcParams& p, size_t tok0, int hh, int L, float* bc, float* wsum) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     if (tid < kC) {
@@ -117,38 +132,38 @@ __device__ __forceinline__ void chunk_decay(const BwdTcParams& p, size_t tok0, i
         if (lane == 31) wsum[warp] = x;
         bc[tid] = x;
     }
-    named_bar_sync(kNamedBar, kRowThreads);
+    named_bar_sync(kNamedBar, NRT);
     if (tid < kC) {
         float add = 0.f;
         for (int w = 0; w < warp; ++w) add += wsum[w];
         bc[tid] += add;
     }
-    named_bar_sync(kNamedBar, kRowThreads);
+    named_bar_sync(kNamedBar, NRT);
 }
 
-// ---- 1. per chunk: e^{b_L} and inc_c = sum_s e^{b_L - b_s} k_s^T v_s into
-// slot c of incg ([d][j] fp32).  K~ = diag(e^{b_L - b}) K is formed in shared
-// memory as a bf16 pair; the MMA is D[d][j] = K~^T V (A = K~ MN-major,
-// B = V MN-major), two passes.
-template <int DV>
+// ---- 1. per chunk and 128-channel half of d_v: e^{b_L} and the increment
+// inc_c = sum_s e^{b_L - b_s} k_s^T v_s into slot c of incg ([d][j] fp32).
+// K~ = diag(e^{b_L - b}) K is formed in shared memory as a bf16 pair; the MMA
+// is D[d][j] = K~^T V (A = K~ MN-major, B = V MN-major), two passes.  96 KB of
+// shared memory and 128 tensor-memory columns: two CTAs share an SM.
 struct IncCfg {
     static constexpr int OFF_K = 0;                    // K~ hi (in place of K)
     static constexpr int OFF_KL = kTile;               // K~ lo
-    static constexpr int OFF_V = 2 * kTile;            // DV / 64 boxes
-    static constexpr int OFF_BC = OFF_V + DV / 64 * kBox;
+    static constexpr int OFF_V = 2 * kTile;            // 128 channels of V
+    static constexpr int OFF_BC = 3 * kTile;
     static constexpr int OFF_BAR = OFF_BC + kC * 4 + 64;
     static constexpr int OFF_MISC = OFF_BAR + 64;
     static constexpr int SMEM = OFF_MISC + 64 + 1024;  // + alignment slack
 };
 
-template <int DV>
-__global__ void __launch_bounds__(kThreads, 1) bwd_inc_tc(const __grid_constant__ BwdTcParams p) {
-    using CF = IncCfg<DV>;
+__global__ void __launch_bounds__(kThreads, 2) bwd_inc_tc(const __grid_constant__ BwdTcParams p) {
+    using CF = IncCfg;
     extern __shared__ uint8_t smraw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int nc = p.nc, u = blockIdx.x / nc, c = blockIdx.x - u * nc, b = u / p.H, hh = u - b * p.H;
+    const int halves = p.dv / 128, item = blockIdx.x / halves, ch0 = 128 * (blockIdx.x - item * halves);
+    const int nc = p.nc, u = item / nc, c = item - u * nc, b = u / p.H, hh = u - b * p.H;
     const int n0 = c * kC, L = min(kC, p.N - n0);
     const size_t tok0 = (size_t)b * p.N + n0;
     const bool need = c + 1 < nc;   // the last chunk's increment is never used
@@ -164,15 +179,15 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_inc_tc(const __grid_constant_
         *abort_flag = 0;
         fence_mbar_init();
         if (need) {
-            mbar_arrive_expect_tx(bar_ld, kTile + DV / 64 * kBox);
-            for (int x = 0; x < 2; ++x)
+            mbar_arrive_expect_tx(bar_ld, 2 * kTile);
+            for (int x = 0; x < 2; ++x) {
                 tma_load_4d(sb + CF::OFF_K + x * kBox, &p.tmK, x * 64, hh, n0, b, bar_ld);
-            for (int x = 0; x < DV / 64; ++x)
-                tma_load_4d(sb + CF::OFF_V + x * kBox, &p.tmV, x * 64, hh, n0, b, bar_ld);
+                tma_load_4d(sb + CF::OFF_V + x * kBox, &p.tmV, ch0 + x * 64, hh, n0, b, bar_ld);
+            }
         }
     }
     if (warp == kRowThreads / 32) {
-        tmem_alloc(smem_u32(tmem_slot), DV);
+        tmem_alloc(smem_u32(tmem_slot), 128);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -183,10 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_inc_tc(const __grid_constant_
     if (tid < kRowThreads) {
         chunk_decay(p, tok0, hh, L, bc, wsum);
         const float bL = bc[kC - 1];
-        if (tid == 0) {
-            p.decay[(size_t)u * nc + c] = __expf(bL);
-            p.xs[(size_t)u * nc + c] = 0.f;   // the reverse scan accumulates here
-        }
+        if (tid == 0 && ch0 == 0) p.decay[(size_t)u * nc + c] = __expf(bL);
         // K~ = e^{b_L - b_s} k_s as a bf16 pair: row s, 64 columns per thread
         const int s = tid & 127, xb = tid >> 7;
         const float w = s < L ? __expf(bL - bc[s]) : 0.f;
@@ -211,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_inc_tc(const __grid_constant_
         if (lane == 0) mbar_arrive(bar_rdy);
     } else if (lane == 0) {
         // ============================================================ MMA issuer
-        constexpr uint32_t id = idesc_bf16(128, DV, true, true);
+        constexpr uint32_t id = idesc_bf16(128, 128, true, true);
         if (mbar_wait(bar_rdy, 0, p.status, abort_flag) && need) {
             tc_fence_after();
             for (int pass = 0; pass < 2; ++pass) {
@@ -224,16 +236,16 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_inc_tc(const __grid_constant_
         }
         mma_commit(bar_mma);
     }
-    // store: row d of the increment (TMEM lane d), DV / 2 columns per thread
+    // store: row d of the increment (TMEM lane d), 64 columns per thread
     if (tid < kRowThreads) {
         const int q = warp & 3, half = warp >> 2, d = 32 * q + lane;
         if (mbar_wait(bar_mma, 0, p.status, abort_flag) && need) {
             tc_fence_after();
-            float* dst = p.incg + (((size_t)u * nc + c) * kDK + d) * DV + half * (DV / 2);
+            float* dst = p.incg + (((size_t)u * nc + c) * kDK + d) * p.dv + ch0 + 64 * half;
 #pragma unroll 1
-            for (int cb = 0; cb < DV / 64; ++cb) {
+            for (int cb = 0; cb < 2; ++cb) {
                 uint32_t r[32];
-                tmem_ld_x32(tm + ((uint32_t)(32 * q) << 16) + half * (DV / 2) + cb * 32, r);
+                tmem_ld_x32(tm + ((uint32_t)(32 * q) << 16) + 64 * half + cb * 32, r);
                 tmem_wait_ld();
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
@@ -247,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_inc_tc(const __grid_constant_
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == kRowThreads / 32) tmem_dealloc(tm, DV);
+    if (warp == kRowThreads / 32) tmem_dealloc(tm, 128);
 }
 
 // ---- 2. per state element (4 per thread): S_0 = S0 (or 0), S_{c+1} =
@@ -284,58 +296,54 @@ __global__ void __launch_bounds__(kScanThreads) bwd_scan_fwd(const __grid_consta
 }
 
 // ---- 4. per state element, from the last chunk back: cur = dS_final (or 0);
-// for c = nc-1 .. 0: X_c += e^{b_L} <cur, S_c> (S_c from its bf16 pair, read
-// before it is overwritten), slot c <- cur as a bf16 pair, cur = e^{b_L} cur
-// + G_c; dS0 = cur
+// for c = nc-1 .. 0: slot c <- cur as a bf16 pair (S_c is read from the slot
+// first), cur = e^{b_L} cur + G_c; dS0 = cur.  Each warp also writes its
+// 128 elements' share of e^{b_L} <cur, S_c> to xs[u][c][warp]; the dk/dv
+// kernel adds a chunk's d_v shares.
 __global__ void __launch_bounds__(kScanThreads) bwd_scan_rev(const __grid_constant__ BwdTcParams p) {
-    __shared__ float red[kScanThreads / 32];
-    const size_t E4 = (size_t)kDK * p.dv / 4;
+    const size_t E4 = (size_t)kDK * p.dv / 4, W = E4 / 32;
     const int nc = p.nc;
     const size_t u = blockIdx.y, e4 = (size_t)blockIdx.x * kScanThreads + threadIdx.x;
-    const bool on = e4 < E4;
+    if (e4 >= E4) return;
     const float4* gc = reinterpret_cast<const float4*>(p.incg) + u * nc * E4 + e4;
     uint2* hi = reinterpret_cast<uint2*>(p.sh) + u * nc * E4 + e4;
     uint2* lo = reinterpret_cast<uint2*>(p.sl) + u * nc * E4 + e4;
+    float* xw = p.xs + u * nc * W + (e4 >> 5);
     const float* dec = p.decay + u * nc;
     float4 cur = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (on && p.dS_final) cur = reinterpret_cast<const float4*>(p.dS_final)[u * E4 + e4];
+    if (p.dS_final) cur = reinterpret_cast<const float4*>(p.dS_final)[u * E4 + e4];
+    float4 gn = gc[(size_t)(nc - 1) * E4];
+    uint2 hn = hi[(size_t)(nc - 1) * E4], ln = lo[(size_t)(nc - 1) * E4];
     for (int c = nc - 1; c >= 0; --c) {
-        float acc = 0.f;
-        float4 g = make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 g = gn;
+        const uint2 h = hn, l = ln;
+        if (c > 0) {
+            gn = gc[(size_t)(c - 1) * E4];
+            hn = hi[(size_t)(c - 1) * E4];
+            ln = lo[(size_t)(c - 1) * E4];
+        }
         const float e = dec[c];
-        if (on) {
-            g = gc[(size_t)c * E4];
-            const uint2 h = hi[(size_t)c * E4], l = lo[(size_t)c * E4];
-            const float s0 = u2f(h.x << 16) + u2f(l.x << 16), s1 = u2f(h.x & 0xffff0000u) + u2f(l.x & 0xffff0000u);
-            const float s2 = u2f(h.y << 16) + u2f(l.y << 16), s3 = u2f(h.y & 0xffff0000u) + u2f(l.y & 0xffff0000u);
-            acc = e * (cur.x * s0 + cur.y * s1 + cur.z * s2 + cur.w * s3);
-            uint2 nh, nl;
-            split2(cur.x, cur.y, nh.x, nl.x);
-            split2(cur.z, cur.w, nh.y, nl.y);
-            hi[(size_t)c * E4] = nh;
-            lo[(size_t)c * E4] = nl;
-            cur.x = fmaf(e, cur.x, g.x);
-            cur.y = fmaf(e, cur.y, g.y);
-            cur.z = fmaf(e, cur.z, g.z);
-            cur.w = fmaf(e, cur.w, g.w);
-        }
+        const float s0 = u2f(h.x << 16) + u2f(l.x << 16), s1 = u2f(h.x & 0xffff0000u) + u2f(l.x & 0xffff0000u);
+        const float s2 = u2f(h.y << 16) + u2f(l.y << 16), s3 = u2f(h.y & 0xffff0000u) + u2f(l.y & 0xffff0000u);
+        float acc = e * (cur.x * s0 + cur.y * s1 + cur.z * s2 + cur.w * s3);
+        uint2 nh, nl;
+        split2(cur.x, cur.y, nh.x, nl.x);
+        split2(cur.z, cur.w, nh.y, nl.y);
+        hi[(size_t)c * E4] = nh;
+        lo[(size_t)c * E4] = nl;
+        cur.x = fmaf(e, cur.x, g.x);
+        cur.y = fmaf(e, cur.y, g.y);
+        cur.z = fmaf(e, cur.z, g.z);
+        cur.w = fmaf(e, cur.w, g.w);
         acc = warp_sum(acc);
-        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            float t = 0.f;
-            for (int w = 0; w < kScanThreads / 32; ++w) t += red[w];
-            atomicAdd(p.xs + u * nc + c, t);
-        }
-        __syncthreads();
+        if ((threadIdx.x & 31) == 0) xw[(size_t)c * W] = acc;
     }
-    if (on && p.dS0) reinterpret_cast<float4*>(p.dS0)[u * E4 + e4] = cur;
+    if (p.dS0) reinterpret_cast<float4*>(p.dS0)[u * E4 + e4] = cur;
 }
 
 // Shared-memory layout of the two per-chunk gradient kernels: seven
 // [128][128] bf16 tiles (two 64-column swizzled boxes each), then small arrays.
 struct GradCfg {
-    static constexpr int OFF_T0 = 0;
     static constexpr int OFF_BC = 7 * kTile;          // b_t [128], 4 warp sums
     static constexpr int OFF_AUX = OFF_BC + 528;      // 2 KB: exchange buffers / row sums
     static constexpr int NUM_BARS = 18;
@@ -404,6 +412,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dyq_tc(const __grid_constant_
         tma_prefetch_desc(&p.tmV);
         tma_prefetch_desc(&p.tmSH);
         tma_prefetch_desc(&p.tmSL);
+        tma_prefetch_desc(&p.tmDyH);
+        tma_prefetch_desc(&p.tmDyL);
     }
     if (warp == kRowThreads / 32) {
         tmem_alloc(smem_u32(tmem_slot), 512);
@@ -424,6 +434,25 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dyq_tc(const __grid_constant_
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(i));
         };
+        // G and dO of this thread's row and 64 channels, requested now (volatile
+        // loads stay where they are written) and used by the GroupNorm backward
+        const size_t rowoff = ((tok0 + t) * p.H + hh) * (size_t)DV + ch0 + 64 * half;
+        uint4 gv[8], ov[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            ov[k] = make_uint4(0u, 0u, 0u, 0u);
+            gv[k] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        if (t < L) {
+            const uint4* og = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.dO) + rowoff);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) ov[k] = ldg_nc_v4(og + k);
+            if (p.gn) {
+                const uint4* gg = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.G) + rowoff);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) gv[k] = ldg_nc_v4(gg + k);
+            }
+        }
         chunk_decay(p, tok0, hh, L, bc, wsum);
         const float bt = bc[t], ebt = __expf(bt);
 
@@ -450,15 +479,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dyq_tc(const __grid_constant_
         warp_arrive(BP);
 
         // ---------------------------------------------------- GroupNorm * swish backward
-        const size_t rowoff = ((tok0 + t) * p.H + hh) * (size_t)DV + ch0 + 64 * half;
-        uint4 gv[8], ov[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            ov[k] = t < L ? reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.dO) + rowoff)[k]
-                          : make_uint4(0u, 0u, 0u, 0u);
-            gv[k] = (t < L && p.gn) ? reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.G) + rowoff)[k]
-                                    : make_uint4(0u, 0u, 0u, 0u);
-        }
         // sum over the row's d_v channels of (a, b): the two column-half warps
         // through `scr`, the pair through distributed shared memory
         auto row_sum = [&](int slot, int xbar, float a, float bv, bool two, float& ra, float& rb) {
@@ -541,7 +561,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dyq_tc(const __grid_constant_
                         const int j = 8 * k + 2 * e + hf;
                         const float g = hf ? u2f(ge[e] & 0xffff0000u) : u2f(ge[e] << 16);
                         const float o = hf ? u2f(oe[e] & 0xffff0000u) : u2f(oe[e] << 16);
-                        const float sg = sigmoidf_(g);
+                        const float sg = sigmoid_fast(g);
                         const float n = y[j] * rstd;
                         y[j] = n;
                         // d/dg [g sigmoid(g)] = sigmoid(g) (1 + g (1 - sigmoid(g)))
@@ -568,7 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dyq_tc(const __grid_constant_
                         const int j = 8 * k + 2 * e + hf;
                         const float g = hf ? u2f(ge[e] & 0xffff0000u) : u2f(ge[e] << 16);
                         const float o = hf ? u2f(oe[e] & 0xffff0000u) : u2f(oe[e] << 16);
-                        const float dn = o * g * sigmoidf_(g);
+                        const float dn = o * g * sigmoid_fast(g);
                         y[j] = rstd * (dn - m1 - y[j] * m2);
                     }
             }
@@ -603,11 +623,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dyq_tc(const __grid_constant_
             if (!half && t < L) p.rr[(size_t)rank * p.B * p.N * p.H + (tok0 + t) * p.H + hh] = rp + scr[8 * kC + t];
             named_bar_sync(kNamedBar, kRowThreads);   // the scratch is overwritten by dy below
         }
-        // dy as a bf16 pair: shared-memory tiles (row t, box `half`) and the workspace
+        // dy as a bf16 pair into the shared-memory tiles (row t, box `half`); the
+        // issuer stores the tiles to the workspace
         {
             uint8_t* rh = sm + OFF_DYH + half * kBox;
             uint8_t* rl = sm + OFF_DYL + half * kBox;
-            const size_t go = ((tok0 + t) * p.H + hh) * (size_t)DV + ch0 + 64 * half;
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
                 uint4 h, l;
@@ -617,10 +637,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dyq_tc(const __grid_constant_
                 split2(y[8 * k + 6], y[8 * k + 7], h.w, l.w);
                 *reinterpret_cast<uint4*>(rh + sw128(t, 8 * k)) = h;
                 *reinterpret_cast<uint4*>(rl + sw128(t, 8 * k)) = l;
-                if (t < L) {
-                    reinterpret_cast<uint4*>(p.dyh + go)[k] = h;
-                    reinterpret_cast<uint4*>(p.dyl + go)[k] = l;
-                }
             }
         }
         fence_proxy_async_smem();
@@ -760,6 +776,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dyq_tc(const __grid_constant_
         mma_commit(bar(BY));
         ok = ok && mbar_wait(bar(BDY), 0, p.status, abort_flag);
         if (ok) {
+            // dy (both halves of the pair) to the workspace; rows past the end of the
+            // sequence fall outside the tensor map and are not written
+            for (int x = 0; x < 2; ++x) {
+                tma_store_4d(&p.tmDyH, sb + OFF_DYH + x * kBox, ch0 + x * 64, hh, n0, b);
+                tma_store_4d(&p.tmDyL, sb + OFF_DYL + x * kBox, ch0 + x * 64, hh, n0, b);
+            }
+            bulk_commit();
             tc_fence_after();
             // D = dy V^T (dy as a bf16 pair)
             for (int pass = 0; pass < 2; ++pass)
@@ -799,6 +822,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dyq_tc(const __grid_constant_
         mma_commit(bar(BDQ));
         mma_commit(bar(BDRAIN));
         mbar_wait_drain(bar(BDRAIN), 0, kWaitCycles);
+        bulk_wait<0>();   // the dy tiles are read before the CTA leaves
         if (*abort_flag) {
             mbar_wait_drain(bar(BQK), 0, kWaitCycles);
             mbar_wait_drain(bar(BVS), 0, kWaitCycles);
@@ -865,17 +889,26 @@ __device__ __forceinline__ float transpose_reduce32(float (&v)[32], int lane) {
 // that (A o E)^T and (D o E)^T serve as A operands from tensor memory.  With
 // PAIR the CTA of cluster rank h owns channels 128 h .. + 127 (the dv columns,
 // a partial dk, F and us) and rows 64 h .. 64 h + 63 of dk; rank 0 forms dz.
+// Persistent: a CTA (pair) takes chunks cid, cid + ncl, ...; the issuer loads
+// the next chunk's tiles as the current one releases them (V after its last
+// product, K after the rows' last read, Q and dy after the last products, dS'
+// after the dk exchange, whose buffer is the dS' lo tile).
 //
 // Tensor memory: [0,128) A^T, then (A o E)^T (bf16); [128,256) D^T, then
 // (D o E)^T; [256,384) V dS'^T, scaled, + (D o E)^T Q; [384,512) K dS',
 // scaled, + (A o E)^T dy.  Shared tiles: Q, K, V, dy hi, dy lo, dS' hi, dS' lo.
+constexpr int kRowThreads16 = 512;   // sixteen row warps: lane quarter q = w & 3, column quarter w >> 2
+constexpr int kThreads16 = kRowThreads16 + 32;
+
 template <bool PAIR>
-__global__ void __launch_bounds__(kThreads, 1) bwd_kv_tc(const __grid_constant__ BwdTcParams p) {
+__global__ void __launch_bounds__(kThreads16, 1) bwd_kv_tc(const __grid_constant__ BwdTcParams p) {
     using CF = GradCfg;
+    constexpr int RT = kRowThreads16;
     constexpr int OFF_Q = 0, OFF_K = kTile, OFF_V = 2 * kTile, OFF_DYH = 3 * kTile, OFF_DYL = 4 * kTile,
                   OFF_DSH = 5 * kTile, OFF_DSL = 6 * kTile;
     constexpr uint32_t R_AT = 0, R_DT = 128, R_DK = 256, R_DV = 384;
-    constexpr int BQK = 0, BVD = 1, BS = 2, BADT = 3, BINTER = 4, BROWS = 5, BOUT = 6, BXK = 7, BDRAIN = 8;
+    constexpr int BQ = 0, BK = 1, BV = 2, BDY = 3, BS = 4, BADT = 5, BINTER = 6, BROWS = 7, BOUT = 8, BXK = 9,
+                  BXDONE = 10, BDRAIN = 11;
     extern __shared__ __align__(1024) uint8_t sm[];
     const uint32_t sb = smem_u32(sm);
     if (sb & 1023u) {
@@ -884,25 +917,24 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kv_tc(const __grid_constant__
     }
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int rank = PAIR ? (int)cluster_ctarank() : 0;
-    const int item = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
-    const int nc = p.nc, u = item / nc, c = item - u * nc, b = u / p.H, hh = u - b * p.H;
-    const int n0 = c * kC, L = min(kC, p.N - n0);
-    const size_t tok0 = (size_t)b * p.N + n0;
+    const int cid = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+    const int ncl = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+    const int nc = p.nc, nitems = p.B * p.H * nc;
+    const int niter = cid < nitems ? (nitems - 1 - cid) / ncl + 1 : 0;
     const int DV = p.dv, ch0 = 128 * rank;
     auto bar = [&](int i) -> uint32_t { return sb + CF::OFF_BAR + 8 * i; };
     float* bc = reinterpret_cast<float*>(sm + CF::OFF_BC);
     float* wsum = bc + kC;
     float* Facc = reinterpret_cast<float*>(sm + CF::OFF_AUX);   // [128] F_j over this CTA's channels
-    float* T1 = Facc + kC;                                       // [128] scratch
-    float* ush = T1 + kC;                                        // [2][128] us_s per column half
+    float* ush = Facc + kC;                                      // [128] us_s over this CTA's channels
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + CF::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + CF::OFF_MISC + 4);
 
-    if (tid == kRowThreads) {
-        for (int i = 0; i < CF::NUM_BARS; ++i) mbar_init(bar(i), i == BROWS ? kRowThreads / 32 : 1);
+    if (tid == RT) {
+        for (int i = 0; i < CF::NUM_BARS; ++i) mbar_init(bar(i), (i == BROWS || i == BXDONE) ? RT / 32 : 1);
         *abort_flag = 0;
         fence_mbar_init();
-        if (PAIR) mbar_arrive_expect_tx(bar(BXK), 64 * 128 * 4);
+        if (PAIR && niter > 0) mbar_arrive_expect_tx(bar(BXK), 64 * 128 * 4);
         tma_prefetch_desc(&p.tmQ);
         tma_prefetch_desc(&p.tmK);
         tma_prefetch_desc(&p.tmV);
@@ -911,7 +943,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kv_tc(const __grid_constant__
         tma_prefetch_desc(&p.tmSH);
         tma_prefetch_desc(&p.tmSL);
     }
-    if (warp == kRowThreads / 32) {
+    if (warp == RT / 32) {
         tmem_alloc(smem_u32(tmem_slot), 512);
         tmem_relinquish();
     }
@@ -922,94 +954,102 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kv_tc(const __grid_constant__
     const uint32_t tm = *tmem_slot;
     const uint32_t peer = (uint32_t)(rank ^ 1);
 
-    float dk[64];
-    if (tid < kRowThreads) {
-        const int q = warp & 3, half = warp >> 2, s = 32 * q + lane;
+    if (tid < RT) {
+        const int q = warp & 3, cq = warp >> 2, s = 32 * q + lane;
         const uint32_t lq = (uint32_t)(32 * q) << 16;
         auto warp_arrive = [&](int i) {
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(i));
         };
-        chunk_decay(p, tok0, hh, L, bc, wsum);
-        if (tid < kC) Facc[tid] = 0.f;
-        const float bs = bc[s], bL = bc[kC - 1];
-        const float ws = s < L ? __expf(bL - bs) : 0.f;
-        named_bar_sync(kNamedBar, kRowThreads);
+        for (int it = 0; it < niter; ++it) {
+            const uint32_t par = it & 1;
+            const int item = cid + it * ncl;
+            const int u = item / nc, c = item - u * nc, b = u / p.H, hh = u - b * p.H;
+            const int n0 = c * kC, L = min(kC, p.N - n0);
+            const size_t tok0 = (size_t)b * p.N + n0;
+            chunk_decay<RT>(p, tok0, hh, L, bc, wsum);
+            if (tid < kC) {
+                Facc[tid] = 0.f;
+                ush[tid] = 0.f;
+            }
+            const float bs = bc[s], bL = bc[kC - 1];
+            const float ws = s < L ? __expf(bL - bs) : 0.f;
+            named_bar_sync(kNamedBar, RT);
 
-        // ---------------------------------------------------- (A o E)^T, (D o E)^T and F
-        const bool ok = mbar_wait(bar(BADT), 0, p.status, abort_flag);
-        tc_fence_after();
-        uint32_t pa[32], pd[32];
-        {
-            float m[64];
-            if (ok) {
-#pragma unroll
-                for (int cb = 0; cb < 2; ++cb) {
+            // ------------------------------------------------ (A o E)^T, (D o E)^T and F
+            // thread (s, cq): key token s, query tokens t = 32 cq .. 32 cq + 31
+            const bool ok = mbar_wait(bar(BADT), par, p.status, abort_flag);
+            tc_fence_after();
+            {
+                float m[32];
+                uint32_t pa[16], pd[16];
+                if (ok) {
                     uint32_t ra[32], rd[32];
-                    tmem_ld_x32(tm + lq + R_AT + 64 * half + 32 * cb, ra);
-                    tmem_ld_x32(tm + lq + R_DT + 64 * half + 32 * cb, rd);
+                    tmem_ld_x32(tm + lq + R_AT + 32 * cq, ra);
+                    tmem_ld_x32(tm + lq + R_DT + 32 * cq, rd);
                     tmem_wait_ld();
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         float av[2], dv2[2];
 #pragma unroll
                         for (int hf = 0; hf < 2; ++hf) {
-                            const int jj = 32 * cb + 2 * j + hf, t = 64 * half + jj;
+                            const int jj = 2 * j + hf, t = 32 * cq + jj;
                             const float e = (t >= s && t < L) ? __expf(fminf(bc[t] - bs, 0.f)) : 0.f;
-                            const float a = u2f(ra[2 * j + hf]), d = u2f(rd[2 * j + hf]);
+                            const float a = u2f(ra[jj]), d = u2f(rd[jj]);
                             av[hf] = a * e;
                             dv2[hf] = d * e;
                             m[jj] = av[hf] * d;
                         }
-                        pa[16 * cb + j] = pack_bf16x2(av[0], av[1]);
-                        pd[16 * cb + j] = pack_bf16x2(dv2[0], dv2[1]);
+                        pa[j] = pack_bf16x2(av[0], av[1]);
+                        pd[j] = pack_bf16x2(dv2[0], dv2[1]);
                     }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) m[j] = 0.f;
                 }
-            } else {
+                // C_s(j) = sum_{t >= j} M_ts: suffix within this column quarter, plus
+                // the later quarters' row totals (exchanged through tensor-memory
+                // columns 64..71, free once every warp has read A^T)
+                float run = 0.f;
 #pragma unroll
-                for (int j = 0; j < 64; ++j) m[j] = 0.f;
-            }
-            // C_s(j) = sum_{t >= j} M_ts: suffix within this half, plus the second
-            // half's row total for the first half
-            float run = 0.f;
+                for (int j = 31; j >= 0; --j) {
+                    run += m[j];
+                    m[j] = run;
+                }
+                named_bar_sync(kNamedBar, RT);   // every row warp has read A^T and D^T
+                if (ok) {
+                    tmem_st_x16(tm + lq + R_AT + 16 * cq, pa);
+                    tmem_st_x16(tm + lq + R_DT + 16 * cq, pd);
+                    const uint32_t tv[2] = {f2u(run), 0u};
+                    tmem_st_x2(tm + lq + R_AT + 64 + 2 * cq, tv);
+                    tmem_wait_st();
+                }
+                named_bar_sync(kNamedBar, RT);
+                float add = 0.f;
+                if (ok) {
+                    uint32_t tr[8];
+                    tmem_ld_x8(tm + lq + R_AT + 64, tr);
+                    tmem_wait_ld();
 #pragma unroll
-            for (int j = 63; j >= 0; --j) {
-                run += m[j];
-                m[j] = run;
-            }
-            if (half) T1[s] = run;
-            named_bar_sync(kNamedBar, kRowThreads);
-            const float add = half ? 0.f : T1[s];
-#pragma unroll
-            for (int g = 0; g < 2; ++g) {
+                    for (int k = 0; k < 4; ++k)
+                        if (k > cq) add += u2f(tr[2 * k]);
+                }
                 float v[32];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int j = 64 * half + 32 * g + i;   // the token j of F_j
-                    v[i] = s < j ? m[32 * g + i] + add : 0.f;
-                }
-                atomicAdd(Facc + 64 * half + 32 * g + lane, transpose_reduce32(v, lane));
+                for (int i = 0; i < 32; ++i) v[i] = s < 32 * cq + i ? m[i] + add : 0.f;   // the token j of F_j
+                atomicAdd(Facc + 32 * cq + lane, transpose_reduce32(v, lane));
             }
-        }
-        // every row warp has read A^T and D^T before their first 64 columns are overwritten
-        named_bar_sync(kNamedBar, kRowThreads);
-        if (ok) {
-            tmem_st_x32(tm + lq + R_AT + 32 * half, pa);
-            tmem_st_x32(tm + lq + R_DT + 32 * half, pd);
-        }
-        // ---------------------------------------------------- e^{b_L - b_s} on the dS' products, us_s
-        float usp = 0.f;
-        if (mbar_wait(bar(BINTER), 0, p.status, abort_flag)) {
-            tc_fence_after();
-            const uint8_t* krow = sm + OFF_K + half * kBox;
-#pragma unroll
-            for (int cb = 0; cb < 2; ++cb) {
+            // ------------------------------------------------ e^{b_L - b_s} on the dS' products, us_s
+            float usp = 0.f;
+            if (mbar_wait(bar(BINTER), par, p.status, abort_flag)) {
+                tc_fence_after();
+                const uint8_t* krow = sm + OFF_K + (cq >> 1) * kBox;
                 uint32_t v[32];
-                tmem_ld_x32(tm + lq + R_DK + 64 * half + 32 * cb, v);
+                tmem_ld_x32(tm + lq + R_DK + 32 * cq, v);
                 tmem_wait_ld();
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    const uint4 kw = *reinterpret_cast<const uint4*>(krow + sw128(s, 32 * cb + 8 * k));
+                    const uint4 kw = *reinterpret_cast<const uint4*>(krow + sw128(s, 32 * (cq & 1) + 8 * k));
                     const uint32_t* ke = reinterpret_cast<const uint32_t*>(&kw);
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
@@ -1019,203 +1059,267 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kv_tc(const __grid_constant__
                         v[8 * k + 2 * e + 1] = f2u(x1);
                     }
                 }
-                tmem_st_x32(tm + lq + R_DK + 64 * half + 32 * cb, v);
-                tmem_ld_x32(tm + lq + R_DV + 64 * half + 32 * cb, v);
+                tmem_st_x32(tm + lq + R_DK + 32 * cq, v);
+                tmem_ld_x32(tm + lq + R_DV + 32 * cq, v);
                 tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < 32; ++j) v[j] = f2u(u2f(v[j]) * ws);
-                tmem_st_x32(tm + lq + R_DV + 64 * half + 32 * cb, v);
+                tmem_st_x32(tm + lq + R_DV + 32 * cq, v);
             }
-        }
-        ush[half * kC + s] = usp;
-        tmem_wait_st();
-        tc_fence_before();
-        warp_arrive(BROWS);
+            atomicAdd(ush + s, usp);
+            tmem_wait_st();
+            tc_fence_before();
+            warp_arrive(BROWS);
 
-        // ---------------------------------------------------- dv rows out, dk partial rows
-        if (mbar_wait(bar(BOUT), 0, p.status, abort_flag)) {
-            tc_fence_after();
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dV) + ((tok0 + s) * p.H + hh) * DV +
-                                                  ch0 + 64 * half);
-#pragma unroll
-            for (int cb = 0; cb < 2; ++cb) {
+            // ------------------------------------------------ dv rows out, dk partial rows
+            float dk[32];
+            if (mbar_wait(bar(BOUT), par, p.status, abort_flag)) {
+                tc_fence_after();
                 uint32_t v[32];
-                tmem_ld_x32(tm + lq + R_DV + 64 * half + 32 * cb, v);
+                tmem_ld_x32(tm + lq + R_DV + 32 * cq, v);
                 tmem_wait_ld();
-                if (s < L)
+                if (s < L) {
+                    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dV) +
+                                                          ((tok0 + s) * p.H + hh) * DV + ch0 + 32 * cq);
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
-                        dst[4 * cb + k] = make_uint4(pack_bf16x2(u2f(v[8 * k]), u2f(v[8 * k + 1])),
-                                                     pack_bf16x2(u2f(v[8 * k + 2]), u2f(v[8 * k + 3])),
-                                                     pack_bf16x2(u2f(v[8 * k + 4]), u2f(v[8 * k + 5])),
-                                                     pack_bf16x2(u2f(v[8 * k + 6]), u2f(v[8 * k + 7])));
-                tmem_ld_x32(tm + lq + R_DK + 64 * half + 32 * cb, v);
+                        dst[k] = make_uint4(pack_bf16x2(u2f(v[8 * k]), u2f(v[8 * k + 1])),
+                                            pack_bf16x2(u2f(v[8 * k + 2]), u2f(v[8 * k + 3])),
+                                            pack_bf16x2(u2f(v[8 * k + 4]), u2f(v[8 * k + 5])),
+                                            pack_bf16x2(u2f(v[8 * k + 6]), u2f(v[8 * k + 7])));
+                }
+                tmem_ld_x32(tm + lq + R_DK + 32 * cq, v);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) dk[32 * cb + j] = u2f(v[j]);
-            }
-        } else {
+                for (int j = 0; j < 32; ++j) dk[j] = u2f(v[j]);
+            } else {
 #pragma unroll
-            for (int j = 0; j < 64; ++j) dk[j] = 0.f;
+                for (int j = 0; j < 32; ++j) dk[j] = 0.f;
+            }
+            tc_fence_before();
+            named_bar_sync(kNamedBar, RT);   // F and us of this CTA are complete
+            if (tid < kC) {
+                float* dst = p.fus + ((size_t)item * 2 + rank) * 2 * kC;
+                dst[tid] = Facc[tid];
+                dst[kC + tid] = ush[tid];
+            }
+            // ------------------------------------------------ dk rows
+            bool mine = true;
+            if constexpr (PAIR) {
+                // the rows of the other CTA's half go to it in one bulk copy: staged
+                // in this CTA's dS' hi tile ([64 rows][128] fp32, 16-byte chunks
+                // swizzled by row), received in its dS' lo tile
+                float* stage = reinterpret_cast<float*>(sm + OFF_DSH);
+                const float* recv = reinterpret_cast<const float*>(sm + OFF_DSL);
+                const int r = s & 63;
+                mine = (s >> 6) == rank;
+                if (!mine)
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        reinterpret_cast<float4*>(stage + r * 128)[8 * cq + (k ^ (r & 7))] =
+                            make_float4(dk[4 * k], dk[4 * k + 1], dk[4 * k + 2], dk[4 * k + 3]);
+                fence_proxy_async_smem();
+                named_bar_sync(kNamedBar, RT);
+                // both CTAs are past this chunk's last product: the dS' tiles are free
+                cluster_sync_all();
+                if (tid == 0) {
+                    bulk_copy_to_cluster(cluster_map(sb + OFF_DSL, peer), sb + OFF_DSH, 64 * 128 * 4,
+                                         cluster_map(bar(BXK), peer));
+                    bulk_commit();
+                }
+                if (mine && mbar_wait_cluster(bar(BXK), par, p.status, abort_flag)) {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const float4 x = reinterpret_cast<const float4*>(recv + r * 128)[8 * cq + (k ^ (r & 7))];
+                        dk[4 * k] += x.x;
+                        dk[4 * k + 1] += x.y;
+                        dk[4 * k + 2] += x.z;
+                        dk[4 * k + 3] += x.w;
+                    }
+                }
+                if (tid == 0) bulk_wait_read<0>();   // the staging tile is read before the next dS' loads
+            }
+            if (mine && s < L) {
+                uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dK) +
+                                                      ((tok0 + s) * p.H + hh) * kDK + 32 * cq);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    dst[k] = make_uint4(pack_bf16x2(dk[8 * k], dk[8 * k + 1]), pack_bf16x2(dk[8 * k + 2], dk[8 * k + 3]),
+                                        pack_bf16x2(dk[8 * k + 4], dk[8 * k + 5]),
+                                        pack_bf16x2(dk[8 * k + 6], dk[8 * k + 7]));
+            }
+            // the exchange tiles have been read: the issuer may load the next dS'
+            warp_arrive(BXDONE);
         }
-        named_bar_sync(kNamedBar, kRowThreads);   // F and us of this CTA are complete
-        if (PAIR && rank == 1 && tid < kC) {
-            float* dst = p.fus + (size_t)item * 2 * kC;
-            dst[tid] = Facc[tid];
-            dst[kC + tid] = ush[tid] + ush[kC + tid];
-            __threadfence();   // read by the other CTA after the cluster barrier
-        }
-    } else if (lane == 0) {
-        // ============================================================ TMA + MMA issuer
+    } else {
+        // ============================================================ TMA + MMA issuer (lane 0)
         constexpr uint32_t id_kk = idesc_bf16(128, 128, false, false);
         constexpr uint32_t id_kn = idesc_bf16(128, 128, false, true);
         auto kmaj = [&](uint32_t base, int k) { return sdesc_sw128(base + (k >> 2) * kBox + (k & 3) * 32, 16, 1024); };
         auto mnmaj = [&](uint32_t base, int k) { return sdesc_sw128(base + k * 2048, kBox, 1024); };
-        const int srow = (u * nc + c) * kDK;
-        mbar_arrive_expect_tx(bar(BQK), 2 * kTile);
-        for (int x = 0; x < 2; ++x) {
-            tma_load_4d(sb + OFF_Q + x * kBox, &p.tmQ, x * 64, hh, n0, b, bar(BQK));
-            tma_load_4d(sb + OFF_K + x * kBox, &p.tmK, x * 64, hh, n0, b, bar(BQK));
-        }
-        mbar_arrive_expect_tx(bar(BVD), 3 * kTile);
-        for (int x = 0; x < 2; ++x) {
-            tma_load_4d(sb + OFF_V + x * kBox, &p.tmV, ch0 + x * 64, hh, n0, b, bar(BVD));
-            tma_load_4d(sb + OFF_DYH + x * kBox, &p.tmDyH, ch0 + x * 64, hh, n0, b, bar(BVD));
-            tma_load_4d(sb + OFF_DYL + x * kBox, &p.tmDyL, ch0 + x * 64, hh, n0, b, bar(BVD));
-        }
-        mbar_arrive_expect_tx(bar(BS), 2 * kTile);
-        for (int x = 0; x < 2; ++x) {
-            tma_load_2d(sb + OFF_DSH + x * kBox, &p.tmSH, ch0 + x * 64, srow, bar(BS));
-            tma_load_2d(sb + OFF_DSL + x * kBox, &p.tmSL, ch0 + x * 64, srow, bar(BS));
-        }
-        bool ok = mbar_wait(bar(BQK), 0, p.status, abort_flag);
-        if (ok) {
-            tc_fence_after();
-            // A^T = K Q^T
-#pragma unroll
-            for (int k = 0; k < 8; ++k) mma_ss(tm + R_AT, kmaj(sb + OFF_K, k), kmaj(sb + OFF_Q, k), id_kk, k > 0);
-        }
-        ok = ok && mbar_wait(bar(BVD), 0, p.status, abort_flag);
-        if (ok) {
-            tc_fence_after();
-            // D^T = V dy^T (dy as a bf16 pair)
-            for (int pass = 0; pass < 2; ++pass)
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mma_ss(tm + R_DT, kmaj(sb + OFF_V, k), kmaj(sb + (pass ? OFF_DYL : OFF_DYH), k), id_kk,
-                           pass > 0 || k > 0);
-        }
-        mma_commit(bar(BADT));
-        ok = ok && mbar_wait(bar(BS), 0, p.status, abort_flag);
-        if (ok) {
-            tc_fence_after();
-            // V dS'^T and K dS' (dS' as a bf16 pair)
-            for (int pass = 0; pass < 2; ++pass)
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mma_ss(tm + R_DK, kmaj(sb + OFF_V, k), kmaj(sb + (pass ? OFF_DSL : OFF_DSH), k), id_kk,
-                           pass > 0 || k > 0);
-            for (int pass = 0; pass < 2; ++pass)
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mma_ss(tm + R_DV, kmaj(sb + OFF_K, k), mnmaj(sb + (pass ? OFF_DSL : OFF_DSH), k), id_kn,
-                           pass > 0 || k > 0);
-        }
-        mma_commit(bar(BINTER));
-        ok = ok && mbar_wait(bar(BROWS), 0, p.status, abort_flag);
-        if (ok) {
-            tc_fence_after();
-            // dk += (D o E)^T Q, dv += (A o E)^T dy
-#pragma unroll
-            for (int k = 0; k < 8; ++k) mma_ts(tm + R_DK, tm + R_DT + k * 8, mnmaj(sb + OFF_Q, k), id_kn, 1);
-            for (int pass = 0; pass < 2; ++pass)
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mma_ts(tm + R_DV, tm + R_AT + k * 8, mnmaj(sb + (pass ? OFF_DYL : OFF_DYH), k), id_kn, 1);
-        }
-        mma_commit(bar(BOUT));
-        mma_commit(bar(BDRAIN));
-        mbar_wait_drain(bar(BDRAIN), 0, kWaitCycles);
-        if (*abort_flag) {
-            mbar_wait_drain(bar(BQK), 0, kWaitCycles);
-            mbar_wait_drain(bar(BVD), 0, kWaitCycles);
-            mbar_wait_drain(bar(BS), 0, kWaitCycles);
-        }
-    }
-    __syncwarp();
-    if constexpr (PAIR) cluster_sync_all();   // both CTAs are past their last MMA; F and us exported
-    if (tid < kRowThreads) {
-        const int q = warp & 3, half = warp >> 2, s = 32 * q + lane;
-        // ---------------------------------------------------- dk rows
-        float* recv = reinterpret_cast<float*>(sm + OFF_DSH);   // [64 rows][128] partials from the other CTA
-        bool mine = true;
-        if constexpr (PAIR) {
-            const int owner = s >> 6;
-            mine = owner == rank;
-            if (!mine) {
-                const uint32_t remote = cluster_map(smem_u32(recv + (s & 63) * 128 + 64 * half), peer);
-                const uint32_t rbar = cluster_map(bar(BXK), peer);
-#pragma unroll
-                for (int k = 0; k < 16; ++k)
-                    st_async_f4(remote + 16 * k, rbar, dk[4 * k], dk[4 * k + 1], dk[4 * k + 2], dk[4 * k + 3]);
-            } else if (mbar_wait_cluster(bar(BXK), 0, p.status, abort_flag)) {
-                const float* src = recv + (s & 63) * 128 + 64 * half;
-#pragma unroll
-                for (int j = 0; j < 64; ++j) dk[j] += src[j];
+        // the tiles of chunk item (coordinates: token n0 of sequence b, head hh)
+        auto coords = [&](int it, int& n0, int& b, int& hh, int& srow) {
+            const int item = cid + it * ncl, u = item / nc, c = item - u * nc;
+            b = u / p.H;
+            hh = u - b * p.H;
+            n0 = c * kC;
+            srow = (u * nc + c) * kDK;
+        };
+        auto load_tok = [&](int it, int bi, const CUtensorMap* m0, const CUtensorMap* m1, uint32_t o0, uint32_t o1,
+                            int x0) {
+            int n0, b, hh, srow;
+            coords(it, n0, b, hh, srow);
+            mbar_arrive_expect_tx(bar(bi), (m1 ? 2 : 1) * kTile);
+            for (int x = 0; x < 2; ++x) {
+                tma_load_4d(sb + o0 + x * kBox, m0, x0 + x * 64, hh, n0, b, bar(bi));
+                if (m1) tma_load_4d(sb + o1 + x * kBox, m1, x0 + x * 64, hh, n0, b, bar(bi));
             }
+        };
+        auto load_q = [&](int it) { load_tok(it, BQ, &p.tmQ, nullptr, OFF_Q, 0, 0); };
+        auto load_k = [&](int it) { load_tok(it, BK, &p.tmK, nullptr, OFF_K, 0, 0); };
+        auto load_v = [&](int it) { load_tok(it, BV, &p.tmV, nullptr, OFF_V, 0, ch0); };
+        auto load_dy = [&](int it) { load_tok(it, BDY, &p.tmDyH, &p.tmDyL, OFF_DYH, OFF_DYL, ch0); };
+        auto load_s = [&](int it) {
+            int n0, b, hh, srow;
+            coords(it, n0, b, hh, srow);
+            mbar_arrive_expect_tx(bar(BS), 2 * kTile);
+            for (int x = 0; x < 2; ++x) {
+                tma_load_2d(sb + OFF_DSH + x * kBox, &p.tmSH, ch0 + x * 64, srow, bar(BS));
+                tma_load_2d(sb + OFF_DSL + x * kBox, &p.tmSL, ch0 + x * 64, srow, bar(BS));
+            }
+        };
+        if (lane == 0 && niter > 0) {
+            load_q(0);
+            load_k(0);
+            load_v(0);
+            load_dy(0);
+            load_s(0);
         }
-        if (mine && s < L) {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dK) + ((tok0 + s) * p.H + hh) * kDK +
-                                                  64 * half);
+        for (int it = 0; it < niter; ++it) {
+            const uint32_t par = it & 1;
+            const bool more = it + 1 < niter;
+            if (lane == 0) {
+                bool ok = mbar_wait(bar(BQ), par, p.status, abort_flag) && mbar_wait(bar(BK), par, p.status, abort_flag);
+                if (ok) {
+                    tc_fence_after();
+                    // A^T = K Q^T
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-                dst[k] = make_uint4(pack_bf16x2(dk[8 * k], dk[8 * k + 1]), pack_bf16x2(dk[8 * k + 2], dk[8 * k + 3]),
-                                    pack_bf16x2(dk[8 * k + 4], dk[8 * k + 5]), pack_bf16x2(dk[8 * k + 6], dk[8 * k + 7]));
-        }
-        // ---------------------------------------------------- dz (rank 0)
-        if (rank == 0 && tid < kC) {
-            const int j = tid;
-            const float* other = PAIR ? p.fus + (size_t)item * 2 * kC : nullptr;
-            const size_t tk = (tok0 + j) * p.H + hh;
-            float F = Facc[j], us = ush[j] + ush[kC + j], rr = 0.f;
-            if (PAIR) {
-                F += other[j];
-                us += other[kC + j];
-            }
-            if (j < L) {
-                rr = p.rr[tk];
-                if (PAIR) rr += p.rr[(size_t)p.B * p.N * p.H + tk];
-            }
-            // R_j = sum_{t >= j} rr_t (suffix), U_j = sum_{s < j} us_s (exclusive prefix)
-            float R = rr, U = us;
+                    for (int k = 0; k < 8; ++k) mma_ss(tm + R_AT, kmaj(sb + OFF_K, k), kmaj(sb + OFF_Q, k), id_kk, k > 0);
+                }
+                ok = ok && mbar_wait(bar(BV), par, p.status, abort_flag) && mbar_wait(bar(BDY), par, p.status, abort_flag);
+                if (ok) {
+                    tc_fence_after();
+                    // D^T = V dy^T (dy as a bf16 pair)
+                    for (int pass = 0; pass < 2; ++pass)
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float r2 = __shfl_down_sync(0xffffffffu, R, o);
-                const float u2 = __shfl_up_sync(0xffffffffu, U, o);
-                if (lane + o < 32) R += r2;
-                if (lane >= o) U += u2;
+                        for (int k = 0; k < 8; ++k)
+                            mma_ss(tm + R_DT, kmaj(sb + OFF_V, k), kmaj(sb + (pass ? OFF_DYL : OFF_DYH), k), id_kk,
+                                   pass > 0 || k > 0);
+                }
+                mma_commit(bar(BADT));
+                ok = ok && mbar_wait(bar(BS), par, p.status, abort_flag);
+                if (ok) {
+                    tc_fence_after();
+                    // V dS'^T and K dS' (dS' as a bf16 pair)
+                    for (int pass = 0; pass < 2; ++pass)
+#pragma unroll
+                        for (int k = 0; k < 8; ++k)
+                            mma_ss(tm + R_DK, kmaj(sb + OFF_V, k), kmaj(sb + (pass ? OFF_DSL : OFF_DSH), k), id_kk,
+                                   pass > 0 || k > 0);
+                    for (int pass = 0; pass < 2; ++pass)
+#pragma unroll
+                        for (int k = 0; k < 8; ++k)
+                            mma_ss(tm + R_DV, kmaj(sb + OFF_K, k), mnmaj(sb + (pass ? OFF_DSL : OFF_DSH), k), id_kn,
+                                   pass > 0 || k > 0);
+                }
+                mma_commit(bar(BINTER));
+                // V is free once the dS' products have read it
+                if (mbar_wait(bar(BINTER), par, p.status, abort_flag) && more) load_v(it + 1);
+                ok = ok && mbar_wait(bar(BROWS), par, p.status, abort_flag);
+                // K is free once the rows have read it (us) and the products above are done
+                if (ok && more) load_k(it + 1);
+                if (ok) {
+                    tc_fence_after();
+                    // dk += (D o E)^T Q, dv += (A o E)^T dy
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) mma_ts(tm + R_DK, tm + R_DT + k * 8, mnmaj(sb + OFF_Q, k), id_kn, 1);
+                    for (int pass = 0; pass < 2; ++pass)
+#pragma unroll
+                        for (int k = 0; k < 8; ++k)
+                            mma_ts(tm + R_DV, tm + R_AT + k * 8, mnmaj(sb + (pass ? OFF_DYL : OFF_DYH), k), id_kn, 1);
+                }
+                mma_commit(bar(BOUT));
+                if (mbar_wait(bar(BOUT), par, p.status, abort_flag) && more) {
+                    load_q(it + 1);
+                    load_dy(it + 1);
+                }
             }
-            U -= us;
-            // warp totals: R of lane 0 is its warp's total, U + us of lane 31 likewise
-            float* tot = T1;   // [4] rr totals, [4] us totals (T1 is no longer needed)
-            named_bar_sync(2, kC);
-            if (lane == 0) tot[warp] = R;
-            if (lane == 31) tot[4 + warp] = U + us;
-            named_bar_sync(2, kC);
-            for (int w = warp + 1; w < 4; ++w) R += tot[w];
-            for (int w = 0; w < warp; ++w) U += tot[4 + w];
-            if (j < L) {
-                const float dlg = F + R + p.xs[(size_t)u * nc + c] + U;
-                const float zj = p.z[tk];
-                const float deriv = log_gamma(zj, p.inv_tau) > kMinLogGamma ? (1.f - sigmoidf_(zj)) * p.inv_tau : 0.f;
-                p.dz[tk] = dlg * deriv;
+            __syncwarp();
+            if constexpr (PAIR) cluster_sync_all();
+            if (lane == 0) {
+                // the dk exchange of this chunk has been read: the next dS' may load
+                // into its buffer, and the exchange barrier is armed for the next chunk
+                if (mbar_wait(bar(BXDONE), par, p.status, abort_flag) && more) {
+                    if (PAIR) mbar_arrive_expect_tx(bar(BXK), 64 * 128 * 4);
+                    load_s(it + 1);
+                }
             }
+            __syncwarp();
         }
+        if (lane == 0) {
+            mma_commit(bar(BDRAIN));
+            mbar_wait_drain(bar(BDRAIN), 0, kWaitCycles);
+        }
+        __syncwarp();
     }
     tc_fence_before();
     __syncthreads();
     if constexpr (PAIR) cluster_sync_all();   // no CTA leaves while the other still sends to it
-    if (warp == kRowThreads / 32) tmem_dealloc(tm, 512);
+    if (warp == RT / 32) tmem_dealloc(tm, 512);
+}
+
+// ---- 6. per chunk, one thread per token: the gate gradient
+//   dz_j = (F_j + sum_{t>=j} rr_t + X_c + sum_{s<j} us_s) (1 - sigmoid(z_j)) / tau
+// from the F and us the dk/dv kernel left per channel half, the rr of the dy
+// kernel and the d_v shares of X_c of the reverse scan; zero where the
+// forward clamps log gamma
+__global__ void __launch_bounds__(kC) bwd_dz(const __grid_constant__ BwdTcParams p) {
+    __shared__ float tot[12];
+    const int item = blockIdx.x, nc = p.nc, u = item / nc, c = item - u * nc, b = u / p.H, hh = u - b * p.H;
+    const int n0 = c * kC, L = min(kC, p.N - n0), j = threadIdx.x, lane = j & 31, warp = j >> 5;
+    const int halves = p.dv / 128, DV = p.dv;
+    const size_t tk = ((size_t)b * p.N + n0 + j) * p.H + hh;
+    float F = 0.f, us = 0.f, rr = 0.f, X = 0.f;
+    for (int h = 0; h < halves; ++h) {
+        const float* src = p.fus + ((size_t)item * 2 + h) * 2 * kC;
+        F += src[j];
+        us += src[kC + j];
+        if (j < L) rr += p.rr[(size_t)h * p.B * p.N * p.H + tk];
+    }
+    for (int w = j; w < DV; w += kC) X += p.xs[((size_t)u * nc + c) * DV + w];
+    X = warp_sum(X);
+    // R_j = sum_{t >= j} rr_t (suffix), U_j = sum_{s < j} us_s (exclusive prefix)
+    float R = rr, U = us;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float r2 = __shfl_down_sync(0xffffffffu, R, o);
+        const float u2 = __shfl_up_sync(0xffffffffu, U, o);
+        if (lane + o < 32) R += r2;
+        if (lane >= o) U += u2;
+    }
+    U -= us;
+    if (lane == 0) tot[warp] = R;
+    if (lane == 31) tot[4 + warp] = U + us;
+    if (lane == 0) tot[8 + warp] = X;
+    __syncthreads();
+    for (int w = warp + 1; w < 4; ++w) R += tot[w];
+    for (int w = 0; w < warp; ++w) U += tot[4 + w];
+    X = tot[8] + tot[9] + tot[10] + tot[11];
+    if (j < L) {
+        const float zj = p.z[tk];
+        const float deriv = log_gamma(zj, p.inv_tau) > kMinLogGamma ? (1.f - sigmoidf_(zj)) * p.inv_tau : 0.f;
+        p.dz[tk] = (F + R + X + U) * deriv;
+    }
 }
 
 // ---------------------------------------------------------------- host side
@@ -1283,19 +1387,19 @@ BwdTcWs bwd_tc_ws(int B, int H, int N, int dv) {
     w.dyh = o; o += a256(tok * dv * 2);
     w.dyl = o; o += a256(tok * dv * 2);
     w.rr = o; o += a256(2 * tok * 4);
-    w.xs = o; o += a256(units * nc * 4);
+    w.xs = o; o += a256(units * nc * dv * 4);
     w.decay = o; o += a256(units * nc * 4);
-    w.fus = o; o += a256(units * nc * 2 * kC * 4);
+    w.fus = o; o += a256(units * nc * 2 * 2 * kC * 4);
     w.total = o;
     return w;
 }
 
 template <typename... KArgs, typename... Args>
 cudaError_t launch_cluster(void (*kernel)(KArgs...), unsigned grid, int cluster, size_t smem, cudaStream_t s,
-                           Args&&... args) {
+                           int threads, Args&&... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(threads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
@@ -1312,22 +1416,31 @@ template <int DV>
 cudaError_t run_bwd_tc(BwdTcParams& p, cudaStream_t s) {
     constexpr bool PAIR = DV == 256;
     const unsigned items = (unsigned)((size_t)p.B * p.H * p.nc);
-    auto k1 = bwd_inc_tc<DV>;
+    auto k1 = bwd_inc_tc;
     auto k3 = bwd_dyq_tc<PAIR>;
     auto k5 = bwd_kv_tc<PAIR>;
     cudaError_t e;
-    if ((e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, IncCfg<DV>::SMEM)) != cudaSuccess)
+    if ((e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, IncCfg::SMEM)) != cudaSuccess)
         return e;
     if ((e = cudaFuncSetAttribute(k3, cudaFuncAttributeMaxDynamicSharedMemorySize, GradCfg::SMEM)) != cudaSuccess)
         return e;
     if ((e = cudaFuncSetAttribute(k5, cudaFuncAttributeMaxDynamicSharedMemorySize, GradCfg::SMEM)) != cudaSuccess)
         return e;
     const dim3 sgrid((unsigned)((kDK * DV / 4 + kScanThreads - 1) / kScanThreads), (unsigned)(p.B * p.H));
-    k1<<<items, kThreads, IncCfg<DV>::SMEM, s>>>(p);
+    k1<<<items * (DV / 128), kThreads, IncCfg::SMEM, s>>>(p);
     bwd_scan_fwd<<<sgrid, kScanThreads, 0, s>>>(p);
-    if ((e = launch_cluster(k3, items * (PAIR ? 2 : 1), PAIR ? 2 : 1, GradCfg::SMEM, s, p)) != cudaSuccess) return e;
+    if ((e = launch_cluster(k3, items * (PAIR ? 2 : 1), PAIR ? 2 : 1, GradCfg::SMEM, s, kThreads, p)) != cudaSuccess)
+        return e;
     bwd_scan_rev<<<sgrid, kScanThreads, 0, s>>>(p);
-    if ((e = launch_cluster(k5, items * (PAIR ? 2 : 1), PAIR ? 2 : 1, GradCfg::SMEM, s, p)) != cudaSuccess) return e;
+    // dk/dv/dz: persistent, one CTA (pair) per SM (pair of SMs)
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    const unsigned ncl = std::min<unsigned>(items, (unsigned)std::max(1, PAIR ? sms / 2 : sms));
+    if ((e = launch_cluster(k5, ncl * (PAIR ? 2 : 1), PAIR ? 2 : 1, GradCfg::SMEM, s, kThreads16, p)) !=
+        cudaSuccess)
+        return e;
+    bwd_dz<<<items, kC, 0, s>>>(p);
     return cudaGetLastError();
 }
 

@@ -156,7 +156,8 @@ struct BackwardArgs {
 };
 size_t prefill_backward_workspace_bytes(int B, int H, int N, int dk, int dv, gret_dtype io);
 bool prefill_backward_supported(int dk, int dv);
-// launches one backward call makes (5 on the chunk-parallel path, 2 on the serial one)
+// launches one backward call makes (6 on the tensor-core path, 5 on the chunk-parallel
+// CUDA-core path, 2 on the serial one)
 int prefill_backward_launches(int B, int H, int N, int dk, int dv, gret_dtype io);
 cudaError_t launch_prefill_backward(const BackwardArgs& a, cudaStream_t s);
 // chunk-parallel backward (gret_backward_chunk.cu): head sizes multiples of 32,
