@@ -62,6 +62,8 @@ constexpr int kTile = 2 * kBox;          // [128 rows][128 bf16]
 constexpr int kRowThreads = 256;         // eight warps: lane quarter q = w & 3, column half w >> 2
 constexpr int kThreads = kRowThreads + 32;
 constexpr int kNamedBar = 1;             // named barrier among the row warps
+constexpr int kRowThreads16 = 512;       // sixteen row warps: lane quarter q = w & 3, column quarter w >> 2
+constexpr int kThreads16 = kRowThreads16 + 32;
 
 struct BwdTcParams {
     CUtensorMap tmQ, tmK, tmV, tmDyH, tmDyL, tmSH, tmSL;
@@ -346,7 +348,7 @@ __global__ void __launch_bounds__(kScanThreads) bwd_scan_rev(const __grid_consta
 struct GradCfg {
     static constexpr int OFF_BC = 7 * kTile;          // b_t [128], 4 warp sums
     static constexpr int OFF_AUX = OFF_BC + 528;      // 2 KB: exchange buffers / row sums
-    static constexpr int NUM_BARS = 18;
+    static constexpr int NUM_BARS = 22;
     static constexpr int OFF_BAR = OFF_AUX + 2048;
     static constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;
     static constexpr int SMEM = OFF_MISC + 16;
@@ -357,21 +359,27 @@ struct GradCfg {
 // (dG; dy as a bf16 pair to the workspace), G_c = sum_t e^{b_t} q_t^T dy_t into
 // slot c of incg, rr_t = dy_t . (e^{b_t} q_t S_c), and
 // dq = (D o E) K + e^{b_t} dy S_c^T.  With PAIR the CTA of cluster rank h owns
-// channels 128 h .. 128 h + 127 and rows 64 h .. 64 h + 63 of dq.
+// channels 128 h .. 128 h + 127 and rows 64 h .. 64 h + 63 of dq.  Persistent
+// like the dk/dv kernel: the issuer loads the next chunk's Q once the rows have
+// built Q~^T, V after D, S after dy S^T and K after the last product.
 //
-// Tensor memory (512 columns): [0,128) scores A, then D, then D o E (bf16);
-// [128,256) Y = P V, then e^{b_t} dy S^T + (D o E) K; [256,384) Yi = Q S, then
-// G_c; [384,512) P (bf16), then Q~^T as a bf16 pair.
+// Tensor memory (512 columns): [0,128) scores A, then row-sum scratch, then D,
+// then D o E (bf16); [128,256) Y = P V, then e^{b_t} dy S^T + (D o E) K;
+// [256,384) Yi = Q S, then G_c; [384,512) P (bf16), then Q~^T as a bf16 pair.
 // Shared memory tiles: Q, K, V (this CTA's channels), S_c hi, S_c lo, dy hi,
-// dy lo; the dy lo tile is scratch for the row sums until dy is written.
+// dy lo; after the chunk's products the dy tiles carry the dq exchange of the
+// pair (lo: the rows sent, hi: the rows received).
 template <bool PAIR>
-__global__ void __launch_bounds__(kThreads, 1) bwd_dyq_tc(const __grid_constant__ BwdTcParams p) {
+__global__ void __launch_bounds__(kThreads16, 1) bwd_dyq_tc(const __grid_constant__ BwdTcParams p) {
     using CF = GradCfg;
+    constexpr int RT = kRowThreads16;
     constexpr int OFF_Q = 0, OFF_K = kTile, OFF_V = 2 * kTile, OFF_SH = 3 * kTile, OFF_SL = 4 * kTile,
                   OFF_DYH = 5 * kTile, OFF_DYL = 6 * kTile;
     constexpr uint32_t R_A = 0, R_Y = 128, R_YI = 256, R_P = 384;
-    constexpr int BQK = 0, BVS = 1, BA = 2, BYI = 3, BP = 4, BY = 5, BDY = 6, BD = 7, BQI = 8, BQT = 9, BGC = 10,
-                  BDS = 11, BDQ = 12, BX0 = 13, BX1 = 14, BX2 = 15, BXQ = 16, BDRAIN = 17;
+    constexpr int BQ = 0, BK = 1, BV = 2, BS = 3, BA = 4, BYI = 5, BP = 6, BY = 7, BDY = 8, BD = 9, BQI = 10,
+                  BQT = 11, BGC = 12, BDS = 13, BDQ = 14, BX0 = 15, BX1 = 16, BX2 = 17, BXQ = 18, BDYRD = 19,
+                  BDRAIN = 20, BEND = 21;
+    static_assert(BEND < CF::NUM_BARS, "barrier count");
     extern __shared__ __align__(1024) uint8_t sm[];
     const uint32_t sb = smem_u32(sm);
     if (sb & 1023u) {
@@ -380,33 +388,33 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dyq_tc(const __grid_constant_
     }
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int rank = PAIR ? (int)cluster_ctarank() : 0;
-    const int item = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
-    const int nc = p.nc, u = item / nc, c = item - u * nc, b = u / p.H, hh = u - b * p.H;
-    const int n0 = c * kC, L = min(kC, p.N - n0);
-    const size_t tok0 = (size_t)b * p.N + n0;
+    const int cid = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+    const int ncl = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+    const int nc = p.nc, nitems = p.B * p.H * nc;
+    const int niter = cid < nitems ? (nitems - 1 - cid) / ncl + 1 : 0;
     const int DV = p.dv, ch0 = 128 * rank;
     auto bar = [&](int i) -> uint32_t { return sb + CF::OFF_BAR + 8 * i; };
     float* bc = reinterpret_cast<float*>(sm + CF::OFF_BC);
     float* wsum = bc + kC;
     float* xch = reinterpret_cast<float*>(sm + CF::OFF_AUX);   // [128] round 0, [128] round 1, [128][2] round 2
-    float* scr = reinterpret_cast<float*>(sm + OFF_DYL);       // [9][128] row partial sums
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + CF::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + CF::OFF_MISC + 4);
+    // one-shot-per-chunk exchange barriers, armed for the bytes the other CTA sends
+    auto arm_exchange = [&]() {
+        if (p.gn) {
+            mbar_arrive_expect_tx(bar(BX0), kC * 4);
+            mbar_arrive_expect_tx(bar(BX1), kC * 4);
+            mbar_arrive_expect_tx(bar(BX2), kC * 8);
+        }
+        mbar_arrive_expect_tx(bar(BXQ), 64 * 128 * 4);
+    };
 
-    if (tid == kRowThreads) {
+    if (tid == RT) {
         for (int i = 0; i < CF::NUM_BARS; ++i)
-            mbar_init(bar(i), (i == BP || i == BDY || i == BQT || i == BDS) ? kRowThreads / 32 : 1);
+            mbar_init(bar(i), (i == BP || i == BDY || i == BQT || i == BDS || i == BEND) ? RT / 32 : 1);
         *abort_flag = 0;
         fence_mbar_init();
-        if (PAIR) {
-            // one-shot exchange barriers, armed for the bytes the other CTA sends
-            if (p.gn) {
-                mbar_arrive_expect_tx(bar(BX0), kC * 4);
-                mbar_arrive_expect_tx(bar(BX1), kC * 4);
-                mbar_arrive_expect_tx(bar(BX2), kC * 8);
-            }
-            mbar_arrive_expect_tx(bar(BXQ), 64 * 128 * 4);
-        }
+        if (PAIR && niter > 0) arm_exchange();
         tma_prefetch_desc(&p.tmQ);
         tma_prefetch_desc(&p.tmK);
         tma_prefetch_desc(&p.tmV);
@@ -415,7 +423,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dyq_tc(const __grid_constant_
         tma_prefetch_desc(&p.tmDyH);
         tma_prefetch_desc(&p.tmDyL);
     }
-    if (warp == kRowThreads / 32) {
+    if (warp == RT / 32) {
         tmem_alloc(smem_u32(tmem_slot), 512);
         tmem_relinquish();
     }
@@ -426,443 +434,483 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dyq_tc(const __grid_constant_
     const uint32_t tm = *tmem_slot;
     const uint32_t peer = (uint32_t)(rank ^ 1);
 
-    float dq[64];
-    if (tid < kRowThreads) {
-        const int q = warp & 3, half = warp >> 2, t = 32 * q + lane;
+    if (tid < RT) {
+        const int q = warp & 3, cq = warp >> 2, t = 32 * q + lane;
         const uint32_t lq = (uint32_t)(32 * q) << 16;
         auto warp_arrive = [&](int i) {
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(i));
         };
-        // G and dO of this thread's row and 64 channels, requested now (volatile
-        // loads stay where they are written) and used by the GroupNorm backward
-        const size_t rowoff = ((tok0 + t) * p.H + hh) * (size_t)DV + ch0 + 64 * half;
-        uint4 gv[8], ov[8];
+        for (int it = 0; it < niter; ++it) {
+            const uint32_t par = it & 1;
+            const int item = cid + it * ncl;
+            const int u = item / nc, c = item - u * nc, b = u / p.H, hh = u - b * p.H;
+            const int n0 = c * kC, L = min(kC, p.N - n0);
+            const size_t tok0 = (size_t)b * p.N + n0;
+            // G and dO of this thread's row and 32 channels, requested now
+            // (volatile loads stay where they are written)
+            const size_t rowoff = ((tok0 + t) * p.H + hh) * (size_t)DV + ch0 + 32 * cq;
+            uint4 gv[4], ov[4];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            ov[k] = make_uint4(0u, 0u, 0u, 0u);
-            gv[k] = make_uint4(0u, 0u, 0u, 0u);
-        }
-        if (t < L) {
-            const uint4* og = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.dO) + rowoff);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) ov[k] = ldg_nc_v4(og + k);
-            if (p.gn) {
-                const uint4* gg = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.G) + rowoff);
-#pragma unroll
-                for (int k = 0; k < 8; ++k) gv[k] = ldg_nc_v4(gg + k);
+            for (int k = 0; k < 4; ++k) {
+                ov[k] = make_uint4(0u, 0u, 0u, 0u);
+                gv[k] = make_uint4(0u, 0u, 0u, 0u);
             }
-        }
-        chunk_decay(p, tok0, hh, L, bc, wsum);
-        const float bt = bc[t], ebt = __expf(bt);
+            if (t < L) {
+                const uint4* og = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.dO) + rowoff);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) ov[k] = ldg_nc_v4(og + k);
+                if (p.gn) {
+                    const uint4* gg = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.G) + rowoff);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) gv[k] = ldg_nc_v4(gg + k);
+                }
+            }
+            chunk_decay<RT>(p, tok0, hh, L, bc, wsum);
+            const float bt = bc[t], ebt = __expf(bt);
 
-        // ---------------------------------------------------- P = A o E, masked
-        if (mbar_wait(bar(BA), 0, p.status, abort_flag)) {
-            tc_fence_after();
-            uint32_t r[32], pk[16];
-#pragma unroll 1
-            for (int cb = 0; cb < 2; ++cb) {
-                tmem_ld_x32(tm + lq + R_A + 64 * half + 32 * cb, r);
+            // ------------------------------------------------ P = A o E, masked
+            if (mbar_wait(bar(BA), par, p.status, abort_flag)) {
+                tc_fence_after();
+                uint32_t r[32], pk[16];
+                tmem_ld_x32(tm + lq + R_A + 32 * cq, r);
                 tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
-                    const int s0 = 64 * half + 32 * cb + 2 * j;
+                    const int s0 = 32 * cq + 2 * j;
                     const float v0 = s0 <= t ? u2f(r[2 * j]) * __expf(fminf(bt - bc[s0], 0.f)) : 0.f;
                     const float v1 = s0 + 1 <= t ? u2f(r[2 * j + 1]) * __expf(fminf(bt - bc[s0 + 1], 0.f)) : 0.f;
                     pk[j] = pack_bf16x2(v0, v1);
                 }
-                tmem_st_x16(tm + lq + R_P + 32 * half + 16 * cb, pk);
+                tmem_st_x16(tm + lq + R_P + 16 * cq, pk);
+                tmem_wait_st();
             }
-            tmem_wait_st();
-        }
-        tc_fence_before();
-        warp_arrive(BP);
+            tc_fence_before();
+            warp_arrive(BP);
 
-        // ---------------------------------------------------- GroupNorm * swish backward
-        // sum over the row's d_v channels of (a, b): the two column-half warps
-        // through `scr`, the pair through distributed shared memory
-        auto row_sum = [&](int slot, int xbar, float a, float bv, bool two, float& ra, float& rb) {
-            if (half) {
-                scr[(2 * slot) * kC + t] = a;
-                if (two) scr[(2 * slot + 1) * kC + t] = bv;
-            }
-            named_bar_sync(kNamedBar, kRowThreads);
-            if (!half) {
-                a += scr[(2 * slot) * kC + t];
-                if (two) bv += scr[(2 * slot + 1) * kC + t];
-                if constexpr (PAIR) {
+            // ------------------------------------------------ GroupNorm * swish backward
+            // Row sums over the d_v channels: the four column-quarter warps of a lane
+            // quarter through tensor-memory columns 8 slot .. 8 slot + 7 (the scores'
+            // columns, free after P), the pair through distributed shared memory.
+            auto row_sum = [&](int slot, int xbar, float a, float bv, bool two, bool pair, float& ra, float& rb) {
+                const uint32_t col = tm + lq + R_A + 8 * slot;
+                const uint32_t w2[2] = {f2u(a), f2u(bv)};
+                tmem_st_x2(col + 2 * cq, w2);
+                tmem_wait_st();
+                named_bar_sync(kNamedBar, RT);
+                uint32_t r8[8];
+                tmem_ld_x8(col, r8);
+                tmem_wait_ld();
+                ra = u2f(r8[0]) + u2f(r8[2]) + u2f(r8[4]) + u2f(r8[6]);
+                rb = u2f(r8[1]) + u2f(r8[3]) + u2f(r8[5]) + u2f(r8[7]);
+                if (PAIR && pair) {
                     const int off = slot == 0 ? t : slot == 1 ? kC + t : 2 * kC + 2 * t;
-                    const uint32_t remote = cluster_map(smem_u32(xch + off), peer);
-                    const uint32_t rbar = cluster_map(bar(xbar), peer);
-                    if (two)
-                        st_async_f2(remote, rbar, a, bv);
-                    else
-                        st_async_f1(remote, rbar, a);
-                    if (mbar_wait_cluster(bar(xbar), 0, p.status, abort_flag)) {
-                        a += xch[off];
-                        if (two) bv += xch[off + 1];
+                    if (cq == 0) {
+                        const uint32_t remote = cluster_map(smem_u32(xch + off), peer);
+                        const uint32_t rbar = cluster_map(bar(xbar), peer);
+                        if (two)
+                            st_async_f2(remote, rbar, ra, rb);
+                        else
+                            st_async_f1(remote, rbar, ra);
+                    }
+                    if (mbar_wait_cluster(bar(xbar), par, p.status, abort_flag)) {
+                        ra += xch[off];
+                        if (two) rb += xch[off + 1];
                     }
                 }
-                scr[(2 * slot) * kC + t] = a;
-                if (two) scr[(2 * slot + 1) * kC + t] = bv;
-            }
-            named_bar_sync(kNamedBar, kRowThreads);
-            ra = scr[(2 * slot) * kC + t];
-            rb = two ? scr[(2 * slot + 1) * kC + t] : 0.f;
-            named_bar_sync(kNamedBar, kRowThreads);
-        };
-        float y[64];
-        const bool ok_y = mbar_wait(bar(BY), 0, p.status, abort_flag) && mbar_wait(bar(BYI), 0, p.status, abort_flag);
-        tc_fence_after();
-        if (ok_y) {
-            uint32_t r[32], ri[32];
-#pragma unroll
-            for (int cb = 0; cb < 2; ++cb) {
-                tmem_ld_x32(tm + lq + R_Y + 64 * half + 32 * cb, r);
-                tmem_ld_x32(tm + lq + R_YI + 64 * half + 32 * cb, ri);
+            };
+            float y[32];
+            const bool ok_y =
+                mbar_wait(bar(BY), par, p.status, abort_flag) && mbar_wait(bar(BYI), par, p.status, abort_flag);
+            tc_fence_after();
+            if (ok_y) {
+                uint32_t r[32], ri[32];
+                tmem_ld_x32(tm + lq + R_Y + 32 * cq, r);
+                tmem_ld_x32(tm + lq + R_YI + 32 * cq, ri);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) y[32 * cb + j] = fmaf(ebt, u2f(ri[j]), u2f(r[j]));
+                for (int j = 0; j < 32; ++j) y[j] = fmaf(ebt, u2f(ri[j]), u2f(r[j]));
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) y[j] = 0.f;
             }
-        } else {
+            if (p.gn) {
+                const float inv_dv = 1.0f / (float)DV;
+                float s1 = 0.f, dummy;
 #pragma unroll
-            for (int j = 0; j < 64; ++j) y[j] = 0.f;
-        }
-        if (p.gn) {
-            const float inv_dv = 1.0f / (float)DV;
-            float s1 = 0.f, dummy;
+                for (int j = 0; j < 32; ++j) s1 += y[j];
+                float mean;
+                row_sum(0, BX0, s1, 0.f, false, true, mean, dummy);
+                mean *= inv_dv;
+                float s2 = 0.f;
 #pragma unroll
-            for (int j = 0; j < 64; ++j) s1 += y[j];
-            float mean;
-            row_sum(0, BX0, s1, 0.f, false, mean, dummy);
-            mean *= inv_dv;
-            float s2 = 0.f;
-#pragma unroll
-            for (int j = 0; j < 64; ++j) {
-                y[j] -= mean;
-                s2 = fmaf(y[j], y[j], s2);
-            }
-            float var;
-            row_sum(1, BX1, s2, 0.f, false, var, dummy);
-            const float rstd = rsqrtf(var * inv_dv + p.eps);
-            float m1 = 0.f, m2 = 0.f;
-            __nv_bfloat16* dGg = static_cast<__nv_bfloat16*>(p.dG) + rowoff;
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const uint32_t* ge = reinterpret_cast<const uint32_t*>(&gv[k]);
-                const uint32_t* oe = reinterpret_cast<const uint32_t*>(&ov[k]);
-                uint4 dg;
-                uint32_t* dge = reinterpret_cast<uint32_t*>(&dg);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    float out[2];
-#pragma unroll
-                    for (int hf = 0; hf < 2; ++hf) {
-                        const int j = 8 * k + 2 * e + hf;
-                        const float g = hf ? u2f(ge[e] & 0xffff0000u) : u2f(ge[e] << 16);
-                        const float o = hf ? u2f(oe[e] & 0xffff0000u) : u2f(oe[e] << 16);
-                        const float sg = sigmoid_fast(g);
-                        const float n = y[j] * rstd;
-                        y[j] = n;
-                        // d/dg [g sigmoid(g)] = sigmoid(g) (1 + g (1 - sigmoid(g)))
-                        out[hf] = o * n * sg * (1.f + g * (1.f - sg));
-                        const float dn = o * g * sg;
-                        m1 += dn;
-                        m2 = fmaf(dn, n, m2);
-                    }
-                    dge[e] = pack_bf16x2(out[0], out[1]);
+                for (int j = 0; j < 32; ++j) {
+                    y[j] -= mean;
+                    s2 = fmaf(y[j], y[j], s2);
                 }
-                if (t < L) reinterpret_cast<uint4*>(dGg)[k] = dg;
-            }
-            row_sum(2, BX2, m1, m2, true, m1, m2);
-            m1 *= inv_dv;
-            m2 *= inv_dv;
+                float var;
+                row_sum(1, BX1, s2, 0.f, false, true, var, dummy);
+                const float rstd = rsqrtf(var * inv_dv + p.eps);
+                float m1 = 0.f, m2 = 0.f;
+                __nv_bfloat16* dGg = static_cast<__nv_bfloat16*>(p.dG) + rowoff;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const uint32_t* ge = reinterpret_cast<const uint32_t*>(&gv[k]);
-                const uint32_t* oe = reinterpret_cast<const uint32_t*>(&ov[k]);
+                for (int k = 0; k < 4; ++k) {
+                    const uint32_t* ge = reinterpret_cast<const uint32_t*>(&gv[k]);
+                    const uint32_t* oe = reinterpret_cast<const uint32_t*>(&ov[k]);
+                    uint4 dg;
+                    uint32_t* dge = reinterpret_cast<uint32_t*>(&dg);
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
+                    for (int e = 0; e < 4; ++e) {
+                        float out[2];
 #pragma unroll
-                    for (int hf = 0; hf < 2; ++hf) {
-                        const int j = 8 * k + 2 * e + hf;
-                        const float g = hf ? u2f(ge[e] & 0xffff0000u) : u2f(ge[e] << 16);
-                        const float o = hf ? u2f(oe[e] & 0xffff0000u) : u2f(oe[e] << 16);
-                        const float dn = o * g * sigmoid_fast(g);
-                        y[j] = rstd * (dn - m1 - y[j] * m2);
+                        for (int hf = 0; hf < 2; ++hf) {
+                            const int j = 8 * k + 2 * e + hf;
+                            const float g = hf ? u2f(ge[e] & 0xffff0000u) : u2f(ge[e] << 16);
+                            const float o = hf ? u2f(oe[e] & 0xffff0000u) : u2f(oe[e] << 16);
+                            const float sg = sigmoid_fast(g);
+                            const float n = y[j] * rstd;
+                            y[j] = n;
+                            // d/dg [g sigmoid(g)] = sigmoid(g) (1 + g (1 - sigmoid(g)))
+                            out[hf] = o * n * sg * (1.f + g * (1.f - sg));
+                            const float dn = o * g * sg;
+                            m1 += dn;
+                            m2 = fmaf(dn, n, m2);
+                        }
+                        dge[e] = pack_bf16x2(out[0], out[1]);
                     }
-            }
-        } else {
+                    if (t < L) reinterpret_cast<uint4*>(dGg)[k] = dg;
+                }
+                row_sum(2, BX2, m1, m2, true, true, m1, m2);
+                m1 *= inv_dv;
+                m2 *= inv_dv;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const uint32_t* oe = reinterpret_cast<const uint32_t*>(&ov[k]);
+                for (int k = 0; k < 4; ++k) {
+                    const uint32_t* ge = reinterpret_cast<const uint32_t*>(&gv[k]);
+                    const uint32_t* oe = reinterpret_cast<const uint32_t*>(&ov[k]);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    y[8 * k + 2 * e] = u2f(oe[e] << 16);
-                    y[8 * k + 2 * e + 1] = u2f(oe[e] & 0xffff0000u);
+                    for (int e = 0; e < 4; ++e)
+#pragma unroll
+                        for (int hf = 0; hf < 2; ++hf) {
+                            const int j = 8 * k + 2 * e + hf;
+                            const float g = hf ? u2f(ge[e] & 0xffff0000u) : u2f(ge[e] << 16);
+                            const float o = hf ? u2f(oe[e] & 0xffff0000u) : u2f(oe[e] << 16);
+                            const float dn = o * g * sigmoid_fast(g);
+                            y[j] = rstd * (dn - m1 - y[j] * m2);
+                        }
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint32_t* oe = reinterpret_cast<const uint32_t*>(&ov[k]);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        y[8 * k + 2 * e] = u2f(oe[e] << 16);
+                        y[8 * k + 2 * e + 1] = u2f(oe[e] & 0xffff0000u);
+                    }
                 }
             }
-        }
-        // rr_t = dy_t . (e^{b_t} q_t S_c) over this CTA's channels (Yi is still in
-        // tensor memory: G_c overwrites it only after every row warp arrived on BQT)
-        {
-            float rp = 0.f;
-            if (ok_y) {
-                uint32_t ri[32];
-#pragma unroll
-                for (int cb = 0; cb < 2; ++cb) {
-                    tmem_ld_x32(tm + lq + R_YI + 64 * half + 32 * cb, ri);
+            // rr_t = dy_t . (e^{b_t} q_t S_c) over this CTA's channels (Yi is still in
+            // tensor memory: G_c overwrites it only after every row warp arrived on BQT)
+            {
+                float rp = 0.f, dummy;
+                if (ok_y) {
+                    uint32_t ri[32];
+                    tmem_ld_x32(tm + lq + R_YI + 32 * cq, ri);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) rp = fmaf(y[32 * cb + j], u2f(ri[j]), rp);
+                    for (int j = 0; j < 32; ++j) rp = fmaf(y[j], u2f(ri[j]), rp);
+                }
+                float rt;
+                row_sum(3, 0, rp * ebt, 0.f, false, false, rt, dummy);
+                if (cq == 0 && t < L) p.rr[(size_t)rank * p.B * p.N * p.H + (tok0 + t) * p.H + hh] = rt;
+            }
+            // dy as a bf16 pair into the shared-memory tiles (row t, box cq / 2); the
+            // issuer stores the tiles to the workspace
+            {
+                uint8_t* rh = sm + OFF_DYH + (cq >> 1) * kBox;
+                uint8_t* rl = sm + OFF_DYL + (cq >> 1) * kBox;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    uint4 h, l;
+                    split2(y[8 * k], y[8 * k + 1], h.x, l.x);
+                    split2(y[8 * k + 2], y[8 * k + 3], h.y, l.y);
+                    split2(y[8 * k + 4], y[8 * k + 5], h.z, l.z);
+                    split2(y[8 * k + 6], y[8 * k + 7], h.w, l.w);
+                    *reinterpret_cast<uint4*>(rh + sw128(t, 32 * (cq & 1) + 8 * k)) = h;
+                    *reinterpret_cast<uint4*>(rl + sw128(t, 32 * (cq & 1) + 8 * k)) = l;
                 }
             }
-            rp *= ebt;
-            if (half) scr[8 * kC + t] = rp;
-            named_bar_sync(kNamedBar, kRowThreads);
-            if (!half && t < L) p.rr[(size_t)rank * p.B * p.N * p.H + (tok0 + t) * p.H + hh] = rp + scr[8 * kC + t];
-            named_bar_sync(kNamedBar, kRowThreads);   // the scratch is overwritten by dy below
-        }
-        // dy as a bf16 pair into the shared-memory tiles (row t, box `half`); the
-        // issuer stores the tiles to the workspace
-        {
-            uint8_t* rh = sm + OFF_DYH + half * kBox;
-            uint8_t* rl = sm + OFF_DYL + half * kBox;
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                uint4 h, l;
-                split2(y[8 * k], y[8 * k + 1], h.x, l.x);
-                split2(y[8 * k + 2], y[8 * k + 3], h.y, l.y);
-                split2(y[8 * k + 4], y[8 * k + 5], h.z, l.z);
-                split2(y[8 * k + 6], y[8 * k + 7], h.w, l.w);
-                *reinterpret_cast<uint4*>(rh + sw128(t, 8 * k)) = h;
-                *reinterpret_cast<uint4*>(rl + sw128(t, 8 * k)) = l;
-            }
-        }
-        fence_proxy_async_smem();
-        warp_arrive(BDY);
+            fence_proxy_async_smem();
+            warp_arrive(BDY);
 
-        // ---------------------------------------------------- Q~^T = (diag(e^{b}) Q)^T as a bf16 pair
-        if (ok_y) {
-            const int d = 32 * q + lane;
-            const uint8_t* qb = sm + OFF_Q + (q >> 1) * kBox;
-            const int xq = 32 * (q & 1) + lane;
-            uint32_t hi[32], lo[32];
+            // ------------------------------------------------ Q~^T = (diag(e^{b}) Q)^T as a bf16 pair
+            if (ok_y) {
+                const uint8_t* qb = sm + OFF_Q + (q >> 1) * kBox;
+                const int xq = 32 * (q & 1) + lane;   // column d = 32 q + lane of Q
+                uint32_t hi[16], lo[16];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int t0 = 64 * half + 2 * j;
-                const float x0 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(qb + sw128(t0, xq)));
-                const float x1 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(qb + sw128(t0 + 1, xq)));
-                split2(x0 * __expf(bc[t0]), x1 * __expf(bc[t0 + 1]), hi[j], lo[j]);
+                for (int j = 0; j < 16; ++j) {
+                    const int t0 = 32 * cq + 2 * j;
+                    const float x0 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(qb + sw128(t0, xq)));
+                    const float x1 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(qb + sw128(t0 + 1, xq)));
+                    split2(x0 * __expf(bc[t0]), x1 * __expf(bc[t0 + 1]), hi[j], lo[j]);
+                }
+                tmem_st_x16(tm + lq + R_P + 16 * cq, hi);
+                tmem_st_x16(tm + lq + R_P + 64 + 16 * cq, lo);
+                tmem_wait_st();
             }
-            (void)d;
-            tmem_st_x32(tm + lq + R_P + 32 * half, hi);
-            tmem_st_x32(tm + lq + R_P + 64 + 32 * half, lo);
-            tmem_wait_st();
-        }
-        tc_fence_before();
-        warp_arrive(BQT);
+            tc_fence_before();
+            warp_arrive(BQT);
 
-        // ---------------------------------------------------- D o E (bf16) and e^{b_t} dy S^T
-        if (mbar_wait(bar(BD), 0, p.status, abort_flag)) {
-            tc_fence_after();
-            uint32_t r[64], pk[32];
-            tmem_ld_x32(tm + lq + R_A + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(r));
-            tmem_ld_x32(tm + lq + R_A + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int s0 = 64 * half + 2 * j;
-                const float v0 = s0 <= t ? u2f(r[2 * j]) * __expf(fminf(bt - bc[s0], 0.f)) : 0.f;
-                const float v1 = s0 + 1 <= t ? u2f(r[2 * j + 1]) * __expf(fminf(bt - bc[s0 + 1], 0.f)) : 0.f;
-                pk[j] = pack_bf16x2(v0, v1);
-            }
-            // every row warp has read D before D o E overwrites its first 64 columns
-            named_bar_sync(kNamedBar, kRowThreads);
-            tmem_st_x32(tm + lq + R_A + 32 * half, pk);
-            if (mbar_wait(bar(BQI), 0, p.status, abort_flag)) {
+            // ------------------------------------------------ D o E (bf16) and e^{b_t} dy S^T
+            if (mbar_wait(bar(BD), par, p.status, abort_flag)) {
                 tc_fence_after();
+                uint32_t r[32], pk[16];
+                tmem_ld_x32(tm + lq + R_A + 32 * cq, r);
+                tmem_wait_ld();
 #pragma unroll
-                for (int cb = 0; cb < 2; ++cb) {
+                for (int j = 0; j < 16; ++j) {
+                    const int s0 = 32 * cq + 2 * j;
+                    const float v0 = s0 <= t ? u2f(r[2 * j]) * __expf(fminf(bt - bc[s0], 0.f)) : 0.f;
+                    const float v1 = s0 + 1 <= t ? u2f(r[2 * j + 1]) * __expf(fminf(bt - bc[s0 + 1], 0.f)) : 0.f;
+                    pk[j] = pack_bf16x2(v0, v1);
+                }
+                // every row warp has read D before D o E overwrites its first 64 columns
+                named_bar_sync(kNamedBar, RT);
+                tmem_st_x16(tm + lq + R_A + 16 * cq, pk);
+                if (mbar_wait(bar(BQI), par, p.status, abort_flag)) {
+                    tc_fence_after();
                     uint32_t v[32];
-                    tmem_ld_x32(tm + lq + R_Y + 64 * half + 32 * cb, v);
+                    tmem_ld_x32(tm + lq + R_Y + 32 * cq, v);
                     tmem_wait_ld();
 #pragma unroll
                     for (int j = 0; j < 32; ++j) v[j] = f2u(u2f(v[j]) * ebt);
-                    tmem_st_x32(tm + lq + R_Y + 64 * half + 32 * cb, v);
+                    tmem_st_x32(tm + lq + R_Y + 32 * cq, v);
                 }
+                tmem_wait_st();
+            } else {
+                named_bar_sync(kNamedBar, RT);
             }
-            tmem_wait_st();
-        } else {
-            named_bar_sync(kNamedBar, kRowThreads);
-        }
-        tc_fence_before();
-        warp_arrive(BDS);
+            tc_fence_before();
+            warp_arrive(BDS);
 
-        // ---------------------------------------------------- G_c rows (lane = d_k row)
-        if (mbar_wait(bar(BGC), 0, p.status, abort_flag)) {
-            tc_fence_after();
-            float* dst = p.incg + (((size_t)u * nc + c) * kDK + t) * DV + ch0 + 64 * half;
-#pragma unroll 1
-            for (int cb = 0; cb < 2; ++cb) {
+            // ------------------------------------------------ G_c rows (lane = d_k row)
+            if (mbar_wait(bar(BGC), par, p.status, abort_flag)) {
+                tc_fence_after();
+                float* dst = p.incg + (((size_t)u * nc + c) * kDK + t) * DV + ch0 + 32 * cq;
                 uint32_t v[32];
-                tmem_ld_x32(tm + lq + R_YI + 64 * half + 32 * cb, v);
+                tmem_ld_x32(tm + lq + R_YI + 32 * cq, v);
                 tmem_wait_ld();
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    reinterpret_cast<float4*>(dst + 32 * cb)[k] =
+                    reinterpret_cast<float4*>(dst)[k] =
                         make_float4(u2f(v[4 * k]), u2f(v[4 * k + 1]), u2f(v[4 * k + 2]), u2f(v[4 * k + 3]));
             }
-        }
-        // ---------------------------------------------------- dq (this CTA's channel half)
-        if (mbar_wait(bar(BDQ), 0, p.status, abort_flag)) {
-            tc_fence_after();
-#pragma unroll
-            for (int cb = 0; cb < 2; ++cb) {
+            // ------------------------------------------------ dq (this CTA's channel half)
+            float dq[32];
+            if (mbar_wait(bar(BDQ), par, p.status, abort_flag)) {
+                tc_fence_after();
                 uint32_t v[32];
-                tmem_ld_x32(tm + lq + R_Y + 64 * half + 32 * cb, v);
+                tmem_ld_x32(tm + lq + R_Y + 32 * cq, v);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) dq[32 * cb + j] = u2f(v[j]);
-            }
-        } else {
+                for (int j = 0; j < 32; ++j) dq[j] = u2f(v[j]);
+            } else {
 #pragma unroll
-            for (int j = 0; j < 64; ++j) dq[j] = 0.f;
+                for (int j = 0; j < 32; ++j) dq[j] = 0.f;
+            }
+            tc_fence_before();
+            warp_arrive(BEND);   // this chunk's tensor memory has been read
+            // the dy tiles have been stored (and read by every product of the chunk)
+            mbar_wait(bar(BDYRD), par, p.status, abort_flag);
+            bool mine = true;
+            if constexpr (PAIR) {
+                // rows of the other CTA's half leave in one bulk copy, staged in the dy
+                // lo tile ([64 rows][128] fp32, 16-byte chunks swizzled by row) and
+                // received in the other CTA's dy hi tile
+                float* stage = reinterpret_cast<float*>(sm + OFF_DYL);
+                const float* recv = reinterpret_cast<const float*>(sm + OFF_DYH);
+                const int r = t & 63;
+                mine = (t >> 6) == rank;
+                if (!mine)
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        reinterpret_cast<float4*>(stage + r * 128)[8 * cq + (k ^ (r & 7))] =
+                            make_float4(dq[4 * k], dq[4 * k + 1], dq[4 * k + 2], dq[4 * k + 3]);
+                fence_proxy_async_smem();
+                named_bar_sync(kNamedBar, RT);
+                cluster_sync_all();   // both CTAs are past the chunk's last product
+                if (tid == 0) {
+                    bulk_copy_to_cluster(cluster_map(sb + OFF_DYH, peer), sb + OFF_DYL, 64 * 128 * 4,
+                                         cluster_map(bar(BXQ), peer));
+                    bulk_commit();
+                }
+                if (mine && mbar_wait_cluster(bar(BXQ), par, p.status, abort_flag)) {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const float4 x = reinterpret_cast<const float4*>(recv + r * 128)[8 * cq + (k ^ (r & 7))];
+                        dq[4 * k] += x.x;
+                        dq[4 * k + 1] += x.y;
+                        dq[4 * k + 2] += x.z;
+                        dq[4 * k + 3] += x.w;
+                    }
+                }
+                if (tid == 0) bulk_wait_read<0>();   // the staging tile is read before dy is written again
+            }
+            if (mine && t < L) {
+                uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dQ) +
+                                                      ((tok0 + t) * p.H + hh) * kDK + 32 * cq);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    dst[k] = make_uint4(pack_bf16x2(dq[8 * k], dq[8 * k + 1]), pack_bf16x2(dq[8 * k + 2], dq[8 * k + 3]),
+                                        pack_bf16x2(dq[8 * k + 4], dq[8 * k + 5]),
+                                        pack_bf16x2(dq[8 * k + 6], dq[8 * k + 7]));
+            }
         }
-    } else if (lane == 0) {
-        // ============================================================ TMA + MMA issuer
+    } else {
+        // ============================================================ TMA + MMA issuer (lane 0)
         constexpr uint32_t id_kk = idesc_bf16(128, 128, false, false);
         constexpr uint32_t id_kn = idesc_bf16(128, 128, false, true);
         auto kmaj = [&](uint32_t base, int k) { return sdesc_sw128(base + (k >> 2) * kBox + (k & 3) * 32, 16, 1024); };
         auto mnmaj = [&](uint32_t base, int k) { return sdesc_sw128(base + k * 2048, kBox, 1024); };
-        const int srow = (u * nc + c) * kDK;
-        mbar_arrive_expect_tx(bar(BQK), 2 * kTile);
-        for (int x = 0; x < 2; ++x) {
-            tma_load_4d(sb + OFF_Q + x * kBox, &p.tmQ, x * 64, hh, n0, b, bar(BQK));
-            tma_load_4d(sb + OFF_K + x * kBox, &p.tmK, x * 64, hh, n0, b, bar(BQK));
-        }
-        mbar_arrive_expect_tx(bar(BVS), 3 * kTile);
-        for (int x = 0; x < 2; ++x) {
-            tma_load_4d(sb + OFF_V + x * kBox, &p.tmV, ch0 + x * 64, hh, n0, b, bar(BVS));
-            tma_load_2d(sb + OFF_SH + x * kBox, &p.tmSH, ch0 + x * 64, srow, bar(BVS));
-            tma_load_2d(sb + OFF_SL + x * kBox, &p.tmSL, ch0 + x * 64, srow, bar(BVS));
-        }
-        bool ok = mbar_wait(bar(BQK), 0, p.status, abort_flag);
-        if (ok) {
-            tc_fence_after();
-            // scores A = Q K^T
-#pragma unroll
-            for (int k = 0; k < 8; ++k) mma_ss(tm + R_A, kmaj(sb + OFF_Q, k), kmaj(sb + OFF_K, k), id_kk, k > 0);
-        }
-        mma_commit(bar(BA));
-        ok = ok && mbar_wait(bar(BVS), 0, p.status, abort_flag);
-        if (ok) {
-            tc_fence_after();
-            // Yi = Q S_c (S as a bf16 pair)
-            for (int pass = 0; pass < 2; ++pass)
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mma_ss(tm + R_YI, kmaj(sb + OFF_Q, k), mnmaj(sb + (pass ? OFF_SL : OFF_SH), k), id_kn,
-                           pass > 0 || k > 0);
-        }
-        mma_commit(bar(BYI));
-        ok = ok && mbar_wait(bar(BP), 0, p.status, abort_flag);
-        if (ok) {
-            tc_fence_after();
-            // Y = P V
-#pragma unroll
-            for (int k = 0; k < 8; ++k) mma_ts(tm + R_Y, tm + R_P + k * 8, mnmaj(sb + OFF_V, k), id_kn, k > 0);
-        }
-        mma_commit(bar(BY));
-        ok = ok && mbar_wait(bar(BDY), 0, p.status, abort_flag);
-        if (ok) {
-            // dy (both halves of the pair) to the workspace; rows past the end of the
-            // sequence fall outside the tensor map and are not written
+        auto coords = [&](int it, int& n0, int& b, int& hh, int& srow) {
+            const int item = cid + it * ncl, u = item / nc, c = item - u * nc;
+            b = u / p.H;
+            hh = u - b * p.H;
+            n0 = c * kC;
+            srow = (u * nc + c) * kDK;
+        };
+        auto load_tile = [&](int it, int bi, const CUtensorMap* m, uint32_t off, int x0) {
+            int n0, b, hh, srow;
+            coords(it, n0, b, hh, srow);
+            mbar_arrive_expect_tx(bar(bi), kTile);
+            for (int x = 0; x < 2; ++x) tma_load_4d(sb + off + x * kBox, m, x0 + x * 64, hh, n0, b, bar(bi));
+        };
+        auto load_s = [&](int it) {
+            int n0, b, hh, srow;
+            coords(it, n0, b, hh, srow);
+            mbar_arrive_expect_tx(bar(BS), 2 * kTile);
             for (int x = 0; x < 2; ++x) {
-                tma_store_4d(&p.tmDyH, sb + OFF_DYH + x * kBox, ch0 + x * 64, hh, n0, b);
-                tma_store_4d(&p.tmDyL, sb + OFF_DYL + x * kBox, ch0 + x * 64, hh, n0, b);
+                tma_load_2d(sb + OFF_SH + x * kBox, &p.tmSH, ch0 + x * 64, srow, bar(BS));
+                tma_load_2d(sb + OFF_SL + x * kBox, &p.tmSL, ch0 + x * 64, srow, bar(BS));
             }
-            bulk_commit();
-            tc_fence_after();
-            // D = dy V^T (dy as a bf16 pair)
-            for (int pass = 0; pass < 2; ++pass)
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mma_ss(tm + R_A, kmaj(sb + (pass ? OFF_DYL : OFF_DYH), k), kmaj(sb + OFF_V, k), id_kk,
-                           pass > 0 || k > 0);
+        };
+        if (lane == 0 && niter > 0) {
+            load_tile(0, BQ, &p.tmQ, OFF_Q, 0);
+            load_tile(0, BK, &p.tmK, OFF_K, 0);
+            load_tile(0, BV, &p.tmV, OFF_V, ch0);
+            load_s(0);
         }
-        mma_commit(bar(BD));
-        if (ok) {
-            // dy S^T: hi hi + hi lo + lo hi
-            for (int pass = 0; pass < 3; ++pass)
+        for (int it = 0; it < niter; ++it) {
+            const uint32_t par = it & 1;
+            const bool more = it + 1 < niter;
+            if (lane == 0) {
+                bool ok = mbar_wait(bar(BQ), par, p.status, abort_flag) && mbar_wait(bar(BK), par, p.status, abort_flag);
+                // the rows have read the previous chunk's tensor memory
+                ok = ok && (it == 0 || mbar_wait(bar(BEND), par ^ 1, p.status, abort_flag));
+                if (ok) {
+                    tc_fence_after();
+                    // scores A = Q K^T
 #pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mma_ss(tm + R_Y, kmaj(sb + (pass == 2 ? OFF_DYL : OFF_DYH), k),
-                           kmaj(sb + (pass == 1 ? OFF_SL : OFF_SH), k), id_kk, pass > 0 || k > 0);
-        }
-        mma_commit(bar(BQI));
-        ok = ok && mbar_wait(bar(BQT), 0, p.status, abort_flag);
-        if (ok) {
-            tc_fence_after();
-            // G_c = Q~^T dy: A = Q~^T from tensor memory (lane = d_k row), B = dy MN-major
-            for (int pass = 0; pass < 3; ++pass)
+                    for (int k = 0; k < 8; ++k) mma_ss(tm + R_A, kmaj(sb + OFF_Q, k), kmaj(sb + OFF_K, k), id_kk, k > 0);
+                }
+                mma_commit(bar(BA));
+                ok = ok && mbar_wait(bar(BS), par, p.status, abort_flag);
+                if (ok) {
+                    tc_fence_after();
+                    // Yi = Q S_c (S as a bf16 pair)
+                    for (int pass = 0; pass < 2; ++pass)
 #pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mma_ts(tm + R_YI, tm + R_P + (pass == 2 ? 64 : 0) + k * 8,
-                           mnmaj(sb + (pass == 1 ? OFF_DYL : OFF_DYH), k), id_kn, pass > 0 || k > 0);
-        }
-        mma_commit(bar(BGC));
-        ok = ok && mbar_wait(bar(BDS), 0, p.status, abort_flag);
-        if (ok) {
-            tc_fence_after();
-            // dq += (D o E) K
+                        for (int k = 0; k < 8; ++k)
+                            mma_ss(tm + R_YI, kmaj(sb + OFF_Q, k), mnmaj(sb + (pass ? OFF_SL : OFF_SH), k), id_kn,
+                                   pass > 0 || k > 0);
+                }
+                mma_commit(bar(BYI));
+                ok = ok && mbar_wait(bar(BP), par, p.status, abort_flag) && mbar_wait(bar(BV), par, p.status, abort_flag);
+                if (ok) {
+                    tc_fence_after();
+                    // Y = P V
 #pragma unroll
-            for (int k = 0; k < 8; ++k) mma_ts(tm + R_Y, tm + R_A + k * 8, mnmaj(sb + OFF_K, k), id_kn, 1);
-        }
-        mma_commit(bar(BDQ));
-        mma_commit(bar(BDRAIN));
-        mbar_wait_drain(bar(BDRAIN), 0, kWaitCycles);
-        bulk_wait<0>();   // the dy tiles are read before the CTA leaves
-        if (*abort_flag) {
-            mbar_wait_drain(bar(BQK), 0, kWaitCycles);
-            mbar_wait_drain(bar(BVS), 0, kWaitCycles);
-        }
-    }
-    __syncwarp();
-    // ---------------------------------------------------------------- dq rows
-    if constexpr (PAIR) cluster_sync_all();   // both CTAs are past their last MMA: the S tiles are free
-    if (tid < kRowThreads) {
-        const int q = warp & 3, half = warp >> 2, t = 32 * q + lane;
-        float* recv = reinterpret_cast<float*>(sm + OFF_SH);   // [64 rows][128] partials from the other CTA
-        bool mine = true;
-        if constexpr (PAIR) {
-            const int owner = t >> 6;
-            mine = owner == rank;
-            if (!mine) {
-                const uint32_t remote = cluster_map(smem_u32(recv + (t & 63) * 128 + 64 * half), peer);
-                const uint32_t rbar = cluster_map(bar(BXQ), peer);
+                    for (int k = 0; k < 8; ++k) mma_ts(tm + R_Y, tm + R_P + k * 8, mnmaj(sb + OFF_V, k), id_kn, k > 0);
+                }
+                mma_commit(bar(BY));
+                ok = ok && mbar_wait(bar(BDY), par, p.status, abort_flag);
+                if (ok) {
+                    // dy (both halves of the pair) to the workspace; rows past the end of
+                    // the sequence fall outside the tensor map and are not written
+                    int n0, b, hh, srow;
+                    coords(it, n0, b, hh, srow);
+                    for (int x = 0; x < 2; ++x) {
+                        tma_store_4d(&p.tmDyH, sb + OFF_DYH + x * kBox, ch0 + x * 64, hh, n0, b);
+                        tma_store_4d(&p.tmDyL, sb + OFF_DYL + x * kBox, ch0 + x * 64, hh, n0, b);
+                    }
+                    bulk_commit();
+                    tc_fence_after();
+                    // D = dy V^T (dy as a bf16 pair)
+                    for (int pass = 0; pass < 2; ++pass)
 #pragma unroll
-                for (int k = 0; k < 16; ++k)
-                    st_async_f4(remote + 16 * k, rbar, dq[4 * k], dq[4 * k + 1], dq[4 * k + 2], dq[4 * k + 3]);
-            } else if (mbar_wait_cluster(bar(BXQ), 0, p.status, abort_flag)) {
-                const float* src = recv + (t & 63) * 128 + 64 * half;
+                        for (int k = 0; k < 8; ++k)
+                            mma_ss(tm + R_A, kmaj(sb + (pass ? OFF_DYL : OFF_DYH), k), kmaj(sb + OFF_V, k), id_kk,
+                                   pass > 0 || k > 0);
+                }
+                mma_commit(bar(BD));
+                if (ok) {
+                    // dy S^T: hi hi + hi lo + lo hi
+                    for (int pass = 0; pass < 3; ++pass)
 #pragma unroll
-                for (int j = 0; j < 64; ++j) dq[j] += src[j];
+                        for (int k = 0; k < 8; ++k)
+                            mma_ss(tm + R_Y, kmaj(sb + (pass == 2 ? OFF_DYL : OFF_DYH), k),
+                                   kmaj(sb + (pass == 1 ? OFF_SL : OFF_SH), k), id_kk, pass > 0 || k > 0);
+                }
+                mma_commit(bar(BQI));
+                // V is free after D, S after dy S^T: the next chunk's tiles may load
+                if (mbar_wait(bar(BD), par, p.status, abort_flag) && more) load_tile(it + 1, BV, &p.tmV, OFF_V, ch0);
+                if (mbar_wait(bar(BQI), par, p.status, abort_flag) && more) load_s(it + 1);
+                ok = ok && mbar_wait(bar(BQT), par, p.status, abort_flag);
+                // Q is free once the rows have built Q~^T
+                if (ok && more) load_tile(it + 1, BQ, &p.tmQ, OFF_Q, 0);
+                if (ok) {
+                    tc_fence_after();
+                    // G_c = Q~^T dy: A = Q~^T from tensor memory (lane = d_k row), B = dy MN-major
+                    for (int pass = 0; pass < 3; ++pass)
+#pragma unroll
+                        for (int k = 0; k < 8; ++k)
+                            mma_ts(tm + R_YI, tm + R_P + (pass == 2 ? 64 : 0) + k * 8,
+                                   mnmaj(sb + (pass == 1 ? OFF_DYL : OFF_DYH), k), id_kn, pass > 0 || k > 0);
+                }
+                mma_commit(bar(BGC));
+                ok = ok && mbar_wait(bar(BDS), par, p.status, abort_flag);
+                if (ok) {
+                    tc_fence_after();
+                    // dq += (D o E) K
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) mma_ts(tm + R_Y, tm + R_A + k * 8, mnmaj(sb + OFF_K, k), id_kn, 1);
+                }
+                mma_commit(bar(BDQ));
+                // K is free after the last product
+                if (mbar_wait(bar(BDQ), par, p.status, abort_flag) && more) load_tile(it + 1, BK, &p.tmK, OFF_K, 0);
+                bulk_wait_read<0>();   // the dy store has read its tiles
+                mbar_arrive(bar(BDYRD));
+            }
+            __syncwarp();
+            if constexpr (PAIR) {
+                cluster_sync_all();
+                // the next chunk's exchanges, once this chunk's dq has arrived
+                if (lane == 0 && more && mbar_wait_cluster(bar(BXQ), par, p.status, abort_flag)) arm_exchange();
+                __syncwarp();
             }
         }
-        if (mine && t < L) {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dQ) + ((tok0 + t) * p.H + hh) * kDK +
-                                                  64 * half);
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-                dst[k] = make_uint4(pack_bf16x2(dq[8 * k], dq[8 * k + 1]), pack_bf16x2(dq[8 * k + 2], dq[8 * k + 3]),
-                                    pack_bf16x2(dq[8 * k + 4], dq[8 * k + 5]), pack_bf16x2(dq[8 * k + 6], dq[8 * k + 7]));
+        if (lane == 0) {
+            mma_commit(bar(BDRAIN));
+            mbar_wait_drain(bar(BDRAIN), 0, kWaitCycles);
+            bulk_wait<0>();
         }
+        __syncwarp();
     }
     tc_fence_before();
     __syncthreads();
     if constexpr (PAIR) cluster_sync_all();   // no CTA leaves while the other still sends to it
-    if (warp == kRowThreads / 32) tmem_dealloc(tm, 512);
+    if (warp == RT / 32) tmem_dealloc(tm, 512);
 }
 
 // Sum of v[0..31] over the warp's lanes for each of the 32 columns at once:
@@ -897,9 +945,6 @@ __device__ __forceinline__ float transpose_reduce32(float (&v)[32], int lane) {
 // Tensor memory: [0,128) A^T, then (A o E)^T (bf16); [128,256) D^T, then
 // (D o E)^T; [256,384) V dS'^T, scaled, + (D o E)^T Q; [384,512) K dS',
 // scaled, + (A o E)^T dy.  Shared tiles: Q, K, V, dy hi, dy lo, dS' hi, dS' lo.
-constexpr int kRowThreads16 = 512;   // sixteen row warps: lane quarter q = w & 3, column quarter w >> 2
-constexpr int kThreads16 = kRowThreads16 + 32;
-
 template <bool PAIR>
 __global__ void __launch_bounds__(kThreads16, 1) bwd_kv_tc(const __grid_constant__ BwdTcParams p) {
     using CF = GradCfg;
@@ -1429,14 +1474,15 @@ cudaError_t run_bwd_tc(BwdTcParams& p, cudaStream_t s) {
     const dim3 sgrid((unsigned)((kDK * DV / 4 + kScanThreads - 1) / kScanThreads), (unsigned)(p.B * p.H));
     k1<<<items * (DV / 128), kThreads, IncCfg::SMEM, s>>>(p);
     bwd_scan_fwd<<<sgrid, kScanThreads, 0, s>>>(p);
-    if ((e = launch_cluster(k3, items * (PAIR ? 2 : 1), PAIR ? 2 : 1, GradCfg::SMEM, s, kThreads, p)) != cudaSuccess)
-        return e;
-    bwd_scan_rev<<<sgrid, kScanThreads, 0, s>>>(p);
-    // dk/dv/dz: persistent, one CTA (pair) per SM (pair of SMs)
     int dev = 0, sms = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    // the two gradient kernels are persistent: one CTA (pair) per SM (pair of SMs)
     const unsigned ncl = std::min<unsigned>(items, (unsigned)std::max(1, PAIR ? sms / 2 : sms));
+    if ((e = launch_cluster(k3, ncl * (PAIR ? 2 : 1), PAIR ? 2 : 1, GradCfg::SMEM, s, kThreads16, p)) !=
+        cudaSuccess)
+        return e;
+    bwd_scan_rev<<<sgrid, kScanThreads, 0, s>>>(p);
     if ((e = launch_cluster(k5, ncl * (PAIR ? 2 : 1), PAIR ? 2 : 1, GradCfg::SMEM, s, kThreads16, p)) !=
         cudaSuccess)
         return e;
