@@ -658,9 +658,7 @@ def backward_alg(cfg):
 
 
 # chunk length of the backward (bf16 inputs); the flop count below depends on it
-BACKWARD_CHUNK = 64
-# tf32 / bf16 dense tensor peak (nominal 1.1 / 2.25 PFLOP/s per GPU)
-TF32_OVER_BF16 = 1.1 / 2.25
+BACKWARD_CHUNK = 128
 
 
 def backward_alg_flops(cfg, chunk=BACKWARD_CHUNK):
@@ -678,15 +676,15 @@ def backward_summary(cfg, steps, ms, world, peaks, launches_per_call):
     flops = backward_alg_flops(cfg)
     step_s = ms / 1e3 / steps
     tflops = flops / step_s / 1e12
-    peak = peaks["bf16_tflops"] * TF32_OVER_BF16
+    peak = peaks["bf16_tflops"]
     return {"workload": cfg.name, "steps": steps, "warmup": 2, "ms_per_step": ms / steps,
             "value": job_throughput(world, cfg.B * cfg.N, steps, ms) / 1e6, "unit": "Mtok/s",
-            "kernels": "bwd_inc_mma, bwd_fwd_scan, bwd_dy_mma, bwd_rev_scan, bwd_grad_mma "
-                       "(mma.sync m16n8k8 tf32 with split operands, fp32 accumulation)",
-            "roofline": {"kernel": "whole backward (5 launches)", "bound": "tensor", "achieved": tflops,
+            "kernels": "bwd_inc_tc, bwd_scan_fwd, bwd_dyq_tc, bwd_scan_rev, bwd_kv_tc, bwd_dz "
+                       "(tcgen05 kind::f16, states and dy as bf16 pairs, fp32 accumulation in tensor memory)",
+            "roofline": {"kernel": "whole backward (6 launches)", "bound": "tensor", "achieved": tflops,
                          "peak": peak, "unit": "TFLOP/s", "frac": tflops / peak, "traffic": None,
                          "alg_flops_per_call": flops,
-                         "peak_source": peaks["source"] + " bf16 burst x nominal tf32/bf16 ratio"},
+                         "peak_source": peaks["source"] + " bf16 burst"},
             "path_hbm": {"alg_bytes": bytes_, "alg_gbs": bytes_ / step_s / 1e9,
                          "frac": bytes_ / step_s / 1e9 / peaks["hbm_gbs"]},
             "gpu_launches": launches_per_call * steps}

@@ -3,9 +3,12 @@
 
 Cases: the fp32 path (1e-4 of max|ref|) with an initial state and a gradient
 on the final state, both epilogues, ragged chunk tails; bf16 inputs and
-gradients at the benchmark's head sizes (bf16 tolerance) over one and several
-chunks; a gate-stress mix of fast- and slow-decaying heads; head sizes that are
-not multiples of 32 (the serial path)."""
+gradients at the benchmark's head sizes on the tensor-core path (bf16
+tolerance; d_v 256 runs on CTA pairs, d_v 128 on single CTAs) over one and
+several chunks, and the benchmark's full length on sampled units; a
+gate-stress mix of fast- and slow-decaying heads; bf16 with d_k 64 (the
+CUDA-core chunk kernels); head sizes that are not multiples of 32 (the serial
+path)."""
 import numpy as np
 import pytest
 import torch
@@ -89,7 +92,7 @@ def test_serial_path_odd_head_sizes(io):
 
 
 def test_bf16_tensor_core_path_prenorm():
-    # d_k 128 bf16 takes the mma.sync kernels; the plain epilogue (dy = dO)
+    # d_k 128 bf16 takes the tensor-core (tcgen05) kernels; the plain epilogue (dy = dO)
     _run(gi.C2.scaled(B=1, H=2, N=200, seed=78), epilogue="none")
 
 
@@ -125,3 +128,43 @@ def test_bf16_full_benchmark_length_sampled_units():
             assert_close(u(got[name]), ref[name], "bf16", f"{name} unit {(b, h)}")
         assert_close(got["dz"][b:b + 1, :, h:h + 1], ref["dz"], "bf16", f"dz unit {(b, h)}")
         assert_close(got["dS0"][b:b + 1, h:h + 1], ref["dS0"], "bf16", f"dS0 unit {(b, h)}")
+
+
+def _sampled_units(cfg, units, seed_s0=911):
+    """The whole backward of cfg on the GPU; the listed (batch, head) units
+    against the oracle run on that unit alone."""
+    inp = gi.prefill_inputs(cfg)
+    shape_o = (cfg.B, cfg.N, cfg.H, cfg.dv)
+    shape_s = (cfg.B, cfg.H, cfg.dk, cfg.dv)
+    dO = gi.random_unit(cfg.seed, 910, shape_o, io=cfg.io)
+    S0 = gi.random_unit(cfg.seed, seed_s0, shape_s, var=0.04)
+    dSf = gi.random_unit(cfg.seed, 912, shape_s, var=0.01)
+    d = {k: v.cuda() for k, v in inp.items()}
+    got = gret.prefill_backward(d["Q"], d["K"], d["V"], d["z"], d["G"], dO.cuda(), cfg.tau, eps=cfg.eps,
+                                S0=S0.cuda(), dS_final=dSf.cuda())
+    gret.check_device_status()
+    for b, h in units:
+        u = lambda x: x[b:b + 1, :, h:h + 1]  # noqa: E731
+        ref = og.prefill_backward(u(inp["Q"]), u(inp["K"]), u(inp["V"]), u(inp["z"]), u(inp["G"]), cfg.tau,
+                                  cfg.eps, u(dO), S0=S0[b:b + 1, h:h + 1], dS_final=dSf[b:b + 1, h:h + 1])
+        for name in ("dQ", "dK", "dV", "dG"):
+            assert_close(u(got[name]), ref[name], "bf16", f"{name} unit {(b, h)}")
+        assert_close(got["dz"][b:b + 1, :, h:h + 1], ref["dz"], "bf16", f"dz unit {(b, h)}")
+        assert_close(got["dS0"][b:b + 1, h:h + 1], ref["dS0"], "bf16", f"dS0 unit {(b, h)}")
+
+
+@pytest.mark.slow
+def test_bf16_dv128_more_chunks_than_ctas():
+    """d_v 128 (one CTA per chunk): 2 heads x 81 chunks of a ragged 10300-token
+    sequence are more chunks than SMs, so the persistent gradient kernels take
+    several chunks each; fast-decaying gates."""
+    cfg = gi.C2.scaled(B=1, H=2, N=10300, dv=128, seed=81, z_dist=((-2.0, 1.0),))
+    _sampled_units(cfg, [(0, 1)])
+
+
+@pytest.mark.slow
+def test_bf16_dv256_pairs_more_chunks_than_pairs():
+    """d_v 256 (a CTA pair per chunk): 3 heads x 26 chunks of a 3288-token
+    sequence (the last chunk 88 tokens) are more chunks than SM pairs."""
+    cfg = gi.C2.scaled(B=1, H=3, N=3288, seed=82)
+    _sampled_units(cfg, [(0, 0), (0, 2)])
