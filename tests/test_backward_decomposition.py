@@ -102,6 +102,7 @@ def _chunked_backward(Q, K, V, z, G, dO, tau, eps, S0, dSf, C, gn):
     (2, 16, 1, 3, 5, 4, False),     # plain epilogue, chunks that divide N
     (1, 70, 1, 8, 8, 64, True),     # one full chunk and a short one
     (1, 9, 1, 2, 3, 16, True),      # a single partial chunk
+    (1, 300, 1, 8, 8, 128, True),   # the tensor-core kernels' chunk: two full chunks and a 44-token one
 ])
 def test_chunk_decomposition_matches_the_oracle(B, N, H, dk, dv, C, gn):
     rng = np.random.default_rng(100 + N)
