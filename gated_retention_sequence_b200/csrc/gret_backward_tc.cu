@@ -67,6 +67,7 @@ constexpr int kThreads16 = kRowThreads16 + 32;
 
 struct BwdTcParams {
     CUtensorMap tmQ, tmK, tmV, tmDyH, tmDyL, tmSH, tmSL;
+    CUtensorMap tmInc;        // incg as [rows][dv] fp32, box (32, 128): stores of state-shaped rows
     const void *Q, *K, *V, *G, *dO;
     const float *z, *S0, *dS_final;
     void *dQ, *dK, *dV, *dG;
@@ -238,22 +239,26 @@ __global__ void __launch_bounds__(kThreads, 2) bwd_inc_tc(const __grid_constant_
         }
         mma_commit(bar_mma);
     }
-    // store: row d of the increment (TMEM lane d), 64 columns per thread
+    // store: row d of the increment (TMEM lane d), 64 columns per thread, staged
+    // in the dead K~ tiles as four [128][32] fp32 boxes in the 128-byte swizzle
+    // layout and stored by TMA (rows of 512 bytes, written whole)
+    const bool stored = mbar_wait(bar_mma, 0, p.status, abort_flag) && need;
     if (tid < kRowThreads) {
         const int q = warp & 3, half = warp >> 2, d = 32 * q + lane;
-        if (mbar_wait(bar_mma, 0, p.status, abort_flag) && need) {
+        if (stored) {
             tc_fence_after();
-            float* dst = p.incg + (((size_t)u * nc + c) * kDK + d) * p.dv + ch0 + 64 * half;
 #pragma unroll 1
             for (int cb = 0; cb < 2; ++cb) {
                 uint32_t r[32];
                 tmem_ld_x32(tm + ((uint32_t)(32 * q) << 16) + 64 * half + cb * 32, r);
                 tmem_wait_ld();
+                uint8_t* box = sm + (2 * half + cb) * kBox;   // [128 rows][32 fp32] = 16 KB
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    reinterpret_cast<float4*>(dst + cb * 32)[k] =
-                        make_float4(u2f(r[4 * k]), u2f(r[4 * k + 1]), u2f(r[4 * k + 2]), u2f(r[4 * k + 3]));
+                    *reinterpret_cast<uint4*>(box + d * 128 + ((k ^ (d & 7)) << 4)) =
+                        make_uint4(r[4 * k], r[4 * k + 1], r[4 * k + 2], r[4 * k + 3]);
             }
+            fence_proxy_async_smem();
         }
     } else if (lane == 0 && *abort_flag) {
         if (need) mbar_wait_drain(bar_ld, 0, kWaitCycles);
@@ -261,6 +266,12 @@ __global__ void __launch_bounds__(kThreads, 2) bwd_inc_tc(const __grid_constant_
     }
     tc_fence_before();
     __syncthreads();
+    if (tid == 0 && stored) {
+        const int row0 = (u * nc + c) * kDK;
+        for (int x = 0; x < 4; ++x) tma_store_2d(&p.tmInc, sb + x * kBox, ch0 + 32 * x, row0);
+        bulk_commit();
+        bulk_wait<0>();
+    }
     if (warp == kRowThreads / 32) tmem_dealloc(tm, 128);
 }
 
@@ -422,6 +433,7 @@ __global__ void __launch_bounds__(kThreads16, 1) bwd_dyq_tc(const __grid_constan
         tma_prefetch_desc(&p.tmSL);
         tma_prefetch_desc(&p.tmDyH);
         tma_prefetch_desc(&p.tmDyL);
+        tma_prefetch_desc(&p.tmInc);
     }
     if (warp == RT / 32) {
         tmem_alloc(smem_u32(tmem_slot), 512);
@@ -695,16 +707,25 @@ __global__ void __launch_bounds__(kThreads16, 1) bwd_dyq_tc(const __grid_constan
             warp_arrive(BDS);
 
             // ------------------------------------------------ G_c rows (lane = d_k row)
-            if (mbar_wait(bar(BGC), par, p.status, abort_flag)) {
+            // staged in the dy tiles (free once G_c and the dy store have read them) as
+            // four [128][32] fp32 boxes in the 128-byte swizzle layout, stored by TMA
+            if (mbar_wait(bar(BGC), par, p.status, abort_flag) && mbar_wait(bar(BDYRD), par, p.status, abort_flag)) {
                 tc_fence_after();
-                float* dst = p.incg + (((size_t)u * nc + c) * kDK + t) * DV + ch0 + 32 * cq;
                 uint32_t v[32];
                 tmem_ld_x32(tm + lq + R_YI + 32 * cq, v);
                 tmem_wait_ld();
+                uint8_t* box = sm + OFF_DYH + cq * kBox;
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    reinterpret_cast<float4*>(dst)[k] =
-                        make_float4(u2f(v[4 * k]), u2f(v[4 * k + 1]), u2f(v[4 * k + 2]), u2f(v[4 * k + 3]));
+                    *reinterpret_cast<uint4*>(box + t * 128 + ((k ^ (t & 7)) << 4)) =
+                        make_uint4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+            }
+            fence_proxy_async_smem();
+            named_bar_sync(kNamedBar, RT);
+            if (tid == 0 && !*abort_flag) {
+                for (int x = 0; x < 4; ++x)
+                    tma_store_2d(&p.tmInc, sb + OFF_DYH + x * kBox, ch0 + 32 * x, (u * nc + c) * kDK);
+                bulk_commit();
             }
             // ------------------------------------------------ dq (this CTA's channel half)
             float dq[32];
@@ -721,8 +742,9 @@ __global__ void __launch_bounds__(kThreads16, 1) bwd_dyq_tc(const __grid_constan
             }
             tc_fence_before();
             warp_arrive(BEND);   // this chunk's tensor memory has been read
-            // the dy tiles have been stored (and read by every product of the chunk)
-            mbar_wait(bar(BDYRD), par, p.status, abort_flag);
+            // the G_c store has read the dy tiles
+            if (tid == 0) bulk_wait_read<0>();
+            named_bar_sync(kNamedBar, RT);
             bool mine = true;
             if constexpr (PAIR) {
                 // rows of the other CTA's half leave in one bulk copy, staged in the dy
@@ -879,6 +901,8 @@ __global__ void __launch_bounds__(kThreads16, 1) bwd_dyq_tc(const __grid_constan
                                    mnmaj(sb + (pass == 1 ? OFF_DYL : OFF_DYH), k), id_kn, pass > 0 || k > 0);
                 }
                 mma_commit(bar(BGC));
+                bulk_wait_read<0>();   // the dy store has read its tiles
+                mbar_arrive(bar(BDYRD));
                 ok = ok && mbar_wait(bar(BDS), par, p.status, abort_flag);
                 if (ok) {
                     tc_fence_after();
@@ -889,8 +913,6 @@ __global__ void __launch_bounds__(kThreads16, 1) bwd_dyq_tc(const __grid_constan
                 mma_commit(bar(BDQ));
                 // K is free after the last product
                 if (mbar_wait(bar(BDQ), par, p.status, abort_flag) && more) load_tile(it + 1, BK, &p.tmK, OFF_K, 0);
-                bulk_wait_read<0>();   // the dy store has read its tiles
-                mbar_arrive(bar(BDYRD));
             }
             __syncwarp();
             if constexpr (PAIR) {
@@ -1384,21 +1406,33 @@ EncodeTiledFn encode_fn_bwd() {
     return fn;
 }
 
-// bf16 tensor of `rank` dimensions (innermost first), 128-byte swizzle, box
-// (64, 1, ..., 128 at dimension `rowdim`, ...)
-bool encode_bf16(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint32_t* box) {
+// tensor of `rank` dimensions (innermost first) of bf16 or fp32 elements,
+// 128-byte swizzle
+bool encode_tile(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint32_t* box,
+                 bool f32) {
     EncodeTiledFn fn = encode_fn_bwd();
     if (!fn) return false;
     cuuint64_t strides[4];
-    cuuint64_t st = 2;
+    cuuint64_t st = f32 ? 4 : 2;
     for (int i = 0; i + 1 < rank; ++i) {
         st *= dims[i];
         strides[i] = st;
     }
     cuuint32_t estr[4] = {1, 1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    return fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank,
+              const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+bool encode_bf16(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint32_t* box) {
+    return encode_tile(m, base, rank, dims, box, false);
+}
+
+// state-shaped fp32 rows [rows][dv], box (32, 128): 128-byte rows in the swizzle layout
+bool map_state_rows_f32(CUtensorMap* m, const void* base, int dv, size_t rows) {
+    const cuuint64_t dims[2] = {(cuuint64_t)dv, (cuuint64_t)rows};
+    const cuuint32_t box[2] = {32, 128};
+    return encode_tile(m, base, 2, dims, box, true);
 }
 
 // [B][N][H][d] viewed as (d, H, N, B), box (64, 1, 128, 1)
@@ -1526,7 +1560,7 @@ cudaError_t launch_bwd_tc(const BackwardArgs& in, cudaStream_t s) {
     if (!map_tokens(&p.tmQ, in.Q, kDK, in.H, in.N, in.B) || !map_tokens(&p.tmK, in.K, kDK, in.H, in.N, in.B) ||
         !map_tokens(&p.tmV, in.V, in.dv, in.H, in.N, in.B) || !map_tokens(&p.tmDyH, p.dyh, in.dv, in.H, in.N, in.B) ||
         !map_tokens(&p.tmDyL, p.dyl, in.dv, in.H, in.N, in.B) || !map_states(&p.tmSH, p.sh, in.dv, srows) ||
-        !map_states(&p.tmSL, p.sl, in.dv, srows))
+        !map_states(&p.tmSL, p.sl, in.dv, srows) || !map_state_rows_f32(&p.tmInc, p.incg, in.dv, srows))
         return cudaErrorInvalidValue;
     return in.dv == 256 ? run_bwd_tc<256>(p, s) : run_bwd_tc<128>(p, s);
 }
