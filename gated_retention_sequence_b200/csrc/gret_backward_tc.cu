@@ -359,7 +359,7 @@ __global__ void __launch_bounds__(kScanThreads) bwd_scan_rev(const __grid_consta
 struct GradCfg {
     static constexpr int OFF_BC = 7 * kTile;          // b_t [128], 4 warp sums
     static constexpr int OFF_AUX = OFF_BC + 528;      // 2 KB: exchange buffers / row sums
-    static constexpr int NUM_BARS = 22;
+    static constexpr int NUM_BARS = 23;
     static constexpr int OFF_BAR = OFF_AUX + 2048;
     static constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;
     static constexpr int SMEM = OFF_MISC + 16;
@@ -389,8 +389,8 @@ __global__ void __launch_bounds__(kThreads16, 1) bwd_dyq_tc(const __grid_constan
     constexpr uint32_t R_A = 0, R_Y = 128, R_YI = 256, R_P = 384;
     constexpr int BQ = 0, BK = 1, BV = 2, BS = 3, BA = 4, BYI = 5, BP = 6, BY = 7, BDY = 8, BD = 9, BQI = 10,
                   BQT = 11, BGC = 12, BDS = 13, BDQ = 14, BX0 = 15, BX1 = 16, BX2 = 17, BXQ = 18, BDYRD = 19,
-                  BDRAIN = 20, BEND = 21;
-    static_assert(BEND < CF::NUM_BARS, "barrier count");
+                  BDRAIN = 20, BEND = 21, BPR = 22;
+    static_assert(BPR < CF::NUM_BARS, "barrier count");
     extern __shared__ __align__(1024) uint8_t sm[];
     const uint32_t sb = smem_u32(sm);
     if (sb & 1023u) {
@@ -742,8 +742,11 @@ __global__ void __launch_bounds__(kThreads16, 1) bwd_dyq_tc(const __grid_constan
             }
             tc_fence_before();
             warp_arrive(BEND);   // this chunk's tensor memory has been read
-            // the G_c store has read the dy tiles
-            if (tid == 0) bulk_wait_read<0>();
+            // the G_c store has read the dy tiles; the other CTA may send into dy hi
+            if (tid == 0) {
+                bulk_wait_read<0>();
+                if (PAIR) mbar_arrive_remote(cluster_map(bar(BPR), peer));
+            }
             named_bar_sync(kNamedBar, RT);
             bool mine = true;
             if constexpr (PAIR) {
@@ -761,8 +764,8 @@ __global__ void __launch_bounds__(kThreads16, 1) bwd_dyq_tc(const __grid_constan
                             make_float4(dq[4 * k], dq[4 * k + 1], dq[4 * k + 2], dq[4 * k + 3]);
                 fence_proxy_async_smem();
                 named_bar_sync(kNamedBar, RT);
-                cluster_sync_all();   // both CTAs are past the chunk's last product
-                if (tid == 0) {
+                // the other CTA's dy hi tile is free
+                if (tid == 0 && mbar_wait_cluster(bar(BPR), par, p.status, abort_flag)) {
                     bulk_copy_to_cluster(cluster_map(sb + OFF_DYH, peer), sb + OFF_DYL, 64 * 128 * 4,
                                          cluster_map(bar(BXQ), peer));
                     bulk_commit();
@@ -916,7 +919,6 @@ __global__ void __launch_bounds__(kThreads16, 1) bwd_dyq_tc(const __grid_constan
             }
             __syncwarp();
             if constexpr (PAIR) {
-                cluster_sync_all();
                 // the next chunk's exchanges, once this chunk's dq has arrived
                 if (lane == 0 && more && mbar_wait_cluster(bar(BXQ), par, p.status, abort_flag)) arm_exchange();
                 __syncwarp();
@@ -975,7 +977,7 @@ __global__ void __launch_bounds__(kThreads16, 1) bwd_kv_tc(const __grid_constant
                   OFF_DSH = 5 * kTile, OFF_DSL = 6 * kTile;
     constexpr uint32_t R_AT = 0, R_DT = 128, R_DK = 256, R_DV = 384;
     constexpr int BQ = 0, BK = 1, BV = 2, BDY = 3, BS = 4, BADT = 5, BINTER = 6, BROWS = 7, BOUT = 8, BXK = 9,
-                  BXDONE = 10, BDRAIN = 11;
+                  BXDONE = 10, BDRAIN = 11, BPR = 12;
     extern __shared__ __align__(1024) uint8_t sm[];
     const uint32_t sb = smem_u32(sm);
     if (sb & 1023u) {
@@ -1142,6 +1144,8 @@ __global__ void __launch_bounds__(kThreads16, 1) bwd_kv_tc(const __grid_constant
             float dk[32];
             if (mbar_wait(bar(BOUT), par, p.status, abort_flag)) {
                 tc_fence_after();
+                // this CTA's dS' products are done: the other CTA may send into dS' lo
+                if (PAIR && tid == 0) mbar_arrive_remote(cluster_map(bar(BPR), peer));
                 uint32_t v[32];
                 tmem_ld_x32(tm + lq + R_DV + 32 * cq, v);
                 tmem_wait_ld();
@@ -1187,9 +1191,8 @@ __global__ void __launch_bounds__(kThreads16, 1) bwd_kv_tc(const __grid_constant
                             make_float4(dk[4 * k], dk[4 * k + 1], dk[4 * k + 2], dk[4 * k + 3]);
                 fence_proxy_async_smem();
                 named_bar_sync(kNamedBar, RT);
-                // both CTAs are past this chunk's last product: the dS' tiles are free
-                cluster_sync_all();
-                if (tid == 0) {
+                // the other CTA is past its dS' products: its dS' lo tile is free
+                if (tid == 0 && mbar_wait_cluster(bar(BPR), par, p.status, abort_flag)) {
                     bulk_copy_to_cluster(cluster_map(sb + OFF_DSL, peer), sb + OFF_DSH, 64 * 128 * 4,
                                          cluster_map(bar(BXK), peer));
                     bulk_commit();
@@ -1322,7 +1325,6 @@ __global__ void __launch_bounds__(kThreads16, 1) bwd_kv_tc(const __grid_constant
                 }
             }
             __syncwarp();
-            if constexpr (PAIR) cluster_sync_all();
             if (lane == 0) {
                 // the dk exchange of this chunk has been read: the next dS' may load
                 // into its buffer, and the exchange barrier is armed for the next chunk
