@@ -221,20 +221,24 @@ gret_status gret_state_fold(const float* dS_all, const float* decay_all, int num
  * and the initial state dS0 (fp32 [B][H][dk][dv]; may be NULL).  S0 and
  * dS_final may be NULL (zero).  Accumulation is fp32 throughout.
  *
- * Head sizes that are multiples of 32 with dk <= 128 and dv <= 256 take the
- * chunk-parallel path (5 launches; chunks of 64 tokens for bf16, 32 for fp32).
- * With bf16 inputs, dk = 128 and dv = 128 or 256 its products run on the
- * tensor cores (mma.sync tf32; every operand that is not a bf16 input is split
- * into two tf32 parts, which keeps the products at fp32-level accuracy);
- * otherwise on CUDA cores in fp32.
- * The workspace holds the state before every chunk and the gradient at every
- * chunk's end (2 * B*H*ceil(N/chunk)*dk*dv*4 bytes), the gradient of the
- * pre-norm output (B*N*H*dv*4) and one decay per chunk.  Other head sizes
+ * bf16 inputs with dk = 128 and dv = 128 or 256 take the tensor-core path
+ * (6 launches, chunks of 128 tokens, tcgen05 products with fp32 accumulation;
+ * the per-chunk states, state gradients and dy enter the products as bf16
+ * pairs hi + lo, about 16 mantissa bits).  Its workspace holds, per chunk, an
+ * fp32 state-shaped buffer and a state as a bf16 pair (2 * B*H*ceil(N/128)*
+ * dk*dv*(4 + 4) bytes in all), dy as a bf16 pair (B*N*H*dv*4), two fp32 terms
+ * per token and head, and per chunk dv + 513 fp32 values.  Other head sizes
+ * that are multiples of 32 with dk <= 128 and dv <= 256 take the chunk-parallel
+ * path on CUDA cores in fp32 (5 launches; chunks of 64 tokens for bf16, 32 for
+ * fp32), whose workspace holds the state before every chunk and the gradient
+ * at every chunk's end (2 * B*H*ceil(N/chunk)*dk*dv*4 bytes), the gradient of
+ * the pre-norm output (B*N*H*dv*4) and one decay per chunk.  Other head sizes
  * (multiples of 16 up to 256) take a serial path (2 launches) that keeps the
  * state at every 32-token block (B*H*ceil(N/32)*dk*dv*4 plus one state per
  * unit) and walks the blocks in reverse.  The size depends on io_dtype; 0 for
  * an unsupported shape.  Where the forward clamps a log-decay at -64 the gate
- * gradient is zero.
+ * gradient is zero.  A bounded device wait that gives up on the tensor-core
+ * path is reported by gret_last_device_status.
  */
 size_t gret_prefill_backward_workspace_size(int B, int H, int N, int dk, int dv, gret_dtype io_dtype);
 /* Kernel launches one gret_prefill_backward call makes for this shape (0 if unsupported). */
