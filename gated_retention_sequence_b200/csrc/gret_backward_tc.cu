@@ -407,14 +407,13 @@ __global__ void __launch_bounds__(kThreads16, 1) bwd_dyq_tc(const __grid_constan
     auto bar = [&](int i) -> uint32_t { return sb + CF::OFF_BAR + 8 * i; };
     float* bc = reinterpret_cast<float*>(sm + CF::OFF_BC);
     float* wsum = bc + kC;
-    float* xch = reinterpret_cast<float*>(sm + CF::OFF_AUX);   // [128] round 0, [128] round 1, [128][2] round 2
+    float* xch = reinterpret_cast<float*>(sm + CF::OFF_AUX);   // [128][2] round 0, [128][2] round 2
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + CF::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + CF::OFF_MISC + 4);
     // one-shot-per-chunk exchange barriers, armed for the bytes the other CTA sends
     auto arm_exchange = [&]() {
         if (p.gn) {
-            mbar_arrive_expect_tx(bar(BX0), kC * 4);
-            mbar_arrive_expect_tx(bar(BX1), kC * 4);
+            mbar_arrive_expect_tx(bar(BX0), kC * 8);
             mbar_arrive_expect_tx(bar(BX2), kC * 8);
         }
         mbar_arrive_expect_tx(bar(BXQ), 64 * 128 * 4);
@@ -516,7 +515,7 @@ __global__ void __launch_bounds__(kThreads16, 1) bwd_dyq_tc(const __grid_constan
                 ra = u2f(r8[0]) + u2f(r8[2]) + u2f(r8[4]) + u2f(r8[6]);
                 rb = u2f(r8[1]) + u2f(r8[3]) + u2f(r8[5]) + u2f(r8[7]);
                 if (PAIR && pair) {
-                    const int off = slot == 0 ? t : slot == 1 ? kC + t : 2 * kC + 2 * t;
+                    const int off = slot == 0 ? 2 * t : 2 * kC + 2 * t;
                     if (cq == 0) {
                         const uint32_t remote = cluster_map(smem_u32(xch + off), peer);
                         const uint32_t rbar = cluster_map(bar(xbar), peer);
@@ -548,21 +547,20 @@ __global__ void __launch_bounds__(kThreads16, 1) bwd_dyq_tc(const __grid_constan
             }
             if (p.gn) {
                 const float inv_dv = 1.0f / (float)DV;
-                float s1 = 0.f, dummy;
-#pragma unroll
-                for (int j = 0; j < 32; ++j) s1 += y[j];
-                float mean;
-                row_sum(0, BX0, s1, 0.f, false, true, mean, dummy);
-                mean *= inv_dv;
-                float s2 = 0.f;
+                // mean and variance from the sums of y and y^2 in one exchange (as the
+                // forward's epilogue forms them)
+                float s1 = 0.f, s2 = 0.f;
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
-                    y[j] -= mean;
+                    s1 += y[j];
                     s2 = fmaf(y[j], y[j], s2);
                 }
-                float var;
-                row_sum(1, BX1, s2, 0.f, false, true, var, dummy);
-                const float rstd = rsqrtf(var * inv_dv + p.eps);
+                row_sum(0, BX0, s1, s2, true, true, s1, s2);
+                const float mean = s1 * inv_dv;
+                const float var = fmaxf(s2 * inv_dv - mean * mean, 0.f);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) y[j] -= mean;
+                const float rstd = rsqrtf(var + p.eps);
                 float m1 = 0.f, m2 = 0.f;
                 __nv_bfloat16* dGg = static_cast<__nv_bfloat16*>(p.dG) + rowoff;
 #pragma unroll
