@@ -168,3 +168,11 @@ def test_bf16_dv256_pairs_more_chunks_than_pairs():
     sequence (the last chunk 88 tokens) are more chunks than SM pairs."""
     cfg = gi.C2.scaled(B=1, H=3, N=3288, seed=82)
     _sampled_units(cfg, [(0, 0), (0, 2)])
+
+
+@pytest.mark.parametrize("dv,N", [(256, 1), (256, 129), (128, 1), (128, 129)])
+def test_bf16_tensor_core_edge_lengths(dv, N):
+    """The tensor-core backward on a single token and on one chunk plus one token
+    (the last chunk's one row), without states: nearly every launched CTA of the
+    persistent kernels has no chunk to take."""
+    _run(gi.C2.scaled(B=1, H=1, N=N, dv=dv, seed=90 + N + dv), with_s0=False, with_dsf=False)
