@@ -131,6 +131,7 @@ struct Cfg {
 
 struct TcParams {
     CUtensorMap tmQ, tmK, tmV, tmG, tmO;
+    CUtensorMap tmKs, tmVs;  // K and V in the state pass's sub-chunk tiles
     const float* bcum;       // [units][Npad] chunk-local cumulative log-decay
     const float* eblk;       // [units][Npad] block factors of the P columns (gate scan)
     float* seg_state;        // [units][slots][DV][DK]  (S^T, fp32)
@@ -894,24 +895,32 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_tc_kernel(const __gr
 // Segment state pass: dS_p = sum over the segment's tokens of
 // e^{a_p - B_s} K_s^T V_s (B_s the log-decay from the segment start through s,
 // a_p the segment total), from K, V and the decay sums alone.  The same
-// lazy/eager state scaling as the fused kernels; a 3-4 stage ring of K/V
-// tiles keeps about 190 KB of loads in flight per SM.
+// lazy/eager state scaling as the fused kernels, decided per chunk of C tokens;
+// the K/V tiles stream through a ring of sub-chunks of SUB tokens (64 where a
+// whole 128-token chunk of d_v = 256 would leave room for two stages only), so
+// that three or more stages of loads stay in flight per SM.
 constexpr int kStateThreads = 256;
+
+// tokens per staged K/V tile of the state pass
+constexpr int state_sub(int dv, int C) { return (C == 128 && dv == 256) ? 64 : C; }
 
 template <int DV, int C>
 struct StateCfg {
     static constexpr int NH = DV / 128;
-    static constexpr int BOX = C * 128;
+    static constexpr int SUB = state_sub(DV, C);
+    static constexpr int NSUB = C / SUB;                    // sub-chunks per chunk
+    static constexpr int BOX = SUB * 128;
     static constexpr int K_BYTES = 2 * BOX;
     static constexpr int V_BYTES = (DV / 64) * BOX;
     // as many K + V stages as about 210 KB hold (2-6), to keep loads in flight
-    static constexpr int NS_FIT = (210 * 1024) / (K_BYTES + V_BYTES);
+    static constexpr int NS_FIT = (210 * 1024) / (K_BYTES + V_BYTES + C * 4);
     static constexpr int NS = NS_FIT > 6 ? 6 : NS_FIT;
     static_assert(NS >= 2, "state pass stages");
     static constexpr int W = NH * 64;                       // state columns per thread
     static constexpr int TM_ALLOC = NH * 128 <= 128 ? 128 : 256;
     static constexpr int OFF_K = 0;
     static constexpr int OFF_V = OFF_K + NS * K_BYTES;
+    // the decay sums of the whole chunk a sub-chunk belongs to
     static constexpr int OFF_B = OFF_V + NS * V_BYTES;
     static constexpr int OFF_BAR = OFF_B + NS * C * 4;
     // full and empty barrier per stage, then the drain barrier of the last commit
@@ -923,7 +932,7 @@ struct StateCfg {
 template <int DV, int C, bool PACKED>
 __global__ void __launch_bounds__(kStateThreads, 1) prefill_state_kernel(const __grid_constant__ TcParams p) {
     using CF = StateCfg<DV, C>;
-    constexpr int NS = CF::NS, NH = CF::NH, W = CF::W;
+    constexpr int NS = CF::NS, NH = CF::NH, W = CF::W, SUB = CF::SUB, NSUB = CF::NSUB;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_u32(sm);
@@ -976,8 +985,8 @@ __global__ void __launch_bounds__(kStateThreads, 1) prefill_state_kernel(const _
         for (int i = 0; i < 2 * NS + 1; ++i) mbar_init(sb + CF::OFF_BAR + 8 * i, 1);
         *abort_flag = 0;
         fence_mbar_init();
-        tma_prefetch_desc(&p.tmK);
-        tma_prefetch_desc(&p.tmV);
+        tma_prefetch_desc(&p.tmKs);
+        tma_prefetch_desc(&p.tmVs);
     }
     if (warp == 0) {
         tmem_alloc(smem_u32(tmem_slot), CF::TM_ALLOC);
@@ -1000,20 +1009,21 @@ __global__ void __launch_bounds__(kStateThreads, 1) prefill_state_kernel(const _
         Nu = min(Nu, p.N);                    // tokens past max_seqlen are not processed
     }
     const int n_end = min(Nu, n_begin + piece_len);
-    const int nchunks = n_end > n_begin ? (n_end - n_begin + C - 1) / C : 0;
-    int last_issued = -1;     // thread 0: the last chunk whose loads it issued
+    // sub-chunks of SUB tokens; the pieces start on chunk boundaries
+    const int nsub = n_end > n_begin ? (n_end - n_begin + SUB - 1) / SUB : 0;
+    int last_issued = -1;     // thread 0: the last sub-chunk whose loads it issued
     auto issue = [&](int j) {
-        const int s = j % NS, n0 = n_begin + j * C;
+        const int s = j % NS, nc0 = n_begin + (j / NSUB) * C, n0 = nc0 + (j % NSUB) * SUB;
         last_issued = j;
         mbar_arrive_expect_tx(full(s), CF::K_BYTES + CF::V_BYTES + C * 4);
         for (int x = 0; x < 2; ++x)
-            tma_load_4d(sb + CF::OFF_K + s * CF::K_BYTES + x * CF::BOX, &p.tmK, x * 64, hh, row0 + n0, bb, full(s));
+            tma_load_4d(sb + CF::OFF_K + s * CF::K_BYTES + x * CF::BOX, &p.tmKs, x * 64, hh, row0 + n0, bb, full(s));
         for (int x = 0; x < DV / 64; ++x)
-            tma_load_4d(sb + CF::OFF_V + s * CF::V_BYTES + x * CF::BOX, &p.tmV, x * 64, hh, row0 + n0, bb, full(s));
-        bulk_load(sb + CF::OFF_B + s * C * 4, p.bcum + (size_t)u * p.Npad + n0, C * 4, full(s));
+            tma_load_4d(sb + CF::OFF_V + s * CF::V_BYTES + x * CF::BOX, &p.tmVs, x * 64, hh, row0 + n0, bb, full(s));
+        bulk_load(sb + CF::OFF_B + s * C * 4, p.bcum + (size_t)u * p.Npad + nc0, C * 4, full(s));
     };
     if (tid == 0)
-        for (int j = 0; j < NS && j < nchunks; ++j) issue(j);
+        for (int j = 0; j < NS && j < nsub; ++j) issue(j);
 
     const int col0 = gi * W;
 #pragma unroll 1
@@ -1026,28 +1036,30 @@ __global__ void __launch_bounds__(kStateThreads, 1) prefill_state_kernel(const _
     tmem_wait_st();
 
     float lam = 0.f, seg_decay = 0.f;
-    for (int i = 0; i < nchunks; ++i) {
-        const int s = i % NS;
+    for (int i = 0; i < nsub; ++i) {
+        const int s = i % NS, hs = i % NSUB;             // stage; sub-chunk within its chunk
         const float* bc = reinterpret_cast<const float*>(sm + CF::OFF_B + s * C * 4);
         mbar_wait(full(s), (i / NS) & 1, p.status, abort_flag);
         const float bC = bc[C - 1];
+        // lam and the decision change only at chunk ends, so every sub-chunk
+        // of a chunk takes the same one
         const bool eager = (-bC - lam) > kLazyMax;
         uint8_t* Kp = sm + CF::OFF_K + s * CF::K_BYTES;
         {
-            constexpr int NIT = C * 16 / kStateThreads;   // 4 or 8 items per thread
+            constexpr int NIT = SUB * 16 / kStateThreads;   // 4 or 8 items per thread
             uint4 w[NIT];
             float e[NIT];
 #pragma unroll
             for (int k = 0; k < NIT; ++k) {
                 const int ci = tid + k * kStateThreads;
                 w[k] = *reinterpret_cast<const uint4*>(Kp + ci * 16);
-                e[k] = bc[(ci >> 3) % C];
+                e[k] = bc[hs * SUB + (ci >> 3) % SUB];
             }
-            const int valid = n_end - (n_begin + i * C);   // rows of this unit in the chunk
+            const int valid = n_end - (n_begin + i * SUB);   // rows of this unit in the sub-chunk
 #pragma unroll
             for (int k = 0; k < NIT; ++k) {
                 // rows past the unit's end (the next packed sequence's) add nothing
-                const float sc = (!PACKED || ((tid + k * kStateThreads) >> 3) % C < valid)
+                const float sc = (!PACKED || ((tid + k * kStateThreads) >> 3) % SUB < valid)
                                      ? __expf(eager ? (bC - e[k]) : (-e[k] - lam)) : 0.f;
                 uint32_t* x = reinterpret_cast<uint32_t*>(&w[k]);
 #pragma unroll
@@ -1058,7 +1070,7 @@ __global__ void __launch_bounds__(kStateThreads, 1) prefill_state_kernel(const _
                 *reinterpret_cast<uint4*>(Kp + (tid + k * kStateThreads) * 16) = w[k];
             }
         }
-        if (eager) {
+        if (eager && hs == 0) {
             // T *= e^{Lambda + b_C}, after the previous chunk's state MMA
             if (i > 0) {
                 mbar_wait(empty((i - 1) % NS), ((i - 1) / NS) & 1, p.status, abort_flag);
@@ -1086,19 +1098,21 @@ __global__ void __launch_bounds__(kStateThreads, 1) prefill_state_kernel(const _
 #pragma unroll
             for (int h = 0; h < NH; ++h) {
 #pragma unroll
-                for (int k = 0; k < C / 16; ++k)
+                for (int k = 0; k < SUB / 16; ++k)
                     mma_ss(tm + h * 128, sdesc_sw128(sV + 2 * h * CF::BOX + k * 2048, CF::BOX, 1024),
                            sdesc_sw128(sK + k * 2048, CF::BOX, 1024), id_kv, 1);
             }
             mma_commit(empty(s));
-            // the stage the previous chunk used is free once its MMAs are done
-            // (they run before this chunk's, which queue behind them)
-            if (i > 0 && i - 1 + NS < nchunks &&
+            // the stage the previous sub-chunk used is free once its MMAs are
+            // done (they run before this one's, which queue behind them)
+            if (i > 0 && i - 1 + NS < nsub &&
                 mbar_wait(empty((i - 1) % NS), ((i - 1) / NS) & 1, p.status, abort_flag))
                 issue(i - 1 + NS);
         }
-        seg_decay += bC;
-        lam = eager ? 0.f : lam + bC;
+        if (hs == NSUB - 1 || i == nsub - 1) {
+            seg_decay += bC;
+            lam = eager ? 0.f : lam + bC;
+        }
     }
     if (tid == 0) {
         // every MMA issued has completed, and on the give-up path every load
@@ -1111,8 +1125,8 @@ __global__ void __launch_bounds__(kStateThreads, 1) prefill_state_kernel(const _
             for (int j = last_issued; j >= 0 && j > last_issued - NS; --j)
                 mbar_wait_drain(full(j % NS), (j / NS) & 1, kWaitCycles);
     }
-    if (nchunks > 0) {
-        mbar_wait(empty((nchunks - 1) % NS), ((nchunks - 1) / NS) & 1, p.status, abort_flag);
+    if (nsub > 0) {
+        mbar_wait(empty((nsub - 1) % NS), ((nsub - 1) / NS) & 1, p.status, abort_flag);
         tc_fence_after();
     }
     {
@@ -1346,24 +1360,42 @@ __global__ void seg_combine_kernel(float* __restrict__ seg_state, const float* _
     }
 }
 
-// State-only pass: the folded pieces (the last slot, S^T layout [DV][DK]) become
-// the slice's increment dS [DK][DV] through a shared-memory tile transpose, and
-// the pieces' log-decays sum to the slice's total.
+// State-only pass: each piece's increment is folded from the zero state in
+// place -- slot j <- e^{a_j} slot(j - 1) + slot j, the increment from the
+// slice's start through piece j, which a resumed prefill reads -- and the last
+// fold, S^T [DV][DK], becomes the slice's increment dS [DK][DV] through a
+// shared-memory tile transpose; the pieces' log-decays sum to the slice's total.
+// One block per 32 x 32 tile of a unit's state, each thread four rows of it.
 template <int DV>
-__global__ void state_finish_kernel(const float* __restrict__ seg_state, const float* __restrict__ seg_decay,
-                                    int slots, float* __restrict__ dS, float* __restrict__ decay) {
+__global__ void state_finish_kernel(float* __restrict__ seg_state, const float* __restrict__ seg_decay, int slots,
+                                    float* __restrict__ dS, float* __restrict__ decay) {
     __shared__ float tile[32][33];
+    grid_dep_launch();
+    grid_dep_wait();       // the state pass's pieces
     const int u = blockIdx.x;
     const int d0 = (blockIdx.y % (DV / 32)) * 32, k0 = (blockIdx.y / (DV / 32)) * 32;   // tile of S^T
-    const float* src = seg_state + ((size_t)u * slots + slots - 1) * DV * DK;
-    for (int r = threadIdx.y; r < 32; r += blockDim.y) tile[r][threadIdx.x] = src[(size_t)(d0 + r) * DK + k0 + threadIdx.x];
+    const int x = threadIdx.x, y = threadIdx.y;
+    float run[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < slots; ++j) {
+        float* src = seg_state + ((size_t)u * slots + j) * DV * DK + (size_t)d0 * DK + k0 + x;
+        const float f = __expf(seg_decay[(size_t)u * slots + j]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float* at = src + (size_t)(y + 8 * i) * DK;
+            run[i] = fmaf(f, run[i], *at);
+            *at = run[i];
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) tile[y + 8 * i][x] = run[i];
     __syncthreads();
     float* dst = dS + (size_t)u * DK * DV;
-    for (int r = threadIdx.y; r < 32; r += blockDim.y) dst[(size_t)(k0 + r) * DV + d0 + threadIdx.x] = tile[threadIdx.x][r];
-    if (blockIdx.y == 0 && threadIdx.x == 0 && threadIdx.y == 0) {
-        float a = 0.f;
-        for (int k = 0; k < slots; ++k) a += seg_decay[(size_t)u * slots + k];
-        decay[u] = a;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) dst[(size_t)(k0 + y + 8 * i) * DV + d0 + x] = tile[x][y + 8 * i];
+    if (blockIdx.y == 0 && x == 0 && y == 0) {
+        float acc = 0.f;
+        for (int k = 0; k < slots; ++k) acc += seg_decay[(size_t)u * slots + k];
+        decay[u] = acc;
     }
 }
 
@@ -1395,17 +1427,27 @@ __global__ void seg_shift_kernel(float* __restrict__ seg_state, const float* __r
 }
 
 // Sequence-parallel fold: S_in = e^{a_{p-1}} (... (e^{a_0} S0 + dS_0) ...) + dS_{p-1}
-// over the slices before `slice`, elementwise.
-__global__ void state_fold_kernel(const float* __restrict__ dS_all, const float* __restrict__ decay_all,
-                                  int slice, const float* __restrict__ S0, float* __restrict__ S_in, int units,
-                                  int elems) {
+// over the slices before `slice`, elementwise, VW elements (float or float4)
+// per thread.
+__device__ __forceinline__ float fold_fma(float f, float r, float d) { return fmaf(f, r, d); }
+__device__ __forceinline__ float4 fold_fma(float f, float4 r, float4 d) {
+    return make_float4(fmaf(f, r.x, d.x), fmaf(f, r.y, d.y), fmaf(f, r.z, d.z), fmaf(f, r.w, d.w));
+}
+
+template <typename T>
+__global__ void state_fold_kernel(const T* __restrict__ dS_all, const float* __restrict__ decay_all, int slice,
+                                  const T* S0, T* S_in, int units, int nvec) {
+    grid_dep_launch();
+    grid_dep_wait();       // the increments may come from the kernel before this one
     const int u = blockIdx.x;
     const int e = blockIdx.y * blockDim.x + threadIdx.x;
-    if (e >= elems) return;
-    const size_t at = (size_t)u * elems + e;
-    float run = S0 ? S0[at] : 0.f;
+    if (e >= nvec) return;
+    const size_t at = (size_t)u * nvec + e;
+    T run;
+    if (S0) run = S0[at];                      // S0 may be S_in itself: read before the write
+    else memset(&run, 0, sizeof(T));
     for (int q = 0; q < slice; ++q)
-        run = fmaf(__expf(decay_all[(size_t)q * units + u]), run, dS_all[(size_t)q * units * elems + at]);
+        run = fold_fma(__expf(decay_all[(size_t)q * units + u]), run, dS_all[(size_t)q * units * nvec + at]);
     S_in[at] = run;
 }
 
@@ -2393,7 +2435,9 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
     const int mN = a.cu_seqlens ? a.total : a.N, mB = a.cu_seqlens ? 1 : a.B;
     if (!make_map(&tp.tmQ, a.Q, DK, a.H, mN, mB, C) || !make_map(&tp.tmK, a.K, DK, a.H, mN, mB, C) ||
         !make_map(&tp.tmV, a.V, a.dv, a.H, mN, mB, C) || !make_map(&tp.tmO, a.O, a.dv, a.H, mN, mB, C) ||
-        !make_map(&tp.tmG, a.G ? a.G : a.O, a.dv, a.H, mN, mB, C))
+        !make_map(&tp.tmG, a.G ? a.G : a.O, a.dv, a.H, mN, mB, C) ||
+        !make_map(&tp.tmKs, a.K, DK, a.H, mN, mB, state_sub(a.dv, C)) ||
+        !make_map(&tp.tmVs, a.V, a.dv, a.H, mN, mB, state_sub(a.dv, C)))
         return cudaErrorInvalidValue;
     tp.cu = a.cu_seqlens;
     tp.total = a.total;
@@ -2479,24 +2523,19 @@ static cudaError_t run_state_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t
     if (e != cudaSuccess) return e;
     e = launch_pdl(ks, dim3(units * tp.slots), dim3(kStateThreads), StateCfg<DV, C>::SMEM, s, tp);
     if (e != cudaSuccess) return e;
-    // fold every piece from the zero state, in place: slot j becomes the
-    // increment from the slice's start through piece j
-    const int elems4 = DV * DK / 4;
-    e = launch_pdl(seg_combine_kernel, dim3(units, (elems4 + 255) / 256), dim3(256), 0, s, tp.seg_state,
-                   static_cast<const float*>(tp.seg_decay), static_cast<const float*>(nullptr), tp.slots, DK, DV,
-                   static_cast<const int4*>(nullptr), static_cast<const int2*>(nullptr),
-                   static_cast<const int*>(nullptr));
-    if (e != cudaSuccess) return e;
-    state_finish_kernel<DV><<<dim3(units, (DV / 32) * (DK / 32)), dim3(32, 8), 0, s>>>(tp.seg_state, tp.seg_decay,
-                                                                                  tp.slots, a.S_final, a.decay_out);
-    return cudaGetLastError();
+    // fold every piece from the zero state, in place (slot j becomes the
+    // increment from the slice's start through piece j), and write the last
+    // fold as the slice's increment
+    return launch_pdl(state_finish_kernel<DV>, dim3(units, (DV / 32) * (DK / 32)), dim3(32, 8), 0, s, tp.seg_state,
+                      static_cast<const float*>(tp.seg_decay), tp.slots, a.S_final, a.decay_out);
 }
 
 cudaError_t launch_prefill_state_tc(const PrefillArgs& a, int num_sms, cudaStream_t s) {
     TcParams tp;
     memset(&tp, 0, sizeof(tp));
     const int C = a.chunk;
-    if (!make_map(&tp.tmK, a.K, DK, a.H, a.N, a.B, C) || !make_map(&tp.tmV, a.V, a.dv, a.H, a.N, a.B, C))
+    if (!make_map(&tp.tmKs, a.K, DK, a.H, a.N, a.B, state_sub(a.dv, C)) ||
+        !make_map(&tp.tmVs, a.V, a.dv, a.H, a.N, a.B, state_sub(a.dv, C)))
         return cudaErrorInvalidValue;
     const int nchunks = (a.N + C - 1) / C;
     int P = 1, seg_len = a.N, Kp = 1;
@@ -2527,9 +2566,15 @@ cudaError_t launch_prefill_state_tc(const PrefillArgs& a, int num_sms, cudaStrea
 cudaError_t launch_state_fold(const float* dS_all, const float* decay_all, int num_slices, int slice,
                               const float* S0, float* S_in, int units, int elems, cudaStream_t s) {
     (void)num_slices;
-    state_fold_kernel<<<dim3(units, (elems + 255) / 256), 256, 0, s>>>(dS_all, decay_all, slice, S0, S_in, units,
-                                                                      elems);
-    return cudaGetLastError();
+    auto a16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
+    if (elems % 4 == 0 && a16(dS_all) && a16(S0) && a16(S_in)) {
+        const int nvec = elems / 4;
+        return launch_pdl(state_fold_kernel<float4>, dim3(units, (nvec + 255) / 256), dim3(256), 0, s,
+                          reinterpret_cast<const float4*>(dS_all), decay_all, slice,
+                          reinterpret_cast<const float4*>(S0), reinterpret_cast<float4*>(S_in), units, nvec);
+    }
+    return launch_pdl(state_fold_kernel<float>, dim3(units, (elems + 255) / 256), dim3(256), 0, s, dS_all, decay_all,
+                      slice, S0, S_in, units, elems);
 }
 
 }  // namespace gret
