@@ -1177,10 +1177,14 @@ __global__ void __launch_bounds__(kScanThreads) gate_scan_kernel(const float* __
     int row0 = 0, Nu = N;
     if (cu_seqlens) packed_range(cu_seqlens, b, total, row0, Nu);
     const size_t base = cu_seqlens ? (size_t)row0 : (size_t)b * N;
+    // a packed unit's chunks end with its own tokens (the kernels after this
+    // one read no further), a uniform unit's at Npad
+    const int nend = cu_seqlens ? min(Npad, (Nu + C - 1) / C * C) : Npad;
     // blocks of kScanThreads / C chunks, strided over the grid's y extent
     for (int by = blockIdx.y; by < nyb; by += gridDim.y) {
+        if (by * kScanThreads >= nend) break;          // the same for every thread of the block
         const int ch = by * (kScanThreads / C) + threadIdx.x / C;
-        const bool live = ch * C < Npad;
+        const bool live = ch * C < nend;
         const int n = ch * C + t;
         float x = (live && n < Nu) ? log_gamma(z[(base + n) * H + h], inv_tau) : 0.f;
 #pragma unroll
@@ -1290,7 +1294,9 @@ __global__ void __launch_bounds__(kPlanThreads) varlen_plan_kernel(const PlanArg
         a.seq_order[atomicAdd(&offs[bucket_of(a.seq_info[b].y)], 1)] = b;
     __syncthreads();
     // in that order: the fused items (sequence, segment, head) and, per split
-    // sequence, its state slots
+    // sequence, its state slots; a block of up to kPlanThreads sequences at a
+    // time, its (sequence, head) pairs spread over the threads
+    __shared__ int4 blk[kPlanThreads];   // sequence, segments, first fused item, first state item
     int carry_f = 0, carry_s = 0;
     for (int r0 = 0; r0 < a.S; r0 += kPlanThreads) {
         const int r = r0 + tid;
@@ -1299,19 +1305,23 @@ __global__ void __launch_bounds__(kPlanThreads) varlen_plan_kernel(const PlanArg
         int tf = 0, ts = 0;
         const int ef = block_exclusive_sum(si.x, warp_sums, &tf) + carry_f;
         const int es = block_exclusive_sum(b >= 0 ? si.x - 1 : 0, warp_sums, &ts) + carry_s;
-        if (b >= 0) {
-            for (int h = 0; h < a.H; ++h) {
-                const int u = b * a.H + h;
-                const int slot0 = es * a.H + h * (si.x - 1);
-                a.unit_info[u] = make_int4(si.x, si.y * a.C, slot0, 0);
-                for (int sg = 0; sg < si.x; ++sg) {
-                    const int it = (ef + sg) * a.H + h;
-                    if (it < a.max_fused) a.fused_items[it] = make_int2(u, sg);
-                }
-                for (int sg = 0; sg + 1 < si.x; ++sg)
-                    if (slot0 + sg < a.max_state) a.state_items[slot0 + sg] = make_int2(u, sg);
+        blk[tid] = make_int4(b, si.x, ef, es);
+        __syncthreads();
+        const int nb = min(kPlanThreads, a.S - r0);
+        for (int q = tid; q < nb * a.H; q += kPlanThreads) {
+            const int4 e = blk[q / a.H];
+            const int h = q % a.H, bq = e.x, P = e.y;
+            const int u = bq * a.H + h;
+            const int slot0 = e.w * a.H + h * (P - 1);
+            a.unit_info[u] = make_int4(P, a.seq_info[bq].y * a.C, slot0, 0);
+            for (int sg = 0; sg < P; ++sg) {
+                const int it = (e.z + sg) * a.H + h;
+                if (it < a.max_fused) a.fused_items[it] = make_int2(u, sg);
             }
+            for (int sg = 0; sg + 1 < P; ++sg)
+                if (slot0 + sg < a.max_state) a.state_items[slot0 + sg] = make_int2(u, sg);
         }
+        __syncthreads();                 // blk is rewritten by the next block of sequences
         carry_f += tf;
         carry_s += ts;
     }
@@ -1360,15 +1370,16 @@ __global__ void seg_combine_kernel(float* __restrict__ seg_state, const float* _
     }
 }
 
-// State-only pass: each piece's increment is folded from the zero state in
-// place -- slot j <- e^{a_j} slot(j - 1) + slot j, the increment from the
-// slice's start through piece j, which a resumed prefill reads -- and the last
-// fold, S^T [DV][DK], becomes the slice's increment dS [DK][DV] through a
-// shared-memory tile transpose; the pieces' log-decays sum to the slice's total.
+// State-only pass: the pieces' increments are folded from the zero state --
+// the fold through piece j is e^{a_j} (fold through piece j - 1) + slot j --
+// and the last fold, S^T [DV][DK], becomes the slice's increment dS [DK][DV]
+// through a shared-memory tile transpose; the pieces' log-decays sum to the
+// slice's total.  The folds a resumed prefill reads, those that end a segment
+// of `pieces` pieces before the last, are written back to their slots.
 // One block per 32 x 32 tile of a unit's state, each thread four rows of it.
 template <int DV>
 __global__ void state_finish_kernel(float* __restrict__ seg_state, const float* __restrict__ seg_decay, int slots,
-                                    float* __restrict__ dS, float* __restrict__ decay) {
+                                    int pieces, float* __restrict__ dS, float* __restrict__ decay) {
     __shared__ float tile[32][33];
     grid_dep_launch();
     grid_dep_wait();       // the state pass's pieces
@@ -1380,10 +1391,10 @@ __global__ void state_finish_kernel(float* __restrict__ seg_state, const float* 
         float* src = seg_state + ((size_t)u * slots + j) * DV * DK + (size_t)d0 * DK + k0 + x;
         const float f = __expf(seg_decay[(size_t)u * slots + j]);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            float* at = src + (size_t)(y + 8 * i) * DK;
-            run[i] = fmaf(f, run[i], *at);
-            *at = run[i];
+        for (int i = 0; i < 4; ++i) run[i] = fmaf(f, run[i], src[(size_t)(y + 8 * i) * DK]);
+        if ((j + 1) % pieces == 0 && j + 1 < slots) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) src[(size_t)(y + 8 * i) * DK] = run[i];
         }
     }
 #pragma unroll
@@ -1399,13 +1410,13 @@ __global__ void state_finish_kernel(float* __restrict__ seg_state, const float* 
     }
 }
 
-// Prefill resumed after a state-only pass of the same tokens, whose pieces
-// were folded from the zero state: every folded slot j (the state after piece
-// j, S^T layout) gains the initial state carried through the pieces' decays,
-// slot_j += e^{a_0 + ... + a_j} S0 -- the state decomposition with S0 as the
-// state before the first piece.
+// Prefill resumed after a state-only pass of the same tokens, whose folds from
+// the zero state end each segment (`pieces` pieces) in slot seg * pieces - 1:
+// each such slot j (the state after piece j, S^T layout) gains the initial
+// state carried through the pieces' decays, slot_j += e^{a_0 + ... + a_j} S0
+// -- the state decomposition with S0 as the state before the first piece.
 __global__ void seg_shift_kernel(float* __restrict__ seg_state, const float* __restrict__ seg_decay,
-                                 const float* __restrict__ S0, int slots, int dk, int dv) {
+                                 const float* __restrict__ S0, int slots, int pieces, int dk, int dv) {
     grid_dep_launch();
     grid_dep_wait();
     const int u = blockIdx.x;
@@ -1418,6 +1429,7 @@ __global__ void seg_shift_kernel(float* __restrict__ seg_state, const float* __r
     float a = 0.f;
     for (int j = 0; j < slots; ++j) {
         a += seg_decay[(size_t)u * slots + j];
+        if ((j + 1) % pieces != 0 || j + 1 == slots) continue;
         const float f = __expf(a);
         float4* slot = reinterpret_cast<float4*>(seg_state) + ((size_t)u * slots + j) * elems4 + e;
         float4 v = *slot;
@@ -2282,7 +2294,7 @@ cudaError_t run_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t s, const Pla
         if (tp.P > 1 && tp.S0) {
             const int elems4 = DV * DK / 4;
             e = launch_pdl(seg_shift_kernel, dim3(units, (elems4 + 255) / 256), dim3(256), 0, s, tp.seg_state,
-                           static_cast<const float*>(tp.seg_decay), tp.S0, tp.slots, DK, DV);
+                           static_cast<const float*>(tp.seg_decay), tp.S0, tp.slots, tp.K, DK, DV);
         }
     } else if (a.X) {
         // gate logits from the projection z = X W_gamma, fused with the scan
@@ -2527,7 +2539,7 @@ static cudaError_t run_state_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t
     // increment from the slice's start through piece j), and write the last
     // fold as the slice's increment
     return launch_pdl(state_finish_kernel<DV>, dim3(units, (DV / 32) * (DK / 32)), dim3(32, 8), 0, s, tp.seg_state,
-                      static_cast<const float*>(tp.seg_decay), tp.slots, a.S_final, a.decay_out);
+                      static_cast<const float*>(tp.seg_decay), tp.slots, tp.K, a.S_final, a.decay_out);
 }
 
 cudaError_t launch_prefill_state_tc(const PrefillArgs& a, int num_sms, cudaStream_t s) {
