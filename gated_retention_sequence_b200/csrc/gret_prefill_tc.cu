@@ -2137,10 +2137,14 @@ WsLayout ws_layout(int B, int H, int N, int dk, int dv, int chunk, int segments,
 }
 
 // Workspace of a packed batch on the tensor-core path: decay sums, the state
-// pass's slots (at most max_state), and the plan.  seg_max is half of one SM's
-// share of the batch's token-heads (at least four chunks), so that the
-// longest-first order has pieces fine enough to even out; the item bounds follow
-// from sum over sequences of ceil(chunks / (seg_max / C)) <= S + (total / C + S) / (seg_max / C).
+// pass's slots (at most max_state), and the plan.  seg_max is one and a half
+// times one work slot's share of the batch's token-heads (at least four
+// chunks): a sequence is cut only when it is much longer than that share, since
+// the state pass over the segments before its last re-reads their K and V (about
+// 0.37 of the bytes a prefill moves) and adds two launches, which costs more than
+// the imbalance of a longest-first order whose longest item is up to 1.5 shares.
+// The item bounds follow from
+// sum over sequences of ceil(chunks / (seg_max / C)) <= S + (total / C + S) / (seg_max / C).
 struct VarlenLayout {
     size_t bcum, eblk, state, decay, unit_info, fused, sitems, count, seq_info, seq_order, total;
     int seg_max, max_fused, max_state, npad;
@@ -2151,7 +2155,7 @@ VarlenLayout varlen_layout(int S, int H, int max_seqlen, int total, int dk, int 
     const long long units = (long long)S * H;
     // concurrent work items: one per SM, or per pair of SMs for the d_v = 256 pair
     const long long slots = std::max<long long>(1, num_sms / prefill_tc_ctas_per_item(dv, chunk));
-    const long long share = ((long long)total * H + 2LL * slots - 1) / (2LL * slots);
+    const long long share = (3LL * total * H + 2LL * slots - 1) / (2LL * slots);
     long long seg_max = (share + chunk - 1) / chunk * chunk;
     if (seg_max < 4LL * chunk) seg_max = 4LL * chunk;
     if (seg_max > (1LL << 30)) seg_max = (1LL << 30) / chunk * chunk;

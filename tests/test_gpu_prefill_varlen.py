@@ -86,9 +86,9 @@ def test_simt_fp32():
 
 
 @pytest.mark.parametrize("lengths,dv,chunk,H", [
-    # half of one SM's share of these batches is a few chunks, so the long
-    # sequences are cut on the device into several segments each (12 and 3, 5 and
-    # 2, 8 and 3) that a state pass joins; empty and one-token sequences stay whole
+    # one and a half work slots' share of these batches is a few chunks, so the
+    # long sequences are cut on the device into several segments each (3; 5 and
+    # 2; 6 and 2) that a state pass joins; the others stay whole
     ([3000, 50, 1, 64, 200, 0, 700], 256, 64, 16),
     ([2500, 130, 1, 0, 1000], 128, 128, 8),
     ([1900, 3, 640], 128, 64, 12),
