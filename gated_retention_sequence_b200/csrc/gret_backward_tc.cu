@@ -80,6 +80,7 @@ struct BwdTcParams {
     float* rr;                // [2][B][N][H] per channel half: dy_t . (e^{b_t} q_t S_c)
     float* xs;                // [units][nc][dv]: e^{b_L} <dS'_c, S_c> in shares of 128 elements
     float* decay;             // [units][nc] e^{b_L}
+    float* bcg;               // [units][nc][128] chunk-local decay sums b_t (flat past the sequence's end)
     float* fus;               // [units][nc][2][256]: F and us per channel half
     unsigned int* status;
     int B, H, N, dv, nc;
@@ -202,6 +203,8 @@ __global__ void __launch_bounds__(kThreads, 2) bwd_inc_tc(const __grid_constant_
         chunk_decay(p, tok0, hh, L, bc, wsum);
         const float bL = bc[kC - 1];
         if (tid == 0 && ch0 == 0) p.decay[(size_t)u * nc + c] = __expf(bL);
+        // the gradient kernels load the chunk's sums instead of scanning again
+        if (tid < kC && ch0 == 0) p.bcg[((size_t)u * nc + c) * kC + tid] = bc[tid];
         // K~ = e^{b_L - b_s} k_s as a bf16 pair: row s, 64 columns per thread
         const int s = tid & 127, xb = tid >> 7;
         const float w = s < L ? __expf(bL - bc[s]) : 0.f;
@@ -357,9 +360,9 @@ __global__ void __launch_bounds__(kScanThreads) bwd_scan_rev(const __grid_consta
 // Shared-memory layout of the two per-chunk gradient kernels: seven
 // [128][128] bf16 tiles (two 64-column swizzled boxes each), then small arrays.
 struct GradCfg {
-    static constexpr int OFF_BC = 7 * kTile;          // b_t [128], 4 warp sums
+    static constexpr int OFF_BC = 7 * kTile;          // b_t [128] of the chunk (bulk-loaded), 16 B spare
     static constexpr int OFF_AUX = OFF_BC + 528;      // 2 KB: exchange buffers / row sums
-    static constexpr int NUM_BARS = 23;
+    static constexpr int NUM_BARS = 24;
     static constexpr int OFF_BAR = OFF_AUX + 2048;
     static constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;
     static constexpr int SMEM = OFF_MISC + 16;
@@ -389,8 +392,8 @@ __global__ void __launch_bounds__(kThreads16, 1) bwd_dyq_tc(const __grid_constan
     constexpr uint32_t R_A = 0, R_Y = 128, R_YI = 256, R_P = 384;
     constexpr int BQ = 0, BK = 1, BV = 2, BS = 3, BA = 4, BYI = 5, BP = 6, BY = 7, BDY = 8, BD = 9, BQI = 10,
                   BQT = 11, BGC = 12, BDS = 13, BDQ = 14, BX0 = 15, BX1 = 16, BX2 = 17, BXQ = 18, BDYRD = 19,
-                  BDRAIN = 20, BEND = 21, BPR = 22;
-    static_assert(BPR < CF::NUM_BARS, "barrier count");
+                  BDRAIN = 20, BEND = 21, BPR = 22, BBC = 23;
+    static_assert(BBC < CF::NUM_BARS, "barrier count");
     extern __shared__ __align__(1024) uint8_t sm[];
     const uint32_t sb = smem_u32(sm);
     if (sb & 1023u) {
@@ -405,8 +408,7 @@ __global__ void __launch_bounds__(kThreads16, 1) bwd_dyq_tc(const __grid_constan
     const int niter = cid < nitems ? (nitems - 1 - cid) / ncl + 1 : 0;
     const int DV = p.dv, ch0 = 128 * rank;
     auto bar = [&](int i) -> uint32_t { return sb + CF::OFF_BAR + 8 * i; };
-    float* bc = reinterpret_cast<float*>(sm + CF::OFF_BC);
-    float* wsum = bc + kC;
+    float* bc = reinterpret_cast<float*>(sm + CF::OFF_BC);    // the chunk's decay sums (bulk-loaded)
     float* xch = reinterpret_cast<float*>(sm + CF::OFF_AUX);   // [128][2] round 0, [128][2] round 2
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + CF::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + CF::OFF_MISC + 4);
@@ -477,7 +479,8 @@ __global__ void __launch_bounds__(kThreads16, 1) bwd_dyq_tc(const __grid_constan
                     for (int k = 0; k < 4; ++k) gv[k] = ldg_nc_v4(gg + k);
                 }
             }
-            chunk_decay<RT>(p, tok0, hh, L, bc, wsum);
+            // the chunk's decay sums b_t (loaded with the tiles)
+            mbar_wait(bar(BBC), par, p.status, abort_flag);
             const float bt = bc[t], ebt = __expf(bt);
 
             // ------------------------------------------------ P = A o E, masked
@@ -818,7 +821,12 @@ __global__ void __launch_bounds__(kThreads16, 1) bwd_dyq_tc(const __grid_constan
                 tma_load_2d(sb + OFF_SL + x * kBox, &p.tmSL, ch0 + x * 64, srow, bar(BS));
             }
         };
+        auto load_bc = [&](int it) {
+            mbar_arrive_expect_tx(bar(BBC), kC * 4);
+            bulk_load(sb + CF::OFF_BC, p.bcg + (size_t)(cid + it * ncl) * kC, kC * 4, bar(BBC));
+        };
         if (lane == 0 && niter > 0) {
+            load_bc(0);
             load_tile(0, BQ, &p.tmQ, OFF_Q, 0);
             load_tile(0, BK, &p.tmK, OFF_K, 0);
             load_tile(0, BV, &p.tmV, OFF_V, ch0);
@@ -905,6 +913,8 @@ __global__ void __launch_bounds__(kThreads16, 1) bwd_dyq_tc(const __grid_constan
                 bulk_wait_read<0>();   // the dy store has read its tiles
                 mbar_arrive(bar(BDYRD));
                 ok = ok && mbar_wait(bar(BDS), par, p.status, abort_flag);
+                // the rows have read this chunk's decay sums
+                if (ok && more) load_bc(it + 1);
                 if (ok) {
                     tc_fence_after();
                     // dq += (D o E) K
@@ -975,7 +985,7 @@ __global__ void __launch_bounds__(kThreads16, 1) bwd_kv_tc(const __grid_constant
                   OFF_DSH = 5 * kTile, OFF_DSL = 6 * kTile;
     constexpr uint32_t R_AT = 0, R_DT = 128, R_DK = 256, R_DV = 384;
     constexpr int BQ = 0, BK = 1, BV = 2, BDY = 3, BS = 4, BADT = 5, BINTER = 6, BROWS = 7, BOUT = 8, BXK = 9,
-                  BXDONE = 10, BDRAIN = 11, BPR = 12;
+                  BXDONE = 10, BDRAIN = 11, BPR = 12, BBC = 13;
     extern __shared__ __align__(1024) uint8_t sm[];
     const uint32_t sb = smem_u32(sm);
     if (sb & 1023u) {
@@ -990,8 +1000,7 @@ __global__ void __launch_bounds__(kThreads16, 1) bwd_kv_tc(const __grid_constant
     const int niter = cid < nitems ? (nitems - 1 - cid) / ncl + 1 : 0;
     const int DV = p.dv, ch0 = 128 * rank;
     auto bar = [&](int i) -> uint32_t { return sb + CF::OFF_BAR + 8 * i; };
-    float* bc = reinterpret_cast<float*>(sm + CF::OFF_BC);
-    float* wsum = bc + kC;
+    float* bc = reinterpret_cast<float*>(sm + CF::OFF_BC);    // the chunk's decay sums (bulk-loaded)
     float* Facc = reinterpret_cast<float*>(sm + CF::OFF_AUX);   // [128] F_j over this CTA's channels
     float* ush = Facc + kC;                                      // [128] us_s over this CTA's channels
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + CF::OFF_MISC);
@@ -1034,7 +1043,8 @@ __global__ void __launch_bounds__(kThreads16, 1) bwd_kv_tc(const __grid_constant
             const int u = item / nc, c = item - u * nc, b = u / p.H, hh = u - b * p.H;
             const int n0 = c * kC, L = min(kC, p.N - n0);
             const size_t tok0 = (size_t)b * p.N + n0;
-            chunk_decay<RT>(p, tok0, hh, L, bc, wsum);
+            // the chunk's decay sums b_t (loaded with the tiles)
+            mbar_wait(bar(BBC), par, p.status, abort_flag);
             if (tid < kC) {
                 Facc[tid] = 0.f;
                 ush[tid] = 0.f;
@@ -1256,7 +1266,12 @@ __global__ void __launch_bounds__(kThreads16, 1) bwd_kv_tc(const __grid_constant
                 tma_load_2d(sb + OFF_DSL + x * kBox, &p.tmSL, ch0 + x * 64, srow, bar(BS));
             }
         };
+        auto load_bc = [&](int it) {
+            mbar_arrive_expect_tx(bar(BBC), kC * 4);
+            bulk_load(sb + CF::OFF_BC, p.bcg + (size_t)(cid + it * ncl) * kC, kC * 4, bar(BBC));
+        };
         if (lane == 0 && niter > 0) {
+            load_bc(0);
             load_q(0);
             load_k(0);
             load_v(0);
@@ -1304,8 +1319,12 @@ __global__ void __launch_bounds__(kThreads16, 1) bwd_kv_tc(const __grid_constant
                 // V is free once the dS' products have read it
                 if (mbar_wait(bar(BINTER), par, p.status, abort_flag) && more) load_v(it + 1);
                 ok = ok && mbar_wait(bar(BROWS), par, p.status, abort_flag);
-                // K is free once the rows have read it (us) and the products above are done
-                if (ok && more) load_k(it + 1);
+                // K is free once the rows have read it (us) and the products above are done;
+                // the rows have read the chunk's decay sums
+                if (ok && more) {
+                    load_k(it + 1);
+                    load_bc(it + 1);
+                }
                 if (ok) {
                     tc_fence_after();
                     // dk += (D o E)^T Q, dv += (A o E)^T dy
@@ -1452,7 +1471,7 @@ bool map_states(CUtensorMap* m, const void* base, int dv, size_t rows) {
 size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct BwdTcWs {
-    size_t incg, sh, sl, dyh, dyl, rr, xs, decay, fus, total;
+    size_t incg, sh, sl, dyh, dyl, rr, xs, decay, bcg, fus, total;
 };
 
 BwdTcWs bwd_tc_ws(int B, int H, int N, int dv) {
@@ -1468,6 +1487,7 @@ BwdTcWs bwd_tc_ws(int B, int H, int N, int dv) {
     w.rr = o; o += a256(2 * tok * 4);
     w.xs = o; o += a256(units * nc * dv * 4);
     w.decay = o; o += a256(units * nc * 4);
+    w.bcg = o; o += a256(units * nc * kC * 4);
     w.fus = o; o += a256(units * nc * 2 * 2 * kC * 4);
     w.total = o;
     return w;
@@ -1555,6 +1575,7 @@ cudaError_t launch_bwd_tc(const BackwardArgs& in, cudaStream_t s) {
     p.rr = reinterpret_cast<float*>(ws + w.rr);
     p.xs = reinterpret_cast<float*>(ws + w.xs);
     p.decay = reinterpret_cast<float*>(ws + w.decay);
+    p.bcg = reinterpret_cast<float*>(ws + w.bcg);
     p.fus = reinterpret_cast<float*>(ws + w.fus);
     const size_t srows = (size_t)in.B * in.H * p.nc * kDK;
     if (!map_tokens(&p.tmQ, in.Q, kDK, in.H, in.N, in.B) || !map_tokens(&p.tmK, in.K, kDK, in.H, in.N, in.B) ||

@@ -225,9 +225,10 @@ gret_status gret_state_fold(const float* dS_all, const float* decay_all, int num
  * (6 launches, chunks of 128 tokens, tcgen05 products with fp32 accumulation;
  * the per-chunk states, state gradients and dy enter the products as bf16
  * pairs hi + lo, about 16 mantissa bits).  Its workspace holds, per chunk, an
- * fp32 state-shaped buffer and a state as a bf16 pair (2 * B*H*ceil(N/128)*
+ * fp32 state-shaped buffer and a state as a bf16 pair (B*H*ceil(N/128)*
  * dk*dv*(4 + 4) bytes in all), dy as a bf16 pair (B*N*H*dv*4), two fp32 terms
- * per token and head, and per chunk dv + 513 fp32 values.  Other head sizes
+ * per token and head, and per chunk dv + 641 fp32 values (among them the
+ * decay sums of its 128 tokens).  Other head sizes
  * that are multiples of 32 with dk <= 128 and dv <= 256 take the chunk-parallel
  * path on CUDA cores in fp32 (5 launches; chunks of 64 tokens for bf16, 32 for
  * fp32), whose workspace holds the state before every chunk and the gradient

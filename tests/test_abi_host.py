@@ -129,12 +129,12 @@ def test_backward_path_and_workspace(lib):
     # tensor-core path (bf16, d_k 128): chunks of 128 tokens; per chunk an fp32
     # state-shaped buffer (increments, then G_c) and a state as a bf16 pair
     # (S_c, then dS'_c); dy as a bf16 pair; per token the two channel halves'
-    # inter-chunk terms; per chunk the d_v shares of X_c, e^{b_L} and the F/us
-    # partials of each channel half
+    # inter-chunk terms; per chunk the d_v shares of X_c, e^{b_L}, the decay sums
+    # of its 128 tokens and the F/us partials of each channel half
     assert gret.gret_prefill_backward_launches(4, 16, 4096, 128, 256, bf) == 6
     units, nc128, tok = 64, 32, 4 * 4096 * 16
     want = (units * nc128 * E * 4 + 2 * units * nc128 * E * 2 + 2 * tok * 256 * 2 + 2 * tok * 4
-            + units * nc128 * 256 * 4 + units * nc128 * 4 + units * nc128 * 512 * 4)
+            + units * nc128 * 256 * 4 + units * nc128 * 4 + units * nc128 * 128 * 4 + units * nc128 * 512 * 4)
     assert gret.gret_prefill_backward_workspace_size(4, 16, 4096, 128, 256, bf) == want
     nc = (100 + 31) // 32
     assert gret.gret_prefill_backward_launches(1, 2, 100, 64, 64, f32) == 5
