@@ -128,10 +128,12 @@ __global__ void __launch_bounds__(kProjThreads, 1) gate_project_scan_kernel(cons
                     mma_ss(tm, sdesc_sw128(st + kk * 32, 16, 1024), sdesc_sw128(st + CF::XB + kk * 32, 16, 1024),
                            idesc, (k | kk) != 0);
                 mma_commit(empty(s));
-                if (k + NS < p.nk) {
-                    // the stage is free once its MMAs have read it
-                    if (!mbar_wait(empty(s), (k / NS) & 1, p.status, abort_flag)) break;
-                    issue(k + NS);
+                // the previous step's stage is free once its MMAs have read it
+                // (they run before this step's, which queue behind them), so the
+                // issuer never waits on the MMAs it has just committed
+                if (k > 0 && k - 1 + NS < p.nk) {
+                    if (!mbar_wait(empty((k - 1) % NS), ((k - 1) / NS) & 1, p.status, abort_flag)) break;
+                    issue(k - 1 + NS);
                 }
             }
             mma_commit(done);

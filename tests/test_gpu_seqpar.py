@@ -99,3 +99,32 @@ def test_tc_resumed_from_the_state_pass(dv, chunk, N, cuts):
 def test_simt_resumed_is_from_state():
     cfg = gi.C1.scaled(N=256, seed=66)
     _run(cfg, (0, 100, 256), gret.Path.SIMT, with_s0=True, resume=True)
+
+
+def test_fold_on_unaligned_buffers():
+    """gret_state_fold with its increments, initial state and output one float
+    past a 16-byte boundary (the fold's element-wise variant): folding the
+    state-only passes of two slices from S0 gives the oracle's state after the
+    whole sequence."""
+    cfg = gi.C2.scaled(B=1, H=2, N=700, chunk=64, seed=67)
+    inp = gi.prefill_inputs(cfg)
+    d = {k: v.cuda() for k, v in inp.items()}
+    S0 = gi.random_unit(cfg.seed, 904, (cfg.B, cfg.H, cfg.dk, cfg.dv), var=0.04)
+    parts = [gret.prefill_state(d["K"][:, a:b].contiguous(), d["V"][:, a:b].contiguous(),
+                                d["z"][:, a:b].contiguous(), cfg.tau, cfg.chunk) for a, b in ((0, 300), (300, 700))]
+
+    def off_by_one_float(x):
+        buf = torch.empty(x.numel() + 1, dtype=torch.float32, device="cuda")
+        v = buf[1:].view(x.shape)
+        v.copy_(x)
+        assert v.data_ptr() % 16 == 4
+        return v
+
+    dS_all = off_by_one_float(torch.stack([p[0] for p in parts]))
+    decay_all = torch.stack([p[1] for p in parts])
+    out = off_by_one_float(torch.zeros((cfg.B, cfg.H, cfg.dk, cfg.dv), device="cuda"))
+    S = gret.state_fold(dS_all, decay_all, 2, S0=off_by_one_float(S0.cuda()), out=out)
+    gret.check_device_status()
+    lg = oracle.log_gamma(inp["z"], cfg.tau)
+    _, S_ref = oracle.recurrent(inp["K"], inp["K"], inp["V"], lg, S0=S0)
+    assert_close(S, S_ref, cfg.io, "fold of both slices from S0")
