@@ -315,8 +315,10 @@ int gret_prefill_varlen_launches(int num_seqs, int total_tokens, int max_seqlen,
     int sms = 148;
     device_info(nullptr, &sms);
     const gret_path p = select_path(num_seqs, H, max_seqlen, dk, dv, chunk, io_dtype, sms, nullptr, nullptr);
-    // tensor cores: gate scan, plan, state pass, combine, fused loop
-    return p == GRET_PATH_TC ? 5 : p == GRET_PATH_SIMT ? 1 : 0;
+    // tensor cores: gate scan, plan, (where a sequence may be cut) state pass
+    // and combine, fused loop
+    if (p == GRET_PATH_TC) return prefill_tc_varlen_launches(num_seqs, H, max_seqlen, total_tokens, dk, dv, chunk, sms);
+    return p == GRET_PATH_SIMT ? 1 : 0;
 }
 
 gret_status gret_prefill_varlen(const void* Q, const void* K, const void* V, const float* gate_logits,

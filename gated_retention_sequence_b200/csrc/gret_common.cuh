@@ -192,6 +192,9 @@ int prefill_tc_ctas_per_item(int dv, int chunk);
 size_t prefill_tc_workspace_bytes(int B, int H, int N, int dk, int dv, int chunk, int segments, int pieces);
 size_t prefill_tc_varlen_workspace_bytes(int S, int H, int max_seqlen, int total, int dk, int dv, int chunk,
                                          int num_sms);
+// Launches of a packed batch on the tensor-core path: 3, or 5 where max_seqlen
+// allows a sequence to be cut (state pass and combine).
+int prefill_tc_varlen_launches(int S, int H, int max_seqlen, int total, int dk, int dv, int chunk, int num_sms);
 int prefill_tc_launches(int segments, int pieces);
 
 }  // namespace gret

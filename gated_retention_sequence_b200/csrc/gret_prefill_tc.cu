@@ -2270,13 +2270,17 @@ cudaError_t run_tc(const PrefillArgs& a, TcParams& tp, cudaStream_t s, const Pla
         if (e != cudaSuccess) return e;
         e = launch_pdl(varlen_plan_kernel, dim3(1), dim3(kPlanThreads), 0, s, *plan);
         if (e != cudaSuccess) return e;
-        e = launch_pdl(ks, dim3(plan->max_state), dim3(kStateThreads), StateCfg<DV, C>::SMEM, s, tp);
-        if (e != cudaSuccess) return e;
-        const int elems4 = DV * DK / 4;
-        e = launch_pdl(seg_combine_kernel, dim3(plan->max_state, (elems4 + 255) / 256), dim3(256), 0, s,
-                       tp.seg_state, static_cast<const float*>(tp.seg_decay), tp.S0, 0, DK, DV, tp.unit_info,
-                       tp.state_items, tp.plan_count);
-        if (e != cudaSuccess) return e;
+        // a sequence is cut only when longer than seg_max (the plan clamps
+        // lengths to max_len): otherwise there is no state pass to run
+        if (plan->max_len > plan->seg_max) {
+            e = launch_pdl(ks, dim3(plan->max_state), dim3(kStateThreads), StateCfg<DV, C>::SMEM, s, tp);
+            if (e != cudaSuccess) return e;
+            const int elems4 = DV * DK / 4;
+            e = launch_pdl(seg_combine_kernel, dim3(plan->max_state, (elems4 + 255) / 256), dim3(256), 0, s,
+                           tp.seg_state, static_cast<const float*>(tp.seg_decay), tp.S0, 0, DK, DV, tp.unit_info,
+                           tp.state_items, tp.plan_count);
+            if (e != cudaSuccess) return e;
+        }
         if (g_profile_start) cudaEventRecord(g_profile_start, s);
         if constexpr (ROWS) {
             auto kr = prefill_rows_kernel<DV == 256, true>;
@@ -2440,6 +2444,10 @@ size_t prefill_tc_workspace_bytes(int B, int H, int N, int dk, int dv, int chunk
 size_t prefill_tc_varlen_workspace_bytes(int S, int H, int max_seqlen, int total, int dk, int dv, int chunk,
                                          int num_sms) {
     return varlen_layout(S, H, max_seqlen, total, dk, dv, chunk, num_sms).total;
+}
+
+int prefill_tc_varlen_launches(int S, int H, int max_seqlen, int total, int dk, int dv, int chunk, int num_sms) {
+    return max_seqlen > varlen_layout(S, H, max_seqlen, total, dk, dv, chunk, num_sms).seg_max ? 5 : 3;
 }
 
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {

@@ -138,11 +138,13 @@ gret_status gret_prefill_from_state(const void* Q, const void* K, const void* V,
  * aligned; total_tokens > 0.
  *
  * On the tensor-core path the work is planned on the device from cu_seqlens
- * (no host synchronisation): a sequence longer than half of one SM's share of the
- * batch's tokens and heads is cut into segments of equal length -- a state
- * pass gives each segment its initial state -- while the others stay whole,
- * and the segments start longest first, so that one long prompt among short
- * ones does not finish alone.  The call then makes
+ * (no host synchronisation): a sequence longer than one and a half work
+ * slots' share (a slot is an SM, or an SM pair for dv = 256) of the batch's
+ * tokens and heads is cut into segments of equal length -- a state pass gives
+ * each segment its initial state -- while the others stay whole, and the
+ * segments start longest first, so that one long prompt among short ones does
+ * not finish alone.  Where max_seqlen is within that bound no sequence is cut
+ * and the state pass is not launched.  The call then makes
  * gret_prefill_varlen_launches(...) launches.
  */
 gret_status gret_prefill_varlen(const void* Q, const void* K, const void* V, const float* gate_logits,
