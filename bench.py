@@ -669,15 +669,16 @@ def backward_alg_flops(cfg, chunk=BACKWARD_CHUNK):
     return cfg.B * cfg.N * cfg.H * (12 * cfg.dk * cfg.dv + chunk * (4 * cfg.dk + 3 * cfg.dv))
 
 
-def backward_summary(cfg, steps, ms, world, peaks, launches_per_call):
-    """The ``backward`` object of the JSON line for `steps` calls that took
-    `ms` (max over ranks) on each of `world` ranks."""
+def backward_summary(cfg, steps, ms, world, peaks, launches_per_call, warmup=3):
+    """The ``backward`` object of the JSON line for `steps` calls, after
+    `warmup` untimed ones, that took `ms` (max over ranks) on each of `world`
+    ranks."""
     bytes_ = backward_alg(cfg)
     flops = backward_alg_flops(cfg)
     step_s = ms / 1e3 / steps
     tflops = flops / step_s / 1e12
     peak = peaks["bf16_tflops"]
-    return {"workload": cfg.name, "steps": steps, "warmup": 2, "ms_per_step": ms / steps,
+    return {"workload": cfg.name, "steps": steps, "warmup": warmup, "ms_per_step": ms / steps,
             "value": job_throughput(world, cfg.B * cfg.N, steps, ms) / 1e6, "unit": "Mtok/s",
             "kernels": "bwd_inc_tc, bwd_scan_fwd, bwd_dyq_tc, bwd_scan_rev, bwd_kv_tc, bwd_dz "
                        "(tcgen05 kind::f16, states and dy as bf16 pairs, fp32 accumulation in tensor memory)",
@@ -703,6 +704,7 @@ def run_backward(args, world, dev, stream, d, O, cfg, peaks):
         d = {k: v[:nb] for k, v in d.items()}
         O = O[:nb]
     steps = max(1, min(args.steps, 5))
+    warmup = max(3, min(args.warmup, 5))
     dO = O.clone()
     io = gret.Dtype.BF16
     ws_bytes = gret.gret_prefill_backward_workspace_size(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, io)
@@ -712,7 +714,7 @@ def run_backward(args, world, dev, stream, d, O, cfg, peaks):
         return gret.prefill_backward(d["Q"], d["K"], d["V"], d["z"], d["G"], dO, cfg.tau, eps=cfg.eps,
                                      workspace=ws, stream=stream)
 
-    for _ in range(2):
+    for _ in range(warmup):
         step()
     gret.check_device_status()
     barrier(world)
@@ -725,7 +727,7 @@ def run_backward(args, world, dev, stream, d, O, cfg, peaks):
     gret.check_device_status()
     ms = max_over_ranks(e0.elapsed_time(e1), world)
     return backward_summary(cfg, steps, ms, world, peaks,
-                            gret.gret_prefill_backward_launches(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, io))
+                            gret.gret_prefill_backward_launches(cfg.B, cfg.H, cfg.N, cfg.dk, cfg.dv, io), warmup)
 
 
 def projection_alg(cfg, d_model):
